@@ -1,0 +1,230 @@
+"""TQ4_1S CPU oracle -- test infrastructure, not part of the product.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline
+leg may import this package.  It wraps ``tq4_1s_oracle.c`` (plain scalar C,
+compiled with gcc without FMA contraction or fast-math) through ctypes and
+shares nothing with the CUDA path.
+
+Every function follows the Nemotron-TheHobbit-30B-A3B model card, section
+"What Config-I means" (per-32-block Walsh-Hadamard rotation, 16-level
+Lloyd-Max codes, two half-block scales, ~5 bits/weight), with the readings
+listed at the top of the C file.  Parity status of each function:
+
+- codebook, sign_mask, hadamard32, fwht32, quantize, dequantize, levels,
+  linear, moe_route: pinned by ``tests/test_oracle_pins.py``.
+- moe: pinned through closed-form special cases (single slot, constant-level
+  experts) and composition with the pinned linear; the squared-ReLU and the
+  bf16 rounding of the hidden activation are fixed by the workload
+  definition, not by the pages.
+- reconstruction cosine 0.997 quoted on the model card for real weights:
+  parity unpinned (real weights are not available; synthetic weights are
+  checked against the >= 0.99 bound instead).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "tq4_1s_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle_tq4.so")
+CFLAGS = ["-O2", "-std=gnu11", "-ffp-contract=off", "-fexcess-precision=standard", "-fno-fast-math",
+          "-shared", "-fPIC"]
+_lock = threading.Lock()
+_lib = None
+
+BLOCK = 32
+HALF = 16
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle shared library with gcc (idempotent)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + ".tmp%d" % os.getpid()
+        subprocess.check_call(["gcc", *CFLAGS, "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is None:
+            lib = ctypes.CDLL(build())
+            P = ctypes.c_void_p
+            I64 = ctypes.c_int64
+            lib.orc_codebook.argtypes = [P, P, P, P]
+            lib.orc_codebook.restype = ctypes.c_int
+            lib.orc_splitmix64_first.argtypes = [ctypes.c_uint64]
+            lib.orc_splitmix64_first.restype = ctypes.c_uint64
+            lib.orc_sign_mask.argtypes = [ctypes.c_uint64]
+            lib.orc_sign_mask.restype = ctypes.c_uint32
+            lib.orc_hadamard32.argtypes = [P]
+            lib.orc_fwht32_f32.argtypes = [P]
+            lib.orc_rotate_block.argtypes = [P, ctypes.c_uint32, P]
+            lib.orc_f16_to_f32.argtypes = [ctypes.c_uint16]
+            lib.orc_f16_to_f32.restype = ctypes.c_float
+            lib.orc_f32_to_f16_sat.argtypes = [ctypes.c_float]
+            lib.orc_f32_to_f16_sat.restype = ctypes.c_uint16
+            lib.orc_f64_to_bf16.argtypes = [ctypes.c_double]
+            lib.orc_f64_to_bf16.restype = ctypes.c_uint16
+            lib.orc_quantize.argtypes = [P, I64, I64, ctypes.c_uint64, P, P]
+            lib.orc_quantize.restype = I64
+            lib.orc_dequantize.argtypes = [P, P, I64, I64, ctypes.c_uint64, P]
+            lib.orc_levels.argtypes = [P, P, I64, I64, P]
+            lib.orc_linear.argtypes = [P, I64, I64, P, I64, P]
+            lib.orc_round_bf16.argtypes = [P, I64, P]
+            lib.orc_moe_route.argtypes = [P, I64, ctypes.c_int, ctypes.c_int, P, P]
+            lib.orc_moe_route.restype = I64
+            lib.orc_moe.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, ctypes.c_int,
+                                    P, P, ctypes.c_uint64, P, P, ctypes.c_uint64, P]
+            lib.orc_moe.restype = I64
+            _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# ---------------------------------------------------------------------------
+def codebook():
+    """Lloyd-Max levels of N(0,1), 16 levels.  Returns (c, t, c32, t32)."""
+    c = np.zeros(16); t = np.zeros(15)
+    c32 = np.zeros(16, np.float32); t32 = np.zeros(15, np.float32)
+    it = _load().orc_codebook(_ptr(c), _ptr(t), _ptr(c32), _ptr(t32))
+    if it < 0:
+        raise RuntimeError("Lloyd iteration did not converge")
+    return c, t, c32, t32
+
+
+def splitmix64_first(state: int) -> int:
+    return int(_load().orc_splitmix64_first(state))
+
+
+def sign_mask(seed: int) -> int:
+    return int(_load().orc_sign_mask(seed))
+
+
+def hadamard32() -> np.ndarray:
+    H = np.zeros((32, 32), np.int8)
+    _load().orc_hadamard32(_ptr(H))
+    return H
+
+
+def fwht32(a) -> np.ndarray:
+    a = _c(a, np.float32).copy()
+    assert a.shape == (32,)
+    _load().orc_fwht32_f32(_ptr(a))
+    return a
+
+
+def rotate_block(w, mask: int) -> np.ndarray:
+    w = _c(w, np.float32)
+    v = np.zeros(32, np.float32)
+    _load().orc_rotate_block(_ptr(w), mask, _ptr(v))
+    return v
+
+
+def f16_to_f32(h: int) -> float:
+    return float(_load().orc_f16_to_f32(h))
+
+
+def f32_to_f16_sat(x: float) -> int:
+    return int(_load().orc_f32_to_f16_sat(x))
+
+
+def f64_to_bf16(x: float) -> int:
+    return int(_load().orc_f64_to_bf16(x))
+
+
+def quantize(W, seed: int):
+    """W fp32 [n][k] -> (codes uint8 [n][k/2], scales uint16 [n][k/16], nonfinite_blocks)."""
+    W = _c(W, np.float32)
+    n, k = W.shape
+    assert k % BLOCK == 0
+    codes = np.zeros((n, k // 2), np.uint8)
+    scales = np.zeros((n, k // HALF), np.uint16)
+    bad = _load().orc_quantize(_ptr(W), n, k, seed, _ptr(codes), _ptr(scales))
+    return codes, scales, int(bad)
+
+
+def dequantize(codes, scales, seed: int) -> np.ndarray:
+    codes = _c(codes, np.uint8); scales = _c(scales, np.uint16)
+    n, k = codes.shape[0], codes.shape[1] * 2
+    W = np.zeros((n, k), np.float32)
+    _load().orc_dequantize(_ptr(codes), _ptr(scales), n, k, seed, _ptr(W))
+    return W
+
+
+def levels(codes, scales) -> np.ndarray:
+    """Rotated-domain dequantized values (codebook level times half-block scale)."""
+    codes = _c(codes, np.uint8); scales = _c(scales, np.uint16)
+    n, k = codes.shape[0], codes.shape[1] * 2
+    wn = np.zeros((n, k), np.float32)
+    _load().orc_levels(_ptr(codes), _ptr(scales), n, k, _ptr(wn))
+    return wn
+
+
+def linear_f64(x_bf16, W_hat) -> np.ndarray:
+    """y = x * W_hat^T in fp64 (x as bf16 bits [m][k], W_hat fp32 [n][k])."""
+    x = _c(x_bf16, np.uint16); W = _c(W_hat, np.float32)
+    m, k = x.shape
+    n = W.shape[0]
+    assert W.shape[1] == k
+    y = np.zeros((m, n), np.float64)
+    _load().orc_linear(_ptr(x), m, k, _ptr(W), n, _ptr(y))
+    return y
+
+
+def round_bf16(y) -> np.ndarray:
+    y = _c(y, np.float64)
+    out = np.zeros(y.shape, np.uint16)
+    _load().orc_round_bf16(_ptr(y), y.size, _ptr(out))
+    return out
+
+
+def linear(x_bf16, codes, scales, seed: int):
+    """The TQ4_1S linear layer: returns (y_f64, y_bf16_bits)."""
+    y = linear_f64(x_bf16, dequantize(codes, scales, seed))
+    return y, round_bf16(y)
+
+
+def moe_route(ids, num_experts: int):
+    ids = _c(ids, np.int32)
+    m, topk = ids.shape
+    offsets = np.zeros(num_experts + 1, np.int32)
+    pairs = np.full(m * topk, -1, np.int32)
+    bad = _load().orc_moe_route(_ptr(ids), m, topk, num_experts, _ptr(offsets), _ptr(pairs))
+    return offsets, pairs[: offsets[-1]], int(bad)
+
+
+def moe(x_bf16, ids, w, up_codes, up_scales, up_seed, dn_codes, dn_scales, dn_seed):
+    """MoE layer.  up_*: [E][I][H/2], [E][I][H/16]; dn_*: [E][H][I/2], [E][H][I/16].
+
+    Returns (y_f64 [m][H], y_bf16_bits, skipped_pairs)."""
+    x = _c(x_bf16, np.uint16); ids = _c(ids, np.int32); w = _c(w, np.float32)
+    uc = _c(up_codes, np.uint8); us = _c(up_scales, np.uint16)
+    dc = _c(dn_codes, np.uint8); ds = _c(dn_scales, np.uint16)
+    m, H = x.shape
+    E, I = uc.shape[0], uc.shape[1]
+    topk = ids.shape[1]
+    assert uc.shape == (E, I, H // 2) and dc.shape == (E, H, I // 2)
+    y = np.zeros((m, H), np.float64)
+    bad = _load().orc_moe(_ptr(x), m, H, I, _ptr(ids), _ptr(w), topk, E, _ptr(uc), _ptr(us), up_seed,
+                          _ptr(dc), _ptr(ds), dn_seed, _ptr(y))
+    return y, round_bf16(y), int(bad)
+
+
+def packed_bytes(n: int, k: int, num_experts: int = 1):
+    """Bytes of the two planes: codes 4 bits/weight, scales 2 x fp16 per 32."""
+    return num_experts * n * k // 2, num_experts * n * (k // HALF) * 2

@@ -1,0 +1,348 @@
+"""Pins that tie the CPU oracle to facts other than itself.
+
+Each test checks one oracle function against a closed form, a textbook or
+published value, a library routine used independently, or brute force, so
+that a dropped term, a wrong sign or index, or a transposed operand in the
+oracle fails here.  CPU only.
+"""
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+from scipy.stats import norm
+
+import oracle
+import synth
+
+
+def test_hadamard_is_orthogonal_and_symmetric():
+    # Closed form: the 32-point Sylvester Hadamard matrix satisfies H H^T = 32 I.
+    H = oracle.hadamard32().astype(np.int64)
+    assert np.array_equal(H @ H.T, 32 * np.eye(32, dtype=np.int64))
+    assert np.array_equal(H, H.T)
+    assert np.all(H[0] == 1) and np.all(H[:, 0] == 1)
+    # Sylvester recursion H_2n = [[H_n, H_n], [H_n, -H_n]] in natural order.
+    h = np.array([[1]])
+    for _ in range(5):
+        h = np.block([[h, h], [h, -h]])
+    assert np.array_equal(H, h)
+
+
+def test_fwht_matches_matrix_product():
+    H = oracle.hadamard32().astype(np.float64)
+    for i in range(32):   # unit vectors: exact columns of H
+        e = np.zeros(32, np.float32); e[i] = 1.0
+        assert np.array_equal(oracle.fwht32(e).astype(np.float64), H[:, i])
+    a = synth.normal_f32(32, 11)
+    ref = H @ a.astype(np.float64)
+    got = oracle.fwht32(a).astype(np.float64)
+    # five fp32 additions per output: |err| <= 5 * 2^-24 * sum|a| (generous)
+    assert np.max(np.abs(got - ref)) <= 5 * 2.0 ** -24 * np.abs(a).sum() * 4
+
+
+def test_rotate_block_applies_signs_then_hadamard():
+    mask = 0b1011_0000_0000_0000_0000_0000_0000_0101
+    H = oracle.hadamard32().astype(np.float64)
+    s = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(32)])
+    w = synth.normal_f32(32, 12)
+    ref = (H @ (s * w.astype(np.float64))) / np.sqrt(32.0)
+    got = oracle.rotate_block(w, mask).astype(np.float64)
+    assert np.max(np.abs(got - ref)) < 1e-5 * np.abs(w).max()
+
+
+def test_codebook_is_lloyd_fixed_point():
+    c, t, c32, t32 = oracle.codebook()
+    edges = np.concatenate([[-np.inf], t, [np.inf]])
+    # centroid condition, with scipy's normal pdf/cdf (independent library)
+    cent = (norm.pdf(edges[:-1]) - norm.pdf(edges[1:])) / (norm.cdf(edges[1:]) - norm.cdf(edges[:-1]))
+    assert np.max(np.abs(cent - c)) < 1e-9
+    # midpoint (nearest-neighbour) condition
+    assert np.max(np.abs(t - 0.5 * (c[:-1] + c[1:]))) < 1e-15
+    assert np.all(np.diff(c) > 0)
+    assert np.array_equal(c[::-1], -c) and t[7] == 0.0
+    assert np.array_equal(c32, c.astype(np.float32)) and np.array_equal(t32, t.astype(np.float32))
+
+
+def test_codebook_matches_max_1960_table(golden_dir):
+    c, t, _, _ = oracle.codebook()
+    outs, ths = {}, {}
+    for line in open(os.path.join(golden_dir, "max1960_gaussian_16_levels.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        kind, idx, val = line.split()
+        (outs if kind == "output" else ths)[int(idx)] = float(val)
+    for i, v in outs.items():
+        assert abs(c[7 + i] - v) <= 6e-4, (i, c[7 + i], v)
+    for i, v in ths.items():
+        assert abs((0.0 if i == 1 else t[6 + i]) - v) <= 6e-4, (i, v)
+
+
+def test_codebook_distortion():
+    # MSE of the 16-level Lloyd-Max quantizer of N(0,1) by numerical integration.
+    c, t, _, _ = oracle.codebook()
+    from scipy.integrate import quad
+    edges = np.concatenate([[-np.inf], t, [np.inf]])
+    mse = sum(quad(lambda x, cj=cj: (x - cj) ** 2 * norm.pdf(x), a, b)[0]
+              for cj, a, b in zip(c, edges[:-1], edges[1:]))
+    assert 0.0094 < mse < 0.0096
+
+
+def test_sign_mask_published_splitmix64(golden_dir):
+    for line in open(os.path.join(golden_dir, "splitmix64_first_outputs.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        state, hx = line.split()
+        assert oracle.splitmix64_first(int(state)) == int(hx, 16)
+        assert oracle.sign_mask(int(state)) == int(hx, 16) & 0xFFFFFFFF
+
+
+def test_f16_rounding_matches_numpy():
+    g = synth.rng(21)
+    vals = np.concatenate([
+        (g.standard_normal(20000) * 10.0 ** g.uniform(-9, 4.8, 20000)).astype(np.float32),
+        np.array([0.0, -0.0, 6.1035156e-05, 5.9604645e-08, 2.9802322e-08, 65504.0, 65519.0, 1e-3], np.float32),
+    ])
+    vals = vals[np.abs(vals) < 65520.0]   # numpy overflows to inf beyond; saturation is checked below
+    for v in vals:
+        assert oracle.f32_to_f16_sat(float(v)) == int(np.array(v, np.float32).astype(np.float16).view(np.uint16))
+    # saturation instead of overflow to infinity
+    for v, bits in [(65520.0, 0x7BFF), (1e6, 0x7BFF), (-np.inf, 0xFBFF), (np.inf, 0x7BFF)]:
+        assert oracle.f32_to_f16_sat(v) == bits
+    for h in [0x0001, 0x03FF, 0x0400, 0x3C00, 0x7BFF, 0x8001, 0xBC00]:
+        assert oracle.f16_to_f32(h) == float(np.array(h, np.uint16).view(np.float16))
+
+
+def _bf16_brute(x: float) -> int:
+    """Round x to bf16 by enumerating bf16 neighbours in exact rational arithmetic."""
+    f = Fraction(x)
+    sign = 0x8000 if x < 0 else 0
+    f = abs(f)
+    # bracket by the float32 neighbours: find bf16 values just below/above
+    b = np.array(abs(x), np.float64).astype(np.float32).view(np.uint32) >> 16
+    cands = [int(b) - 1, int(b), int(b) + 1, int(b) + 2]
+    best = None
+    for cb in cands:
+        if cb < 0 or cb > 0x7F80:
+            continue
+        val = Fraction(float(np.array(cb << 16, np.uint32).view(np.float32)))
+        d = abs(val - f)
+        key = (d, cb & 1)
+        if best is None or key < best[0]:
+            best = (key, cb)
+    return sign | best[1]
+
+
+def test_bf16_rounding_from_double_brute_force():
+    g = synth.rng(22)
+    vals = list(g.standard_normal(3000) * 10.0 ** g.uniform(-30, 30, 3000))
+    # exact ties between two bf16 values: must go to the even one
+    vals += [1.0 + 2.0 ** -8, 1.0 + 3 * 2.0 ** -8, -(1.0 + 2.0 ** -8), 1.0 + 2.0 ** -8 + 2.0 ** -40]
+    for v in vals:
+        assert oracle.f64_to_bf16(float(v)) == _bf16_brute(float(v)), v
+
+
+def test_threshold_search_equals_nearest_level():
+    _, _, c32, t32 = oracle.codebook()
+    u = synth.rng(23).standard_normal(1_000_000).astype(np.float32) * 1.3
+    by_threshold = (u[:, None] > t32[None, :]).sum(axis=1)
+    by_distance = np.argmin(np.abs(u[:, None].astype(np.float64) - c32[None, :].astype(np.float64)), axis=1)
+    near = np.min(np.abs(u[:, None].astype(np.float64) - t32[None, :].astype(np.float64)), axis=1) < 1e-6
+    assert np.all((by_threshold == by_distance) | near)
+    assert near.sum() < 20
+
+
+def _unpack(codes):
+    lo = codes & 0xF
+    hi = codes >> 4
+    out = np.empty((codes.shape[0], codes.shape[1] * 2), np.int64)
+    out[:, 0::2] = lo
+    out[:, 1::2] = hi
+    return out
+
+
+def test_quantize_brute_force_tiny():
+    """Codes and scales against an independent formulation: explicit Hadamard
+    matrix in fp64, numpy's fp16 rounding, argmin over the 16 levels."""
+    c, t, c32, t32 = oracle.codebook()
+    H = oracle.hadamard32().astype(np.float64)
+    seed = 5
+    mask = oracle.sign_mask(seed)
+    s = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(32)])
+    W = np.concatenate([synth.normal_f32((6, 96), 31, 0.02), synth.student_t_f32((6, 96), 32, 5.0, 0.3)])
+    codes, scales, bad = oracle.quantize(W, seed)
+    assert bad == 0 and codes.shape == (12, 48) and scales.shape == (12, 6)
+    q = _unpack(codes)
+    boundary, midpoint = 0, 0
+    for r in range(W.shape[0]):
+        for kb in range(3):
+            v = (H @ (s * W[r, 32 * kb:32 * kb + 32].astype(np.float64))) / np.sqrt(32.0)
+            for h in range(2):
+                vh = v[16 * h:16 * h + 16]
+                rms = np.sqrt(np.mean(vh * vh))
+                d16 = np.array(rms, np.float64).astype(np.float16)
+                got_d = scales[r, 2 * kb + h]
+                if got_d != int(d16.view(np.uint16)):
+                    # only allowed within 1e-6 (relative) of an fp16 rounding midpoint
+                    lo = float(np.array(got_d, np.uint16).view(np.float16))
+                    ref = float(d16)
+                    assert abs(rms - 0.5 * (lo + ref)) <= 1e-6 * rms
+                    midpoint += 1
+                    continue
+                d = float(d16)
+                u = vh / d
+                want = np.argmin(np.abs(u[:, None] - c32[None, :].astype(np.float64)), axis=1)
+                got = q[r, 32 * kb + 16 * h:32 * kb + 16 * h + 16]
+                for i in range(16):
+                    if got[i] != want[i]:
+                        assert np.min(np.abs(u[i] - t)) < 1e-6
+                        boundary += 1
+    assert boundary + midpoint <= 2
+
+
+def test_quantize_special_blocks():
+    W = np.zeros((2, 64), np.float32)
+    W[1, 32:] = synth.normal_f32(32, 41)
+    W[1, 3] = np.nan
+    codes, scales, bad = oracle.quantize(W, 0)
+    assert bad == 1
+    # all-zero block: both scales 0 and every code is 7
+    assert np.all(scales[0] == 0) and np.all(codes[0] == 0x77)
+    # a NaN spreads through the butterfly: scale is the fp16 NaN, codes 0
+    assert np.all(scales[1, :2] == 0x7E00) and np.all(codes[1, :16] == 0)
+    assert np.all(scales[1, 2:] != 0)
+
+
+def test_levels_and_dequantize_closed_form():
+    _, _, c32, _ = oracle.codebook()
+    seed = 77
+    mask = oracle.sign_mask(seed)
+    s = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(32)])
+    H = oracle.hadamard32().astype(np.float64)
+    g = synth.rng(42)
+    codes = g.integers(0, 256, (5, 48), dtype=np.uint8)
+    scales = np.array(g.uniform(0.001, 2.0, (5, 6)), np.float32).astype(np.float16).view(np.uint16)
+    q = _unpack(codes)
+    d = scales.view(np.float16).astype(np.float64)
+    wn_ref = c32[q].astype(np.float64) * np.repeat(d, 16, axis=1)
+    wn = oracle.levels(codes, scales)
+    assert np.allclose(wn, wn_ref, rtol=2 ** -23, atol=0)
+    W = oracle.dequantize(codes, scales, seed).astype(np.float64)
+    for kb in range(3):
+        blk = wn_ref[:, 32 * kb:32 * kb + 32]
+        ref = (blk @ H.T) / np.sqrt(32.0) * s[None, :]
+        assert np.max(np.abs(W[:, 32 * kb:32 * kb + 32] - ref)) < 1e-5 * np.abs(ref).max()
+    # constant codes: H * (level * 1) = 32 * level * e_0, so only element 0 survives
+    codes_c = np.full((1, 16), 0xFF, np.uint8)
+    scales_c = np.array([[0x3C00, 0x3C00]], np.uint16)  # d = 1.0
+    Wc = oracle.dequantize(codes_c, scales_c, seed)[0]
+    expect0 = np.float32(np.float32(np.float32(32.0) * c32[15]) * np.float32(1 / np.sqrt(32.0)))
+    assert Wc[0] == pytest.approx(s[0] * float(expect0), rel=1e-6)
+    assert np.all(Wc[1:] == 0.0)
+
+
+def test_bits_per_weight_is_five():
+    codes_b, scales_b = oracle.packed_bytes(4096, 4096)
+    assert codes_b + scales_b == 10_485_760           # "~10.5 MB" packed
+    assert (codes_b + scales_b) * 8 / (4096 * 4096) == 5.0
+    W = synth.normal_f32((4, 64), 1, 0.02)
+    codes, scales, _ = oracle.quantize(W, 0)
+    assert (codes.nbytes + scales.nbytes) * 8 / W.size == 5.0
+
+
+@pytest.mark.parametrize("dist", ["normal", "student_t5", "laplace"])
+def test_reconstruction_cosine(dist):
+    if dist == "normal":
+        W = synth.normal_f32((128, 1024), 51, 0.02)
+    elif dist == "student_t5":
+        W = synth.student_t_f32((128, 1024), 52, 5.0, 0.02)
+    else:
+        W = (synth.rng(53).laplace(0.0, 0.02, (128, 1024))).astype(np.float32)
+    codes, scales, _ = oracle.quantize(W, 9)
+    Wh = oracle.dequantize(codes, scales, 9).astype(np.float64)
+    W = W.astype(np.float64)
+    cos = (W * Wh).sum() / np.sqrt((W * W).sum() * (Wh * Wh).sum())
+    assert cos >= 0.99
+
+
+def test_rotation_equivalence_route_a_equals_route_b():
+    """x * W_hat^T == (R x) * w_n^T per 32-slice, with R = r H diag(s) orthogonal."""
+    seed = 13
+    W = synth.normal_f32((8, 128), 61, 0.02)
+    codes, scales, _ = oracle.quantize(W, seed)
+    x = synth.activations_bf16(3, 128, 62)
+    xf = synth.bf16_bits_to_f32(x).astype(np.float64)
+    wn = oracle.levels(codes, scales).astype(np.float64)
+    mask = oracle.sign_mask(seed)
+    s = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(32)])
+    H = oracle.hadamard32().astype(np.float64)
+    R = (H * s[None, :]) / np.sqrt(32.0)
+    xr = np.concatenate([xf[:, 32 * b:32 * b + 32] @ R.T for b in range(4)], axis=1)
+    route_b = xr @ wn.T
+    # route A with the exactly inverse-rotated (fp64) weights
+    What = np.concatenate([wn[:, 32 * b:32 * b + 32] @ R for b in range(4)], axis=1)
+    route_a = xf @ What.T
+    assert np.max(np.abs(route_a - route_b)) < 1e-12 * np.abs(route_a).max()
+    # and the oracle's linear (fp32 inverse rotation) agrees to fp32 accuracy
+    y, _ = oracle.linear(x, codes, scales, seed)
+    assert np.max(np.abs(y - route_b)) < 1e-5 * np.abs(route_b).max()
+
+
+def test_linear_matches_library_matmul_and_rounding():
+    W = synth.normal_f32((40, 96), 71, 0.02)
+    codes, scales, _ = oracle.quantize(W, 3)
+    x = synth.activations_bf16(5, 96, 72)
+    Wh = oracle.dequantize(codes, scales, 3)
+    y, yb = oracle.linear(x, codes, scales, 3)
+    ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ Wh.astype(np.float64).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-15)
+    flat = y.ravel()
+    for i in range(0, flat.size, 7):
+        assert yb.ravel()[i] == _bf16_brute(float(flat[i]))
+
+
+def test_moe_route_brute_force():
+    ids, _ = synth.gumbel_topk_router(16, 128, 6, 7)
+    offsets, pairs, bad = oracle.moe_route(ids, 128)
+    assert bad == 0
+    flat = ids.ravel()
+    want = sorted(range(flat.size), key=lambda p: (flat[p], p))
+    assert list(pairs) == want
+    counts = np.bincount(flat, minlength=128)
+    assert np.array_equal(np.diff(offsets), counts)
+    ids2 = ids.copy(); ids2[3, 2] = 128; ids2[5, 0] = -1
+    offsets2, pairs2, bad2 = oracle.moe_route(ids2, 128)
+    assert bad2 == 2 and len(pairs2) == flat.size - 2 and 3 * 6 + 2 not in pairs2
+
+
+def test_router_weights_are_normalised():
+    ids, w = synth.gumbel_topk_router(16, 128, 6, 7)
+    assert ids.shape == (16, 6) and np.allclose(w.sum(axis=1), 1.0, atol=1e-6)
+    assert all(len(set(r)) == 6 for r in ids)
+
+
+def test_moe_composes_linear_relu2_and_slot_sum():
+    E, H, I, m, topk = 4, 64, 96, 5, 2
+    up = synth.normal_f32((E, I, H), 81, 0.05)
+    dn = synth.normal_f32((E, H, I), 82, 0.05)
+    uq = [oracle.quantize(up[e], 4)[:2] for e in range(E)]
+    dq = [oracle.quantize(dn[e], 5)[:2] for e in range(E)]
+    uc = np.stack([a for a, _ in uq]); us = np.stack([b for _, b in uq])
+    dc = np.stack([a for a, _ in dq]); ds = np.stack([b for _, b in dq])
+    ids, w = synth.gumbel_topk_router(m, E, topk, 83)
+    ids[1, 1] = E + 3  # out of range: skipped
+    x = synth.activations_bf16(m, H, 84)
+    y, yb, bad = oracle.moe(x, ids, w, uc, us, 4, dc, ds, 5)
+    assert bad == 1
+    ref = np.zeros((m, H))
+    for t in range(m):
+        for j in range(topk):
+            e = ids[t, j]
+            if not 0 <= e < E:
+                continue
+            u = oracle.linear_f64(x[t:t + 1], oracle.dequantize(uc[e], us[e], 4))
+            h = oracle.round_bf16(np.maximum(u, 0.0) ** 2)
+            z = oracle.linear_f64(h, oracle.dequantize(dc[e], ds[e], 5))
+            ref[t] += float(w[t, j]) * z[0]
+    assert np.array_equal(y, ref)
+    assert np.array_equal(yb, oracle.round_bf16(ref))
