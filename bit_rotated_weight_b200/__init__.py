@@ -1,0 +1,254 @@
+"""Python binding of libtq4_1s.so, the B200 (sm_100a) TQ4_1S layer.
+
+Argument marshalling only: PyTorch supplies device memory and the current
+stream; every step of quantize, dequantize, linear and MoE runs in the CUDA
+kernels behind the C ABI declared in ``include/tq4_1s.h``.  There is no CPU
+or PyTorch fallback: if the shared library is missing or the device is not
+an sm_100 GPU, the calls raise.
+
+TQ4_1S ("Config-I") is the weight format of the Nemotron-TheHobbit-30B-A3B
+model card, section "What Config-I means": a randomized Walsh-Hadamard
+rotation per 32-element block, 4-bit codes into a 16-level Lloyd-Max
+codebook, two half-block scales, about 5 bits per weight.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from dataclasses import dataclass
+
+import torch
+
+__all__ = [
+    "LIB_PATH", "TQ4Error", "Packed", "load_library",
+    "tq4_1s_version", "tq4_1s_error_string", "tq4_1s_packed_bytes", "tq4_1s_sign_mask", "tq4_1s_codebook",
+    "tq4_1s_quantize", "tq4_1s_dequantize", "tq4_1s_linear_workspace", "tq4_1s_linear",
+    "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_route", "tq4_1s_get_status",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtq4_1s.so")
+
+TQ_OK = 0
+TQ_DTYPE_F32, TQ_DTYPE_BF16 = 0, 1
+TQ_DEV_TIMEOUT, TQ_DEV_BAD_ROUTING, TQ_DEV_NONFINITE = 1, 2, 4
+
+
+class TQ4Error(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {tq4_1s_error_string(code)} (code {code})")
+
+
+class _Weight(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("num_experts", ctypes.c_int32),
+        ("reserved", ctypes.c_int32), ("seed", ctypes.c_uint64),
+        ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+    ]
+
+
+_lock = threading.Lock()
+_lib = None
+
+
+def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
+    """Load libtq4_1s.so (built by ``__graft_entry__.build()``); raise if absent."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(path):
+                raise ImportError(f"libtq4_1s.so not built (expected at {path}); run __graft_entry__.build()")
+            lib = ctypes.CDLL(path)
+            P, I64, I32, SZ = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int32, ctypes.c_size_t
+            W = ctypes.POINTER(_Weight)
+            sig = {
+                "tq4_1s_version": ([], ctypes.c_int),
+                "tq4_1s_error_string": ([ctypes.c_int], ctypes.c_char_p),
+                "tq4_1s_packed_bytes": ([I64, I64, I32, ctypes.POINTER(SZ), ctypes.POINTER(SZ)], ctypes.c_int),
+                "tq4_1s_sign_mask": ([ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
+                "tq4_1s_codebook": ([P, P], ctypes.c_int),
+                "tq4_1s_quantize": ([P, ctypes.c_int, W, P], ctypes.c_int),
+                "tq4_1s_dequantize": ([W, P, P], ctypes.c_int),
+                "tq4_1s_linear_workspace": ([I64, W], SZ),
+                "tq4_1s_linear": ([P, I64, W, P, P, SZ, P], ctypes.c_int),
+                "tq4_1s_moe_workspace": ([I64, I32, W, W], SZ),
+                "tq4_1s_moe": ([P, I64, P, P, I32, W, W, P, P, SZ, P], ctypes.c_int),
+                "tq4_1s_moe_route": ([P, I64, I32, I32, P, P, P], ctypes.c_int),
+                "tq4_1s_get_status": ([P, ctypes.POINTER(I32)], ctypes.c_int),
+            }
+            for name, (args, res) in sig.items():
+                fn = getattr(lib, name)
+                fn.argtypes = args
+                fn.restype = res
+            _lib = lib
+    return _lib
+
+
+def _check(rc: int, what: str):
+    if rc != TQ_OK:
+        raise TQ4Error(rc, what)
+
+
+def _stream(device: torch.device | None = None):
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t: torch.Tensor | None):
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+@dataclass
+class Packed:
+    """A packed TQ4_1S tensor (stack): codes [E][n][k/2] uint8, scales [E][n][k/16] fp16 bits."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    n: int
+    k: int
+    num_experts: int
+    seed: int
+
+    def c_struct(self) -> _Weight:
+        return _Weight(self.n, self.k, self.num_experts, 0, self.seed, self.codes.data_ptr(), self.scales.data_ptr())
+
+    @property
+    def nbytes(self) -> int:
+        return self.codes.numel() + self.scales.numel() * 2
+
+
+def tq4_1s_version() -> int:
+    return load_library().tq4_1s_version()
+
+
+def tq4_1s_error_string(code: int) -> str:
+    return load_library().tq4_1s_error_string(code).decode()
+
+
+def tq4_1s_packed_bytes(n: int, k: int, num_experts: int = 1):
+    c, s = ctypes.c_size_t(), ctypes.c_size_t()
+    _check(load_library().tq4_1s_packed_bytes(n, k, num_experts, ctypes.byref(c), ctypes.byref(s)), "packed_bytes")
+    return c.value, s.value
+
+
+def tq4_1s_sign_mask(seed: int) -> int:
+    m = ctypes.c_uint32()
+    _check(load_library().tq4_1s_sign_mask(seed, ctypes.byref(m)), "sign_mask")
+    return m.value
+
+
+def tq4_1s_codebook():
+    """(levels[16], thresholds[15]) as float32 CPU tensors, as the kernels use them."""
+    lv = torch.zeros(16, dtype=torch.float32)
+    th = torch.zeros(15, dtype=torch.float32)
+    _check(load_library().tq4_1s_codebook(_ptr(lv), _ptr(th)), "codebook")
+    return lv, th
+
+
+def _empty_packed(n: int, k: int, num_experts: int, seed: int, device) -> Packed:
+    cb, sb = tq4_1s_packed_bytes(n, k, num_experts)
+    codes = torch.empty(cb, dtype=torch.uint8, device=device).view(num_experts, n, k // 2)
+    scales = torch.empty(sb // 2, dtype=torch.int16, device=device).view(num_experts, n, k // 16)
+    return Packed(codes, scales, n, k, num_experts, seed)
+
+
+def tq4_1s_quantize(W: torch.Tensor, seed: int, out: Packed | None = None) -> Packed:
+    """Quantize W ([n][k] or [E][n][k], float32 or bfloat16, CUDA) to TQ4_1S."""
+    if W.dim() == 2:
+        W = W.unsqueeze(0)
+    if W.dim() != 3 or not W.is_cuda or W.dtype not in (torch.float32, torch.bfloat16):
+        raise ValueError("W must be a CUDA float32/bfloat16 tensor of shape [n][k] or [E][n][k]")
+    W = W.contiguous()
+    E, n, k = W.shape
+    if out is None:
+        out = _empty_packed(n, k, E, seed, W.device)
+    dt = TQ_DTYPE_F32 if W.dtype == torch.float32 else TQ_DTYPE_BF16
+    ws = out.c_struct()
+    _check(load_library().tq4_1s_quantize(_ptr(W), dt, ctypes.byref(ws), _stream(W.device)), "quantize")
+    return out
+
+
+def tq4_1s_dequantize(w: Packed) -> torch.Tensor:
+    out = torch.empty((w.num_experts, w.n, w.k), dtype=torch.float32, device=w.codes.device)
+    ws = w.c_struct()
+    _check(load_library().tq4_1s_dequantize(ctypes.byref(ws), _ptr(out), _stream(out.device)), "dequantize")
+    return out
+
+
+_ws_cache: dict = {}
+
+
+def _workspace(nbytes: int, device) -> torch.Tensor:
+    key = (str(device),)
+    buf = _ws_cache.get(key)
+    if buf is None or buf.numel() < nbytes:
+        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        _ws_cache[key] = buf
+    return buf
+
+
+def tq4_1s_linear_workspace(m: int, w: Packed) -> int:
+    ws = w.c_struct()
+    return load_library().tq4_1s_linear_workspace(m, ctypes.byref(ws))
+
+
+def tq4_1s_linear(x: torch.Tensor, w: Packed, out: torch.Tensor | None = None,
+                  workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """y = bf16(x @ W_hat^T) for x bfloat16 [m][k] on CUDA."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a CUDA bfloat16 [m][k] tensor")
+    x = x.contiguous()
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device)
+    wst = w.c_struct()
+    need = load_library().tq4_1s_linear_workspace(m, ctypes.byref(wst))
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    _check(load_library().tq4_1s_linear(_ptr(x), m, ctypes.byref(wst), _ptr(out), _ptr(workspace),
+                                        workspace.numel(), _stream(x.device)), "linear")
+    return out
+
+
+def tq4_1s_moe_workspace(m: int, topk: int, up: Packed, down: Packed) -> int:
+    u, d = up.c_struct(), down.c_struct()
+    return load_library().tq4_1s_moe_workspace(m, topk, ctypes.byref(u), ctypes.byref(d))
+
+
+def tq4_1s_moe(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, up: Packed, down: Packed,
+               out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """Sync-free MoE: y_t = bf16(sum_j w_tj * down_e(bf16(relu(up_e(x_t))^2)))."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a CUDA bfloat16 [m][H] tensor")
+    x = x.contiguous()
+    topk_ids = topk_ids.to(torch.int32).contiguous()
+    topk_w = topk_w.to(torch.float32).contiguous()
+    m, topk = topk_ids.shape
+    if out is None:
+        out = torch.empty((m, up.k), dtype=torch.bfloat16, device=x.device)
+    u, d = up.c_struct(), down.c_struct()
+    need = load_library().tq4_1s_moe_workspace(m, topk, ctypes.byref(u), ctypes.byref(d))
+    if workspace is None:
+        workspace = _workspace(need, x.device)
+    _check(load_library().tq4_1s_moe(_ptr(x), m, _ptr(topk_ids), _ptr(topk_w), topk, ctypes.byref(u),
+                                     ctypes.byref(d), _ptr(out), _ptr(workspace), workspace.numel(),
+                                     _stream(x.device)), "moe")
+    return out
+
+
+def tq4_1s_moe_route(topk_ids: torch.Tensor, num_experts: int):
+    """(offsets [E+1], pairs [m*topk]) -- the routing step of tq4_1s_moe."""
+    topk_ids = topk_ids.to(torch.int32).contiguous()
+    m, topk = topk_ids.shape
+    offsets = torch.empty(num_experts + 1, dtype=torch.int32, device=topk_ids.device)
+    pairs = torch.empty(m * topk, dtype=torch.int32, device=topk_ids.device)
+    _check(load_library().tq4_1s_moe_route(_ptr(topk_ids), m, topk, num_experts, _ptr(offsets), _ptr(pairs),
+                                           _stream(topk_ids.device)), "moe_route")
+    return offsets, pairs
+
+
+def tq4_1s_get_status(device=None) -> int:
+    """Synchronize the current stream and read-and-clear the device status word."""
+    s = ctypes.c_int32()
+    _check(load_library().tq4_1s_get_status(_stream(device), ctypes.byref(s)), "get_status")
+    return s.value

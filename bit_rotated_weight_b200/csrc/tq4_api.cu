@@ -1,0 +1,484 @@
+// Host side of libtq4_1s.so: the extern "C" entry points declared in
+// include/tq4_1s.h -- argument validation, the codebook, the RHT sign mask,
+// TMA tensor-map construction and the launch sequences of each call.
+#include <cmath>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+
+#include "tq4_internal.h"
+
+#define TQ_API extern "C" __attribute__((visibility("default")))
+
+namespace tq4 {
+
+// ------------------------------------------------------------------ codebook
+// 16-level Lloyd-Max quantizer of N(0,1) ("16-level Lloyd-Max", model card
+// section "What Config-I means").  The quantizer of a symmetric density is
+// odd-symmetric, so only the 8 positive levels m_0 < ... < m_7 are iterated,
+// with interval edges b_0 = 0, b_j = (m_{j-1} + m_j) / 2, b_8 = +inf and the
+// centroid update m_j = E[X | b_j < X < b_{j+1}].
+static CodebookF32 compute_codebook() {
+  const double inv_sqrt2 = 0.70710678118654752440;
+  const double inv_sqrt2pi = 0.39894228040143267794;
+  auto pdf = [&](double x) { return std::isinf(x) ? 0.0 : inv_sqrt2pi * std::exp(-0.5 * x * x); };
+  auto upper_tail = [&](double x) { return std::isinf(x) ? 0.0 : 0.5 * std::erfc(x * inv_sqrt2); };  // P(X > x)
+  double mlev[8];
+  for (int j = 0; j < 8; ++j) mlev[j] = 0.35 * (j + 0.5);
+  for (int iter = 0; iter < 100000; ++iter) {
+    double edge[9];
+    edge[0] = 0.0;
+    for (int j = 1; j < 8; ++j) edge[j] = 0.5 * (mlev[j - 1] + mlev[j]);
+    edge[8] = INFINITY;
+    double change = 0.0;
+    for (int j = 0; j < 8; ++j) {
+      const double mass = upper_tail(edge[j]) - upper_tail(edge[j + 1]);
+      const double next = (pdf(edge[j]) - pdf(edge[j + 1])) / mass;
+      change = std::fmax(change, std::fabs(next - mlev[j]));
+      mlev[j] = next;
+    }
+    if (change < 1e-14) break;
+  }
+  CodebookF32 cb{};
+  for (int j = 0; j < 8; ++j) {
+    cb.levels[8 + j] = static_cast<float>(mlev[j]);
+    cb.levels[7 - j] = -static_cast<float>(mlev[j]);
+  }
+  cb.thresholds[7] = 0.0f;
+  for (int j = 1; j < 8; ++j) {
+    const float tj = static_cast<float>(0.5 * (mlev[j - 1] + mlev[j]));
+    cb.thresholds[7 + j] = tj;
+    cb.thresholds[7 - j] = -tj;
+  }
+  cb.thresholds[15] = INFINITY;
+  return cb;
+}
+
+const CodebookF32& codebook() {
+  static const CodebookF32 cb = compute_codebook();
+  return cb;
+}
+
+// SplitMix64 (Steele, Lea, Flood, OOPSLA 2014): first output from `state`.
+static uint32_t sign_mask_of(uint64_t state) {
+  uint64_t z = state + 0x9E3779B97F4A7C15ull;
+  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
+  z ^= z >> 31;
+  return static_cast<uint32_t>(z);
+}
+
+// ------------------------------------------------------------------ helpers
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct DeviceInfo {
+  int ok = -1;   // -1 unknown, 0 unsupported, 1 sm_100
+  int sms = 0;
+};
+
+static int check_device(int* sms_out) {
+  static std::mutex mu;
+  static DeviceInfo info[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return TQ_ERR_UNSUPPORTED_DEVICE;
+  }
+  std::lock_guard<std::mutex> g(mu);
+  if (info[dev].ok < 0) {
+    int major = 0, minor = 0, sms = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+      cudaGetLastError();
+      return TQ_ERR_UNSUPPORTED_DEVICE;
+    }
+    info[dev].ok = (major == 10 && minor == 0) ? 1 : 0;
+    info[dev].sms = sms;
+  }
+  if (info[dev].ok != 1) return TQ_ERR_UNSUPPORTED_DEVICE;
+  if (sms_out) *sms_out = info[dev].sms;
+  return TQ_OK;
+}
+
+static int weight_ok(const tq4_1s_weight* w, bool need_ptrs) {
+  if (!w) return TQ_ERR_INVALID_ARG;
+  if (w->n <= 0 || w->k <= 0 || (w->k % 32) != 0 || w->num_experts <= 0 || w->reserved != 0)
+    return TQ_ERR_INVALID_ARG;
+  if (w->n > (1ll << 30) || w->k > (1ll << 30) || w->num_experts > (1 << 20)) return TQ_ERR_INVALID_ARG;
+  if (need_ptrs) {
+    if (!w->codes || !w->scales) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(w->codes) || !aligned16(w->scales)) return TQ_ERR_ALIGNMENT;
+  }
+  return TQ_OK;
+}
+
+// cuTensorMapEncodeTiled through the runtime's driver entry point, so the
+// library does not link libcuda directly.
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+    else
+      cudaGetLastError();
+  });
+  return fn;
+}
+
+static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const void* base, const uint64_t* dims,
+                     const uint64_t* strides_bytes, const uint32_t* box, CUtensorMapSwizzle sw) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t gd[3], gs[2];
+  cuuint32_t bx[3], es[3];
+  for (int i = 0; i < rank; ++i) {
+    gd[i] = dims[i];
+    bx[i] = box[i];
+    es[i] = 1;
+  }
+  for (int i = 0; i < rank - 1; ++i) gs[i] = strides_bytes[i];
+  CUresult r = fn(m, dt, static_cast<cuuint32_t>(rank), const_cast<void*>(base), gd, gs, bx, es,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// Codes plane [E][n][k/2] bytes, box 64 B x 128 rows, 64-byte swizzle.
+static bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
+  const uint64_t dims[3] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n),
+                            static_cast<uint64_t>(w->num_experts)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n * (w->k / 2))};
+  const uint32_t box[3] = {64, 128, 1};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+}
+
+// bf16 matrix [rows][cols] row-major, box 64 x box_rows, 128-byte swizzle.
+static bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(cols * 2)};
+  const uint32_t box[2] = {64, box_rows};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+// Small-m path threshold: up to this many rows, the stream-K kernel streams
+// the packed weight once per 32-row segment; above it, dequantize + GEMM.
+constexpr int64_t kSmallM = 128;
+
+struct SmallLayout {
+  size_t xh, xl, partials, counters, total;
+  int grid;
+  int64_t tiles;
+};
+
+static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
+  SmallLayout L{};
+  const int64_t nseg = (m + kSegRows - 1) / kSegRows;
+  const int64_t rt = (w->n + 127) / 128, ki = (w->k + 127) / 128;
+  L.tiles = nseg * rt;
+  const int64_t T = L.tiles * ki;
+  L.grid = static_cast<int>(T < sms ? T : sms);
+  size_t off = 0;
+  L.xh = off;
+  off = align256(off + static_cast<size_t>(m * w->k) * 2);
+  L.xl = off;
+  off = align256(off + static_cast<size_t>(m * w->k) * 2);
+  L.partials = off;
+  off = align256(off + static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
+  L.counters = off;
+  off = align256(off + static_cast<size_t>(L.tiles) * 4);
+  L.total = off;
+  return L;
+}
+
+struct MoeLayout {
+  size_t offsets, pairs, segs, nseg, npv, xh, xl, hh, hl, zw, partials, cnt_up, cnt_dn, total;
+  int64_t P, maxseg, rt_up, rt_dn;
+};
+
+static MoeLayout moe_layout(int64_t m, int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* dn, int sms) {
+  MoeLayout L{};
+  const int64_t E = up->num_experts;
+  const int64_t H = up->k, I = up->n;
+  L.P = m * topk;
+  L.maxseg = (L.P + kSegRows - 1) / kSegRows + (E < L.P ? E : L.P) + 1;
+  L.rt_up = (I + 127) / 128;
+  L.rt_dn = (dn->n + 127) / 128;
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.offsets = take((E + 1) * 4);
+  L.pairs = take(L.P * 4);
+  L.segs = take(L.maxseg * 16);
+  L.nseg = take(4);
+  L.npv = take(4);
+  L.xh = take(L.P * H * 2);
+  L.xl = take(L.P * H * 2);
+  L.hh = take(L.P * I * 2);
+  L.hl = take(L.P * I * 2);
+  L.zw = take(L.P * H * 4);
+  L.partials = take(static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
+  L.cnt_up = take(L.maxseg * L.rt_up * 4);
+  L.cnt_dn = take(L.maxseg * L.rt_dn * 4);
+  L.total = off;
+  return L;
+}
+
+static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUDA; }
+
+}  // namespace tq4
+
+using namespace tq4;
+
+// ==================================================================== ABI
+TQ_API int tq4_1s_version(void) { return 100; }
+
+TQ_API const char* tq4_1s_error_string(int code) {
+  switch (code) {
+    case TQ_OK: return "ok";
+    case TQ_ERR_INVALID_ARG: return "invalid argument";
+    case TQ_ERR_ALIGNMENT: return "pointer not 16-byte aligned";
+    case TQ_ERR_UNSUPPORTED_DEVICE: return "current device is not an sm_100 (B200) GPU";
+    case TQ_ERR_WORKSPACE: return "workspace missing or too small";
+    case TQ_ERR_CUDA: return "CUDA call failed";
+    case TQ_ERR_TIMEOUT: return "a bounded device wait timed out";
+    case TQ_ERR_BAD_ROUTING: return "routing expert id out of range";
+    case TQ_ERR_NONFINITE: return "non-finite value in quantize input";
+    default: return "unknown error code";
+  }
+}
+
+TQ_API int tq4_1s_packed_bytes(int64_t n, int64_t k, int32_t num_experts, size_t* codes_bytes,
+                               size_t* scales_bytes) {
+  if (n <= 0 || k <= 0 || k % 32 != 0 || num_experts <= 0 || !codes_bytes || !scales_bytes) return TQ_ERR_INVALID_ARG;
+  *codes_bytes = static_cast<size_t>(num_experts) * static_cast<size_t>(n) * static_cast<size_t>(k / 2);
+  *scales_bytes = static_cast<size_t>(num_experts) * static_cast<size_t>(n) * static_cast<size_t>(k / 16) * 2;
+  return TQ_OK;
+}
+
+TQ_API int tq4_1s_sign_mask(uint64_t seed, uint32_t* mask) {
+  if (!mask) return TQ_ERR_INVALID_ARG;
+  *mask = sign_mask_of(seed);
+  return TQ_OK;
+}
+
+TQ_API int tq4_1s_codebook(float* levels, float* thresholds) {
+  const CodebookF32& cb = codebook();
+  if (levels) std::memcpy(levels, cb.levels, sizeof(float) * 16);
+  if (thresholds) std::memcpy(thresholds, cb.thresholds, sizeof(float) * 15);
+  return TQ_OK;
+}
+
+TQ_API int tq4_1s_quantize(const void* W, int dtype, const tq4_1s_weight* out, tq4_stream_t stream) {
+  int rc = weight_ok(out, true);
+  if (rc) return rc;
+  if (!W || (dtype != TQ_DTYPE_F32 && dtype != TQ_DTYPE_BF16)) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(W)) return TQ_ERR_ALIGNMENT;
+  if ((rc = check_device(nullptr))) return rc;
+  const int64_t rows = out->n * out->num_experts;
+  return cuda_rc(launch_quantize(W, dtype, out->codes, out->scales, rows, out->k, sign_mask_of(out->seed),
+                                 codebook(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+TQ_API int tq4_1s_dequantize(const tq4_1s_weight* w, float* W_out, tq4_stream_t stream) {
+  int rc = weight_ok(w, true);
+  if (rc) return rc;
+  if (!W_out) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(W_out)) return TQ_ERR_ALIGNMENT;
+  if ((rc = check_device(nullptr))) return rc;
+  return cuda_rc(launch_dequantize_f32(w->codes, w->scales, W_out, w->n * w->num_experts, w->k,
+                                       sign_mask_of(w->seed), codebook(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int sms_or_default() {
+  int sms = 148;
+  if (check_device(&sms) != TQ_OK) sms = 148;
+  return sms;
+}
+
+TQ_API size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w) {
+  if (m < 0 || weight_ok(w, false) != TQ_OK || w->num_experts != 1) return 0;
+  if (m == 0) return 0;
+  if (m <= kSmallM) return small_layout(m, w, sms_or_default()).total;
+  return align256(static_cast<size_t>(w->n) * static_cast<size_t>(w->k) * 2);
+}
+
+TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, void* ws,
+                         size_t ws_bytes, tq4_stream_t stream) {
+  int rc = weight_ok(w, true);
+  if (rc) return rc;
+  if (w->num_experts != 1 || m < 0 || m > (1ll << 24)) return TQ_ERR_INVALID_ARG;
+  if (m == 0) return TQ_OK;
+  if (!x || !y) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return TQ_ERR_ALIGNMENT;
+  int sms = 0;
+  if ((rc = check_device(&sms))) return rc;
+  const size_t need = tq4_1s_linear_workspace(m, w);
+  if (!ws || ws_bytes < need) return TQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const uint32_t mask = sign_mask_of(w->seed);
+
+  if (m <= kSmallM) {
+    const SmallLayout L = small_layout(m, w, sms);
+    uint16_t* xh = reinterpret_cast<uint16_t*>(base + L.xh);
+    uint16_t* xl = reinterpret_cast<uint16_t*>(base + L.xl);
+    int32_t* counters = reinterpret_cast<int32_t*>(base + L.counters);
+    cudaError_t e = launch_rotate_act(x, w->k, nullptr, 1, nullptr, m, m, xh, xl, mask, counters, L.tiles, st);
+    if (e != cudaSuccess) return TQ_ERR_CUDA;
+    alignas(64) CUtensorMap tc, th, tl;
+    if (!map_codes(&tc, w) || !map_bf16(&th, xh, m, w->k, 16) || !map_bf16(&tl, xl, m, w->k, 16))
+      return TQ_ERR_CUDA;
+    StreamKArgs a{};
+    a.n = static_cast<int32_t>(w->n);
+    a.k = static_cast<int32_t>(w->k);
+    a.row_tiles = static_cast<int32_t>((w->n + 127) / 128);
+    a.k_iters = static_cast<int32_t>((w->k + 127) / 128);
+    a.nseg_host = static_cast<int32_t>((m + kSegRows - 1) / kSegRows);
+    a.m_host = static_cast<int32_t>(m);
+    a.scales = w->scales;
+    a.mode = EPI_DENSE;
+    a.out_a = y;
+    a.partials = reinterpret_cast<float*>(base + L.partials);
+    a.counters = counters;
+    a.max_tiles = static_cast<int32_t>(L.tiles);
+    return cuda_rc(launch_streamk(&tc, &th, &tl, a, L.grid, st));
+  }
+  // large m: W_hat in bf16, then the tensor-core GEMM
+  uint16_t* wh = reinterpret_cast<uint16_t*>(base);
+  cudaError_t e = launch_dequantize_bf16(w->codes, w->scales, wh, w->n, w->k, mask, codebook(), st);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+  alignas(64) CUtensorMap tx, tw;
+  if (!map_bf16(&tx, x, m, w->k, 128) || !map_bf16(&tw, wh, w->n, w->k, 256)) return TQ_ERR_CUDA;
+  const int64_t tiles = ((m + 127) / 128) * ((w->n + 255) / 256);
+  const int grid = static_cast<int>(tiles < sms ? tiles : sms);
+  return cuda_rc(launch_gemm_bf16(&tx, &tw, y, static_cast<int32_t>(m), static_cast<int32_t>(w->n),
+                                  static_cast<int32_t>(w->k), grid, st));
+}
+
+static int moe_check(int64_t m, int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* down, bool ptrs) {
+  int rc = weight_ok(up, ptrs);
+  if (rc) return rc;
+  if ((rc = weight_ok(down, ptrs))) return rc;
+  if (m < 0 || topk <= 0 || topk > 64 || m * topk > (1ll << 26)) return TQ_ERR_INVALID_ARG;
+  if (up->num_experts != down->num_experts || up->k != down->n || up->n != down->k) return TQ_ERR_INVALID_ARG;
+  if (up->num_experts > 4096) return TQ_ERR_INVALID_ARG;
+  return TQ_OK;
+}
+
+TQ_API size_t tq4_1s_moe_workspace(int64_t m, int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* down) {
+  if (moe_check(m, topk, up, down, false) != TQ_OK) return 0;
+  if (m == 0) return 0;
+  return moe_layout(m, topk, up, down, sms_or_default()).total;
+}
+
+TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, const float* topk_w, int32_t topk,
+                      const tq4_1s_weight* up, const tq4_1s_weight* down, uint16_t* y, void* ws, size_t ws_bytes,
+                      tq4_stream_t stream) {
+  int rc = moe_check(m, topk, up, down, true);
+  if (rc) return rc;
+  if (m == 0) return TQ_OK;
+  if (!x || !topk_ids || !topk_w || !y) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y) || !aligned16(topk_ids) || !aligned16(topk_w)) return TQ_ERR_ALIGNMENT;
+  int sms = 0;
+  if ((rc = check_device(&sms))) return rc;
+  const MoeLayout L = moe_layout(m, topk, up, down, sms);
+  if (!ws || ws_bytes < L.total) return TQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint8_t* base = static_cast<uint8_t*>(ws);
+  const int64_t E = up->num_experts, H = up->k, I = up->n;
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + L.offsets);
+  int32_t* pairs = reinterpret_cast<int32_t*>(base + L.pairs);
+  int4* segs = reinterpret_cast<int4*>(base + L.segs);
+  int32_t* nseg = reinterpret_cast<int32_t*>(base + L.nseg);
+  int32_t* npv = reinterpret_cast<int32_t*>(base + L.npv);
+  uint16_t* xh = reinterpret_cast<uint16_t*>(base + L.xh);
+  uint16_t* xl = reinterpret_cast<uint16_t*>(base + L.xl);
+  uint16_t* hh = reinterpret_cast<uint16_t*>(base + L.hh);
+  uint16_t* hl = reinterpret_cast<uint16_t*>(base + L.hl);
+  float* zw = reinterpret_cast<float*>(base + L.zw);
+  int32_t* cnt_up = reinterpret_cast<int32_t*>(base + L.cnt_up);
+  const int64_t ncnt = L.maxseg * (L.rt_up + L.rt_dn);   // cnt_up and cnt_dn are contiguous
+  cudaError_t e = launch_moe_route(topk_ids, L.P, static_cast<int32_t>(E), offsets, pairs, segs, nseg, kSegRows,
+                                   npv, cnt_up, ncnt, st);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+  e = launch_rotate_act(x, H, pairs, topk, npv, 0, L.P, xh, xl, sign_mask_of(up->seed), nullptr, 0, st);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
+
+  alignas(64) CUtensorMap tcu, txh, txl, tcd, thh, thl;
+  if (!map_codes(&tcu, up) || !map_bf16(&txh, xh, L.P, H, 16) || !map_bf16(&txl, xl, L.P, H, 16) ||
+      !map_codes(&tcd, down) || !map_bf16(&thh, hh, L.P, I, 16) || !map_bf16(&thl, hl, L.P, I, 16))
+    return TQ_ERR_CUDA;
+  StreamKArgs a{};
+  a.n = static_cast<int32_t>(I);
+  a.k = static_cast<int32_t>(H);
+  a.row_tiles = static_cast<int32_t>(L.rt_up);
+  a.k_iters = static_cast<int32_t>((H + 127) / 128);
+  a.segs = segs;
+  a.nseg_dev = nseg;
+  a.scales = up->scales;
+  a.mode = EPI_UP;
+  a.out_a = hh;
+  a.out_b = hl;
+  a.next_mask = sign_mask_of(down->seed);
+  a.partials = reinterpret_cast<float*>(base + L.partials);
+  a.counters = cnt_up;
+  a.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_up);
+  if ((e = launch_streamk(&tcu, &txh, &txl, a, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
+
+  StreamKArgs b = a;
+  b.n = static_cast<int32_t>(H);
+  b.k = static_cast<int32_t>(I);
+  b.row_tiles = static_cast<int32_t>(L.rt_dn);
+  b.k_iters = static_cast<int32_t>((I + 127) / 128);
+  b.scales = down->scales;
+  b.mode = EPI_DOWN;
+  b.out_a = nullptr;
+  b.out_b = nullptr;
+  b.out_f = zw;
+  b.pairs = pairs;
+  b.topk_w = topk_w;
+  b.counters = reinterpret_cast<int32_t*>(base + L.cnt_dn);
+  b.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_dn);
+  if ((e = launch_streamk(&tcd, &thh, &thl, b, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
+  return cuda_rc(launch_moe_combine(zw, topk_ids, m, topk, H, static_cast<int32_t>(E), y, st));
+}
+
+TQ_API int tq4_1s_moe_route(const int32_t* topk_ids, int64_t m, int32_t topk, int32_t num_experts, int32_t* offsets,
+                            int32_t* pairs, tq4_stream_t stream) {
+  if (m < 0 || topk <= 0 || num_experts <= 0 || num_experts > 4096 || m * topk > (1ll << 26))
+    return TQ_ERR_INVALID_ARG;
+  if (!topk_ids || !offsets || !pairs) return TQ_ERR_INVALID_ARG;
+  int rc = check_device(nullptr);
+  if (rc) return rc;
+  return cuda_rc(launch_moe_route(topk_ids, m * topk, num_experts, offsets, pairs, nullptr, nullptr, kSegRows,
+                                  nullptr, nullptr, 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+TQ_API int tq4_1s_get_status(tq4_stream_t stream, int32_t* status) {
+  if (!status) return TQ_ERR_INVALID_ARG;
+  int rc = check_device(nullptr);
+  if (rc) return rc;
+  if (cudaStreamSynchronize(reinterpret_cast<cudaStream_t>(stream)) != cudaSuccess) return TQ_ERR_CUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_status, sizeof(int)) != cudaSuccess) return TQ_ERR_CUDA;
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(g_status, &zero, sizeof(int)) != cudaSuccess) return TQ_ERR_CUDA;
+  *status = v;
+  return TQ_OK;
+}

@@ -1,0 +1,75 @@
+// Internal declarations shared by the library's translation units.
+#pragma once
+#include <cstdint>
+#include <cuda_runtime.h>
+
+#include "tq4_common.cuh"
+
+namespace tq4 {
+
+// The fp32 codebook handed to kernels by value (kernel parameter space).
+struct CodebookF32 {
+  float levels[16];       // ascending, levels[15 - j] == -levels[j]
+  float thresholds[16];   // 15 used: midpoints of adjacent levels
+};
+
+// Host-side codebook computation (Lloyd iteration), run once per process.
+const CodebookF32& codebook();
+
+// One segment of rows of the rotated activations multiplied by one expert:
+// x = expert, y = first row, z = row count (<= kSegRows), w unused.
+constexpr int kSegRows = 32;
+
+cudaError_t launch_quantize(const void* W, int dtype, uint8_t* codes, uint16_t* scales, int64_t rows, int64_t k,
+                            uint32_t mask, const CodebookF32& cb, cudaStream_t st);
+cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, float* out, int64_t rows, int64_t k,
+                                  uint32_t mask, const CodebookF32& cb, cudaStream_t st);
+cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales, uint16_t* out, int64_t rows,
+                                   int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st);
+cudaError_t launch_rotate_act(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
+                              const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
+                              uint16_t* xh, uint16_t* xl, uint32_t mask, int32_t* zero_ptr, int64_t nzero,
+                              cudaStream_t st);
+cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
+                             int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
+                             int32_t* zero_ptr, int64_t nzero, cudaStream_t st);
+cudaError_t launch_moe_combine(const float* zw, const int32_t* ids, int64_t m, int32_t topk, int64_t h,
+                               int32_t num_experts, uint16_t* y, cudaStream_t st);
+
+// ---------------------------------------------------------------- stream-K
+enum EpilogueMode : int32_t { EPI_DENSE = 0, EPI_UP = 1, EPI_DOWN = 2 };
+
+struct StreamKArgs {
+  int32_t n, k;              // rows / columns of one expert's weight
+  int32_t row_tiles;         // ceil(n / 128)
+  int32_t k_iters;           // ceil(k / 128)
+  int32_t nseg_host;         // segment count when segs == nullptr (dense): ceil(m / kSegRows)
+  int32_t m_host;            // dense row count
+  const int4* segs;          // device segment list (MoE) or nullptr
+  const int32_t* nseg_dev;   // device segment count (MoE) or nullptr
+  const uint16_t* scales;    // [E][n][k/16]
+  int32_t mode;              // EpilogueMode
+  uint16_t* out_a;           // dense: y [m][n]; up: next-stage hi [P][n]
+  uint16_t* out_b;           // up: next-stage lo [P][n]
+  float* out_f;              // down: z*w [m*topk][n]
+  const int32_t* pairs;      // MoE: flat slot index of each sorted row
+  const float* topk_w;       // MoE: router weights (flat)
+  uint32_t next_mask;        // up: sign mask of the down projection
+  float* partials;           // [grid][2][128][kSegRows]
+  int32_t* counters;         // [tiles]
+  int32_t max_tiles;         // capacity of counters
+};
+
+// Bytes of dynamic shared memory the stream-K kernel uses.
+size_t streamk_smem_bytes();
+
+cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void* tm_xlo, const StreamKArgs& a,
+                           int grid, cudaStream_t st);
+
+// ---------------------------------------------------------------- GEMM
+// y[m][n] = bf16( x[m][k] * w[n][k]^T ), bf16 operands via TMA tensor maps.
+cudaError_t launch_gemm_bf16(const void* tm_x, const void* tm_w, uint16_t* y, int32_t m, int32_t n, int32_t k,
+                             int grid, cudaStream_t st);
+size_t gemm_smem_bytes();
+
+}  // namespace tq4

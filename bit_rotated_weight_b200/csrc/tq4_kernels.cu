@@ -1,0 +1,317 @@
+// TQ4_1S streaming kernels for sm_100a: quantize, dequantize, activation
+// rotation, and the MoE routing and combine steps.
+//
+// Format and arithmetic follow the Nemotron-TheHobbit-30B-A3B model card,
+// section "What Config-I means" (per-32-block RHT rotation, 16-level
+// Lloyd-Max codes, two half-block scales).  One warp handles one 32-element
+// block: lane i owns element i, and the 32-point butterfly runs in registers
+// through shfl_xor, stage h exchanging lanes i and i^h.
+#include "tq4_internal.h"
+
+namespace tq4 {
+
+__device__ int g_status = 0;
+
+// r = fp32(1/sqrt(32))
+__device__ __forceinline__ float rsqrt32() { return __uint_as_float(0x3E3504F3u); }
+
+// In-register 32-point Sylvester Hadamard butterfly across the warp
+// (stages h = 1, 2, 4, 8, 16): the lane with bit h clear keeps a + partner,
+// the other keeps partner - a.
+__device__ __forceinline__ float warp_fwht32(float a, int lane) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+    const float p = __shfl_xor_sync(0xFFFFFFFFu, a, h);
+    a = (lane & h) ? __fsub_rn(p, a) : __fadd_rn(a, p);
+  }
+  return a;
+}
+
+// fp32 -> fp16 bits, round to nearest even, saturating at 65504, NaN -> 0x7E00.
+__device__ __forceinline__ uint16_t f16_sat_bits(float x) {
+  if (x != x) return 0x7E00u;
+  const float ax = fabsf(x);
+  if (ax >= 65520.0f) return (x < 0.0f) ? 0xFBFFu : 0x7BFFu;
+  return __half_as_ushort(__float2half_rn(x));
+}
+
+// ------------------------------------------------------------------ quantize
+template <typename T>
+__device__ __forceinline__ float load_w(const T* p);
+template <>
+__device__ __forceinline__ float load_w<float>(const float* p) { return __ldg(p); }
+template <>
+__device__ __forceinline__ float load_w<uint16_t>(const uint16_t* p) { return bf16_bits_to_f32(__ldg(p)); }
+
+template <typename T>
+__global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ W, uint8_t* __restrict__ codes,
+                                                       uint16_t* __restrict__ scales, int64_t rows, int64_t k,
+                                                       uint32_t mask, CodebookF32 cb) {
+  __shared__ float s_t[16];
+  if (threadIdx.x < 15) s_t[threadIdx.x] = cb.thresholds[threadIdx.x];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const float sgn_neg = ((mask >> lane) & 1u) ? -1.0f : 1.0f;
+  const int64_t kb_per_row = k / 32;
+  const int64_t nblocks = rows * kb_per_row;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const float r = rsqrt32();
+  for (int64_t b = warp; b < nblocks; b += nwarps) {
+    const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
+    const float w = load_w<T>(W + row * k + kb * 32 + lane);
+    if (__any_sync(0xFFFFFFFFu, !isfinite(w)) && lane == 0) raise_status(TQ_DEV_NONFINITE);
+    const float a = warp_fwht32(w * sgn_neg, lane);  // sign flip is exact
+    const float v = __fmul_rn(a, r);
+    // half-block mean square: pairwise tree with strides 8, 4, 2, 1
+    float p = __fmul_rn(v, v);
+#pragma unroll
+    for (int s = 8; s >= 1; s >>= 1) p = __fadd_rn(p, __shfl_down_sync(0xFFFFFFFFu, p, s, 16));
+    const float S = __shfl_sync(0xFFFFFFFFu, p, 0, 16);
+    const float rms = __fsqrt_rn(__fmul_rn(S, 0.0625f));
+    const uint16_t dbits = f16_sat_bits(rms);
+    const float d = __half2float(__ushort_as_half(dbits));
+    uint32_t code;
+    if (d == 0.0f) {
+      code = 7u;
+    } else {
+      const float u = __fdiv_rn(v, d);
+      // number of thresholds strictly below u (binary search over sorted t)
+      code = 0u;
+      code += (u > s_t[7]) ? 8u : 0u;
+      code += (u > s_t[code + 3]) ? 4u : 0u;
+      code += (u > s_t[code + 1]) ? 2u : 0u;
+      code += (u > s_t[code]) ? 1u : 0u;
+    }
+    // pack: byte i/2 <- code(2i) | code(2i+1) << 4 ; 16 bytes per block
+    const uint32_t hi = __shfl_down_sync(0xFFFFFFFFu, code, 1);
+    const uint32_t byte = code | (hi << 4);
+    const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, byte, 2);
+    const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, byte, 4);
+    const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, byte, 6);
+    const uint32_t word = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);  // valid on lanes 0, 8, 16, 24
+    const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, word, 8);
+    const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, word, 16);
+    const uint32_t w3 = __shfl_sync(0xFFFFFFFFu, word, 24);
+    const uint32_t d1 = __shfl_sync(0xFFFFFFFFu, static_cast<uint32_t>(dbits), 16);
+    if (lane == 0) {
+      *reinterpret_cast<uint4*>(codes + row * (k / 2) + kb * 16) = make_uint4(word, w1, w2, w3);
+      *reinterpret_cast<uint32_t*>(scales + row * (k / 16) + kb * 2) = static_cast<uint32_t>(dbits) | (d1 << 16);
+    }
+  }
+}
+
+// ------------------------------------------------------------------ dequantize
+// W_hat = diag(s) * r * H * (c[code] * d), fp32 or bf16 output.
+template <typename TO>
+__global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                         const uint16_t* __restrict__ scales, TO* __restrict__ out,
+                                                         int64_t rows, int64_t k, uint32_t mask, CodebookF32 cb) {
+  __shared__ float s_c[16];
+  if (threadIdx.x < 16) s_c[threadIdx.x] = cb.levels[threadIdx.x];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const bool neg = (mask >> lane) & 1u;
+  const int64_t kb_per_row = k / 32;
+  const int64_t nblocks = rows * kb_per_row;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const float r = rsqrt32();
+  for (int64_t b = warp; b < nblocks; b += nwarps) {
+    const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
+    const uint32_t byte = __ldg(codes + row * (k / 2) + kb * 16 + (lane >> 1));
+    const uint32_t code = (lane & 1) ? (byte >> 4) : (byte & 0xFu);
+    const float d = __half2float(__ushort_as_half(__ldg(scales + row * (k / 16) + kb * 2 + (lane >> 4))));
+    const float wn = __fmul_rn(s_c[code], d);
+    const float a = __fmul_rn(warp_fwht32(wn, lane), r);
+    const float o = neg ? -a : a;
+    if constexpr (sizeof(TO) == 4) {
+      out[row * k + kb * 32 + lane] = o;
+    } else {
+      out[row * k + kb * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+    }
+  }
+}
+
+// ------------------------------------------------------------------ activations
+// x' = r * H * diag(s) * x per 32-slice, split into bf16 hi = bf16(x') and
+// lo = bf16(x' - hi).  Row r of the outputs takes x row gather[r] / topk when a
+// gather list is given (MoE: rows in expert order), else row r.  Rows in
+// [rows_valid, rows_alloc) are zero-filled.  Also zeroes `nzero` ints at
+// `zero_ptr` (stream-K tile counters of the launches that follow).
+__global__ void __launch_bounds__(256) rotate_act_kernel(const uint16_t* __restrict__ x, int64_t k,
+                                                         const int32_t* __restrict__ gather, int32_t topk,
+                                                         const int32_t* __restrict__ rows_valid_dev,
+                                                         int64_t rows_valid_host, int64_t rows_alloc,
+                                                         uint16_t* __restrict__ xh, uint16_t* __restrict__ xl,
+                                                         uint32_t mask, int32_t* __restrict__ zero_ptr,
+                                                         int64_t nzero) {
+  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  for (int64_t i = tid; i < nzero; i += static_cast<int64_t>(gridDim.x) * blockDim.x) zero_ptr[i] = 0;
+  const int lane = threadIdx.x & 31;
+  const bool neg = (mask >> lane) & 1u;
+  const int64_t rows_valid = rows_valid_dev ? static_cast<int64_t>(*rows_valid_dev) : rows_valid_host;
+  const int64_t kb_per_row = k / 32;
+  const int64_t nblocks = rows_alloc * kb_per_row;
+  const int64_t warp = tid >> 5;
+  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  const float r = rsqrt32();
+  for (int64_t b = warp; b < nblocks; b += nwarps) {
+    const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
+    const int64_t off = row * k + kb * 32 + lane;
+    if (row >= rows_valid) {
+      xh[off] = 0;
+      xl[off] = 0;
+      continue;
+    }
+    const int64_t src = gather ? static_cast<int64_t>(gather[row] / topk) : row;
+    const float xv = bf16_bits_to_f32(x[src * k + kb * 32 + lane]);
+    const float v = __fmul_rn(warp_fwht32(neg ? -xv : xv, lane), r);
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
+    xh[off] = __bfloat16_as_ushort(h);
+    xl[off] = __bfloat16_as_ushort(l);
+  }
+}
+
+// ------------------------------------------------------------------ MoE routing
+// One CTA: per-expert counts, exclusive prefix (offsets), and a stable
+// bucketing of flat slot indices p = t*topk + j by expert.  Stability comes
+// from assigning positions in p order: each thread handles a contiguous run
+// of p, and runs are ranked by a second pass over the per-thread counts.
+// Also writes (when the pointers are non-null) the segment list used by the
+// grouped stream-K launches -- chunks of at most `chunk` consecutive rows of
+// one expert -- the segment and valid-pair counts, and zeroes the stream-K
+// counters.
+__global__ void __launch_bounds__(1024) moe_route_kernel(const int32_t* __restrict__ ids, int64_t npairs,
+                                                         int32_t num_experts, int32_t* __restrict__ offsets,
+                                                         int32_t* __restrict__ pairs, int4* __restrict__ segs,
+                                                         int32_t* __restrict__ nseg_out, int32_t chunk,
+                                                         int32_t* __restrict__ npairs_valid,
+                                                         int32_t* __restrict__ zero_ptr, int64_t nzero) {
+  extern __shared__ int32_t sh[];
+  int32_t* cnt = sh;                       // [num_experts]
+  int32_t* base = sh + num_experts;        // [num_experts]
+  __shared__ int32_t s_bad;
+  const int tid = threadIdx.x;
+  for (int64_t i = tid; i < nzero; i += blockDim.x) zero_ptr[i] = 0;
+  for (int e = tid; e < num_experts; e += blockDim.x) cnt[e] = 0;
+  if (tid == 0) s_bad = 0;
+  __syncthreads();
+  for (int64_t p = tid; p < npairs; p += blockDim.x) {
+    const int e = ids[p];
+    if (e >= 0 && e < num_experts) atomicAdd(&cnt[e], 1);
+    else atomicAdd(&s_bad, 1);
+  }
+  __syncthreads();
+  if (tid == 0) {
+    int32_t run = 0, ns = 0;
+    for (int e = 0; e < num_experts; ++e) {
+      offsets[e] = run;
+      base[e] = run;
+      for (int32_t c = 0; c < cnt[e]; c += chunk) {
+        if (segs) segs[ns] = make_int4(e, run + c, min(chunk, cnt[e] - c), 0);
+        ++ns;
+      }
+      run += cnt[e];
+    }
+    offsets[num_experts] = run;
+    if (npairs_valid) *npairs_valid = run;
+    if (nseg_out) *nseg_out = ns;
+    if (s_bad) raise_status(TQ_DEV_BAD_ROUTING);
+  }
+  __syncthreads();
+  // Stable scatter by warp 0, 32 slots at a time in p order: lanes holding
+  // the same expert take consecutive positions in lane order.
+  if (tid < 32) {
+    const unsigned lt_mask = (1u << tid) - 1u;
+    for (int64_t p0 = 0; p0 < npairs; p0 += 32) {
+      const int64_t p = p0 + tid;
+      const int e = (p < npairs) ? ids[p] : -1;
+      const bool ok = e >= 0 && e < num_experts;
+      const int key = ok ? e : -1 - tid;   // invalid slots group with nobody
+      const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
+      const int rank = __popc(peers & lt_mask);
+      if (ok) pairs[base[e] + rank] = static_cast<int32_t>(p);
+      __syncwarp();
+      if (ok && rank == 0) base[e] += __popc(peers);
+      __syncwarp();
+    }
+  }
+}
+
+// y[t][n] = bf16( sum_j zw[t*topk + j][n] ) over slots with a valid expert id.
+__global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restrict__ zw, const int32_t* __restrict__ ids,
+                                                          int64_t m, int32_t topk, int64_t h, int32_t num_experts,
+                                                          uint16_t* __restrict__ y) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= m * h) return;
+  const int64_t t = i / h, n = i - t * h;
+  float s = 0.0f;
+  for (int j = 0; j < topk; ++j) {
+    const int64_t p = t * topk + j;
+    const int e = ids[p];
+    if (e >= 0 && e < num_experts) s = __fadd_rn(s, zw[p * h + n]);
+  }
+  y[i] = __bfloat16_as_ushort(__float2bfloat16_rn(s));
+}
+
+// ------------------------------------------------------------------ launchers
+static int grid_for(int64_t warps_needed, int threads) {
+  int64_t blocks = (warps_needed * 32 + threads - 1) / threads;
+  const int64_t cap = 148LL * 16;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return static_cast<int>(blocks);
+}
+
+cudaError_t launch_quantize(const void* W, int dtype, uint8_t* codes, uint16_t* scales, int64_t rows, int64_t k,
+                            uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
+  const int g = grid_for(rows * (k / 32), 256);
+  if (dtype == TQ_DTYPE_F32)
+    quantize_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(W), codes, scales, rows, k, mask, cb);
+  else
+    quantize_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(W), codes, scales, rows, k, mask, cb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, float* out, int64_t rows, int64_t k,
+                                  uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
+  dequantize_kernel<float><<<grid_for(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k, mask, cb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales, uint16_t* out, int64_t rows,
+                                   int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
+  dequantize_kernel<uint16_t><<<grid_for(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k, mask, cb);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rotate_act(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
+                              const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
+                              uint16_t* xh, uint16_t* xl, uint32_t mask, int32_t* zero_ptr, int64_t nzero,
+                              cudaStream_t st) {
+  int g = grid_for(rows_alloc * (k / 32), 256);
+  rotate_act_kernel<<<g, 256, 0, st>>>(x, k, gather, topk, rows_valid_dev, rows_valid_host, rows_alloc, xh, xl,
+                                       mask, zero_ptr, nzero);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
+                             int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
+                             int32_t* zero_ptr, int64_t nzero, cudaStream_t st) {
+  const size_t sh = sizeof(int32_t) * 2 * static_cast<size_t>(num_experts);
+  moe_route_kernel<<<1, 1024, sh, st>>>(ids, npairs, num_experts, offsets, pairs, segs, nseg, chunk, npairs_valid,
+                                        zero_ptr, nzero);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_moe_combine(const float* zw, const int32_t* ids, int64_t m, int32_t topk, int64_t h,
+                               int32_t num_experts, uint16_t* y, cudaStream_t st) {
+  const int64_t n = m * h;
+  const int g = static_cast<int>((n + 255) / 256);
+  moe_combine_kernel<<<g, 256, 0, st>>>(zw, ids, m, topk, h, num_experts, y);
+  return cudaGetLastError();
+}
+
+}  // namespace tq4

@@ -1,0 +1,177 @@
+/*
+ * tq4_1s.h -- C ABI of libtq4_1s.so, the B200 (sm_100a) TQ4_1S layer.
+ *
+ * TQ4_1S ("Config-I") is the weight format of the Nemotron-TheHobbit-30B-A3B
+ * model card, section "What Config-I means": each 32-element block of a
+ * weight row (along K) is rotated by a randomized Walsh-Hadamard transform,
+ * then coded with 4-bit indices into a fixed 16-level Lloyd-Max codebook of
+ * N(0,1), with two half-block scales -- about 5 bits per weight.  Section
+ * "Running it" swaps quantized Linears for an on-the-fly dequant layer;
+ * section "Performance" adds a sync-free MoE and bf16 tensor-core matmuls;
+ * section "The model underneath" gives the 128-expert, top-6 MoE.
+ *
+ * Format (readings of what the card leaves open):
+ *   - signs: s_i = -1 where bit i of sign_mask is set, one 32-sign vector per
+ *     tensor (per expert stack), sign_mask = low 32 bits of the first
+ *     SplitMix64 output for the tensor's seed;
+ *   - rotation R = r * H * diag(s), H the natural-order 32-point Sylvester
+ *     Hadamard matrix, r = fp32(1/sqrt(32));
+ *   - per 16-element half h of a rotated block v: d_h = fp16(rms(v_h))
+ *     (round to nearest even, saturating at 65504);
+ *     code_i = #{ j : v_i / d_h > t_j } over the 15 fp32 midpoints of the
+ *     codebook (all codes 7 when d_h == 0);
+ *   - codes plane  uint8 [E][n][k/2]: element 2i of a row in the low nibble
+ *     of byte i, 2i+1 in the high nibble;
+ *     scales plane uint16 [E][n][k/16]: fp16 bits, scale of half (k/16).
+ *   - dequantized weight: W_hat = diag(s) * r * H * (c[code] * d) per block.
+ *
+ * Conventions for every entry point:
+ *   - All pointers named as device pointers must point to device memory of
+ *     the current CUDA device; host pointers are noted as such.  The caller
+ *     owns every buffer; the library allocates nothing on these paths.
+ *   - Calls are asynchronous on the given stream (a cudaStream_t; NULL is
+ *     the legacy default stream) and do not synchronize, except
+ *     tq4_1s_get_status().
+ *   - Arguments are validated on the host before any launch; a failed check
+ *     returns its error code and launches nothing.
+ *   - Conditions found on the device (a routing id out of range, a bounded
+ *     wait that timed out, a non-finite input to quantize) set bits of a
+ *     per-device status word, read and cleared by tq4_1s_get_status().
+ */
+#ifndef TQ4_1S_H_
+#define TQ4_1S_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* A cudaStream_t, without requiring the CUDA headers. */
+typedef struct CUstream_st* tq4_stream_t;
+
+/* Return codes. */
+enum {
+  TQ_OK = 0,
+  TQ_ERR_INVALID_ARG = 1,         /* null pointer, bad size, k % 32 != 0, m < 0, ... */
+  TQ_ERR_ALIGNMENT = 2,           /* a device pointer not 16-byte aligned */
+  TQ_ERR_UNSUPPORTED_DEVICE = 3,  /* current device is not compute capability 10.0 */
+  TQ_ERR_WORKSPACE = 4,           /* workspace null or smaller than the query says */
+  TQ_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
+  TQ_ERR_TIMEOUT = 6,             /* status: a bounded device wait gave up */
+  TQ_ERR_BAD_ROUTING = 7,         /* status: a routing expert id was out of range */
+  TQ_ERR_NONFINITE = 8            /* status: quantize saw a NaN or infinity */
+};
+
+/* Bits of the device status word (tq4_1s_get_status). */
+enum {
+  TQ_DEV_TIMEOUT = 1,
+  TQ_DEV_BAD_ROUTING = 2,
+  TQ_DEV_NONFINITE = 4
+};
+
+/* Input dtypes of tq4_1s_quantize. */
+enum { TQ_DTYPE_F32 = 0, TQ_DTYPE_BF16 = 1 };
+
+/* A packed TQ4_1S tensor or stack of num_experts tensors of shape [n][k]. */
+typedef struct {
+  int64_t n;            /* rows (output features), > 0                          */
+  int64_t k;            /* columns (input features), > 0, multiple of 32        */
+  int32_t num_experts;  /* 1 for a dense layer                                  */
+  int32_t reserved;     /* must be 0                                            */
+  uint64_t seed;        /* RHT seed; the sign mask is derived from it           */
+  uint8_t* codes;       /* device, [num_experts][n][k/2], 16-byte aligned       */
+  uint16_t* scales;     /* device, [num_experts][n][k/16], 16-byte aligned      */
+} tq4_1s_weight;
+
+/* ABI version of this header (major * 100 + minor). */
+int tq4_1s_version(void);
+
+/* Human-readable text for a return code or status bit.  Never NULL. */
+const char* tq4_1s_error_string(int code);
+
+/* Host, pure.  Bytes of the codes and scales planes of an [e][n][k] stack
+ * (n*k/2*e and n*(k/16)*2*e: exactly 5 bits per weight, per the ~5 bits per
+ * weight of "What Config-I means").  INVALID_ARG for bad sizes. */
+int tq4_1s_packed_bytes(int64_t n, int64_t k, int32_t num_experts, size_t* codes_bytes, size_t* scales_bytes);
+
+/* Host, pure.  The RHT sign mask of a seed: low 32 bits of the first output
+ * of SplitMix64 (Steele, Lea and Flood, OOPSLA 2014) from state `seed`.
+ * Reading of the randomized rotation of "What Config-I means", whose signs
+ * the card does not specify. */
+int tq4_1s_sign_mask(uint64_t seed, uint32_t* mask);
+
+/* Host, pure.  The fp32 codebook the kernels use: levels[16], the 16-level
+ * Lloyd-Max quantizer of N(0,1) ("16-level Lloyd-Max", What Config-I means),
+ * ascending; thresholds[15], the fp32 midpoints.  Either pointer may be NULL. */
+int tq4_1s_codebook(float* levels, float* thresholds);
+
+/* Quantize W (device, [num_experts][n][k], dtype F32 or BF16, row-major,
+ * 16-byte aligned) into out->codes / out->scales (device buffers sized by
+ * tq4_1s_packed_bytes) with the RHT seed out->seed.  Steps: sign flip,
+ * 32-point butterfly, x r, half-block RMS, fp16 scale, nearest level by the
+ * 15 midpoints, nibble packing ("What Config-I means").  A block holding a
+ * NaN or infinity sets TQ_DEV_NONFINITE; its output follows the same
+ * arithmetic (NaN scales are stored as 0x7E00, NaN codes as 0). */
+int tq4_1s_quantize(const void* W, int dtype, const tq4_1s_weight* out, tq4_stream_t stream);
+
+/* Dequantize a packed tensor stack to fp32 W_out (device, [E][n][k]):
+ * W_hat = diag(s) * r * H * (c[code] * d) per block.  Test/debug path. */
+int tq4_1s_dequantize(const tq4_1s_weight* w, float* W_out, tq4_stream_t stream);
+
+/* Bytes of workspace tq4_1s_linear needs for m rows with weight w (dense,
+ * num_experts == 1).  0 on invalid arguments. */
+size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
+
+/* The quantized linear layer of "Running it": y[m][n] = bf16(x * W_hat^T),
+ * fp32 accumulation on the tensor cores, no bias.
+ *   x  device bf16 bits [m][k], row-major, 16-byte aligned;
+ *   y  device bf16 bits [m][n], row-major, 16-byte aligned (n*2 % 16 == 0);
+ *   ws device workspace of at least tq4_1s_linear_workspace(m, w) bytes,
+ *      16-byte aligned, owned by the caller, contents need no initialisation.
+ * Small m rotates each 32-slice of x (x' = R x, split into bf16 hi + lo) and
+ * multiplies the rotated-domain levels c[code]*d on the tensor cores with a
+ * stream-K split of the weight stream; large m dequantizes W_hat to bf16 in
+ * the workspace and runs a tensor-core GEMM.  m == 0 is a no-op. */
+int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, void* ws, size_t ws_bytes,
+                  tq4_stream_t stream);
+
+/* Bytes of workspace tq4_1s_moe needs.  0 on invalid arguments. */
+size_t tq4_1s_moe_workspace(int64_t m, int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* down);
+
+/* The sync-free MoE layer ("Performance"; 128 experts top-6 in "The model
+ * underneath"):  for each token t and slot j < topk with expert
+ * e = topk_ids[t][j] and weight w = topk_w[t][j]:
+ *     u = x_t * W_up[e]^T,  h = bf16(relu(u)^2),  z = h * W_down[e]^T,
+ *     y_t = bf16(sum_j w_tj * z_tj)      (slots in order)
+ *   x        device bf16 bits [m][H]            (H = up->k = down->n)
+ *   topk_ids device int32 [m][topk]; ids outside [0, E) are skipped and set
+ *            TQ_DEV_BAD_ROUTING
+ *   topk_w   device float [m][topk]
+ *   up       stack of E experts [I][H]; down stack of E experts [H][I]
+ *   y        device bf16 bits [m][H]
+ *   ws       device workspace of tq4_1s_moe_workspace() bytes.
+ * Routing, gathering, both projections and the combine all run on the
+ * device; nothing synchronizes with the host. */
+int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, const float* topk_w, int32_t topk,
+               const tq4_1s_weight* up, const tq4_1s_weight* down, uint16_t* y, void* ws, size_t ws_bytes,
+               tq4_stream_t stream);
+
+/* The routing step of tq4_1s_moe on its own (exposed for parity tests):
+ * offsets (device int32 [num_experts + 1]) = exclusive prefix of per-expert
+ * counts; pairs (device int32 [m*topk]) = flat slot indices t*topk + j
+ * grouped by expert, ascending within an expert.  Entries past
+ * offsets[num_experts] are left unspecified. */
+int tq4_1s_moe_route(const int32_t* topk_ids, int64_t m, int32_t topk, int32_t num_experts, int32_t* offsets,
+                     int32_t* pairs, tq4_stream_t stream);
+
+/* Synchronize `stream`, then read and clear the current device's status
+ * word (a mask of TQ_DEV_* bits) into *status (host). */
+int tq4_1s_get_status(tq4_stream_t stream, int32_t* status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* TQ4_1S_H_ */

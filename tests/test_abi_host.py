@@ -1,0 +1,129 @@
+"""Host-side checks of the C ABI: the library loads without a GPU, exports
+every symbol the header declares, and its host-only logic (sizes, sign mask,
+codebook, argument validation) behaves as documented.  No GPU compute."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+import torch
+
+import bit_rotated_weight_b200 as tq
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tq4_1s.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(tq4_1s_\w+)\s*\(", text)))
+
+
+def test_library_exports_every_declared_symbol():
+    lib = tq.load_library()
+    names = declared_functions()
+    assert len(names) >= 13
+    for name in names:
+        assert hasattr(lib, name), name
+    out = os.popen(f"nm -D --defined-only {tq.LIB_PATH}").read()
+    exported = set(re.findall(r" T (tq4_1s_\w+)", out))
+    assert exported == set(names), exported ^ set(names)
+
+
+def test_version_and_error_strings():
+    assert tq.tq4_1s_version() == 100
+    for code in range(0, 9):
+        s = tq.tq4_1s_error_string(code)
+        assert s and s != "unknown error code"
+    assert tq.tq4_1s_error_string(99) == "unknown error code"
+
+
+def test_packed_bytes_is_five_bits_per_weight():
+    c, s = tq.tq4_1s_packed_bytes(4096, 4096)
+    assert (c, s) == (8_388_608, 2_097_152) and c + s == 10_485_760
+    c, s = tq.tq4_1s_packed_bytes(1856, 2688, 128)
+    assert (c + s) * 8 == 5 * 128 * 1856 * 2688
+    with pytest.raises(tq.TQ4Error):
+        tq.tq4_1s_packed_bytes(4096, 4016)   # k % 32 != 0
+
+
+def test_sign_mask_matches_oracle_and_published_value():
+    assert tq.tq4_1s_sign_mask(0) == 0x7B1DCDAF
+    for seed in [1, 2, 3, 1000, 2 ** 63 + 5, 2 ** 64 - 1]:
+        assert tq.tq4_1s_sign_mask(seed) == oracle.sign_mask(seed)
+
+
+def test_library_codebook_equals_oracle_codebook():
+    # two independent Lloyd iterations (positive half vs full) agree in fp32
+    lv, th = tq.tq4_1s_codebook()
+    _, _, c32, t32 = oracle.codebook()
+    assert np.array_equal(lv.numpy().view(np.uint32), c32.view(np.uint32))
+    assert np.array_equal(th.numpy().view(np.uint32), t32.view(np.uint32))
+
+
+def _weight(n=64, k=64, e=1, codes=16, scales=16):
+    return tq._Weight(n, k, e, 0, 0, codes, scales)
+
+
+def test_validation_rejects_before_any_launch():
+    lib = tq.load_library()
+    null = ctypes.c_void_p(0)
+    good = ctypes.c_void_p(4096)
+    w = _weight(k=48)                                          # k % 32 != 0
+    assert lib.tq4_1s_linear(good, 16, ctypes.byref(w), good, good, 1 << 20, null) == 1
+    w = _weight(codes=0)                                       # null codes
+    assert lib.tq4_1s_linear(good, 16, ctypes.byref(w), good, good, 1 << 20, null) == 1
+    w = _weight(codes=4104)                                    # misaligned codes
+    assert lib.tq4_1s_linear(good, 16, ctypes.byref(w), good, good, 1 << 20, null) == 2
+    w = _weight()
+    assert lib.tq4_1s_linear(good, -1, ctypes.byref(w), good, good, 1 << 20, null) == 1
+    assert lib.tq4_1s_linear(good, 0, ctypes.byref(w), good, good, 0, null) == 0     # m == 0: no-op
+    assert lib.tq4_1s_linear(null, 16, ctypes.byref(w), good, good, 1 << 20, null) == 1
+    assert lib.tq4_1s_linear(ctypes.c_void_p(4100), 16, ctypes.byref(w), good, good, 1 << 20, null) == 2
+    w2 = _weight(e=2)                                          # linear wants a dense weight
+    assert lib.tq4_1s_linear(good, 16, ctypes.byref(w2), good, good, 1 << 20, null) == 1
+    assert lib.tq4_1s_quantize(good, 7, ctypes.byref(w), null) == 1          # bad dtype
+    assert lib.tq4_1s_quantize(null, 0, ctypes.byref(w), null) == 1
+    assert lib.tq4_1s_dequantize(ctypes.byref(w), null, null) == 1
+    assert lib.tq4_1s_get_status(null, None) == 1
+    up, dn = _weight(n=128, k=64, e=4), _weight(n=64, k=96, e=4)            # up.n != down.k
+    assert lib.tq4_1s_moe(good, 4, good, good, 2, ctypes.byref(up), ctypes.byref(dn), good, good, 1 << 20,
+                          null) == 1
+    assert lib.tq4_1s_moe_workspace(4, 2, ctypes.byref(up), ctypes.byref(dn)) == 0
+    assert lib.tq4_1s_moe_route(good, 4, 0, 8, good, good, null) == 1
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
+def test_valid_call_without_gpu_fails_loudly():
+    lib = tq.load_library()
+    good = ctypes.c_void_p(4096)
+    w = _weight()
+    need = lib.tq4_1s_linear_workspace(16, ctypes.byref(w))
+    assert need > 0
+    assert lib.tq4_1s_linear(good, 16, ctypes.byref(w), good, good, need, ctypes.c_void_p(0)) == 3
+    assert lib.tq4_1s_quantize(good, 0, ctypes.byref(w), ctypes.c_void_p(0)) == 3
+
+
+def test_workspace_queries():
+    lib = tq.load_library()
+    w = _weight(n=4096, k=4096)
+    small = lib.tq4_1s_linear_workspace(16, ctypes.byref(w))
+    large = lib.tq4_1s_linear_workspace(8192, ctypes.byref(w))
+    assert 0 < small < large and large >= 4096 * 4096 * 2
+    assert lib.tq4_1s_linear_workspace(0, ctypes.byref(w)) == 0
+    up, dn = _weight(n=1856, k=2688, e=128), _weight(n=2688, k=1856, e=128)
+    assert lib.tq4_1s_moe_workspace(16, 6, ctypes.byref(up), ctypes.byref(dn)) > 0
+
+
+def test_missing_library_raises(tmp_path):
+    import importlib
+    with pytest.raises(ImportError):
+        tq._lib_saved = tq._lib
+        tq._lib = None
+        try:
+            tq.load_library(str(tmp_path / "nope.so"))
+        finally:
+            tq._lib = tq._lib_saved

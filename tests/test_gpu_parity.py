@@ -1,0 +1,214 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.  Packing, unpacking and routing are compared bit for bit;
+GEMM outputs against the stated max/mean relative tolerances."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import synth
+from tests._parity import assert_close, errors
+
+pytestmark = pytest.mark.gpu
+
+tq = pytest.importorskip("bit_rotated_weight_b200")
+DEV = torch.device("cuda:0") if torch.cuda.is_available() else None
+
+
+def _bf16_dev(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(DEV).view(torch.bfloat16)
+
+
+def _bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _quantize_both(W, seed):
+    p = tq.tq4_1s_quantize(torch.from_numpy(W).to(DEV), seed=seed)
+    torch.cuda.synchronize()
+    codes, scales, bad = oracle.quantize(W.reshape(-1, W.shape[-1]), seed)
+    return p, codes.reshape(p.codes.shape), scales.reshape(p.scales.shape), bad
+
+
+@pytest.fixture(autouse=True)
+def _clear_status():
+    if torch.cuda.is_available():
+        tq.tq4_1s_get_status()
+    yield
+
+
+# ----------------------------------------------------------------- quantize
+@pytest.mark.parametrize("shape,seed,dist", [
+    ((256, 256), 0, "normal"),             # tiny single linear
+    ((200, 96), 11, "student_t"),          # ragged rows, 3 blocks per row
+    ((1, 32), 12, "normal"),               # one block
+    ((4096, 4096), 2, "student_t"),        # dense decode-block weight
+    ((4, 64, 160), 13, "normal"),          # expert stack
+])
+def test_quantize_bit_exact(shape, seed, dist):
+    W = (synth.normal_f32(shape, seed, 0.02) if dist == "normal"
+         else synth.student_t_f32(shape, seed, 5.0, 0.02))
+    p, codes, scales, _ = _quantize_both(W, seed)
+    assert np.array_equal(p.codes.cpu().numpy(), codes)
+    assert np.array_equal(p.scales.cpu().numpy().view(np.uint16), scales)
+    assert tq.tq4_1s_get_status() == 0
+
+
+def test_quantize_bf16_input_bit_exact():
+    Wb = synth.f32_to_bf16_bits(synth.normal_f32((128, 256), 21, 0.05))
+    Wf = synth.bf16_bits_to_f32(Wb)
+    p = tq.tq4_1s_quantize(_bf16_dev(Wb), seed=21)
+    codes, scales, _ = oracle.quantize(Wf, 21)
+    assert np.array_equal(p.codes[0].cpu().numpy(), codes)
+    assert np.array_equal(p.scales[0].cpu().numpy().view(np.uint16), scales)
+
+
+def test_quantize_special_blocks_and_status():
+    W = np.zeros((3, 64), np.float32)
+    W[1, 32:] = synth.normal_f32(32, 41)
+    W[2, 3] = np.nan
+    W[2, 40] = np.inf
+    p, codes, scales, bad = _quantize_both(W, 0)
+    assert bad == 2
+    assert np.array_equal(p.codes.cpu().numpy()[0], codes)
+    assert np.array_equal(p.scales.cpu().numpy()[0].view(np.uint16), scales)
+    assert tq.tq4_1s_get_status() & tq.TQ_DEV_NONFINITE
+    assert tq.tq4_1s_get_status() == 0     # read clears
+
+
+# ----------------------------------------------------------------- dequantize
+@pytest.mark.parametrize("shape,seed", [((256, 256), 0), ((77, 320), 5), ((3, 64, 96), 6)])
+def test_dequantize_bit_exact(shape, seed):
+    W = synth.student_t_f32(shape, seed, 5.0, 0.02)
+    p, codes, scales, _ = _quantize_both(W, seed)
+    Wg = tq.tq4_1s_dequantize(p).cpu().numpy()
+    Wo = oracle.dequantize(codes.reshape(-1, codes.shape[-1]), scales.reshape(-1, scales.shape[-1]), seed)
+    assert np.array_equal(Wg.reshape(Wo.shape).view(np.uint32), Wo.view(np.uint32))
+
+
+# ----------------------------------------------------------------- linear
+LINEAR_CASES = [
+    # (m, n, k, seed)  -- small-m stream-K path
+    (16, 256, 256, 0),      # tiny single linear: split tiles on a 4-CTA grid
+    (1, 128, 128, 30),
+    (5, 200, 96, 31),       # ragged rows and a ragged k tail (96 = 0.75 of a 128 k step)
+    (16, 1000, 544, 32),
+    (32, 384, 512, 33),     # two 16-row boxes per operand
+    (33, 256, 256, 34),     # two segments, the second with one row
+    (100, 640, 384, 35),    # four segments
+    (16, 4096, 4096, 2),    # dense decode-block linear, full size
+    # large-m path (dequantize + GEMM)
+    (129, 256, 256, 40),
+    (300, 520, 224, 41),    # ragged m, n, k
+    (512, 1024, 512, 42),
+]
+
+
+@pytest.mark.parametrize("m,n,k,seed", LINEAR_CASES)
+def test_linear_parity(m, n, k, seed):
+    W = synth.student_t_f32((n, k), seed, 5.0, 0.02)
+    x = synth.activations_bf16(m, k, seed + 1)
+    p, codes, scales, _ = _quantize_both(W, seed)
+    y = tq.tq4_1s_linear(_bf16_dev(x), p)
+    torch.cuda.synchronize()
+    y_ref, _ = oracle.linear(x, codes[0], scales[0], seed)
+    assert_close(_bits(y), y_ref, f"linear m={m} n={n} k={k}")
+    assert tq.tq4_1s_get_status() == 0
+
+
+def test_linear_deterministic_repeats():
+    W = synth.student_t_f32((4096, 4096), 2, 5.0, 0.02)
+    x = synth.activations_bf16(16, 4096, 3)
+    p = tq.tq4_1s_quantize(torch.from_numpy(W).to(DEV), seed=2)
+    xd = _bf16_dev(x)
+    first = _bits(tq.tq4_1s_linear(xd, p))
+    for _ in range(20):
+        assert np.array_equal(_bits(tq.tq4_1s_linear(xd, p)), first)
+
+
+def test_linear_prefill_8192_sampled_rows():
+    """M=8192 x K=4096 against W 14336 x 4096: sampled output rows vs oracle."""
+    m, n, k, seed = 8192, 14336, 4096, 8
+    W = synth.normal_f32((n, k), seed, 0.02)
+    x = synth.activations_bf16(m, k, 9)
+    p, codes, scales, _ = _quantize_both(W, seed)
+    y = tq.tq4_1s_linear(_bf16_dev(x), p)
+    torch.cuda.synchronize()
+    rows = np.sort(synth.rng(99).choice(m, 12, replace=False))
+    rows = np.concatenate([rows, [0, m - 1]])
+    Wh = oracle.dequantize(codes[0], scales[0], seed)
+    y_ref = oracle.linear_f64(x[rows], Wh)
+    assert_close(_bits(y)[rows], y_ref, "prefill sampled rows")
+
+
+# ----------------------------------------------------------------- MoE
+def test_moe_route_bit_exact():
+    for m, E, topk, seed in [(16, 128, 6, 7), (512, 128, 6, 77), (3, 8, 2, 78)]:
+        ids, _ = synth.gumbel_topk_router(m, E, topk, seed)
+        off, pairs = tq.tq4_1s_moe_route(torch.from_numpy(ids).to(DEV), E)
+        o_off, o_pairs, _ = oracle.moe_route(ids, E)
+        assert np.array_equal(off.cpu().numpy(), o_off)
+        assert np.array_equal(pairs.cpu().numpy()[: len(o_pairs)], o_pairs)
+
+
+def test_moe_route_bad_ids_flagged():
+    ids, _ = synth.gumbel_topk_router(8, 16, 2, 5)
+    ids[2, 1] = 16
+    ids[5, 0] = -3
+    off, pairs = tq.tq4_1s_moe_route(torch.from_numpy(ids).to(DEV), 16)
+    o_off, o_pairs, bad = oracle.moe_route(ids, 16)
+    assert bad == 2
+    assert np.array_equal(off.cpu().numpy(), o_off)
+    assert np.array_equal(pairs.cpu().numpy()[: len(o_pairs)], o_pairs)
+    assert tq.tq4_1s_get_status() & tq.TQ_DEV_BAD_ROUTING
+
+
+def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False):
+    up_seed, dn_seed, x_seed, r_seed = seeds
+    up = synth.normal_f32((E, I, H), up_seed, dist_std)
+    dn = synth.normal_f32((E, H, I), dn_seed, dist_std)
+    ids, w = synth.gumbel_topk_router(m, E, topk, r_seed)
+    if bad_ids:
+        ids[0, 1] = E + 1
+    x = synth.activations_bf16(m, H, x_seed)
+    pu = tq.tq4_1s_quantize(torch.from_numpy(up).to(DEV), seed=up_seed)
+    pd = tq.tq4_1s_quantize(torch.from_numpy(dn).to(DEV), seed=dn_seed)
+    y = tq.tq4_1s_moe(_bf16_dev(x), torch.from_numpy(ids).to(DEV), torch.from_numpy(w).to(DEV), pu, pd)
+    torch.cuda.synchronize()
+    # the oracle quantizes only the experts the routing touches (others cannot
+    # influence y); unused experts keep zero planes on the oracle side
+    used = sorted(set(int(e) for e in ids.ravel() if 0 <= e < E))
+    uc = np.zeros((E, I, H // 2), np.uint8); us = np.zeros((E, I, H // 16), np.uint16)
+    dc = np.zeros((E, H, I // 2), np.uint8); ds = np.zeros((E, H, I // 16), np.uint16)
+    for e in used:
+        uc[e], us[e], _ = oracle.quantize(up[e], up_seed)
+        dc[e], ds[e], _ = oracle.quantize(dn[e], dn_seed)
+    y_ref, _, bad = oracle.moe(x, ids, w, uc, us, up_seed, dc, ds, dn_seed)
+    return y, y_ref, bad
+
+
+def test_moe_small_parity():
+    y, y_ref, _ = _moe_case(8, 256, 128, 4, 2, (4, 5, 6, 7))
+    assert_close(_bits(y), y_ref, "moe small")
+    assert tq.tq4_1s_get_status() == 0
+
+
+def test_moe_many_tokens_per_expert():
+    # 40 tokens, 4 experts, top-2: 20 rows per expert on average, some experts
+    # take more than one 32-row segment
+    y, y_ref, _ = _moe_case(4, 256, 192, 40, 2, (14, 15, 16, 17))
+    assert_close(_bits(y), y_ref, "moe segments")
+
+
+def test_moe_bad_id_skipped():
+    y, y_ref, bad = _moe_case(8, 128, 96, 5, 2, (24, 25, 26, 27), bad_ids=True)
+    assert bad == 1
+    assert_close(_bits(y), y_ref, "moe bad id")
+    assert tq.tq4_1s_get_status() & tq.TQ_DEV_BAD_ROUTING
+
+
+def test_moe_128_experts_top6_full():
+    """128 experts (up 2688->1856, down 1856->2688), 16 tokens, top-6."""
+    y, y_ref, _ = _moe_case(128, 2688, 1856, 16, 6, (4, 5, 6, 7))
+    e = assert_close(_bits(y), y_ref, "moe 128x top6")
+    print("moe errors", e)
