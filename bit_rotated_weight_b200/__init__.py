@@ -24,7 +24,7 @@ __all__ = [
     "LIB_PATH", "TQ4Error", "Packed", "load_library",
     "tq4_1s_version", "tq4_1s_error_string", "tq4_1s_packed_bytes", "tq4_1s_sign_mask", "tq4_1s_codebook",
     "tq4_1s_quantize", "tq4_1s_dequantize", "tq4_1s_linear_workspace", "tq4_1s_linear",
-    "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_route", "tq4_1s_get_status",
+    "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_route", "tq4_1s_get_status", "tq4_1s_launch_count",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -77,6 +77,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                 "tq4_1s_moe": ([P, I64, P, P, I32, W, W, P, P, SZ, P], ctypes.c_int),
                 "tq4_1s_moe_route": ([P, I64, I32, I32, P, P, P], ctypes.c_int),
                 "tq4_1s_get_status": ([P, ctypes.POINTER(I32)], ctypes.c_int),
+                "tq4_1s_launch_count": ([], ctypes.c_uint64),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -252,3 +253,8 @@ def tq4_1s_get_status(device=None) -> int:
     s = ctypes.c_int32()
     _check(load_library().tq4_1s_get_status(_stream(device), ctypes.byref(s)), "get_status")
     return s.value
+
+
+def tq4_1s_launch_count() -> int:
+    """Kernel launches issued through the library by this process so far."""
+    return int(load_library().tq4_1s_launch_count())

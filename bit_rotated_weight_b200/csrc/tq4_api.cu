@@ -1,6 +1,7 @@
 // Host side of libtq4_1s.so: the extern "C" entry points declared in
 // include/tq4_1s.h -- argument validation, the codebook, the RHT sign mask,
 // TMA tensor-map construction and the launch sequences of each call.
+#include <atomic>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -58,6 +59,9 @@ const CodebookF32& codebook() {
   static const CodebookF32 cb = compute_codebook();
   return cb;
 }
+
+static std::atomic<uint64_t> g_launches{0};
+void note_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
 // SplitMix64 (Steele, Lea, Flood, OOPSLA 2014): first output from `state`.
 static uint32_t sign_mask_of(uint64_t state) {
@@ -161,12 +165,13 @@ static bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
-// bf16 matrix [rows][cols] row-major, box 64 x box_rows, 128-byte swizzle.
+// 16-bit matrix [rows][cols] row-major (bf16 or fp16), box 64 x box_rows,
+// 128-byte swizzle.
 static bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
   const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(cols * 2)};
   const uint32_t box[2] = {64, box_rows};
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -202,7 +207,7 @@ static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
 }
 
 struct MoeLayout {
-  size_t offsets, pairs, segs, nseg, npv, xh, xl, hh, hl, zw, partials, cnt_up, cnt_dn, total;
+  size_t offsets, pairs, segs, nseg, npv, xh, xl, xscale, hh, hl, zw, partials, cnt_up, cnt_dn, total;
   int64_t P, maxseg, rt_up, rt_dn;
 };
 
@@ -227,12 +232,14 @@ static MoeLayout moe_layout(int64_t m, int32_t topk, const tq4_1s_weight* up, co
   L.npv = take(4);
   L.xh = take(L.P * H * 2);
   L.xl = take(L.P * H * 2);
+  L.xscale = take(L.P * 4);
   L.hh = take(L.P * I * 2);
   L.hl = take(L.P * I * 2);
   L.zw = take(L.P * H * 4);
   L.partials = take(static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
-  L.cnt_up = take(L.maxseg * L.rt_up * 4);
-  L.cnt_dn = take(L.maxseg * L.rt_dn * 4);
+  // the two counter arrays are one block: the route kernel zeroes it at once
+  L.cnt_up = take(L.maxseg * (L.rt_up + L.rt_dn) * 4);
+  L.cnt_dn = L.cnt_up + static_cast<size_t>(L.maxseg * L.rt_up) * 4;
   L.total = off;
   return L;
 }
@@ -417,13 +424,17 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   cudaError_t e = launch_moe_route(topk_ids, L.P, static_cast<int32_t>(E), offsets, pairs, segs, nseg, kSegRows,
                                    npv, cnt_up, ncnt, st);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
-  e = launch_rotate_act(x, H, pairs, topk, npv, 0, L.P, xh, xl, sign_mask_of(up->seed), nullptr, 0, st);
+  float* xscale = reinterpret_cast<float*>(base + L.xscale);
+  e = launch_rotate_rows_f16(x, H, pairs, topk, npv, L.P, xh, xl, xscale, sign_mask_of(up->seed), st);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
 
   alignas(64) CUtensorMap tcu, txh, txl, tcd, thh, thl;
   if (!map_codes(&tcu, up) || !map_bf16(&txh, xh, L.P, H, 16) || !map_bf16(&txl, xl, L.P, H, 16) ||
       !map_codes(&tcd, down) || !map_bf16(&thh, hh, L.P, I, 16) || !map_bf16(&thl, hl, L.P, I, 16))
     return TQ_ERR_CUDA;
+  // Up projection in fp16 operands: its error is doubled by the squared ReLU,
+  // and fp16 levels round 8x finer than bf16.  Rows of x' carry a power-of-two
+  // scale (xscale) that keeps them inside the fp16 range.
   StreamKArgs a{};
   a.n = static_cast<int32_t>(I);
   a.k = static_cast<int32_t>(H);
@@ -432,6 +443,8 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   a.segs = segs;
   a.nseg_dev = nseg;
   a.scales = up->scales;
+  a.f16 = 1;
+  a.row_scale = xscale;
   a.mode = EPI_UP;
   a.out_a = hh;
   a.out_b = hl;
@@ -447,6 +460,8 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   b.row_tiles = static_cast<int32_t>(L.rt_dn);
   b.k_iters = static_cast<int32_t>((I + 127) / 128);
   b.scales = down->scales;
+  b.f16 = 0;
+  b.row_scale = nullptr;
   b.mode = EPI_DOWN;
   b.out_a = nullptr;
   b.out_b = nullptr;
@@ -469,6 +484,8 @@ TQ_API int tq4_1s_moe_route(const int32_t* topk_ids, int64_t m, int32_t topk, in
   return cuda_rc(launch_moe_route(topk_ids, m * topk, num_experts, offsets, pairs, nullptr, nullptr, kSegRows,
                                   nullptr, nullptr, 0, reinterpret_cast<cudaStream_t>(stream)));
 }
+
+TQ_API uint64_t tq4_1s_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 TQ_API int tq4_1s_get_status(tq4_stream_t stream, int32_t* status) {
   if (!status) return TQ_ERR_INVALID_ARG;

@@ -211,6 +211,7 @@ cudaError_t launch_gemm_bf16(const void* tm_x, const void* tm_w, uint16_t* y, in
   }
   gemm_bf16_kernel<<<grid, kThreads, smem, st>>>(*static_cast<const CUtensorMap*>(tm_x),
                                                  *static_cast<const CUtensorMap*>(tm_w), y, m, n, k);
+  note_launches(1);
   return cudaGetLastError();
 }
 

@@ -13,6 +13,9 @@ struct CodebookF32 {
   float thresholds[16];   // 15 used: midpoints of adjacent levels
 };
 
+// Count of kernel launches issued by the library (tq4_1s_launch_count).
+void note_launches(int n);
+
 // Host-side codebook computation (Lloyd iteration), run once per process.
 const CodebookF32& codebook();
 
@@ -30,6 +33,9 @@ cudaError_t launch_rotate_act(const uint16_t* x, int64_t k, const int32_t* gathe
                               const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
                               uint16_t* xh, uint16_t* xl, uint32_t mask, int32_t* zero_ptr, int64_t nzero,
                               cudaStream_t st);
+cudaError_t launch_rotate_rows_f16(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
+                                   const int32_t* rows_valid_dev, int64_t rows_alloc, uint16_t* xh, uint16_t* xl,
+                                   float* row_scale, uint32_t mask, cudaStream_t st);
 cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
                              int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
                              int32_t* zero_ptr, int64_t nzero, cudaStream_t st);
@@ -55,6 +61,8 @@ struct StreamKArgs {
   const int32_t* pairs;      // MoE: flat slot index of each sorted row
   const float* topk_w;       // MoE: router weights (flat)
   uint32_t next_mask;        // up: sign mask of the down projection
+  int32_t f16;               // operands: 0 = bf16 (x' hi/lo), 1 = fp16 (x' hi/lo scaled by row_scale)
+  const float* row_scale;    // fp16 mode: x' row r was multiplied by 1/row_scale[r]
   float* partials;           // [grid][2][128][kSegRows]
   int32_t* counters;         // [tiles]
   int32_t max_tiles;         // capacity of counters

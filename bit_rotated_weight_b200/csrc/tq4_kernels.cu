@@ -174,6 +174,65 @@ __global__ void __launch_bounds__(256) rotate_act_kernel(const uint16_t* __restr
   }
 }
 
+// One CTA per row: the fp16 variant of the activation rotation.  x' = R x per
+// 32-slice is scaled by 2^-e, where e puts the largest value x' can take,
+// sqrt(32) * max|x| (each x'_i is r times a signed sum of 32 entries), in
+// [2^13, 2^14): every row then uses the full fp16 precision and cannot
+// overflow.  Split into fp16 hi = f16(x' 2^-e) and lo = f16(x' 2^-e - hi);
+// row_scale[row] = 2^e undoes the scaling in the GEMM epilogue (an exact
+// power of two).  Rows at or past the valid count are zero with scale 1.
+__global__ void __launch_bounds__(256) rotate_rows_f16_kernel(const uint16_t* __restrict__ x, int64_t k,
+                                                              const int32_t* __restrict__ gather, int32_t topk,
+                                                              const int32_t* __restrict__ rows_valid_dev,
+                                                              int64_t rows_alloc, uint16_t* __restrict__ xh,
+                                                              uint16_t* __restrict__ xl,
+                                                              float* __restrict__ row_scale, uint32_t mask) {
+  __shared__ float s_max[8];
+  const int64_t row = blockIdx.x;
+  if (row >= rows_alloc) return;
+  const int64_t rows_valid = rows_valid_dev ? static_cast<int64_t>(*rows_valid_dev) : rows_alloc;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  uint16_t* oh = xh + row * k;
+  uint16_t* ol = xl + row * k;
+  if (row >= rows_valid) {
+    for (int64_t i = threadIdx.x; i < k; i += blockDim.x) {
+      oh[i] = 0;
+      ol[i] = 0;
+    }
+    if (threadIdx.x == 0) row_scale[row] = 1.0f;
+    return;
+  }
+  const int64_t src = gather ? static_cast<int64_t>(gather[row] / topk) : row;
+  const uint16_t* xr = x + src * k;
+  float mx = 0.0f;
+  for (int64_t i = threadIdx.x; i < k; i += blockDim.x) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(xr[i])));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+  if (lane == 0) s_max[warp] = mx;
+  __syncthreads();
+  mx = s_max[0];
+  for (int w = 1; w < nwarps; ++w) mx = fmaxf(mx, s_max[w]);
+  int e = 0;
+  if (mx > 0.0f && isfinite(mx)) {
+    int ex;
+    frexpf(__fmul_rn(mx, 5.65685415f), &ex);   // bound in [2^(ex-1), 2^ex)
+    e = ex - 14;
+    e = e < -100 ? -100 : (e > 100 ? 100 : e);
+  }
+  const float down = ldexpf(1.0f, -e);
+  if (threadIdx.x == 0) row_scale[row] = ldexpf(1.0f, e);
+  const bool neg = (mask >> lane) & 1u;
+  const float r = rsqrt32();
+  for (int64_t kb = warp; kb < k / 32; kb += nwarps) {
+    const float xv = bf16_bits_to_f32(xr[kb * 32 + lane]);
+    const float v = __fmul_rn(__fmul_rn(warp_fwht32(neg ? -xv : xv, lane), r), down);
+    const __half h = __float2half_rn(v);
+    const __half l = __float2half_rn(__fsub_rn(v, __half2float(h)));
+    oh[kb * 32 + lane] = __half_as_ushort(h);
+    ol[kb * 32 + lane] = __half_as_ushort(l);
+  }
+}
+
 // ------------------------------------------------------------------ MoE routing
 // One CTA: per-expert counts, exclusive prefix (offsets), and a stable
 // bucketing of flat slot indices p = t*topk + j by expert.  Stability comes
@@ -272,18 +331,21 @@ cudaError_t launch_quantize(const void* W, int dtype, uint8_t* codes, uint16_t* 
     quantize_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(W), codes, scales, rows, k, mask, cb);
   else
     quantize_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(W), codes, scales, rows, k, mask, cb);
+  note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, float* out, int64_t rows, int64_t k,
                                   uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
   dequantize_kernel<float><<<grid_for(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k, mask, cb);
+  note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales, uint16_t* out, int64_t rows,
                                    int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
   dequantize_kernel<uint16_t><<<grid_for(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k, mask, cb);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -294,6 +356,17 @@ cudaError_t launch_rotate_act(const uint16_t* x, int64_t k, const int32_t* gathe
   int g = grid_for(rows_alloc * (k / 32), 256);
   rotate_act_kernel<<<g, 256, 0, st>>>(x, k, gather, topk, rows_valid_dev, rows_valid_host, rows_alloc, xh, xl,
                                        mask, zero_ptr, nzero);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rotate_rows_f16(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
+                                   const int32_t* rows_valid_dev, int64_t rows_alloc, uint16_t* xh, uint16_t* xl,
+                                   float* row_scale, uint32_t mask, cudaStream_t st) {
+  if (rows_alloc <= 0) return cudaSuccess;
+  rotate_rows_f16_kernel<<<static_cast<unsigned>(rows_alloc), 256, 0, st>>>(x, k, gather, topk, rows_valid_dev,
+                                                                            rows_alloc, xh, xl, row_scale, mask);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -303,6 +376,7 @@ cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_exp
   const size_t sh = sizeof(int32_t) * 2 * static_cast<size_t>(num_experts);
   moe_route_kernel<<<1, 1024, sh, st>>>(ids, npairs, num_experts, offsets, pairs, segs, nseg, chunk, npairs_valid,
                                         zero_ptr, nzero);
+  note_launches(1);
   return cudaGetLastError();
 }
 
@@ -311,6 +385,7 @@ cudaError_t launch_moe_combine(const float* zw, const int32_t* ids, int64_t m, i
   const int64_t n = m * h;
   const int g = static_cast<int>((n + 255) / 256);
   moe_combine_kernel<<<g, 256, 0, st>>>(zw, ids, m, topk, h, num_experts, y);
+  note_launches(1);
   return cudaGetLastError();
 }
 

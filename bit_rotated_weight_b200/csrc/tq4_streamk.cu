@@ -104,14 +104,21 @@ __device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
 __device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
   return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
 }
-__device__ __forceinline__ uint32_t bf16x2_from_f32x2(uint64_t v) {
-  return pack_bf16x2(__uint_as_float(static_cast<uint32_t>(v)), __uint_as_float(static_cast<uint32_t>(v >> 32)));
+template <bool kF16>
+__device__ __forceinline__ uint32_t x2_from_f32x2(uint64_t v) {
+  const float lo = __uint_as_float(static_cast<uint32_t>(v)), hi = __uint_as_float(static_cast<uint32_t>(v >> 32));
+  if constexpr (kF16) {
+    __half2 h = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&h);
+  } else {
+    return pack_bf16x2(lo, hi);
+  }
 }
 
 // Dequantize one half-block (16 codes in q0 = elements 0..7, q1 = 8..15, one
 // nibble each, low nibble first) with scale d into 8 registers of bf16 pairs
-// {element 2i, element 2i+1}, value bf16(c[code] * d) with one rounding of
-// the fp32 product.
+// {element 2i, element 2i+1}, value bf16(c[code] * d) (or fp16 when kF16)
+// with one rounding of the fp32 product.
 //
 // The codebook is odd-symmetric (c[15-j] = -c[j]), so a code j maps to a
 // magnitude index m = j-8 (j >= 8) or 7-j (j < 8) and a sign (j < 8).  The 8
@@ -119,13 +126,14 @@ __device__ __forceinline__ uint32_t bf16x2_from_f32x2(uint64_t v) {
 // low-byte plane and a high-byte plane (two registers each); prmt then looks
 // up four codes at a time by byte index, the sign is OR-ed into the high
 // bytes, and a last prmt interleaves low/high bytes into bf16 pairs.
+template <bool kF16>
 __device__ __forceinline__ void dequant_half(uint32_t q0, uint32_t q1, float d, const uint64_t (&cm2)[4],
                                              uint32_t* out) {
   const uint64_t dd = pack_f32x2(d, d);
-  const uint32_t p01 = bf16x2_from_f32x2(fmul2(cm2[0], dd));
-  const uint32_t p23 = bf16x2_from_f32x2(fmul2(cm2[1], dd));
-  const uint32_t p45 = bf16x2_from_f32x2(fmul2(cm2[2], dd));
-  const uint32_t p67 = bf16x2_from_f32x2(fmul2(cm2[3], dd));
+  const uint32_t p01 = x2_from_f32x2<kF16>(fmul2(cm2[0], dd));
+  const uint32_t p23 = x2_from_f32x2<kF16>(fmul2(cm2[1], dd));
+  const uint32_t p45 = x2_from_f32x2<kF16>(fmul2(cm2[2], dd));
+  const uint32_t p67 = x2_from_f32x2<kF16>(fmul2(cm2[3], dd));
   const uint32_t lo0 = prmt(p01, p23, 0x6420u), lo1 = prmt(p45, p67, 0x6420u);
   const uint32_t hi0 = prmt(p01, p23, 0x7531u), hi1 = prmt(p45, p67, 0x7531u);
 #pragma unroll
@@ -163,8 +171,13 @@ __device__ __forceinline__ float warp_fwht32_epi(float a, int lane) {
 }
 
 // The per-mode store of one finished tile row (thread = weight row `row`).
-__device__ __forceinline__ void epilogue_store(const StreamKArgs& a, const float (&v)[kSegRows], int row, int lane,
+__device__ __forceinline__ void epilogue_store(const StreamKArgs& a, float (&v)[kSegRows], int row, int lane,
                                                const Seg& sg) {
+  if (a.row_scale) {
+#pragma unroll
+    for (int j = 0; j < kSegRows; ++j)
+      if (j < sg.count) v[j] = __fmul_rn(v[j], a.row_scale[sg.row0 + j]);
+  }
   if (a.mode == EPI_DENSE) {
     if (row < a.n) {
 #pragma unroll
@@ -209,6 +222,7 @@ struct Codemag {
   float v[8];   // levels[8..15]: the positive magnitudes, ascending
 };
 
+template <bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
     streamk_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_xhi,
                    const __grid_constant__ CUtensorMap tm_xlo, const StreamKArgs a, const Codemag cmag) {
@@ -318,7 +332,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int sgi = static_cast<int>(tile / a.row_tiles);
         const Seg sg = get_seg(a, sgi);
         const int nb = (sg.count + 15) >> 4;
-        const uint32_t idesc = idesc_bf16(128, 32 * nb);
+        const uint32_t idesc = kF16 ? idesc_f16(128, 32 * nb) : idesc_bf16(128, 32 * nb);
         const uint32_t d_addr = tmem + (pi & 1) * kDCols;
         const uint32_t a_addr = tmem + kACol0 + as * kAColsPerStage;
         const uint32_t xb = smem_u32(smem + s * kStageBytes + kCodesBytes);
@@ -373,8 +387,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int kb = 0; kb < 4; ++kb) {
         const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((t >> 1) & 3)));
         uint32_t o[16];
-        dequant_half(c.x, c.y, dsc[2 * kb], cm2, o);
-        dequant_half(c.z, c.w, dsc[2 * kb + 1], cm2, o + 8);
+        dequant_half<kF16>(c.x, c.y, dsc[2 * kb], cm2, o);
+        dequant_half<kF16>(c.z, c.w, dsc[2 * kb + 1], cm2, o + 8);
         tmem_st16(tbase + 16 * kb, o);
       }
       tmem_wait_st();
@@ -502,17 +516,25 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void*
   static bool attr_set = false;
   const size_t smem = streamk_smem_bytes();
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(streamk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    cudaError_t e = cudaFuncSetAttribute(streamk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          static_cast<int>(smem));
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(streamk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               static_cast<int>(smem));
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
   Codemag cm;
   const CodebookF32& cb = codebook();
   for (int i = 0; i < 8; ++i) cm.v[i] = cb.levels[8 + i];
-  streamk_kernel<<<grid, kThreads, smem, st>>>(*static_cast<const CUtensorMap*>(tm_codes),
-                                               *static_cast<const CUtensorMap*>(tm_xhi),
-                                               *static_cast<const CUtensorMap*>(tm_xlo), a, cm);
+  const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
+  const CUtensorMap& m1 = *static_cast<const CUtensorMap*>(tm_xhi);
+  const CUtensorMap& m2 = *static_cast<const CUtensorMap*>(tm_xlo);
+  if (a.f16)
+    streamk_kernel<true><<<grid, kThreads, smem, st>>>(m0, m1, m2, a, cm);
+  else
+    streamk_kernel<false><<<grid, kThreads, smem, st>>>(m0, m1, m2, a, cm);
+  note_launches(1);
   return cudaGetLastError();
 }
 

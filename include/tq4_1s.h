@@ -166,6 +166,11 @@ int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, const floa
 int tq4_1s_moe_route(const int32_t* topk_ids, int64_t m, int32_t topk, int32_t num_experts, int32_t* offsets,
                      int32_t* pairs, tq4_stream_t stream);
 
+/* Host, pure.  Number of kernel launches this process has issued through
+ * the library so far (all devices); a launch captured into a CUDA graph
+ * counts once, at capture. */
+uint64_t tq4_1s_launch_count(void);
+
 /* Synchronize `stream`, then read and clear the current device's status
  * word (a mask of TQ_DEV_* bits) into *status (host). */
 int tq4_1s_get_status(tq4_stream_t stream, int32_t* status);

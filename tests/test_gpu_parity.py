@@ -70,8 +70,8 @@ def test_quantize_special_blocks_and_status():
     W[2, 40] = np.inf
     p, codes, scales, bad = _quantize_both(W, 0)
     assert bad == 2
-    assert np.array_equal(p.codes.cpu().numpy()[0], codes)
-    assert np.array_equal(p.scales.cpu().numpy()[0].view(np.uint16), scales)
+    assert np.array_equal(p.codes.cpu().numpy(), codes)
+    assert np.array_equal(p.scales.cpu().numpy().view(np.uint16), scales)
     assert tq.tq4_1s_get_status() & tq.TQ_DEV_NONFINITE
     assert tq.tq4_1s_get_status() == 0     # read clears
 
@@ -163,14 +163,14 @@ def test_moe_route_bad_ids_flagged():
     assert tq.tq4_1s_get_status() & tq.TQ_DEV_BAD_ROUTING
 
 
-def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False):
+def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False, x_std=1.0):
     up_seed, dn_seed, x_seed, r_seed = seeds
     up = synth.normal_f32((E, I, H), up_seed, dist_std)
     dn = synth.normal_f32((E, H, I), dn_seed, dist_std)
     ids, w = synth.gumbel_topk_router(m, E, topk, r_seed)
     if bad_ids:
         ids[0, 1] = E + 1
-    x = synth.activations_bf16(m, H, x_seed)
+    x = synth.f32_to_bf16_bits(synth.normal_f32((m, H), x_seed, x_std))
     pu = tq.tq4_1s_quantize(torch.from_numpy(up).to(DEV), seed=up_seed)
     pd = tq.tq4_1s_quantize(torch.from_numpy(dn).to(DEV), seed=dn_seed)
     y = tq.tq4_1s_moe(_bf16_dev(x), torch.from_numpy(ids).to(DEV), torch.from_numpy(w).to(DEV), pu, pd)
@@ -205,6 +205,15 @@ def test_moe_bad_id_skipped():
     assert bad == 1
     assert_close(_bits(y), y_ref, "moe bad id")
     assert tq.tq4_1s_get_status() & tq.TQ_DEV_BAD_ROUTING
+
+
+@pytest.mark.parametrize("x_std,w_std", [(3000.0, 0.0005), (1e-5, 30.0)])
+def test_moe_activation_range(x_std, w_std):
+    # activations far outside (and far inside) the fp16 range: the per-row
+    # power-of-two scaling of the rotated activations keeps full precision
+    y, y_ref, _ = _moe_case(4, 128, 96, 6, 2, (34, 35, 36, 37), dist_std=w_std, x_std=x_std)
+    assert np.all(np.isfinite(y.float().cpu().numpy()))
+    assert_close(_bits(y), y_ref, f"moe range x_std={x_std}")
 
 
 def test_moe_128_experts_top6_full():
