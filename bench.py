@@ -325,8 +325,56 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     return out
 
 
+def profile_arm(args):
+    """Eager calls of one workload for ncu captures (no graphs, no oracle).
+
+    decode:  16-token linear on 16 distinct 4096x4096 weight copies (168 MB,
+             larger than L2), args.iters calls;
+    moe:     128 experts top-6, 16 tokens, args.iters calls;
+    prefill: M=8192 linear, args.iters calls."""
+    import numpy as np
+    import torch
+
+    import bit_rotated_weight_b200 as tq
+    import synth
+    dev = torch.device("cuda:0")
+    torch.cuda.set_device(dev)
+    if args.profile == "decode":
+        W = torch.from_numpy(synth.student_t_f32((N_OUT, K_IN), 2, 5.0, 0.02)).to(dev)
+        base = tq.tq4_1s_quantize(W, seed=2)
+        copies = [tq.Packed(base.codes.clone(), base.scales.clone(), N_OUT, K_IN, 1, 2) for _ in range(16)]
+        x = torch.from_numpy(synth.activations_bf16(M_TOK, K_IN, 3).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((M_TOK, N_OUT), dtype=torch.bfloat16, device=dev)
+        for i in range(args.iters):
+            tq.tq4_1s_linear(x, copies[i % 16], out=y)
+    elif args.profile == "moe":
+        E, H, I, mt, topk = 128, 2688, 1856, 16, 6
+        up = tq.tq4_1s_quantize(torch.from_numpy(synth.normal_f32((E, I, H), 4, 0.02)).to(dev), seed=4)
+        dn = tq.tq4_1s_quantize(torch.from_numpy(synth.normal_f32((E, H, I), 5, 0.02)).to(dev), seed=5)
+        torch.cuda.empty_cache()
+        ids, w = synth.gumbel_topk_router(mt, E, topk, 7)
+        xm = torch.from_numpy(synth.activations_bf16(mt, H, 6).view(np.int16)).to(dev).view(torch.bfloat16)
+        ids_d, w_d = torch.from_numpy(ids).to(dev), torch.from_numpy(w).to(dev)
+        for _ in range(args.iters):
+            tq.tq4_1s_moe(xm, ids_d, w_d, up, dn)
+    else:
+        m, n, k = 8192, 14336, 4096
+        p = tq.tq4_1s_quantize(torch.from_numpy(synth.normal_f32((n, k), 8, 0.02)).to(dev), seed=8)
+        torch.cuda.empty_cache()
+        x = torch.from_numpy(synth.activations_bf16(m, k, 9).view(np.int16)).to(dev).view(torch.bfloat16)
+        y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+        for _ in range(args.iters):
+            tq.tq4_1s_linear(x, p, out=y)
+    torch.cuda.synchronize()
+    assert tq.tq4_1s_get_status() == 0
+    print(json.dumps({"profile": args.profile, "iters": args.iters, "launches": tq.tq4_1s_launch_count()}))
+
+
 def main():
     ap = argparse.ArgumentParser()
+    ap.add_argument("--profile", choices=["decode", "moe", "prefill"], default=None,
+                    help="run eager calls of one workload (for ncu) instead of the benchmark")
+    ap.add_argument("--iters", type=int, default=8)
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
@@ -335,7 +383,9 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
-    if args.impl == "reference":
+    if args.profile:
+        profile_arm(args)
+    elif args.impl == "reference":
         reference_arm(args)
     else:
         ours_arm(args)
