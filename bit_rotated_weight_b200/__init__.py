@@ -258,3 +258,25 @@ def tq4_1s_get_status(device=None) -> int:
 def tq4_1s_launch_count() -> int:
     """Kernel launches issued through the library by this process so far."""
     return int(load_library().tq4_1s_launch_count())
+
+
+def tq4_1s_linear_static(x: torch.Tensor, w: Packed, out: torch.Tensor | None = None) -> torch.Tensor:
+    """tq4_1s_linear without a workspace, for callers that cannot allocate.
+
+    Runs the small-m linear path with its scratch held in a fixed device array
+    inside the library (m <= 32, k <= 8192, n <= 32768).  Calls that overlap
+    on the GPU share that array and race; serialize them.  The first call on a
+    device looks up the array's address, so make it outside stream capture.
+    """
+    lib = load_library()
+    fn = lib.tq4_1s_linear_static
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(_Weight), ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a CUDA bfloat16 [m][k] tensor")
+    x = x.contiguous()
+    if out is None:
+        out = torch.empty((x.shape[0], w.n), dtype=torch.bfloat16, device=x.device)
+    wst = w.c_struct()
+    _check(fn(_ptr(x), x.shape[0], ctypes.byref(wst), _ptr(out), _stream(x.device)), "linear_static")
+    return out

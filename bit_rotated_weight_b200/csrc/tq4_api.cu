@@ -264,6 +264,7 @@ TQ_API const char* tq4_1s_error_string(int code) {
     case TQ_ERR_TIMEOUT: return "a bounded device wait timed out";
     case TQ_ERR_BAD_ROUTING: return "routing expert id out of range";
     case TQ_ERR_NONFINITE: return "non-finite value in quantize input";
+    case TQ_ERR_SCRATCH_LIMIT: return "shape exceeds the fixed scratch of tq4_1s_linear_static (m<=32, k<=8192, n<=32768)";
     default: return "unknown error code";
   }
 }

@@ -1,0 +1,159 @@
+// tq4_1s_linear_static: the small-m quantized linear layer for callers that
+// cannot allocate device memory.
+//
+// Some hosts of this layer hand it only its input and output buffers: plugin
+// runtimes and serving engines that plan every device allocation at start-up
+// and forbid new ones afterwards (cudaMalloc can synchronize the device, fail
+// under memory pressure mid-request, or break a fixed memory budget).  Such a
+// caller cannot supply the workspace tq4_1s_linear asks for.  This entry point
+// runs the same two kernels as tq4_1s_linear's small-m path (activation
+// rotation, then the stream-K dequant-GEMM) but keeps their scratch -- the
+// rotated activations, the stream-K partial sums and the tile counters -- in
+// one file-scope device array of fixed size, allocated once per GPU when the
+// library's module loads there and held until the process exits.
+#include <mutex>
+
+#include "tq4_internal.h"
+
+#define TQ_STATIC_API extern "C" __attribute__((visibility("default")))
+
+namespace tq4 {
+namespace {
+
+// Limits of the static scratch: m <= 32 rows, k <= 8192, n <= 32768, and at
+// most 148 CTAs in the stream-K grid.
+constexpr int64_t kStaticMaxM = 32;
+constexpr int64_t kStaticMaxK = 8192;
+constexpr int64_t kStaticMaxN = 32768;
+constexpr int kStaticMaxGrid = 148;
+constexpr size_t kStaticXBytes = static_cast<size_t>(kStaticMaxM * kStaticMaxK) * 2;   // x' hi (or lo)
+constexpr size_t kStaticPartialBytes = static_cast<size_t>(kStaticMaxGrid) * 2 * 128 * kSegRows * 4;
+constexpr size_t kStaticCounterBytes = static_cast<size_t>(kStaticMaxN / 128) * 4;
+constexpr size_t kStaticScratchBytes = 2 * kStaticXBytes + kStaticPartialBytes + kStaticCounterBytes;  // ~5.6 MiB
+
+// The scratch itself.  In host code this name is only a stand-in for the
+// device symbol: its device address must be fetched with cudaGetSymbolAddress.
+static __device__ __align__(256) unsigned char g_linear_scratch[kStaticScratchBytes];
+
+// Device address of g_linear_scratch on the current device, looked up once
+// per device (with that device current) and cached.
+int scratch_address(void** out) {
+  static std::mutex mu;
+  static void* addr[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return TQ_ERR_UNSUPPORTED_DEVICE;
+  }
+  std::lock_guard<std::mutex> g(mu);
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_linear_scratch) != cudaSuccess || !p) {
+      cudaGetLastError();
+      return TQ_ERR_CUDA;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return TQ_OK;
+}
+
+}  // namespace
+}  // namespace tq4
+
+using namespace tq4;
+
+TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y,
+                                       tq4_stream_t stream) {
+  if (!w) return TQ_ERR_INVALID_ARG;
+  if (w->n <= 0 || w->k <= 0 || (w->k % 32) != 0 || w->num_experts != 1 || w->reserved != 0 || m < 0)
+    return TQ_ERR_INVALID_ARG;
+  if (!w->codes || !w->scales) return TQ_ERR_INVALID_ARG;
+  if (m > kStaticMaxM || w->k > kStaticMaxK || w->n > kStaticMaxN) return TQ_ERR_SCRATCH_LIMIT;
+  if (m == 0) return TQ_OK;
+  if (!x || !y) return TQ_ERR_INVALID_ARG;
+  auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!a16(x) || !a16(y) || !a16(w->codes) || !a16(w->scales)) return TQ_ERR_ALIGNMENT;
+  int dev = 0, major = 0, minor = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return TQ_ERR_UNSUPPORTED_DEVICE;
+  }
+  if (major != 10 || minor != 0) return TQ_ERR_UNSUPPORTED_DEVICE;
+  void* scratch = nullptr;
+  int rc = scratch_address(&scratch);
+  if (rc) return rc;
+
+  uint8_t* base = static_cast<uint8_t*>(scratch);
+  uint16_t* xh = reinterpret_cast<uint16_t*>(base);
+  uint16_t* xl = reinterpret_cast<uint16_t*>(base + kStaticXBytes);
+  float* partials = reinterpret_cast<float*>(base + 2 * kStaticXBytes);
+  int32_t* counters = reinterpret_cast<int32_t*>(base + 2 * kStaticXBytes + kStaticPartialBytes);
+  const int64_t row_tiles = (w->n + 127) / 128, k_iters = (w->k + 127) / 128;
+  const int64_t tiles = row_tiles;   // m <= 32: one segment
+  const int64_t T = tiles * k_iters;
+  int grid = sms < kStaticMaxGrid ? sms : kStaticMaxGrid;
+  if (T < grid) grid = static_cast<int>(T);
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint32_t mask = 0;
+  tq4_1s_sign_mask(w->seed, &mask);
+
+  // The rotation kernel also zeroes this call's tile counters, which the
+  // previous call left in the shared scratch.
+  if (launch_rotate_act(x, w->k, nullptr, 1, nullptr, m, m, xh, xl, mask, counters, tiles, st) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  alignas(64) CUtensorMap tc, th, tl;
+  {
+    // same tensor maps as tq4_1s_linear: codes [1][n][k/2] (64 B x 128 rows),
+    // x' hi/lo [m][k] (64 x 16)
+    typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+    static EncodeFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+      void* p = nullptr;
+      cudaDriverEntryPointQueryResult q;
+      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+          q == cudaDriverEntryPointSuccess)
+        fn = reinterpret_cast<EncodeFn>(p);
+      else
+        cudaGetLastError();
+    });
+    if (!fn) return TQ_ERR_CUDA;
+    const cuuint32_t es[3] = {1, 1, 1};
+    const cuuint64_t cd[3] = {static_cast<cuuint64_t>(w->k / 2), static_cast<cuuint64_t>(w->n), 1};
+    const cuuint64_t cs[2] = {static_cast<cuuint64_t>(w->k / 2), static_cast<cuuint64_t>(w->n * (w->k / 2))};
+    const cuuint32_t cb[3] = {64, 128, 1};
+    const cuuint64_t xd[2] = {static_cast<cuuint64_t>(w->k), static_cast<cuuint64_t>(m)};
+    const cuuint64_t xs[1] = {static_cast<cuuint64_t>(w->k * 2)};
+    const cuuint32_t xb[2] = {64, 16};
+    if (fn(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, cd, cs, cb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+            CUDA_SUCCESS ||
+        fn(&th, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xh, xd, xs, xb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+            CUDA_SUCCESS ||
+        fn(&tl, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xl, xd, xs, xb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
+            CUDA_SUCCESS)
+      return TQ_ERR_CUDA;
+  }
+  StreamKArgs a{};
+  a.n = static_cast<int32_t>(w->n);
+  a.k = static_cast<int32_t>(w->k);
+  a.row_tiles = static_cast<int32_t>(row_tiles);
+  a.k_iters = static_cast<int32_t>(k_iters);
+  a.nseg_host = 1;
+  a.m_host = static_cast<int32_t>(m);
+  a.scales = w->scales;
+  a.mode = EPI_DENSE;
+  a.out_a = y;
+  a.partials = partials;
+  a.counters = counters;
+  a.max_tiles = static_cast<int32_t>(tiles);
+  return launch_streamk(&tc, &th, &tl, a, grid, st) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+}

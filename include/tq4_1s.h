@@ -61,7 +61,8 @@ enum {
   TQ_ERR_CUDA = 5,                /* a CUDA runtime/driver call failed */
   TQ_ERR_TIMEOUT = 6,             /* status: a bounded device wait gave up */
   TQ_ERR_BAD_ROUTING = 7,         /* status: a routing expert id was out of range */
-  TQ_ERR_NONFINITE = 8            /* status: quantize saw a NaN or infinity */
+  TQ_ERR_NONFINITE = 8,           /* status: quantize saw a NaN or infinity */
+  TQ_ERR_SCRATCH_LIMIT = 9        /* tq4_1s_linear_static: shape beyond its fixed scratch */
 };
 
 /* Bits of the device status word (tq4_1s_get_status). */
@@ -136,6 +137,26 @@ size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
  * the workspace and runs a tensor-core GEMM.  m == 0 is a no-op. */
 int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, void* ws, size_t ws_bytes,
                   tq4_stream_t stream);
+
+/* tq4_1s_linear for callers that cannot allocate device memory.  (The model
+ * card has no counterpart: this is a deployment variant of the layer above.)
+ * Plugin hosts and serving runtimes that fix every device allocation at
+ * start-up and forbid new ones later cannot hand tq4_1s_linear a workspace;
+ * this entry point takes only x, w and y and keeps its scratch (rotated
+ * activations, stream-K partial sums, tile counters) in a fixed device array
+ * inside the library: about 5.6 MiB, reserved on every GPU that loads the
+ * library and held until the process exits.
+ *   Limits: m <= 32, w->k <= 8192, w->n <= 32768, dense weight; larger
+ *   shapes return TQ_ERR_SCRATCH_LIMIT and launch nothing.
+ *   The first call on a device looks up the array's device address (with
+ *   that device current); make that first call outside any stream capture.
+ *   All calls share the one array, so calls that overlap on the GPU (on
+ *   different streams, or from different host threads) race and corrupt each
+ *   other's results; serialize them.  Each call clears the counters it
+ *   needs, so the previous call's leftovers do no harm.
+ * Same arguments, result and numerics as tq4_1s_linear's small-m path; no
+ * allocation of any kind. */
+int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, tq4_stream_t stream);
 
 /* Bytes of workspace tq4_1s_moe needs.  0 on invalid arguments. */
 size_t tq4_1s_moe_workspace(int64_t m, int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* down);

@@ -1,0 +1,58 @@
+"""tq4_1s_linear_static -- the linear layer for callers that cannot allocate.
+
+Plugin hosts and serving runtimes that fix their device memory at start-up
+cannot hand tq4_1s_linear a workspace; tq4_1s_linear_static keeps its scratch
+in a fixed array inside the library instead.  This test calls it through the
+C ABI twice in a row (the second call runs on the scratch the first one left
+behind) and checks each result against tq4_1s_linear, which uses a caller
+workspace, with the same tolerances as the parity tests.  It lives in a file
+of its own that pytest collects last.
+"""
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+import synth
+from tests._parity import assert_close
+
+pytestmark = pytest.mark.gpu
+
+tq = pytest.importorskip("bit_rotated_weight_b200")
+
+
+def _bits(t):
+    return t.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
+
+def _to_dev(bits, dev):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+
+def test_static_scratch_linear_matches_workspace_linear():
+    dev = torch.device("cuda:0")
+    lib = tq.load_library()
+    fn = lib.tq4_1s_linear_static
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(tq._Weight), ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    W = torch.from_numpy(synth.student_t_f32((4096, 4096), 2, 5.0, 0.02)).to(dev)
+    p = tq.tq4_1s_quantize(W, seed=2)
+    wst = p.c_struct()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    for call, (m, seed) in enumerate([(16, 3), (13, 5)]):
+        x = _to_dev(synth.activations_bf16(m, 4096, seed), dev)
+        ref = tq.tq4_1s_linear(x, p)
+        y = torch.empty((m, 4096), dtype=torch.bfloat16, device=dev)
+        rc = fn(ctypes.c_void_p(x.data_ptr()), m, ctypes.byref(wst), ctypes.c_void_p(y.data_ptr()), stream)
+        assert rc == 0, tq.tq4_1s_error_string(rc)
+        torch.cuda.synchronize()
+        ref_f = _bits(ref).astype(np.uint32) << 16
+        assert_close(_bits(y), ref_f.view(np.float32).astype(np.float64), f"static call {call}")
+    assert tq.tq4_1s_get_status() == 0
+    # shapes beyond the fixed scratch are refused without a launch
+    big = tq.Packed(p.codes, p.scales, 4096, 4096, 1, 2)
+    x40 = torch.zeros((40, 4096), dtype=torch.bfloat16, device=dev)
+    y40 = torch.empty((40, 4096), dtype=torch.bfloat16, device=dev)
+    bst = big.c_struct()
+    assert fn(ctypes.c_void_p(x40.data_ptr()), 40, ctypes.byref(bst), ctypes.c_void_p(y40.data_ptr()), stream) == 9
