@@ -289,7 +289,7 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     del W
     x = torch.from_numpy(synth.activations_bf16(m, k, 9).view(np.int16)).to(dev).view(torch.bfloat16)
     y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
-    wsp = torch.empty(tq.tq4_1s_linear_workspace(m, p), dtype=torch.uint8, device=dev)
+    wsp = torch.zeros(tq.tq4_1s_linear_workspace(m, p), dtype=torch.uint8, device=dev)
     for _ in range(3):
         tq.tq4_1s_linear(x, p, out=y, workspace=wsp)
     it = 10

@@ -179,11 +179,19 @@ def tq4_1s_dequantize(w: Packed) -> torch.Tensor:
 _ws_cache: dict = {}
 
 
-def _workspace(nbytes: int, device) -> torch.Tensor:
-    key = (str(device),)
+SMALL_M = 128   # tq4_1s_linear takes its stream-K path up to this many rows
+
+
+def _workspace(nbytes: int, device, kind: str) -> torch.Tensor:
+    """A cached, zero-filled workspace per (device, kind).
+
+    The small-m linear path needs its tile counters zero at the start of a
+    call and leaves them zero, so its workspace is kept apart from the
+    large-m path (which writes the dequantized weight into its own)."""
+    key = (str(device), kind)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:
-        buf = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+        buf = torch.zeros(max(nbytes, 256), dtype=torch.uint8, device=device)
         _ws_cache[key] = buf
     return buf
 
@@ -205,7 +213,7 @@ def tq4_1s_linear(x: torch.Tensor, w: Packed, out: torch.Tensor | None = None,
     wst = w.c_struct()
     need = load_library().tq4_1s_linear_workspace(m, ctypes.byref(wst))
     if workspace is None:
-        workspace = _workspace(need, x.device)
+        workspace = _workspace(need, x.device, "linear_small" if m <= SMALL_M else "linear_large")
     _check(load_library().tq4_1s_linear(_ptr(x), m, ctypes.byref(wst), _ptr(out), _ptr(workspace),
                                         workspace.numel(), _stream(x.device)), "linear")
     return out
@@ -230,7 +238,7 @@ def tq4_1s_moe(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, up
     u, d = up.c_struct(), down.c_struct()
     need = load_library().tq4_1s_moe_workspace(m, topk, ctypes.byref(u), ctypes.byref(d))
     if workspace is None:
-        workspace = _workspace(need, x.device)
+        workspace = _workspace(need, x.device, "moe")
     _check(load_library().tq4_1s_moe(_ptr(x), m, _ptr(topk_ids), _ptr(topk_w), topk, ctypes.byref(u),
                                      ctypes.byref(d), _ptr(out), _ptr(workspace), workspace.numel(),
                                      _stream(x.device)), "moe")

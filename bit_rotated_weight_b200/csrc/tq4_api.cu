@@ -2,6 +2,7 @@
 // include/tq4_1s.h -- argument validation, the codebook, the RHT sign mask,
 // TMA tensor-map construction and the launch sequences of each call.
 #include <atomic>
+#include <climits>
 #include <cmath>
 #include <cstdio>
 #include <cstring>
@@ -181,11 +182,15 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int64_t kSmallM = 128;
 
 struct SmallLayout {
-  size_t xh, xl, partials, counters, total;
+  size_t partials, counters, total;
   int grid;
   int64_t tiles;
 };
 
+// Small-m workspace: the fp32 partials first (their size depends only on the
+// SM count), the tile counters after them.  The counters therefore start at
+// the same offset for every shape, so a workspace shared by small-m calls of
+// different shapes never sees another call's partials in its counters.
 static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
   SmallLayout L{};
   const int64_t nseg = (m + kSegRows - 1) / kSegRows;
@@ -194,10 +199,6 @@ static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
   const int64_t T = L.tiles * ki;
   L.grid = static_cast<int>(T < sms ? T : sms);
   size_t off = 0;
-  L.xh = off;
-  off = align256(off + static_cast<size_t>(m * w->k) * 2);
-  L.xl = off;
-  off = align256(off + static_cast<size_t>(m * w->k) * 2);
   L.partials = off;
   off = align256(off + static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
   L.counters = off;
@@ -343,13 +344,12 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
 
   if (m <= kSmallM) {
     const SmallLayout L = small_layout(m, w, sms);
-    uint16_t* xh = reinterpret_cast<uint16_t*>(base + L.xh);
-    uint16_t* xl = reinterpret_cast<uint16_t*>(base + L.xl);
+    if (L.tiles * ((w->k + 127) / 128) > INT32_MAX) return TQ_ERR_INVALID_ARG;   // 32-bit iteration space
     int32_t* counters = reinterpret_cast<int32_t*>(base + L.counters);
-    cudaError_t e = launch_rotate_act(x, w->k, nullptr, 1, nullptr, m, m, xh, xl, mask, counters, L.tiles, st);
-    if (e != cudaSuccess) return TQ_ERR_CUDA;
+    // One launch: the kernel rotates x itself (no x' round trip through
+    // memory).  The x' maps are unused in this mode; they point at x.
     alignas(64) CUtensorMap tc, th, tl;
-    if (!map_codes(&tc, w) || !map_bf16(&th, xh, m, w->k, 16) || !map_bf16(&tl, xl, m, w->k, 16))
+    if (!map_codes(&tc, w) || !map_bf16(&th, x, m, w->k, 16) || !map_bf16(&tl, x, m, w->k, 16))
       return TQ_ERR_CUDA;
     StreamKArgs a{};
     a.n = static_cast<int32_t>(w->n);
@@ -358,9 +358,12 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     a.k_iters = static_cast<int32_t>((w->k + 127) / 128);
     a.nseg_host = static_cast<int32_t>((m + kSegRows - 1) / kSegRows);
     a.m_host = static_cast<int32_t>(m);
+    a.nb_max = m > 16 ? 2 : 1;
     a.scales = w->scales;
     a.mode = EPI_DENSE;
     a.out_a = y;
+    a.x_raw = x;
+    a.x_mask = mask;
     a.partials = reinterpret_cast<float*>(base + L.partials);
     a.counters = counters;
     a.max_tiles = static_cast<int32_t>(L.tiles);
@@ -377,6 +380,8 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
   return cuda_rc(launch_gemm_bf16(&tx, &tw, y, static_cast<int32_t>(m), static_cast<int32_t>(w->n),
                                   static_cast<int32_t>(w->k), grid, st));
 }
+
+static int64_t H_of(const tq4_1s_weight* up) { return up->k; }
 
 static int moe_check(int64_t m, int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* down, bool ptrs) {
   int rc = weight_ok(up, ptrs);
@@ -405,6 +410,9 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   int sms = 0;
   if ((rc = check_device(&sms))) return rc;
   const MoeLayout L = moe_layout(m, topk, up, down, sms);
+  if (L.maxseg * L.rt_up * ((H_of(up) + 127) / 128) > INT32_MAX ||
+      L.maxseg * L.rt_dn * ((up->n + 127) / 128) > INT32_MAX)
+    return TQ_ERR_INVALID_ARG;   // 32-bit iteration space
   if (!ws || ws_bytes < L.total) return TQ_ERR_WORKSPACE;
   if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
@@ -443,6 +451,7 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   a.k_iters = static_cast<int32_t>((H + 127) / 128);
   a.segs = segs;
   a.nseg_dev = nseg;
+  a.nb_max = m > 16 ? 2 : 1;   // an expert takes each token at most once (top-k ids are distinct)
   a.scales = up->scales;
   a.f16 = 1;
   a.row_scale = xscale;

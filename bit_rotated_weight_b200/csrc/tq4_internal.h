@@ -51,6 +51,7 @@ struct StreamKArgs {
   int32_t k_iters;           // ceil(k / 128)
   int32_t nseg_host;         // segment count when segs == nullptr (dense): ceil(m / kSegRows)
   int32_t m_host;            // dense row count
+  int32_t nb_max;            // max 16-row blocks per segment (1 or 2): accumulator layout
   const int4* segs;          // device segment list (MoE) or nullptr
   const int32_t* nseg_dev;   // device segment count (MoE) or nullptr
   const uint16_t* scales;    // [E][n][k/16]
@@ -63,6 +64,8 @@ struct StreamKArgs {
   uint32_t next_mask;        // up: sign mask of the down projection
   int32_t f16;               // operands: 0 = bf16 (x' hi/lo), 1 = fp16 (x' hi/lo scaled by row_scale)
   const float* row_scale;    // fp16 mode: x' row r was multiplied by 1/row_scale[r]
+  const uint16_t* x_raw;     // dense bf16 mode: raw x [m][k]; warps of the kernel rotate it (x' hi/lo)
+  uint32_t x_mask;           // sign mask of the weight (for the fused rotation)
   float* partials;           // [grid][2][128][kSegRows]
   int32_t* counters;         // [tiles]
   int32_t max_tiles;         // capacity of counters

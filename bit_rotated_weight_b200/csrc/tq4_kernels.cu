@@ -43,66 +43,120 @@ __device__ __forceinline__ float load_w<float>(const float* p) { return __ldg(p)
 template <>
 __device__ __forceinline__ float load_w<uint16_t>(const uint16_t* p) { return bf16_bits_to_f32(__ldg(p)); }
 
+// One thread per 32-element block: the whole butterfly runs in registers in
+// the fixed order (stage h pairs elements j and j+h for j with bit h clear),
+// so the result is bit-identical to the warp-shuffle form and to the oracle.
+__device__ __forceinline__ void fwht32_regs(float (&a)[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (!(j & h)) {
+        const float x = a[j], y = a[j + h];
+        a[j] = __fadd_rn(x, y);
+        a[j + h] = __fsub_rn(x, y);
+      }
+    }
+  }
+}
+
+template <typename T>
+__device__ __forceinline__ void load_block(const T* p, float (&w)[32]);
+template <>
+__device__ __forceinline__ void load_block<float>(const float* p, float (&w)[32]) {
+  const float4* q = reinterpret_cast<const float4*>(p);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float4 f = __ldg(q + i);
+    w[4 * i] = f.x;
+    w[4 * i + 1] = f.y;
+    w[4 * i + 2] = f.z;
+    w[4 * i + 3] = f.w;
+  }
+}
+template <>
+__device__ __forceinline__ void load_block<uint16_t>(const uint16_t* p, float (&w)[32]) {
+  const uint4* q = reinterpret_cast<const uint4*>(p);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const uint4 u = __ldg(q + i);
+    const uint32_t v[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      w[8 * i + 2 * j] = __uint_as_float(v[j] << 16);
+      w[8 * i + 2 * j + 1] = __uint_as_float(v[j] & 0xFFFF0000u);
+    }
+  }
+}
+
+// Quantize: one thread per 32-block (sign flip, butterfly, x r, per-half RMS
+// by the pairwise tree, fp16 scale, nearest level by the thresholds, nibble
+// packing).  Consecutive threads take consecutive blocks of a row.
 template <typename T>
 __global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ W, uint8_t* __restrict__ codes,
                                                        uint16_t* __restrict__ scales, int64_t rows, int64_t k,
                                                        uint32_t mask, CodebookF32 cb) {
   __shared__ float s_t[16];
-  if (threadIdx.x < 15) s_t[threadIdx.x] = cb.thresholds[threadIdx.x];
+  if (threadIdx.x < 16) s_t[threadIdx.x] = cb.thresholds[threadIdx.x];
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const float sgn_neg = ((mask >> lane) & 1u) ? -1.0f : 1.0f;
   const int64_t kb_per_row = k / 32;
   const int64_t nblocks = rows * kb_per_row;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float r = rsqrt32();
-  for (int64_t b = warp; b < nblocks; b += nwarps) {
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
-    const float w = load_w<T>(W + row * k + kb * 32 + lane);
-    if (__any_sync(0xFFFFFFFFu, !isfinite(w)) && lane == 0) raise_status(TQ_DEV_NONFINITE);
-    const float a = warp_fwht32(w * sgn_neg, lane);  // sign flip is exact
-    const float v = __fmul_rn(a, r);
-    // half-block mean square: pairwise tree with strides 8, 4, 2, 1
-    float p = __fmul_rn(v, v);
+    float a[32];
+    load_block<T>(W + row * k + kb * 32, a);
+    bool finite = true;
 #pragma unroll
-    for (int s = 8; s >= 1; s >>= 1) p = __fadd_rn(p, __shfl_down_sync(0xFFFFFFFFu, p, s, 16));
-    const float S = __shfl_sync(0xFFFFFFFFu, p, 0, 16);
-    const float rms = __fsqrt_rn(__fmul_rn(S, 0.0625f));
-    const uint16_t dbits = f16_sat_bits(rms);
-    const float d = __half2float(__ushort_as_half(dbits));
-    uint32_t code;
-    if (d == 0.0f) {
-      code = 7u;
-    } else {
-      const float u = __fdiv_rn(v, d);
-      // number of thresholds strictly below u (binary search over sorted t)
-      code = 0u;
-      code += (u > s_t[7]) ? 8u : 0u;
-      code += (u > s_t[code + 3]) ? 4u : 0u;
-      code += (u > s_t[code + 1]) ? 2u : 0u;
-      code += (u > s_t[code]) ? 1u : 0u;
+    for (int i = 0; i < 32; ++i) {
+      finite = finite && isfinite(a[i]);
+      if ((mask >> i) & 1u) a[i] = -a[i];
     }
-    // pack: byte i/2 <- code(2i) | code(2i+1) << 4 ; 16 bytes per block
-    const uint32_t hi = __shfl_down_sync(0xFFFFFFFFu, code, 1);
-    const uint32_t byte = code | (hi << 4);
-    const uint32_t b1 = __shfl_down_sync(0xFFFFFFFFu, byte, 2);
-    const uint32_t b2 = __shfl_down_sync(0xFFFFFFFFu, byte, 4);
-    const uint32_t b3 = __shfl_down_sync(0xFFFFFFFFu, byte, 6);
-    const uint32_t word = byte | (b1 << 8) | (b2 << 16) | (b3 << 24);  // valid on lanes 0, 8, 16, 24
-    const uint32_t w1 = __shfl_sync(0xFFFFFFFFu, word, 8);
-    const uint32_t w2 = __shfl_sync(0xFFFFFFFFu, word, 16);
-    const uint32_t w3 = __shfl_sync(0xFFFFFFFFu, word, 24);
-    const uint32_t d1 = __shfl_sync(0xFFFFFFFFu, static_cast<uint32_t>(dbits), 16);
-    if (lane == 0) {
-      *reinterpret_cast<uint4*>(codes + row * (k / 2) + kb * 16) = make_uint4(word, w1, w2, w3);
-      *reinterpret_cast<uint32_t*>(scales + row * (k / 16) + kb * 2) = static_cast<uint32_t>(dbits) | (d1 << 16);
+    if (!finite) raise_status(TQ_DEV_NONFINITE);
+    fwht32_regs(a);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) a[i] = __fmul_rn(a[i], r);
+    uint32_t words[4] = {0u, 0u, 0u, 0u};
+    uint32_t dpair = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      float p[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) p[i] = __fmul_rn(a[16 * h + i], a[16 * h + i]);
+#pragma unroll
+      for (int st = 8; st >= 1; st >>= 1)
+#pragma unroll
+        for (int i = 0; i < st; ++i) p[i] = __fadd_rn(p[i], p[i + st]);
+      const float rms = __fsqrt_rn(__fmul_rn(p[0], 0.0625f));
+      const uint16_t dbits = f16_sat_bits(rms);
+      dpair |= static_cast<uint32_t>(dbits) << (16 * h);
+      const float d = __half2float(__ushort_as_half(dbits));
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        uint32_t code;
+        if (d == 0.0f) {
+          code = 7u;
+        } else {
+          const float u = __fdiv_rn(a[16 * h + i], d);
+          // number of thresholds strictly below u (binary search, sorted t)
+          code = (u > s_t[7]) ? 8u : 0u;
+          code += (u > s_t[code + 3]) ? 4u : 0u;
+          code += (u > s_t[code + 1]) ? 2u : 0u;
+          code += (u > s_t[code]) ? 1u : 0u;
+        }
+        const int e = 16 * h + i;   // element index; nibble e of the 16-byte block
+        words[e >> 3] |= code << (4 * (e & 7));
+      }
     }
+    *reinterpret_cast<uint4*>(codes + row * (k / 2) + kb * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+    *reinterpret_cast<uint32_t*>(scales + row * (k / 16) + kb * 2) = dpair;
   }
 }
 
 // ------------------------------------------------------------------ dequantize
-// W_hat = diag(s) * r * H * (c[code] * d), fp32 or bf16 output.
+// W_hat = diag(s) * r * H * (c[code] * d), fp32 or bf16 output; one thread per
+// 32-block, butterfly in registers.
 template <typename TO>
 __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restrict__ codes,
                                                          const uint16_t* __restrict__ scales, TO* __restrict__ out,
@@ -110,25 +164,40 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
   __shared__ float s_c[16];
   if (threadIdx.x < 16) s_c[threadIdx.x] = cb.levels[threadIdx.x];
   __syncthreads();
-  const int lane = threadIdx.x & 31;
-  const bool neg = (mask >> lane) & 1u;
   const int64_t kb_per_row = k / 32;
   const int64_t nblocks = rows * kb_per_row;
-  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   const float r = rsqrt32();
-  for (int64_t b = warp; b < nblocks; b += nwarps) {
+  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
+       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
-    const uint32_t byte = __ldg(codes + row * (k / 2) + kb * 16 + (lane >> 1));
-    const uint32_t code = (lane & 1) ? (byte >> 4) : (byte & 0xFu);
-    const float d = __half2float(__ushort_as_half(__ldg(scales + row * (k / 16) + kb * 2 + (lane >> 4))));
-    const float wn = __fmul_rn(s_c[code], d);
-    const float a = __fmul_rn(warp_fwht32(wn, lane), r);
-    const float o = neg ? -a : a;
+    const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes + row * (k / 2) + kb * 16));
+    const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(scales + row * (k / 16) + kb * 2));
+    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+    const float d0 = __half2float(__ushort_as_half(static_cast<uint16_t>(sw & 0xFFFFu)));
+    const float d1 = __half2float(__ushort_as_half(static_cast<uint16_t>(sw >> 16)));
+    float a[32];
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const uint32_t code = (words[e >> 3] >> (4 * (e & 7))) & 0xFu;
+      a[e] = __fmul_rn(s_c[code], e < 16 ? d0 : d1);
+    }
+    fwht32_regs(a);
+    TO* o = out + row * k + kb * 32;
+#pragma unroll
+    for (int e = 0; e < 32; ++e) {
+      const float x = __fmul_rn(a[e], r);
+      a[e] = ((mask >> e) & 1u) ? -x : x;
+    }
     if constexpr (sizeof(TO) == 4) {
-      out[row * k + kb * 32 + lane] = o;
+      float4* o4 = reinterpret_cast<float4*>(o);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o4[i] = make_float4(a[4 * i], a[4 * i + 1], a[4 * i + 2], a[4 * i + 3]);
     } else {
-      out[row * k + kb * 32 + lane] = __bfloat16_as_ushort(__float2bfloat16_rn(o));
+      uint4* o4 = reinterpret_cast<uint4*>(o);
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        o4[i] = make_uint4(pack_bf16x2(a[8 * i], a[8 * i + 1]), pack_bf16x2(a[8 * i + 2], a[8 * i + 3]),
+                           pack_bf16x2(a[8 * i + 4], a[8 * i + 5]), pack_bf16x2(a[8 * i + 6], a[8 * i + 7]));
     }
   }
 }
@@ -263,20 +332,58 @@ __global__ void __launch_bounds__(1024) moe_route_kernel(const int32_t* __restri
     else atomicAdd(&s_bad, 1);
   }
   __syncthreads();
+  // Exclusive scans over experts of (count, segment count), one expert per
+  // thread per pass of the block, carried across passes.
+  __shared__ int32_t s_wsum[2][32];
+  __shared__ int32_t s_carry[2];
   if (tid == 0) {
-    int32_t run = 0, ns = 0;
-    for (int e = 0; e < num_experts; ++e) {
-      offsets[e] = run;
-      base[e] = run;
-      for (int32_t c = 0; c < cnt[e]; c += chunk) {
-        if (segs) segs[ns] = make_int4(e, run + c, min(chunk, cnt[e] - c), 0);
-        ++ns;
+    s_carry[0] = 0;
+    s_carry[1] = 0;
+  }
+  __syncthreads();
+  const int lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+  for (int e0 = 0; e0 < num_experts; e0 += blockDim.x) {
+    const int e = e0 + tid;
+    const int32_t c = (e < num_experts) ? cnt[e] : 0;
+    const int32_t ns = (c + chunk - 1) / chunk;
+    int32_t ic = c, is = ns;   // inclusive warp scans
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t yc = __shfl_up_sync(0xFFFFFFFFu, ic, o), ys = __shfl_up_sync(0xFFFFFFFFu, is, o);
+      if (lane >= o) {
+        ic += yc;
+        is += ys;
       }
-      run += cnt[e];
     }
-    offsets[num_experts] = run;
-    if (npairs_valid) *npairs_valid = run;
-    if (nseg_out) *nseg_out = ns;
+    if (lane == 31) {
+      s_wsum[0][wid] = ic;
+      s_wsum[1][wid] = is;
+    }
+    __syncthreads();
+    int32_t pc = s_carry[0], ps = s_carry[1];
+    for (int w = 0; w < wid; ++w) {
+      pc += s_wsum[0][w];
+      ps += s_wsum[1][w];
+    }
+    const int32_t off = pc + ic - c, soff = ps + is - ns;
+    if (e < num_experts) {
+      offsets[e] = off;
+      base[e] = off;
+      if (segs)
+        for (int32_t k = 0; k < ns; ++k) segs[soff + k] = make_int4(e, off + k * chunk, min(chunk, c - k * chunk), 0);
+    }
+    __syncthreads();
+    if (tid == blockDim.x - 1) {
+      s_carry[0] = pc + ic;
+      s_carry[1] = ps + is;
+    }
+    __syncthreads();
+    (void)nw;
+  }
+  if (tid == 0) {
+    offsets[num_experts] = s_carry[0];
+    if (npairs_valid) *npairs_valid = s_carry[0];
+    if (nseg_out) *nseg_out = s_carry[1];
     if (s_bad) raise_status(TQ_DEV_BAD_ROUTING);
   }
   __syncthreads();
@@ -318,7 +425,15 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restric
 // ------------------------------------------------------------------ launchers
 static int grid_for(int64_t warps_needed, int threads) {
   int64_t blocks = (warps_needed * 32 + threads - 1) / threads;
-  const int64_t cap = 148LL * 16;
+  const int64_t cap = 148LL * (2048 / threads);   // one wave of resident threads
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  return static_cast<int>(blocks);
+}
+
+static int grid_threads(int64_t threads_needed, int threads) {
+  int64_t blocks = (threads_needed + threads - 1) / threads;
+  const int64_t cap = 148LL * (2048 / threads);
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   return static_cast<int>(blocks);
@@ -326,7 +441,7 @@ static int grid_for(int64_t warps_needed, int threads) {
 
 cudaError_t launch_quantize(const void* W, int dtype, uint8_t* codes, uint16_t* scales, int64_t rows, int64_t k,
                             uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
-  const int g = grid_for(rows * (k / 32), 256);
+  const int g = grid_threads(rows * (k / 32), 256);
   if (dtype == TQ_DTYPE_F32)
     quantize_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(W), codes, scales, rows, k, mask, cb);
   else
@@ -337,14 +452,16 @@ cudaError_t launch_quantize(const void* W, int dtype, uint8_t* codes, uint16_t* 
 
 cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, float* out, int64_t rows, int64_t k,
                                   uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
-  dequantize_kernel<float><<<grid_for(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k, mask, cb);
+  dequantize_kernel<float><<<grid_threads(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k, mask,
+                                                                                cb);
   note_launches(1);
   return cudaGetLastError();
 }
 
 cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales, uint16_t* out, int64_t rows,
                                    int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
-  dequantize_kernel<uint16_t><<<grid_for(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k, mask, cb);
+  dequantize_kernel<uint16_t><<<grid_threads(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k,
+                                                                                   mask, cb);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -149,6 +149,7 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   a.k_iters = static_cast<int32_t>(k_iters);
   a.nseg_host = 1;
   a.m_host = static_cast<int32_t>(m);
+  a.nb_max = m > 16 ? 2 : 1;
   a.scales = w->scales;
   a.mode = EPI_DENSE;
   a.out_a = y;

@@ -11,15 +11,18 @@
 //   warp 0      TMA: packed codes tile [128 x 64 B] (64-byte swizzle) and the
 //               x' hi/lo tiles [rows x 128 k] (128-byte swizzle) into a
 //               shared-memory stage, completing on an mbarrier;
-//   warps 4-11  two dequant warpgroups (alternate iterations), thread = row:
+//   warps 4-19  four dequant warpgroups (round-robin iterations), thread = row:
 //               16 B of codes + 8 fp16 scales -> 128 bf16 levels through a
 //               per-half-block scaled table looked up with byte permutes,
 //               written to tensor memory with tcgen05.st (the MMA A operand);
-//   warp 1      one thread issues 8 tcgen05.mma (M=128, N=32*nb, K=16,
-//               A from tensor memory, B from shared memory) into a TMEM
-//               accumulator and commits to the stage / A-stage barriers;
-//   warps 12-15 epilogue, thread = row: tcgen05.ld of the accumulator,
-//               hi + lo columns summed, then the mode's store.
+//               one thread of the group then issues 8 tcgen05.mma (M=128,
+//               N=32*nb, K=16, A from tensor memory, B from shared memory)
+//               into the group's own accumulator -- four concurrent issuers;
+//   warps 2-3   (dense bf16 mode) rotate x per 32-slice in registers and
+//               write the x' hi/lo B tiles into the stage, 128-byte swizzled;
+//   warp 1      allocates / frees tensor memory;
+//   warps 20-23 epilogue, thread = row: tcgen05.ld of the accumulator in
+//               16-token chunks, hi + lo columns summed, then the mode's store.
 // The flattened (segment, row tile, k iteration) space is split evenly over
 // the CTAs (stream-K).  A tile split between CTAs is finished by whichever
 // contributor arrives last on the tile's counter: it sums all contributors'
@@ -30,28 +33,37 @@
 namespace tq4 {
 namespace {
 
-constexpr int kThreads = 512;
+constexpr int kThreads = 768;
+constexpr int kDequantGroups = 4;
+constexpr int kFirstDequantWarp = 4;
+constexpr int kFirstEpilogueWarp = kFirstDequantWarp + 4 * kDequantGroups;
 constexpr int kStages = 8;
-constexpr int kAStages = 6;
+constexpr int kAStages = 4;
 constexpr int kCodesBytes = 128 * 64;    // 128 rows x 128 k codes
 constexpr int kXHalfBytes = 64 * 128;    // 64 rows x 64 k bf16 (one 128-B swizzle span)
 constexpr int kXBytes = 2 * kXHalfBytes; // two k-halves
 constexpr int kStageBytes = kCodesBytes + kXBytes;
 constexpr int kTmemCols = 512;
-constexpr int kDCols = 64;
-constexpr int kACol0 = 2 * kDCols;
+// Tensor memory: columns [0, 256) hold the accumulators, [256, 512) the four
+// A stages (one per dequant warpgroup, 64 columns = 128 k of bf16 levels).
+// Each warpgroup issues the MMAs of its own iterations into its own
+// accumulator (N = 32 * nb columns): single-thread tcgen05.mma issue costs
+// ~66-98 cycles per instruction at small N, so four concurrent issuers are
+// needed to keep pace with the weight stream.  With nb = 1 (<= 16 tokens per
+// segment) the four accumulators take 128 columns and two accumulator sets
+// alternate between tile portions; with nb = 2 one set of 256 columns.
+constexpr int kAccRegion = 256;
+constexpr int kACol0 = kAccRegion;
 constexpr int kAColsPerStage = 64;
 static_assert(kACol0 + kAStages * kAColsPerStage <= kTmemCols, "tensor memory budget");
-static_assert(kStages % 2 == 0 && kAStages % 2 == 0, "two dequant warpgroups alternate");
+static_assert(kAStages == kDequantGroups, "one A stage per dequant warpgroup");
 
 struct SharedState {
-  uint64_t full[kStages];
-  uint64_t empty[kStages];
-  uint64_t afull[kAStages];
-  uint64_t aempty[kAStages];
-  uint64_t dfull[2];
-  uint64_t dempty[2];
-  uint64_t mma_done;
+  uint64_t full[kStages];      // TMA landed (codes, x') and rotated x' written
+  uint64_t done[kStages];      // the MMAs of the iteration that used this stage completed
+  uint64_t dfull[2];           // all four warpgroups finished a portion (4 arrivals)
+  uint64_t dempty[2];          // the epilogue drained an accumulator set (128 arrivals)
+  uint64_t wg_done[kDequantGroups];
   uint32_t tmem_base;
   int abort_flag;
   int last_flag;
@@ -75,6 +87,29 @@ __device__ __forceinline__ Seg get_seg(const StreamKArgs& a, int s) {
 __device__ __forceinline__ int64_t range_begin(int64_t c, int64_t T, int64_t G) { return c * T / G; }
 // The CTA whose range holds iteration i.
 __device__ __forceinline__ int64_t owner_of(int64_t i, int64_t T, int64_t G) { return ((i + 1) * G + T - 1) / T - 1; }
+
+// Position of an iteration in the (segment, row tile, k iteration) space,
+// advanced incrementally so the loops do no integer division.
+struct Cursor {
+  int tile, kit, sgi, rt;
+  __device__ __forceinline__ void init(int64_t it, int KI, int RT) {
+    tile = static_cast<int>(it / KI);
+    kit = static_cast<int>(it - static_cast<int64_t>(tile) * KI);
+    sgi = tile / RT;
+    rt = tile - sgi * RT;
+  }
+  __device__ __forceinline__ void advance(int n, int KI, int RT) {
+    kit += n;
+    while (kit >= KI) {
+      kit -= KI;
+      ++tile;
+      if (++rt == RT) {
+        rt = 0;
+        ++sgi;
+      }
+    }
+  }
+};
 
 // Bounded wait that ignores the abort flag (used while winding down).
 __device__ __forceinline__ void drain_wait(uint64_t* bar, uint32_t parity) {
@@ -156,6 +191,21 @@ __device__ __forceinline__ void dequant_half(uint32_t q0, uint32_t q1, float d, 
   }
 }
 
+// 32-point Sylvester butterfly on a register array (stages h = 1..16).
+__device__ __forceinline__ void fwht32_regs_sk(float (&a)[32]) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+      if (!(j & h)) {
+        const float x = a[j], y = a[j + h];
+        a[j] = __fadd_rn(x, y);
+        a[j + h] = __fsub_rn(x, y);
+      }
+    }
+  }
+}
+
 __device__ __forceinline__ float relu2_bf16(float v) {
   const float r = fmaxf(v, 0.0f);
   return __bfloat162float(__float2bfloat16_rn(__fmul_rn(r, r)));
@@ -170,20 +220,23 @@ __device__ __forceinline__ float warp_fwht32_epi(float a, int lane) {
   return a;
 }
 
-// The per-mode store of one finished tile row (thread = weight row `row`).
-__device__ __forceinline__ void epilogue_store(const StreamKArgs& a, float (&v)[kSegRows], int row, int lane,
+// The per-mode store of 16 tokens [j0, j0 + 16) of one finished tile row
+// (thread = weight row `row`).
+__device__ __forceinline__ void epilogue_store(const StreamKArgs& a, float (&v)[16], int j0, int row, int lane,
                                                const Seg& sg) {
+  const int cnt = sg.count - j0;
   if (a.row_scale) {
 #pragma unroll
-    for (int j = 0; j < kSegRows; ++j)
-      if (j < sg.count) v[j] = __fmul_rn(v[j], a.row_scale[sg.row0 + j]);
+    for (int j = 0; j < 16; ++j)
+      if (j < cnt) v[j] = __fmul_rn(v[j], a.row_scale[sg.row0 + j0 + j]);
   }
   if (a.mode == EPI_DENSE) {
     if (row < a.n) {
 #pragma unroll
-      for (int j = 0; j < kSegRows; ++j)
-        if (j < sg.count)
-          a.out_a[static_cast<int64_t>(sg.row0 + j) * a.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+      for (int j = 0; j < 16; ++j)
+        if (j < cnt)
+          a.out_a[static_cast<int64_t>(sg.row0 + j0 + j) * a.n + row] =
+              __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
     }
   } else if (a.mode == EPI_UP) {
     // h = bf16(relu(u)^2), then rotate the 32-slice held by this warp with the
@@ -193,13 +246,13 @@ __device__ __forceinline__ void epilogue_store(const StreamKArgs& a, float (&v)[
       const bool neg = (a.next_mask >> lane) & 1u;
       const float r = __uint_as_float(0x3E3504F3u);
 #pragma unroll
-      for (int j = 0; j < kSegRows; ++j) {
-        if (j < sg.count) {
+      for (int j = 0; j < 16; ++j) {
+        if (j < cnt) {
           const float hv = relu2_bf16(v[j]);
           const float t = __fmul_rn(warp_fwht32_epi(neg ? -hv : hv, lane), r);
           const __nv_bfloat16 hi = __float2bfloat16_rn(t);
           const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(t, __bfloat162float(hi)));
-          const int64_t off = static_cast<int64_t>(sg.row0 + j) * a.n + row;
+          const int64_t off = static_cast<int64_t>(sg.row0 + j0 + j) * a.n + row;
           a.out_a[off] = __bfloat16_as_ushort(hi);
           a.out_b[off] = __bfloat16_as_ushort(lo);
         }
@@ -208,9 +261,9 @@ __device__ __forceinline__ void epilogue_store(const StreamKArgs& a, float (&v)[
   } else {
     if (row < a.n) {
 #pragma unroll
-      for (int j = 0; j < kSegRows; ++j) {
-        if (j < sg.count) {
-          const int p = a.pairs[sg.row0 + j];
+      for (int j = 0; j < 16; ++j) {
+        if (j < cnt) {
+          const int p = a.pairs[sg.row0 + j0 + j];
           a.out_f[static_cast<int64_t>(p) * a.n + row] = __fmul_rn(a.topk_w[p], v[j]);
         }
       }
@@ -231,29 +284,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  // Grouped (MoE) mode reads the routing kernel's segment list right away;
+  // the dense mode defers the dependency wait to the roles that need it.
+  if (a.segs) pdl_wait();
   const int nseg = a.segs ? *a.nseg_dev : a.nseg_host;
-  const int64_t KI = a.k_iters;
+  const int KI = a.k_iters;
   const int64_t T = static_cast<int64_t>(nseg) * a.row_tiles * KI;
   const int64_t G = gridDim.x;
   const int64_t it_begin = range_begin(blockIdx.x, T, G);
   const int64_t it_end = range_begin(blockIdx.x + 1, T, G);
   const int cnt = static_cast<int>(it_end - it_begin);
   if (cnt <= 0) return;
+  // accumulator layout (see kAccRegion): width per warpgroup, number of sets
+  const int acc_w = 32 * a.nb_max;
+  const int nsets = (a.nb_max == 1) ? 2 : 1;
+  const int64_t tile_begin = it_begin / KI, tile_last = (it_end - 1) / KI;
+  const int nportions = static_cast<int>(tile_last - tile_begin + 1);
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sh.full[i], 1);
-      mbar_init(&sh.empty[i], 1);
-    }
-    for (int i = 0; i < kAStages; ++i) {
-      mbar_init(&sh.afull[i], 128);
-      mbar_init(&sh.aempty[i], 1);
+      mbar_init(&sh.full[i], a.x_raw ? 3 : 1);   // producer (+ the two rotation warps)
+      mbar_init(&sh.done[i], 1);
     }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.dfull[i], 1);
+      mbar_init(&sh.dfull[i], kDequantGroups);
       mbar_init(&sh.dempty[i], 128);
     }
-    mbar_init(&sh.mma_done, 1);
+    for (int i = 0; i < kDequantGroups; ++i) mbar_init(&sh.wg_done[i], 1);
     sh.abort_flag = 0;
     sh.last_flag = 0;
     fence_mbar_init();
@@ -263,7 +320,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tma_prefetch_desc(&tm_xhi);
     tma_prefetch_desc(&tm_xlo);
   }
-  if (warp == 2) {
+  if (warp == 1) {
     tmem_alloc(&sh.tmem_base, kTmemCols);
     tmem_relinquish();
   }
@@ -272,29 +329,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
   volatile int* abortp = &sh.abort_flag;
+  if (threadIdx.x == 0) pdl_launch_dependents();
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
+      if (!a.x_raw) pdl_wait();   // x' tiles are the previous kernel's output
       int armed[kStages];
 #pragma unroll
       for (int i = 0; i < kStages; ++i) armed[i] = -1;
-      for (int li = 0; li < cnt; ++li) {
+      Cursor cur;
+      cur.init(it_begin, KI, a.row_tiles);
+      Seg sg = get_seg(a, cur.sgi);
+      int seg_of = cur.sgi;
+      for (int li = 0; li < cnt; ++li, cur.advance(1, KI, a.row_tiles)) {
         const int s = li % kStages;
         const uint32_t ph = (li / kStages) & 1;
-        if (!mbar_wait(&sh.empty[s], ph ^ 1u, abortp)) break;
-        const int64_t it = it_begin + li;
-        const int64_t tile = it / KI;
-        const int kit = static_cast<int>(it - tile * KI);
-        const int sgi = static_cast<int>(tile / a.row_tiles);
-        const int rt = static_cast<int>(tile - static_cast<int64_t>(sgi) * a.row_tiles);
-        const Seg sg = get_seg(a, sgi);
+        if (!mbar_wait(&sh.done[s], ph ^ 1u, abortp)) break;
+        if (cur.sgi != seg_of) {
+          seg_of = cur.sgi;
+          sg = get_seg(a, seg_of);
+        }
+        const int kit = cur.kit, rt = cur.rt;
         const int nb = (sg.count + 15) >> 4;
         uint8_t* st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&sh.full[s], kCodesBytes + nb * 4 * 2048);
+        mbar_arrive_expect_tx(&sh.full[s], kCodesBytes + (a.x_raw ? 0 : nb * 4 * 2048));
         armed[s] = static_cast<int>(ph);
         tma_load_3d(st, &tm_codes, &sh.full[s], kit * 64, rt * 128, sg.e);
-        for (int b = 0; b < nb; ++b) {
+        for (int b = 0; b < nb && !a.x_raw; ++b) {
 #pragma unroll
           for (int kh = 0; kh < 2; ++kh) {
             uint8_t* xb = st + kCodesBytes + kh * kXHalfBytes;
@@ -310,159 +372,254 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (armed[i] >= 0) drain_wait(&sh.full[i], static_cast<uint32_t>(armed[i]));
       }
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      int pi = -1;
-      for (int li = 0; li < cnt; ++li) {
-        const int64_t it = it_begin + li;
-        const int64_t tile = it / KI;
-        const int kit = static_cast<int>(it - tile * KI);
-        const bool first = (li == 0) || (kit == 0);
-        const bool last = (li == cnt - 1) || (kit == KI - 1);
-        if (first) {
-          ++pi;
-          if (!mbar_wait(&sh.dempty[pi & 1], ((pi >> 1) & 1) ^ 1u, abortp)) break;
-        }
+  } else if (warp == 2 || warp == 3) {
+    // ------------------------------------------------------------ rotation
+    // Dense bf16 mode: x' = r H diag(s) x per 32-slice, split into bf16 hi and
+    // lo, written straight into the stage's B tile.  Unit u = (token j, slice
+    // sl) of the iteration's 128 k; the 64 threads take units u and u + 64.
+    if (a.x_raw) {
+      pdl_wait();   // x may be the previous kernel's output
+      const int tid = (warp - 2) * 32 + lane;
+      const float r = __uint_as_float(0x3E3504F3u);
+      Cursor cur;
+      cur.init(it_begin, KI, a.row_tiles);
+      for (int li = 0; li < cnt; ++li, cur.advance(1, KI, a.row_tiles)) {
         const int s = li % kStages;
-        if (!mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) break;
-        const int as = li % kAStages;
-        if (!mbar_wait(&sh.afull[as], (li / kAStages) & 1, abortp)) break;
-        tc_fence_after();
-        const int sgi = static_cast<int>(tile / a.row_tiles);
-        const Seg sg = get_seg(a, sgi);
+        if (!warp_wait(&sh.done[s], ((li / kStages) & 1) ^ 1u, abortp)) break;
+        const Seg sg = get_seg(a, cur.sgi);
         const int nb = (sg.count + 15) >> 4;
-        const uint32_t idesc = kF16 ? idesc_f16(128, 32 * nb) : idesc_bf16(128, 32 * nb);
-        const uint32_t d_addr = tmem + (pi & 1) * kDCols;
-        const uint32_t a_addr = tmem + kACol0 + as * kAColsPerStage;
-        const uint32_t xb = smem_u32(smem + s * kStageBytes + kCodesBytes);
+        uint8_t* xb = smem + s * kStageBytes + kCodesBytes;
+        for (int u = tid; u < 64 * nb; u += 64) {
+          const int j = u >> 2, sl = u & 3;
+          const int k0 = cur.kit * 128 + 32 * sl;
+          float v[32];
+          if (j < sg.count && k0 < a.k) {
+            const uint4* src =
+                reinterpret_cast<const uint4*>(a.x_raw + static_cast<int64_t>(sg.row0 + j) * a.k + k0);
 #pragma unroll
-        for (int k16 = 0; k16 < 8; ++k16) {
-          const uint64_t bdesc = sdesc_k128(xb + (k16 >> 2) * kXHalfBytes + (k16 & 3) * 32);
-          mma_ts(d_addr, a_addr + 8 * k16, bdesc, idesc, (k16 > 0 || !first) ? 1u : 0u);
+            for (int q = 0; q < 4; ++q) {
+              const uint4 w = __ldg(src + q);
+              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                v[8 * q + 2 * e] = __uint_as_float(ww[e] << 16);
+                v[8 * q + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+              }
+            }
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              if ((a.x_mask >> i) & 1u) v[i] = -v[i];
+            fwht32_regs_sk(v);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+          }
+          // hi row j, lo row 16nb + j; slice sl covers bytes [(sl&1)*64, +64)
+          // of the 128-byte row in k-half (sl >> 1); 16-byte chunk c of row
+          // `row` sits at chunk c ^ (row & 7) (128-byte swizzle)
+          uint8_t* half = xb + (sl >> 1) * kXHalfBytes;
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t hw[4], lw[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              const float f0 = __fmul_rn(v[8 * q + 2 * e], r), f1 = __fmul_rn(v[8 * q + 2 * e + 1], r);
+              const __nv_bfloat16 h0 = __float2bfloat16_rn(f0), h1 = __float2bfloat16_rn(f1);
+              const __nv_bfloat16 l0 = __float2bfloat16_rn(__fsub_rn(f0, __bfloat162float(h0)));
+              const __nv_bfloat16 l1 = __float2bfloat16_rn(__fsub_rn(f1, __bfloat162float(h1)));
+              hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
+                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
+              lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
+                      (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
+            }
+            const int c = (sl & 1) * 4 + q;
+            const int rh = j, rl = 16 * nb + j;
+            *reinterpret_cast<uint4*>(half + rh * 128 + ((c ^ (rh & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+            *reinterpret_cast<uint4*>(half + rl * 128 + ((c ^ (rl & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+          }
         }
-        mma_commit(&sh.empty[s]);
-        mma_commit(&sh.aempty[as]);
-        if (last) mma_commit(&sh.dfull[pi & 1]);
+        fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.full[s]);
       }
-      mma_commit(&sh.mma_done);
-      drain_wait(&sh.mma_done, 0);
     }
-  } else if (warp >= 4 && warp < 12) {
-    // ------------------------------------------------------------ dequant
-    const int wg = (warp - 4) >> 2;
+  } else if (warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp) {
+    // ------------------------------------------------------------ dequant + MMA
+    // Warpgroup wg takes the iterations li = wg (mod 4).  Per iteration: the
+    // 8 fp16 scales (fetched one iteration ahead), 16 B of codes per row from
+    // the stage, 128 levels per row written to the group's A stage with
+    // tcgen05.st; then one elected thread issues the 8 MMAs (K = 16 each)
+    // into the group's accumulator and commits to the stage's `done`.
+    const int wg = (warp - kFirstDequantWarp) >> 2;
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int t = q * 32 + lane;            // row within the tile
+    const bool issuer = (t == 0);
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
+    const uint32_t a_stage = tmem + kACol0 + wg * kAColsPerStage;
     uint64_t cm2[4];
 #pragma unroll
     for (int i = 0; i < 4; ++i) cm2[i] = pack_f32x2(cmag.v[2 * i], cmag.v[2 * i + 1]);
     const int kh16 = a.k / 16;
-    for (int li = wg; li < cnt; li += 2) {
-      const int64_t it = it_begin + li;
-      const int64_t tile = it / KI;
-      const int kit = static_cast<int>(it - tile * KI);
-      const int sgi = static_cast<int>(tile / a.row_tiles);
-      const int rt = static_cast<int>(tile - static_cast<int64_t>(sgi) * a.row_tiles);
-      const Seg sg = get_seg(a, sgi);
+    auto fetch_scales = [&](const Cursor& c, uint32_t (&raw)[4]) {
+      const int kit = c.kit, rt = c.rt;
+      const int e = get_seg(a, c.sgi).e;
       const int row = rt * 128 + t;
-      float dsc[8];
-      {
-        const bool rv = row < a.n;
-        const uint16_t* sp = a.scales + (static_cast<int64_t>(sg.e) * a.n + (rv ? row : 0)) * kh16 + kit * 8;
+      const bool rv = row < a.n;
+      const uint32_t* sp = reinterpret_cast<const uint32_t*>(
+          a.scales + (static_cast<int64_t>(e) * a.n + (rv ? row : 0)) * kh16 + kit * 8);
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const bool ok = rv && (kit * 8 + j < kh16);
-          dsc[j] = ok ? __half2float(__ushort_as_half(__ldg(sp + j))) : 0.0f;
+      for (int j = 0; j < 4; ++j) raw[j] = (rv && kit * 8 + 2 * j < kh16) ? __ldg(sp + j) : 0u;
+    };
+    uint32_t next_raw[4] = {0u, 0u, 0u, 0u};
+    Cursor ahead;   // the iteration whose scales are in flight
+    ahead.init(it_begin + wg, KI, a.row_tiles);
+    if (wg < cnt) fetch_scales(ahead, next_raw);
+    // Every exit from these loops is decided by a reducing group barrier, so
+    // the four warps of the group always leave together (a timeout anywhere
+    // sets the CTA abort flag, which the next reduction picks up).
+    int li = wg;    // this group's next iteration
+    bool stop = false;
+    for (int pi = 0; pi < nportions && !stop; ++pi) {
+      const int64_t tile = tile_begin + pi;
+      const int pe = static_cast<int>(((tile + 1) * KI < it_end ? (tile + 1) * KI : it_end) - it_begin);
+      const int db = pi % nsets;
+      const uint32_t dpar = static_cast<uint32_t>((pi / nsets) & 1);
+      const uint32_t acc = tmem + db * (kAccRegion / nsets) + wg * acc_w;
+      if (li >= pe) {
+        // no iteration of this portion falls to this group: once the
+        // accumulator set is free (so the arrival lands in the right phase),
+        // count this group as done with the portion
+        if (issuer && mbar_wait(&sh.dempty[db], dpar ^ 1u, abortp)) mbar_arrive(&sh.dfull[db]);
+        continue;
+      }
+      bool first = true;
+      for (; li < pe; li += kDequantGroups) {
+        float dsc[8];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const __half2 h2 = *reinterpret_cast<const __half2*>(&next_raw[j]);
+          const float2 f2 = __half22float2(h2);
+          dsc[2 * j] = f2.x;
+          dsc[2 * j + 1] = f2.y;
         }
-      }
-      const int s = li % kStages;
-      if (!warp_wait(&sh.full[s], (li / kStages) & 1, abortp)) break;
-      const int as = li % kAStages;
-      if (!warp_wait(&sh.aempty[as], ((li / kAStages) & 1) ^ 1u, abortp)) break;
-      tc_fence_after();
-      const uint8_t* cb = smem + s * kStageBytes + t * 64;
-      const uint32_t tbase = tmem + lane_base + kACol0 + as * kAColsPerStage;
+        const int nbcur = (get_seg(a, ahead.sgi).count + 15) >> 4;   // `ahead` is this iteration
+        if (li + kDequantGroups < cnt) {
+          ahead.advance(kDequantGroups, KI, a.row_tiles);
+          fetch_scales(ahead, next_raw);
+        }
+        const int s = li % kStages;
+        bool okw = warp_wait(&sh.full[s], (li / kStages) & 1, abortp);
+        // the group's A stage was last read by its MMAs of iteration li - 4
+        if (okw && li >= kDequantGroups) {
+          const int prev = li - kDequantGroups;
+          okw = warp_wait(&sh.done[prev % kStages], (prev / kStages) & 1, abortp);
+        }
+        // the issuer's warp also waits for the accumulator set to be free
+        if (okw && first && q == 0) okw = warp_wait(&sh.dempty[db], dpar ^ 1u, abortp);
+        if (okw) {
+          tc_fence_after();
+          const uint8_t* cb = smem + s * kStageBytes + t * 64;
 #pragma unroll
-      for (int kb = 0; kb < 4; ++kb) {
-        const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((t >> 1) & 3)));
-        uint32_t o[16];
-        dequant_half<kF16>(c.x, c.y, dsc[2 * kb], cm2, o);
-        dequant_half<kF16>(c.z, c.w, dsc[2 * kb + 1], cm2, o + 8);
-        tmem_st16(tbase + 16 * kb, o);
+          for (int kb = 0; kb < 4; ++kb) {
+            const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((t >> 1) & 3)));
+            uint32_t o[16];
+            dequant_half<kF16>(c.x, c.y, dsc[2 * kb], cm2, o);
+            dequant_half<kF16>(c.z, c.w, dsc[2 * kb + 1], cm2, o + 8);
+            tmem_st16(a_stage + lane_base + 16 * kb, o);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        if (bar_any(2 + wg, 128, !okw || *abortp)) {
+          stop = true;
+          break;
+        }
+        if (issuer) {
+          tc_fence_after();
+          const uint32_t idesc = kF16 ? idesc_f16(128, 32 * nbcur) : idesc_bf16(128, 32 * nbcur);
+          const uint32_t xb = smem_u32(smem + s * kStageBytes + kCodesBytes);
+#pragma unroll
+          for (int k16 = 0; k16 < 8; ++k16) {
+            const uint64_t bdesc = sdesc_k128(xb + (k16 >> 2) * kXHalfBytes + (k16 & 3) * 32);
+            mma_ts(acc, a_stage + 8 * k16, bdesc, idesc, (first && k16 == 0) ? 0u : 1u);
+          }
+          mma_commit(&sh.done[s]);
+        }
+        first = false;
       }
-      tmem_wait_st();
-      tc_fence_before();
-      mbar_arrive(&sh.afull[as]);
+      if (!stop && issuer) mma_commit(&sh.dfull[db]);
     }
-  } else if (warp >= 12) {
+    if (issuer) {
+      mma_commit(&sh.wg_done[wg]);
+      drain_wait(&sh.wg_done[wg], 0);
+    }
+  } else if (warp >= kFirstEpilogueWarp) {
     // ------------------------------------------------------------ epilogue
+    pdl_wait();   // y, the partials and the counters may still be in use upstream
     const int q = warp & 3;
     const int t = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    int pi = -1;
-    for (int li = 0; li < cnt; ++li) {
-      const int64_t it = it_begin + li;
-      const int64_t tile = it / KI;
-      const int kit = static_cast<int>(it - tile * KI);
-      if (!((li == cnt - 1) || (kit == KI - 1))) continue;
-      ++pi;
-      const int db = pi & 1;
-      // one thread waits; the decision is published before the group barrier
-      // so all four epilogue warps leave together on a timeout
-      if (t == 0) sh.epi_ok[db] = mbar_wait(&sh.dfull[db], (pi >> 1) & 1, abortp) ? 1 : 0;
-      named_bar_sync(1, 128);
-      if (!sh.epi_ok[db]) break;
-      tc_fence_after();
-      const int sgi = static_cast<int>(tile / a.row_tiles);
-      const int rt = static_cast<int>(tile - static_cast<int64_t>(sgi) * a.row_tiles);
-      const Seg sg = get_seg(a, sgi);
-      const int nb = (sg.count + 15) >> 4;
-      float v[kSegRows];
-      {
-        uint32_t r0[16], r1[16];
-        const uint32_t dbase = tmem + lane_base + db * kDCols;
-        if (nb == 1) {
-          tmem_ld16(dbase, r0);
-          tmem_ld16(dbase + 16, r1);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            v[j] = __fadd_rn(__uint_as_float(r0[j]), __uint_as_float(r1[j]));
-            v[16 + j] = 0.0f;
-          }
-        } else {
-          uint32_t r2[16], r3[16];
-          tmem_ld16(dbase, r0);
-          tmem_ld16(dbase + 16, r1);
-          tmem_ld16(dbase + 32, r2);
-          tmem_ld16(dbase + 48, r3);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            v[j] = __fadd_rn(__uint_as_float(r0[j]), __uint_as_float(r2[j]));
-            v[16 + j] = __fadd_rn(__uint_as_float(r1[j]), __uint_as_float(r3[j]));
-          }
-        }
+    int sgi = static_cast<int>(tile_begin / a.row_tiles);
+    int rt = static_cast<int>(tile_begin - static_cast<int64_t>(sgi) * a.row_tiles);
+    for (int pi = 0; pi < nportions; ++pi) {
+      const int64_t tile = tile_begin + pi;
+      if (pi > 0 && ++rt == a.row_tiles) {
+        rt = 0;
+        ++sgi;
       }
-      tc_fence_before();
-      mbar_arrive(&sh.dempty[db]);
-
       const int64_t tile_first = tile * KI;
       const int64_t portion_first = it_begin > tile_first ? it_begin : tile_first;
-      const bool whole = (portion_first == tile_first) && (kit == KI - 1);
+      const int64_t portion_end = (tile + 1) * KI < it_end ? (tile + 1) * KI : it_end;
+      const int db = pi % nsets;
+      // one thread waits; the decision is published before the group barrier
+      // so all four epilogue warps leave together on a timeout
+      if (t == 0) sh.epi_ok[pi & 1] = mbar_wait(&sh.dfull[db], (pi / nsets) & 1, abortp) ? 1 : 0;
+      named_bar_sync(1, 128);
+      if (!sh.epi_ok[pi & 1]) break;
+      tc_fence_after();
+      const Seg sg = get_seg(a, sgi);
+      const int nb = (sg.count + 15) >> 4;
       const int row = rt * 128 + t;
-      if (whole) {
-        epilogue_store(a, v, row, lane, sg);
-        continue;
-      }
-      // split tile: publish the partial, the last contributor finishes it
+      // warpgroup w wrote an accumulator iff one of the portion's local
+      // iterations is congruent to w mod 4
+      const int lpf = static_cast<int>(portion_first - it_begin), plen = static_cast<int>(portion_end - portion_first);
+      const uint32_t dbase = tmem + lane_base + db * (kAccRegion / nsets);
+      const bool whole = (portion_first == tile_first) && (portion_end == tile_first + KI);
       const int slot = (pi == 0) ? 0 : 1;
-      float4* pp = reinterpret_cast<float4*>(a.partials +
-                                             ((static_cast<int64_t>(blockIdx.x) * 2 + slot) * 128 + t) * kSegRows);
+      float* pbase = a.partials + ((static_cast<int64_t>(blockIdx.x) * 2 + slot) * 128 + t) * kSegRows;
+      for (int c = 0; c < nb; ++c) {
+        // hi columns [16c, 16c+16), lo columns [16nb + 16c, +16) of each accumulator
+        float v[16];
 #pragma unroll
-      for (int j = 0; j < kSegRows / 4; ++j) pp[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
-      __threadfence();
+        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+        for (int w = 0; w < kDequantGroups; ++w) {
+          const int off = ((w - lpf) % kDequantGroups + kDequantGroups) % kDequantGroups;
+          if (off >= plen) continue;
+          uint32_t rh[16], rl[16];
+          tmem_ld16(dbase + w * acc_w + 16 * c, rh);
+          tmem_ld16(dbase + w * acc_w + 16 * nb + 16 * c, rl);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            v[j] = __fadd_rn(v[j], __fadd_rn(__uint_as_float(rh[j]), __uint_as_float(rl[j])));
+        }
+        if (c == nb - 1) {
+          tc_fence_before();
+          mbar_arrive(&sh.dempty[db]);
+        }
+        if (whole) {
+          epilogue_store(a, v, 16 * c, row, lane, sg);
+        } else {
+          float4* pp = reinterpret_cast<float4*>(pbase + 16 * c);
+#pragma unroll
+          for (int j = 0; j < 4; ++j) pp[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
+        }
+      }
+      if (whole) continue;
+      // split tile: publish the partial, the last contributor finishes it.
+      // The group barrier orders the 128 threads' partial stores before thread
+      // 0's release (acq_rel, gpu scope) on the tile counter; the last
+      // arriver's acquire orders its reads of the others' partials after it.
       named_bar_sync(1, 128);
       const int64_t c_first = owner_of(tile_first, T, G);
       const int64_t c_last = owner_of(tile_first + KI - 1, T, G);
@@ -470,31 +627,33 @@ __global__ void __launch_bounds__(kThreads, 1)
         int ncontrib = 0;
         for (int64_t c = c_first; c <= c_last; ++c)
           if (range_begin(c + 1, T, G) > range_begin(c, T, G)) ++ncontrib;
-        const int old = atomicAdd(&a.counters[tile], 1);
+        int old;
+        asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(&a.counters[tile]) : "memory");
         sh.last_flag = (old == ncontrib - 1) ? 1 : 0;
       }
       named_bar_sync(1, 128);
       if (sh.last_flag) {
-        __threadfence();
-        float acc[kSegRows];
+        for (int ch = 0; ch < nb; ++ch) {
+          float acc[16];
 #pragma unroll
-        for (int j = 0; j < kSegRows; ++j) acc[j] = 0.0f;
-        for (int64_t c = c_first; c <= c_last; ++c) {
-          const int64_t cb0 = range_begin(c, T, G);
-          if (range_begin(c + 1, T, G) <= cb0) continue;
-          const int cslot = (cb0 / KI == tile) ? 0 : 1;
-          const float4* src = reinterpret_cast<const float4*>(
-              a.partials + ((c * 2 + cslot) * 128 + t) * kSegRows);
+          for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
+          for (int64_t c = c_first; c <= c_last; ++c) {
+            const int64_t cb0 = range_begin(c, T, G);
+            if (range_begin(c + 1, T, G) <= cb0) continue;
+            const int cslot = (cb0 / KI == tile) ? 0 : 1;
+            const float4* src =
+                reinterpret_cast<const float4*>(a.partials + ((c * 2 + cslot) * 128 + t) * kSegRows + 16 * ch);
 #pragma unroll
-          for (int j = 0; j < kSegRows / 4; ++j) {
-            const float4 f = __ldcg(src + j);
-            acc[4 * j] = __fadd_rn(acc[4 * j], f.x);
-            acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], f.y);
-            acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], f.z);
-            acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], f.w);
+            for (int j = 0; j < 4; ++j) {
+              const float4 f = __ldcg(src + j);
+              acc[4 * j] = __fadd_rn(acc[4 * j], f.x);
+              acc[4 * j + 1] = __fadd_rn(acc[4 * j + 1], f.y);
+              acc[4 * j + 2] = __fadd_rn(acc[4 * j + 2], f.z);
+              acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], f.w);
+            }
           }
+          epilogue_store(a, acc, 16 * ch, row, lane, sg);
         }
-        epilogue_store(a, acc, row, lane, sg);
         if (t == 0) a.counters[tile] = 0;
       }
       named_bar_sync(1, 128);
@@ -504,7 +663,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 2) tmem_dealloc(tmem, kTmemCols);
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
@@ -530,10 +689,19 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void*
   const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
   const CUtensorMap& m1 = *static_cast<const CUtensorMap*>(tm_xhi);
   const CUtensorMap& m2 = *static_cast<const CUtensorMap*>(tm_xlo);
-  if (a.f16)
-    streamk_kernel<true><<<grid, kThreads, smem, st>>>(m0, m1, m2, a, cm);
-  else
-    streamk_kernel<false><<<grid, kThreads, smem, st>>>(m0, m1, m2, a, cm);
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = a.f16 ? cudaLaunchKernelEx(&cfg, streamk_kernel<true>, m0, m1, m2, a, cm)
+                        : cudaLaunchKernelEx(&cfg, streamk_kernel<false>, m0, m1, m2, a, cm);
+  if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();
 }

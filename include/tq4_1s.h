@@ -122,19 +122,28 @@ int tq4_1s_quantize(const void* W, int dtype, const tq4_1s_weight* out, tq4_stre
 int tq4_1s_dequantize(const tq4_1s_weight* w, float* W_out, tq4_stream_t stream);
 
 /* Bytes of workspace tq4_1s_linear needs for m rows with weight w (dense,
- * num_experts == 1).  0 on invalid arguments. */
+ * num_experts == 1).  0 on invalid arguments.
+ * Small m (<= 128): the workspace holds stream-K partial sums and tile
+ * counters; the counters must be zero when a call starts, and every call
+ * leaves them zero again.  So zero-fill the workspace once, then use it only
+ * for small-m tq4_1s_linear calls (any shapes, one call at a time); zero it
+ * again after anything else wrote to it or after a call reported
+ * TQ_DEV_TIMEOUT.  Large m: the workspace receives the bf16 dequantized
+ * weight; no initialisation is needed. */
 size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
 
 /* The quantized linear layer of "Running it": y[m][n] = bf16(x * W_hat^T),
  * fp32 accumulation on the tensor cores, no bias.
  *   x  device bf16 bits [m][k], row-major, 16-byte aligned;
- *   y  device bf16 bits [m][n], row-major, 16-byte aligned (n*2 % 16 == 0);
+ *   y  device bf16 bits [m][n], row-major, 16-byte aligned;
  *   ws device workspace of at least tq4_1s_linear_workspace(m, w) bytes,
- *      16-byte aligned, owned by the caller, contents need no initialisation.
- * Small m rotates each 32-slice of x (x' = R x, split into bf16 hi + lo) and
- * multiplies the rotated-domain levels c[code]*d on the tensor cores with a
- * stream-K split of the weight stream; large m dequantizes W_hat to bf16 in
- * the workspace and runs a tensor-core GEMM.  m == 0 is a no-op. */
+ *      16-byte aligned, owned by the caller; for m <= 128 it must satisfy the
+ *      zero-counter rule of tq4_1s_linear_workspace.
+ * Small m (<= 128) is one kernel launch: it rotates each 32-slice of x
+ * (x' = R x, split into bf16 hi + lo) and multiplies the rotated-domain levels
+ * c[code]*d on the tensor cores with a stream-K split of the weight stream;
+ * large m dequantizes W_hat to bf16 in the workspace and runs a tensor-core
+ * GEMM.  m == 0 is a no-op. */
 int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, void* ws, size_t ws_bytes,
                   tq4_stream_t stream);
 

@@ -116,6 +116,28 @@ def test_linear_parity(m, n, k, seed):
     assert tq.tq4_1s_get_status() == 0
 
 
+def test_linear_shared_workspace_across_shapes_and_paths():
+    # one zero-filled workspace reused by small-m calls of different shapes
+    # (different tile counts) stays valid: each call leaves its counters zero;
+    # a large-m call in between uses the binding's separate large-m workspace
+    cases = [(16, 256, 256, 50), (16, 4096, 1024, 51), (300, 520, 224, 52), (8, 1000, 544, 53), (16, 256, 256, 50)]
+    ws = None
+    for m, n, k, seed in cases:
+        W = synth.student_t_f32((n, k), seed, 5.0, 0.02)
+        x = synth.activations_bf16(m, k, seed + 1)
+        p, codes, scales, _ = _quantize_both(W, seed)
+        if m <= 128:
+            need = tq.tq4_1s_linear_workspace(m, p)
+            if ws is None or ws.numel() < need:
+                ws = torch.zeros(4 << 20 if need < (4 << 20) else need, dtype=torch.uint8, device=DEV)
+            y = tq.tq4_1s_linear(_bf16_dev(x), p, workspace=ws)
+        else:
+            y = tq.tq4_1s_linear(_bf16_dev(x), p)
+        torch.cuda.synchronize()
+        y_ref, _ = oracle.linear(x, codes[0], scales[0], seed)
+        assert_close(_bits(y), y_ref, f"shared workspace m={m} n={n} k={k}")
+
+
 def test_linear_deterministic_repeats():
     W = synth.student_t_f32((4096, 4096), 2, 5.0, 0.02)
     x = synth.activations_bf16(16, 4096, 3)
