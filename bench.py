@@ -52,6 +52,30 @@ def peaks():
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x: float) -> float:
+    """The maximum of x over all ranks (x itself when not distributed).
+
+    The job's step time is the slowest rank's device time; each rank runs an
+    independent replica, so no data moves between ranks except this scalar."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    if dist.get_backend() == "nccl":
+        dev = torch.device("cuda", torch.cuda.current_device())
+    else:
+        dev = torch.device("cpu")
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_gbs(world: int, bytes_per_rank_step: float, ms_per_step: float) -> float:
+    """Whole-job throughput in GB/s: every rank's bytes over the slowest rank's step."""
+    return world * bytes_per_rank_step / (ms_per_step * 1e-3) / 1e9
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -207,12 +231,7 @@ def ours_arm(args):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1))
 
     clocks = ClockSampler(local)
     clocks.start()
@@ -220,7 +239,7 @@ def ours_arm(args):
     ms = timed(lambda i: graphs[i % ngraphs].replay(), args.steps)
     clk = clocks.stop()
     ms_step = ms / args.steps
-    value = world * CALLS * PACKED_PER_CALL / (ms_step * 1e-3) / 1e9
+    value = job_gbs(world, CALLS * PACKED_PER_CALL, ms_step)
     per_call_ms = ms_step / CALLS
     achieved = PACKED_PER_CALL / (per_call_ms * 1e-3) / 1e9
     assert tq.tq4_1s_get_status() == 0, "device status word set during the timed region"
@@ -242,7 +261,7 @@ def ours_arm(args):
     for i in range(2):
         e2e_step(i)
     e2e_ms = timed(e2e_step, max(3, args.steps // 2)) / max(3, args.steps // 2)
-    e2e = {"value": world * CALLS * PACKED_PER_CALL / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+    e2e = {"value": job_gbs(world, CALLS * PACKED_PER_CALL, e2e_ms), "unit": "GB/s",
            "h2d_bytes_per_step": x_host.numel() * 2, "d2h_bytes_per_step": y_host.numel() * 2,
            "ms_per_step": e2e_ms}
 

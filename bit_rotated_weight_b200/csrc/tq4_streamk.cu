@@ -33,10 +33,14 @@
 namespace tq4 {
 namespace {
 
-constexpr int kThreads = 768;
+constexpr int kThreads = 800;
 constexpr int kDequantGroups = 4;
 constexpr int kFirstDequantWarp = 4;
 constexpr int kFirstEpilogueWarp = kFirstDequantWarp + 4 * kDequantGroups;
+// Two MMA-issuing threads: lane 0 of warp 1 serves dequant groups 0 and 1,
+// lane 0 of the last warp (24) groups 2 and 3.
+constexpr int kIssuerWarpB = kFirstEpilogueWarp + 4;
+static_assert((kIssuerWarpB + 1) * 32 == kThreads, "warp roles cover the block");
 constexpr int kStages = 8;
 constexpr int kAStages = 4;
 constexpr int kCodesBytes = 128 * 64;    // 128 rows x 128 k codes
@@ -61,9 +65,11 @@ static_assert(kAStages == kDequantGroups, "one A stage per dequant warpgroup");
 struct SharedState {
   uint64_t full[kStages];      // TMA landed (codes, x') and rotated x' written
   uint64_t done[kStages];      // the MMAs of the iteration that used this stage completed
+  uint64_t afull[kDequantGroups][2];   // a half A stage (64 k) holds fresh levels (128 arrivals)
+  uint64_t afree[kDequantGroups][2];   // the MMAs reading a half A stage completed
   uint64_t dfull[2];           // all four warpgroups finished a portion (4 arrivals)
   uint64_t dempty[2];          // the epilogue drained an accumulator set (128 arrivals)
-  uint64_t wg_done[kDequantGroups];
+  uint64_t issuer_done[2];
   uint32_t tmem_base;
   int abort_flag;
   int last_flag;
@@ -310,7 +316,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh.dfull[i], kDequantGroups);
       mbar_init(&sh.dempty[i], 128);
     }
-    for (int i = 0; i < kDequantGroups; ++i) mbar_init(&sh.wg_done[i], 1);
+    for (int i = 0; i < kDequantGroups; ++i)
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(&sh.afull[i][h], 128);
+        mbar_init(&sh.afree[i][h], 1);
+      }
+    for (int i = 0; i < 2; ++i) mbar_init(&sh.issuer_done[i], 1);
     sh.abort_flag = 0;
     sh.last_flag = 0;
     fence_mbar_init();
@@ -444,16 +455,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   } else if (warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp) {
-    // ------------------------------------------------------------ dequant + MMA
+    // ------------------------------------------------------------ dequant
     // Warpgroup wg takes the iterations li = wg (mod 4).  Per iteration: the
     // 8 fp16 scales (fetched one iteration ahead), 16 B of codes per row from
-    // the stage, 128 levels per row written to the group's A stage with
-    // tcgen05.st; then one elected thread issues the 8 MMAs (K = 16 each)
-    // into the group's accumulator and commits to the stage's `done`.
+    // the stage, and 128 levels per row written with tcgen05.st into the
+    // group's A stage -- as two 64-k halves, each signalled separately, so the
+    // tensor core reads one half while the group fills the other.
     const int wg = (warp - kFirstDequantWarp) >> 2;
     const int q = warp & 3;                 // TMEM lane quarter of this warp
     const int t = q * 32 + lane;            // row within the tile
-    const bool issuer = (t == 0);
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t a_stage = tmem + kACol0 + wg * kAColsPerStage;
     uint64_t cm2[4];
@@ -474,86 +484,122 @@ __global__ void __launch_bounds__(kThreads, 1)
     Cursor ahead;   // the iteration whose scales are in flight
     ahead.init(it_begin + wg, KI, a.row_tiles);
     if (wg < cnt) fetch_scales(ahead, next_raw);
-    // Every exit from these loops is decided by a reducing group barrier, so
-    // the four warps of the group always leave together (a timeout anywhere
-    // sets the CTA abort flag, which the next reduction picks up).
-    int li = wg;    // this group's next iteration
-    bool stop = false;
-    for (int pi = 0; pi < nportions && !stop; ++pi) {
+    int use = 0;    // how many times this group has filled its A stage
+    for (int li = wg; li < cnt; li += kDequantGroups, ++use) {
+      float dsc[8];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const __half2 h2 = *reinterpret_cast<const __half2*>(&next_raw[j]);
+        const float2 f2 = __half22float2(h2);
+        dsc[2 * j] = f2.x;
+        dsc[2 * j + 1] = f2.y;
+      }
+      if (li + kDequantGroups < cnt) {
+        ahead.advance(kDequantGroups, KI, a.row_tiles);
+        fetch_scales(ahead, next_raw);
+      }
+      const int s = li % kStages;
+      if (!warp_wait(&sh.full[s], (li / kStages) & 1, abortp)) break;
+      const uint8_t* cb = smem + s * kStageBytes + t * 64;
+      bool ok = true;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        // this half was last read by the MMAs of the group's previous use
+        if (use > 0 && !warp_wait(&sh.afree[wg][h], (use - 1) & 1, abortp)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kb2 = 0; kb2 < 2; ++kb2) {
+          const int kb = 2 * h + kb2;
+          const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((t >> 1) & 3)));
+          uint32_t o[16];
+          dequant_half<kF16>(c.x, c.y, dsc[2 * kb], cm2, o);
+          dequant_half<kF16>(c.z, c.w, dsc[2 * kb + 1], cm2, o + 8);
+          tmem_st16(a_stage + lane_base + 16 * kb, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&sh.afull[wg][h]);
+      }
+      if (!ok) break;
+    }
+  } else if ((warp == 1 || warp == kIssuerWarpB) && lane == 0) {
+    // ------------------------------------------------------------ MMA issue
+    // Issuer A (warp 1) serves groups 0-1, issuer B groups 2-3: the
+    // iterations li with li % 4 in {gb, gb + 1}, in order.  Per half A stage:
+    // wait until the group filled it, issue 4 MMAs (K = 16) into the group's
+    // accumulator, commit to the half's `afree`; after the second half commit
+    // to the stage's `done`; at the end of a portion commit to `dfull`.
+    const int gb = (warp == 1) ? 0 : 2;
+    const int ib = (warp == 1) ? 0 : 1;
+    int use0 = 0, use1 = 0;   // fills of group gb / gb + 1 consumed so far
+    bool ok = true;
+    for (int pi = 0; pi < nportions && ok; ++pi) {
       const int64_t tile = tile_begin + pi;
+      const int pf = static_cast<int>((tile * KI > it_begin ? tile * KI : it_begin) - it_begin);
       const int pe = static_cast<int>(((tile + 1) * KI < it_end ? (tile + 1) * KI : it_end) - it_begin);
       const int db = pi % nsets;
       const uint32_t dpar = static_cast<uint32_t>((pi / nsets) & 1);
-      const uint32_t acc = tmem + db * (kAccRegion / nsets) + wg * acc_w;
-      if (li >= pe) {
-        // no iteration of this portion falls to this group: once the
-        // accumulator set is free (so the arrival lands in the right phase),
-        // count this group as done with the portion
-        if (issuer && mbar_wait(&sh.dempty[db], dpar ^ 1u, abortp)) mbar_arrive(&sh.dfull[db]);
-        continue;
+      // the accumulator set must be free before any MMA or arrival of this portion
+      if (!mbar_wait(&sh.dempty[db], dpar ^ 1u, abortp)) {
+        ok = false;
+        break;
       }
-      bool first = true;
-      for (; li < pe; li += kDequantGroups) {
-        float dsc[8];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const __half2 h2 = *reinterpret_cast<const __half2*>(&next_raw[j]);
-          const float2 f2 = __half22float2(h2);
-          dsc[2 * j] = f2.x;
-          dsc[2 * j + 1] = f2.y;
-        }
-        const int nbcur = (get_seg(a, ahead.sgi).count + 15) >> 4;   // `ahead` is this iteration
-        if (li + kDequantGroups < cnt) {
-          ahead.advance(kDequantGroups, KI, a.row_tiles);
-          fetch_scales(ahead, next_raw);
-        }
+      const Seg sg = get_seg(a, static_cast<int>(tile / a.row_tiles));
+      const int nb = (sg.count + 15) >> 4;
+      const uint32_t idesc = kF16 ? idesc_f16(128, 32 * nb) : idesc_bf16(128, 32 * nb);
+      bool started0 = false, started1 = false;
+      for (int li = pf; li < pe && ok; ++li) {
+        const int w = li % kDequantGroups;
+        if (w != gb && w != gb + 1) continue;
+        const bool second = (w != gb);
+        const int use = second ? use1 : use0;
+        const bool started = second ? started1 : started0;
         const int s = li % kStages;
-        bool okw = warp_wait(&sh.full[s], (li / kStages) & 1, abortp);
-        // the group's A stage was last read by its MMAs of iteration li - 4
-        if (okw && li >= kDequantGroups) {
-          const int prev = li - kDequantGroups;
-          okw = warp_wait(&sh.done[prev % kStages], (prev / kStages) & 1, abortp);
-        }
-        // the issuer's warp also waits for the accumulator set to be free
-        if (okw && first && q == 0) okw = warp_wait(&sh.dempty[db], dpar ^ 1u, abortp);
-        if (okw) {
-          tc_fence_after();
-          const uint8_t* cb = smem + s * kStageBytes + t * 64;
-#pragma unroll
-          for (int kb = 0; kb < 4; ++kb) {
-            const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((t >> 1) & 3)));
-            uint32_t o[16];
-            dequant_half<kF16>(c.x, c.y, dsc[2 * kb], cm2, o);
-            dequant_half<kF16>(c.z, c.w, dsc[2 * kb + 1], cm2, o + 8);
-            tmem_st16(a_stage + lane_base + 16 * kb, o);
-          }
-          tmem_wait_st();
-        }
-        tc_fence_before();
-        if (bar_any(2 + wg, 128, !okw || *abortp)) {
-          stop = true;
+        const uint32_t acc = tmem + db * (kAccRegion / nsets) + w * acc_w;
+        const uint32_t a_stage = tmem + kACol0 + w * kAColsPerStage;
+        const uint32_t xb = smem_u32(smem + s * kStageBytes + kCodesBytes);
+        // the B tile (x') of this stage must have landed too
+        if (!mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) {
+          ok = false;
           break;
         }
-        if (issuer) {
-          tc_fence_after();
-          const uint32_t idesc = kF16 ? idesc_f16(128, 32 * nbcur) : idesc_bf16(128, 32 * nbcur);
-          const uint32_t xb = smem_u32(smem + s * kStageBytes + kCodesBytes);
-#pragma unroll
-          for (int k16 = 0; k16 < 8; ++k16) {
-            const uint64_t bdesc = sdesc_k128(xb + (k16 >> 2) * kXHalfBytes + (k16 & 3) * 32);
-            mma_ts(acc, a_stage + 8 * k16, bdesc, idesc, (first && k16 == 0) ? 0u : 1u);
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(&sh.afull[w][h], use & 1, abortp)) {
+            ok = false;
+            break;
           }
-          mma_commit(&sh.done[s]);
+          tc_fence_after();
+          // half h of the stage's B tile is k-half h of x'; the descriptor's
+          // start address (16-byte units) advances by 2 per 16-k step
+          const uint64_t bdesc0 = sdesc_k128(xb + h * kXHalfBytes);
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc0 + static_cast<uint64_t>(2 * kk), idesc,
+                   (!started && h == 0 && kk == 0) ? 0u : 1u);
+          mma_commit(&sh.afree[w][h]);
         }
-        first = false;
+        if (!ok) break;
+        mma_commit(&sh.done[s]);
+        if (second) {
+          started1 = true;
+          ++use1;
+        } else {
+          started0 = true;
+          ++use0;
+        }
       }
-      if (!stop && issuer) mma_commit(&sh.dfull[db]);
+      if (!ok) break;
+      if (started0) mma_commit(&sh.dfull[db]);
+      else mbar_arrive(&sh.dfull[db]);
+      if (started1) mma_commit(&sh.dfull[db]);
+      else mbar_arrive(&sh.dfull[db]);
     }
-    if (issuer) {
-      mma_commit(&sh.wg_done[wg]);
-      drain_wait(&sh.wg_done[wg], 0);
-    }
-  } else if (warp >= kFirstEpilogueWarp) {
+    mma_commit(&sh.issuer_done[ib]);
+    drain_wait(&sh.issuer_done[ib], 0);
+  } else if (warp >= kFirstEpilogueWarp && warp < kFirstEpilogueWarp + 4) {
     // ------------------------------------------------------------ epilogue
     pdl_wait();   // y, the partials and the counters may still be in use upstream
     const int q = warp & 3;
@@ -595,13 +641,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int w = 0; w < kDequantGroups; ++w) {
           const int off = ((w - lpf) % kDequantGroups + kDequantGroups) % kDequantGroups;
           if (off >= plen) continue;
-          uint32_t rh[16], rl[16];
-          tmem_ld16(dbase + w * acc_w + 16 * c, rh);
-          tmem_ld16(dbase + w * acc_w + 16 * nb + 16 * c, rl);
-          tmem_wait_ld();
+          for (int part = 0; part < 2; ++part) {   // hi columns, then lo columns
+            uint32_t rr[16];
+            tmem_ld16(dbase + w * acc_w + 16 * nb * part + 16 * c, rr);
+            tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            v[j] = __fadd_rn(v[j], __fadd_rn(__uint_as_float(rh[j]), __uint_as_float(rl[j])));
+            for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __uint_as_float(rr[j]));
+          }
         }
         if (c == nb - 1) {
           tc_fence_before();
