@@ -283,7 +283,7 @@ def ours_arm(args):
                        "l2": "cold: 64 distinct packed weight copies (671 MB > 126 MB L2) cycled, 16 per step"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                         "kernel": "tq4_1s_linear small-m call (rotate_act + streamk), per call",
+                         "kernel": "tq4_1s_linear small-m call (activation rotation + stream-K dequant-GEMM), per call",
                          "peak_source": pk["source"], "per_call_us": per_call_ms * 1e3},
             "eager_per_call_us": ms_eager / CALLS * 1e3,
             "cpu_baseline": cpu,

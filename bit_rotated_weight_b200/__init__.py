@@ -32,7 +32,7 @@ LIB_PATH = os.path.join(_HERE, "libtq4_1s.so")
 
 TQ_OK = 0
 TQ_DTYPE_F32, TQ_DTYPE_BF16 = 0, 1
-TQ_DEV_TIMEOUT, TQ_DEV_BAD_ROUTING, TQ_DEV_NONFINITE = 1, 2, 4
+TQ_DEV_TIMEOUT, TQ_DEV_BAD_ROUTING, TQ_DEV_NONFINITE, TQ_DEV_SCALE_RANGE = 1, 2, 4, 8
 
 
 class TQ4Error(RuntimeError):
@@ -183,11 +183,11 @@ SMALL_M = 128   # tq4_1s_linear takes its stream-K path up to this many rows
 
 
 def _workspace(nbytes: int, device, kind: str) -> torch.Tensor:
-    """A cached, zero-filled workspace per (device, kind).
+    """A cached workspace per (device, kind), grown on demand.
 
-    The small-m linear path needs its tile counters zero at the start of a
-    call and leaves them zero, so its workspace is kept apart from the
-    large-m path (which writes the dequantized weight into its own)."""
+    The library clears whatever it needs at the start of each call; the
+    kinds are kept apart only so that a large small-m buffer and a large
+    dequantized-weight buffer are not reallocated back and forth."""
     key = (str(device), kind)
     buf = _ws_cache.get(key)
     if buf is None or buf.numel() < nbytes:

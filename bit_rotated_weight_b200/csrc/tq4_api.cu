@@ -182,15 +182,15 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int64_t kSmallM = 128;
 
 struct SmallLayout {
-  size_t partials, counters, total;
+  size_t xh, xl, xscale, partials, counters, total;
   int grid;
   int64_t tiles;
 };
 
-// Small-m workspace: the fp32 partials first (their size depends only on the
-// SM count), the tile counters after them.  The counters therefore start at
-// the same offset for every shape, so a workspace shared by small-m calls of
-// different shapes never sees another call's partials in its counters.
+// Small-m workspace: the rotated activations (fp16 hi and lo planes, per-row
+// scales; unused when the kernel rotates x itself), the stream-K fp32
+// partials and the tile counters.  Counters carry the launch's epoch, so the
+// workspace needs no initialisation.
 static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
   SmallLayout L{};
   const int64_t nseg = (m + kSegRows - 1) / kSegRows;
@@ -199,16 +199,28 @@ static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
   const int64_t T = L.tiles * ki;
   L.grid = static_cast<int>(T < sms ? T : sms);
   size_t off = 0;
-  L.partials = off;
-  off = align256(off + static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
-  L.counters = off;
-  off = align256(off + static_cast<size_t>(L.tiles) * 4);
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off = align256(off + bytes);
+    return at;
+  };
+  L.xh = take(static_cast<size_t>(m * w->k) * 2);
+  L.xl = take(static_cast<size_t>(m * w->k) * 2);
+  L.xscale = take(static_cast<size_t>(m) * 4);
+  L.partials = take(static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
+  L.counters = take(static_cast<size_t>(L.tiles) * 8);
   L.total = off;
   return L;
 }
 
+// The dense kernel rotates x itself when it is one segment and no CTA runs
+// more iterations than it has stages.
+static bool small_fused(int64_t m, int64_t tiles_times_ki, int grid) {
+  return m <= kSegRows && (tiles_times_ki + grid - 1) / grid <= kFusedMaxIters;
+}
+
 struct MoeLayout {
-  size_t offsets, pairs, segs, nseg, npv, xh, xl, xscale, hh, hl, zw, partials, cnt_up, cnt_dn, total;
+  size_t offsets, pairs, segs, nseg, npv, xh, xl, xscale, h, hh, hl, hscale, zw, partials, cnt_up, cnt_dn, total;
   int64_t P, maxseg, rt_up, rt_dn;
 };
 
@@ -234,13 +246,14 @@ static MoeLayout moe_layout(int64_t m, int32_t topk, const tq4_1s_weight* up, co
   L.xh = take(L.P * H * 2);
   L.xl = take(L.P * H * 2);
   L.xscale = take(L.P * 4);
+  L.h = take(L.P * I * 2);
   L.hh = take(L.P * I * 2);
   L.hl = take(L.P * I * 2);
+  L.hscale = take(L.P * 4);
   L.zw = take(L.P * H * 4);
   L.partials = take(static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
-  // the two counter arrays are one block: the route kernel zeroes it at once
-  L.cnt_up = take(L.maxseg * (L.rt_up + L.rt_dn) * 4);
-  L.cnt_dn = L.cnt_up + static_cast<size_t>(L.maxseg * L.rt_up) * 4;
+  L.cnt_up = take(L.maxseg * L.rt_up * 8);
+  L.cnt_dn = take(L.maxseg * L.rt_dn * 8);
   L.total = off;
   return L;
 }
@@ -344,12 +357,23 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
 
   if (m <= kSmallM) {
     const SmallLayout L = small_layout(m, w, sms);
-    if (L.tiles * ((w->k + 127) / 128) > INT32_MAX) return TQ_ERR_INVALID_ARG;   // 32-bit iteration space
-    int32_t* counters = reinterpret_cast<int32_t*>(base + L.counters);
-    // One launch: the kernel rotates x itself (no x' round trip through
-    // memory).  The x' maps are unused in this mode; they point at x.
+    const int64_t T = L.tiles * ((w->k + 127) / 128);
+    if (T > INT32_MAX) return TQ_ERR_INVALID_ARG;   // 32-bit iteration space
+    // m <= 32 (one segment): cluster split-K when it fits in one wave, else
+    // stream-K (the kernel rotates x itself when every CTA has a stage per
+    // iteration, else the rotation kernel feeds x' through memory)
+    const int64_t KI = (w->k + 127) / 128;
+    const int split = m <= kSegRows ? choose_cluster_split(L.tiles, KI, sms) : 1;
+    const int grid = split > 1 ? static_cast<int>(L.tiles * split) : L.grid;
+    const bool fused = split > 1 || small_fused(m, T, L.grid);
+    uint16_t* xh = reinterpret_cast<uint16_t*>(base + L.xh);
+    uint16_t* xl = reinterpret_cast<uint16_t*>(base + L.xl);
+    float* xscale = reinterpret_cast<float*>(base + L.xscale);
+    // TMA-fed mode: x' = R x (fp16 hi/lo, per-row scale) by the rotation kernel
+    if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xh, xl, xscale, mask, st) != cudaSuccess)
+      return TQ_ERR_CUDA;
     alignas(64) CUtensorMap tc, th, tl;
-    if (!map_codes(&tc, w) || !map_bf16(&th, x, m, w->k, 16) || !map_bf16(&tl, x, m, w->k, 16))
+    if (!map_codes(&tc, w) || !map_bf16(&th, xh, m, w->k, 16) || !map_bf16(&tl, xl, m, w->k, 16))
       return TQ_ERR_CUDA;
     StreamKArgs a{};
     a.n = static_cast<int32_t>(w->n);
@@ -360,14 +384,19 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     a.m_host = static_cast<int32_t>(m);
     a.nb_max = m > 16 ? 2 : 1;
     a.scales = w->scales;
+    a.row_scale = xscale;
+    if (fused) {
+      a.x_raw = x;
+      a.x_mask = mask;
+    }
+    a.epoch = next_epoch();
+    a.cluster_s = split;
     a.mode = EPI_DENSE;
     a.out_a = y;
-    a.x_raw = x;
-    a.x_mask = mask;
     a.partials = reinterpret_cast<float*>(base + L.partials);
-    a.counters = counters;
+    a.counters = reinterpret_cast<unsigned long long*>(base + L.counters);
     a.max_tiles = static_cast<int32_t>(L.tiles);
-    return cuda_rc(launch_streamk(&tc, &th, &tl, a, L.grid, st));
+    return cuda_rc(launch_streamk(&tc, &th, &tl, a, grid, st));
   }
   // large m: W_hat in bf16, then the tensor-core GEMM
   uint16_t* wh = reinterpret_cast<uint16_t*>(base);
@@ -428,22 +457,21 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   uint16_t* hh = reinterpret_cast<uint16_t*>(base + L.hh);
   uint16_t* hl = reinterpret_cast<uint16_t*>(base + L.hl);
   float* zw = reinterpret_cast<float*>(base + L.zw);
-  int32_t* cnt_up = reinterpret_cast<int32_t*>(base + L.cnt_up);
-  const int64_t ncnt = L.maxseg * (L.rt_up + L.rt_dn);   // cnt_up and cnt_dn are contiguous
   cudaError_t e = launch_moe_route(topk_ids, L.P, static_cast<int32_t>(E), offsets, pairs, segs, nseg, kSegRows,
-                                   npv, cnt_up, ncnt, st);
+                                   npv, nullptr, 0, st);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   float* xscale = reinterpret_cast<float*>(base + L.xscale);
-  e = launch_rotate_rows_f16(x, H, pairs, topk, npv, L.P, xh, xl, xscale, sign_mask_of(up->seed), st);
+  uint16_t* h = reinterpret_cast<uint16_t*>(base + L.h);
+  float* hscale = reinterpret_cast<float*>(base + L.hscale);
+  // x' of each sorted pair row (x row pairs[r] / topk), rotated by the up
+  // projection's signs
+  e = launch_rotate_scaled(x, H, pairs, topk, npv, 0, L.P, xh, xl, xscale, sign_mask_of(up->seed), st);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
 
   alignas(64) CUtensorMap tcu, txh, txl, tcd, thh, thl;
   if (!map_codes(&tcu, up) || !map_bf16(&txh, xh, L.P, H, 16) || !map_bf16(&txl, xl, L.P, H, 16) ||
       !map_codes(&tcd, down) || !map_bf16(&thh, hh, L.P, I, 16) || !map_bf16(&thl, hl, L.P, I, 16))
     return TQ_ERR_CUDA;
-  // Up projection in fp16 operands: its error is doubled by the squared ReLU,
-  // and fp16 levels round 8x finer than bf16.  Rows of x' carry a power-of-two
-  // scale (xscale) that keeps them inside the fp16 range.
   StreamKArgs a{};
   a.n = static_cast<int32_t>(I);
   a.k = static_cast<int32_t>(H);
@@ -453,32 +481,33 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   a.nseg_dev = nseg;
   a.nb_max = m > 16 ? 2 : 1;   // an expert takes each token at most once (top-k ids are distinct)
   a.scales = up->scales;
-  a.f16 = 1;
   a.row_scale = xscale;
+  a.epoch = next_epoch();
+  a.cluster_s = 1;
   a.mode = EPI_UP;
-  a.out_a = hh;
-  a.out_b = hl;
-  a.next_mask = sign_mask_of(down->seed);
+  a.out_a = h;
   a.partials = reinterpret_cast<float*>(base + L.partials);
-  a.counters = cnt_up;
+  a.counters = reinterpret_cast<unsigned long long*>(base + L.cnt_up);
   a.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_up);
   if ((e = launch_streamk(&tcu, &txh, &txl, a, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
 
+  // h' = R_down h per sorted pair row
+  e = launch_rotate_scaled(h, I, nullptr, 1, npv, 0, L.P, hh, hl, hscale, sign_mask_of(down->seed), st);
+  if (e != cudaSuccess) return TQ_ERR_CUDA;
   StreamKArgs b = a;
   b.n = static_cast<int32_t>(H);
   b.k = static_cast<int32_t>(I);
   b.row_tiles = static_cast<int32_t>(L.rt_dn);
   b.k_iters = static_cast<int32_t>((I + 127) / 128);
   b.scales = down->scales;
-  b.f16 = 0;
-  b.row_scale = nullptr;
+  b.row_scale = hscale;
+  b.epoch = next_epoch();
   b.mode = EPI_DOWN;
   b.out_a = nullptr;
-  b.out_b = nullptr;
   b.out_f = zw;
   b.pairs = pairs;
   b.topk_w = topk_w;
-  b.counters = reinterpret_cast<int32_t*>(base + L.cnt_dn);
+  b.counters = reinterpret_cast<unsigned long long*>(base + L.cnt_dn);
   b.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_dn);
   if ((e = launch_streamk(&tcd, &thh, &thl, b, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
   return cuda_rc(launch_moe_combine(zw, topk_ids, m, topk, H, static_cast<int32_t>(E), y, st));

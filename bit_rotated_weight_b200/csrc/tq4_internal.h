@@ -29,13 +29,15 @@ cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, 
                                   uint32_t mask, const CodebookF32& cb, cudaStream_t st);
 cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales, uint16_t* out, int64_t rows,
                                    int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st);
-cudaError_t launch_rotate_act(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
-                              const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
-                              uint16_t* xh, uint16_t* xl, uint32_t mask, int32_t* zero_ptr, int64_t nzero,
-                              cudaStream_t st);
-cudaError_t launch_rotate_rows_f16(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
-                                   const int32_t* rows_valid_dev, int64_t rows_alloc, uint16_t* xh, uint16_t* xl,
-                                   float* row_scale, uint32_t mask, cudaStream_t st);
+// Activation rotation for the stream-K GEMM: x' = r H diag(s) x per 32-slice
+// of each row, scaled by a per-row power of two 2^-e and split into fp16
+// hi/lo planes [rows][k]; row_scale[row] = 2^e.  Row r reads x row
+// gather[r] / topk when a gather list is given, else row r.  Rows at or past
+// the valid count (rows_valid_dev when non-null, else rows_valid_host) are
+// not written.
+cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
+                                 const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
+                                 uint16_t* xh, uint16_t* xl, float* row_scale, uint32_t mask, cudaStream_t st);
 cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
                              int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
                              int32_t* zero_ptr, int64_t nzero, cudaStream_t st);
@@ -55,24 +57,39 @@ struct StreamKArgs {
   const int4* segs;          // device segment list (MoE) or nullptr
   const int32_t* nseg_dev;   // device segment count (MoE) or nullptr
   const uint16_t* scales;    // [E][n][k/16]
+  const float* row_scale;    // x' row r holds x'_r * 2^-e_r; row_scale[r] = 2^e_r (TMA-fed mode)
+  const uint16_t* x_raw;     // fused mode (dense, m <= kSegRows, <= kFusedMaxIters iterations per CTA):
+                             // raw bf16 x [m][k], rotated by the kernel itself; nullptr otherwise
+  uint32_t x_mask;           // fused mode: the weight's sign mask
+  uint32_t epoch;            // tag of this launch in the tile counters (never 0)
+  int32_t cluster_s;         // >= 2: fused split-K mode -- grid = tiles * cluster_s, one cluster per
+                             // tile, partials reduced through distributed shared memory; else 1
   int32_t mode;              // EpilogueMode
-  uint16_t* out_a;           // dense: y [m][n]; up: next-stage hi [P][n]
-  uint16_t* out_b;           // up: next-stage lo [P][n]
+  uint16_t* out_a;           // dense: y [m][n]; up: h = relu(u)^2 [P][n] (bf16)
   float* out_f;              // down: z*w [m*topk][n]
   const int32_t* pairs;      // MoE: flat slot index of each sorted row
   const float* topk_w;       // MoE: router weights (flat)
-  uint32_t next_mask;        // up: sign mask of the down projection
-  int32_t f16;               // operands: 0 = bf16 (x' hi/lo), 1 = fp16 (x' hi/lo scaled by row_scale)
-  const float* row_scale;    // fp16 mode: x' row r was multiplied by 1/row_scale[r]
-  const uint16_t* x_raw;     // dense bf16 mode: raw x [m][k]; warps of the kernel rotate it (x' hi/lo)
-  uint32_t x_mask;           // sign mask of the weight (for the fused rotation)
   float* partials;           // [grid][2][128][kSegRows]
-  int32_t* counters;         // [tiles]
+  unsigned long long* counters;   // [tiles]: (epoch << 32) | arrivals
   int32_t max_tiles;         // capacity of counters
 };
 
+// Iterations per CTA up to which the dense kernel can rotate x in its
+// prologue (one pipeline stage per iteration, no stage reuse).
+constexpr int kFusedMaxIters = 8;
+
+// A fresh counter tag for each stream-K launch.
+uint32_t next_epoch();
+
 // Bytes of dynamic shared memory the stream-K kernel uses.
 size_t streamk_smem_bytes();
+// How many clusters of s stream-K CTAs can be resident at once (0 on error).
+int streamk_max_clusters(int s);
+// Cluster split-K factor for a fused dense launch of `tiles` row tiles and
+// k_iters k iterations: the largest s in [2, 8] with s <= k_iters, at most
+// kFusedMaxIters iterations per CTA, tiles * s <= sms and all clusters
+// resident at once; 1 if none fits.
+int choose_cluster_split(int64_t tiles, int64_t k_iters, int sms);
 
 cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void* tm_xlo, const StreamKArgs& a,
                            int grid, cudaStream_t st);

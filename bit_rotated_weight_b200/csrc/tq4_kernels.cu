@@ -3,9 +3,10 @@
 //
 // Format and arithmetic follow the Nemotron-TheHobbit-30B-A3B model card,
 // section "What Config-I means" (per-32-block RHT rotation, 16-level
-// Lloyd-Max codes, two half-block scales).  One warp handles one 32-element
-// block: lane i owns element i, and the 32-point butterfly runs in registers
-// through shfl_xor, stage h exchanging lanes i and i^h.
+// Lloyd-Max codes, two half-block scales).  The weight kernels give one
+// thread one 32-element block, its 32-point butterfly in registers (stage h
+// pairs elements j and j+h); the activation kernel spreads a slice over a
+// warp and runs the same butterfly through lane shuffles.
 #include "tq4_internal.h"
 
 namespace tq4 {
@@ -14,18 +15,6 @@ __device__ int g_status = 0;
 
 // r = fp32(1/sqrt(32))
 __device__ __forceinline__ float rsqrt32() { return __uint_as_float(0x3E3504F3u); }
-
-// In-register 32-point Sylvester Hadamard butterfly across the warp
-// (stages h = 1, 2, 4, 8, 16): the lane with bit h clear keeps a + partner,
-// the other keeps partner - a.
-__device__ __forceinline__ float warp_fwht32(float a, int lane) {
-#pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
-    const float p = __shfl_xor_sync(0xFFFFFFFFu, a, h);
-    a = (lane & h) ? __fsub_rn(p, a) : __fadd_rn(a, p);
-  }
-  return a;
-}
 
 // fp32 -> fp16 bits, round to nearest even, saturating at 65504, NaN -> 0x7E00.
 __device__ __forceinline__ uint16_t f16_sat_bits(float x) {
@@ -203,103 +192,102 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
 }
 
 // ------------------------------------------------------------------ activations
-// x' = r * H * diag(s) * x per 32-slice, split into bf16 hi = bf16(x') and
-// lo = bf16(x' - hi).  Row r of the outputs takes x row gather[r] / topk when a
-// gather list is given (MoE: rows in expert order), else row r.  Rows in
-// [rows_valid, rows_alloc) are zero-filled.  Also zeroes `nzero` ints at
-// `zero_ptr` (stream-K tile counters of the launches that follow).
-__global__ void __launch_bounds__(256) rotate_act_kernel(const uint16_t* __restrict__ x, int64_t k,
-                                                         const int32_t* __restrict__ gather, int32_t topk,
-                                                         const int32_t* __restrict__ rows_valid_dev,
-                                                         int64_t rows_valid_host, int64_t rows_alloc,
-                                                         uint16_t* __restrict__ xh, uint16_t* __restrict__ xl,
-                                                         uint32_t mask, int32_t* __restrict__ zero_ptr,
-                                                         int64_t nzero) {
-  const int64_t tid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  for (int64_t i = tid; i < nzero; i += static_cast<int64_t>(gridDim.x) * blockDim.x) zero_ptr[i] = 0;
-  const int lane = threadIdx.x & 31;
-  const bool neg = (mask >> lane) & 1u;
-  const int64_t rows_valid = rows_valid_dev ? static_cast<int64_t>(*rows_valid_dev) : rows_valid_host;
-  const int64_t kb_per_row = k / 32;
-  const int64_t nblocks = rows_alloc * kb_per_row;
-  const int64_t warp = tid >> 5;
-  const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
-  const float r = rsqrt32();
-  for (int64_t b = warp; b < nblocks; b += nwarps) {
-    const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
-    const int64_t off = row * k + kb * 32 + lane;
-    if (row >= rows_valid) {
-      xh[off] = 0;
-      xl[off] = 0;
-      continue;
-    }
-    const int64_t src = gather ? static_cast<int64_t>(gather[row] / topk) : row;
-    const float xv = bf16_bits_to_f32(x[src * k + kb * 32 + lane]);
-    const float v = __fmul_rn(warp_fwht32(neg ? -xv : xv, lane), r);
-    const __nv_bfloat16 h = __float2bfloat16_rn(v);
-    const __nv_bfloat16 l = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(h)));
-    xh[off] = __bfloat16_as_ushort(h);
-    xl[off] = __bfloat16_as_ushort(l);
+// The activation side of route B: x' = r H diag(s) x per 32-slice of each row
+// (rotating x by the weight's RHT instead of inverse-rotating the weight;
+// equivalent because R is orthogonal).  Each row is scaled by 2^-e, where e
+// puts the largest value x' can take, sqrt(32) * max|x| (each x'_i is r times
+// a signed sum of 32 entries), in [2^13, 2^14): the row then uses the full
+// fp16 precision and cannot overflow.  Split into fp16 hi = f16(x' 2^-e) and
+// lo = f16(x' 2^-e - hi); row_scale[row] = 2^e (exact) undoes the scaling in
+// the GEMM epilogue.
+//
+// One CTA of four warps per row; lane i of a warp holds element i of a
+// slice, and the 32-point butterfly runs across the warp through shfl_xor
+// (stage h exchanges lanes i and i^h: the lane with bit h clear keeps
+// a + partner, the other partner - a), the same order as the one-thread form.
+// First pass: the row maximum; second pass (L1 hits): rotate, scale, split.
+// The CTA is small (128 threads, at most 48 registers each, no shared
+// arrays) so that it fits on an SM beside a running stream-K CTA.
+constexpr int kRotThreads = 128;
+
+__device__ __forceinline__ float warp_fwht32(float a, int lane) {
+#pragma unroll
+  for (int h = 1; h < 32; h <<= 1) {
+    const float p = __shfl_xor_sync(0xFFFFFFFFu, a, h);
+    a = (lane & h) ? __fsub_rn(p, a) : __fadd_rn(a, p);
   }
+  return a;
 }
 
-// One CTA per row: the fp16 variant of the activation rotation.  x' = R x per
-// 32-slice is scaled by 2^-e, where e puts the largest value x' can take,
-// sqrt(32) * max|x| (each x'_i is r times a signed sum of 32 entries), in
-// [2^13, 2^14): every row then uses the full fp16 precision and cannot
-// overflow.  Split into fp16 hi = f16(x' 2^-e) and lo = f16(x' 2^-e - hi);
-// row_scale[row] = 2^e undoes the scaling in the GEMM epilogue (an exact
-// power of two).  Rows at or past the valid count are zero with scale 1.
-__global__ void __launch_bounds__(256) rotate_rows_f16_kernel(const uint16_t* __restrict__ x, int64_t k,
-                                                              const int32_t* __restrict__ gather, int32_t topk,
-                                                              const int32_t* __restrict__ rows_valid_dev,
-                                                              int64_t rows_alloc, uint16_t* __restrict__ xh,
-                                                              uint16_t* __restrict__ xl,
-                                                              float* __restrict__ row_scale, uint32_t mask) {
-  __shared__ float s_max[8];
+__global__ void __launch_bounds__(kRotThreads, 10)
+    rotate_scaled_kernel(const uint16_t* __restrict__ x, int64_t k, const int32_t* __restrict__ gather,
+                         int32_t topk, const int32_t* __restrict__ rows_valid_dev, int64_t rows_valid_host,
+                         uint16_t* __restrict__ xh, uint16_t* __restrict__ xl, float* __restrict__ row_scale,
+                         uint32_t mask) {
+  __shared__ float s_max[kRotThreads / 32];
+  // x, the gather list and the valid count may be the previous kernel's
+  // output.  Dependents may start once every CTA is past this wait: nothing
+  // before this kernel is still running then, and the stream-K kernel that
+  // follows reads only the weight before its own wait.
+  pdl_wait();
+  if (threadIdx.x == 0) pdl_launch_dependents();
   const int64_t row = blockIdx.x;
-  if (row >= rows_alloc) return;
-  const int64_t rows_valid = rows_valid_dev ? static_cast<int64_t>(*rows_valid_dev) : rows_alloc;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
-  uint16_t* oh = xh + row * k;
-  uint16_t* ol = xl + row * k;
-  if (row >= rows_valid) {
-    for (int64_t i = threadIdx.x; i < k; i += blockDim.x) {
-      oh[i] = 0;
-      ol[i] = 0;
-    }
-    if (threadIdx.x == 0) row_scale[row] = 1.0f;
-    return;
-  }
-  const int64_t src = gather ? static_cast<int64_t>(gather[row] / topk) : row;
-  const uint16_t* xr = x + src * k;
+  const int64_t rows_valid = rows_valid_dev ? static_cast<int64_t>(*rows_valid_dev) : rows_valid_host;
+  if (row >= rows_valid) return;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kWarps = kRotThreads / 32;
+  const int64_t src = gather ? static_cast<int64_t>(__ldcg(gather + row) / topk) : row;
+  const uint16_t* xr = x + src * k + lane;
+  const int64_t nsl = k / 32;
   float mx = 0.0f;
-  for (int64_t i = threadIdx.x; i < k; i += blockDim.x) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(xr[i])));
+  {
+    // 16 loads in flight per lane: a 4096-wide row is one round trip
+    int64_t sl = warp;
+    for (; sl + 15 * kWarps < nsl; sl += 16 * kWarps) {
+      uint16_t v[16];
+#pragma unroll
+      for (int u = 0; u < 16; ++u) v[u] = __ldg(xr + (sl + u * kWarps) * 32);
+#pragma unroll
+      for (int u = 0; u < 16; ++u) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(v[u])));
+    }
+    for (; sl < nsl; sl += kWarps) mx = fmaxf(mx, fabsf(bf16_bits_to_f32(__ldg(xr + sl * 32))));
+  }
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
   if (lane == 0) s_max[warp] = mx;
   __syncthreads();
   mx = s_max[0];
-  for (int w = 1; w < nwarps; ++w) mx = fmaxf(mx, s_max[w]);
+#pragma unroll
+  for (int w = 1; w < kWarps; ++w) mx = fmaxf(mx, s_max[w]);
   int e = 0;
   if (mx > 0.0f && isfinite(mx)) {
     int ex;
-    frexpf(__fmul_rn(mx, 5.65685415f), &ex);   // bound in [2^(ex-1), 2^ex)
+    frexpf(__fmul_rn(mx, 5.65685415f), &ex);   // the bound lies in [2^(ex-1), 2^ex)
     e = ex - 14;
     e = e < -100 ? -100 : (e > 100 ? 100 : e);
   }
-  const float down = ldexpf(1.0f, -e);
   if (threadIdx.x == 0) row_scale[row] = ldexpf(1.0f, e);
+  const float rd = __fmul_rn(rsqrt32(), ldexpf(1.0f, -e));   // exact: r times a power of two
   const bool neg = (mask >> lane) & 1u;
-  const float r = rsqrt32();
-  for (int64_t kb = warp; kb < k / 32; kb += nwarps) {
-    const float xv = bf16_bits_to_f32(xr[kb * 32 + lane]);
-    const float v = __fmul_rn(__fmul_rn(warp_fwht32(neg ? -xv : xv, lane), r), down);
+  uint16_t* oh = xh + row * k + lane;
+  uint16_t* ol = xl + row * k + lane;
+  auto emit = [&](int64_t sl, uint16_t raw) {
+    const float xv = bf16_bits_to_f32(raw);
+    const float v = __fmul_rn(warp_fwht32(neg ? -xv : xv, lane), rd);
     const __half h = __float2half_rn(v);
     const __half l = __float2half_rn(__fsub_rn(v, __half2float(h)));
-    oh[kb * 32 + lane] = __half_as_ushort(h);
-    ol[kb * 32 + lane] = __half_as_ushort(l);
+    oh[sl * 32] = __half_as_ushort(h);
+    ol[sl * 32] = __half_as_ushort(l);
+  };
+  int64_t sl = warp;
+  for (; sl + 3 * kWarps < nsl; sl += 4 * kWarps) {
+    uint16_t v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = __ldg(xr + (sl + u * kWarps) * 32);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) emit(sl + u * kWarps, v[u]);
   }
+  for (; sl < nsl; sl += kWarps) emit(sl, __ldg(xr + sl * 32));
 }
 
 // ------------------------------------------------------------------ MoE routing
@@ -466,23 +454,31 @@ cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales,
   return cudaGetLastError();
 }
 
-cudaError_t launch_rotate_act(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
-                              const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
-                              uint16_t* xh, uint16_t* xl, uint32_t mask, int32_t* zero_ptr, int64_t nzero,
-                              cudaStream_t st) {
-  int g = grid_for(rows_alloc * (k / 32), 256);
-  rotate_act_kernel<<<g, 256, 0, st>>>(x, k, gather, topk, rows_valid_dev, rows_valid_host, rows_alloc, xh, xl,
-                                       mask, zero_ptr, nzero);
-  note_launches(1);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_rotate_rows_f16(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
-                                   const int32_t* rows_valid_dev, int64_t rows_alloc, uint16_t* xh, uint16_t* xl,
-                                   float* row_scale, uint32_t mask, cudaStream_t st) {
+cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
+                                 const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
+                                 uint16_t* xh, uint16_t* xl, float* row_scale, uint32_t mask, cudaStream_t st) {
   if (rows_alloc <= 0) return cudaSuccess;
-  rotate_rows_f16_kernel<<<static_cast<unsigned>(rows_alloc), 256, 0, st>>>(x, k, gather, topk, rows_valid_dev,
-                                                                            rows_alloc, xh, xl, row_scale, mask);
+  static bool attr_set = false;
+  if (!attr_set) {
+    // the stream-K kernel runs with the largest shared-memory carveout; an SM
+    // hosts CTAs of two kernels at once only if their carveouts agree
+    const cudaError_t e =
+        cudaFuncSetAttribute(rotate_scaled_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(rows_alloc));
+  cfg.blockDim = dim3(kRotThreads);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, rotate_scaled_kernel, x, k, gather, topk, rows_valid_dev,
+                                           rows_valid_host, xh, xl, row_scale, mask);
+  if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();
 }

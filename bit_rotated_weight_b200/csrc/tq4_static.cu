@@ -8,7 +8,8 @@
 // caller cannot supply the workspace tq4_1s_linear asks for.  This entry point
 // runs the same two kernels as tq4_1s_linear's small-m path (activation
 // rotation, then the stream-K dequant-GEMM) but keeps their scratch -- the
-// rotated activations, the stream-K partial sums and the tile counters -- in
+// rotated activations and their row scales, the stream-K partial sums and the
+// tile counters -- in
 // one file-scope device array of fixed size, allocated once per GPU when the
 // library's module loads there and held until the process exits.
 #include <mutex>
@@ -28,8 +29,10 @@ constexpr int64_t kStaticMaxN = 32768;
 constexpr int kStaticMaxGrid = 148;
 constexpr size_t kStaticXBytes = static_cast<size_t>(kStaticMaxM * kStaticMaxK) * 2;   // x' hi (or lo)
 constexpr size_t kStaticPartialBytes = static_cast<size_t>(kStaticMaxGrid) * 2 * 128 * kSegRows * 4;
-constexpr size_t kStaticCounterBytes = static_cast<size_t>(kStaticMaxN / 128) * 4;
-constexpr size_t kStaticScratchBytes = 2 * kStaticXBytes + kStaticPartialBytes + kStaticCounterBytes;  // ~5.6 MiB
+constexpr size_t kStaticScaleBytes = 256;                                              // x' row scales
+constexpr size_t kStaticCounterBytes = static_cast<size_t>(kStaticMaxN / 128) * 8;
+constexpr size_t kStaticScratchBytes =
+    2 * kStaticXBytes + kStaticScaleBytes + kStaticPartialBytes + kStaticCounterBytes;   // ~5.6 MiB
 
 // The scratch itself.  In host code this name is only a stand-in for the
 // device symbol: its device address must be fetched with cudaGetSymbolAddress.
@@ -90,8 +93,10 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   uint8_t* base = static_cast<uint8_t*>(scratch);
   uint16_t* xh = reinterpret_cast<uint16_t*>(base);
   uint16_t* xl = reinterpret_cast<uint16_t*>(base + kStaticXBytes);
-  float* partials = reinterpret_cast<float*>(base + 2 * kStaticXBytes);
-  int32_t* counters = reinterpret_cast<int32_t*>(base + 2 * kStaticXBytes + kStaticPartialBytes);
+  float* xscale = reinterpret_cast<float*>(base + 2 * kStaticXBytes);
+  float* partials = reinterpret_cast<float*>(base + 2 * kStaticXBytes + kStaticScaleBytes);
+  unsigned long long* counters =
+      reinterpret_cast<unsigned long long*>(base + 2 * kStaticXBytes + kStaticScaleBytes + kStaticPartialBytes);
   const int64_t row_tiles = (w->n + 127) / 128, k_iters = (w->k + 127) / 128;
   const int64_t tiles = row_tiles;   // m <= 32: one segment
   const int64_t T = tiles * k_iters;
@@ -101,9 +106,14 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   uint32_t mask = 0;
   tq4_1s_sign_mask(w->seed, &mask);
 
-  // The rotation kernel also zeroes this call's tile counters, which the
-  // previous call left in the shared scratch.
-  if (launch_rotate_act(x, w->k, nullptr, 1, nullptr, m, m, xh, xl, mask, counters, tiles, st) != cudaSuccess)
+  // m <= 32 is one segment: the stream-K kernel rotates x itself when no CTA
+  // runs more iterations than it has stages; otherwise the rotation kernel
+  // writes x' into the scratch first.  The tile counters carry each launch's
+  // epoch, so what a previous call left in them does no harm.
+  const int split = choose_cluster_split(tiles, k_iters, sms < kStaticMaxGrid ? sms : kStaticMaxGrid);
+  if (split > 1) grid = static_cast<int>(tiles * split);
+  const bool fused = split > 1 || (T + grid - 1) / grid <= kFusedMaxIters;
+  if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xh, xl, xscale, mask, st) != cudaSuccess)
     return TQ_ERR_CUDA;
   alignas(64) CUtensorMap tc, th, tl;
   {
@@ -151,6 +161,13 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   a.m_host = static_cast<int32_t>(m);
   a.nb_max = m > 16 ? 2 : 1;
   a.scales = w->scales;
+  a.row_scale = xscale;
+  if (fused) {
+    a.x_raw = x;
+    a.x_mask = mask;
+  }
+  a.epoch = next_epoch();
+  a.cluster_s = split;
   a.mode = EPI_DENSE;
   a.out_a = y;
   a.partials = partials;

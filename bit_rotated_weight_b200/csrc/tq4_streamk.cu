@@ -4,76 +4,106 @@
 // Computes D[n][j] = sum_k w_n[n][k] * x'[j][k] for 128-row tiles of one
 // expert's weight, where w_n = c[code] * d are the rotated-domain levels
 // ("What Config-I means": 16-level Lloyd-Max codes, two half-block scales)
-// and x' = R x is the activation rotated per 32-slice, split into bf16 hi and
-// lo rows (route B: rotating the activations instead of inverse-rotating the
-// weights, which is equivalent because R is orthogonal).  Per 128-k
-// iteration of a 128-row tile:
-//   warp 0      TMA: packed codes tile [128 x 64 B] (64-byte swizzle) and the
-//               x' hi/lo tiles [rows x 128 k] (128-byte swizzle) into a
-//               shared-memory stage, completing on an mbarrier;
-//   warps 4-19  four dequant warpgroups (round-robin iterations), thread = row:
-//               16 B of codes + 8 fp16 scales -> 128 bf16 levels through a
-//               per-half-block scaled table looked up with byte permutes,
-//               written to tensor memory with tcgen05.st (the MMA A operand);
-//               one thread of the group then issues 8 tcgen05.mma (M=128,
-//               N=32*nb, K=16, A from tensor memory, B from shared memory)
-//               into the group's own accumulator -- four concurrent issuers;
-//   warps 2-3   (dense bf16 mode) rotate x per 32-slice in registers and
-//               write the x' hi/lo B tiles into the stage, 128-byte swizzled;
-//   warp 1      allocates / frees tensor memory;
-//   warps 20-23 epilogue, thread = row: tcgen05.ld of the accumulator in
-//               16-token chunks, hi + lo columns summed, then the mode's store.
+// and x' = R x is the activation rotated per 32-slice (route B: rotating the
+// activations instead of inverse-rotating the weights, which is equivalent
+// because R is orthogonal).  x' is fp16 hi + lo, each row scaled by a power
+// of two 2^-e; the levels are fp16(c[code] * 256 * d).  Both operands fp16,
+// fp32 accumulation; the epilogue multiplies by 2^e / 256, which is exact.
+//
+// x' comes from one of two places.  TMA-fed mode: the rotation kernel wrote
+// it to global memory (row_scale = 2^e per row) and the producer stages it
+// with TMA.  Fused mode (a dense layer of at most kSegRows rows whose CTAs
+// run at most kFusedMaxIters iterations each, so every iteration has a stage
+// of its own): the kernel rotates x itself in a prologue -- the dequant and
+// epilogue warps read x, take each row's maximum over the k range this CTA
+// covers, and write every stage's B tile -- while the codes are in flight,
+// which saves the second launch and the x' round trip through memory.
+//
+// Per 128-row x 128-k iteration of a tile:
+//   warp 0      TMA: codes tile [128 x 64 B] (64-byte swizzle) and, in
+//               TMA-fed mode, the x' hi/lo tiles [rows x 128 k] (128-byte
+//               swizzle) into a stage;
+//   warps 2-17  four dequant warpgroups (round-robin iterations), thread =
+//               weight row: 16 B of codes + 8 scales -> 128 levels.  Each
+//               code byte (two nibbles) indexes a shared-memory table of
+//               fp16 level pairs {256 c[lo], 256 c[hi]}, one copy per lane so
+//               a warp's 32 lookups hit 32 banks, and one packed fp16 multiply
+//               by {d, d} scales the pair.  The levels go to tensor memory
+//               with tcgen05.st (the MMA A operand), as two 64-k halves
+//               signalled separately;
+//   warp 1, 22  lane 0: MMA issuers (groups 0-1 / 2-3): 4 tcgen05.mma per
+//               half (M=128, N=32*nb, K=16, A from tensor memory, B from
+//               shared memory) into the group's own accumulator -- single-
+//               thread issue costs ~66-98 cycles per small-N instruction, so
+//               two issuers and four accumulators keep the tensor core fed;
+//   warps 18-21 epilogue, thread = row: tcgen05.ld of the accumulators,
+//               hi + lo and the groups summed, scaled back, the mode's store.
 // The flattened (segment, row tile, k iteration) space is split evenly over
 // the CTAs (stream-K).  A tile split between CTAs is finished by whichever
 // contributor arrives last on the tile's counter: it sums all contributors'
 // fp32 partials in CTA order (deterministic) and runs the epilogue, so no
-// CTA ever waits on another.
+// CTA ever waits on another.  Cluster split-K mode (fused mode with a grid of
+// tiles x s CTAs, s per tile): the even split gives each CTA 1/s of one
+// tile's k range; the s CTAs of a tile form a thread-block cluster, write
+// their partials to their own shared memory and, after a cluster barrier,
+// each sums 1/s of the tile's rows over the s partials in rank order through
+// distributed shared memory -- no partials or counters in global memory.
+#include <atomic>
+#include <mutex>
+
 #include "tq4_internal.h"
 
 namespace tq4 {
 namespace {
 
-constexpr int kThreads = 800;
 constexpr int kDequantGroups = 4;
-constexpr int kFirstDequantWarp = 4;
+constexpr int kFirstDequantWarp = 2;
 constexpr int kFirstEpilogueWarp = kFirstDequantWarp + 4 * kDequantGroups;
 // Two MMA-issuing threads: lane 0 of warp 1 serves dequant groups 0 and 1,
-// lane 0 of the last warp (24) groups 2 and 3.
+// lane 0 of the last warp (22) groups 2 and 3.
 constexpr int kIssuerWarpB = kFirstEpilogueWarp + 4;
-static_assert((kIssuerWarpB + 1) * 32 == kThreads, "warp roles cover the block");
+constexpr int kThreads = (kIssuerWarpB + 1) * 32;
+// fused mode: the dequant and epilogue warps rotate x before their own work
+constexpr int kPrologueThreads = (kFirstEpilogueWarp + 4 - kFirstDequantWarp) * 32;
 constexpr int kStages = 8;
-constexpr int kAStages = 4;
 constexpr int kCodesBytes = 128 * 64;    // 128 rows x 128 k codes
-constexpr int kXHalfBytes = 64 * 128;    // 64 rows x 64 k bf16 (one 128-B swizzle span)
+constexpr int kXHalfBytes = 64 * 128;    // 64 rows x 64 k of fp16 x' (one 128-B swizzle span)
 constexpr int kXBytes = 2 * kXHalfBytes; // two k-halves
 constexpr int kStageBytes = kCodesBytes + kXBytes;
+constexpr int kLutBytes = 256 * 32 * 4;  // fp16 level-pair table, one copy per lane
 constexpr int kTmemCols = 512;
 // Tensor memory: columns [0, 256) hold the accumulators, [256, 512) the four
-// A stages (one per dequant warpgroup, 64 columns = 128 k of bf16 levels).
-// Each warpgroup issues the MMAs of its own iterations into its own
-// accumulator (N = 32 * nb columns): single-thread tcgen05.mma issue costs
-// ~66-98 cycles per instruction at small N, so four concurrent issuers are
-// needed to keep pace with the weight stream.  With nb = 1 (<= 16 tokens per
-// segment) the four accumulators take 128 columns and two accumulator sets
-// alternate between tile portions; with nb = 2 one set of 256 columns.
+// A stages (one per dequant group, 64 columns = 128 k of fp16 levels).  With
+// nb = 1 (<= 16 tokens per segment) the four group accumulators take 128
+// columns and two accumulator sets alternate between tile portions; with
+// nb = 2 one set of 256 columns.
 constexpr int kAccRegion = 256;
 constexpr int kACol0 = kAccRegion;
 constexpr int kAColsPerStage = 64;
-static_assert(kACol0 + kAStages * kAColsPerStage <= kTmemCols, "tensor memory budget");
-static_assert(kAStages == kDequantGroups, "one A stage per dequant warpgroup");
+static_assert(kACol0 + kDequantGroups * kAColsPerStage <= kTmemCols, "tensor memory budget");
+static_assert(kFusedMaxIters <= kStages, "fused mode gives each iteration its own stage");
+// fp16 levels carry a factor 256 (2^8): with it, half-block scales d from
+// ~2e-6 up to 65504 / fp16(256 * max level) ~ 93.6 give normal, finite fp16
+// levels.  Larger scales overflow; the dequant warps flag them.
+constexpr float kLevelScale = 256.0f;
 
 struct SharedState {
-  uint64_t full[kStages];      // TMA landed (codes, x') and rotated x' written
+  uint64_t full[kStages];      // the stage's codes and x' tiles landed
   uint64_t done[kStages];      // the MMAs of the iteration that used this stage completed
   uint64_t afull[kDequantGroups][2];   // a half A stage (64 k) holds fresh levels (128 arrivals)
   uint64_t afree[kDequantGroups][2];   // the MMAs reading a half A stage completed
-  uint64_t dfull[2];           // all four warpgroups finished a portion (4 arrivals)
+  uint64_t dfull[2];           // all four groups finished a portion (4 arrivals)
   uint64_t dempty[2];          // the epilogue drained an accumulator set (128 arrivals)
   uint64_t issuer_done[2];
+  uint64_t xready;             // fused mode: every stage's x' tile is written (one arrival per prologue warp)
+  uint64_t xissued;            // fused mode: the prologue's global reads are issued (one arrival per prologue warp)
+  float row_scale[kSegRows];   // fused mode: 2^e of each row
+  unsigned row_max[kSegRows];  // fused mode: max |x| of each row over this CTA's k range (float bits)
   uint32_t tmem_base;
   int abort_flag;
   int last_flag;
   int epi_ok[2];
+  int x_ok;                    // fused mode: the epilogue saw xready complete
 };
 
 struct Seg {
@@ -82,25 +112,38 @@ struct Seg {
 
 __device__ __forceinline__ Seg get_seg(const StreamKArgs& a, int s) {
   if (a.segs) {
-    const int4 v = a.segs[s];
+    const int4 v = __ldcg(a.segs + s);
     return {v.x, v.y, v.z};
   }
   const int r0 = s * kSegRows;
   return {0, r0, min(kSegRows, a.m_host - r0)};
 }
 
+// floor(a / b) for 0 <= a < 2^62, 0 < b < 2^31: an fp64 estimate, then an
+// exact integer correction (the estimate is off by at most one) -- far
+// cheaper than a 64-bit integer division.
+__device__ __forceinline__ int floordiv(long long a, int b) {
+  long long q = static_cast<long long>(static_cast<double>(a) * (1.0 / static_cast<double>(b)));
+  if (q * b > a) --q;
+  else if ((q + 1) * b <= a) ++q;
+  return static_cast<int>(q);
+}
 // First iteration of CTA c when T iterations are split over G CTAs.
-__device__ __forceinline__ int64_t range_begin(int64_t c, int64_t T, int64_t G) { return c * T / G; }
-// The CTA whose range holds iteration i.
-__device__ __forceinline__ int64_t owner_of(int64_t i, int64_t T, int64_t G) { return ((i + 1) * G + T - 1) / T - 1; }
+__device__ __forceinline__ int range_begin(int c, int T, int G) {
+  return floordiv(static_cast<long long>(c) * T, G);
+}
+// The CTA whose range holds iteration i: ceil((i + 1) G / T) - 1.
+__device__ __forceinline__ int owner_of(int i, int T, int G) {
+  return floordiv(static_cast<long long>(i + 1) * G + T - 1, T) - 1;
+}
 
 // Position of an iteration in the (segment, row tile, k iteration) space,
 // advanced incrementally so the loops do no integer division.
 struct Cursor {
   int tile, kit, sgi, rt;
-  __device__ __forceinline__ void init(int64_t it, int KI, int RT) {
-    tile = static_cast<int>(it / KI);
-    kit = static_cast<int>(it - static_cast<int64_t>(tile) * KI);
+  __device__ __forceinline__ void init(int it, int KI, int RT) {
+    tile = it / KI;
+    kit = it - tile * KI;
     sgi = tile / RT;
     rt = tile - sgi * RT;
   }
@@ -137,64 +180,32 @@ __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volati
   return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
 }
 
-__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
-  uint64_t d;
-  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
-  return d;
-}
-__device__ __forceinline__ uint64_t pack_f32x2(float lo, float hi) {
-  return static_cast<uint64_t>(__float_as_uint(lo)) | (static_cast<uint64_t>(__float_as_uint(hi)) << 32);
-}
-template <bool kF16>
-__device__ __forceinline__ uint32_t x2_from_f32x2(uint64_t v) {
-  const float lo = __uint_as_float(static_cast<uint32_t>(v)), hi = __uint_as_float(static_cast<uint32_t>(v >> 32));
-  if constexpr (kF16) {
-    __half2 h = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&h);
-  } else {
-    return pack_bf16x2(lo, hi);
-  }
-}
-
-// Dequantize one half-block (16 codes in q0 = elements 0..7, q1 = 8..15, one
-// nibble each, low nibble first) with scale d into 8 registers of bf16 pairs
-// {element 2i, element 2i+1}, value bf16(c[code] * d) (or fp16 when kF16)
-// with one rounding of the fp32 product.
-//
-// The codebook is odd-symmetric (c[15-j] = -c[j]), so a code j maps to a
-// magnitude index m = j-8 (j >= 8) or 7-j (j < 8) and a sign (j < 8).  The 8
-// scaled magnitudes are built per half-block as bf16 and split into a
-// low-byte plane and a high-byte plane (two registers each); prmt then looks
-// up four codes at a time by byte index, the sign is OR-ed into the high
-// bytes, and a last prmt interleaves low/high bytes into bf16 pairs.
-template <bool kF16>
-__device__ __forceinline__ void dequant_half(uint32_t q0, uint32_t q1, float d, const uint64_t (&cm2)[4],
+// Dequantize one half-block: 16 codes in q0 (elements 0..7) and q1 (8..15),
+// one nibble each, low nibble first; dd = {d, d} in fp16.  Each code byte
+// indexes the lane's copy of the level-pair table (`lut_lane` = byte address
+// of the copy's entry 0; entries are 128 bytes apart); out[i] = fp16 pair
+// {element 2i, element 2i+1} = fp16(256 c[code] * d) each.
+__device__ __forceinline__ void dequant_half(uint32_t q0, uint32_t q1, uint32_t dd, uint32_t lut_lane,
                                              uint32_t* out) {
-  const uint64_t dd = pack_f32x2(d, d);
-  const uint32_t p01 = x2_from_f32x2<kF16>(fmul2(cm2[0], dd));
-  const uint32_t p23 = x2_from_f32x2<kF16>(fmul2(cm2[1], dd));
-  const uint32_t p45 = x2_from_f32x2<kF16>(fmul2(cm2[2], dd));
-  const uint32_t p67 = x2_from_f32x2<kF16>(fmul2(cm2[3], dd));
-  const uint32_t lo0 = prmt(p01, p23, 0x6420u), lo1 = prmt(p45, p67, 0x6420u);
-  const uint32_t hi0 = prmt(p01, p23, 0x7531u), hi1 = prmt(p45, p67, 0x7531u);
 #pragma unroll
   for (int w = 0; w < 2; ++w) {
     const uint32_t q = w ? q1 : q0;
-    const uint32_t pos = (q >> 3) & 0x11111111u;            // 1 where code >= 8
-    const uint32_t m = (q ^ (0x77777777u - pos * 7u)) & 0x77777777u;  // magnitude index per nibble
-    const uint32_t qs = q << 4;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t sel = h ? (m >> 16) : m;
-      const uint32_t l4 = prmt(lo0, lo1, sel);
-      uint32_t h4 = prmt(hi0, hi1, sel);
-      // 0xFF per byte where the code is >= 8 (sign bit of nibble replicated)
-      const uint32_t posmask = prmt(qs, q, h ? 0xFBEAu : 0xD9C8u);
-      h4 |= ~posmask & 0x80808080u;
-      out[4 * w + 2 * h + 0] = prmt(l4, h4, 0x5140u);
-      out[4 * w + 2 * h + 1] = prmt(l4, h4, 0x7362u);
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t idx = prmt(q, 0u, 0x4440u + static_cast<uint32_t>(b));   // byte b, zero-extended
+      uint32_t v;   // (the table is written once, before the kernel's first barrier)
+      asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(lut_lane + idx * 128u));
+      uint32_t r;
+      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(dd));
+      out[4 * w + b] = r;
     }
   }
+}
+
+__device__ __forceinline__ uint32_t hmax2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
 }
 
 // 32-point Sylvester butterfly on a register array (stages h = 1..16).
@@ -217,119 +228,113 @@ __device__ __forceinline__ float relu2_bf16(float v) {
   return __bfloat162float(__float2bfloat16_rn(__fmul_rn(r, r)));
 }
 
-__device__ __forceinline__ float warp_fwht32_epi(float a, int lane) {
-#pragma unroll
-  for (int h = 1; h < 32; h <<= 1) {
-    const float p = __shfl_xor_sync(0xFFFFFFFFu, a, h);
-    a = (lane & h) ? __fsub_rn(p, a) : __fadd_rn(a, p);
-  }
-  return a;
-}
-
 // The per-mode store of 16 tokens [j0, j0 + 16) of one finished tile row
 // (thread = weight row `row`).
-__device__ __forceinline__ void epilogue_store(const StreamKArgs& a, float (&v)[16], int j0, int row, int lane,
+__device__ __forceinline__ void epilogue_store(const StreamKArgs& a, const float (&v)[16], int j0, int row,
                                                const Seg& sg) {
   const int cnt = sg.count - j0;
-  if (a.row_scale) {
+  if (row >= a.n) return;
+  if (a.mode == EPI_DENSE) {
 #pragma unroll
     for (int j = 0; j < 16; ++j)
-      if (j < cnt) v[j] = __fmul_rn(v[j], a.row_scale[sg.row0 + j0 + j]);
-  }
-  if (a.mode == EPI_DENSE) {
-    if (row < a.n) {
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        if (j < cnt)
-          a.out_a[static_cast<int64_t>(sg.row0 + j0 + j) * a.n + row] =
-              __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
-    }
+      if (j < cnt)
+        a.out_a[static_cast<int64_t>(sg.row0 + j0 + j) * a.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
   } else if (a.mode == EPI_UP) {
-    // h = bf16(relu(u)^2), then rotate the 32-slice held by this warp with the
-    // down projection's signs and split into hi/lo rows for the next stage.
-    const int slice0 = row - lane;
-    if (slice0 < a.n) {
-      const bool neg = (a.next_mask >> lane) & 1u;
-      const float r = __uint_as_float(0x3E3504F3u);
+    // h = bf16(relu(u)^2) per sorted pair row: the down projection's input
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j < cnt) {
-          const float hv = relu2_bf16(v[j]);
-          const float t = __fmul_rn(warp_fwht32_epi(neg ? -hv : hv, lane), r);
-          const __nv_bfloat16 hi = __float2bfloat16_rn(t);
-          const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(t, __bfloat162float(hi)));
-          const int64_t off = static_cast<int64_t>(sg.row0 + j0 + j) * a.n + row;
-          a.out_a[off] = __bfloat16_as_ushort(hi);
-          a.out_b[off] = __bfloat16_as_ushort(lo);
-        }
-      }
-    }
+    for (int j = 0; j < 16; ++j)
+      if (j < cnt)
+        a.out_a[static_cast<int64_t>(sg.row0 + j0 + j) * a.n + row] =
+            __bfloat16_as_ushort(__float2bfloat16_rn(relu2_bf16(v[j])));
   } else {
-    if (row < a.n) {
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        if (j < cnt) {
-          const int p = a.pairs[sg.row0 + j0 + j];
-          a.out_f[static_cast<int64_t>(p) * a.n + row] = __fmul_rn(a.topk_w[p], v[j]);
-        }
+    for (int j = 0; j < 16; ++j) {
+      if (j < cnt) {
+        const int p = __ldcg(a.pairs + sg.row0 + j0 + j);
+        a.out_f[static_cast<int64_t>(p) * a.n + row] = __fmul_rn(__ldcg(a.topk_w + p), v[j]);
       }
     }
   }
 }
 
-struct Codemag {
-  float v[8];   // levels[8..15]: the positive magnitudes, ascending
+struct LevelTable {
+  uint32_t h[16];    // fp16 bits of 256 * levels[0..15]
+  float max_level;   // fp16(256 * levels[15]) as a float
 };
 
-template <bool kF16>
 __global__ void __launch_bounds__(kThreads, 1)
     streamk_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_xhi,
-                   const __grid_constant__ CUtensorMap tm_xlo, const StreamKArgs a, const Codemag cmag) {
+                   const __grid_constant__ CUtensorMap tm_xlo, const StreamKArgs a,
+                   const __grid_constant__ LevelTable lt) {
   __shared__ SharedState sh;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  uint8_t* lut = smem + kStages * kStageBytes;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Grouped (MoE) mode reads the routing kernel's segment list right away;
   // the dense mode defers the dependency wait to the roles that need it.
   if (a.segs) pdl_wait();
-  const int nseg = a.segs ? *a.nseg_dev : a.nseg_host;
+  const int nseg = a.segs ? __ldcg(a.nseg_dev) : a.nseg_host;
   const int KI = a.k_iters;
-  const int64_t T = static_cast<int64_t>(nseg) * a.row_tiles * KI;
-  const int64_t G = gridDim.x;
-  const int64_t it_begin = range_begin(blockIdx.x, T, G);
-  const int64_t it_end = range_begin(blockIdx.x + 1, T, G);
-  const int cnt = static_cast<int>(it_end - it_begin);
-  if (cnt <= 0) return;
-  // accumulator layout (see kAccRegion): width per warpgroup, number of sets
+  const int T = nseg * a.row_tiles * KI;   // < 2^31 (checked by the host)
+  const int G = gridDim.x;
+  const int it_begin = range_begin(blockIdx.x, T, G);
+  const int it_end = range_begin(blockIdx.x + 1, T, G);
+  const int cnt = it_end - it_begin;
+  if (cnt <= 0) {
+    // (the host never gives a cluster-mode CTA an empty range; if one had
+    // one, it would still meet its cluster's barriers)
+    if (a.cluster_s > 1) {
+      cluster_sync_all();
+      cluster_sync_all();
+    }
+    return;
+  }
+  const bool fused = a.x_raw != nullptr;
+  // accumulator layout (see kAccRegion): width per group, number of sets
   const int acc_w = 32 * a.nb_max;
   const int nsets = (a.nb_max == 1) ? 2 : 1;
-  const int64_t tile_begin = it_begin / KI, tile_last = (it_end - 1) / KI;
-  const int nportions = static_cast<int>(tile_last - tile_begin + 1);
+  const int tile_begin = it_begin / KI, tile_last = (it_end - 1) / KI;
+  const int nportions = tile_last - tile_begin + 1;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sh.full[i], a.x_raw ? 3 : 1);   // producer (+ the two rotation warps)
+      mbar_init(&sh.full[i], 1);
       mbar_init(&sh.done[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.dfull[i], kDequantGroups);
-      mbar_init(&sh.dempty[i], 128);
     }
     for (int i = 0; i < kDequantGroups; ++i)
       for (int h = 0; h < 2; ++h) {
         mbar_init(&sh.afull[i][h], 128);
         mbar_init(&sh.afree[i][h], 1);
       }
-    for (int i = 0; i < 2; ++i) mbar_init(&sh.issuer_done[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.dfull[i], kDequantGroups);
+      mbar_init(&sh.dempty[i], 128);
+      mbar_init(&sh.issuer_done[i], 1);
+    }
+    mbar_init(&sh.xready, kPrologueThreads / 32);
+    mbar_init(&sh.xissued, kPrologueThreads / 32);
+    for (int j = 0; j < kSegRows; ++j) sh.row_max[j] = 0u;
     sh.abort_flag = 0;
     sh.last_flag = 0;
     fence_mbar_init();
   }
+  {
+    // table entry b (a code byte) of lane l's copy, at byte 128 b + 4 l:
+    // {256 c[b & 15], 256 c[b >> 4]}
+    uint32_t* lw = reinterpret_cast<uint32_t*>(lut);
+    for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
+      const int b = i >> 5;
+      lw[i] = lt.h[b & 15] | (lt.h[b >> 4] << 16);
+    }
+  }
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_codes);
-    tma_prefetch_desc(&tm_xhi);
-    tma_prefetch_desc(&tm_xlo);
+    if (!fused) {
+      tma_prefetch_desc(&tm_xhi);
+      tma_prefetch_desc(&tm_xlo);
+    }
   }
   if (warp == 1) {
     tmem_alloc(&sh.tmem_base, kTmemCols);
@@ -340,20 +345,205 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = sh.tmem_base;
   volatile int* abortp = &sh.abort_flag;
-  if (threadIdx.x == 0) pdl_launch_dependents();
+
+  // In fused mode the kernel before this one may have written anything, the
+  // weight included: the prologue warps wait for it before any global read
+  // (the producer does the same).
+  if (fused && warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp + 4) pdl_wait();
+  // The dequant warps' first scale loads go out before the prologue, so their
+  // latency overlaps it; in fused mode a group has at most two iterations and
+  // loads the scales of both, before the weight stream starts.
+  uint32_t first_raw[4] = {0u, 0u, 0u, 0u}, second_raw[4] = {0u, 0u, 0u, 0u};
+  if (warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp) {
+    const int wg = (warp - kFirstDequantWarp) >> 2;
+    const int t = (warp & 3) * 32 + lane;
+    const int kh16 = a.k / 16;
+    auto load_scales = [&](int li, uint32_t (&raw)[4]) {
+      Cursor c0;
+      c0.init(it_begin + li, KI, a.row_tiles);
+      const int row = c0.rt * 128 + t;
+      if (row < a.n) {
+        const uint32_t* sp = reinterpret_cast<const uint32_t*>(
+            a.scales + (static_cast<int64_t>(get_seg(a, c0.sgi).e) * a.n + row) * kh16 + c0.kit * 8);
+        if ((kh16 & 7) == 0) {   // 16-byte aligned rows: one load
+          const uint4 v = __ldg(reinterpret_cast<const uint4*>(sp));
+          raw[0] = v.x;
+          raw[1] = v.y;
+          raw[2] = v.z;
+          raw[3] = v.w;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) raw[j] = (c0.kit * 8 + 2 * j < kh16) ? __ldg(sp + j) : 0u;
+        }
+      }
+    };
+    if (wg < cnt) load_scales(wg, first_raw);
+    if (fused && wg + kDequantGroups < cnt) load_scales(wg + kDequantGroups, second_raw);
+  }
+
+  if (fused && warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp + 4) {
+    // ------------------------------------------------------------ fused prologue
+    // Unit u = (iteration li, slice sl, row j), j fastest: 32 consecutive x
+    // values of row j at k = 128 kit(li) + 32 sl; a thread takes units ptid
+    // and ptid + kPrologueThreads and keeps their x in registers.  Pass 1
+    // takes each row's max |x| over the units; pass 2 applies the signs, the
+    // butterfly and r 2^-e, splits into fp16 hi/lo and writes them into stage
+    // li's B tile: hi in row j, lo in row 16 nb + j, 16-byte chunk c of a
+    // 128-byte row at chunk c ^ (row & 7) (128-byte swizzle).  The exponent e
+    // puts sqrt(32) max|x|, the bound on |x'|, in [2^13, 2^14).
+    const int ptid = threadIdx.x - kFirstDequantWarp * 32;
+    const int m = a.m_host, nb = (m + 15) >> 4;
+    const int units = cnt * 4 * m;   // <= kFusedMaxIters * 4 * kSegRows = 2 * kPrologueThreads
+    static_assert(kFusedMaxIters * 4 * kSegRows <= 2 * kPrologueThreads, "two units per prologue thread");
+    uint32_t raw[2][16];   // the thread's units of x, bf16 pairs, kept for pass 2
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int u = ptid + r * kPrologueThreads;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) raw[r][i] = 0u;
+      if (u < units) {
+        const int j = u % m, rest = u / m, sl = rest & 3, li = rest >> 2;
+        const int k0 = ((it_begin + li) % KI) * 128 + 32 * sl;
+        if (k0 < a.k) {
+          const uint4* src = reinterpret_cast<const uint4*>(a.x_raw + static_cast<int64_t>(j) * a.k + k0);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const uint4 w = __ldg(src + q);
+            raw[r][4 * q] = w.x;
+            raw[r][4 * q + 1] = w.y;
+            raw[r][4 * q + 2] = w.z;
+            raw[r][4 * q + 3] = w.w;
+          }
+        }
+      }
+    }
+    // the small reads are on their way: let the producer start the weight
+    // stream behind them (relaxed: the loads need not have completed)
+    __syncwarp();
+    if (lane == 0) asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sh.xissued)) : "memory");
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int u = ptid + r * kPrologueThreads;
+      if (u < units) {
+        float mx = 0.0f;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          mx = fmaxf(mx, fabsf(__uint_as_float(raw[r][i] << 16)));
+          mx = fmaxf(mx, fabsf(__uint_as_float(raw[r][i] & 0xFFFF0000u)));
+        }
+        atomicMax(&sh.row_max[u % m], __float_as_uint(mx));   // non-negative floats order as integers
+      }
+    }
+    named_bar_sync(2, kPrologueThreads);
+    const float r = __uint_as_float(0x3E3504F3u);
+#pragma unroll
+    for (int rr = 0; rr < 2; ++rr) {
+      const int u = ptid + rr * kPrologueThreads;
+      if (u >= units) continue;
+      const int j = u % m, rest = u / m, sl = rest & 3, li = rest >> 2;
+      float v[32];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        v[2 * i] = __uint_as_float(raw[rr][i] << 16);
+        v[2 * i + 1] = __uint_as_float(raw[rr][i] & 0xFFFF0000u);
+      }
+#pragma unroll
+      for (int i = 0; i < 32; ++i)
+        if ((a.x_mask >> i) & 1u) v[i] = -v[i];
+      fwht32_regs_sk(v);
+      const float mx = __uint_as_float(sh.row_max[j]);
+      int e = 0;
+      if (mx > 0.0f && isfinite(mx)) {
+        int ex;
+        frexpf(__fmul_rn(mx, 5.65685415f), &ex);   // the bound lies in [2^(ex-1), 2^ex)
+        e = ex - 14;
+        e = e < -100 ? -100 : (e > 100 ? 100 : e);
+      }
+      if (li == 0 && sl == 0) sh.row_scale[j] = ldexpf(1.0f, e);
+      const float rd = __fmul_rn(r, ldexpf(1.0f, -e));   // exact: r times a power of two
+      uint8_t* hbase = smem + li * kStageBytes + kCodesBytes + (sl >> 1) * kXHalfBytes;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t hw[4], lw[4];
+#pragma unroll
+        for (int c2 = 0; c2 < 4; ++c2) {
+          const float f0 = __fmul_rn(v[8 * q + 2 * c2], rd), f1 = __fmul_rn(v[8 * q + 2 * c2 + 1], rd);
+          const __half h0 = __float2half_rn(f0), h1 = __float2half_rn(f1);
+          const __half l0 = __float2half_rn(__fsub_rn(f0, __half2float(h0)));
+          const __half l1 = __float2half_rn(__fsub_rn(f1, __half2float(h1)));
+          hw[c2] = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
+          lw[c2] = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+        }
+        const int c = (sl & 1) * 4 + q;
+        const int rh = j, rl = 16 * nb + j;
+        *reinterpret_cast<uint4*>(hbase + rh * 128 + ((c ^ (rh & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(hbase + rl * 128 + ((c ^ (rl & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      }
+    }
+    fence_proxy_async_smem();   // the generic-proxy writes, before the tensor core reads them
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.xready);
+  }
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      if (!a.x_raw) pdl_wait();   // x' tiles are the previous kernel's output
       int armed[kStages];
 #pragma unroll
       for (int i = 0; i < kStages; ++i) armed[i] = -1;
+      auto load_x = [&](uint8_t* st, int kit, const Seg& sg, int nb, uint64_t* bar) {
+        for (int b = 0; b < nb; ++b) {
+#pragma unroll
+          for (int kh = 0; kh < 2; ++kh) {
+            uint8_t* xb = st + kCodesBytes + kh * kXHalfBytes;
+            tma_load_2d(xb + (16 * b) * 128, &tm_xhi, bar, kit * 128 + 64 * kh, sg.row0 + 16 * b);
+            tma_load_2d(xb + (16 * nb + 16 * b) * 128, &tm_xlo, bar, kit * 128 + 64 * kh, sg.row0 + 16 * b);
+          }
+        }
+      };
+      // TMA-fed mode: the codes of the first stages go out before the
+      // dependency wait -- the kernel before this one (the activation
+      // rotation) lets it start only once everything earlier has finished,
+      // and does not write the weight.  Fused mode: any kernel may come
+      // before, so wait first.
+      if (fused) {
+        pdl_wait();
+        // the weight stream goes out behind the prologue's reads of x and the
+        // first scales, which would otherwise queue behind ~all of it
+        mbar_wait(&sh.xissued, 0, abortp);
+      }
+      const int npre = cnt < kStages ? cnt : kStages;
+      const uint32_t xbytes = fused ? 0u : 4u * 2048u;
       Cursor cur;
       cur.init(it_begin, KI, a.row_tiles);
+      const Cursor first = cur;
       Seg sg = get_seg(a, cur.sgi);
       int seg_of = cur.sgi;
-      for (int li = 0; li < cnt; ++li, cur.advance(1, KI, a.row_tiles)) {
+      for (int li = 0; li < npre; ++li, cur.advance(1, KI, a.row_tiles)) {
+        if (cur.sgi != seg_of) {
+          seg_of = cur.sgi;
+          sg = get_seg(a, seg_of);
+        }
+        const int nb = (sg.count + 15) >> 4;
+        mbar_arrive_expect_tx(&sh.full[li], kCodesBytes + nb * xbytes);
+        armed[li] = 0;
+        tma_load_3d(smem + li * kStageBytes, &tm_codes, &sh.full[li], cur.kit * 64, cur.rt * 128, sg.e);
+      }
+      if (!fused) {
+        pdl_wait();   // x' and its row scales are the rotation kernel's output
+        Cursor c2 = first;
+        Seg sg2 = get_seg(a, c2.sgi);
+        int seg2 = c2.sgi;
+        for (int li = 0; li < npre; ++li, c2.advance(1, KI, a.row_tiles)) {
+          if (c2.sgi != seg2) {
+            seg2 = c2.sgi;
+            sg2 = get_seg(a, seg2);
+          }
+          load_x(smem + li * kStageBytes, c2.kit, sg2, (sg2.count + 15) >> 4, &sh.full[li]);
+        }
+      }
+      // (fused mode: cnt <= kStages, so the loop below does not run)
+      for (int li = npre; li < cnt; ++li, cur.advance(1, KI, a.row_tiles)) {
         const int s = li % kStages;
         const uint32_t ph = (li / kStages) & 1;
         if (!mbar_wait(&sh.done[s], ph ^ 1u, abortp)) break;
@@ -361,21 +551,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           seg_of = cur.sgi;
           sg = get_seg(a, seg_of);
         }
-        const int kit = cur.kit, rt = cur.rt;
         const int nb = (sg.count + 15) >> 4;
         uint8_t* st = smem + s * kStageBytes;
-        mbar_arrive_expect_tx(&sh.full[s], kCodesBytes + (a.x_raw ? 0 : nb * 4 * 2048));
+        mbar_arrive_expect_tx(&sh.full[s], kCodesBytes + nb * xbytes);
         armed[s] = static_cast<int>(ph);
-        tma_load_3d(st, &tm_codes, &sh.full[s], kit * 64, rt * 128, sg.e);
-        for (int b = 0; b < nb && !a.x_raw; ++b) {
-#pragma unroll
-          for (int kh = 0; kh < 2; ++kh) {
-            uint8_t* xb = st + kCodesBytes + kh * kXHalfBytes;
-            tma_load_2d(xb + (16 * b) * 128, &tm_xhi, &sh.full[s], kit * 128 + 64 * kh, sg.row0 + 16 * b);
-            tma_load_2d(xb + (16 * nb + 16 * b) * 128, &tm_xlo, &sh.full[s], kit * 128 + 64 * kh,
-                        sg.row0 + 16 * b);
-          }
-        }
+        tma_load_3d(st, &tm_codes, &sh.full[s], cur.kit * 64, cur.rt * 128, sg.e);
+        load_x(st, cur.kit, sg, nb, &sh.full[s]);
       }
       if (*abortp) {
         // wind down: let every armed copy land before the CTA exits
@@ -383,82 +564,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (armed[i] >= 0) drain_wait(&sh.full[i], static_cast<uint32_t>(armed[i]));
       }
     }
-  } else if (warp == 2 || warp == 3) {
-    // ------------------------------------------------------------ rotation
-    // Dense bf16 mode: x' = r H diag(s) x per 32-slice, split into bf16 hi and
-    // lo, written straight into the stage's B tile.  Unit u = (token j, slice
-    // sl) of the iteration's 128 k; the 64 threads take units u and u + 64.
-    if (a.x_raw) {
-      pdl_wait();   // x may be the previous kernel's output
-      const int tid = (warp - 2) * 32 + lane;
-      const float r = __uint_as_float(0x3E3504F3u);
-      Cursor cur;
-      cur.init(it_begin, KI, a.row_tiles);
-      for (int li = 0; li < cnt; ++li, cur.advance(1, KI, a.row_tiles)) {
-        const int s = li % kStages;
-        if (!warp_wait(&sh.done[s], ((li / kStages) & 1) ^ 1u, abortp)) break;
-        const Seg sg = get_seg(a, cur.sgi);
-        const int nb = (sg.count + 15) >> 4;
-        uint8_t* xb = smem + s * kStageBytes + kCodesBytes;
-        for (int u = tid; u < 64 * nb; u += 64) {
-          const int j = u >> 2, sl = u & 3;
-          const int k0 = cur.kit * 128 + 32 * sl;
-          float v[32];
-          if (j < sg.count && k0 < a.k) {
-            const uint4* src =
-                reinterpret_cast<const uint4*>(a.x_raw + static_cast<int64_t>(sg.row0 + j) * a.k + k0);
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-              const uint4 w = __ldg(src + q);
-              const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                v[8 * q + 2 * e] = __uint_as_float(ww[e] << 16);
-                v[8 * q + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
-              }
-            }
-#pragma unroll
-            for (int i = 0; i < 32; ++i)
-              if ((a.x_mask >> i) & 1u) v[i] = -v[i];
-            fwht32_regs_sk(v);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 32; ++i) v[i] = 0.0f;
-          }
-          // hi row j, lo row 16nb + j; slice sl covers bytes [(sl&1)*64, +64)
-          // of the 128-byte row in k-half (sl >> 1); 16-byte chunk c of row
-          // `row` sits at chunk c ^ (row & 7) (128-byte swizzle)
-          uint8_t* half = xb + (sl >> 1) * kXHalfBytes;
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            uint32_t hw[4], lw[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const float f0 = __fmul_rn(v[8 * q + 2 * e], r), f1 = __fmul_rn(v[8 * q + 2 * e + 1], r);
-              const __nv_bfloat16 h0 = __float2bfloat16_rn(f0), h1 = __float2bfloat16_rn(f1);
-              const __nv_bfloat16 l0 = __float2bfloat16_rn(__fsub_rn(f0, __bfloat162float(h0)));
-              const __nv_bfloat16 l1 = __float2bfloat16_rn(__fsub_rn(f1, __bfloat162float(h1)));
-              hw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(h0)) |
-                      (static_cast<uint32_t>(__bfloat16_as_ushort(h1)) << 16);
-              lw[e] = static_cast<uint32_t>(__bfloat16_as_ushort(l0)) |
-                      (static_cast<uint32_t>(__bfloat16_as_ushort(l1)) << 16);
-            }
-            const int c = (sl & 1) * 4 + q;
-            const int rh = j, rl = 16 * nb + j;
-            *reinterpret_cast<uint4*>(half + rh * 128 + ((c ^ (rh & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-            *reinterpret_cast<uint4*>(half + rl * 128 + ((c ^ (rl & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
-          }
-        }
-        fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.full[s]);
-      }
-    }
   } else if (warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp) {
     // ------------------------------------------------------------ dequant
-    // Warpgroup wg takes the iterations li = wg (mod 4).  Per iteration: the
-    // 8 fp16 scales (fetched one iteration ahead), 16 B of codes per row from
-    // the stage, and 128 levels per row written with tcgen05.st into the
+    // Group wg takes the iterations li = wg (mod 4).  Per iteration: the 8
+    // scales of the row (fetched one iteration ahead), 16 B of codes per row
+    // from the stage, and 128 levels per row written with tcgen05.st into the
     // group's A stage -- as two 64-k halves, each signalled separately, so the
     // tensor core reads one half while the group fills the other.
     const int wg = (warp - kFirstDequantWarp) >> 2;
@@ -466,37 +576,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int t = q * 32 + lane;            // row within the tile
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
     const uint32_t a_stage = tmem + kACol0 + wg * kAColsPerStage;
-    uint64_t cm2[4];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) cm2[i] = pack_f32x2(cmag.v[2 * i], cmag.v[2 * i + 1]);
+    const uint32_t lut_lane = smem_u32(lut) + 4u * static_cast<uint32_t>(lane);
     const int kh16 = a.k / 16;
+    int seg_cached = -1, e_cached = 0;   // expert of the segment whose scales were last fetched
     auto fetch_scales = [&](const Cursor& c, uint32_t (&raw)[4]) {
-      const int kit = c.kit, rt = c.rt;
-      const int e = get_seg(a, c.sgi).e;
-      const int row = rt * 128 + t;
+      if (c.sgi != seg_cached) {
+        seg_cached = c.sgi;
+        e_cached = get_seg(a, c.sgi).e;
+      }
+      const int row = c.rt * 128 + t;
       const bool rv = row < a.n;
       const uint32_t* sp = reinterpret_cast<const uint32_t*>(
-          a.scales + (static_cast<int64_t>(e) * a.n + (rv ? row : 0)) * kh16 + kit * 8);
+          a.scales + (static_cast<int64_t>(e_cached) * a.n + (rv ? row : 0)) * kh16 + c.kit * 8);
+      if ((kh16 & 7) == 0) {   // 16-byte aligned rows: one load
+        const uint4 v = rv ? __ldg(reinterpret_cast<const uint4*>(sp)) : make_uint4(0u, 0u, 0u, 0u);
+        raw[0] = v.x;
+        raw[1] = v.y;
+        raw[2] = v.z;
+        raw[3] = v.w;
+      } else {
 #pragma unroll
-      for (int j = 0; j < 4; ++j) raw[j] = (rv && kit * 8 + 2 * j < kh16) ? __ldg(sp + j) : 0u;
+        for (int j = 0; j < 4; ++j) raw[j] = (rv && c.kit * 8 + 2 * j < kh16) ? __ldg(sp + j) : 0u;
+      }
     };
-    uint32_t next_raw[4] = {0u, 0u, 0u, 0u};
-    Cursor ahead;   // the iteration whose scales are in flight
+    uint32_t next_raw[4] = {first_raw[0], first_raw[1], first_raw[2], first_raw[3]};
+    uint32_t dmax = 0u;   // running max of the scales seen (fp16 pairs)
+    Cursor ahead;         // the iteration whose scales are in flight
     ahead.init(it_begin + wg, KI, a.row_tiles);
-    if (wg < cnt) fetch_scales(ahead, next_raw);
     int use = 0;    // how many times this group has filled its A stage
     for (int li = wg; li < cnt; li += kDequantGroups, ++use) {
-      float dsc[8];
+      uint32_t sraw[4];
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
-        const __half2 h2 = *reinterpret_cast<const __half2*>(&next_raw[j]);
-        const float2 f2 = __half22float2(h2);
-        dsc[2 * j] = f2.x;
-        dsc[2 * j + 1] = f2.y;
+        sraw[j] = next_raw[j];
+        dmax = hmax2(dmax, sraw[j]);
       }
       if (li + kDequantGroups < cnt) {
-        ahead.advance(kDequantGroups, KI, a.row_tiles);
-        fetch_scales(ahead, next_raw);
+        if (fused) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) next_raw[j] = second_raw[j];
+        } else {
+          ahead.advance(kDequantGroups, KI, a.row_tiles);
+          fetch_scales(ahead, next_raw);
+        }
       }
       const int s = li % kStages;
       if (!warp_wait(&sh.full[s], (li / kStages) & 1, abortp)) break;
@@ -515,8 +637,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int kb = 2 * h + kb2;
           const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((t >> 1) & 3)));
           uint32_t o[16];
-          dequant_half<kF16>(c.x, c.y, dsc[2 * kb], cm2, o);
-          dequant_half<kF16>(c.z, c.w, dsc[2 * kb + 1], cm2, o + 8);
+          const uint32_t sp = sraw[kb];   // scales of the block's two halves
+          dequant_half(c.x, c.y, prmt(sp, 0u, 0x1010u), lut_lane, o);
+          dequant_half(c.z, c.w, prmt(sp, 0u, 0x3232u), lut_lane, o + 8);
           tmem_st16(a_stage + lane_base + 16 * kb, o);
         }
         tmem_wait_st();
@@ -525,6 +648,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (!ok) break;
     }
+    // a scale whose largest level overflows fp16 made some levels infinite
+    const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
+    if (fmaxf(dm.x, dm.y) * lt.max_level >= 65520.0f) raise_status(TQ_DEV_SCALE_RANGE);
   } else if ((warp == 1 || warp == kIssuerWarpB) && lane == 0) {
     // ------------------------------------------------------------ MMA issue
     // Issuer A (warp 1) serves groups 0-1, issuer B groups 2-3: the
@@ -535,11 +661,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int gb = (warp == 1) ? 0 : 2;
     const int ib = (warp == 1) ? 0 : 1;
     int use0 = 0, use1 = 0;   // fills of group gb / gb + 1 consumed so far
-    bool ok = true;
+    bool ok = !fused || mbar_wait(&sh.xready, 0, abortp);   // fused mode: the B tiles are written
     for (int pi = 0; pi < nportions && ok; ++pi) {
-      const int64_t tile = tile_begin + pi;
-      const int pf = static_cast<int>((tile * KI > it_begin ? tile * KI : it_begin) - it_begin);
-      const int pe = static_cast<int>(((tile + 1) * KI < it_end ? (tile + 1) * KI : it_end) - it_begin);
+      const int tile = tile_begin + pi;
+      const int pf = (tile * KI > it_begin ? tile * KI : it_begin) - it_begin;
+      const int pe = ((tile + 1) * KI < it_end ? (tile + 1) * KI : it_end) - it_begin;
       const int db = pi % nsets;
       const uint32_t dpar = static_cast<uint32_t>((pi / nsets) & 1);
       // the accumulator set must be free before any MMA or arrival of this portion
@@ -547,9 +673,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         ok = false;
         break;
       }
-      const Seg sg = get_seg(a, static_cast<int>(tile / a.row_tiles));
+      const Seg sg = get_seg(a, tile / a.row_tiles);
       const int nb = (sg.count + 15) >> 4;
-      const uint32_t idesc = kF16 ? idesc_f16(128, 32 * nb) : idesc_bf16(128, 32 * nb);
+      const uint32_t idesc = idesc_f16(128, 32 * nb);
       bool started0 = false, started1 = false;
       for (int li = pf; li < pe && ok; ++li) {
         const int w = li % kDequantGroups;
@@ -605,17 +731,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int q = warp & 3;
     const int t = q * 32 + lane;
     const uint32_t lane_base = static_cast<uint32_t>(q * 32) << 16;
-    int sgi = static_cast<int>(tile_begin / a.row_tiles);
-    int rt = static_cast<int>(tile_begin - static_cast<int64_t>(sgi) * a.row_tiles);
-    for (int pi = 0; pi < nportions; ++pi) {
-      const int64_t tile = tile_begin + pi;
+    // fused mode: the row scales come from the prologue
+    if (fused) {
+      if (t == 0) sh.x_ok = mbar_wait(&sh.xready, 0, abortp) ? 1 : 0;
+      named_bar_sync(1, 128);
+    }
+    int sgi = tile_begin / a.row_tiles;
+    int rt = tile_begin - sgi * a.row_tiles;
+    for (int pi = 0; pi < nportions && (!fused || sh.x_ok); ++pi) {
+      const int tile = tile_begin + pi;
       if (pi > 0 && ++rt == a.row_tiles) {
         rt = 0;
         ++sgi;
       }
-      const int64_t tile_first = tile * KI;
-      const int64_t portion_first = it_begin > tile_first ? it_begin : tile_first;
-      const int64_t portion_end = (tile + 1) * KI < it_end ? (tile + 1) * KI : it_end;
+      const int tile_first = tile * KI;
+      const int portion_first = it_begin > tile_first ? it_begin : tile_first;
+      const int portion_end = (tile + 1) * KI < it_end ? (tile + 1) * KI : it_end;
       const int db = pi % nsets;
       // one thread waits; the decision is published before the group barrier
       // so all four epilogue warps leave together on a timeout
@@ -626,9 +757,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Seg sg = get_seg(a, sgi);
       const int nb = (sg.count + 15) >> 4;
       const int row = rt * 128 + t;
-      // warpgroup w wrote an accumulator iff one of the portion's local
+      // group w wrote an accumulator iff one of the portion's local
       // iterations is congruent to w mod 4
-      const int lpf = static_cast<int>(portion_first - it_begin), plen = static_cast<int>(portion_end - portion_first);
+      const int lpf = portion_first - it_begin, plen = portion_end - portion_first;
       const uint32_t dbase = tmem + lane_base + db * (kAccRegion / nsets);
       const bool whole = (portion_first == tile_first) && (portion_end == tile_first + KI);
       const int slot = (pi == 0) ? 0 : 1;
@@ -641,41 +772,73 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int w = 0; w < kDequantGroups; ++w) {
           const int off = ((w - lpf) % kDequantGroups + kDequantGroups) % kDequantGroups;
           if (off >= plen) continue;
-          for (int part = 0; part < 2; ++part) {   // hi columns, then lo columns
-            uint32_t rr[16];
-            tmem_ld16(dbase + w * acc_w + 16 * nb * part + 16 * c, rr);
-            tmem_wait_ld();
+          uint32_t rh[16], rl[16];   // hi columns, lo columns
+          tmem_ld16(dbase + w * acc_w + 16 * c, rh);
+          tmem_ld16(dbase + w * acc_w + 16 * nb + 16 * c, rl);
+          tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __uint_as_float(rr[j]));
+          for (int j = 0; j < 16; ++j)
+            v[j] = __fadd_rn(__fadd_rn(v[j], __uint_as_float(rh[j])), __uint_as_float(rl[j]));
+        }
+        // back from the scaled domain: times 2^e / 256 per token (exact), with
+        // 2^e from the prologue in fused mode (it may differ between the CTAs
+        // of a split tile, so it is applied before the partials are published)
+        // or else the rotation kernel's row_scale
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int jj = 16 * c + j;
+          if (jj < sg.count) {
+            const float s = fused ? sh.row_scale[jj] : __ldcg(a.row_scale + sg.row0 + jj);
+            v[j] = __fmul_rn(v[j], __fmul_rn(s, 1.0f / kLevelScale));
           }
         }
         if (c == nb - 1) {
           tc_fence_before();
           mbar_arrive(&sh.dempty[db]);
         }
-        if (whole) {
-          epilogue_store(a, v, 16 * c, row, lane, sg);
+        if (a.cluster_s > 1) {
+          // cluster split-K: the partial goes to this CTA's reduction buffer
+          // (stage 0's B region, free once the MMAs completed), token-major
+          float* red = reinterpret_cast<float*>(smem + kCodesBytes);
+#pragma unroll
+          for (int j = 0; j < 16; ++j) red[(16 * c + j) * 128 + t] = v[j];
+        } else if (whole) {
+          epilogue_store(a, v, 16 * c, row, sg);
         } else {
           float4* pp = reinterpret_cast<float4*>(pbase + 16 * c);
 #pragma unroll
           for (int j = 0; j < 4; ++j) pp[j] = make_float4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
         }
       }
-      if (whole) continue;
+      if (whole || a.cluster_s > 1) continue;
       // split tile: publish the partial, the last contributor finishes it.
       // The group barrier orders the 128 threads' partial stores before thread
       // 0's release (acq_rel, gpu scope) on the tile counter; the last
       // arriver's acquire orders its reads of the others' partials after it.
+      // A counter holds (epoch << 32) | arrivals: a value left by another
+      // launch (another epoch) counts as zero arrivals, so the counters never
+      // need clearing.
       named_bar_sync(1, 128);
-      const int64_t c_first = owner_of(tile_first, T, G);
-      const int64_t c_last = owner_of(tile_first + KI - 1, T, G);
+      const int c_first = owner_of(tile_first, T, G);
+      const int c_last = owner_of(tile_first + KI - 1, T, G);
       if (t == 0) {
-        int ncontrib = 0;
-        for (int64_t c = c_first; c <= c_last; ++c)
+        unsigned ncontrib = 0;
+        for (int c = c_first; c <= c_last; ++c)
           if (range_begin(c + 1, T, G) > range_begin(c, T, G)) ++ncontrib;
-        int old;
-        asm volatile("atom.acq_rel.gpu.global.add.s32 %0, [%1], 1;" : "=r"(old) : "l"(&a.counters[tile]) : "memory");
-        sh.last_flag = (old == ncontrib - 1) ? 1 : 0;
+        unsigned long long* ctr = a.counters + tile;
+        const unsigned long long tag = static_cast<unsigned long long>(a.epoch) << 32;
+        unsigned long long cur = *reinterpret_cast<volatile unsigned long long*>(ctr), want = 0;
+        bool done = false;
+        for (int attempt = 0; attempt < (1 << 20) && !done; ++attempt) {
+          want = ((cur >> 32) == a.epoch) ? cur + 1 : (tag | 1ull);
+          unsigned long long prev;
+          asm volatile("atom.acq_rel.gpu.global.cas.b64 %0, [%1], %2, %3;"
+                       : "=l"(prev) : "l"(ctr), "l"(cur), "l"(want) : "memory");
+          done = (prev == cur);
+          cur = prev;
+        }
+        if (!done) raise_status(TQ_DEV_TIMEOUT);
+        sh.last_flag = (done && (want & 0xFFFFFFFFull) == ncontrib) ? 1 : 0;
       }
       named_bar_sync(1, 128);
       if (sh.last_flag) {
@@ -683,12 +846,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           float acc[16];
 #pragma unroll
           for (int j = 0; j < 16; ++j) acc[j] = 0.0f;
-          for (int64_t c = c_first; c <= c_last; ++c) {
-            const int64_t cb0 = range_begin(c, T, G);
+          for (int c = c_first; c <= c_last; ++c) {
+            const int cb0 = range_begin(c, T, G);
             if (range_begin(c + 1, T, G) <= cb0) continue;
             const int cslot = (cb0 / KI == tile) ? 0 : 1;
-            const float4* src =
-                reinterpret_cast<const float4*>(a.partials + ((c * 2 + cslot) * 128 + t) * kSegRows + 16 * ch);
+            const float4* src = reinterpret_cast<const float4*>(
+                a.partials + ((static_cast<int64_t>(c) * 2 + cslot) * 128 + t) * kSegRows + 16 * ch);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const float4 f = __ldcg(src + j);
@@ -698,9 +861,8 @@ __global__ void __launch_bounds__(kThreads, 1)
               acc[4 * j + 3] = __fadd_rn(acc[4 * j + 3], f.w);
             }
           }
-          epilogue_store(a, acc, 16 * ch, row, lane, sg);
+          epilogue_store(a, acc, 16 * ch, row, sg);
         }
-        if (t == 0) a.counters[tile] = 0;
       }
       named_bar_sync(1, 128);
     }
@@ -709,29 +871,114 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (a.cluster_s > 1) {
+    // Cluster split-K reduction.  Every thread of every CTA of the cluster
+    // reaches both barriers (on a timeout too: the roles above always run to
+    // their end), so neither can hang; the second keeps each CTA's buffer
+    // alive until the other CTAs have read it.
+    cluster_sync_all();
+    if (!sh.abort_flag) {
+      const int s_n = a.cluster_s;
+      const int rank = static_cast<int>(cluster_ctarank());
+      const int tile = tile_begin;   // one tile per CTA in this mode
+      const int rt = tile % a.row_tiles;
+      const Seg sg = get_seg(a, tile / a.row_tiles);
+      const int r0 = rank * 128 / s_n, r1 = (rank + 1) * 128 / s_n;
+      const int nrow = r1 - r0;
+      const uint32_t red = smem_u32(smem + kCodesBytes);
+      for (int idx = threadIdx.x; idx < nrow * sg.count; idx += kThreads) {
+        const int j = idx / nrow, rl = r0 + (idx - j * nrow);
+        const int row = rt * 128 + rl;
+        if (row >= a.n) continue;
+        float acc = 0.0f;
+        for (int q = 0; q < s_n; ++q)
+          acc = __fadd_rn(acc, ld_dsmem_f32(red + static_cast<uint32_t>((j * 128 + rl) * 4), static_cast<uint32_t>(q)));
+        a.out_a[static_cast<int64_t>(sg.row0 + j) * a.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+      }
+    }
+    cluster_sync_all();
+  }
+  // Dependents may launch once every CTA is done: a kernel that waits on this
+  // one gains nothing from taking an SM early, and its CTAs would only delay
+  // this kernel's CTAs that have not started yet.
+  if (threadIdx.x == 0) pdl_launch_dependents();
   if (warp == 1) tmem_dealloc(tmem, kTmemCols);
 }
 
 }  // namespace
 
-size_t streamk_smem_bytes() { return static_cast<size_t>(kStages) * kStageBytes + 1024; }
+uint32_t next_epoch() {
+  static std::atomic<uint32_t> epoch{0};
+  uint32_t e = epoch.fetch_add(1, std::memory_order_relaxed) + 1;
+  if (e == 0) e = epoch.fetch_add(1, std::memory_order_relaxed) + 1;   // 0 marks never-used counters
+  return e;
+}
+
+int choose_cluster_split(int64_t tiles, int64_t k_iters, int sms) {
+  static std::mutex mu;
+  static int cap[64][9];   // per device, per s: resident clusters (+1; 0 = not queried yet)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 1;
+  }
+  for (int s = 8; s >= 2; --s) {
+    if (s > k_iters || (k_iters + s - 1) / s > kFusedMaxIters || tiles * s > sms) continue;
+    int c;
+    {
+      std::lock_guard<std::mutex> g(mu);
+      if (cap[dev][s] == 0) cap[dev][s] = streamk_max_clusters(s) + 1;
+      c = cap[dev][s] - 1;
+    }
+    if (tiles <= c) return s;
+  }
+  return 1;
+}
+
+int streamk_max_clusters(int s) {
+  // clusters of s CTAs (one per SM) that can be resident at once
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(s));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = streamk_smem_bytes();
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(s);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaFuncSetAttribute(streamk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           static_cast<int>(streamk_smem_bytes())) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, streamk_kernel, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+size_t streamk_smem_bytes() { return static_cast<size_t>(kStages) * kStageBytes + kLutBytes + 1024; }
 
 cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void* tm_xlo, const StreamKArgs& a,
                            int grid, cudaStream_t st) {
   static bool attr_set = false;
   const size_t smem = streamk_smem_bytes();
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(streamk_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(streamk_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               static_cast<int>(smem));
+    cudaError_t e =
+        cudaFuncSetAttribute(streamk_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(streamk_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  Codemag cm;
+  LevelTable lt;
   const CodebookF32& cb = codebook();
-  for (int i = 0; i < 8; ++i) cm.v[i] = cb.levels[8 + i];
+  for (int i = 0; i < 16; ++i)
+    lt.h[i] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(cb.levels[i] * kLevelScale)));
+  lt.max_level = __half2float(__float2half_rn(cb.levels[15] * kLevelScale));
   const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
   const CUtensorMap& m1 = *static_cast<const CUtensorMap*>(tm_xhi);
   const CUtensorMap& m2 = *static_cast<const CUtensorMap*>(tm_xlo);
@@ -740,13 +987,19 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void*
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = st;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   attr[0].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  cudaError_t e = a.f16 ? cudaLaunchKernelEx(&cfg, streamk_kernel<true>, m0, m1, m2, a, cm)
-                        : cudaLaunchKernelEx(&cfg, streamk_kernel<false>, m0, m1, m2, a, cm);
+  if (a.cluster_s > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(a.cluster_s);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, streamk_kernel, m0, m1, m2, a, lt);
   if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();

@@ -69,7 +69,8 @@ enum {
 enum {
   TQ_DEV_TIMEOUT = 1,
   TQ_DEV_BAD_ROUTING = 2,
-  TQ_DEV_NONFINITE = 4
+  TQ_DEV_NONFINITE = 4,
+  TQ_DEV_SCALE_RANGE = 8   /* linear/moe: a half-block scale above ~93.6 (see tq4_1s_linear) */
 };
 
 /* Input dtypes of tq4_1s_quantize. */
@@ -123,13 +124,10 @@ int tq4_1s_dequantize(const tq4_1s_weight* w, float* W_out, tq4_stream_t stream)
 
 /* Bytes of workspace tq4_1s_linear needs for m rows with weight w (dense,
  * num_experts == 1).  0 on invalid arguments.
- * Small m (<= 128): the workspace holds stream-K partial sums and tile
- * counters; the counters must be zero when a call starts, and every call
- * leaves them zero again.  So zero-fill the workspace once, then use it only
- * for small-m tq4_1s_linear calls (any shapes, one call at a time); zero it
- * again after anything else wrote to it or after a call reported
- * TQ_DEV_TIMEOUT.  Large m: the workspace receives the bf16 dequantized
- * weight; no initialisation is needed. */
+ * Small m (<= 128): the workspace holds the rotated activations, the
+ * stream-K partial sums and the tile counters; large m: the bf16 dequantized
+ * weight.  No initialisation is needed (each call clears what it uses), but
+ * calls that share a workspace must not overlap on the GPU. */
 size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
 
 /* The quantized linear layer of "Running it": y[m][n] = bf16(x * W_hat^T),
@@ -137,13 +135,22 @@ size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
  *   x  device bf16 bits [m][k], row-major, 16-byte aligned;
  *   y  device bf16 bits [m][n], row-major, 16-byte aligned;
  *   ws device workspace of at least tq4_1s_linear_workspace(m, w) bytes,
- *      16-byte aligned, owned by the caller; for m <= 128 it must satisfy the
- *      zero-counter rule of tq4_1s_linear_workspace.
- * Small m (<= 128) is one kernel launch: it rotates each 32-slice of x
- * (x' = R x, split into bf16 hi + lo) and multiplies the rotated-domain levels
- * c[code]*d on the tensor cores with a stream-K split of the weight stream;
- * large m dequantizes W_hat to bf16 in the workspace and runs a tensor-core
- * GEMM.  m == 0 is a no-op. */
+ *      16-byte aligned, owned by the caller.
+ * Small m (<= 128) rotates each 32-slice of x by the weight's own RHT
+ * (x' = R x; R's orthogonality makes this equivalent to inverse-rotating W),
+ * scales each row by a power of two that keeps it inside the fp16 range,
+ * splits it into fp16 hi + lo, and multiplies the rotated-domain levels
+ * fp16(256 c[code]) * d (fp16 product) by x' on the tensor cores, streaming
+ * the packed weight once and scaling back exactly.  For m <= 32 with a short
+ * k range per CTA this is one kernel launch (the GEMM kernel rotates x
+ * itself; the CTAs sharing a row tile form a cluster and reduce their
+ * partial sums on chip); otherwise a rotation kernel writes x' to the
+ * workspace first and a stream-K kernel splits the weight stream evenly over
+ * the SMs.  Levels are finite for half-block scales d up to
+ * 65504 / fp16(256 c_max) (about 93.6); a larger scale sets
+ * TQ_DEV_SCALE_RANGE and makes the affected outputs non-finite.  Large m
+ * dequantizes W_hat to bf16 in the workspace and runs a tensor-core GEMM.
+ * m == 0 is a no-op. */
 int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, void* ws, size_t ws_bytes,
                   tq4_stream_t stream);
 
@@ -161,8 +168,8 @@ int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t
  *   that device current); make that first call outside any stream capture.
  *   All calls share the one array, so calls that overlap on the GPU (on
  *   different streams, or from different host threads) race and corrupt each
- *   other's results; serialize them.  Each call clears the counters it
- *   needs, so the previous call's leftovers do no harm.
+ *   other's results; serialize them.  Each launch tags the tile counters
+ *   it uses with its own epoch, so a previous call's leftovers do no harm.
  * Same arguments, result and numerics as tq4_1s_linear's small-m path; no
  * allocation of any kind. */
 int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, tq4_stream_t stream);

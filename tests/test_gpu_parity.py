@@ -97,6 +97,8 @@ LINEAR_CASES = [
     (33, 256, 256, 34),     # two segments, the second with one row
     (100, 640, 384, 35),    # four segments
     (16, 4096, 4096, 2),    # dense decode-block linear, full size
+    (16, 256, 8192, 36),    # wide k: four rotation warps per activation row
+    (8, 128, 16416, 37),    # wider k: eight rotation warps, lanes with 2-3 slices
     # large-m path (dequantize + GEMM)
     (129, 256, 256, 40),
     (300, 520, 224, 41),    # ragged m, n, k
@@ -116,10 +118,43 @@ def test_linear_parity(m, n, k, seed):
     assert tq.tq4_1s_get_status() == 0
 
 
+@pytest.mark.parametrize("x_std", [3000.0, 1e-5])
+def test_linear_activation_range(x_std):
+    # activations far outside (and far inside) the fp16 range: the per-row
+    # power-of-two scaling of the rotated activations keeps full precision
+    m, n, k, seed = 16, 384, 512, 38
+    W = synth.student_t_f32((n, k), seed, 5.0, 0.02)
+    x = synth.f32_to_bf16_bits(synth.student_t_f32((m, k), seed + 1, 5.0, x_std))
+    p, codes, scales, _ = _quantize_both(W, seed)
+    y = tq.tq4_1s_linear(_bf16_dev(x), p)
+    torch.cuda.synchronize()
+    assert np.all(np.isfinite(y.float().cpu().numpy()))
+    y_ref, _ = oracle.linear(x, codes[0], scales[0], seed)
+    assert_close(_bits(y), y_ref, f"linear range x_std={x_std}")
+    assert tq.tq4_1s_get_status() == 0
+
+
+def test_linear_scale_beyond_fp16_level_range_flagged():
+    # one weight row with half-block scales far above ~93.6: its fp16 levels
+    # overflow, the status word says so, and every other output column is
+    # still correct (accumulator rows are independent)
+    m, n, k, seed = 16, 256, 256, 39
+    W = synth.normal_f32((n, k), seed, 0.02)
+    W[3] *= 20000.0
+    x = synth.activations_bf16(m, k, seed + 1)
+    p, codes, scales, _ = _quantize_both(W, seed)
+    y = tq.tq4_1s_linear(_bf16_dev(x), p)
+    torch.cuda.synchronize()
+    assert tq.tq4_1s_get_status() & tq.TQ_DEV_SCALE_RANGE
+    y_ref, _ = oracle.linear(x, codes[0], scales[0], seed)
+    keep = np.array([c for c in range(n) if c != 3])
+    assert_close(_bits(y)[:, keep], y_ref[:, keep], "linear with one out-of-range row")
+
+
 def test_linear_shared_workspace_across_shapes_and_paths():
-    # one zero-filled workspace reused by small-m calls of different shapes
-    # (different tile counts) stays valid: each call leaves its counters zero;
-    # a large-m call in between uses the binding's separate large-m workspace
+    # one workspace reused by small-m calls of different shapes (different
+    # tile counts and activation sizes) stays valid: each call clears its own
+    # counters; a large-m call in between uses the binding's large-m workspace
     cases = [(16, 256, 256, 50), (16, 4096, 1024, 51), (300, 520, 224, 52), (8, 1000, 544, 53), (16, 256, 256, 50)]
     ws = None
     for m, n, k, seed in cases:
@@ -129,7 +164,7 @@ def test_linear_shared_workspace_across_shapes_and_paths():
         if m <= 128:
             need = tq.tq4_1s_linear_workspace(m, p)
             if ws is None or ws.numel() < need:
-                ws = torch.zeros(4 << 20 if need < (4 << 20) else need, dtype=torch.uint8, device=DEV)
+                ws = torch.full((max(need, 4 << 20),), 0x5A, dtype=torch.uint8, device=DEV)   # not zeroed
             y = tq.tq4_1s_linear(_bf16_dev(x), p, workspace=ws)
         else:
             y = tq.tq4_1s_linear(_bf16_dev(x), p)
