@@ -182,13 +182,13 @@ static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 constexpr int64_t kSmallM = 128;
 
 struct SmallLayout {
-  size_t xh, xl, xscale, partials, counters, total;
+  size_t xr, xscale, partials, counters, total;
   int grid;
   int64_t tiles;
 };
 
-// Small-m workspace: the rotated activations (fp16 hi and lo planes, per-row
-// scales; unused when the kernel rotates x itself), the stream-K fp32
+// Small-m workspace: the rotated activations (fp16, per-row scales; unused
+// when the kernel rotates x itself), the stream-K fp32
 // partials and the tile counters.  Counters carry the launch's epoch, so the
 // workspace needs no initialisation.
 static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
@@ -204,8 +204,7 @@ static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
     off = align256(off + bytes);
     return at;
   };
-  L.xh = take(static_cast<size_t>(m * w->k) * 2);
-  L.xl = take(static_cast<size_t>(m * w->k) * 2);
+  L.xr = take(static_cast<size_t>(m * w->k) * 2);
   L.xscale = take(static_cast<size_t>(m) * 4);
   L.partials = take(static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
   L.counters = take(static_cast<size_t>(L.tiles) * 8);
@@ -220,7 +219,7 @@ static bool small_fused(int64_t m, int64_t tiles_times_ki, int grid) {
 }
 
 struct MoeLayout {
-  size_t offsets, pairs, segs, nseg, npv, xh, xl, xscale, h, hh, hl, hscale, zw, partials, cnt_up, cnt_dn, total;
+  size_t offsets, pairs, segs, nseg, npv, xr, xscale, h, hr, hscale, zw, partials, cnt_up, cnt_dn, total;
   int64_t P, maxseg, rt_up, rt_dn;
 };
 
@@ -243,12 +242,10 @@ static MoeLayout moe_layout(int64_t m, int32_t topk, const tq4_1s_weight* up, co
   L.segs = take(L.maxseg * 16);
   L.nseg = take(4);
   L.npv = take(4);
-  L.xh = take(L.P * H * 2);
-  L.xl = take(L.P * H * 2);
+  L.xr = take(L.P * H * 2);
   L.xscale = take(L.P * 4);
   L.h = take(L.P * I * 2);
-  L.hh = take(L.P * I * 2);
-  L.hl = take(L.P * I * 2);
+  L.hr = take(L.P * I * 2);
   L.hscale = take(L.P * 4);
   L.zw = take(L.P * H * 4);
   L.partials = take(static_cast<size_t>(sms) * 2 * 128 * kSegRows * 4);
@@ -366,15 +363,13 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     const int split = m <= kSegRows ? choose_cluster_split(L.tiles, KI, sms) : 1;
     const int grid = split > 1 ? static_cast<int>(L.tiles * split) : L.grid;
     const bool fused = split > 1 || small_fused(m, T, L.grid);
-    uint16_t* xh = reinterpret_cast<uint16_t*>(base + L.xh);
-    uint16_t* xl = reinterpret_cast<uint16_t*>(base + L.xl);
+    uint16_t* xr = reinterpret_cast<uint16_t*>(base + L.xr);
     float* xscale = reinterpret_cast<float*>(base + L.xscale);
-    // TMA-fed mode: x' = R x (fp16 hi/lo, per-row scale) by the rotation kernel
-    if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xh, xl, xscale, mask, st) != cudaSuccess)
+    // TMA-fed mode: x' = R x (fp16, per-row scale) by the rotation kernel
+    if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xr, xscale, mask, st) != cudaSuccess)
       return TQ_ERR_CUDA;
-    alignas(64) CUtensorMap tc, th, tl;
-    if (!map_codes(&tc, w) || !map_bf16(&th, xh, m, w->k, 16) || !map_bf16(&tl, xl, m, w->k, 16))
-      return TQ_ERR_CUDA;
+    alignas(64) CUtensorMap tc, tx;
+    if (!map_codes(&tc, w) || !map_bf16(&tx, xr, m, w->k, 16)) return TQ_ERR_CUDA;
     StreamKArgs a{};
     a.n = static_cast<int32_t>(w->n);
     a.k = static_cast<int32_t>(w->k);
@@ -396,7 +391,7 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     a.partials = reinterpret_cast<float*>(base + L.partials);
     a.counters = reinterpret_cast<unsigned long long*>(base + L.counters);
     a.max_tiles = static_cast<int32_t>(L.tiles);
-    return cuda_rc(launch_streamk(&tc, &th, &tl, a, grid, st));
+    return cuda_rc(launch_streamk(&tc, &tx, a, grid, st));
   }
   // large m: W_hat in bf16, then the tensor-core GEMM
   uint16_t* wh = reinterpret_cast<uint16_t*>(base);
@@ -452,10 +447,8 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   int4* segs = reinterpret_cast<int4*>(base + L.segs);
   int32_t* nseg = reinterpret_cast<int32_t*>(base + L.nseg);
   int32_t* npv = reinterpret_cast<int32_t*>(base + L.npv);
-  uint16_t* xh = reinterpret_cast<uint16_t*>(base + L.xh);
-  uint16_t* xl = reinterpret_cast<uint16_t*>(base + L.xl);
-  uint16_t* hh = reinterpret_cast<uint16_t*>(base + L.hh);
-  uint16_t* hl = reinterpret_cast<uint16_t*>(base + L.hl);
+  uint16_t* xr = reinterpret_cast<uint16_t*>(base + L.xr);
+  uint16_t* hr = reinterpret_cast<uint16_t*>(base + L.hr);
   float* zw = reinterpret_cast<float*>(base + L.zw);
   cudaError_t e = launch_moe_route(topk_ids, L.P, static_cast<int32_t>(E), offsets, pairs, segs, nseg, kSegRows,
                                    npv, nullptr, 0, st);
@@ -465,12 +458,12 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   float* hscale = reinterpret_cast<float*>(base + L.hscale);
   // x' of each sorted pair row (x row pairs[r] / topk), rotated by the up
   // projection's signs
-  e = launch_rotate_scaled(x, H, pairs, topk, npv, 0, L.P, xh, xl, xscale, sign_mask_of(up->seed), st);
+  e = launch_rotate_scaled(x, H, pairs, topk, npv, 0, L.P, xr, xscale, sign_mask_of(up->seed), st);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
 
-  alignas(64) CUtensorMap tcu, txh, txl, tcd, thh, thl;
-  if (!map_codes(&tcu, up) || !map_bf16(&txh, xh, L.P, H, 16) || !map_bf16(&txl, xl, L.P, H, 16) ||
-      !map_codes(&tcd, down) || !map_bf16(&thh, hh, L.P, I, 16) || !map_bf16(&thl, hl, L.P, I, 16))
+  alignas(64) CUtensorMap tcu, txr, tcd, thr;
+  if (!map_codes(&tcu, up) || !map_bf16(&txr, xr, L.P, H, 16) || !map_codes(&tcd, down) ||
+      !map_bf16(&thr, hr, L.P, I, 16))
     return TQ_ERR_CUDA;
   StreamKArgs a{};
   a.n = static_cast<int32_t>(I);
@@ -489,10 +482,10 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   a.partials = reinterpret_cast<float*>(base + L.partials);
   a.counters = reinterpret_cast<unsigned long long*>(base + L.cnt_up);
   a.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_up);
-  if ((e = launch_streamk(&tcu, &txh, &txl, a, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
+  if ((e = launch_streamk(&tcu, &txr, a, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
 
   // h' = R_down h per sorted pair row
-  e = launch_rotate_scaled(h, I, nullptr, 1, npv, 0, L.P, hh, hl, hscale, sign_mask_of(down->seed), st);
+  e = launch_rotate_scaled(h, I, nullptr, 1, npv, 0, L.P, hr, hscale, sign_mask_of(down->seed), st);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   StreamKArgs b = a;
   b.n = static_cast<int32_t>(H);
@@ -509,7 +502,7 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   b.topk_w = topk_w;
   b.counters = reinterpret_cast<unsigned long long*>(base + L.cnt_dn);
   b.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_dn);
-  if ((e = launch_streamk(&tcd, &thh, &thl, b, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
+  if ((e = launch_streamk(&tcd, &thr, b, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
   return cuda_rc(launch_moe_combine(zw, topk_ids, m, topk, H, static_cast<int32_t>(E), y, st));
 }
 

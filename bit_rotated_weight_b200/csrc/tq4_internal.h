@@ -30,14 +30,14 @@ cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, 
 cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales, uint16_t* out, int64_t rows,
                                    int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st);
 // Activation rotation for the stream-K GEMM: x' = r H diag(s) x per 32-slice
-// of each row, scaled by a per-row power of two 2^-e and split into fp16
-// hi/lo planes [rows][k]; row_scale[row] = 2^e.  Row r reads x row
+// of each row, scaled by a per-row power of two 2^-e and rounded to fp16
+// [rows][k]; row_scale[row] = 2^e.  Row r reads x row
 // gather[r] / topk when a gather list is given, else row r.  Rows at or past
 // the valid count (rows_valid_dev when non-null, else rows_valid_host) are
 // not written.
 cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
                                  const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
-                                 uint16_t* xh, uint16_t* xl, float* row_scale, uint32_t mask, cudaStream_t st);
+                                 uint16_t* xr, float* row_scale, uint32_t mask, cudaStream_t st);
 cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
                              int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
                              int32_t* zero_ptr, int64_t nzero, cudaStream_t st);
@@ -91,8 +91,7 @@ int streamk_max_clusters(int s);
 // resident at once; 1 if none fits.
 int choose_cluster_split(int64_t tiles, int64_t k_iters, int sms);
 
-cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void* tm_xlo, const StreamKArgs& a,
-                           int grid, cudaStream_t st);
+cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const StreamKArgs& a, int grid, cudaStream_t st);
 
 // ---------------------------------------------------------------- GEMM
 // y[m][n] = bf16( x[m][k] * w[n][k]^T ), bf16 operands via TMA tensor maps.

@@ -197,15 +197,14 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
 // equivalent because R is orthogonal).  Each row is scaled by 2^-e, where e
 // puts the largest value x' can take, sqrt(32) * max|x| (each x'_i is r times
 // a signed sum of 32 entries), in [2^13, 2^14): the row then uses the full
-// fp16 precision and cannot overflow.  Split into fp16 hi = f16(x' 2^-e) and
-// lo = f16(x' 2^-e - hi); row_scale[row] = 2^e (exact) undoes the scaling in
-// the GEMM epilogue.
+// fp16 precision and cannot overflow; the result is rounded to fp16, and
+// row_scale[row] = 2^e (exact) undoes the scaling in the GEMM epilogue.
 //
 // One CTA of four warps per row; lane i of a warp holds element i of a
 // slice, and the 32-point butterfly runs across the warp through shfl_xor
 // (stage h exchanges lanes i and i^h: the lane with bit h clear keeps
 // a + partner, the other partner - a), the same order as the one-thread form.
-// First pass: the row maximum; second pass (L1 hits): rotate, scale, split.
+// First pass: the row maximum; second pass (L1 hits): rotate, scale, round.
 // The CTA is small (128 threads, at most 48 registers each, no shared
 // arrays) so that it fits on an SM beside a running stream-K CTA.
 constexpr int kRotThreads = 128;
@@ -222,8 +221,7 @@ __device__ __forceinline__ float warp_fwht32(float a, int lane) {
 __global__ void __launch_bounds__(kRotThreads, 10)
     rotate_scaled_kernel(const uint16_t* __restrict__ x, int64_t k, const int32_t* __restrict__ gather,
                          int32_t topk, const int32_t* __restrict__ rows_valid_dev, int64_t rows_valid_host,
-                         uint16_t* __restrict__ xh, uint16_t* __restrict__ xl, float* __restrict__ row_scale,
-                         uint32_t mask) {
+                         uint16_t* __restrict__ xr_out, float* __restrict__ row_scale, uint32_t mask) {
   __shared__ float s_max[kRotThreads / 32];
   // x, the gather list and the valid count may be the previous kernel's
   // output.  Dependents may start once every CTA is past this wait: nothing
@@ -269,15 +267,11 @@ __global__ void __launch_bounds__(kRotThreads, 10)
   if (threadIdx.x == 0) row_scale[row] = ldexpf(1.0f, e);
   const float rd = __fmul_rn(rsqrt32(), ldexpf(1.0f, -e));   // exact: r times a power of two
   const bool neg = (mask >> lane) & 1u;
-  uint16_t* oh = xh + row * k + lane;
-  uint16_t* ol = xl + row * k + lane;
+  uint16_t* oh = xr_out + row * k + lane;
   auto emit = [&](int64_t sl, uint16_t raw) {
     const float xv = bf16_bits_to_f32(raw);
     const float v = __fmul_rn(warp_fwht32(neg ? -xv : xv, lane), rd);
-    const __half h = __float2half_rn(v);
-    const __half l = __float2half_rn(__fsub_rn(v, __half2float(h)));
-    oh[sl * 32] = __half_as_ushort(h);
-    ol[sl * 32] = __half_as_ushort(l);
+    oh[sl * 32] = __half_as_ushort(__float2half_rn(v));
   };
   int64_t sl = warp;
   for (; sl + 3 * kWarps < nsl; sl += 4 * kWarps) {
@@ -456,7 +450,7 @@ cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales,
 
 cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
                                  const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
-                                 uint16_t* xh, uint16_t* xl, float* row_scale, uint32_t mask, cudaStream_t st) {
+                                 uint16_t* xr, float* row_scale, uint32_t mask, cudaStream_t st) {
   if (rows_alloc <= 0) return cudaSuccess;
   static bool attr_set = false;
   if (!attr_set) {
@@ -477,7 +471,7 @@ cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* ga
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, rotate_scaled_kernel, x, k, gather, topk, rows_valid_dev,
-                                           rows_valid_host, xh, xl, row_scale, mask);
+                                           rows_valid_host, xr, row_scale, mask);
   if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();

@@ -27,12 +27,12 @@ constexpr int64_t kStaticMaxM = 32;
 constexpr int64_t kStaticMaxK = 8192;
 constexpr int64_t kStaticMaxN = 32768;
 constexpr int kStaticMaxGrid = 148;
-constexpr size_t kStaticXBytes = static_cast<size_t>(kStaticMaxM * kStaticMaxK) * 2;   // x' hi (or lo)
+constexpr size_t kStaticXBytes = static_cast<size_t>(kStaticMaxM * kStaticMaxK) * 2;   // x' (fp16)
 constexpr size_t kStaticPartialBytes = static_cast<size_t>(kStaticMaxGrid) * 2 * 128 * kSegRows * 4;
 constexpr size_t kStaticScaleBytes = 256;                                              // x' row scales
 constexpr size_t kStaticCounterBytes = static_cast<size_t>(kStaticMaxN / 128) * 8;
 constexpr size_t kStaticScratchBytes =
-    2 * kStaticXBytes + kStaticScaleBytes + kStaticPartialBytes + kStaticCounterBytes;   // ~5.6 MiB
+    kStaticXBytes + kStaticScaleBytes + kStaticPartialBytes + kStaticCounterBytes;   // ~5.2 MiB
 
 // The scratch itself.  In host code this name is only a stand-in for the
 // device symbol: its device address must be fetched with cudaGetSymbolAddress.
@@ -91,12 +91,11 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   if (rc) return rc;
 
   uint8_t* base = static_cast<uint8_t*>(scratch);
-  uint16_t* xh = reinterpret_cast<uint16_t*>(base);
-  uint16_t* xl = reinterpret_cast<uint16_t*>(base + kStaticXBytes);
-  float* xscale = reinterpret_cast<float*>(base + 2 * kStaticXBytes);
-  float* partials = reinterpret_cast<float*>(base + 2 * kStaticXBytes + kStaticScaleBytes);
+  uint16_t* xr = reinterpret_cast<uint16_t*>(base);
+  float* xscale = reinterpret_cast<float*>(base + kStaticXBytes);
+  float* partials = reinterpret_cast<float*>(base + kStaticXBytes + kStaticScaleBytes);
   unsigned long long* counters =
-      reinterpret_cast<unsigned long long*>(base + 2 * kStaticXBytes + kStaticScaleBytes + kStaticPartialBytes);
+      reinterpret_cast<unsigned long long*>(base + kStaticXBytes + kStaticScaleBytes + kStaticPartialBytes);
   const int64_t row_tiles = (w->n + 127) / 128, k_iters = (w->k + 127) / 128;
   const int64_t tiles = row_tiles;   // m <= 32: one segment
   const int64_t T = tiles * k_iters;
@@ -113,12 +112,12 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   const int split = choose_cluster_split(tiles, k_iters, sms < kStaticMaxGrid ? sms : kStaticMaxGrid);
   if (split > 1) grid = static_cast<int>(tiles * split);
   const bool fused = split > 1 || (T + grid - 1) / grid <= kFusedMaxIters;
-  if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xh, xl, xscale, mask, st) != cudaSuccess)
+  if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xr, xscale, mask, st) != cudaSuccess)
     return TQ_ERR_CUDA;
-  alignas(64) CUtensorMap tc, th, tl;
+  alignas(64) CUtensorMap tc, tx;
   {
     // same tensor maps as tq4_1s_linear: codes [1][n][k/2] (64 B x 128 rows),
-    // x' hi/lo [m][k] (64 x 16)
+    // x' [m][k] (64 x 16)
     typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -144,10 +143,7 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
     if (fn(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, cd, cs, cb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
             CUDA_SUCCESS ||
-        fn(&th, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xh, xd, xs, xb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-            CUDA_SUCCESS ||
-        fn(&tl, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xl, xd, xs, xb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        fn(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xr, xd, xs, xb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
             CUDA_SUCCESS)
       return TQ_ERR_CUDA;
@@ -173,5 +169,5 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   a.partials = partials;
   a.counters = counters;
   a.max_tiles = static_cast<int32_t>(tiles);
-  return launch_streamk(&tc, &th, &tl, a, grid, st) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  return launch_streamk(&tc, &tx, a, grid, st) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

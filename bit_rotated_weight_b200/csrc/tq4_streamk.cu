@@ -6,9 +6,11 @@
 // ("What Config-I means": 16-level Lloyd-Max codes, two half-block scales)
 // and x' = R x is the activation rotated per 32-slice (route B: rotating the
 // activations instead of inverse-rotating the weights, which is equivalent
-// because R is orthogonal).  x' is fp16 hi + lo, each row scaled by a power
-// of two 2^-e; the levels are fp16(c[code] * 256 * d).  Both operands fp16,
-// fp32 accumulation; the epilogue multiplies by 2^e / 256, which is exact.
+// because R is orthogonal).  x' is fp16, each row scaled by a power of two
+// 2^-e that puts its largest possible value in [2^13, 2^14); the levels are
+// fp16(c[code] * 256 * d).  Both operands fp16 (relative rounding 2^-11,
+// well inside the layer's tolerance), fp32 accumulation; the epilogue
+// multiplies by 2^e / 256, which is exact.
 //
 // x' comes from one of two places.  TMA-fed mode: the rotation kernel wrote
 // it to global memory (row_scale = 2^e per row) and the producer stages it
@@ -21,8 +23,8 @@
 //
 // Per 128-row x 128-k iteration of a tile:
 //   warp 0      TMA: codes tile [128 x 64 B] (64-byte swizzle) and, in
-//               TMA-fed mode, the x' hi/lo tiles [rows x 128 k] (128-byte
-//               swizzle) into a stage;
+//               TMA-fed mode, the x' tiles [rows x 128 k] (128-byte swizzle)
+//               into a stage;
 //   warps 2-17  four dequant warpgroups (round-robin iterations), thread =
 //               weight row: 16 B of codes + 8 scales -> 128 levels.  Each
 //               code byte (two nibbles) indexes a shared-memory table of
@@ -31,13 +33,13 @@
 //               by {d, d} scales the pair.  The levels go to tensor memory
 //               with tcgen05.st (the MMA A operand), as two 64-k halves
 //               signalled separately;
-//   warp 1, 22  lane 0: MMA issuers (groups 0-1 / 2-3): 4 tcgen05.mma per
-//               half (M=128, N=32*nb, K=16, A from tensor memory, B from
-//               shared memory) into the group's own accumulator -- single-
-//               thread issue costs ~66-98 cycles per small-N instruction, so
-//               two issuers and four accumulators keep the tensor core fed;
-//   warps 18-21 epilogue, thread = row: tcgen05.ld of the accumulators,
-//               hi + lo and the groups summed, scaled back, the mode's store.
+//   warps 1, 22-24  lane 0: one MMA issuer per dequant group: 4 tcgen05.mma
+//               per half (M=128, N=16*nb, K=16, A from tensor memory, B from
+//               shared memory) into the group's own accumulator --
+//               single-thread issue costs ~66-98 cycles per small-N
+//               instruction, so the four groups issue in parallel;
+//   warps 18-21 epilogue, thread = row: tcgen05.ld of the accumulators, the
+//               groups summed, scaled back, the mode's store.
 // The flattened (segment, row tile, k iteration) space is split evenly over
 // the CTAs (stream-K).  A tile split between CTAs is finished by whichever
 // contributor arrives last on the tile's counter: it sums all contributors'
@@ -59,24 +61,25 @@ namespace {
 constexpr int kDequantGroups = 4;
 constexpr int kFirstDequantWarp = 2;
 constexpr int kFirstEpilogueWarp = kFirstDequantWarp + 4 * kDequantGroups;
-// Two MMA-issuing threads: lane 0 of warp 1 serves dequant groups 0 and 1,
-// lane 0 of the last warp (22) groups 2 and 3.
-constexpr int kIssuerWarpB = kFirstEpilogueWarp + 4;
-constexpr int kThreads = (kIssuerWarpB + 1) * 32;
+// MMA-issuing threads: lane 0 of warp 1 serves dequant group 0, lane 0 of
+// warps 22, 23, 24 groups 1, 2, 3 (the four land on four different SMSPs).
+constexpr int kFirstIssuerWarp = kFirstEpilogueWarp + 4;
+constexpr int kThreads = (kFirstIssuerWarp + kDequantGroups - 1) * 32;
+__device__ __forceinline__ int issuer_group(int warp) { return warp == 1 ? 0 : warp - kFirstIssuerWarp + 1; }
 // fused mode: the dequant and epilogue warps rotate x before their own work
 constexpr int kPrologueThreads = (kFirstEpilogueWarp + 4 - kFirstDequantWarp) * 32;
-constexpr int kStages = 8;
+constexpr int kStages = 12;
 constexpr int kCodesBytes = 128 * 64;    // 128 rows x 128 k codes
-constexpr int kXHalfBytes = 64 * 128;    // 64 rows x 64 k of fp16 x' (one 128-B swizzle span)
+constexpr int kXHalfBytes = kSegRows * 128;   // up to 32 token rows x 64 k of fp16 x' (128-B swizzle span)
 constexpr int kXBytes = 2 * kXHalfBytes; // two k-halves
 constexpr int kStageBytes = kCodesBytes + kXBytes;
 constexpr int kLutBytes = 256 * 32 * 4;  // fp16 level-pair table, one copy per lane
 constexpr int kTmemCols = 512;
 // Tensor memory: columns [0, 256) hold the accumulators, [256, 512) the four
 // A stages (one per dequant group, 64 columns = 128 k of fp16 levels).  With
-// nb = 1 (<= 16 tokens per segment) the four group accumulators take 128
-// columns and two accumulator sets alternate between tile portions; with
-// nb = 2 one set of 256 columns.
+// 16 nb columns per group accumulator (nb = 16-token blocks per segment),
+// so 64 nb columns per set of four, and 256 / (64 nb) sets (4 or 2)
+// rotate between tile portions.
 constexpr int kAccRegion = 256;
 constexpr int kACol0 = kAccRegion;
 constexpr int kAColsPerStage = 64;
@@ -92,9 +95,9 @@ struct SharedState {
   uint64_t done[kStages];      // the MMAs of the iteration that used this stage completed
   uint64_t afull[kDequantGroups][2];   // a half A stage (64 k) holds fresh levels (128 arrivals)
   uint64_t afree[kDequantGroups][2];   // the MMAs reading a half A stage completed
-  uint64_t dfull[2];           // all four groups finished a portion (4 arrivals)
-  uint64_t dempty[2];          // the epilogue drained an accumulator set (128 arrivals)
-  uint64_t issuer_done[2];
+  uint64_t dfull[4];           // all four groups finished a portion (4 arrivals), per set
+  uint64_t dempty[4];          // the epilogue drained an accumulator set (128 arrivals)
+  uint64_t issuer_done[kDequantGroups];
   uint64_t xready;             // fused mode: every stage's x' tile is written (one arrival per prologue warp)
   uint64_t xissued;            // fused mode: the prologue's global reads are issued (one arrival per prologue warp)
   float row_scale[kSegRows];   // fused mode: 2^e of each row
@@ -263,8 +266,8 @@ struct LevelTable {
 };
 
 __global__ void __launch_bounds__(kThreads, 1)
-    streamk_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_xhi,
-                   const __grid_constant__ CUtensorMap tm_xlo, const StreamKArgs a,
+    streamk_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
+                   const StreamKArgs a,
                    const __grid_constant__ LevelTable lt) {
   __shared__ SharedState sh;
   extern __shared__ uint8_t dyn_smem[];
@@ -293,8 +296,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   const bool fused = a.x_raw != nullptr;
   // accumulator layout (see kAccRegion): width per group, number of sets
-  const int acc_w = 32 * a.nb_max;
-  const int nsets = (a.nb_max == 1) ? 2 : 1;
+  const int acc_w = 16 * a.nb_max;
+  const int nsets = kAccRegion / (kDequantGroups * acc_w);
   const int tile_begin = it_begin / KI, tile_last = (it_end - 1) / KI;
   const int nportions = tile_last - tile_begin + 1;
 
@@ -308,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sh.afull[i][h], 128);
         mbar_init(&sh.afree[i][h], 1);
       }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < 4; ++i) {
       mbar_init(&sh.dfull[i], kDequantGroups);
       mbar_init(&sh.dempty[i], 128);
       mbar_init(&sh.issuer_done[i], 1);
@@ -332,8 +335,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0 && lane == 0) {
     tma_prefetch_desc(&tm_codes);
     if (!fused) {
-      tma_prefetch_desc(&tm_xhi);
-      tma_prefetch_desc(&tm_xlo);
+      tma_prefetch_desc(&tm_x);
     }
   }
   if (warp == 1) {
@@ -387,12 +389,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     // values of row j at k = 128 kit(li) + 32 sl; a thread takes units ptid
     // and ptid + kPrologueThreads and keeps their x in registers.  Pass 1
     // takes each row's max |x| over the units; pass 2 applies the signs, the
-    // butterfly and r 2^-e, splits into fp16 hi/lo and writes them into stage
-    // li's B tile: hi in row j, lo in row 16 nb + j, 16-byte chunk c of a
-    // 128-byte row at chunk c ^ (row & 7) (128-byte swizzle).  The exponent e
-    // puts sqrt(32) max|x|, the bound on |x'|, in [2^13, 2^14).
+    // butterfly and r 2^-e, rounds to fp16 and writes row j of stage li's B
+    // tile, 16-byte chunk c of a 128-byte row at chunk c ^ (j & 7) (128-byte
+    // swizzle).  The exponent e puts sqrt(32) max|x|, the bound on |x'|, in
+    // [2^13, 2^14).
     const int ptid = threadIdx.x - kFirstDequantWarp * 32;
-    const int m = a.m_host, nb = (m + 15) >> 4;
+    const int m = a.m_host;
     const int units = cnt * 4 * m;   // <= kFusedMaxIters * 4 * kSegRows = 2 * kPrologueThreads
     static_assert(kFusedMaxIters * 4 * kSegRows <= 2 * kPrologueThreads, "two units per prologue thread");
     uint32_t raw[2][16];   // the thread's units of x, bf16 pairs, kept for pass 2
@@ -464,20 +466,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint8_t* hbase = smem + li * kStageBytes + kCodesBytes + (sl >> 1) * kXHalfBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
-        uint32_t hw[4], lw[4];
+        uint32_t hw[4];
 #pragma unroll
         for (int c2 = 0; c2 < 4; ++c2) {
-          const float f0 = __fmul_rn(v[8 * q + 2 * c2], rd), f1 = __fmul_rn(v[8 * q + 2 * c2 + 1], rd);
-          const __half h0 = __float2half_rn(f0), h1 = __float2half_rn(f1);
-          const __half l0 = __float2half_rn(__fsub_rn(f0, __half2float(h0)));
-          const __half l1 = __float2half_rn(__fsub_rn(f1, __half2float(h1)));
-          hw[c2] = static_cast<uint32_t>(__half_as_ushort(h0)) | (static_cast<uint32_t>(__half_as_ushort(h1)) << 16);
-          lw[c2] = static_cast<uint32_t>(__half_as_ushort(l0)) | (static_cast<uint32_t>(__half_as_ushort(l1)) << 16);
+          const __half2 h = __floats2half2_rn(__fmul_rn(v[8 * q + 2 * c2], rd), __fmul_rn(v[8 * q + 2 * c2 + 1], rd));
+          hw[c2] = *reinterpret_cast<const uint32_t*>(&h);
         }
         const int c = (sl & 1) * 4 + q;
-        const int rh = j, rl = 16 * nb + j;
-        *reinterpret_cast<uint4*>(hbase + rh * 128 + ((c ^ (rh & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-        *reinterpret_cast<uint4*>(hbase + rl * 128 + ((c ^ (rl & 7)) << 4)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        *reinterpret_cast<uint4*>(hbase + j * 128 + ((c ^ (j & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       }
     }
     fence_proxy_async_smem();   // the generic-proxy writes, before the tensor core reads them
@@ -494,11 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       auto load_x = [&](uint8_t* st, int kit, const Seg& sg, int nb, uint64_t* bar) {
         for (int b = 0; b < nb; ++b) {
 #pragma unroll
-          for (int kh = 0; kh < 2; ++kh) {
-            uint8_t* xb = st + kCodesBytes + kh * kXHalfBytes;
-            tma_load_2d(xb + (16 * b) * 128, &tm_xhi, bar, kit * 128 + 64 * kh, sg.row0 + 16 * b);
-            tma_load_2d(xb + (16 * nb + 16 * b) * 128, &tm_xlo, bar, kit * 128 + 64 * kh, sg.row0 + 16 * b);
-          }
+          for (int kh = 0; kh < 2; ++kh)
+            tma_load_2d(st + kCodesBytes + kh * kXHalfBytes + (16 * b) * 128, &tm_x, bar, kit * 128 + 64 * kh,
+                        sg.row0 + 16 * b);
         }
       };
       // TMA-fed mode: the codes of the first stages go out before the
@@ -513,7 +507,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_wait(&sh.xissued, 0, abortp);
       }
       const int npre = cnt < kStages ? cnt : kStages;
-      const uint32_t xbytes = fused ? 0u : 4u * 2048u;
+      const uint32_t xbytes = fused ? 0u : 2u * 2048u;   // per 16-row block: two k-halves of 16 x 128 B
       Cursor cur;
       cur.init(it_begin, KI, a.row_tiles);
       const Cursor first = cur;
@@ -651,16 +645,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     // a scale whose largest level overflows fp16 made some levels infinite
     const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
     if (fmaxf(dm.x, dm.y) * lt.max_level >= 65520.0f) raise_status(TQ_DEV_SCALE_RANGE);
-  } else if ((warp == 1 || warp == kIssuerWarpB) && lane == 0) {
+  } else if ((warp == 1 || warp >= kFirstIssuerWarp) && lane == 0) {
     // ------------------------------------------------------------ MMA issue
-    // Issuer A (warp 1) serves groups 0-1, issuer B groups 2-3: the
-    // iterations li with li % 4 in {gb, gb + 1}, in order.  Per half A stage:
-    // wait until the group filled it, issue 4 MMAs (K = 16) into the group's
-    // accumulator, commit to the half's `afree`; after the second half commit
-    // to the stage's `done`; at the end of a portion commit to `dfull`.
-    const int gb = (warp == 1) ? 0 : 2;
-    const int ib = (warp == 1) ? 0 : 1;
-    int use0 = 0, use1 = 0;   // fills of group gb / gb + 1 consumed so far
+    // Issuer of group w: the iterations li = w (mod 4), in order.  Per half A
+    // stage: wait until the group filled it, issue 4 MMAs (K = 16) into the
+    // group's accumulator, commit to the half's `afree`; after the second
+    // half commit to the stage's `done`; at the end of a portion commit (or,
+    // with no iteration in it, arrive) on `dfull`.
+    const int w = issuer_group(warp);
+    int use = 0;   // fills of the group's A stage consumed so far
     bool ok = !fused || mbar_wait(&sh.xready, 0, abortp);   // fused mode: the B tiles are written
     for (int pi = 0; pi < nportions && ok; ++pi) {
       const int tile = tile_begin + pi;
@@ -675,17 +668,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const Seg sg = get_seg(a, tile / a.row_tiles);
       const int nb = (sg.count + 15) >> 4;
-      const uint32_t idesc = idesc_f16(128, 32 * nb);
-      bool started0 = false, started1 = false;
-      for (int li = pf; li < pe && ok; ++li) {
-        const int w = li % kDequantGroups;
-        if (w != gb && w != gb + 1) continue;
-        const bool second = (w != gb);
-        const int use = second ? use1 : use0;
-        const bool started = second ? started1 : started0;
+      const uint32_t idesc = idesc_f16(128, 16 * nb);
+      const uint32_t acc = tmem + db * (kAccRegion / nsets) + w * acc_w;
+      const uint32_t a_stage = tmem + kACol0 + w * kAColsPerStage;
+      bool started = false;
+      // first local iteration of this portion that belongs to group w
+      for (int li = pf + ((w - pf) % kDequantGroups + kDequantGroups) % kDequantGroups; li < pe && ok;
+           li += kDequantGroups) {
         const int s = li % kStages;
-        const uint32_t acc = tmem + db * (kAccRegion / nsets) + w * acc_w;
-        const uint32_t a_stage = tmem + kACol0 + w * kAColsPerStage;
         const uint32_t xb = smem_u32(smem + s * kStageBytes + kCodesBytes);
         // the B tile (x') of this stage must have landed too
         if (!mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) {
@@ -709,22 +699,15 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (!ok) break;
         mma_commit(&sh.done[s]);
-        if (second) {
-          started1 = true;
-          ++use1;
-        } else {
-          started0 = true;
-          ++use0;
-        }
+        started = true;
+        ++use;
       }
       if (!ok) break;
-      if (started0) mma_commit(&sh.dfull[db]);
-      else mbar_arrive(&sh.dfull[db]);
-      if (started1) mma_commit(&sh.dfull[db]);
+      if (started) mma_commit(&sh.dfull[db]);
       else mbar_arrive(&sh.dfull[db]);
     }
-    mma_commit(&sh.issuer_done[ib]);
-    drain_wait(&sh.issuer_done[ib], 0);
+    mma_commit(&sh.issuer_done[w]);
+    drain_wait(&sh.issuer_done[w], 0);
   } else if (warp >= kFirstEpilogueWarp && warp < kFirstEpilogueWarp + 4) {
     // ------------------------------------------------------------ epilogue
     pdl_wait();   // y, the partials and the counters may still be in use upstream
@@ -765,20 +748,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int slot = (pi == 0) ? 0 : 1;
       float* pbase = a.partials + ((static_cast<int64_t>(blockIdx.x) * 2 + slot) * 128 + t) * kSegRows;
       for (int c = 0; c < nb; ++c) {
-        // hi columns [16c, 16c+16), lo columns [16nb + 16c, +16) of each accumulator
+        // columns [16c, 16c+16) of each group's accumulator
         float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.0f;
         for (int w = 0; w < kDequantGroups; ++w) {
           const int off = ((w - lpf) % kDequantGroups + kDequantGroups) % kDequantGroups;
           if (off >= plen) continue;
-          uint32_t rh[16], rl[16];   // hi columns, lo columns
-          tmem_ld16(dbase + w * acc_w + 16 * c, rh);
-          tmem_ld16(dbase + w * acc_w + 16 * nb + 16 * c, rl);
+          uint32_t rr[16];
+          tmem_ld16(dbase + w * acc_w + 16 * c, rr);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            v[j] = __fadd_rn(__fadd_rn(v[j], __uint_as_float(rh[j])), __uint_as_float(rl[j]));
+          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __uint_as_float(rr[j]));
         }
         // back from the scaled domain: times 2^e / 256 per token (exact), with
         // 2^e from the prologue in fused mode (it may differ between the CTAs
@@ -798,8 +779,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (a.cluster_s > 1) {
           // cluster split-K: the partial goes to this CTA's reduction buffer
-          // (stage 0's B region, free once the MMAs completed), token-major
-          float* red = reinterpret_cast<float*>(smem + kCodesBytes);
+          // (stage 0, free once the MMAs completed), token-major
+          float* red = reinterpret_cast<float*>(smem);
 #pragma unroll
           for (int j = 0; j < 16; ++j) red[(16 * c + j) * 128 + t] = v[j];
         } else if (whole) {
@@ -885,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Seg sg = get_seg(a, tile / a.row_tiles);
       const int r0 = rank * 128 / s_n, r1 = (rank + 1) * 128 / s_n;
       const int nrow = r1 - r0;
-      const uint32_t red = smem_u32(smem + kCodesBytes);
+      const uint32_t red = smem_u32(smem);
       for (int idx = threadIdx.x; idx < nrow * sg.count; idx += kThreads) {
         const int j = idx / nrow, rl = r0 + (idx - j * nrow);
         const int row = rt * 128 + rl;
@@ -963,7 +944,7 @@ int streamk_max_clusters(int s) {
 
 size_t streamk_smem_bytes() { return static_cast<size_t>(kStages) * kStageBytes + kLutBytes + 1024; }
 
-cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void* tm_xlo, const StreamKArgs& a,
+cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const StreamKArgs& a,
                            int grid, cudaStream_t st) {
   static bool attr_set = false;
   const size_t smem = streamk_smem_bytes();
@@ -980,8 +961,7 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void*
     lt.h[i] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(cb.levels[i] * kLevelScale)));
   lt.max_level = __half2float(__float2half_rn(cb.levels[15] * kLevelScale));
   const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
-  const CUtensorMap& m1 = *static_cast<const CUtensorMap*>(tm_xhi);
-  const CUtensorMap& m2 = *static_cast<const CUtensorMap*>(tm_xlo);
+  const CUtensorMap& m1 = *static_cast<const CUtensorMap*>(tm_x);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
@@ -999,7 +979,7 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_xhi, const void*
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, streamk_kernel, m0, m1, m2, a, lt);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, streamk_kernel, m0, m1, a, lt);
   if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();

@@ -139,7 +139,7 @@ size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
  * Small m (<= 128) rotates each 32-slice of x by the weight's own RHT
  * (x' = R x; R's orthogonality makes this equivalent to inverse-rotating W),
  * scales each row by a power of two that keeps it inside the fp16 range,
- * splits it into fp16 hi + lo, and multiplies the rotated-domain levels
+ * rounds it to fp16, and multiplies the rotated-domain levels
  * fp16(256 c[code]) * d (fp16 product) by x' on the tensor cores, streaming
  * the packed weight once and scaling back exactly.  For m <= 32 with a short
  * k range per CTA this is one kernel launch (the GEMM kernel rotates x
@@ -160,7 +160,7 @@ int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t
  * start-up and forbid new ones later cannot hand tq4_1s_linear a workspace;
  * this entry point takes only x, w and y and keeps its scratch (rotated
  * activations, stream-K partial sums, tile counters) in a fixed device array
- * inside the library: about 5.6 MiB, reserved on every GPU that loads the
+ * inside the library: about 5.2 MiB, reserved on every GPU that loads the
  * library and held until the process exits.
  *   Limits: m <= 32, w->k <= 8192, w->n <= 32768, dense weight; larger
  *   shapes return TQ_ERR_SCRATCH_LIMIT and launch nothing.
