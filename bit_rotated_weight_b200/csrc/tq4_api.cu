@@ -369,7 +369,9 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xr, xscale, mask, st) != cudaSuccess)
       return TQ_ERR_CUDA;
     alignas(64) CUtensorMap tc, tx;
-    if (!map_codes(&tc, w) || !map_bf16(&tx, xr, m, w->k, 16)) return TQ_ERR_CUDA;
+    // the producer stages x' (TMA-fed mode) or the raw x (fused mode)
+    if (!map_codes(&tc, w) || !map_bf16(&tx, fused ? static_cast<const void*>(x) : xr, m, w->k, 16))
+      return TQ_ERR_CUDA;
     StreamKArgs a{};
     a.n = static_cast<int32_t>(w->n);
     a.k = static_cast<int32_t>(w->k);

@@ -117,7 +117,7 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   alignas(64) CUtensorMap tc, tx;
   {
     // same tensor maps as tq4_1s_linear: codes [1][n][k/2] (64 B x 128 rows),
-    // x' [m][k] (64 x 16)
+    // x' (TMA-fed mode) or x (fused mode) [m][k] (64 x 16)
     typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -143,7 +143,8 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
     if (fn(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, cd, cs, cb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
             CUDA_SUCCESS ||
-        fn(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, xr, xd, xs, xb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+        fn(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, fused ? const_cast<uint16_t*>(x) : xr, xd, xs, xb, es,
+           CU_TENSOR_MAP_INTERLEAVE_NONE,
            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
             CUDA_SUCCESS)
       return TQ_ERR_CUDA;

@@ -16,10 +16,11 @@
 // it to global memory (row_scale = 2^e per row) and the producer stages it
 // with TMA.  Fused mode (a dense layer of at most kSegRows rows whose CTAs
 // run at most kFusedMaxIters iterations each, so every iteration has a stage
-// of its own): the kernel rotates x itself in a prologue -- the dequant and
-// epilogue warps read x, take each row's maximum over the k range this CTA
-// covers, and write every stage's B tile -- while the codes are in flight,
-// which saves the second launch and the x' round trip through memory.
+// of its own): the producer stages the raw bf16 x tiles into the B regions
+// first, then the codes; the dequant and epilogue warps take each row's
+// maximum over the k range this CTA covers and rotate the tiles in place
+// while the codes are in flight -- no second launch, no x' round trip
+// through memory.
 //
 // Per 128-row x 128-k iteration of a tile:
 //   warp 0      TMA: codes tile [128 x 64 B] (64-byte swizzle) and, in
@@ -99,7 +100,7 @@ struct SharedState {
   uint64_t dempty[4];          // the epilogue drained an accumulator set (128 arrivals)
   uint64_t issuer_done[kDequantGroups];
   uint64_t xready;             // fused mode: every stage's x' tile is written (one arrival per prologue warp)
-  uint64_t xissued;            // fused mode: the prologue's global reads are issued (one arrival per prologue warp)
+  uint64_t xland[kFusedMaxIters];   // fused mode: the raw x tiles of a stage landed (TMA)
   float row_scale[kSegRows];   // fused mode: 2^e of each row
   unsigned row_max[kSegRows];  // fused mode: max |x| of each row over this CTA's k range (float bits)
   uint32_t tmem_base;
@@ -317,7 +318,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&sh.issuer_done[i], 1);
     }
     mbar_init(&sh.xready, kPrologueThreads / 32);
-    mbar_init(&sh.xissued, kPrologueThreads / 32);
+    for (int i = 0; i < kFusedMaxIters; ++i) mbar_init(&sh.xland[i], 1);
     for (int j = 0; j < kSegRows; ++j) sh.row_max[j] = 0u;
     sh.abort_flag = 0;
     sh.last_flag = 0;
@@ -385,69 +386,58 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (fused && warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp + 4) {
     // ------------------------------------------------------------ fused prologue
-    // Unit u = (iteration li, slice sl, row j), j fastest: 32 consecutive x
-    // values of row j at k = 128 kit(li) + 32 sl; a thread takes units ptid
-    // and ptid + kPrologueThreads and keeps their x in registers.  Pass 1
-    // takes each row's max |x| over the units; pass 2 applies the signs, the
-    // butterfly and r 2^-e, rounds to fp16 and writes row j of stage li's B
-    // tile, 16-byte chunk c of a 128-byte row at chunk c ^ (j & 7) (128-byte
-    // swizzle).  The exponent e puts sqrt(32) max|x|, the bound on |x'|, in
-    // [2^13, 2^14).
+    // Stage li's B region holds the bf16 x tile of its k range, as the TMA
+    // wrote it: row j at 128 j within each 64-k half, 16-byte chunk c at
+    // chunk c ^ (j & 7) (128-byte swizzle); rows past m and k past the end
+    // are zero.  Unit u = (iteration li, slice sl, row j), j fastest: the 32
+    // values of row j at k = 128 kit(li) + 32 sl, chunks (sl & 1) * 4 + q of
+    // half sl >> 1.  Pass 1 takes each row's max |x| over the units; pass 2
+    // applies the signs, the butterfly and r 2^-e, rounds to fp16 and writes
+    // the slice back in place.  The exponent e puts sqrt(32) max|x|, the
+    // bound on |x'|, in [2^13, 2^14).
     const int ptid = threadIdx.x - kFirstDequantWarp * 32;
     const int m = a.m_host;
-    const int units = cnt * 4 * m;   // <= kFusedMaxIters * 4 * kSegRows = 2 * kPrologueThreads
-    static_assert(kFusedMaxIters * 4 * kSegRows <= 2 * kPrologueThreads, "two units per prologue thread");
-    uint32_t raw[2][16];   // the thread's units of x, bf16 pairs, kept for pass 2
+    const int units = cnt * 4 * m;
+    bool xok = true;
+    for (int li = 0; li < cnt; ++li) xok = xok && warp_wait(&sh.xland[li], 0, abortp);
+    // a unit's row base in shared memory and the XOR giving its 4 chunks
+    auto unit_row = [&](int u, int& cx) -> uint8_t* {
+      const int j = u % m, rest = u / m, sl = rest & 3, li = rest >> 2;
+      cx = ((sl & 1) * 4) ^ (j & 7);   // chunk q sits at chunk q ^ cx
+      return smem + li * kStageBytes + kCodesBytes + (sl >> 1) * kXHalfBytes + j * 128;
+    };
+    for (int u = ptid; xok && u < units; u += kPrologueThreads) {
+      float mx = 0.0f;
+      int cx;
+      const uint8_t* rowp = unit_row(u, cx);
 #pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int u = ptid + r * kPrologueThreads;
+      for (int q = 0; q < 4; ++q) {
+        const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((q ^ cx) << 4));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-      for (int i = 0; i < 16; ++i) raw[r][i] = 0u;
-      if (u < units) {
-        const int j = u % m, rest = u / m, sl = rest & 3, li = rest >> 2;
-        const int k0 = ((it_begin + li) % KI) * 128 + 32 * sl;
-        if (k0 < a.k) {
-          const uint4* src = reinterpret_cast<const uint4*>(a.x_raw + static_cast<int64_t>(j) * a.k + k0);
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const uint4 w = __ldg(src + q);
-            raw[r][4 * q] = w.x;
-            raw[r][4 * q + 1] = w.y;
-            raw[r][4 * q + 2] = w.z;
-            raw[r][4 * q + 3] = w.w;
-          }
+        for (int e = 0; e < 4; ++e) {
+          mx = fmaxf(mx, fabsf(__uint_as_float(ww[e] << 16)));
+          mx = fmaxf(mx, fabsf(__uint_as_float(ww[e] & 0xFFFF0000u)));
         }
       }
-    }
-    // the small reads are on their way: let the producer start the weight
-    // stream behind them (relaxed: the loads need not have completed)
-    __syncwarp();
-    if (lane == 0) asm volatile("mbarrier.arrive.relaxed.cta.shared::cta.b64 _, [%0];" ::"r"(smem_u32(&sh.xissued)) : "memory");
-#pragma unroll
-    for (int r = 0; r < 2; ++r) {
-      const int u = ptid + r * kPrologueThreads;
-      if (u < units) {
-        float mx = 0.0f;
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          mx = fmaxf(mx, fabsf(__uint_as_float(raw[r][i] << 16)));
-          mx = fmaxf(mx, fabsf(__uint_as_float(raw[r][i] & 0xFFFF0000u)));
-        }
-        atomicMax(&sh.row_max[u % m], __float_as_uint(mx));   // non-negative floats order as integers
-      }
+      atomicMax(&sh.row_max[u % m], __float_as_uint(mx));   // non-negative floats order as integers
     }
     named_bar_sync(2, kPrologueThreads);
     const float r = __uint_as_float(0x3E3504F3u);
-#pragma unroll
-    for (int rr = 0; rr < 2; ++rr) {
-      const int u = ptid + rr * kPrologueThreads;
-      if (u >= units) continue;
+    for (int u = ptid; xok && u < units; u += kPrologueThreads) {
       const int j = u % m, rest = u / m, sl = rest & 3, li = rest >> 2;
+      int cx;
+      uint8_t* rowp = unit_row(u, cx);
       float v[32];
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        v[2 * i] = __uint_as_float(raw[rr][i] << 16);
-        v[2 * i + 1] = __uint_as_float(raw[rr][i] & 0xFFFF0000u);
+      for (int q = 0; q < 4; ++q) {
+        const uint4 w = *reinterpret_cast<const uint4*>(rowp + ((q ^ cx) << 4));
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          v[8 * q + 2 * e] = __uint_as_float(ww[e] << 16);
+          v[8 * q + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+        }
       }
 #pragma unroll
       for (int i = 0; i < 32; ++i)
@@ -463,7 +453,6 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (li == 0 && sl == 0) sh.row_scale[j] = ldexpf(1.0f, e);
       const float rd = __fmul_rn(r, ldexpf(1.0f, -e));   // exact: r times a power of two
-      uint8_t* hbase = smem + li * kStageBytes + kCodesBytes + (sl >> 1) * kXHalfBytes;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         uint32_t hw[4];
@@ -472,8 +461,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const __half2 h = __floats2half2_rn(__fmul_rn(v[8 * q + 2 * c2], rd), __fmul_rn(v[8 * q + 2 * c2 + 1], rd));
           hw[c2] = *reinterpret_cast<const uint32_t*>(&h);
         }
-        const int c = (sl & 1) * 4 + q;
-        *reinterpret_cast<uint4*>(hbase + j * 128 + ((c ^ (j & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        *reinterpret_cast<uint4*>(rowp + ((q ^ cx) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       }
     }
     fence_proxy_async_smem();   // the generic-proxy writes, before the tensor core reads them
@@ -500,17 +488,23 @@ __global__ void __launch_bounds__(kThreads, 1)
       // rotation) lets it start only once everything earlier has finished,
       // and does not write the weight.  Fused mode: any kernel may come
       // before, so wait first.
-      if (fused) {
-        pdl_wait();
-        // the weight stream goes out behind the prologue's reads of x and the
-        // first scales, which would otherwise queue behind ~all of it
-        mbar_wait(&sh.xissued, 0, abortp);
-      }
       const int npre = cnt < kStages ? cnt : kStages;
       const uint32_t xbytes = fused ? 0u : 2u * 2048u;   // per 16-row block: two k-halves of 16 x 128 B
       Cursor cur;
       cur.init(it_begin, KI, a.row_tiles);
       const Cursor first = cur;
+      if (fused) {
+        pdl_wait();
+        // the raw x tiles first (small; the prologue needs them), then the
+        // weight stream behind them (one segment of m <= kSegRows rows)
+        const Seg sx = get_seg(a, 0);
+        const int nbx = (sx.count + 15) >> 4;
+        Cursor cx = first;
+        for (int li = 0; li < cnt; ++li, cx.advance(1, KI, a.row_tiles)) {
+          mbar_arrive_expect_tx(&sh.xland[li], static_cast<uint32_t>(nbx) * 2u * 2048u);
+          load_x(smem + li * kStageBytes, cx.kit, sx, nbx, &sh.xland[li]);
+        }
+      }
       Seg sg = get_seg(a, cur.sgi);
       int seg_of = cur.sgi;
       for (int li = 0; li < npre; ++li, cur.advance(1, KI, a.row_tiles)) {
@@ -556,6 +550,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // wind down: let every armed copy land before the CTA exits
         for (int i = 0; i < kStages; ++i)
           if (armed[i] >= 0) drain_wait(&sh.full[i], static_cast<uint32_t>(armed[i]));
+        if (fused)
+          for (int i = 0; i < cnt; ++i) drain_wait(&sh.xland[i], 0);
       }
     }
   } else if (warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp) {
