@@ -39,6 +39,9 @@ M_TOK, N_OUT, K_IN = 16, 4096, 4096
 CALLS = 16
 COPIES = 64
 PACKED_PER_CALL = N_OUT * K_IN // 2 + N_OUT * (K_IN // 16) * 2   # 10,485,760 B
+# DRAM bytes (read + write) of one decode launch of the kernel, from the ncu
+# capture summarised in profiles/streamk_decode_m16_n4096_k4096.md
+TRAFFIC_PER_CALL = 10_706_944
 WORKLOAD = ("decode_linear_4096: x bf16 [16][4096] N(0,1), W 4096x4096 Student-t(5)*0.02 TQ4_1S, "
             "16 calls per step (denoising steps)")
 
@@ -282,8 +285,12 @@ def ours_arm(args):
                        "parallelism": f"replicas x{world}", "timing": "CUDA graph per step (16 calls)",
                        "l2": "cold: 64 distinct packed weight copies (671 MB > 126 MB L2) cycled, 16 per step"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                         "kernel": "tq4_1s_linear small-m call (activation rotation + stream-K dequant-GEMM), per call",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": TRAFFIC_PER_CALL,
+                         "algorithmic_bytes": PACKED_PER_CALL,
+                         "kernel": "streamk_kernel, fused cluster split-K mode: one launch per tq4_1s_linear "
+                                   "call (x staging and rotation, dequant, MMA, on-chip reduction)",
+                         "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch, "
+                                           "profiles/streamk_decode_m16_n4096_k4096.md",
                          "peak_source": pk["source"], "per_call_us": per_call_ms * 1e3},
             "eager_per_call_us": ms_eager / CALLS * 1e3,
             "cpu_baseline": cpu,
