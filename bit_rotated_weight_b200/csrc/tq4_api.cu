@@ -166,6 +166,16 @@ static bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
   return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
 }
 
+// x [rows][cols] (cols % 64 == 0) viewed as [cols/64][rows][64] 16-bit,
+// box 64 x 32 x 2*kFusedMaxIters, 128-byte swizzle: one copy fills the B
+// tiles of all stages of a fused CTA.
+static bool map_x3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+  const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / 64)};
+  const uint64_t strides[2] = {static_cast<uint64_t>(cols * 2), 128};
+  const uint32_t box[3] = {64, static_cast<uint32_t>(kSegRows), static_cast<uint32_t>(2 * kFusedMaxIters)};
+  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
 // 16-bit matrix [rows][cols] row-major (bf16 or fp16), box 64 x box_rows,
 // 128-byte swizzle.
 static bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
@@ -368,10 +378,12 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     // TMA-fed mode: x' = R x (fp16, per-row scale) by the rotation kernel
     if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xr, xscale, mask, st) != cudaSuccess)
       return TQ_ERR_CUDA;
-    alignas(64) CUtensorMap tc, tx;
+    alignas(64) CUtensorMap tc, tx, tx3;
     // the producer stages x' (TMA-fed mode) or the raw x (fused mode)
     if (!map_codes(&tc, w) || !map_bf16(&tx, fused ? static_cast<const void*>(x) : xr, m, w->k, 16))
       return TQ_ERR_CUDA;
+    const bool box3 = split > 1 && (w->k % 64) == 0;
+    if (box3 && !map_x3(&tx3, x, m, w->k)) return TQ_ERR_CUDA;
     StreamKArgs a{};
     a.n = static_cast<int32_t>(w->n);
     a.k = static_cast<int32_t>(w->k);
@@ -384,16 +396,17 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     a.row_scale = xscale;
     if (fused) {
       a.x_raw = x;
-      a.x_mask = mask;
+      sign_xor_words(mask, a.x_sign);
     }
     a.epoch = next_epoch();
     a.cluster_s = split;
+    a.x_box3 = box3 ? 1 : 0;
     a.mode = EPI_DENSE;
     a.out_a = y;
     a.partials = reinterpret_cast<float*>(base + L.partials);
     a.counters = reinterpret_cast<unsigned long long*>(base + L.counters);
     a.max_tiles = static_cast<int32_t>(L.tiles);
-    return cuda_rc(launch_streamk(&tc, &tx, a, grid, st));
+    return cuda_rc(launch_streamk(&tc, &tx, box3 ? &tx3 : nullptr, a, grid, st));
   }
   // large m: W_hat in bf16, then the tensor-core GEMM
   uint16_t* wh = reinterpret_cast<uint16_t*>(base);
@@ -484,7 +497,7 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   a.partials = reinterpret_cast<float*>(base + L.partials);
   a.counters = reinterpret_cast<unsigned long long*>(base + L.cnt_up);
   a.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_up);
-  if ((e = launch_streamk(&tcu, &txr, a, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
+  if ((e = launch_streamk(&tcu, &txr, nullptr, a, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
 
   // h' = R_down h per sorted pair row
   e = launch_rotate_scaled(h, I, nullptr, 1, npv, 0, L.P, hr, hscale, sign_mask_of(down->seed), st);
@@ -504,7 +517,7 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   b.topk_w = topk_w;
   b.counters = reinterpret_cast<unsigned long long*>(base + L.cnt_dn);
   b.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_dn);
-  if ((e = launch_streamk(&tcd, &thr, b, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
+  if ((e = launch_streamk(&tcd, &thr, nullptr, b, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
   return cuda_rc(launch_moe_combine(zw, topk_ids, m, topk, H, static_cast<int32_t>(E), y, st));
 }
 

@@ -60,10 +60,12 @@ struct StreamKArgs {
   const float* row_scale;    // x' row r holds x'_r * 2^-e_r; row_scale[r] = 2^e_r (TMA-fed mode)
   const uint16_t* x_raw;     // fused mode (dense, m <= kSegRows, <= kFusedMaxIters iterations per CTA):
                              // raw bf16 x [m][k], rotated by the kernel itself; nullptr otherwise
-  uint32_t x_mask;           // fused mode: the weight's sign mask
+  uint32_t x_sign[16];       // fused mode: the weight's sign mask as XOR words on bf16 pairs --
+                             // word i flips bit 15 / bit 31 where sign i*2 / i*2+1 is negative
   uint32_t epoch;            // tag of this launch in the tile counters (never 0)
   int32_t cluster_s;         // >= 2: fused split-K mode -- grid = tiles * cluster_s, one cluster per
                              // tile, partials reduced through distributed shared memory; else 1
+  int32_t x_box3;            // cluster mode with k % 64 == 0: x arrives as one 3-D box (tm_x3)
   int32_t mode;              // EpilogueMode
   uint16_t* out_a;           // dense: y [m][n]; up: h = relu(u)^2 [P][n] (bf16)
   float* out_f;              // down: z*w [m*topk][n]
@@ -81,6 +83,12 @@ constexpr int kFusedMaxIters = 8;
 // A fresh counter tag for each stream-K launch.
 uint32_t next_epoch();
 
+// The sign mask as XOR words over bf16 pairs (StreamKArgs::x_sign).
+inline void sign_xor_words(uint32_t mask, uint32_t (&w)[16]) {
+  for (int i = 0; i < 16; ++i)
+    w[i] = (((mask >> (2 * i)) & 1u) << 15) | (((mask >> (2 * i + 1)) & 1u) << 31);
+}
+
 // Bytes of dynamic shared memory the stream-K kernel uses.
 size_t streamk_smem_bytes();
 // How many clusters of s stream-K CTAs can be resident at once (0 on error).
@@ -91,7 +99,11 @@ int streamk_max_clusters(int s);
 // resident at once; 1 if none fits.
 int choose_cluster_split(int64_t tiles, int64_t k_iters, int sms);
 
-cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const StreamKArgs& a, int grid, cudaStream_t st);
+// tm_x: the x' (TMA-fed) or x (fused) tiles, box 64 x 16; tm_x3 (cluster
+// split-K mode, else may be null): x viewed as [k/64][m][64], box 64 x 32 x
+// 2*kFusedMaxIters.
+cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const void* tm_x3, const StreamKArgs& a, int grid,
+                           cudaStream_t st);
 
 // ---------------------------------------------------------------- GEMM
 // y[m][n] = bf16( x[m][k] * w[n][k]^T ), bf16 operands via TMA tensor maps.

@@ -161,7 +161,7 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   a.row_scale = xscale;
   if (fused) {
     a.x_raw = x;
-    a.x_mask = mask;
+    sign_xor_words(mask, a.x_sign);
   }
   a.epoch = next_epoch();
   a.cluster_s = split;
@@ -170,5 +170,5 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   a.partials = partials;
   a.counters = counters;
   a.max_tiles = static_cast<int32_t>(tiles);
-  return launch_streamk(&tc, &tx, a, grid, st) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  return launch_streamk(&tc, &tx, nullptr, a, grid, st) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

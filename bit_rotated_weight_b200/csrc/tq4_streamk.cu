@@ -47,10 +47,11 @@
 // fp32 partials in CTA order (deterministic) and runs the epilogue, so no
 // CTA ever waits on another.  Cluster split-K mode (fused mode with a grid of
 // tiles x s CTAs, s per tile): the even split gives each CTA 1/s of one
-// tile's k range; the s CTAs of a tile form a thread-block cluster, write
-// their partials to their own shared memory and, after a cluster barrier,
-// each sums 1/s of the tile's rows over the s partials in rank order through
-// distributed shared memory -- no partials or counters in global memory.
+// tile's k range; the s CTAs of a tile form a thread-block cluster, each
+// owns 1/s of the tile's rows: every CTA stores each row of its partial into
+// the owner's shared memory (distributed shared memory), and after one
+// cluster barrier each owner sums its rows over the s partials in rank order
+// -- deterministic, no partials or counters in global memory.
 #include <atomic>
 #include <mutex>
 
@@ -74,6 +75,14 @@ constexpr int kCodesBytes = 128 * 64;    // 128 rows x 128 k codes
 constexpr int kXHalfBytes = kSegRows * 128;   // up to 32 token rows x 64 k of fp16 x' (128-B swizzle span)
 constexpr int kXBytes = 2 * kXHalfBytes; // two k-halves
 constexpr int kStageBytes = kCodesBytes + kXBytes;
+// Shared memory: the codes of the stages [kStages][kCodesBytes], then the B
+// tiles [kStages][kXBytes] (contiguous, so one TMA box can fill several),
+// then the level-pair table.
+constexpr int kBOff = kStages * kCodesBytes;
+// Cluster split-K: each CTA receives the partial rows it reduces into the
+// codes of stages kFusedMaxIters.. (never loaded in fused mode):
+// [source rank][32 tokens][rows per CTA] floats.
+constexpr int kRedOff = kFusedMaxIters * kCodesBytes;
 constexpr int kLutBytes = 256 * 32 * 4;  // fp16 level-pair table, one copy per lane
 constexpr int kTmemCols = 512;
 // Tensor memory: columns [0, 256) hold the accumulators, [256, 512) the four
@@ -268,12 +277,14 @@ struct LevelTable {
 
 __global__ void __launch_bounds__(kThreads, 1)
     streamk_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
-                   const StreamKArgs a,
+                   const __grid_constant__ CUtensorMap tm_x3, const StreamKArgs a,
                    const __grid_constant__ LevelTable lt) {
   __shared__ SharedState sh;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
   uint8_t* lut = smem + kStages * kStageBytes;
+  auto codes_of = [&](int st) { return smem + st * kCodesBytes; };
+  auto btile_of = [&](int st) { return smem + kBOff + st * kXBytes; };
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   // Grouped (MoE) mode reads the routing kernel's segment list right away;
@@ -288,11 +299,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cnt = it_end - it_begin;
   if (cnt <= 0) {
     // (the host never gives a cluster-mode CTA an empty range; if one had
-    // one, it would still meet its cluster's barriers)
-    if (a.cluster_s > 1) {
-      cluster_sync_all();
-      cluster_sync_all();
-    }
+    // one, it would still meet its cluster's barrier)
+    if (a.cluster_s > 1) cluster_sync_all();
     return;
   }
   const bool fused = a.x_raw != nullptr;
@@ -399,12 +407,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int m = a.m_host;
     const int units = cnt * 4 * m;
     bool xok = true;
-    for (int li = 0; li < cnt; ++li) xok = xok && warp_wait(&sh.xland[li], 0, abortp);
+    for (int li = 0; li < (a.x_box3 ? 1 : cnt); ++li) xok = xok && warp_wait(&sh.xland[li], 0, abortp);
     // a unit's row base in shared memory and the XOR giving its 4 chunks
     auto unit_row = [&](int u, int& cx) -> uint8_t* {
       const int j = u % m, rest = u / m, sl = rest & 3, li = rest >> 2;
       cx = ((sl & 1) * 4) ^ (j & 7);   // chunk q sits at chunk q ^ cx
-      return smem + li * kStageBytes + kCodesBytes + (sl >> 1) * kXHalfBytes + j * 128;
+      return btile_of(li) + (sl >> 1) * kXHalfBytes + j * 128;
     };
     for (int u = ptid; xok && u < units; u += kPrologueThreads) {
       float mx = 0.0f;
@@ -435,13 +443,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
-          v[8 * q + 2 * e] = __uint_as_float(ww[e] << 16);
-          v[8 * q + 2 * e + 1] = __uint_as_float(ww[e] & 0xFFFF0000u);
+          const uint32_t sw = ww[e] ^ a.x_sign[4 * q + e];   // the signs s_i, on the bf16 sign bits
+          v[8 * q + 2 * e] = __uint_as_float(sw << 16);
+          v[8 * q + 2 * e + 1] = __uint_as_float(sw & 0xFFFF0000u);
         }
       }
-#pragma unroll
-      for (int i = 0; i < 32; ++i)
-        if ((a.x_mask >> i) & 1u) v[i] = -v[i];
       fwht32_regs_sk(v);
       const float mx = __uint_as_float(sh.row_max[j]);
       int e = 0;
@@ -475,11 +481,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       int armed[kStages];
 #pragma unroll
       for (int i = 0; i < kStages; ++i) armed[i] = -1;
-      auto load_x = [&](uint8_t* st, int kit, const Seg& sg, int nb, uint64_t* bar) {
+      auto load_x = [&](int st, int kit, const Seg& sg, int nb, uint64_t* bar) {
         for (int b = 0; b < nb; ++b) {
 #pragma unroll
           for (int kh = 0; kh < 2; ++kh)
-            tma_load_2d(st + kCodesBytes + kh * kXHalfBytes + (16 * b) * 128, &tm_x, bar, kit * 128 + 64 * kh,
+            tma_load_2d(btile_of(st) + kh * kXHalfBytes + (16 * b) * 128, &tm_x, bar, kit * 128 + 64 * kh,
                         sg.row0 + 16 * b);
         }
       };
@@ -499,10 +505,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         // weight stream behind them (one segment of m <= kSegRows rows)
         const Seg sx = get_seg(a, 0);
         const int nbx = (sx.count + 15) >> 4;
-        Cursor cx = first;
-        for (int li = 0; li < cnt; ++li, cx.advance(1, KI, a.row_tiles)) {
-          mbar_arrive_expect_tx(&sh.xland[li], static_cast<uint32_t>(nbx) * 2u * 2048u);
-          load_x(smem + li * kStageBytes, cx.kit, sx, nbx, &sh.xland[li]);
+        if (a.x_box3) {
+          // one box: the 2 * kFusedMaxIters 64-k chunks from this CTA's first
+          // k, 32 rows each, straight into the contiguous B tiles (chunks past
+          // this CTA's range land in B tiles it does not use)
+          mbar_arrive_expect_tx(&sh.xland[0], 2u * kFusedMaxIters * kXHalfBytes);
+          tma_load_3d(btile_of(0), &tm_x3, &sh.xland[0], 0, 0, 2 * first.kit);
+        } else {
+          Cursor cx = first;
+          for (int li = 0; li < cnt; ++li, cx.advance(1, KI, a.row_tiles)) {
+            mbar_arrive_expect_tx(&sh.xland[li], static_cast<uint32_t>(nbx) * 2u * 2048u);
+            load_x(li, cx.kit, sx, nbx, &sh.xland[li]);
+          }
         }
       }
       Seg sg = get_seg(a, cur.sgi);
@@ -515,7 +529,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int nb = (sg.count + 15) >> 4;
         mbar_arrive_expect_tx(&sh.full[li], kCodesBytes + nb * xbytes);
         armed[li] = 0;
-        tma_load_3d(smem + li * kStageBytes, &tm_codes, &sh.full[li], cur.kit * 64, cur.rt * 128, sg.e);
+        tma_load_3d(codes_of(li), &tm_codes, &sh.full[li], cur.kit * 64, cur.rt * 128, sg.e);
       }
       if (!fused) {
         pdl_wait();   // x' and its row scales are the rotation kernel's output
@@ -527,7 +541,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             seg2 = c2.sgi;
             sg2 = get_seg(a, seg2);
           }
-          load_x(smem + li * kStageBytes, c2.kit, sg2, (sg2.count + 15) >> 4, &sh.full[li]);
+          load_x(li, c2.kit, sg2, (sg2.count + 15) >> 4, &sh.full[li]);
         }
       }
       // (fused mode: cnt <= kStages, so the loop below does not run)
@@ -540,18 +554,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           sg = get_seg(a, seg_of);
         }
         const int nb = (sg.count + 15) >> 4;
-        uint8_t* st = smem + s * kStageBytes;
         mbar_arrive_expect_tx(&sh.full[s], kCodesBytes + nb * xbytes);
         armed[s] = static_cast<int>(ph);
-        tma_load_3d(st, &tm_codes, &sh.full[s], cur.kit * 64, cur.rt * 128, sg.e);
-        load_x(st, cur.kit, sg, nb, &sh.full[s]);
+        tma_load_3d(codes_of(s), &tm_codes, &sh.full[s], cur.kit * 64, cur.rt * 128, sg.e);
+        load_x(s, cur.kit, sg, nb, &sh.full[s]);
       }
       if (*abortp) {
         // wind down: let every armed copy land before the CTA exits
         for (int i = 0; i < kStages; ++i)
           if (armed[i] >= 0) drain_wait(&sh.full[i], static_cast<uint32_t>(armed[i]));
         if (fused)
-          for (int i = 0; i < cnt; ++i) drain_wait(&sh.xland[i], 0);
+          for (int i = 0; i < (a.x_box3 ? 1 : cnt); ++i) drain_wait(&sh.xland[i], 0);
       }
     }
   } else if (warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp) {
@@ -612,7 +625,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       const int s = li % kStages;
       if (!warp_wait(&sh.full[s], (li / kStages) & 1, abortp)) break;
-      const uint8_t* cb = smem + s * kStageBytes + t * 64;
+      const uint8_t* cb = codes_of(s) + t * 64;
       bool ok = true;
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
@@ -672,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int li = pf + ((w - pf) % kDequantGroups + kDequantGroups) % kDequantGroups; li < pe && ok;
            li += kDequantGroups) {
         const int s = li % kStages;
-        const uint32_t xb = smem_u32(smem + s * kStageBytes + kCodesBytes);
+        const uint32_t xb = smem_u32(btile_of(s));
         // the B tile (x') of this stage must have landed too
         if (!mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) {
           ok = false;
@@ -774,11 +787,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           mbar_arrive(&sh.dempty[db]);
         }
         if (a.cluster_s > 1) {
-          // cluster split-K: the partial goes to this CTA's reduction buffer
-          // (stage 0, free once the MMAs completed), token-major
-          float* red = reinterpret_cast<float*>(smem);
+          // cluster split-K: row t goes to the CTA that owns it, slot of this
+          // CTA's rank: [rank][token][row - first row of the owner]
+          const int s_n = a.cluster_s;
+          const int q = (t * s_n) >> 7;                       // owner: floor(t s / 128)
+          const int rpc = (128 + s_n - 1) / s_n;              // rows per CTA (at most)
+          const int tl = t - (q * 128 + s_n - 1) / s_n;       // row within the owner's range
+          const uint32_t dst0 = smem_u32(smem + kRedOff) +
+                                static_cast<uint32_t>(((static_cast<int>(cluster_ctarank()) * 32 + 16 * c) * rpc + tl) * 4);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) red[(16 * c + j) * 128 + t] = v[j];
+          for (int j = 0; j < 16; ++j) st_dsmem_f32(dst0 + static_cast<uint32_t>(j * rpc * 4), static_cast<uint32_t>(q), v[j]);
         } else if (whole) {
           epilogue_store(a, v, 16 * c, row, sg);
         } else {
@@ -850,9 +868,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   if (a.cluster_s > 1) {
     // Cluster split-K reduction.  Every thread of every CTA of the cluster
-    // reaches both barriers (on a timeout too: the roles above always run to
-    // their end), so neither can hang; the second keeps each CTA's buffer
-    // alive until the other CTAs have read it.
+    // reaches the barrier (on a timeout too: the roles above always run to
+    // their end), so it cannot hang; it orders every CTA's stores into the
+    // owners' buffers before the owners read them.  Nothing reads another
+    // CTA's shared memory after it, so no second barrier is needed.
     cluster_sync_all();
     if (!sh.abort_flag) {
       const int s_n = a.cluster_s;
@@ -860,20 +879,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int tile = tile_begin;   // one tile per CTA in this mode
       const int rt = tile % a.row_tiles;
       const Seg sg = get_seg(a, tile / a.row_tiles);
-      const int r0 = rank * 128 / s_n, r1 = (rank + 1) * 128 / s_n;
+      const int rpc = (128 + s_n - 1) / s_n;
+      const int r0 = (rank * 128 + s_n - 1) / s_n, r1 = ((rank + 1) * 128 + s_n - 1) / s_n;
       const int nrow = r1 - r0;
-      const uint32_t red = smem_u32(smem);
+      const float* red = reinterpret_cast<const float*>(smem + kRedOff);
       for (int idx = threadIdx.x; idx < nrow * sg.count; idx += kThreads) {
-        const int j = idx / nrow, rl = r0 + (idx - j * nrow);
-        const int row = rt * 128 + rl;
+        const int j = idx / nrow, tl = idx - j * nrow;
+        const int row = rt * 128 + r0 + tl;
         if (row >= a.n) continue;
         float acc = 0.0f;
-        for (int q = 0; q < s_n; ++q)
-          acc = __fadd_rn(acc, ld_dsmem_f32(red + static_cast<uint32_t>((j * 128 + rl) * 4), static_cast<uint32_t>(q)));
+        for (int q = 0; q < s_n; ++q) acc = __fadd_rn(acc, red[(q * 32 + j) * rpc + tl]);
         a.out_a[static_cast<int64_t>(sg.row0 + j) * a.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
       }
     }
-    cluster_sync_all();
   }
   // Dependents may launch once every CTA is done: a kernel that waits on this
   // one gains nothing from taking an SM early, and its CTAs would only delay
@@ -940,7 +958,7 @@ int streamk_max_clusters(int s) {
 
 size_t streamk_smem_bytes() { return static_cast<size_t>(kStages) * kStageBytes + kLutBytes + 1024; }
 
-cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const StreamKArgs& a,
+cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const void* tm_x3, const StreamKArgs& a,
                            int grid, cudaStream_t st) {
   static bool attr_set = false;
   const size_t smem = streamk_smem_bytes();
@@ -958,6 +976,7 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const StreamK
   lt.max_level = __half2float(__float2half_rn(cb.levels[15] * kLevelScale));
   const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
   const CUtensorMap& m1 = *static_cast<const CUtensorMap*>(tm_x);
+  const CUtensorMap& m3 = *static_cast<const CUtensorMap*>(tm_x3 ? tm_x3 : tm_x);
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
@@ -975,7 +994,7 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const StreamK
     attr[1].val.clusterDim.z = 1;
     cfg.numAttrs = 2;
   }
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, streamk_kernel, m0, m1, a, lt);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, streamk_kernel, m0, m1, m3, a, lt);
   if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();
