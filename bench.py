@@ -288,7 +288,7 @@ def ours_arm(args):
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
             "config": {"workload": WORKLOAD, "global_batch": world * M_TOK, "seq_len": M_TOK,
                        "parallelism": f"replicas x{world}", "timing": "CUDA graph per step (16 calls)",
                        "l2": "cold: 64 distinct packed weight copies (671 MB > 126 MB L2) cycled, 16 per step",

@@ -141,9 +141,14 @@ __device__ __forceinline__ int floordiv(long long a, int b) {
   else if ((q + 1) * b <= a) ++q;
   return static_cast<int>(q);
 }
-// First iteration of CTA c when T iterations are split over G CTAs.
+// First iteration of CTA c when T iterations are split over G CTAs:
+// floor(c T / G) = c q + floor(c r / G) with q = T / G, r = T % G; c r < G^2
+// fits 32 bits for any grid below 2^16 CTAs.
 __device__ __forceinline__ int range_begin(int c, int T, int G) {
-  return floordiv(static_cast<long long>(c) * T, G);
+  const unsigned q = static_cast<unsigned>(T) / static_cast<unsigned>(G);
+  const unsigned r = static_cast<unsigned>(T) - q * static_cast<unsigned>(G);
+  return static_cast<int>(static_cast<unsigned>(c) * q +
+                          static_cast<unsigned>(c) * r / static_cast<unsigned>(G));
 }
 // The CTA whose range holds iteration i: ceil((i + 1) G / T) - 1.
 __device__ __forceinline__ int owner_of(int i, int T, int G) {
@@ -310,33 +315,43 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int tile_begin = it_begin / KI, tile_last = (it_end - 1) / KI;
   const int nportions = tile_last - tile_begin + 1;
 
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&sh.full[i], 1);
-      mbar_init(&sh.done[i], 1);
-    }
-    for (int i = 0; i < kDequantGroups; ++i)
-      for (int h = 0; h < 2; ++h) {
-        mbar_init(&sh.afull[i][h], 128);
-        mbar_init(&sh.afree[i][h], 1);
+  if (warp == 0) {
+    // the barriers, spread over the lanes of warp 0
+    constexpr int kBars = 2 * kStages + 4 * kDequantGroups + 12 + 1 + kFusedMaxIters;
+    for (int i = lane; i < kBars; i += 32) {
+      if (i < kStages) mbar_init(&sh.full[i], 1);
+      else if (i < 2 * kStages) mbar_init(&sh.done[i - kStages], 1);
+      else if (i < 2 * kStages + 2 * kDequantGroups) {
+        const int g = i - 2 * kStages;
+        mbar_init(&sh.afull[g >> 1][g & 1], 128);
+      } else if (i < 2 * kStages + 4 * kDequantGroups) {
+        const int g = i - 2 * kStages - 2 * kDequantGroups;
+        mbar_init(&sh.afree[g >> 1][g & 1], 1);
+      } else if (i < 2 * kStages + 4 * kDequantGroups + 4) {
+        mbar_init(&sh.dfull[i - 2 * kStages - 4 * kDequantGroups], kDequantGroups);
+      } else if (i < 2 * kStages + 4 * kDequantGroups + 8) {
+        mbar_init(&sh.dempty[i - 2 * kStages - 4 * kDequantGroups - 4], 128);
+      } else if (i < 2 * kStages + 4 * kDequantGroups + 12) {
+        mbar_init(&sh.issuer_done[i - 2 * kStages - 4 * kDequantGroups - 8], 1);
+      } else if (i == 2 * kStages + 4 * kDequantGroups + 12) {
+        mbar_init(&sh.xready, kPrologueThreads / 32);
+      } else {
+        mbar_init(&sh.xland[i - 2 * kStages - 4 * kDequantGroups - 13], 1);
       }
-    for (int i = 0; i < 4; ++i) {
-      mbar_init(&sh.dfull[i], kDequantGroups);
-      mbar_init(&sh.dempty[i], 128);
-      mbar_init(&sh.issuer_done[i], 1);
     }
-    mbar_init(&sh.xready, kPrologueThreads / 32);
-    for (int i = 0; i < kFusedMaxIters; ++i) mbar_init(&sh.xland[i], 1);
-    for (int j = 0; j < kSegRows; ++j) sh.row_max[j] = 0u;
-    sh.abort_flag = 0;
-    sh.last_flag = 0;
+    static_assert(kSegRows == 32, "one row maximum per lane");
+    sh.row_max[lane] = 0u;
+    if (lane == 0) {
+      sh.abort_flag = 0;
+      sh.last_flag = 0;
+    }
     fence_mbar_init();
   }
   {
     // table entry b (a code byte) of lane l's copy, at byte 128 b + 4 l:
     // {256 c[b & 15], 256 c[b >> 4]}
     uint32_t* lw = reinterpret_cast<uint32_t*>(lut);
-    for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
+    for (int i = threadIdx.x - 64; warp >= 2 && i < 256 * 32; i += kThreads - 64) {
       const int b = i >> 5;
       lw[i] = lt.h[b & 15] | (lt.h[b >> 4] << 16);
     }
