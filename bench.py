@@ -42,7 +42,7 @@ COPIES = 64
 PACKED_PER_CALL = N_OUT * K_IN // 2 + N_OUT * (K_IN // 16) * 2   # 10,485,760 B
 # DRAM bytes (read + write) of one decode launch of the kernel, from the ncu
 # capture summarised in profiles/streamk_decode_m16_n4096_k4096.md
-TRAFFIC_PER_CALL = 10_706_944
+TRAFFIC_PER_CALL = 10_703_872
 WORKLOAD = ("decode_linear_4096: x bf16 [16][4096] N(0,1), W 4096x4096 Student-t(5)*0.02 TQ4_1S, "
             "16 calls per step (denoising steps)")
 
