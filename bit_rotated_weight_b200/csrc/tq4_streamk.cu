@@ -297,6 +297,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (a.segs) pdl_wait();
   const int nseg = a.segs ? __ldcg(a.nseg_dev) : a.nseg_host;
   const int KI = a.k_iters;
+  if (a.segs && nseg * a.row_tiles > a.max_tiles) {
+    // more segments than the counters were sized for: the routing step is
+    // inconsistent; nothing is computed
+    if (threadIdx.x == 0) raise_status(TQ_DEV_BAD_ROUTING);
+    return;
+  }
   const int T = nseg * a.row_tiles * KI;   // < 2^31 (checked by the host)
   const int G = gridDim.x;
   const int it_begin = range_begin(blockIdx.x, T, G);
