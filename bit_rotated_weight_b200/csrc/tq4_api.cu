@@ -466,7 +466,7 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   uint16_t* hr = reinterpret_cast<uint16_t*>(base + L.hr);
   float* zw = reinterpret_cast<float*>(base + L.zw);
   cudaError_t e = launch_moe_route(topk_ids, L.P, static_cast<int32_t>(E), offsets, pairs, segs, nseg, kSegRows,
-                                   npv, nullptr, 0, st);
+                                   npv, st);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   float* xscale = reinterpret_cast<float*>(base + L.xscale);
   uint16_t* h = reinterpret_cast<uint16_t*>(base + L.h);
@@ -529,7 +529,7 @@ TQ_API int tq4_1s_moe_route(const int32_t* topk_ids, int64_t m, int32_t topk, in
   int rc = check_device(nullptr);
   if (rc) return rc;
   return cuda_rc(launch_moe_route(topk_ids, m * topk, num_experts, offsets, pairs, nullptr, nullptr, kSegRows,
-                                  nullptr, nullptr, 0, reinterpret_cast<cudaStream_t>(stream)));
+                                  nullptr, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 TQ_API uint64_t tq4_1s_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

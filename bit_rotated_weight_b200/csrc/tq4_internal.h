@@ -40,7 +40,7 @@ cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* ga
                                  uint16_t* xr, float* row_scale, uint32_t mask, cudaStream_t st);
 cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
                              int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
-                             int32_t* zero_ptr, int64_t nzero, cudaStream_t st);
+                             cudaStream_t st);
 cudaError_t launch_moe_combine(const float* zw, const int32_t* ids, int64_t m, int32_t topk, int64_t h,
                                int32_t num_experts, uint16_t* y, cudaStream_t st);
 

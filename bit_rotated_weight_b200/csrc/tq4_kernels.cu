@@ -291,20 +291,17 @@ __global__ void __launch_bounds__(kRotThreads, 10)
 // of p, and runs are ranked by a second pass over the per-thread counts.
 // Also writes (when the pointers are non-null) the segment list used by the
 // grouped stream-K launches -- chunks of at most `chunk` consecutive rows of
-// one expert -- the segment and valid-pair counts, and zeroes the stream-K
-// counters.
+// one expert -- and the segment and valid-pair counts.
 __global__ void __launch_bounds__(1024) moe_route_kernel(const int32_t* __restrict__ ids, int64_t npairs,
                                                          int32_t num_experts, int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ pairs, int4* __restrict__ segs,
                                                          int32_t* __restrict__ nseg_out, int32_t chunk,
-                                                         int32_t* __restrict__ npairs_valid,
-                                                         int32_t* __restrict__ zero_ptr, int64_t nzero) {
+                                                         int32_t* __restrict__ npairs_valid) {
   extern __shared__ int32_t sh[];
   int32_t* cnt = sh;                       // [num_experts]
   int32_t* base = sh + num_experts;        // [num_experts]
   __shared__ int32_t s_bad;
   const int tid = threadIdx.x;
-  for (int64_t i = tid; i < nzero; i += blockDim.x) zero_ptr[i] = 0;
   for (int e = tid; e < num_experts; e += blockDim.x) cnt[e] = 0;
   if (tid == 0) s_bad = 0;
   __syncthreads();
@@ -479,10 +476,9 @@ cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* ga
 
 cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
                              int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
-                             int32_t* zero_ptr, int64_t nzero, cudaStream_t st) {
+                             cudaStream_t st) {
   const size_t sh = sizeof(int32_t) * 2 * static_cast<size_t>(num_experts);
-  moe_route_kernel<<<1, 1024, sh, st>>>(ids, npairs, num_experts, offsets, pairs, segs, nseg, chunk, npairs_valid,
-                                        zero_ptr, nzero);
+  moe_route_kernel<<<1, 1024, sh, st>>>(ids, npairs, num_experts, offsets, pairs, segs, nseg, chunk, npairs_valid);
   note_launches(1);
   return cudaGetLastError();
 }
