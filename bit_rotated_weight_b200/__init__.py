@@ -111,7 +111,13 @@ class Packed:
     seed: int
 
     def c_struct(self) -> _Weight:
-        return _Weight(self.n, self.k, self.num_experts, 0, self.seed, self.codes.data_ptr(), self.scales.data_ptr())
+        # built once per (codes, scales) storage; a call only marshals a pointer to it
+        key = (self.codes.data_ptr(), self.scales.data_ptr(), self.n, self.k, self.num_experts, self.seed)
+        cached = self.__dict__.get("_c_struct")
+        if cached is None or cached[0] != key:
+            cached = (key, _Weight(self.n, self.k, self.num_experts, 0, self.seed, key[0], key[1]))
+            self.__dict__["_c_struct"] = cached
+        return cached[1]
 
     @property
     def nbytes(self) -> int:
@@ -211,8 +217,8 @@ def tq4_1s_linear(x: torch.Tensor, w: Packed, out: torch.Tensor | None = None,
     if out is None:
         out = torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device)
     wst = w.c_struct()
-    need = load_library().tq4_1s_linear_workspace(m, ctypes.byref(wst))
-    if workspace is None:
+    if workspace is None:   # (a caller's workspace is checked by the library)
+        need = load_library().tq4_1s_linear_workspace(m, ctypes.byref(wst))
         workspace = _workspace(need, x.device, "linear_small" if m <= SMALL_M else "linear_large")
     _check(load_library().tq4_1s_linear(_ptr(x), m, ctypes.byref(wst), _ptr(out), _ptr(workspace),
                                         workspace.numel(), _stream(x.device)), "linear")

@@ -157,13 +157,38 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
   return r == CUDA_SUCCESS;
 }
 
-// Codes plane [E][n][k/2] bytes, box 64 B x 128 rows, 64-byte swizzle.
+// Codes plane [E][n][k/2] bytes, box 64 B x 128 rows, 64-byte swizzle.  The
+// map depends only on the plane's address and shape, so recent ones are kept
+// (a weight used call after call is encoded once).
 static bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
+  struct Entry {
+    const void* ptr;
+    int64_t n, k;
+    int32_t e;
+    CUtensorMap map;
+  };
+  constexpr int kEntries = 64;
+  static std::mutex mu;
+  static Entry cache[kEntries];
+  static int next = 0;
+  {
+    std::lock_guard<std::mutex> g(mu);
+    for (int i = 0; i < kEntries; ++i)
+      if (cache[i].ptr == w->codes && cache[i].n == w->n && cache[i].k == w->k && cache[i].e == w->num_experts) {
+        *m = cache[i].map;
+        return true;
+      }
+  }
   const uint64_t dims[3] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n),
                             static_cast<uint64_t>(w->num_experts)};
   const uint64_t strides[2] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n * (w->k / 2))};
   const uint32_t box[3] = {64, 128, 1};
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+  if (!make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B))
+    return false;
+  std::lock_guard<std::mutex> g(mu);
+  cache[next] = Entry{w->codes, w->n, w->k, w->num_experts, *m};
+  next = (next + 1) % kEntries;
+  return true;
 }
 
 // x [rows][cols] (cols % 64 == 0) viewed as [cols/64][rows][64] 16-bit,

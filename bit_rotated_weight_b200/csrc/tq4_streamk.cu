@@ -990,11 +990,14 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const void* t
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
-  LevelTable lt;
-  const CodebookF32& cb = codebook();
-  for (int i = 0; i < 16; ++i)
-    lt.h[i] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(cb.levels[i] * kLevelScale)));
-  lt.max_level = __half2float(__float2half_rn(cb.levels[15] * kLevelScale));
+  static const LevelTable lt = [] {
+    LevelTable t;
+    const CodebookF32& cb = codebook();
+    for (int i = 0; i < 16; ++i)
+      t.h[i] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(cb.levels[i] * kLevelScale)));
+    t.max_level = __half2float(__float2half_rn(cb.levels[15] * kLevelScale));
+    return t;
+  }();
   const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
   const CUtensorMap& m1 = *static_cast<const CUtensorMap*>(tm_x);
   const CUtensorMap& m3 = *static_cast<const CUtensorMap*>(tm_x3 ? tm_x3 : tm_x);
