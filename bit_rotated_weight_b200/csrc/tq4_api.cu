@@ -157,57 +157,76 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
   return r == CUDA_SUCCESS;
 }
 
-// Codes plane [E][n][k/2] bytes, box 64 B x 128 rows, 64-byte swizzle.  The
-// map depends only on the plane's address and shape, so recent ones are kept
-// (a weight used call after call is encoded once).
-static bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
+// Tensor maps depend only on the address, shape and box they describe, so
+// recently encoded ones are kept: a weight, or an activation buffer, used
+// call after call is encoded once.
+struct MapKey {
+  int kind;
+  const void* ptr;
+  int64_t d0, d1, d2;
+  bool operator==(const MapKey& o) const {
+    return kind == o.kind && ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && d2 == o.d2;
+  }
+};
+
+template <typename Encode>
+static bool cached_map(CUtensorMap* m, const MapKey& key, Encode encode) {
   struct Entry {
-    const void* ptr;
-    int64_t n, k;
-    int32_t e;
+    MapKey key;
     CUtensorMap map;
   };
-  constexpr int kEntries = 64;
+  constexpr int kEntries = 128;
   static std::mutex mu;
   static Entry cache[kEntries];
-  static int next = 0;
+  static int used = 0, next = 0;
   {
     std::lock_guard<std::mutex> g(mu);
-    for (int i = 0; i < kEntries; ++i)
-      if (cache[i].ptr == w->codes && cache[i].n == w->n && cache[i].k == w->k && cache[i].e == w->num_experts) {
+    for (int i = 0; i < used; ++i)
+      if (cache[i].key == key) {
         *m = cache[i].map;
         return true;
       }
   }
-  const uint64_t dims[3] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n),
-                            static_cast<uint64_t>(w->num_experts)};
-  const uint64_t strides[2] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n * (w->k / 2))};
-  const uint32_t box[3] = {64, 128, 1};
-  if (!make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B))
-    return false;
+  if (!encode(m)) return false;
   std::lock_guard<std::mutex> g(mu);
-  cache[next] = Entry{w->codes, w->n, w->k, w->num_experts, *m};
+  cache[next] = Entry{key, *m};
   next = (next + 1) % kEntries;
+  if (used < kEntries) ++used;
   return true;
+}
+
+// Codes plane [E][n][k/2] bytes, box 64 B x 128 rows, 64-byte swizzle.
+static bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
+  return cached_map(m, MapKey{0, w->codes, w->n, w->k, w->num_experts}, [&](CUtensorMap* out) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n),
+                              static_cast<uint64_t>(w->num_experts)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n * (w->k / 2))};
+    const uint32_t box[3] = {64, 128, 1};
+    return make_map(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_64B);
+  });
 }
 
 // x [rows][cols] (cols % 64 == 0) viewed as [cols/64][rows][64] 16-bit,
 // box 64 x 32 x 2*kFusedMaxIters, 128-byte swizzle: one copy fills the B
 // tiles of all stages of a fused CTA.
 static bool map_x3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
-  const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / 64)};
-  const uint64_t strides[2] = {static_cast<uint64_t>(cols * 2), 128};
-  const uint32_t box[3] = {64, static_cast<uint32_t>(kSegRows), static_cast<uint32_t>(2 * kFusedMaxIters)};
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return cached_map(m, MapKey{1, base, rows, cols, 0}, [&](CUtensorMap* out) {
+    const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / 64)};
+    const uint64_t strides[2] = {static_cast<uint64_t>(cols * 2), 128};
+    const uint32_t box[3] = {64, static_cast<uint32_t>(kSegRows), static_cast<uint32_t>(2 * kFusedMaxIters)};
+    return make_map(out, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  });
 }
 
 // 16-bit matrix [rows][cols] row-major (bf16 or fp16), box 64 x box_rows,
 // 128-byte swizzle.
 static bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
-  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
-  const uint64_t strides[1] = {static_cast<uint64_t>(cols * 2)};
-  const uint32_t box[2] = {64, box_rows};
-  return make_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  return cached_map(m, MapKey{2, base, rows, cols, box_rows}, [&](CUtensorMap* out) {
+    const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+    const uint64_t strides[1] = {static_cast<uint64_t>(cols * 2)};
+    const uint32_t box[2] = {64, box_rows};
+    return make_map(out, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, base, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  });
 }
 
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -380,15 +399,16 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
   if (!aligned16(x) || !aligned16(y)) return TQ_ERR_ALIGNMENT;
   int sms = 0;
   if ((rc = check_device(&sms))) return rc;
-  const size_t need = tq4_1s_linear_workspace(m, w);
+  const bool small = m <= kSmallM;
+  const SmallLayout L = small ? small_layout(m, w, sms) : SmallLayout{};
+  const size_t need = small ? L.total : align256(static_cast<size_t>(w->n) * static_cast<size_t>(w->k) * 2);
   if (!ws || ws_bytes < need) return TQ_ERR_WORKSPACE;
   if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   const uint32_t mask = sign_mask_of(w->seed);
 
-  if (m <= kSmallM) {
-    const SmallLayout L = small_layout(m, w, sms);
+  if (small) {
     const int64_t T = L.tiles * ((w->k + 127) / 128);
     if (T > INT32_MAX) return TQ_ERR_INVALID_ARG;   // 32-bit iteration space
     // m <= 32 (one segment): cluster split-K when it fits in one wave, else
