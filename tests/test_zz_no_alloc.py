@@ -56,3 +56,28 @@ def test_static_scratch_linear_matches_workspace_linear():
     y40 = torch.empty((40, 4096), dtype=torch.bfloat16, device=dev)
     bst = big.c_struct()
     assert fn(ctypes.c_void_p(x40.data_ptr()), 40, ctypes.byref(bst), ctypes.c_void_p(y40.data_ptr()), stream) == 9
+
+
+@pytest.mark.parametrize("m,n,k,seed", [
+    (32, 8192, 8192, 60),   # too long per CTA for the fused modes: rotation kernel + TMA-fed stream-K
+    (7, 4096, 128, 61),     # one k iteration: fused stream-K without a cluster
+])
+def test_static_scratch_other_modes(m, n, k, seed):
+    dev = torch.device("cuda:0")
+    lib = tq.load_library()
+    fn = lib.tq4_1s_linear_static
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(tq._Weight), ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    W = torch.from_numpy(synth.normal_f32((n, k), seed, 0.02)).to(dev)
+    p = tq.tq4_1s_quantize(W, seed=seed)
+    wst = p.c_struct()
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    x = _to_dev(synth.activations_bf16(m, k, seed + 1), dev)
+    ref = tq.tq4_1s_linear(x, p)
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    rc = fn(ctypes.c_void_p(x.data_ptr()), m, ctypes.byref(wst), ctypes.c_void_p(y.data_ptr()), stream)
+    assert rc == 0, tq.tq4_1s_error_string(rc)
+    torch.cuda.synchronize()
+    ref_f = _bits(ref).astype(np.uint32) << 16
+    assert_close(_bits(y), ref_f.view(np.float32).astype(np.float64), f"static m={m} n={n} k={k}")
+    assert tq.tq4_1s_get_status() == 0
