@@ -17,6 +17,13 @@ buffers (e2e), SM clocks sampled during the timed region, and the roofline of
 the dominant kernel against MEASURED_PEAKS.json.
 
 Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                      [--workload decode|sweep]
+``--workload sweep`` times the 52-layer denoise-step weight sweep instead:
+52 layers, each a 128-expert top-6 MoE block (up 2688 -> 1856, down
+1856 -> 2688) plus dense 2688 -> 4096 and 4096 -> 2688 projections, on 512
+tokens (32 sequences x one 16-token block); 67.56 B weights, 42.22 GB packed,
+every expert active.  It reports packed-weight GB/s of the step and the
+quantize throughput of building the 52 layers.
 For N > 1 launch under torch.distributed.run; each rank runs an independent
 replica (the layer's work does not exchange data), reported as weak scaling.
 """
@@ -152,6 +159,8 @@ def reference_arm(args):
         return
     import oracle
     import synth
+    if args.workload == "sweep":
+        return reference_sweep(args)
     W = synth.student_t_f32((N_OUT, K_IN), 2, 5.0, 0.02)
     codes, scales, _ = oracle.quantize(W, 2)
     x = synth.activations_bf16(M_TOK, K_IN, 3)
@@ -168,6 +177,26 @@ def reference_arm(args):
             "config": {"workload": WORKLOAD, "sample": "each step is one of the 16 calls"},
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
                              "sample": f"{args.steps} single-threaded oracle calls (dequantize + fp64 GEMV)"},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def reference_sweep(args):
+    """The oracle on the sweep workload: each step is one bounded sample
+    (a 64-token slice of one dense projection, scaled to 512 tokens)."""
+    for _ in range(args.warmup):
+        sweep_cpu_sample(rows=8)
+    samples = [sweep_cpu_sample() for _ in range(args.steps)]
+    value = statistics.median(s["value"] for s in samples)
+    wl, _ = sweep_shapes()
+    ms_step = sweep_packed_bytes() / (value * 1e9) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": "denoise_sweep_52", "sample": samples[0]["sample"],
+                       "ms_per_step_note": "extrapolated from the sample's GB/s to the step's packed bytes"},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": 1, "kind": "oracle",
+                             "sample": samples[0]["sample"]},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
@@ -361,6 +390,213 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     return out
 
 
+# ------------------------------------------------------------------ denoise sweep
+def sweep_shapes():
+    """Per-layer tensors of the 52-layer sweep: [(name, shape)], weights [E][out][in] or [out][in]."""
+    import synth
+    wl = synth.WORKLOADS["denoise_sweep_52"]
+    E, H, I = wl["num_experts"], wl["hidden"], wl["inter"]
+    (n0, k0), (n1, k1) = wl["dense"]
+    return wl, [("up", (E, I, H)), ("down", (E, H, I)), ("dense_in", (n0, k0)), ("dense_out", (n1, k1))]
+
+
+def sweep_packed_bytes() -> int:
+    """Packed bytes of all 52 layers (codes at 4 bits + two fp16 scales per 32 weights)."""
+    wl, shapes = sweep_shapes()
+    per_layer = 0
+    for _, shp in shapes:
+        e = shp[0] if len(shp) == 3 else 1
+        n, k = shp[-2], shp[-1]
+        per_layer += e * (n * k // 2 + n * (k // 16) * 2)
+    return wl["layers"] * per_layer
+
+
+def sweep_weights() -> int:
+    wl, shapes = sweep_shapes()
+    total = 0
+    for _, shp in shapes:
+        c = 1
+        for d in shp:
+            c *= d
+        total += c
+    return wl["layers"] * total
+
+
+def sweep_cpu_sample(rows: int = 64):
+    """The oracle on a bounded sample of the sweep: layer 0's dense
+    hidden -> 4096 projection on ``rows`` of the 512 tokens, scaled to the
+    512-token step (the oracle's work is linear in the token count)."""
+    import oracle
+    import synth
+    wl, shapes = sweep_shapes()
+    n, k = shapes[2][1]
+    seed = synth.sweep_seed(0, 2)
+    W = synth.normal_f32((n, k), seed, wl["w_std"])
+    codes, scales, _ = oracle.quantize(W, seed)
+    x = synth.activations_bf16(rows, k, synth.sweep_seed(0, 4))
+    t0 = time.perf_counter()
+    oracle.linear(x, codes, scales, seed)
+    el = time.perf_counter() - t0
+    packed = n * k // 2 + n * (k // 16) * 2
+    gbs = packed / (el * wl["m"] / rows) / 1e9
+    return {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle",
+            "sample": f"dequantize + fp64 linear of one {n}x{k} weight on {rows} of {wl['m']} tokens in "
+                      f"{el:.2f} s, single thread, scaled x{wl['m'] // rows} to the 512-token step"}
+
+
+def sweep_arm(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import bit_rotated_weight_b200 as tq
+    import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+    pk = peaks()
+    wl, shapes = sweep_shapes()
+    L, m, topk, E, H = wl["layers"], wl["m"], wl["topk"], wl["num_experts"], wl["hidden"]
+    n_mid = wl["dense"][0][0]
+
+    # ---- build: weights drawn on the device per layer (not timed), quantized
+    # (timed with events on the launching stream)
+    layers = []
+    q_events = []
+    for l in range(L):
+        packed = {}
+        for j, (name, shp) in enumerate(shapes):
+            seed = synth.sweep_seed(l, j)
+            W = synth.normal_f32_device(shp, seed, wl["w_std"], dev)
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record()
+            packed[name] = tq.tq4_1s_quantize(W, seed=seed)
+            e1.record()
+            q_events.append((e0, e1))
+            del W
+        ids, w = synth.gumbel_topk_router(m, E, topk, synth.sweep_seed(l, 5))
+        x = synth.activations_bf16(m, H, synth.sweep_seed(l, 4))
+        packed["touched"] = len(set(ids.ravel().tolist()))
+        packed["ids"] = torch.from_numpy(ids).to(dev)
+        packed["w"] = torch.from_numpy(w).to(dev)
+        packed["x"] = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
+        layers.append(packed)
+    torch.cuda.synchronize()
+    q_ms = sum(a.elapsed_time(b) for a, b in q_events)
+    n_weights = sweep_weights()
+    torch.cuda.empty_cache()
+
+    per_expert = layers[0]["up"].nbytes // E + layers[0]["down"].nbytes // E
+    step_bytes = sum(ly["touched"] * per_expert + ly["dense_in"].nbytes + ly["dense_out"].nbytes for ly in layers)
+    y_moe = torch.empty((m, H), dtype=torch.bfloat16, device=dev)
+    t_mid = torch.empty((m, n_mid), dtype=torch.bfloat16, device=dev)
+    y_out = torch.empty((m, H), dtype=torch.bfloat16, device=dev)
+    ws_moe = torch.empty(tq.tq4_1s_moe_workspace(m, topk, layers[0]["up"], layers[0]["down"]),
+                         dtype=torch.uint8, device=dev)
+    ws_lin = torch.empty(max(tq.tq4_1s_linear_workspace(m, layers[0]["dense_in"]),
+                             tq.tq4_1s_linear_workspace(m, layers[0]["dense_out"])), dtype=torch.uint8, device=dev)
+
+    def step(i, xs=None):
+        # one denoise step: every layer's MoE block and its two dense
+        # projections (the second consumes the first's output)
+        for l, ly in enumerate(layers):
+            x = ly["x"] if xs is None else xs[l]
+            tq.tq4_1s_moe(x, ly["ids"], ly["w"], ly["up"], ly["down"], out=y_moe, workspace=ws_moe)
+            tq.tq4_1s_linear(x, ly["dense_in"], out=t_mid, workspace=ws_lin)
+            tq.tq4_1s_linear(t_mid, ly["dense_out"], out=y_out, workspace=ws_lin)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert tq.tq4_1s_get_status() == 0, "device status word set during warm-up"
+
+    def timed(fn, k):
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for i in range(k):
+            fn(i)
+        e1.record()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        return max_over_ranks(e0.elapsed_time(e1))
+
+    clocks = ClockSampler(local)
+    clocks.start()
+    time.sleep(0.3)
+    l0 = tq.tq4_1s_launch_count()
+    ms = timed(step, args.steps)
+    launches = tq.tq4_1s_launch_count() - l0
+    clk = clocks.stop()
+    assert tq.tq4_1s_get_status() == 0, "device status word set during the timed region"
+    ms_step = ms / args.steps
+    value = job_gbs(world, step_bytes, ms_step)
+    achieved = step_bytes / (ms_step * 1e-3) / 1e9
+
+    # ---- end to end: each step's per-layer input blocks come from pinned
+    # host memory; the last layer's two outputs go back to it
+    x_host = [ly["x"].view(torch.int16).cpu().pin_memory() for ly in layers]
+    x_dev = [torch.empty_like(ly["x"]) for ly in layers]
+    y_host = [torch.empty((m, H), dtype=torch.int16).pin_memory() for _ in range(2)]
+
+    def e2e_step(i):
+        for xh, xd in zip(x_host, x_dev):
+            xd.view(torch.int16).copy_(xh, non_blocking=True)
+        step(i, x_dev)
+        y_host[0].copy_(y_moe.view(torch.int16), non_blocking=True)
+        y_host[1].copy_(y_out.view(torch.int16), non_blocking=True)
+
+    e2e_step(0)
+    ke = max(3, args.steps // 2)
+    e2e_ms = timed(e2e_step, ke) / ke
+    e2e = {"value": job_gbs(world, step_bytes, e2e_ms), "unit": "GB/s",
+           "h2d_bytes_per_step": sum(t.numel() * 2 for t in x_host),
+           "d2h_bytes_per_step": sum(t.numel() * 2 for t in y_host), "ms_per_step": e2e_ms}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        cpu = sweep_cpu_sample() if world == 1 else None
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp16", "data": "synthetic",
+            "config": {"workload": f"denoise_sweep_52: {L} layers x (MoE 128 experts top-6, up {H}->"
+                                   f"{wl['inter']}, down {wl['inter']}->{H}; dense {H}->{n_mid}->{H}), "
+                                   f"{m} tokens (32 sequences x 16-token block) per step",
+                       "global_batch": world * m, "seq_len": 16, "parallelism": f"replicas x{world}",
+                       "timing": "eager calls, one step = all layers",
+                       "l2": f"cold: {step_bytes / 1e9:.2f} GB of packed weights streamed per step (> 126 MB L2)",
+                       "weights": f"{n_weights / 1e9:.2f} B weights, N(0, 0.02^2) drawn on the device per layer"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
+                         "frac": achieved / pk["hbm_gbs"], "traffic": None,
+                         "algorithmic_bytes": step_bytes,
+                         "kernel": "whole step (MoE route, rotations, grouped stream-K up/down, combine; "
+                                   "dense dequantize pre-pass + tcgen05 GEMM), packed bytes per step / step time",
+                         "peak_source": pk["source"]},
+            "quantize": {"weights_per_s": n_weights / (q_ms * 1e-3), "ms_total": q_ms,
+                         "gbs": n_weights * 4.625 / (q_ms * 1e-3) / 1e9,
+                         "bytes_per_weight": "4 read (fp32) + 0.625 written (packed)",
+                         "note": "device time of the 208 quantize calls; weight generation not timed"},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "clocks": clk,
+            "gpu_launches": launches,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+
+
 def profile_arm(args):
     """Eager calls of one workload for ncu captures (no graphs, no oracle).
 
@@ -416,6 +652,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-secondary", action="store_true")
+    ap.add_argument("--workload", choices=["decode", "sweep"], default="decode",
+                    help="decode: the 16-token decode linear (default); sweep: the 52-layer denoise step")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -423,6 +661,8 @@ def main():
         profile_arm(args)
     elif args.impl == "reference":
         reference_arm(args)
+    elif args.workload == "sweep":
+        sweep_arm(args)
     else:
         ours_arm(args)
 

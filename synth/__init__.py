@@ -21,7 +21,7 @@ import numpy as np
 
 __all__ = [
     "rng", "normal_f32", "student_t_f32", "f32_to_bf16_bits", "bf16_bits_to_f32",
-    "activations_bf16", "gumbel_topk_router", "WORKLOADS",
+    "activations_bf16", "gumbel_topk_router", "normal_f32_device", "sweep_seed", "WORKLOADS",
 ]
 
 
@@ -85,6 +85,32 @@ def gumbel_topk_router(m: int, num_experts: int, topk: int, seed: int):
     return order.astype(np.int32), w.astype(np.float32)
 
 
+def normal_f32_device(shape, seed: int, std: float, device):
+    """i.i.d. N(0, std^2) float32 drawn on a CUDA device by torch's Philox
+    generator keyed by ``seed``.
+
+    For tensors too large to draw on the host in reasonable time (a
+    128-expert stack is 638M weights).  Deterministic for a given seed, shape
+    and device type; a different stream from :func:`normal_f32` with the same
+    seed."""
+    import torch
+    g = torch.Generator(device=device)
+    g.manual_seed(int(seed))
+    return torch.randn(tuple(shape), generator=g, device=device, dtype=torch.float32).mul_(std)
+
+
+def sweep_seed(layer: int, tensor: int) -> int:
+    """Seed of one tensor of layer ``layer`` of the 52-layer denoise sweep.
+
+    tensor: 0 up-projection stack, 1 down-projection stack, 2 dense
+    hidden -> 4096 weight, 3 dense 4096 -> hidden weight, 4 activations of the
+    MoE and first dense projection, 5 router, 6 activations of the second
+    dense projection.  The RHT seed of each weight equals its seed here."""
+    if not (0 <= tensor < 8):
+        raise ValueError("tensor index must be in [0, 8)")
+    return WORKLOADS["denoise_sweep_52"]["seed_base"] + 8 * int(layer) + int(tensor)
+
+
 # Seeds and shapes of the five workloads.  The RHT seed of each quantized
 # tensor equals the seed its weights were drawn with.
 WORKLOADS = {
@@ -95,5 +121,6 @@ WORKLOADS = {
                           x_seed=6, router_seed=7, w_std=0.02),
     "prefill_linear_8192": dict(n=14336, k=4096, m=8192, w_seed=8, x_seed=9, w_dist="normal", w_std=0.02),
     "denoise_sweep_52": dict(layers=52, m=512, steps=16, num_experts=128, hidden=2688, inter=1856, topk=6,
-                             dense=((2688, 4096), (4096, 2688)), seed_base=1000, w_std=0.02),
+                             # dense weights as [out][in]: hidden -> 4096, then 4096 -> hidden
+                             dense=((4096, 2688), (2688, 4096)), seed_base=1000, w_std=0.02),
 }
