@@ -1,0 +1,224 @@
+"""Thread roles and named barriers of the tcgen05 kernels, checked on the CPU.
+
+A named barrier (``bar.sync id, count``) cannot time out: if more or fewer
+threads than ``count`` reach it, the block hangs.  These tests read the
+kernels' own source, evaluate their compile-time constants and the role
+dispatch conditions for every thread of the block, and check that:
+  * every thread takes at most one role of the dispatch chain;
+  * each ``named_bar_sync(id, count)`` is reached by exactly ``count``
+    threads -- those of the role (or prologue) block that contains it;
+  * MMA issuers are one thread per dequant group, mapped one to one;
+  * the shared-memory table fill covers every entry exactly once.
+The conditions are taken from the source text, so a change to the dispatch
+is checked as it stands."""
+import os
+import re
+
+import pytest
+
+CSRC = os.path.join(os.path.dirname(__file__), "..", "bit_rotated_weight_b200", "csrc")
+
+
+def _read(name):
+    with open(os.path.join(CSRC, name)) as f:
+        return f.read()
+
+
+_CONST = re.compile(r"^\s*constexpr int (\w+) = ([^;]+);", re.M)
+_SAFE = re.compile(r"^[\w\s+\-*/()]+$")
+
+
+def _constants(*sources):
+    env = {}
+    for src in sources:
+        for name, expr in _CONST.findall(src):
+            expr = expr.split("//")[0].strip()
+            if not _SAFE.match(expr):
+                continue
+            try:
+                env[name] = int(eval(expr.replace("/", "//"), {"__builtins__": {}}, dict(env)))
+            except (NameError, SyntaxError):
+                pass
+    return env
+
+
+def _to_py(cond):
+    cond = cond.replace("&&", " and ").replace("||", " or ")
+    assert "!" not in cond.replace("!=", ""), cond
+    return cond
+
+
+def _kernel_lines(src, marker):
+    """Lines of the kernel whose definition starts at ``marker`` (up to the
+    closing brace at column 0)."""
+    lines = src.splitlines()
+    start = next(i for i, l in enumerate(lines) if marker in l)
+    end = next(i for i in range(start + 1, len(lines)) if lines[i].startswith("}"))
+    return lines, start, end
+
+
+_TOP_IF = re.compile(r"^  if \((.*)\) \{\s*$")
+_TOP_ELSE_IF = re.compile(r"^  \} else if \((.*)\) \{\s*$")
+
+
+def _dispatch(lines, start, end):
+    """(head line, [(line, condition)]) of the role chain: the last top-level
+    ``if (...) {`` before the first top-level ``} else if``, and its arms."""
+    first_else = next(i for i in range(start, end) if _TOP_ELSE_IF.match(lines[i]))
+    head = max(i for i in range(start, first_else) if _TOP_IF.match(lines[i]))
+    arms = [(head, _TOP_IF.match(lines[head]).group(1))]
+    i = head + 1
+    while i < end:
+        m = _TOP_ELSE_IF.match(lines[i])
+        if m:
+            arms.append((i, m.group(1)))
+        elif lines[i].startswith("  }") and not lines[i].startswith("  } else"):
+            return arms, i
+        i += 1
+    raise AssertionError("role chain not closed")
+
+
+def _role_of(arms, env, warp, lane, fused):
+    for idx, (_, cond) in enumerate(arms):
+        if eval(_to_py(cond), {"__builtins__": {}}, dict(env, warp=warp, lane=lane, fused=fused)):
+            return idx
+    return None
+
+
+def _block_end(lines, i):
+    """End line of the top-level block opened at line i."""
+    for j in range(i + 1, len(lines)):
+        if lines[j].startswith("  }"):
+            return j
+    raise AssertionError
+
+
+_BAR = re.compile(r"named_bar_sync\(([^,()]+),\s*([^()]+)\)")
+
+
+def _eval_int(expr, env):
+    assert _SAFE.match(expr), expr
+    return int(eval(expr.replace("/", "//"), {"__builtins__": {}}, dict(env)))
+
+
+def _check_kernel(src_name, marker, extra_sources=(), fused_values=(False, True)):
+    src = _read(src_name)
+    env = _constants(*[_read(s) for s in extra_sources], src)
+    threads = env["kThreads"]
+    assert threads % 32 == 0 and threads <= 1024
+    lines, start, end = _kernel_lines(src, marker)
+    assert "__launch_bounds__(kThreads" in lines[start]
+    arms, chain_end = _dispatch(lines, start, end)
+    # other top-level conditional blocks (set-up, prologue)
+    blocks = [(i, _TOP_IF.match(lines[i]).group(1), _block_end(lines, i))
+              for i in range(start, end) if _TOP_IF.match(lines[i]) and i != arms[0][0]]
+    bars = [(i, m.group(1), m.group(2)) for i in range(start, end) for m in _BAR.finditer(lines[i])]
+    assert bars, "no named barriers found"
+    for fused in fused_values:
+        roles = {}
+        for tid in range(threads):
+            r = _role_of(arms, env, tid // 32, tid % 32, fused)
+            roles.setdefault(r, []).append(tid)
+        for line, bar_id, bar_cnt in bars:
+            cnt = _eval_int(bar_cnt, env)
+            assert _eval_int(bar_id, env) != 0, "barrier 0 is __syncthreads"
+            # innermost enclosing block: a chain arm or another top-level block
+            arm = max((k for k, (l0, _) in enumerate(arms) if l0 < line), default=None)
+            in_chain = arm is not None and line < chain_end
+            if in_chain:
+                n = len(roles.get(arm, []))
+            else:
+                enclosing = [b for b in blocks if b[0] < line < b[2]]
+                assert enclosing, f"{src_name}:{line + 1} named barrier outside any role block"
+                l0, cond, _ = max(enclosing)
+                n = sum(1 for tid in range(threads)
+                        if eval(_to_py(cond), {"__builtins__": {}},
+                                dict(env, warp=tid // 32, lane=tid % 32, fused=fused)))
+                if n == 0:
+                    continue   # the block does not run in this mode
+            assert n == cnt, (f"{src_name}:{line + 1}: named_bar_sync({bar_id}, {bar_cnt}) "
+                              f"reached by {n} threads (fused={fused})")
+    return env, arms, lines
+
+
+def test_streamk_roles_and_named_barriers():
+    env, arms, lines = _check_kernel("tq4_streamk.cu", "__launch_bounds__(kThreads, 1)",
+                                     extra_sources=("tq4_internal.h",))
+    # role sizes: producer warp, 4 dequant groups of 128 rows, one issuer per
+    # group, 128 epilogue threads (one per tensor-memory lane)
+    counts = {}
+    for tid in range(env["kThreads"]):
+        r = _role_of(arms, env, tid // 32, tid % 32, True)
+        counts[r] = counts.get(r, 0) + 1
+    assert len(arms) == 4
+    assert counts[0] == 32
+    assert counts[1] == 128 * env["kDequantGroups"]
+    assert counts[2] == env["kDequantGroups"]
+    assert counts[3] == 128
+
+
+def test_streamk_issuers_map_one_to_one_onto_groups():
+    src = _read("tq4_streamk.cu")
+    env = _constants(_read("tq4_internal.h"), src)
+    m = re.search(r"int issuer_group\(int warp\) \{ return (.*?); \}", src)
+    assert m, "issuer_group not found"
+    expr = m.group(1)
+    # C conditional -> Python
+    c = re.match(r"(.*?) \? (.*?) : (.*)", expr)
+    issuers = [w for w in range(env["kThreads"] // 32) if w == 1 or w >= env["kFirstIssuerWarp"]]
+    groups = [eval(c.group(2) if eval(c.group(1), {}, dict(env, warp=w)) else c.group(3), {}, dict(env, warp=w))
+              for w in issuers]
+    assert sorted(groups) == list(range(env["kDequantGroups"]))
+
+
+def test_streamk_prologue_barrier_and_arrivals():
+    src = _read("tq4_streamk.cu")
+    env = _constants(_read("tq4_internal.h"), src)
+    # the prologue's mbarrier expects one arrival per prologue warp (lane 0)
+    assert "mbar_init(&sh.xready, kPrologueThreads / 32);" in src
+    assert "if (lane == 0) mbar_arrive(&sh.xready);" in src
+    assert env["kPrologueThreads"] % 32 == 0
+    warps = [w for w in range(env["kThreads"] // 32)
+             if env["kFirstDequantWarp"] <= w < env["kFirstEpilogueWarp"] + 4]
+    assert len(warps) * 32 == env["kPrologueThreads"]
+
+
+def test_streamk_table_fill_covers_each_entry_once():
+    src = _read("tq4_streamk.cu")
+    env = _constants(_read("tq4_internal.h"), src)
+    m = re.search(r"for \(int i = threadIdx\.x - (\d+); warp >= (\d+) && i < ([\w *]+); i \+= kThreads - (\d+)\)", src)
+    assert m, "table fill loop not found"
+    off, wmin, lim, step_off = int(m.group(1)), int(m.group(2)), eval(m.group(3), {}, env), int(m.group(4))
+    seen = {}
+    for tid in range(env["kThreads"]):
+        if tid // 32 < wmin:
+            continue
+        i = tid - off
+        while i < lim:
+            seen[i] = seen.get(i, 0) + 1
+            i += env["kThreads"] - step_off
+    assert sorted(seen) == list(range(lim)) and set(seen.values()) == {1}
+    assert lim * 4 == env["kLutBytes"]
+
+
+def test_streamk_shared_memory_and_tensor_memory_budgets():
+    env = _constants(_read("tq4_internal.h"), _read("tq4_streamk.cu"))
+    smem = env["kStages"] * (env["kCodesBytes"] + env["kXBytes"]) + env["kLutBytes"]
+    assert smem + 1024 <= 227 * 1024
+    # cluster split-K: the owner CTA's reduction buffer (codes of the stages
+    # fused mode never loads) holds s partials of 32 token rows x ceil(128/s)
+    # weight rows, for every split s in [2, 8]
+    assert env["kRedOff"] == env["kFusedMaxIters"] * env["kCodesBytes"]
+    room = env["kStages"] * env["kCodesBytes"] - env["kRedOff"]
+    for s in range(2, 9):
+        assert s * env["kSegRows"] * (-(-128 // s)) * 4 <= room
+    assert env["kTmemCols"] <= 512
+
+
+def test_gemm_roles_and_named_barriers():
+    env, arms, _ = _check_kernel("tq4_gemm.cu", "__launch_bounds__(kThreads, 1)", fused_values=(False,))
+    counts = {}
+    for tid in range(env["kThreads"]):
+        r = _role_of(arms, env, tid // 32, tid % 32, False)
+        counts[r] = counts.get(r, 0) + 1
+    assert counts[len(arms) - 1] == 128   # epilogue: one thread per tensor-memory lane
