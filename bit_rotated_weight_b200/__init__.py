@@ -242,8 +242,8 @@ def tq4_1s_moe(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, up
     if out is None:
         out = torch.empty((m, up.k), dtype=torch.bfloat16, device=x.device)
     u, d = up.c_struct(), down.c_struct()
-    need = load_library().tq4_1s_moe_workspace(m, topk, ctypes.byref(u), ctypes.byref(d))
-    if workspace is None:
+    if workspace is None:   # (a caller's workspace is checked by the library)
+        need = load_library().tq4_1s_moe_workspace(m, topk, ctypes.byref(u), ctypes.byref(d))
         workspace = _workspace(need, x.device, "moe")
     _check(load_library().tq4_1s_moe(_ptr(x), m, _ptr(topk_ids), _ptr(topk_w), topk, ctypes.byref(u),
                                      ctypes.byref(d), _ptr(out), _ptr(workspace), workspace.numel(),
