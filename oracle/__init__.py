@@ -16,6 +16,10 @@ listed at the top of the C file.  Parity status of each function:
   experts) and composition with the pinned linear; the squared-ReLU and the
   bf16 rounding of the hidden activation are fixed by the workload
   definition, not by the pages.
+- boundary_near (which code and scale decisions lie within 1e-6 of a
+  threshold or of an fp16 rounding midpoint; a reporting aid beside the
+  bit-exact comparison): pinned by constructed blocks that land exactly on a
+  threshold and on a midpoint, and by perturbed-decision containment.
 - reconstruction cosine 0.997 quoted on the model card for real weights:
   parity unpinned (real weights are not available; synthetic weights are
   checked against the >= 0.99 bound instead).
@@ -156,6 +160,60 @@ def quantize(W, seed: int):
     scales = np.zeros((n, k // HALF), np.uint16)
     bad = _load().orc_quantize(_ptr(W), n, k, seed, _ptr(codes), _ptr(scales))
     return codes, scales, int(bad)
+
+
+def unpack_codes(codes) -> np.ndarray:
+    """codes plane [n][k/2] -> one code per element [n][k] (even k in the low nibble)."""
+    codes = _c(codes, np.uint8)
+    out = np.empty((codes.shape[0], codes.shape[1] * 2), np.uint8)
+    out[:, 0::2] = codes & 0x0F
+    out[:, 1::2] = codes >> 4
+    return out
+
+
+def boundary_near(W, seed: int, scales=None, tol: float = 1e-6):
+    """Which quantization decisions of W sit within ``tol`` of a boundary.
+
+    Two correct fp32 implementations of the quantizer may disagree only on
+    these, so parity of codes and scales is exact everywhere else and the
+    count here is what gets reported beside it.  Computed in fp64 from the
+    definition (explicit Hadamard matrix, not the butterfly): with v = R w
+    per 32-block (r = fp32(1/sqrt(32))) and d the stored fp16 scale of the
+    half block, a code is near when min_j |v/d - t32_j| <= tol; a half-block
+    scale is near when the fp64 RMS of its 16 rotated values lies within
+    ``tol`` (relative) of the midpoint between the two fp16 values around it.
+
+    Returns {"codes": count, "scales": count, "code_mask": bool [n][k],
+    "scale_mask": bool [n][k/16]}."""
+    W = _c(W, np.float32)
+    n, k = W.shape
+    assert k % BLOCK == 0
+    if scales is None:
+        _, scales, _ = quantize(W, seed)
+    mask = sign_mask(seed)
+    s = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(BLOCK)])
+    H = hadamard32().astype(np.float64)
+    r = float(np.float32(1.0 / np.sqrt(32.0)))
+    v = (W.astype(np.float64).reshape(-1, BLOCK) * s) @ H.T * r          # [blocks][32]
+    vh = v.reshape(-1, HALF)                                              # [halves][16]
+    d = _c(scales, np.uint16).reshape(-1).view(np.float16).astype(np.float64)
+    _, _, _, t32 = codebook()
+    t = t32.astype(np.float64)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        u = vh / d[:, None]
+    idx = np.clip(np.searchsorted(t, u), 1, len(t) - 1)
+    dist = np.minimum(np.abs(u - t[idx - 1]), np.abs(u - t[idx]))
+    code_near = (d[:, None] > 0) & np.isfinite(u) & (dist <= tol)
+    rms = np.sqrt(np.mean(vh * vh, axis=1))
+    h = rms.astype(np.float16)
+    lo = np.where(h.astype(np.float64) > rms, np.nextafter(h, np.float16(-np.inf)), h)
+    hi = np.nextafter(lo, np.float16(np.inf))
+    mid = (lo.astype(np.float64) + hi.astype(np.float64)) / 2.0
+    scale_near = (rms > 0) & (rms < 65504.0) & (np.abs(rms - mid) <= tol * rms)
+    code_mask = code_near.reshape(n, k)
+    scale_mask = scale_near.reshape(n, k // HALF)
+    return {"codes": int(code_mask.sum()), "scales": int(scale_mask.sum()),
+            "code_mask": code_mask, "scale_mask": scale_mask}
 
 
 def dequantize(codes, scales, seed: int) -> np.ndarray:

@@ -49,8 +49,19 @@ def test_quantize_bit_exact(shape, seed, dist):
     W = (synth.normal_f32(shape, seed, 0.02) if dist == "normal"
          else synth.student_t_f32(shape, seed, 5.0, 0.02))
     p, codes, scales, _ = _quantize_both(W, seed)
-    assert np.array_equal(p.codes.cpu().numpy(), codes)
-    assert np.array_equal(p.scales.cpu().numpy().view(np.uint16), scales)
+    g_codes = p.codes.cpu().numpy()
+    g_scales = p.scales.cpu().numpy().view(np.uint16)
+    # both sides take every decision in fp32 with the same operation order,
+    # so codes and scales match bit for bit; the decisions within 1e-6 of a
+    # threshold or of an fp16 rounding midpoint are counted and reported
+    k = W.shape[-1]
+    near = oracle.boundary_near(W.reshape(-1, k), seed, scales.reshape(-1, k // 16))
+    n_code = int((oracle.unpack_codes(g_codes.reshape(-1, k // 2)) != oracle.unpack_codes(codes.reshape(-1, k // 2))).sum())
+    n_scale = int((g_scales != scales).sum())
+    print(f"quantize {shape}: {n_code} codes, {n_scale} scales differ; within 1e-6 of a boundary: "
+          f"{near['codes']} codes, {near['scales']} scales")
+    assert np.array_equal(g_codes, codes)
+    assert np.array_equal(g_scales, scales)
     assert tq.tq4_1s_get_status() == 0
 
 

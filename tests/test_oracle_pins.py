@@ -346,3 +346,69 @@ def test_moe_composes_linear_relu2_and_slot_sum():
             ref[t] += float(w[t, j]) * z[0]
     assert np.array_equal(y, ref)
     assert np.array_equal(yb, oracle.round_bf16(ref))
+
+
+# ----------------------------------------------------------- boundary-near count
+def _rotate_inverse_f64(v, seed):
+    """w with R w = v for one 32-block (R = r H diag(s), exact inverse in fp64)."""
+    mask = oracle.sign_mask(seed)
+    s = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(32)])
+    H = oracle.hadamard32().astype(np.float64)
+    r = float(np.float32(1.0 / np.sqrt(32.0)))
+    return s * (H @ np.asarray(v, np.float64)) / (32.0 * r)
+
+
+def test_boundary_near_explains_every_fp32_fp64_code_difference():
+    # codes taken in fp64 from the definition (explicit H, exact division)
+    # against the stored scale may differ from the oracle's fp32 codes only
+    # where the count flags a decision within 1e-6 of a threshold
+    W = synth.student_t_f32((512, 1024), 91, 5.0, 0.02)
+    codes, scales, _ = oracle.quantize(W, 91)
+    near = oracle.boundary_near(W, 91, scales)
+    mask = oracle.sign_mask(91)
+    s = np.array([-1.0 if (mask >> i) & 1 else 1.0 for i in range(32)])
+    H = oracle.hadamard32().astype(np.float64)
+    r = float(np.float32(1.0 / np.sqrt(32.0)))
+    v = ((W.astype(np.float64).reshape(-1, 32) * s) @ H.T * r).reshape(-1, 16)
+    d = scales.reshape(-1).view(np.float16).astype(np.float64)
+    _, _, _, t32 = oracle.codebook()
+    u = v / d[:, None]
+    ideal = (u[:, :, None] > t32.astype(np.float64)[None, None, :]).sum(axis=2).reshape(W.shape)
+    diff = ideal != oracle.unpack_codes(codes)
+    assert not np.any(diff & ~near["code_mask"])
+    assert near["codes"] < 1e-4 * W.size
+    # the mask marks the right elements: scaling u by (1 + 1e-4) moves a code
+    # only where u was within |t_j| * 1e-4 <= 2.5e-4 of threshold t_j, so every
+    # moved code lies inside the mask taken at tol = 3e-4 (and some do move)
+    wide = oracle.boundary_near(W, 91, scales, tol=3e-4)
+    moved = ((u * (1 + 1e-4))[:, :, None] > t32.astype(np.float64)[None, None, :]).sum(axis=2).reshape(W.shape)
+    moved = moved != ideal
+    assert moved.sum() >= 10
+    assert not np.any(moved & ~wide["code_mask"])
+    assert wide["codes"] < 20 * moved.sum()
+
+
+def test_boundary_near_flags_a_value_on_a_threshold_and_a_scale_on_a_midpoint():
+    seed = 5
+    _, _, _, t32 = oracle.codebook()
+    D = 1.5   # an fp16 value: the stored scale of the first half
+    tj = float(t32[11])
+    a = D * np.sqrt((16.0 - tj * tj) / 15.0)
+    v = np.empty(32)
+    v[0] = tj * D                       # u = t_11 exactly
+    v[1:16] = a                         # half-block RMS exactly D
+    M = 1.0 + 2.0 ** -11                # midpoint of fp16 1.0 and 1 + 2^-10
+    v[16:32] = M                        # second half: RMS exactly on a midpoint
+    W = _rotate_inverse_f64(v, seed).astype(np.float32).reshape(1, 32)
+    codes, scales, _ = oracle.quantize(W, seed)
+    assert scales[0, 0] == np.float16(D).view(np.uint16)
+    near = oracle.boundary_near(W, seed, scales)
+    assert near["code_mask"][0, 0] and near["codes"] == 1
+    assert near["scale_mask"][0, 1] and not near["scale_mask"][0, 0] and near["scales"] == 1
+    # nudged off the boundaries, nothing is flagged
+    v[0] = float(t32[11] + t32[12]) / 2 * D
+    v[1:16] = D * np.sqrt((16.0 - (v[0] / D) ** 2) / 15.0)
+    v[16:32] = 1.0 + 2.0 ** -12
+    W = _rotate_inverse_f64(v, seed).astype(np.float32).reshape(1, 32)
+    near = oracle.boundary_near(W, seed)
+    assert near["codes"] == 0 and near["scales"] == 0
