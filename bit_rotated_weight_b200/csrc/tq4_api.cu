@@ -243,8 +243,9 @@ struct SmallLayout {
 
 // Small-m workspace: the rotated activations (fp16, per-row scales; unused
 // when the kernel rotates x itself), the stream-K fp32
-// partials and the tile counters.  Counters carry the launch's epoch, so the
-// workspace needs no initialisation.
+// partials and the tile counters.  Counters carry the launch's epoch and the
+// last arriver of each split tile resets its counter, so the workspace needs
+// no initialisation and a captured call can be replayed.
 static SmallLayout small_layout(int64_t m, const tq4_1s_weight* w, int sms) {
   SmallLayout L{};
   const int64_t nseg = (m + kSegRows - 1) / kSegRows;

@@ -833,7 +833,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       // arriver's acquire orders its reads of the others' partials after it.
       // A counter holds (epoch << 32) | arrivals: a value left by another
       // launch (another epoch) counts as zero arrivals, so the counters never
-      // need clearing.
+      // need clearing; the last arriver resets its counter to zero, which
+      // covers a later launch with the same epoch (a graph replay).
       named_bar_sync(1, 128);
       const int c_first = owner_of(tile_first, T, G);
       const int c_last = owner_of(tile_first + KI - 1, T, G);
@@ -854,7 +855,14 @@ __global__ void __launch_bounds__(kThreads, 1)
           cur = prev;
         }
         if (!done) raise_status(TQ_DEV_TIMEOUT);
-        sh.last_flag = (done && (want & 0xFFFFFFFFull) == ncontrib) ? 1 : 0;
+        const bool last = done && (want & 0xFFFFFFFFull) == ncontrib;
+        // After the last arrival no CTA of this launch touches the counter
+        // again, so it is reset: a launch that reuses this epoch (a CUDA graph
+        // replays its kernels with the arguments they were captured with)
+        // then counts from zero.  The next launch reads the counter only after
+        // this grid has completed (stream order, or its dependent-launch wait).
+        if (last) *reinterpret_cast<volatile unsigned long long*>(ctr) = 0ull;
+        sh.last_flag = last ? 1 : 0;
       }
       named_bar_sync(1, 128);
       if (sh.last_flag) {

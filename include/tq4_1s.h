@@ -126,8 +126,10 @@ int tq4_1s_dequantize(const tq4_1s_weight* w, float* W_out, tq4_stream_t stream)
  * num_experts == 1).  0 on invalid arguments.
  * Small m (<= 128): the workspace holds the rotated activations, the
  * stream-K partial sums and the tile counters; large m: the bf16 dequantized
- * weight.  No initialisation is needed (each call clears what it uses), but
- * calls that share a workspace must not overlap on the GPU. */
+ * weight.  No initialisation is needed: the tile counters carry each launch's
+ * epoch and the launch that finishes a split tile resets its counter, so a
+ * call may also be captured into a CUDA graph and replayed.  Calls that
+ * share a workspace must not overlap on the GPU. */
 size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
 
 /* The quantized linear layer of "Running it": y[m][n] = bf16(x * W_hat^T),
@@ -169,7 +171,8 @@ int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t
  *   All calls share the one array, so calls that overlap on the GPU (on
  *   different streams, or from different host threads) race and corrupt each
  *   other's results; serialize them.  Each launch tags the tile counters
- *   it uses with its own epoch, so a previous call's leftovers do no harm.
+ *   it uses with its own epoch and resets those it finishes, so a previous
+ *   call's leftovers do no harm, also across replays of a CUDA graph.
  * Same arguments, result and numerics as tq4_1s_linear's small-m path; no
  * allocation of any kind. */
 int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, tq4_stream_t stream);
@@ -190,7 +193,8 @@ size_t tq4_1s_moe_workspace(int64_t m, int32_t topk, const tq4_1s_weight* up, co
  *   y        device bf16 bits [m][H]
  *   ws       device workspace of tq4_1s_moe_workspace() bytes.
  * Routing, gathering, both projections and the combine all run on the
- * device; nothing synchronizes with the host. */
+ * device; nothing synchronizes with the host, and the call can be captured
+ * into a CUDA graph and replayed (same workspace rules as tq4_1s_linear). */
 int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, const float* topk_w, int32_t topk,
                const tq4_1s_weight* up, const tq4_1s_weight* down, uint16_t* y, void* ws, size_t ws_bytes,
                tq4_stream_t stream);
