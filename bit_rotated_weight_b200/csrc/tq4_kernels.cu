@@ -402,14 +402,6 @@ __global__ void __launch_bounds__(256) moe_combine_kernel(const float* __restric
 }
 
 // ------------------------------------------------------------------ launchers
-static int grid_for(int64_t warps_needed, int threads) {
-  int64_t blocks = (warps_needed * 32 + threads - 1) / threads;
-  const int64_t cap = 148LL * (2048 / threads);   // one wave of resident threads
-  if (blocks > cap) blocks = cap;
-  if (blocks < 1) blocks = 1;
-  return static_cast<int>(blocks);
-}
-
 static int grid_threads(int64_t threads_needed, int threads) {
   int64_t blocks = (threads_needed + threads - 1) / threads;
   const int64_t cap = 148LL * (2048 / threads);
