@@ -129,6 +129,42 @@ def test_linear_parity(m, n, k, seed):
     assert tq.tq4_1s_get_status() == 0
 
 
+@pytest.mark.parametrize("m,n,k,seed", [
+    (16, 512, 1024, 43),    # fused cluster split-K
+    (48, 512, 1024, 44),    # TMA-fed stream-K (two segments)
+    (200, 512, 1024, 45),   # large-m GEMM
+])
+def test_linear_degenerate_rows_and_blocks(m, n, k, seed):
+    # the method's degenerate inputs: all-zero weight rows and 32-blocks
+    # (scale 0, codes 7), a zero half-block, and all-zero activation rows;
+    # zero rows of x give exactly zero output rows, zero rows of W exactly
+    # zero output columns, the rest matches the oracle
+    W = synth.student_t_f32((n, k), seed, 5.0, 0.02)
+    W[[0, 7, n - 1]] = 0.0
+    W[3, 64:96] = 0.0
+    W[5, 128:144] = 0.0
+    x = synth.activations_bf16(m, k, seed + 1)
+    zero_rows = [0, m // 2, m - 1]
+    x[zero_rows] = 0
+    p, codes, scales, _ = _quantize_both(W, seed)
+    y = tq.tq4_1s_linear(_bf16_dev(x), p)
+    torch.cuda.synchronize()
+    assert tq.tq4_1s_get_status() == 0
+    yf = y.float().cpu().numpy()
+    assert np.all(yf[zero_rows] == 0.0)
+    assert np.all(yf[:, [0, 7, n - 1]] == 0.0)
+    y_ref, _ = oracle.linear(x, codes[0], scales[0], seed)
+    assert_close(_bits(y), y_ref, f"linear degenerate m={m}")
+
+
+def test_moe_zero_token_rows():
+    y, y_ref, _ = _moe_case(8, 256, 128, 12, 2, (46, 47, 48, 49), zero_rows=(0, 5, 11))
+    yf = y.float().cpu().numpy()
+    assert np.all(yf[[0, 5, 11]] == 0.0)
+    assert_close(_bits(y), y_ref, "moe zero rows")
+    assert tq.tq4_1s_get_status() == 0
+
+
 @pytest.mark.parametrize("x_std", [3000.0, 1e-5])
 def test_linear_activation_range(x_std):
     # activations far outside (and far inside) the fp16 range: the per-row
@@ -231,7 +267,7 @@ def test_moe_route_bad_ids_flagged():
     assert tq.tq4_1s_get_status() & tq.TQ_DEV_BAD_ROUTING
 
 
-def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False, x_std=1.0):
+def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False, x_std=1.0, zero_rows=()):
     up_seed, dn_seed, x_seed, r_seed = seeds
     up = synth.normal_f32((E, I, H), up_seed, dist_std)
     dn = synth.normal_f32((E, H, I), dn_seed, dist_std)
@@ -239,6 +275,7 @@ def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False, x_std=1.0):
     if bad_ids:
         ids[0, 1] = E + 1
     x = synth.f32_to_bf16_bits(synth.normal_f32((m, H), x_seed, x_std))
+    x[list(zero_rows)] = 0
     pu = tq.tq4_1s_quantize(torch.from_numpy(up).to(DEV), seed=up_seed)
     pd = tq.tq4_1s_quantize(torch.from_numpy(dn).to(DEV), seed=dn_seed)
     y = tq.tq4_1s_moe(_bf16_dev(x), torch.from_numpy(ids).to(DEV), torch.from_numpy(w).to(DEV), pu, pd)
