@@ -48,8 +48,13 @@ CALLS = 16
 COPIES = 64
 PACKED_PER_CALL = N_OUT * K_IN // 2 + N_OUT * (K_IN // 16) * 2   # 10,485,760 B
 # DRAM bytes (read + write) of one decode launch of the kernel, from the ncu
-# capture summarised in profiles/streamk_decode_m16_n4096_k4096.md
-TRAFFIC_PER_CALL = 10_703_872
+# capture summarised in profiles/streamk_decode_m16_n4096_k4096.md.  The
+# kernel has changed since (the split-tile counter reset of the stream-K
+# fix-up, a path the decode shape's cluster split-K mode does not run), so
+# the line reports traffic as null until the counters are taken again and
+# gives this figure separately.
+TRAFFIC_PER_CALL = None
+TRAFFIC_BEFORE_CHANGE = 10_703_872
 WORKLOAD = ("decode_linear_4096: x bf16 [16][4096] N(0,1), W 4096x4096 Student-t(5)*0.02 TQ4_1S, "
             "16 calls per step (denoising steps)")
 
@@ -325,6 +330,7 @@ def ours_arm(args):
                                       "first input is a fixed N(0,1) block"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": TRAFFIC_PER_CALL,
+                         "traffic_before_last_kernel_change": TRAFFIC_BEFORE_CHANGE,
                          "algorithmic_bytes": PACKED_PER_CALL,
                          "kernel": "streamk_kernel, fused cluster split-K mode: one launch per tq4_1s_linear "
                                    "call (x staging and rotation, dequant, MMA, on-chip reduction)",
