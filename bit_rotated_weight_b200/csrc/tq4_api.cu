@@ -276,6 +276,7 @@ static bool small_fused(int64_t m, int64_t tiles_times_ki, int grid) {
 struct MoeLayout {
   size_t offsets, pairs, segs, nseg, npv, xr, xscale, h, hr, hscale, zw, partials, cnt_up, cnt_dn, total;
   int64_t P, maxseg, rt_up, rt_dn;
+  int nb_max, chunk;
 };
 
 static MoeLayout moe_layout(int64_t m, int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* dn, int sms) {
@@ -283,7 +284,14 @@ static MoeLayout moe_layout(int64_t m, int32_t topk, const tq4_1s_weight* up, co
   const int64_t E = up->num_experts;
   const int64_t H = up->k, I = up->n;
   L.P = m * topk;
-  L.maxseg = (L.P + kSegRows - 1) / kSegRows + (E < L.P ? E : L.P) + 1;
+  // Token columns per segment: the accumulators are sized for 16 * nb_max
+  // columns, so no segment may hold more rows.  With distinct expert ids per
+  // token an expert takes at most m rows, so up to 16 tokens one 16-column
+  // block suffices; a token that names an expert twice adds a row, and the
+  // 16-row segments keep that case correct too.
+  L.nb_max = m > 16 ? 2 : 1;
+  L.chunk = 16 * L.nb_max;
+  L.maxseg = (L.P + L.chunk - 1) / L.chunk + (E < L.P ? E : L.P) + 1;
   L.rt_up = (I + 127) / 128;
   L.rt_dn = (dn->n + 127) / 128;
   size_t off = 0;
@@ -511,7 +519,7 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   uint16_t* xr = reinterpret_cast<uint16_t*>(base + L.xr);
   uint16_t* hr = reinterpret_cast<uint16_t*>(base + L.hr);
   float* zw = reinterpret_cast<float*>(base + L.zw);
-  cudaError_t e = launch_moe_route(topk_ids, L.P, static_cast<int32_t>(E), offsets, pairs, segs, nseg, kSegRows,
+  cudaError_t e = launch_moe_route(topk_ids, L.P, static_cast<int32_t>(E), offsets, pairs, segs, nseg, L.chunk,
                                    npv, st);
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   float* xscale = reinterpret_cast<float*>(base + L.xscale);
@@ -533,7 +541,7 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   a.k_iters = static_cast<int32_t>((H + 127) / 128);
   a.segs = segs;
   a.nseg_dev = nseg;
-  a.nb_max = m > 16 ? 2 : 1;   // an expert takes each token at most once (top-k ids are distinct)
+  a.nb_max = L.nb_max;   // segments hold at most 16 * nb_max rows (the route's chunk)
   a.scales = up->scales;
   a.row_scale = xscale;
   a.epoch = next_epoch();

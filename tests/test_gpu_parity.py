@@ -267,11 +267,12 @@ def test_moe_route_bad_ids_flagged():
     assert tq.tq4_1s_get_status() & tq.TQ_DEV_BAD_ROUTING
 
 
-def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False, x_std=1.0, zero_rows=()):
+def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False, x_std=1.0, zero_rows=(), ids=None):
     up_seed, dn_seed, x_seed, r_seed = seeds
     up = synth.normal_f32((E, I, H), up_seed, dist_std)
     dn = synth.normal_f32((E, H, I), dn_seed, dist_std)
-    ids, w = synth.gumbel_topk_router(m, E, topk, r_seed)
+    routed, w = synth.gumbel_topk_router(m, E, topk, r_seed)
+    ids = routed if ids is None else np.ascontiguousarray(ids, np.int32)
     if bad_ids:
         ids[0, 1] = E + 1
     x = synth.f32_to_bf16_bits(synth.normal_f32((m, H), x_seed, x_std))
@@ -303,6 +304,19 @@ def test_moe_many_tokens_per_expert():
     # take more than one 32-row segment
     y, y_ref, _ = _moe_case(4, 256, 192, 40, 2, (14, 15, 16, 17))
     assert_close(_bits(y), y_ref, "moe segments")
+
+
+@pytest.mark.parametrize("m", [16, 20])
+def test_moe_repeated_expert_ids_in_a_token(m):
+    # a token that names the same expert in several slots (a top-k router
+    # never does, but the call accepts it): every slot contributes, and an
+    # expert's rows (here 3 per token, up to 60) are split into segments no
+    # wider than the accumulators
+    ids = np.tile(np.array([3, 3, 5, 3, 5, 1], np.int32), (m, 1))
+    y, y_ref, bad = _moe_case(8, 256, 128, m, 6, (50, 51, 52, 53), ids=ids)
+    assert bad == 0
+    assert_close(_bits(y), y_ref, f"moe repeated ids m={m}")
+    assert tq.tq4_1s_get_status() == 0
 
 
 def test_moe_bad_id_skipped():
