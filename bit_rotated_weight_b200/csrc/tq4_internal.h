@@ -20,7 +20,8 @@ void note_launches(int n);
 const CodebookF32& codebook();
 
 // One segment of rows of the rotated activations multiplied by one expert:
-// x = expert, y = first row, z = row count (<= kSegRows), w unused.
+// x = expert, y = first row, z = row count (<= 16 * nb_max <= kSegRows),
+// w unused.
 constexpr int kSegRows = 32;
 
 cudaError_t launch_quantize(const void* W, int dtype, uint8_t* codes, uint16_t* scales, int64_t rows, int64_t k,
