@@ -53,7 +53,9 @@
 // cluster barrier each owner sums its rows over the s partials in rank order
 // -- deterministic, no partials or counters in global memory.
 #include <atomic>
+#include <chrono>
 #include <mutex>
+#include <random>
 
 #include "tq4_internal.h"
 
@@ -931,8 +933,24 @@ __global__ void __launch_bounds__(kThreads, 1)
 
 }  // namespace
 
+// Epochs of one process start at a random value, not at 1: a workspace that
+// was never initialised may hold structured data (small integers, indices)
+// where a counter sits, and a counter whose upper word happened to equal the
+// current epoch would be miscounted.  Successive epochs still differ, and 0
+// is never used.
+static uint32_t first_epoch() {
+  uint32_t seed = 0x9E3779B9u;
+  try {
+    std::random_device rd;
+    seed ^= rd();
+  } catch (...) {
+  }
+  seed ^= static_cast<uint32_t>(std::chrono::steady_clock::now().time_since_epoch().count());
+  return seed | 0x40000000u;   // away from the small values structured data is full of
+}
+
 uint32_t next_epoch() {
-  static std::atomic<uint32_t> epoch{0};
+  static std::atomic<uint32_t> epoch{first_epoch()};
   uint32_t e = epoch.fetch_add(1, std::memory_order_relaxed) + 1;
   if (e == 0) e = epoch.fetch_add(1, std::memory_order_relaxed) + 1;   // 0 marks never-used counters
   return e;
