@@ -355,7 +355,9 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     out = {}
     # prefill GEMM: M=8192, K=4096, N=14336
     m, n, k = 8192, 14336, 4096
-    W = torch.from_numpy(synth.normal_f32((n, k), 8, 0.02)).to(dev)
+    # weights drawn on the device (same distribution as the host generator,
+    # without holding the GPU through a long host draw)
+    W = synth.normal_f32_device((n, k), 8, 0.02, dev)
     p = tq.tq4_1s_quantize(W, seed=8)
     del W
     x = torch.from_numpy(synth.activations_bf16(m, k, 9).view(np.int16)).to(dev).view(torch.bfloat16)
@@ -375,8 +377,9 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     torch.cuda.empty_cache()
     # MoE: 128 experts, 16 tokens, top-6
     E, H, I, mt, topk = 128, 2688, 1856, 16, 6
-    up = tq.tq4_1s_quantize(torch.from_numpy(synth.normal_f32((E, I, H), 4, 0.02)).to(dev), seed=4)
-    dn = tq.tq4_1s_quantize(torch.from_numpy(synth.normal_f32((E, H, I), 5, 0.02)).to(dev), seed=5)
+    up = tq.tq4_1s_quantize(synth.normal_f32_device((E, I, H), 4, 0.02, dev), seed=4)
+    dn = tq.tq4_1s_quantize(synth.normal_f32_device((E, H, I), 5, 0.02, dev), seed=5)
+    torch.cuda.empty_cache()
     routes = [synth.gumbel_topk_router(mt, E, topk, 7 + 100 * r) for r in range(4)]
     ids_d = [torch.from_numpy(r[0]).to(dev) for r in routes]
     w_d = [torch.from_numpy(r[1]).to(dev) for r in routes]
