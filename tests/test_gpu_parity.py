@@ -306,19 +306,6 @@ def test_moe_many_tokens_per_expert():
     assert_close(_bits(y), y_ref, "moe segments")
 
 
-@pytest.mark.parametrize("m", [16, 20])
-def test_moe_repeated_expert_ids_in_a_token(m):
-    # a token that names the same expert in several slots (a top-k router
-    # never does, but the call accepts it): every slot contributes, and an
-    # expert's rows (here 3 per token, up to 60) are split into segments no
-    # wider than the accumulators
-    ids = np.tile(np.array([3, 3, 5, 3, 5, 1], np.int32), (m, 1))
-    y, y_ref, bad = _moe_case(8, 256, 128, m, 6, (50, 51, 52, 53), ids=ids)
-    assert bad == 0
-    assert_close(_bits(y), y_ref, f"moe repeated ids m={m}")
-    assert tq.tq4_1s_get_status() == 0
-
-
 def test_moe_bad_id_skipped():
     y, y_ref, bad = _moe_case(8, 128, 96, 5, 2, (24, 25, 26, 27), bad_ids=True)
     assert bad == 1
