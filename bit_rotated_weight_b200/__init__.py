@@ -25,6 +25,7 @@ __all__ = [
     "tq4_1s_version", "tq4_1s_error_string", "tq4_1s_packed_bytes", "tq4_1s_sign_mask", "tq4_1s_codebook",
     "tq4_1s_quantize", "tq4_1s_dequantize", "tq4_1s_linear_workspace", "tq4_1s_linear",
     "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_route", "tq4_1s_get_status", "tq4_1s_launch_count",
+    "tq4_1s_linear_static",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -73,6 +74,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                 "tq4_1s_dequantize": ([W, P, P], ctypes.c_int),
                 "tq4_1s_linear_workspace": ([I64, W], SZ),
                 "tq4_1s_linear": ([P, I64, W, P, P, SZ, P], ctypes.c_int),
+                "tq4_1s_linear_static": ([P, I64, W, P, P], ctypes.c_int),
                 "tq4_1s_moe_workspace": ([I64, I32, W, W], SZ),
                 "tq4_1s_moe": ([P, I64, P, P, I32, W, W, P, P, SZ, P], ctypes.c_int),
                 "tq4_1s_moe_route": ([P, I64, I32, I32, P, P, P], ctypes.c_int),
@@ -282,15 +284,12 @@ def tq4_1s_linear_static(x: torch.Tensor, w: Packed, out: torch.Tensor | None = 
     on the GPU share that array and race; serialize them.  The first call on a
     device looks up the array's address, so make it outside stream capture.
     """
-    lib = load_library()
-    fn = lib.tq4_1s_linear_static
-    fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(_Weight), ctypes.c_void_p, ctypes.c_void_p]
-    fn.restype = ctypes.c_int
     if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
         raise ValueError("x must be a CUDA bfloat16 [m][k] tensor")
     x = x.contiguous()
     if out is None:
         out = torch.empty((x.shape[0], w.n), dtype=torch.bfloat16, device=x.device)
     wst = w.c_struct()
-    _check(fn(_ptr(x), x.shape[0], ctypes.byref(wst), _ptr(out), _stream(x.device)), "linear_static")
+    _check(load_library().tq4_1s_linear_static(_ptr(x), x.shape[0], ctypes.byref(wst), _ptr(out),
+                                               _stream(x.device)), "linear_static")
     return out
