@@ -96,6 +96,25 @@ def test_validation_rejects_before_any_launch():
     assert lib.tq4_1s_moe_route(good, 4, 0, 8, good, good, null) == 1
 
 
+def test_static_entry_validation_and_scratch_limits():
+    lib = tq.load_library()
+    null = ctypes.c_void_p(0)
+    good = ctypes.c_void_p(4096)
+    assert lib.tq4_1s_linear_static(good, 16, None, good, null) == 1                # no weight
+    assert lib.tq4_1s_linear_static(good, 16, ctypes.byref(_weight(k=48)), good, null) == 1
+    assert lib.tq4_1s_linear_static(good, 16, ctypes.byref(_weight(e=2)), good, null) == 1
+    assert lib.tq4_1s_linear_static(good, 16, ctypes.byref(_weight(codes=0)), good, null) == 1
+    # the fixed scratch bounds: m <= 32, k <= 8192, n <= 32768 (TQ_ERR_SCRATCH_LIMIT)
+    assert lib.tq4_1s_linear_static(good, 33, ctypes.byref(_weight()), good, null) == 9
+    assert lib.tq4_1s_linear_static(good, 16, ctypes.byref(_weight(k=8224)), good, null) == 9
+    assert lib.tq4_1s_linear_static(good, 16, ctypes.byref(_weight(n=32769)), good, null) == 9
+    assert lib.tq4_1s_linear_static(good, 0, ctypes.byref(_weight()), good, null) == 0   # m == 0: no-op
+    assert lib.tq4_1s_linear_static(null, 16, ctypes.byref(_weight()), good, null) == 1
+    assert lib.tq4_1s_linear_static(ctypes.c_void_p(4100), 16, ctypes.byref(_weight()), good, null) == 2
+    assert lib.tq4_1s_linear_static(good, 16, ctypes.byref(_weight(scales=24)), good, null) == 2
+    assert tq.tq4_1s_error_string(9).startswith("shape exceeds the fixed scratch")
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
 def test_valid_call_without_gpu_fails_loudly():
     lib = tq.load_library()
@@ -105,6 +124,7 @@ def test_valid_call_without_gpu_fails_loudly():
     assert need > 0
     assert lib.tq4_1s_linear(good, 16, ctypes.byref(w), good, good, need, ctypes.c_void_p(0)) == 3
     assert lib.tq4_1s_quantize(good, 0, ctypes.byref(w), ctypes.c_void_p(0)) == 3
+    assert lib.tq4_1s_linear_static(good, 16, ctypes.byref(w), good, ctypes.c_void_p(0)) == 3
 
 
 def test_workspace_queries():
