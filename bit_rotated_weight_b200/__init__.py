@@ -193,8 +193,9 @@ SMALL_M = 128   # tq4_1s_linear takes its stream-K path up to this many rows
 def _workspace(nbytes: int, device, kind: str) -> torch.Tensor:
     """A cached workspace per (device, kind), grown on demand.
 
-    The library clears whatever it needs at the start of each call; the
-    kinds are kept apart only so that a large small-m buffer and a large
+    The library needs no cleared workspace: its tile counters carry each
+    launch's epoch, so values left by earlier calls read as zero arrivals.
+    The kinds are kept apart only so that a large small-m buffer and a large
     dequantized-weight buffer are not reallocated back and forth."""
     key = (str(device), kind)
     buf = _ws_cache.get(key)
