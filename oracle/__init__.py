@@ -12,6 +12,9 @@ listed at the top of the C file.  Parity status of each function:
 
 - codebook, sign_mask, hadamard32, fwht32, quantize, dequantize, levels,
   linear, moe_route: pinned by ``tests/test_oracle_pins.py``.
+- router_topk: pinned by invariants (distinct ids, descending order, every
+  chosen logit >= every other, weights positive summing to 1), equal-logit
+  and single-choice special cases, and k = E against scipy's softmax.
 - moe: pinned through closed-form special cases (single slot, constant-level
   experts) and composition with the pinned linear; the squared-ReLU and the
   bf16 rounding of the hidden activation are fixed by the workload
@@ -87,6 +90,7 @@ def _load():
             lib.orc_moe.argtypes = [P, I64, I64, I64, P, P, ctypes.c_int, ctypes.c_int,
                                     P, P, ctypes.c_uint64, P, P, ctypes.c_uint64, P]
             lib.orc_moe.restype = I64
+            lib.orc_router_topk.argtypes = [P, I64, ctypes.c_int, ctypes.c_int, P, P]
             _lib = lib
     return _lib
 
@@ -264,6 +268,21 @@ def moe_route(ids, num_experts: int):
     pairs = np.full(m * topk, -1, np.int32)
     bad = _load().orc_moe_route(_ptr(ids), m, topk, num_experts, _ptr(offsets), _ptr(pairs))
     return offsets, pairs[: offsets[-1]], int(bad)
+
+
+def router_topk(z, topk: int):
+    """MoE router: fp32 logits z [m][E] -> (ids int32 [m][topk], w float32 [m][topk]).
+
+    Softmax over all experts (fp64), the topk largest chosen in descending
+    order (equal logits: lower expert id first), their probabilities
+    renormalised to sum to 1 and rounded to fp32."""
+    z = _c(z, np.float32)
+    m, E = z.shape
+    assert 1 <= topk <= E
+    ids = np.zeros((m, topk), np.int32)
+    w = np.zeros((m, topk), np.float32)
+    _load().orc_router_topk(_ptr(z), m, E, topk, _ptr(ids), _ptr(w))
+    return ids, w
 
 
 def moe(x_bf16, ids, w, up_codes, up_scales, up_seed, dn_codes, dn_scales, dn_seed):

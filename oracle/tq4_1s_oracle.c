@@ -326,6 +326,47 @@ int64_t orc_moe_route(const int32_t *ids, int64_t m, int topk, int num_experts,
     return bad;
 }
 
+/* MoE router (model card, "The model underneath": each token is sent to 6 of
+ * 128 experts; "Performance": the MoE runs without host syncs, so routing is
+ * part of the layer).  Reading: the router's fp32 logits z [m][E] give the
+ * softmax p_e = exp(z_e) / sum_i exp(z_i) over all E experts; the topk
+ * experts of largest p are chosen and their p renormalised to sum to 1.
+ * Softmax is monotone in z, so the choice is made on the fp32 z themselves
+ * (equal z: the lower expert id first); selection order is descending.  The
+ * softmax is taken in fp64 with the largest logit subtracted first (which
+ * leaves p unchanged), the weights rounded to fp32 at the end.              */
+void orc_router_topk(const float *z, int64_t m, int num_experts, int topk, int32_t *ids, float *w) {
+    char *taken = (char *)malloc((size_t)num_experts);
+    double *p = (double *)malloc(sizeof(double) * (size_t)num_experts);
+    for (int64_t t = 0; t < m; t++) {
+        const float *zt = z + t * num_experts;
+        double zmax = -INFINITY;
+        for (int e = 0; e < num_experts; e++)
+            if ((double)zt[e] > zmax) zmax = (double)zt[e];
+        double total = 0.0;
+        for (int e = 0; e < num_experts; e++) {
+            p[e] = exp((double)zt[e] - zmax);
+            total += p[e];
+        }
+        for (int e = 0; e < num_experts; e++) p[e] /= total;
+        memset(taken, 0, (size_t)num_experts);
+        double sel = 0.0;
+        for (int j = 0; j < topk; j++) {
+            int best = -1;
+            for (int e = 0; e < num_experts; e++) {
+                if (taken[e]) continue;
+                if (best < 0 || zt[e] > zt[best]) best = e;   /* strict: ties keep the lower id */
+            }
+            taken[best] = 1;
+            ids[t * topk + j] = best;
+            sel += p[best];
+        }
+        for (int j = 0; j < topk; j++) w[t * topk + j] = (float)(p[ids[t * topk + j]] / sel);
+    }
+    free(taken);
+    free(p);
+}
+
 /* MoE layer.  x [m][H] bf16; ids/w [m][topk]; up codes/scales for E experts
  * of shape [I][H]; down codes/scales of shape [H][I].  Result y [m][H] in
  * fp64 before the final bf16 rounding.  Experts are dequantized one at a

@@ -21,7 +21,7 @@ import numpy as np
 
 __all__ = [
     "rng", "normal_f32", "student_t_f32", "f32_to_bf16_bits", "bf16_bits_to_f32",
-    "activations_bf16", "gumbel_topk_router", "normal_f32_device", "sweep_seed", "WORKLOADS",
+    "activations_bf16", "gumbel_topk_router", "router_logits_f32", "normal_f32_device", "sweep_seed", "WORKLOADS",
 ]
 
 
@@ -83,6 +83,18 @@ def gumbel_topk_router(m: int, num_experts: int, topk: int, seed: int):
     w = e / e.sum(axis=1, keepdims=True)
     w = w / w.sum(axis=1, keepdims=True)
     return order.astype(np.int32), w.astype(np.float32)
+
+
+def router_logits_f32(m: int, num_experts: int, seed: int) -> np.ndarray:
+    """Router logits for m tokens as the layer receives them: fp32 [m][E],
+    z = l + g with l ~ N(0,1) and Gumbel noise g = -ln(-ln U), U ~ U(0,1),
+    drawn in float64 exactly as :func:`gumbel_topk_router` draws them (same
+    seed, same stream) and rounded to float32."""
+    g = rng(seed)
+    logits = g.standard_normal((m, num_experts))
+    u = g.random((m, num_experts))
+    u = np.clip(u, np.finfo(np.float64).tiny, 1.0 - 2.0 ** -53)
+    return (logits - np.log(-np.log(u))).astype(np.float32)
 
 
 def normal_f32_device(shape, seed: int, std: float, device):

@@ -321,6 +321,50 @@ def test_router_weights_are_normalised():
     assert all(len(set(r)) == 6 for r in ids)
 
 
+def test_router_topk_invariants_on_gumbel_logits():
+    # Selection: distinct ids in descending logit order, every chosen logit at
+    # least every unchosen one; weights positive, descending, summing to 1.
+    z = synth.router_logits_f32(64, 128, 7)
+    ids, w = oracle.router_topk(z, 6)
+    assert ids.shape == (64, 6) and w.dtype == np.float32
+    for t in range(64):
+        sel = z[t, ids[t]]
+        assert len(set(ids[t].tolist())) == 6
+        assert np.all(np.diff(sel) <= 0)
+        rest = np.delete(z[t], ids[t])
+        assert sel.min() >= rest.max()
+        assert np.all(w[t] > 0) and np.all(np.diff(w[t]) <= 0)
+        assert abs(float(w[t].astype(np.float64).sum()) - 1.0) < 1e-6
+    # the Gumbel-perturbed selection of the input generator chooses the same
+    # experts from the unrounded logits (no fp32 near-ties in this draw)
+    ids_g, w_g = synth.gumbel_topk_router(64, 128, 6, 7)
+    assert np.array_equal(ids, ids_g)
+    assert np.allclose(w, w_g, rtol=1e-6, atol=0)
+
+
+def test_router_topk_special_cases():
+    # equal logits: the lowest ids in order, weights exactly 1/k
+    ids, w = oracle.router_topk(np.zeros((3, 16), np.float32), 4)
+    assert np.array_equal(ids, np.tile(np.arange(4, dtype=np.int32), (3, 1)))
+    assert np.all(w == np.float32(0.25))
+    # ties inside the selection: equal logits ranked by id
+    z = np.array([[0.5, 2.0, 1.0, 2.0, 1.0, -3.0]], np.float32)
+    ids, w = oracle.router_topk(z, 4)
+    assert ids.tolist() == [[1, 3, 2, 4]]
+    assert w[0, 0] == w[0, 1] and w[0, 2] == w[0, 3]
+    # one choice: weight exactly 1
+    ids, w = oracle.router_topk(synth.router_logits_f32(5, 32, 3), 1)
+    assert np.all(w == 1.0)
+    # k = E: the full softmax (scipy, independent of the oracle's loop)
+    from scipy.special import softmax
+    z = synth.router_logits_f32(4, 24, 9)
+    ids, w = oracle.router_topk(z, 24)
+    ref = softmax(z.astype(np.float64), axis=1)
+    for t in range(4):
+        assert np.array_equal(ids[t], np.argsort(-z[t], kind="stable"))
+        assert np.allclose(w[t], ref[t, ids[t]], rtol=2e-7, atol=0)
+
+
 def test_moe_composes_linear_relu2_and_slot_sum():
     E, H, I, m, topk = 4, 64, 96, 5, 2
     up = synth.normal_f32((E, I, H), 81, 0.05)
