@@ -23,8 +23,8 @@ import torch
 __all__ = [
     "LIB_PATH", "TQ4Error", "Packed", "load_library",
     "tq4_1s_version", "tq4_1s_error_string", "tq4_1s_packed_bytes", "tq4_1s_sign_mask", "tq4_1s_codebook",
-    "tq4_1s_quantize", "tq4_1s_dequantize", "tq4_1s_linear_workspace", "tq4_1s_linear",
-    "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_route", "tq4_1s_get_status", "tq4_1s_launch_count",
+    "tq4_1s_quantize", "tq4_1s_quantize_batched", "tq4_1s_dequantize", "tq4_1s_linear_workspace", "tq4_1s_linear",
+    "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_logits", "tq4_1s_router_topk", "tq4_1s_moe_route", "tq4_1s_get_status", "tq4_1s_launch_count",
     "tq4_1s_linear_static",
 ]
 
@@ -71,6 +71,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                 "tq4_1s_sign_mask": ([ctypes.c_uint64, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
                 "tq4_1s_codebook": ([P, P], ctypes.c_int),
                 "tq4_1s_quantize": ([P, ctypes.c_int, W, P], ctypes.c_int),
+                "tq4_1s_quantize_batched": ([P, ctypes.c_int, P, I32, P], ctypes.c_int),
                 "tq4_1s_dequantize": ([W, P, P], ctypes.c_int),
                 "tq4_1s_linear_workspace": ([I64, W], SZ),
                 "tq4_1s_linear": ([P, I64, W, P, P, SZ, P], ctypes.c_int),
@@ -78,6 +79,8 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                 "tq4_1s_moe_workspace": ([I64, I32, W, W], SZ),
                 "tq4_1s_moe": ([P, I64, P, P, I32, W, W, P, P, SZ, P], ctypes.c_int),
                 "tq4_1s_moe_route": ([P, I64, I32, I32, P, P, P], ctypes.c_int),
+                "tq4_1s_moe_logits": ([P, I64, P, I32, W, W, P, P, SZ, P], ctypes.c_int),
+                "tq4_1s_router_topk": ([P, I64, I32, I32, P, P, P], ctypes.c_int),
                 "tq4_1s_get_status": ([P, ctypes.POINTER(I32)], ctypes.c_int),
                 "tq4_1s_launch_count": ([], ctypes.c_uint64),
             }
@@ -177,6 +180,28 @@ def tq4_1s_quantize(W: torch.Tensor, seed: int, out: Packed | None = None) -> Pa
     return out
 
 
+def tq4_1s_quantize_batched(Ws, seeds, outs=None) -> list:
+    """Quantize several tensors (all float32 or all bfloat16, CUDA, [n][k] or
+    [E][n][k]) in batched launches; returns their Packed forms."""
+    Ws = [W.unsqueeze(0) if W.dim() == 2 else W for W in Ws]
+    if not Ws:
+        return []
+    dt0 = Ws[0].dtype
+    for W in Ws:
+        if W.dim() != 3 or not W.is_cuda or W.dtype != dt0 or dt0 not in (torch.float32, torch.bfloat16):
+            raise ValueError("every W must be a CUDA tensor of one dtype (float32 or bfloat16), [n][k] or [E][n][k]")
+    Ws = [W.contiguous() for W in Ws]
+    if outs is None:
+        outs = [_empty_packed(W.shape[1], W.shape[2], W.shape[0], s, W.device) for W, s in zip(Ws, seeds)]
+    structs = (_Weight * len(Ws))(*[o.c_struct() for o in outs])
+    ptrs = (ctypes.c_void_p * len(Ws))(*[W.data_ptr() for W in Ws])
+    dt = TQ_DTYPE_F32 if dt0 == torch.float32 else TQ_DTYPE_BF16
+    _check(load_library().tq4_1s_quantize_batched(ctypes.cast(ptrs, ctypes.c_void_p), dt,
+                                                  ctypes.cast(structs, ctypes.c_void_p), len(Ws),
+                                                  _stream(Ws[0].device)), "quantize_batched")
+    return outs
+
+
 def tq4_1s_dequantize(w: Packed) -> torch.Tensor:
     out = torch.empty((w.num_experts, w.n, w.k), dtype=torch.float32, device=w.codes.device)
     ws = w.c_struct()
@@ -252,6 +277,41 @@ def tq4_1s_moe(x: torch.Tensor, topk_ids: torch.Tensor, topk_w: torch.Tensor, up
                                      ctypes.byref(d), _ptr(out), _ptr(workspace), workspace.numel(),
                                      _stream(x.device)), "moe")
     return out
+
+
+def tq4_1s_moe_logits(x: torch.Tensor, logits: torch.Tensor, topk: int, up: Packed, down: Packed,
+                      out: torch.Tensor | None = None, workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """The MoE with the router on the device: logits float32 [m][E] (CUDA)."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a CUDA bfloat16 [m][H] tensor")
+    if logits.dtype != torch.float32 or logits.dim() != 2 or not logits.is_cuda:
+        raise ValueError("logits must be a CUDA float32 [m][E] tensor")
+    x = x.contiguous()
+    logits = logits.contiguous()
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty((m, up.k), dtype=torch.bfloat16, device=x.device)
+    u, d = up.c_struct(), down.c_struct()
+    if workspace is None:   # (a caller's workspace is checked by the library)
+        need = load_library().tq4_1s_moe_workspace(m, topk, ctypes.byref(u), ctypes.byref(d))
+        workspace = _workspace(need, x.device, "moe")
+    _check(load_library().tq4_1s_moe_logits(_ptr(x), m, _ptr(logits), topk, ctypes.byref(u), ctypes.byref(d),
+                                            _ptr(out), _ptr(workspace), workspace.numel(), _stream(x.device)),
+           "moe_logits")
+    return out
+
+
+def tq4_1s_router_topk(logits: torch.Tensor, topk: int):
+    """(ids int32 [m][topk], weights float32 [m][topk]) from float32 logits [m][E] on CUDA."""
+    if logits.dtype != torch.float32 or logits.dim() != 2 or not logits.is_cuda:
+        raise ValueError("logits must be a CUDA float32 [m][E] tensor")
+    logits = logits.contiguous()
+    m, E = logits.shape
+    ids = torch.empty((m, topk), dtype=torch.int32, device=logits.device)
+    w = torch.empty((m, topk), dtype=torch.float32, device=logits.device)
+    _check(load_library().tq4_1s_router_topk(_ptr(logits), m, E, topk, _ptr(ids), _ptr(w), _stream(logits.device)),
+           "router_topk")
+    return ids, w
 
 
 def tq4_1s_moe_route(topk_ids: torch.Tensor, num_experts: int):

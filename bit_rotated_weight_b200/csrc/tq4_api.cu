@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <vector>
 
 #include "tq4_internal.h"
 
@@ -274,7 +275,7 @@ static bool small_fused(int64_t m, int64_t tiles_times_ki, int grid) {
 }
 
 struct MoeLayout {
-  size_t offsets, pairs, segs, nseg, npv, xr, xscale, h, hr, hscale, zw, partials, cnt_up, cnt_dn, total;
+  size_t offsets, pairs, segs, nseg, npv, ids, wts, xr, xscale, h, hr, hscale, zw, partials, cnt_up, cnt_dn, total;
   int64_t P, maxseg, rt_up, rt_dn;
   int nb_max, chunk;
 };
@@ -305,6 +306,8 @@ static MoeLayout moe_layout(int64_t m, int32_t topk, const tq4_1s_weight* up, co
   L.segs = take(L.maxseg * 16);
   L.nseg = take(4);
   L.npv = take(4);
+  L.ids = take(L.P * 4);   // router output (tq4_1s_moe_logits)
+  L.wts = take(L.P * 4);
   L.xr = take(L.P * H * 2);
   L.xscale = take(L.P * 4);
   L.h = take(L.P * I * 2);
@@ -373,6 +376,26 @@ TQ_API int tq4_1s_quantize(const void* W, int dtype, const tq4_1s_weight* out, t
   const int64_t rows = out->n * out->num_experts;
   return cuda_rc(launch_quantize(W, dtype, out->codes, out->scales, rows, out->k, sign_mask_of(out->seed),
                                  codebook(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+TQ_API int tq4_1s_quantize_batched(const void* const* W, int dtype, const tq4_1s_weight* outs, int32_t count,
+                                   tq4_stream_t stream) {
+  if (count < 0 || (count > 0 && (!W || !outs))) return TQ_ERR_INVALID_ARG;
+  if (dtype != TQ_DTYPE_F32 && dtype != TQ_DTYPE_BF16) return TQ_ERR_INVALID_ARG;
+  if (count == 0) return TQ_OK;
+  for (int32_t i = 0; i < count; ++i) {
+    int rc = weight_ok(&outs[i], true);
+    if (rc) return rc;
+    if (!W[i]) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(W[i])) return TQ_ERR_ALIGNMENT;
+  }
+  int rc = check_device(nullptr);
+  if (rc) return rc;
+  std::vector<QuantItem> items(static_cast<size_t>(count));
+  for (int32_t i = 0; i < count; ++i)
+    items[i] = QuantItem{W[i], outs[i].codes, outs[i].scales, outs[i].n * outs[i].num_experts, outs[i].k,
+                         sign_mask_of(outs[i].seed)};
+  return cuda_rc(launch_quantize_batch(items.data(), count, dtype, codebook(), reinterpret_cast<cudaStream_t>(stream)));
 }
 
 TQ_API int tq4_1s_dequantize(const tq4_1s_weight* w, float* W_out, tq4_stream_t stream) {
@@ -492,14 +515,20 @@ TQ_API size_t tq4_1s_moe_workspace(int64_t m, int32_t topk, const tq4_1s_weight*
   return moe_layout(m, topk, up, down, sms_or_default()).total;
 }
 
-TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, const float* topk_w, int32_t topk,
-                      const tq4_1s_weight* up, const tq4_1s_weight* down, uint16_t* y, void* ws, size_t ws_bytes,
-                      tq4_stream_t stream) {
+// The MoE launch sequence shared by tq4_1s_moe (caller's routing) and
+// tq4_1s_moe_logits (router on the device: `logits` non-null, ids and weights
+// produced into the workspace).
+static int moe_impl(const uint16_t* x, int64_t m, const int32_t* topk_ids, const float* topk_w, const float* logits,
+                    int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* down, uint16_t* y, void* ws,
+                    size_t ws_bytes, tq4_stream_t stream) {
   int rc = moe_check(m, topk, up, down, true);
   if (rc) return rc;
   if (m == 0) return TQ_OK;
-  if (!x || !topk_ids || !topk_w || !y) return TQ_ERR_INVALID_ARG;
-  if (!aligned16(x) || !aligned16(y) || !aligned16(topk_ids) || !aligned16(topk_w)) return TQ_ERR_ALIGNMENT;
+  if (!x || !y || (logits ? false : (!topk_ids || !topk_w))) return TQ_ERR_INVALID_ARG;
+  if (logits && (up->num_experts > 1024 || topk > 32 || topk > up->num_experts))
+    return TQ_ERR_INVALID_ARG;   // router limits
+  if (!aligned16(x) || !aligned16(y)) return TQ_ERR_ALIGNMENT;
+  if (logits ? !aligned16(logits) : (!aligned16(topk_ids) || !aligned16(topk_w))) return TQ_ERR_ALIGNMENT;
   int sms = 0;
   if ((rc = check_device(&sms))) return rc;
   const MoeLayout L = moe_layout(m, topk, up, down, sms);
@@ -519,8 +548,13 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   uint16_t* xr = reinterpret_cast<uint16_t*>(base + L.xr);
   uint16_t* hr = reinterpret_cast<uint16_t*>(base + L.hr);
   float* zw = reinterpret_cast<float*>(base + L.zw);
+  if (logits) {
+    topk_ids = reinterpret_cast<const int32_t*>(base + L.ids);
+    topk_w = reinterpret_cast<const float*>(base + L.wts);
+  }
   cudaError_t e = launch_moe_route(topk_ids, L.P, static_cast<int32_t>(E), offsets, pairs, segs, nseg, L.chunk,
-                                   npv, st);
+                                   npv, st, logits, topk, reinterpret_cast<int32_t*>(base + L.ids),
+                                   reinterpret_cast<float*>(base + L.wts));
   if (e != cudaSuccess) return TQ_ERR_CUDA;
   float* xscale = reinterpret_cast<float*>(base + L.xscale);
   uint16_t* h = reinterpret_cast<uint16_t*>(base + L.h);
@@ -573,6 +607,38 @@ TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, con
   b.max_tiles = static_cast<int32_t>(L.maxseg * L.rt_dn);
   if ((e = launch_streamk(&tcd, &thr, nullptr, b, sms, st)) != cudaSuccess) return TQ_ERR_CUDA;
   return cuda_rc(launch_moe_combine(zw, topk_ids, m, topk, H, static_cast<int32_t>(E), y, st));
+}
+
+TQ_API int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, const float* topk_w, int32_t topk,
+                      const tq4_1s_weight* up, const tq4_1s_weight* down, uint16_t* y, void* ws, size_t ws_bytes,
+                      tq4_stream_t stream) {
+  if (!topk_ids || !topk_w) {
+    const int rc = moe_check(m, topk, up, down, true);
+    return rc ? rc : (m == 0 ? TQ_OK : TQ_ERR_INVALID_ARG);
+  }
+  return moe_impl(x, m, topk_ids, topk_w, nullptr, topk, up, down, y, ws, ws_bytes, stream);
+}
+
+TQ_API int tq4_1s_moe_logits(const uint16_t* x, int64_t m, const float* logits, int32_t topk,
+                             const tq4_1s_weight* up, const tq4_1s_weight* down, uint16_t* y, void* ws,
+                             size_t ws_bytes, tq4_stream_t stream) {
+  if (!logits) {
+    const int rc = moe_check(m, topk, up, down, true);
+    return rc ? rc : (m == 0 ? TQ_OK : TQ_ERR_INVALID_ARG);
+  }
+  return moe_impl(x, m, nullptr, nullptr, logits, topk, up, down, y, ws, ws_bytes, stream);
+}
+
+TQ_API int tq4_1s_router_topk(const float* logits, int64_t m, int32_t num_experts, int32_t topk, int32_t* ids,
+                              float* weights, tq4_stream_t stream) {
+  if (m < 0 || num_experts <= 0 || num_experts > 1024 || topk <= 0 || topk > 32 || topk > num_experts ||
+      m * num_experts > (1ll << 40))
+    return TQ_ERR_INVALID_ARG;
+  if (m == 0) return TQ_OK;
+  if (!logits || !ids || !weights) return TQ_ERR_INVALID_ARG;
+  int rc = check_device(nullptr);
+  if (rc) return rc;
+  return cuda_rc(launch_router(logits, m, num_experts, topk, ids, weights, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 TQ_API int tq4_1s_moe_route(const int32_t* topk_ids, int64_t m, int32_t topk, int32_t num_experts, int32_t* offsets,

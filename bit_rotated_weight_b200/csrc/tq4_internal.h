@@ -24,6 +24,17 @@ const CodebookF32& codebook();
 // w unused.
 constexpr int kSegRows = 32;
 
+// One tensor of a batched quantize launch: rows x k (k % 32 == 0), its sign
+// mask, input W (fp32 or bf16, the batch's dtype) and output planes.
+struct QuantItem {
+  const void* W;
+  uint8_t* codes;
+  uint16_t* scales;
+  int64_t rows, k;
+  uint32_t mask;
+};
+cudaError_t launch_quantize_batch(const QuantItem* items, int count, int dtype, const CodebookF32& cb,
+                                  cudaStream_t st);
 cudaError_t launch_quantize(const void* W, int dtype, uint8_t* codes, uint16_t* scales, int64_t rows, int64_t k,
                             uint32_t mask, const CodebookF32& cb, cudaStream_t st);
 cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, float* out, int64_t rows, int64_t k,
@@ -39,9 +50,18 @@ cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales,
 cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* gather, int32_t topk,
                                  const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
                                  uint16_t* xr, float* row_scale, uint32_t mask, cudaStream_t st);
+// Routing: offsets, stably bucketed pairs, segment list and counts.  With
+// `logits` (fp32 [m][num_experts], m = npairs / topk) the router runs first in
+// the same kernel and writes ids_out / w_out ([m][topk]), which the routing
+// then reads; otherwise `ids` is the caller's.
 cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
                              int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
-                             cudaStream_t st);
+                             cudaStream_t st, const float* logits = nullptr, int32_t topk = 1,
+                             int32_t* ids_out = nullptr, float* w_out = nullptr);
+// The router alone: ids/w [m][topk] from fp32 logits [m][num_experts]
+// (num_experts <= 1024, topk <= 32).
+cudaError_t launch_router(const float* logits, int64_t m, int32_t num_experts, int32_t topk, int32_t* ids, float* w,
+                          cudaStream_t st);
 cudaError_t launch_moe_combine(const float* zw, const int32_t* ids, int64_t m, int32_t topk, int64_t h,
                                int32_t num_experts, uint16_t* y, cudaStream_t st);
 

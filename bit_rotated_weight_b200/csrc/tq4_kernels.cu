@@ -7,6 +7,8 @@
 // thread one 32-element block, its 32-point butterfly in registers (stage h
 // pairs elements j and j+h); the activation kernel spreads a slice over a
 // warp and runs the same butterfly through lane shuffles.
+#include <climits>
+
 #include "tq4_internal.h"
 
 namespace tq4 {
@@ -25,13 +27,6 @@ __device__ __forceinline__ uint16_t f16_sat_bits(float x) {
 }
 
 // ------------------------------------------------------------------ quantize
-template <typename T>
-__device__ __forceinline__ float load_w(const T* p);
-template <>
-__device__ __forceinline__ float load_w<float>(const float* p) { return __ldg(p); }
-template <>
-__device__ __forceinline__ float load_w<uint16_t>(const uint16_t* p) { return bf16_bits_to_f32(__ldg(p)); }
-
 // One thread per 32-element block: the whole butterfly runs in registers in
 // the fixed order (stage h pairs elements j and j+h for j with bit h clear),
 // so the result is bit-identical to the warp-shuffle form and to the oracle.
@@ -49,97 +44,168 @@ __device__ __forceinline__ void fwht32_regs(float (&a)[32]) {
   }
 }
 
-template <typename T>
-__device__ __forceinline__ void load_block(const T* p, float (&w)[32]);
-template <>
-__device__ __forceinline__ void load_block<float>(const float* p, float (&w)[32]) {
-  const float4* q = reinterpret_cast<const float4*>(p);
+// Quantize one 32-element block held in registers (sign flip, butterfly, x r,
+// per-half RMS by the pairwise tree, fp16 scale, nearest level by the
+// thresholds, nibble packing) -- the fixed fp32 operation order that the
+// packing's bit-exactness rests on.  words = the 16 code bytes, dpair = the
+// two fp16 scales (half 0 in the low 16 bits).
+__device__ __forceinline__ void quantize_block(float (&a)[32], uint32_t mask, const float* s_t, uint32_t (&words)[4],
+                                               uint32_t& dpair) {
+  const float r = rsqrt32();
+  bool finite = true;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const float4 f = __ldg(q + i);
-    w[4 * i] = f.x;
-    w[4 * i + 1] = f.y;
-    w[4 * i + 2] = f.z;
-    w[4 * i + 3] = f.w;
+  for (int i = 0; i < 32; ++i) {
+    finite = finite && isfinite(a[i]);
+    if ((mask >> i) & 1u) a[i] = -a[i];
   }
-}
-template <>
-__device__ __forceinline__ void load_block<uint16_t>(const uint16_t* p, float (&w)[32]) {
-  const uint4* q = reinterpret_cast<const uint4*>(p);
+  if (!finite) raise_status(TQ_DEV_NONFINITE);
+  fwht32_regs(a);
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const uint4 u = __ldg(q + i);
-    const uint32_t v[4] = {u.x, u.y, u.z, u.w};
+  for (int i = 0; i < 32; ++i) a[i] = __fmul_rn(a[i], r);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      w[8 * i + 2 * j] = __uint_as_float(v[j] << 16);
-      w[8 * i + 2 * j + 1] = __uint_as_float(v[j] & 0xFFFF0000u);
+  for (int i = 0; i < 4; ++i) words[i] = 0u;
+  dpair = 0u;
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    float p[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) p[i] = __fmul_rn(a[16 * h + i], a[16 * h + i]);
+#pragma unroll
+    for (int st = 8; st >= 1; st >>= 1)
+#pragma unroll
+      for (int i = 0; i < st; ++i) p[i] = __fadd_rn(p[i], p[i + st]);
+    const float rms = __fsqrt_rn(__fmul_rn(p[0], 0.0625f));
+    const uint16_t dbits = f16_sat_bits(rms);
+    dpair |= static_cast<uint32_t>(dbits) << (16 * h);
+    const float d = __half2float(__ushort_as_half(dbits));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      uint32_t code;
+      if (d == 0.0f) {
+        code = 7u;
+      } else {
+        const float u = __fdiv_rn(a[16 * h + i], d);
+        // number of thresholds strictly below u (binary search, sorted t)
+        code = (u > s_t[7]) ? 8u : 0u;
+        code += (u > s_t[code + 3]) ? 4u : 0u;
+        code += (u > s_t[code + 1]) ? 2u : 0u;
+        code += (u > s_t[code]) ? 1u : 0u;
+      }
+      const int e = 16 * h + i;   // element index; nibble e of the 16-byte block
+      words[e >> 3] |= code << (4 * (e & 7));
     }
   }
 }
 
-// Quantize: one thread per 32-block (sign flip, butterfly, x r, per-half RMS
-// by the pairwise tree, fp16 scale, nearest level by the thresholds, nibble
-// packing).  Consecutive threads take consecutive blocks of a row.
+// The tensors of one quantize launch.  A tensor of B blocks (B = rows * k / 32,
+// blocks consecutive in its flat row-major order) owns the warp chunks
+// [chunk0, chunk0 + ceil(B / 32)) of the launch; a chunk is 32 consecutive
+// blocks.  Passed by value (kernel parameter space).
+constexpr int kQuantBatch = 48;
+struct QuantTensor {
+  const void* W;
+  uint8_t* codes;
+  uint16_t* scales;
+  int64_t nblocks;
+  int64_t chunk0;
+  uint32_t mask;
+};
+struct QuantBatch {
+  int32_t count;
+  int64_t nchunks;
+  QuantTensor t[kQuantBatch];
+};
+
+// Quantize.  A warp takes 32 consecutive blocks at a time: it reads them
+// with coalesced 16-byte loads (lane l, load i: bytes 16 l + 512 i of the
+// chunk), writes them to its shared-memory tile, and each lane then quantizes
+// one block from the tile in registers and stores its 16 code bytes and two
+// scales (coalesced too).  Tile rows are one block each, their 16-byte
+// pieces XOR-swizzled so that neither the writes nor the per-lane row reads
+// conflict on banks.  The next chunk's loads are issued before the current
+// chunk is quantized.
 template <typename T>
-__global__ void __launch_bounds__(256) quantize_kernel(const T* __restrict__ W, uint8_t* __restrict__ codes,
-                                                       uint16_t* __restrict__ scales, int64_t rows, int64_t k,
-                                                       uint32_t mask, CodebookF32 cb) {
+__global__ void __launch_bounds__(256) quantize_kernel(const __grid_constant__ QuantBatch qb, CodebookF32 cb) {
+  constexpr int kRowBytes = 32 * static_cast<int>(sizeof(T));   // one block: 128 B (fp32) or 64 B (bf16)
+  constexpr int kPieces = kRowBytes / 16;                        // 16-byte pieces per block
+  constexpr int kLoads = 32 * kPieces / 32;                      // 16-byte loads per lane per chunk
   __shared__ float s_t[16];
+  __shared__ __align__(16) uint8_t tile[8][32 * kRowBytes];
   if (threadIdx.x < 16) s_t[threadIdx.x] = cb.thresholds[threadIdx.x];
   __syncthreads();
-  const int64_t kb_per_row = k / 32;
-  const int64_t nblocks = rows * kb_per_row;
-  const float r = rsqrt32();
-  for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
-       b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
-    float a[32];
-    load_block<T>(W + row * k + kb * 32, a);
-    bool finite = true;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  uint8_t* my = tile[warp];
+  // swizzled byte offset of piece c of block (row) b
+  auto tpos = [](int b, int c) {
+    const int sw = (kPieces == 8) ? (b & 7) : ((b >> 1) & 3);
+    return b * kRowBytes + 16 * (c ^ sw);
+  };
+  const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
+  int tix = 0;   // tensor of the current chunk (chunks are visited in increasing order)
+  auto locate = [&](int64_t ch, int& ti) {
+    while (ti + 1 < qb.count && ch >= qb.t[ti + 1].chunk0) ++ti;
+  };
+  uint4 buf[kLoads];
+  auto load_chunk = [&](int64_t ch, int ti) {
+    const QuantTensor& q = qb.t[ti];
+    const int64_t b0 = (ch - q.chunk0) * 32;
+    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(q.W) + b0 * 32);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) {
-      finite = finite && isfinite(a[i]);
-      if ((mask >> i) & 1u) a[i] = -a[i];
+    for (int i = 0; i < kLoads; ++i) {
+      const int piece = lane + 32 * i;   // 16-byte piece of the chunk
+      const int b = piece / kPieces;
+      buf[i] = (b0 + b < q.nblocks) ? __ldg(src + piece) : make_uint4(0u, 0u, 0u, 0u);
     }
-    if (!finite) raise_status(TQ_DEV_NONFINITE);
-    fwht32_regs(a);
+  };
+  int64_t ch = static_cast<int64_t>(blockIdx.x) * 8 + warp;
+  if (ch < qb.nchunks) {
+    locate(ch, tix);
+    load_chunk(ch, tix);
+  }
+  for (; ch < qb.nchunks; ch += nwarps) {
 #pragma unroll
-    for (int i = 0; i < 32; ++i) a[i] = __fmul_rn(a[i], r);
-    uint32_t words[4] = {0u, 0u, 0u, 0u};
-    uint32_t dpair = 0;
+    for (int i = 0; i < kLoads; ++i) {
+      const int piece = lane + 32 * i;
+      *reinterpret_cast<uint4*>(my + tpos(piece / kPieces, piece % kPieces)) = buf[i];
+    }
+    __syncwarp();
+    const int cur = tix;
+    const int64_t nxt = ch + nwarps;
+    if (nxt < qb.nchunks) {
+      locate(nxt, tix);
+      load_chunk(nxt, tix);
+    }
+    float a[32];
+    if constexpr (sizeof(T) == 4) {
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      float p[16];
+      for (int c = 0; c < kPieces; ++c) {
+        const float4 f = *reinterpret_cast<const float4*>(my + tpos(lane, c));
+        a[4 * c] = f.x;
+        a[4 * c + 1] = f.y;
+        a[4 * c + 2] = f.z;
+        a[4 * c + 3] = f.w;
+      }
+    } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) p[i] = __fmul_rn(a[16 * h + i], a[16 * h + i]);
+      for (int c = 0; c < kPieces; ++c) {
+        const uint4 u = *reinterpret_cast<const uint4*>(my + tpos(lane, c));
+        const uint32_t v[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int st = 8; st >= 1; st >>= 1)
-#pragma unroll
-        for (int i = 0; i < st; ++i) p[i] = __fadd_rn(p[i], p[i + st]);
-      const float rms = __fsqrt_rn(__fmul_rn(p[0], 0.0625f));
-      const uint16_t dbits = f16_sat_bits(rms);
-      dpair |= static_cast<uint32_t>(dbits) << (16 * h);
-      const float d = __half2float(__ushort_as_half(dbits));
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        uint32_t code;
-        if (d == 0.0f) {
-          code = 7u;
-        } else {
-          const float u = __fdiv_rn(a[16 * h + i], d);
-          // number of thresholds strictly below u (binary search, sorted t)
-          code = (u > s_t[7]) ? 8u : 0u;
-          code += (u > s_t[code + 3]) ? 4u : 0u;
-          code += (u > s_t[code + 1]) ? 2u : 0u;
-          code += (u > s_t[code]) ? 1u : 0u;
+        for (int j = 0; j < 4; ++j) {
+          a[8 * c + 2 * j] = __uint_as_float(v[j] << 16);
+          a[8 * c + 2 * j + 1] = __uint_as_float(v[j] & 0xFFFF0000u);
         }
-        const int e = 16 * h + i;   // element index; nibble e of the 16-byte block
-        words[e >> 3] |= code << (4 * (e & 7));
       }
     }
-    *reinterpret_cast<uint4*>(codes + row * (k / 2) + kb * 16) = make_uint4(words[0], words[1], words[2], words[3]);
-    *reinterpret_cast<uint32_t*>(scales + row * (k / 16) + kb * 2) = dpair;
+    __syncwarp();   // the tile is rewritten with the next chunk after this
+    const QuantTensor& q = qb.t[cur];
+    const int64_t b = (ch - q.chunk0) * 32 + lane;
+    if (b < q.nblocks) {
+      uint32_t words[4], dpair;
+      quantize_block(a, q.mask, s_t, words, dpair);
+      *reinterpret_cast<uint4*>(q.codes + b * 16) = make_uint4(words[0], words[1], words[2], words[3]);
+      *reinterpret_cast<uint32_t*>(q.scales + b * 2) = dpair;
+    }
   }
 }
 
@@ -292,12 +358,84 @@ __global__ void __launch_bounds__(kRotThreads, 10)
 // Also writes (when the pointers are non-null) the segment list used by the
 // grouped stream-K launches -- chunks of at most `chunk` consecutive rows of
 // one expert -- and the segment and valid-pair counts.
-__global__ void __launch_bounds__(1024) moe_route_kernel(const int32_t* __restrict__ ids, int64_t npairs,
+//
+// The router (model card, "The model underneath": 6 of 128 experts per token;
+// "Performance": no host syncs in the MoE) runs first when logits are given:
+// softmax over all experts, the topk largest taken (equal logits: lower id
+// first), their probabilities renormalised.  One warp per token; lane l holds
+// the logits of experts l, l + 32, ...; each round the lanes propose their
+// best untaken expert and a shuffle reduction picks the warp's (largest
+// logit, then lowest id).  The selected j-th logit stays with lane j; the
+// weights are exp(z_j - z_max) / sum over the selected, in fp64 (the full
+// softmax's denominator cancels).  A NaN logit is never chosen and sets
+// TQ_DEV_NONFINITE.
+__device__ void router_rows(const float* __restrict__ z, int64_t m, int32_t num_experts, int32_t topk,
+                            int32_t* __restrict__ ids, float* __restrict__ w) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nwarps = blockDim.x >> 5;
+  const int per_lane = (num_experts + 31) / 32;   // <= 32 (num_experts <= 1024)
+  for (int64_t t = warp; t < m; t += nwarps) {
+    const float* zt = z + t * num_experts;
+    uint32_t taken = 0u;   // bit i: expert lane + 32 i already chosen
+    bool nan_seen = false;
+    float myz = 0.0f;
+    int mye = 0;
+    for (int j = 0; j < topk; ++j) {
+      float bz = -INFINITY;
+      int be = INT_MAX;
+      for (int i = 0; i < per_lane; ++i) {
+        const int e = i * 32 + lane;
+        if (e >= num_experts || ((taken >> i) & 1u)) continue;
+        const float v = __ldg(zt + e);
+        if (v != v) {
+          nan_seen = true;
+          continue;
+        }
+        if (v > bz || (v == bz && e < be)) {
+          bz = v;
+          be = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const float oz = __shfl_xor_sync(0xFFFFFFFFu, bz, o);
+        const int oe = __shfl_xor_sync(0xFFFFFFFFu, be, o);
+        if (oz > bz || (oz == bz && oe < be)) {
+          bz = oz;
+          be = oe;
+        }
+      }
+      if (be != INT_MAX && (be & 31) == lane) taken |= 1u << (be >> 5);
+      if (lane == j) {
+        myz = bz;
+        mye = be;
+      }
+    }
+    if (__any_sync(0xFFFFFFFFu, nan_seen) && lane == 0) raise_status(TQ_DEV_NONFINITE);
+    const float zmax = __shfl_sync(0xFFFFFFFFu, myz, 0);
+    const double ex = (lane < topk && mye != INT_MAX) ? exp(static_cast<double>(myz) - static_cast<double>(zmax)) : 0.0;
+    double sum = ex;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) sum += __shfl_xor_sync(0xFFFFFFFFu, sum, o);
+    if (lane < topk) {
+      ids[t * topk + lane] = (mye == INT_MAX) ? -1 : mye;
+      w[t * topk + lane] = static_cast<float>(ex / sum);
+    }
+  }
+}
+
+__global__ void __launch_bounds__(1024) moe_route_kernel(const int32_t* __restrict__ ids_in, int64_t npairs,
                                                          int32_t num_experts, int32_t* __restrict__ offsets,
                                                          int32_t* __restrict__ pairs, int4* __restrict__ segs,
                                                          int32_t* __restrict__ nseg_out, int32_t chunk,
-                                                         int32_t* __restrict__ npairs_valid) {
+                                                         int32_t* __restrict__ npairs_valid,
+                                                         const float* __restrict__ logits, int32_t topk,
+                                                         int32_t* __restrict__ ids_out, float* __restrict__ w_out) {
   extern __shared__ int32_t sh[];
+  if (logits) {
+    router_rows(logits, npairs / topk, num_experts, topk, ids_out, w_out);
+    __syncthreads();   // the ids written above are read by the whole block below
+  }
+  const int32_t* ids = logits ? ids_out : ids_in;
   int32_t* cnt = sh;                       // [num_experts]
   int32_t* base = sh + num_experts;        // [num_experts]
   __shared__ int32_t s_bad;
@@ -410,15 +548,43 @@ static int grid_threads(int64_t threads_needed, int threads) {
   return static_cast<int>(blocks);
 }
 
+cudaError_t launch_quantize_batch(const QuantItem* items, int count, int dtype, const CodebookF32& cb,
+                                  cudaStream_t st) {
+  for (int i0 = 0; i0 < count; i0 += kQuantBatch) {
+    QuantBatch qb{};
+    qb.count = count - i0 < kQuantBatch ? count - i0 : kQuantBatch;
+    int64_t chunks = 0;
+    for (int i = 0; i < qb.count; ++i) {
+      const QuantItem& it = items[i0 + i];
+      QuantTensor& q = qb.t[i];
+      q.W = it.W;
+      q.codes = it.codes;
+      q.scales = it.scales;
+      q.nblocks = it.rows * (it.k / 32);
+      q.chunk0 = chunks;
+      q.mask = it.mask;
+      chunks += (q.nblocks + 31) / 32;
+    }
+    qb.nchunks = chunks;
+    if (chunks == 0) continue;
+    int64_t blocks = (chunks + 7) / 8;
+    const int64_t cap = 148LL * 6;
+    if (blocks > cap) blocks = cap;
+    if (dtype == TQ_DTYPE_F32)
+      quantize_kernel<float><<<static_cast<int>(blocks), 256, 0, st>>>(qb, cb);
+    else
+      quantize_kernel<uint16_t><<<static_cast<int>(blocks), 256, 0, st>>>(qb, cb);
+    note_launches(1);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
 cudaError_t launch_quantize(const void* W, int dtype, uint8_t* codes, uint16_t* scales, int64_t rows, int64_t k,
                             uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
-  const int g = grid_threads(rows * (k / 32), 256);
-  if (dtype == TQ_DTYPE_F32)
-    quantize_kernel<float><<<g, 256, 0, st>>>(static_cast<const float*>(W), codes, scales, rows, k, mask, cb);
-  else
-    quantize_kernel<uint16_t><<<g, 256, 0, st>>>(static_cast<const uint16_t*>(W), codes, scales, rows, k, mask, cb);
-  note_launches(1);
-  return cudaGetLastError();
+  const QuantItem it{W, codes, scales, rows, k, mask};
+  return launch_quantize_batch(&it, 1, dtype, cb, st);
 }
 
 cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, float* out, int64_t rows, int64_t k,
@@ -468,9 +634,25 @@ cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* ga
 
 cudaError_t launch_moe_route(const int32_t* ids, int64_t npairs, int32_t num_experts, int32_t* offsets,
                              int32_t* pairs, int4* segs, int32_t* nseg, int32_t chunk, int32_t* npairs_valid,
-                             cudaStream_t st) {
+                             cudaStream_t st, const float* logits, int32_t topk, int32_t* ids_out, float* w_out) {
   const size_t sh = sizeof(int32_t) * 2 * static_cast<size_t>(num_experts);
-  moe_route_kernel<<<1, 1024, sh, st>>>(ids, npairs, num_experts, offsets, pairs, segs, nseg, chunk, npairs_valid);
+  moe_route_kernel<<<1, 1024, sh, st>>>(ids, npairs, num_experts, offsets, pairs, segs, nseg, chunk, npairs_valid,
+                                        logits, topk, ids_out, w_out);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+// The router alone (parity hook): one CTA of 32 warps per 32 tokens.
+__global__ void __launch_bounds__(1024) router_kernel(const float* __restrict__ logits, int64_t m, int32_t num_experts,
+                                                      int32_t topk, int32_t* __restrict__ ids, float* __restrict__ w) {
+  const int64_t t0 = static_cast<int64_t>(blockIdx.x) * 32;
+  const int64_t rows = m - t0 < 32 ? m - t0 : 32;
+  router_rows(logits + t0 * num_experts, rows, num_experts, topk, ids + t0 * topk, w + t0 * topk);
+}
+
+cudaError_t launch_router(const float* logits, int64_t m, int32_t num_experts, int32_t topk, int32_t* ids, float* w,
+                          cudaStream_t st) {
+  router_kernel<<<static_cast<unsigned>((m + 31) / 32), 1024, 0, st>>>(logits, m, num_experts, topk, ids, w);
   note_launches(1);
   return cudaGetLastError();
 }

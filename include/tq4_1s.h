@@ -118,6 +118,16 @@ int tq4_1s_codebook(float* levels, float* thresholds);
  * arithmetic (NaN scales are stored as 0x7E00, NaN codes as 0). */
 int tq4_1s_quantize(const void* W, int dtype, const tq4_1s_weight* out, tq4_stream_t stream);
 
+/* tq4_1s_quantize for `count` tensors in as few launches as possible (up to
+ * 48 tensors per launch), as when a whole checkpoint is converted
+ * ("Reproduction": the quantizer runs on the GPU).  W is a HOST array of
+ * `count` device pointers, outs a HOST array of `count` weight descriptors;
+ * tensor i is quantized from W[i] into outs[i] exactly as tq4_1s_quantize
+ * would (same bits), all inputs of one dtype.  Every descriptor and pointer
+ * is validated before anything is launched; count == 0 is a no-op. */
+int tq4_1s_quantize_batched(const void* const* W, int dtype, const tq4_1s_weight* outs, int32_t count,
+                            tq4_stream_t stream);
+
 /* Dequantize a packed tensor stack to fp32 W_out (device, [E][n][k]):
  * W_hat = diag(s) * r * H * (c[code] * d) per block.  Test/debug path. */
 int tq4_1s_dequantize(const tq4_1s_weight* w, float* W_out, tq4_stream_t stream);
@@ -198,6 +208,33 @@ size_t tq4_1s_moe_workspace(int64_t m, int32_t topk, const tq4_1s_weight* up, co
 int tq4_1s_moe(const uint16_t* x, int64_t m, const int32_t* topk_ids, const float* topk_w, int32_t topk,
                const tq4_1s_weight* up, const tq4_1s_weight* down, uint16_t* y, void* ws, size_t ws_bytes,
                tq4_stream_t stream);
+
+/* tq4_1s_moe with the router on the device (model card, "Performance": the
+ * MoE made sync-free; "The model underneath": top-6 of 128 experts): the
+ * routing decisions come from the router's logits instead of the caller.
+ *   logits device float [m][E] (E = up->num_experts <= 1024), 16-byte
+ *          aligned; topk <= 32 and <= E.
+ * Per token: softmax over all E experts, the topk of largest probability
+ * chosen (equal logits: the lower expert id first), their probabilities
+ * renormalised to sum to 1 -- as tq4_1s_router_topk -- then the layer of
+ * tq4_1s_moe with those ids and weights.  The router runs inside the routing
+ * kernel, so the call is the same number of launches as tq4_1s_moe, needs no
+ * host sync, and captures into a CUDA graph.  Workspace: tq4_1s_moe_workspace
+ * (it includes room for the router's output).  A NaN logit is never chosen
+ * and sets TQ_DEV_NONFINITE. */
+int tq4_1s_moe_logits(const uint16_t* x, int64_t m, const float* logits, int32_t topk, const tq4_1s_weight* up,
+                      const tq4_1s_weight* down, uint16_t* y, void* ws, size_t ws_bytes, tq4_stream_t stream);
+
+/* The MoE router on its own (parity hook and standalone use):
+ *   logits  device float [m][num_experts] (num_experts <= 1024);
+ *   ids     device int32 [m][topk] (topk <= 32, <= num_experts): the chosen
+ *           experts in descending logit order, equal logits lower id first;
+ *   weights device float [m][topk]: exp(z_j - z_max) / sum over the chosen,
+ *           i.e. the full softmax restricted to the chosen and renormalised
+ *           (computed in fp64, rounded to fp32).
+ * m == 0 is a no-op. */
+int tq4_1s_router_topk(const float* logits, int64_t m, int32_t num_experts, int32_t topk, int32_t* ids,
+                       float* weights, tq4_stream_t stream);
 
 /* The routing step of tq4_1s_moe on its own (exposed for parity tests):
  * offsets (device int32 [num_experts + 1]) = exclusive prefix of per-expert

@@ -115,6 +115,50 @@ def test_static_entry_validation_and_scratch_limits():
     assert tq.tq4_1s_error_string(9).startswith("shape exceeds the fixed scratch")
 
 
+def test_router_and_moe_logits_validation():
+    lib = tq.load_library()
+    null = ctypes.c_void_p(0)
+    good = ctypes.c_void_p(4096)
+    assert lib.tq4_1s_router_topk(good, 0, 128, 6, good, good, null) == 0      # m == 0: no-op
+    assert lib.tq4_1s_router_topk(good, -1, 128, 6, good, good, null) == 1
+    assert lib.tq4_1s_router_topk(good, 4, 1025, 6, good, good, null) == 1     # more than 1024 experts
+    assert lib.tq4_1s_router_topk(good, 4, 128, 33, good, good, null) == 1     # topk > 32
+    assert lib.tq4_1s_router_topk(good, 4, 4, 5, good, good, null) == 1        # topk > E
+    assert lib.tq4_1s_router_topk(null, 4, 128, 6, good, good, null) == 1
+    assert lib.tq4_1s_router_topk(good, 4, 128, 6, good, null, null) == 1
+    up, dn = _weight(n=128, k=64, e=4), _weight(n=64, k=128, e=4)
+    assert lib.tq4_1s_moe_logits(good, 4, null, 2, ctypes.byref(up), ctypes.byref(dn), good, good, 1 << 20,
+                                 null) == 1                                    # no logits
+    assert lib.tq4_1s_moe_logits(good, 4, good, 5, ctypes.byref(up), ctypes.byref(dn), good, good, 1 << 20,
+                                 null) == 1                                    # topk > E
+    assert lib.tq4_1s_moe_logits(good, 4, ctypes.c_void_p(4100), 2, ctypes.byref(up), ctypes.byref(dn), good,
+                                 good, 1 << 20, null) == 2                     # misaligned logits
+    big_u, big_d = _weight(n=128, k=64, e=1025), _weight(n=64, k=128, e=1025)
+    assert lib.tq4_1s_moe_logits(good, 4, good, 2, ctypes.byref(big_u), ctypes.byref(big_d), good, good,
+                                 1 << 20, null) == 1                           # router limit: 1024 experts
+    assert lib.tq4_1s_moe_logits(good, 0, good, 2, ctypes.byref(up), ctypes.byref(dn), good, good, 0,
+                                 null) == 0                                    # m == 0: no-op
+
+
+def test_quantize_batched_validation():
+    lib = tq.load_library()
+    null = ctypes.c_void_p(0)
+    ws = (tq._Weight * 2)(_weight(), _weight())
+    ptrs = (ctypes.c_void_p * 2)(4096, 8192)
+    cw, cp = ctypes.cast(ws, ctypes.c_void_p), ctypes.cast(ptrs, ctypes.c_void_p)
+    assert lib.tq4_1s_quantize_batched(cp, 0, cw, 0, null) == 0           # count 0: no-op
+    assert lib.tq4_1s_quantize_batched(cp, 0, cw, -1, null) == 1
+    assert lib.tq4_1s_quantize_batched(null, 0, cw, 2, null) == 1         # no pointer array
+    assert lib.tq4_1s_quantize_batched(cp, 0, null, 2, null) == 1         # no descriptors
+    assert lib.tq4_1s_quantize_batched(cp, 5, cw, 2, null) == 1           # bad dtype
+    bad = (tq._Weight * 2)(_weight(), _weight(k=48))                       # second one invalid
+    assert lib.tq4_1s_quantize_batched(cp, 0, ctypes.cast(bad, ctypes.c_void_p), 2, null) == 1
+    mis = (ctypes.c_void_p * 2)(4096, 8200)                                # second W misaligned
+    assert lib.tq4_1s_quantize_batched(ctypes.cast(mis, ctypes.c_void_p), 0, cw, 2, null) == 2
+    nul = (ctypes.c_void_p * 2)(4096, 0)
+    assert lib.tq4_1s_quantize_batched(ctypes.cast(nul, ctypes.c_void_p), 0, cw, 2, null) == 1
+
+
 @pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU error path")
 def test_valid_call_without_gpu_fails_loudly():
     lib = tq.load_library()
@@ -124,6 +168,9 @@ def test_valid_call_without_gpu_fails_loudly():
     assert need > 0
     assert lib.tq4_1s_linear(good, 16, ctypes.byref(w), good, good, need, ctypes.c_void_p(0)) == 3
     assert lib.tq4_1s_quantize(good, 0, ctypes.byref(w), ctypes.c_void_p(0)) == 3
+    ws1, p1 = (tq._Weight * 1)(w), (ctypes.c_void_p * 1)(4096)
+    assert lib.tq4_1s_quantize_batched(ctypes.cast(p1, ctypes.c_void_p), 0, ctypes.cast(ws1, ctypes.c_void_p), 1,
+                                       ctypes.c_void_p(0)) == 3
     assert lib.tq4_1s_linear_static(good, 16, ctypes.byref(w), good, ctypes.c_void_p(0)) == 3
 
 

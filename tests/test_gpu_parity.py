@@ -74,6 +74,28 @@ def test_quantize_bf16_input_bit_exact():
     assert np.array_equal(p.scales[0].cpu().numpy().view(np.uint16), scales)
 
 
+def test_quantize_batched_bit_exact_against_oracle():
+    # tensors of different shapes, seeds and block counts (one not a multiple
+    # of 32 blocks, so a warp chunk ends inside it) quantized in one launch
+    shapes = [(200, 96), (1, 32), (3, 64, 160), (257, 128), (64, 4096)]
+    Ws = [synth.normal_f32(s, 50 + i, 0.02) for i, s in enumerate(shapes)]
+    seeds = [50 + i for i in range(len(shapes))]
+    outs = tq.tq4_1s_quantize_batched([torch.from_numpy(W).to(DEV) for W in Ws], seeds)
+    torch.cuda.synchronize()
+    for W, seed, p in zip(Ws, seeds, outs):
+        codes, scales, _ = oracle.quantize(W.reshape(-1, W.shape[-1]), seed)
+        assert np.array_equal(p.codes.cpu().numpy().reshape(codes.shape), codes)
+        assert np.array_equal(p.scales.cpu().numpy().view(np.uint16).reshape(scales.shape), scales)
+    # bf16 inputs, batched
+    Wb = [synth.f32_to_bf16_bits(synth.normal_f32((96, 192), 60 + i, 0.05)) for i in range(3)]
+    outs = tq.tq4_1s_quantize_batched([_bf16_dev(b) for b in Wb], [60, 61, 62])
+    for b, seed, p in zip(Wb, [60, 61, 62], outs):
+        codes, scales, _ = oracle.quantize(synth.bf16_bits_to_f32(b), seed)
+        assert np.array_equal(p.codes[0].cpu().numpy(), codes)
+        assert np.array_equal(p.scales[0].cpu().numpy().view(np.uint16), scales)
+    assert tq.tq4_1s_get_status() == 0
+
+
 def test_quantize_special_blocks_and_status():
     W = np.zeros((3, 64), np.float32)
     W[1, 32:] = synth.normal_f32(32, 41)
