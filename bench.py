@@ -47,14 +47,10 @@ M_TOK, N_OUT, K_IN = 16, 4096, 4096
 CALLS = 16
 COPIES = 64
 PACKED_PER_CALL = N_OUT * K_IN // 2 + N_OUT * (K_IN // 16) * 2   # 10,485,760 B
-# DRAM bytes (read + write) of one decode launch of the kernel, from the ncu
-# capture summarised in profiles/streamk_decode_m16_n4096_k4096.md.  The
-# kernel has changed since (the split-tile counter reset of the stream-K
-# fix-up, a path the decode shape's cluster split-K mode does not run), so
-# the line reports traffic as null until the counters are taken again and
-# gives this figure separately.
+# DRAM bytes (read + write) of one decode launch (ncu dram__bytes_read.sum +
+# dram__bytes_write.sum of decode_kernel); None until taken on the current
+# kernel.
 TRAFFIC_PER_CALL = None
-TRAFFIC_BEFORE_CHANGE = 10_703_872
 WORKLOAD = ("decode_linear_4096: x bf16 [16][4096] N(0,1), W 4096x4096 Student-t(5)*0.02 TQ4_1S, "
             "16 calls per step (denoising steps)")
 
@@ -158,6 +154,38 @@ def cpu_oracle_sample(target_s: float = 12.0):
                       f"in {el:.1f} s, single thread"}
 
 
+def _oracle_decode_worker(args):
+    """One host process of the all-cores oracle baseline: quantize the decode
+    weight with the oracle, then run oracle calls until `seconds` have passed.
+    Returns (calls, seconds spent in calls)."""
+    seconds, wid = args
+    import oracle
+    import synth
+    W = synth.student_t_f32((N_OUT, K_IN), 2, 5.0, 0.02)
+    codes, scales, _ = oracle.quantize(W, 2)
+    calls, t0 = 0, time.perf_counter()
+    while time.perf_counter() - t0 < seconds:
+        oracle.linear(synth.activations_bf16(M_TOK, K_IN, 1000 + 97 * wid + calls), codes, scales, 2)
+        calls += 1
+    return calls, time.perf_counter() - t0
+
+
+def cpu_oracle_all_cores(seconds: float = 8.0):
+    """The oracle on every host core the process may use: one spawned process
+    per core (spawned, not forked, since CUDA is initialised), each running
+    decode calls for `seconds`; throughput = all calls / the slowest worker."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+    cores = len(os.sched_getaffinity(0)) if hasattr(os, "sched_getaffinity") else (os.cpu_count() or 1)
+    with cf.ProcessPoolExecutor(max_workers=cores, mp_context=mp.get_context("spawn")) as ex:
+        res = list(ex.map(_oracle_decode_worker, [(seconds, i) for i in range(cores)]))
+    calls = sum(c for c, _ in res)
+    el = max(t for _, t in res)
+    return {"value": calls * PACKED_PER_CALL / el / 1e9, "unit": "GB/s", "cores": cores, "kind": "oracle",
+            "sample": f"{calls} decode calls (dequantize 4096x4096 + fp64 GEMV) in {el:.1f} s on {cores} "
+                      f"processes, one per core of the affinity mask"}
+
+
 def reference_arm(args):
     rank = int(os.environ.get("RANK", "0"))
     if rank != 0:
@@ -228,7 +256,11 @@ def ours_arm(args):
     W = torch.from_numpy(synth.student_t_f32((N_OUT, K_IN), 2, 5.0, 0.02)).to(dev)
     base = tq.tq4_1s_quantize(W, seed=2)
     del W
-    copies = [tq.Packed(base.codes.clone(), base.scales.clone(), N_OUT, K_IN, 1, 2) for _ in range(COPIES)]
+    # weights quantized once and synchronized: static, as in inference (the
+    # decode kernel may stream them before the previous call has finished)
+    copies = [tq.Packed(base.codes.clone(), base.scales.clone(), N_OUT, K_IN, 1, 2, flags=tq.TQ_WEIGHT_STATIC)
+              for _ in range(COPIES)]
+    torch.cuda.synchronize()
     xs = torch.stack([torch.from_numpy(synth.activations_bf16(M_TOK, K_IN, 3 + j).view(np.int16))
                       for j in range(CALLS)]).to(dev).view(torch.bfloat16)
     ys = torch.empty((CALLS, M_TOK, N_OUT), dtype=torch.bfloat16, device=dev)
@@ -289,6 +321,23 @@ def ours_arm(args):
     # ---- eager (no graph) per-call number, for context
     ms_eager = timed(lambda i: step(i % ngraphs), max(3, args.steps // 2)) / max(3, args.steps // 2)
 
+    # ---- the same graphs with the weights not flagged static: every read of
+    # the weight waits for the previous kernel (the library's default)
+    plain = [tq.Packed(c.codes, c.scales, N_OUT, K_IN, 1, 2) for c in copies]
+    graphs_plain = []
+    saved = copies[:]
+    copies[:] = plain
+    for g in range(ngraphs):
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr, stream=capture_stream):
+            step(g)
+        graphs_plain.append(gr)
+    copies[:] = saved
+    for i in range(3):
+        graphs_plain[i % ngraphs].replay()
+    ms_plain = timed(lambda i: graphs_plain[i % ngraphs].replay(), args.steps) / args.steps
+    del graphs_plain
+
     # ---- end to end through the public API with host buffers: the step's
     # input block comes from pinned host memory, its result goes back to it
     x_host = xs[0].view(torch.int16).cpu().pin_memory()
@@ -318,7 +367,13 @@ def ours_arm(args):
         dist.barrier()
     del graphs
     if rank == 0:
-        cpu = cpu_oracle_sample() if world == 1 else None
+        cpu = None
+        if world == 1:
+            cpu = cpu_oracle_sample()
+            try:
+                cpu["all_cores"] = cpu_oracle_all_cores()
+            except Exception as exc:   # (reported, not fatal: the baseline is context)
+                cpu["all_cores"] = {"unavailable": repr(exc)[:200]}
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
@@ -330,14 +385,17 @@ def ours_arm(args):
                                       "first input is a fixed N(0,1) block"},
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
                          "frac": achieved / pk["hbm_gbs"], "traffic": TRAFFIC_PER_CALL,
-                         "traffic_before_last_kernel_change": TRAFFIC_BEFORE_CHANGE,
                          "algorithmic_bytes": PACKED_PER_CALL,
-                         "kernel": "streamk_kernel, fused cluster split-K mode: one launch per tq4_1s_linear "
-                                   "call (x staging and rotation, dequant, MMA, on-chip reduction)",
-                         "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one launch, "
-                                           "profiles/streamk_decode_m16_n4096_k4096.md",
+                         "kernel": "decode_kernel<1>: one launch per tq4_1s_linear call (x rotation, dequant, "
+                                   "tcgen05 MMA, cluster reduction), 32 row tiles x 4-CTA clusters",
+                         "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one "
+                                           "decode_kernel launch",
                          "peak_source": pk["source"], "per_call_us": per_call_ms * 1e3},
             "eager_per_call_us": ms_eager / CALLS * 1e3,
+            "weights_not_static": {"value": job_gbs(world, CALLS * PACKED_PER_CALL, ms_plain), "unit": "GB/s",
+                                   "per_call_us": ms_plain / CALLS * 1e3,
+                                   "note": "same graphs without TQ_WEIGHT_STATIC: weight reads wait for the "
+                                           "previous kernel"},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": clk,
@@ -369,9 +427,10 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     ms = timed(lambda i: tq.tq4_1s_linear(x, p, out=y, workspace=wsp), it) / it
     fl = 2.0 * m * n * k
     tf = fl / (ms * 1e-3) / 1e12
+    # 10 back-to-back calls (~8 ms) are an isolated timing: the burst peak
     out["prefill_linear_8192"] = {"value": tf, "unit": "TFLOP/s", "ms_per_call": ms,
-                                  "frac_of_bf16_peak": tf / pk["bf16_tflops_sustained"],
-                                  "peak": pk["bf16_tflops_sustained"], "peak_kind": "sustained",
+                                  "frac_of_bf16_peak": tf / pk["bf16_tflops"],
+                                  "peak": pk["bf16_tflops"], "peak_kind": "burst",
                                   "note": "includes the bf16 dequantize pre-pass"}
     del x, y, wsp, p
     torch.cuda.empty_cache()
@@ -396,6 +455,30 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     out["moe_128x_top6_m16"] = {"value": gbs, "unit": "GB/s", "ms_per_call": ms,
                                 "touched_bytes_per_call": sum(touched) / 4,
                                 "frac_of_hbm": gbs / pk["hbm_gbs"]}
+    # quantize throughput: the up-projection expert stack (638M fp32 weights,
+    # 4 B read + 0.625 B written per weight) and the decode weight
+    q = {}
+    for name, shp, seed in (("expert_stack_128x1856x2688_f32", (E, I, H), 4),
+                            ("decode_weight_4096x4096_f32", (4096, 4096), 2)):
+        W = synth.normal_f32_device(shp, seed, 0.02, dev)
+        pq = tq.tq4_1s_quantize(W, seed=seed)
+        for _ in range(2):
+            tq.tq4_1s_quantize(W, seed=seed, out=pq)
+        it = 5
+        ms = timed(lambda i: tq.tq4_1s_quantize(W, seed=seed, out=pq), it) / it
+        nw = W.numel()
+        gb = nw * 4.625 / (ms * 1e-3) / 1e9
+        q[name] = {"weights_per_s": nw / (ms * 1e-3), "gbs": gb, "ms_per_call": ms,
+                   "frac_of_hbm": gb / pk["hbm_gbs"]}
+        del W, pq
+    out["quantize"] = q
+    del up, dn
+    torch.cuda.empty_cache()
+    # the 52-layer denoise sweep: whole step in one CUDA graph, 2 timed steps
+    meas, layers, b, _ = sweep_measure(tq, synth, dev, pk, timed, steps=2, warmup=1)
+    out["denoise_sweep_52"] = meas
+    del layers, b
+    torch.cuda.empty_cache()
     return out
 
 
@@ -453,8 +536,123 @@ def sweep_cpu_sample(rows: int = 64):
                       f"{el:.2f} s, single thread, scaled x{wl['m'] // rows} to the 512-token step"}
 
 
-def sweep_arm(args):
+def build_sweep(tq, synth, dev):
+    """The 52 layers of the sweep, quantized on the device from bf16 weights
+    (a bf16 checkpoint, as the model card's quantizer converts one): each
+    layer's four tensors are drawn on the device (not timed), rounded to
+    bf16, and quantized in one batched launch (timed with CUDA events).
+    Router logits (fp32, Gumbel-perturbed) and activations per layer.
+    Returns (layers, quantize_ms, weights)."""
     import numpy as np
+    import torch
+    wl, shapes = sweep_shapes()
+    L, m, E, H = wl["layers"], wl["m"], wl["num_experts"], wl["hidden"]
+    layers, q_events = [], []
+    for l in range(L):
+        Ws, seeds = [], []
+        for j, (name, shp) in enumerate(shapes):
+            seeds.append(synth.sweep_seed(l, j))
+            Ws.append(synth.normal_f32_device(shp, seeds[-1], wl["w_std"], dev).to(torch.bfloat16))
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        packed = tq.tq4_1s_quantize_batched(Ws, seeds)
+        e1.record()
+        q_events.append((e0, e1))
+        del Ws
+        # weights written by the quantize above are read only after the
+        # synchronize below: static from then on
+        ly = {name: tq.Packed(p.codes, p.scales, p.n, p.k, p.num_experts, p.seed, flags=tq.TQ_WEIGHT_STATIC)
+              for (name, _), p in zip(shapes, packed)}
+        z = synth.router_logits_f32(m, E, synth.sweep_seed(l, 5))
+        top = np.argsort(-z, axis=1, kind="stable")[:, :wl["topk"]]
+        ly["touched"] = len(set(top.ravel().tolist()))
+        ly["logits"] = torch.from_numpy(z).to(dev)
+        ly["x"] = synth.normal_f32_device((m, H), synth.sweep_seed(l, 4), 1.0, dev).to(torch.bfloat16)
+        layers.append(ly)
+    torch.cuda.synchronize()
+    q_ms = sum(a.elapsed_time(b) for a, b in q_events)
+    torch.cuda.empty_cache()
+    return layers, q_ms, sweep_weights()
+
+
+def sweep_buffers(tq, layers, dev):
+    import torch
+    wl, _ = sweep_shapes()
+    m, H, topk, n_mid = wl["m"], wl["hidden"], wl["topk"], wl["dense"][0][0]
+    ly0 = layers[0]
+    return {
+        "y_moe": torch.empty((m, H), dtype=torch.bfloat16, device=dev),
+        "t_mid": torch.empty((m, n_mid), dtype=torch.bfloat16, device=dev),
+        "y_out": torch.empty((m, H), dtype=torch.bfloat16, device=dev),
+        "ws_moe": torch.empty(tq.tq4_1s_moe_workspace(m, topk, ly0["up"], ly0["down"]), dtype=torch.uint8,
+                              device=dev),
+        "ws_lin": torch.empty(max(tq.tq4_1s_linear_workspace(m, ly0["dense_in"]),
+                                  tq.tq4_1s_linear_workspace(m, ly0["dense_out"])), dtype=torch.uint8, device=dev),
+    }
+
+
+def sweep_step(tq, layers, b, xs=None):
+    """One denoise step: per layer the MoE block routed on the device from
+    its logits, and the two dense projections (the second consumes the
+    first's output).  No host sync: the whole step captures into one graph."""
+    wl, _ = sweep_shapes()
+    for l, ly in enumerate(layers):
+        x = ly["x"] if xs is None else xs[l]
+        tq.tq4_1s_moe_logits(x, ly["logits"], wl["topk"], ly["up"], ly["down"], out=b["y_moe"],
+                             workspace=b["ws_moe"])
+        tq.tq4_1s_linear(x, ly["dense_in"], out=b["t_mid"], workspace=b["ws_lin"])
+        tq.tq4_1s_linear(b["t_mid"], ly["dense_out"], out=b["y_out"], workspace=b["ws_lin"])
+
+
+def sweep_measure(tq, synth, dev, pk, timed, steps, warmup):
+    """Build the sweep, capture one step as a CUDA graph, check that a replay
+    reproduces the eager step's outputs bit for bit, and time graph replays
+    (device time, CUDA events).  Returns the measurement dict."""
+    import torch
+    wl, _ = sweep_shapes()
+    E = wl["num_experts"]
+    layers, q_ms, n_weights = build_sweep(tq, synth, dev)
+    b = sweep_buffers(tq, layers, dev)
+    per_expert = layers[0]["up"].nbytes // E + layers[0]["down"].nbytes // E
+    step_bytes = sum(ly["touched"] * per_expert + ly["dense_in"].nbytes + ly["dense_out"].nbytes for ly in layers)
+    l0 = tq.tq4_1s_launch_count()
+    sweep_step(tq, layers, b)
+    launches = tq.tq4_1s_launch_count() - l0
+    torch.cuda.synchronize()
+    assert tq.tq4_1s_get_status() == 0, "device status word set by the eager sweep step"
+    ref = (b["y_moe"].clone(), b["y_out"].clone())
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=torch.cuda.Stream(dev)):
+        sweep_step(tq, layers, b)
+    for t in ("y_moe", "y_out"):
+        b[t].zero_()
+    g.replay()
+    torch.cuda.synchronize()
+    same = torch.equal(b["y_moe"].view(torch.int16), ref[0].view(torch.int16)) and \
+        torch.equal(b["y_out"].view(torch.int16), ref[1].view(torch.int16))
+    for i in range(warmup):
+        g.replay()
+    ms_graph = timed(lambda i: g.replay(), steps) / steps
+    ms_eager = timed(lambda i: sweep_step(tq, layers, b), max(1, steps // 2)) / max(1, steps // 2)
+    assert tq.tq4_1s_get_status() == 0, "device status word set during the sweep"
+    out = {"value": step_bytes / (ms_graph * 1e-3) / 1e9, "unit": "GB/s", "ms_per_step": ms_graph,
+           "frac_of_hbm": step_bytes / (ms_graph * 1e-3) / 1e9 / pk["hbm_gbs"],
+           "packed_bytes_per_step": step_bytes, "launches_per_step": launches,
+           "graph": "whole 52-layer step in one CUDA graph (router on the device, no host sync)",
+           "graph_replay_bit_identical_to_eager": bool(same),
+           "eager_ms_per_step": ms_eager,
+           "quantize": {"weights_per_s": n_weights / (q_ms * 1e-3), "ms_total": q_ms,
+                        "gbs": n_weights * 2.625 / (q_ms * 1e-3) / 1e9,
+                        "bytes_per_weight": "2 read (bf16) + 0.625 written (packed)",
+                        "launches": len(layers), "input": "bf16 (a checkpoint's dtype)",
+                        "weights": n_weights,
+                        "note": "device time of one batched quantize launch per layer (4 tensors); "
+                                "weight generation not timed"}}
+    del g
+    return out, layers, b, step_bytes
+
+
+def sweep_arm(args):
     import torch
     import torch.distributed as dist
 
@@ -470,59 +668,8 @@ def sweep_arm(args):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
     pk = peaks()
     wl, shapes = sweep_shapes()
-    L, m, topk, E, H = wl["layers"], wl["m"], wl["topk"], wl["num_experts"], wl["hidden"]
+    L, m, H = wl["layers"], wl["m"], wl["hidden"]
     n_mid = wl["dense"][0][0]
-
-    # ---- build: weights drawn on the device per layer (not timed), quantized
-    # (timed with events on the launching stream)
-    layers = []
-    q_events = []
-    for l in range(L):
-        packed = {}
-        for j, (name, shp) in enumerate(shapes):
-            seed = synth.sweep_seed(l, j)
-            W = synth.normal_f32_device(shp, seed, wl["w_std"], dev)
-            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-            e0.record()
-            packed[name] = tq.tq4_1s_quantize(W, seed=seed)
-            e1.record()
-            q_events.append((e0, e1))
-            del W
-        ids, w = synth.gumbel_topk_router(m, E, topk, synth.sweep_seed(l, 5))
-        x = synth.activations_bf16(m, H, synth.sweep_seed(l, 4))
-        packed["touched"] = len(set(ids.ravel().tolist()))
-        packed["ids"] = torch.from_numpy(ids).to(dev)
-        packed["w"] = torch.from_numpy(w).to(dev)
-        packed["x"] = torch.from_numpy(x.view(np.int16)).to(dev).view(torch.bfloat16)
-        layers.append(packed)
-    torch.cuda.synchronize()
-    q_ms = sum(a.elapsed_time(b) for a, b in q_events)
-    n_weights = sweep_weights()
-    torch.cuda.empty_cache()
-
-    per_expert = layers[0]["up"].nbytes // E + layers[0]["down"].nbytes // E
-    step_bytes = sum(ly["touched"] * per_expert + ly["dense_in"].nbytes + ly["dense_out"].nbytes for ly in layers)
-    y_moe = torch.empty((m, H), dtype=torch.bfloat16, device=dev)
-    t_mid = torch.empty((m, n_mid), dtype=torch.bfloat16, device=dev)
-    y_out = torch.empty((m, H), dtype=torch.bfloat16, device=dev)
-    ws_moe = torch.empty(tq.tq4_1s_moe_workspace(m, topk, layers[0]["up"], layers[0]["down"]),
-                         dtype=torch.uint8, device=dev)
-    ws_lin = torch.empty(max(tq.tq4_1s_linear_workspace(m, layers[0]["dense_in"]),
-                             tq.tq4_1s_linear_workspace(m, layers[0]["dense_out"])), dtype=torch.uint8, device=dev)
-
-    def step(i, xs=None):
-        # one denoise step: every layer's MoE block and its two dense
-        # projections (the second consumes the first's output)
-        for l, ly in enumerate(layers):
-            x = ly["x"] if xs is None else xs[l]
-            tq.tq4_1s_moe(x, ly["ids"], ly["w"], ly["up"], ly["down"], out=y_moe, workspace=ws_moe)
-            tq.tq4_1s_linear(x, ly["dense_in"], out=t_mid, workspace=ws_lin)
-            tq.tq4_1s_linear(t_mid, ly["dense_out"], out=y_out, workspace=ws_lin)
-
-    for i in range(args.warmup):
-        step(i)
-    torch.cuda.synchronize()
-    assert tq.tq4_1s_get_status() == 0, "device status word set during warm-up"
 
     def timed(fn, k):
         if world > 1:
@@ -542,14 +689,10 @@ def sweep_arm(args):
     clocks = ClockSampler(local)
     clocks.start()
     time.sleep(0.3)
-    l0 = tq.tq4_1s_launch_count()
-    ms = timed(step, args.steps)
-    launches = tq.tq4_1s_launch_count() - l0
+    meas, layers, b, step_bytes = sweep_measure(tq, synth, dev, pk, timed, args.steps, args.warmup)
     clk = clocks.stop()
-    assert tq.tq4_1s_get_status() == 0, "device status word set during the timed region"
-    ms_step = ms / args.steps
+    ms_step = meas["ms_per_step"]
     value = job_gbs(world, step_bytes, ms_step)
-    achieved = step_bytes / (ms_step * 1e-3) / 1e9
 
     # ---- end to end: each step's per-layer input blocks come from pinned
     # host memory; the last layer's two outputs go back to it
@@ -560,9 +703,9 @@ def sweep_arm(args):
     def e2e_step(i):
         for xh, xd in zip(x_host, x_dev):
             xd.view(torch.int16).copy_(xh, non_blocking=True)
-        step(i, x_dev)
-        y_host[0].copy_(y_moe.view(torch.int16), non_blocking=True)
-        y_host[1].copy_(y_out.view(torch.int16), non_blocking=True)
+        sweep_step(tq, layers, b, x_dev)
+        y_host[0].copy_(b["y_moe"].view(torch.int16), non_blocking=True)
+        y_host[1].copy_(b["y_out"].view(torch.int16), non_blocking=True)
 
     e2e_step(0)
     ke = max(3, args.steps // 2)
@@ -583,23 +726,21 @@ def sweep_arm(args):
                                    f"{wl['inter']}, down {wl['inter']}->{H}; dense {H}->{n_mid}->{H}), "
                                    f"{m} tokens (32 sequences x 16-token block) per step",
                        "global_batch": world * m, "seq_len": 16, "parallelism": f"replicas x{world}",
-                       "timing": "eager calls, one step = all layers",
+                       "timing": "one CUDA graph per step (all 52 layers), router on the device",
                        "l2": f"cold: {step_bytes / 1e9:.2f} GB of packed weights streamed per step (> 126 MB L2)",
-                       "weights": f"{n_weights / 1e9:.2f} B weights, N(0, 0.02^2) drawn on the device per layer"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": pk["hbm_gbs"], "unit": "GB/s",
-                         "frac": achieved / pk["hbm_gbs"], "traffic": None,
-                         "algorithmic_bytes": step_bytes,
-                         "kernel": "whole step (MoE route, rotations, grouped stream-K up/down, combine; "
-                                   "dense dequantize pre-pass + tcgen05 GEMM), packed bytes per step / step time",
+                       "weights": f"{meas['quantize']['weights'] / 1e9:.2f} B weights, N(0, 0.02^2) drawn on "
+                                  f"the device per layer, rounded to bf16, quantized"},
+            "roofline": {"bound": "hbm", "achieved": step_bytes / (ms_step * 1e-3) / 1e9, "peak": pk["hbm_gbs"],
+                         "unit": "GB/s", "frac": step_bytes / (ms_step * 1e-3) / 1e9 / pk["hbm_gbs"],
+                         "traffic": None, "algorithmic_bytes": step_bytes,
+                         "kernel": "whole step (MoE router + route, rotations, grouped stream-K up/down, combine; "
+                                   "dense projections), packed bytes per step / step time",
                          "peak_source": pk["source"]},
-            "quantize": {"weights_per_s": n_weights / (q_ms * 1e-3), "ms_total": q_ms,
-                         "gbs": n_weights * 4.625 / (q_ms * 1e-3) / 1e9,
-                         "bytes_per_weight": "4 read (fp32) + 0.625 written (packed)",
-                         "note": "device time of the 208 quantize calls; weight generation not timed"},
+            "sweep": meas,
             "cpu_baseline": cpu,
             "e2e": e2e,
             "clocks": clk,
-            "gpu_launches": launches,
+            "gpu_launches": meas["launches_per_step"] * args.steps,
         }
         print(json.dumps(line), flush=True)
     if world > 1:

@@ -34,6 +34,7 @@ LIB_PATH = os.path.join(_HERE, "libtq4_1s.so")
 TQ_OK = 0
 TQ_DTYPE_F32, TQ_DTYPE_BF16 = 0, 1
 TQ_DEV_TIMEOUT, TQ_DEV_BAD_ROUTING, TQ_DEV_NONFINITE, TQ_DEV_SCALE_RANGE = 1, 2, 4, 8
+TQ_WEIGHT_STATIC = 1
 
 
 class TQ4Error(RuntimeError):
@@ -45,7 +46,7 @@ class TQ4Error(RuntimeError):
 class _Weight(ctypes.Structure):
     _fields_ = [
         ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("num_experts", ctypes.c_int32),
-        ("reserved", ctypes.c_int32), ("seed", ctypes.c_uint64),
+        ("flags", ctypes.c_int32), ("seed", ctypes.c_uint64),
         ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
     ]
 
@@ -114,13 +115,15 @@ class Packed:
     k: int
     num_experts: int
     seed: int
+    flags: int = 0   # TQ_WEIGHT_STATIC: no unfinished kernel writes the planes (see include/tq4_1s.h)
 
     def c_struct(self) -> _Weight:
         # built once per (codes, scales) storage; a call only marshals a pointer to it
-        key = (self.codes.data_ptr(), self.scales.data_ptr(), self.n, self.k, self.num_experts, self.seed)
+        key = (self.codes.data_ptr(), self.scales.data_ptr(), self.n, self.k, self.num_experts, self.seed,
+               self.flags)
         cached = self.__dict__.get("_c_struct")
         if cached is None or cached[0] != key:
-            cached = (key, _Weight(self.n, self.k, self.num_experts, 0, self.seed, key[0], key[1]))
+            cached = (key, _Weight(self.n, self.k, self.num_experts, self.flags, self.seed, key[0], key[1]))
             self.__dict__["_c_struct"] = cached
         return cached[1]
 

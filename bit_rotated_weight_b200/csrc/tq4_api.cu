@@ -109,7 +109,7 @@ static int check_device(int* sms_out) {
 
 static int weight_ok(const tq4_1s_weight* w, bool need_ptrs) {
   if (!w) return TQ_ERR_INVALID_ARG;
-  if (w->n <= 0 || w->k <= 0 || (w->k % 32) != 0 || w->num_experts <= 0 || w->reserved != 0)
+  if (w->n <= 0 || w->k <= 0 || (w->k % 32) != 0 || w->num_experts <= 0 || (w->flags & ~TQ_WEIGHT_STATIC) != 0)
     return TQ_ERR_INVALID_ARG;
   if (w->n > (1ll << 30) || w->k > (1ll << 30) || w->num_experts > (1 << 20)) return TQ_ERR_INVALID_ARG;
   if (need_ptrs) {
@@ -328,7 +328,7 @@ static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUD
 using namespace tq4;
 
 // ==================================================================== ABI
-TQ_API int tq4_1s_version(void) { return 100; }
+TQ_API int tq4_1s_version(void) { return 101; }
 
 TQ_API const char* tq4_1s_error_string(int code) {
   switch (code) {
@@ -440,6 +440,31 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
   uint8_t* base = static_cast<uint8_t*>(ws);
   const uint32_t mask = sign_mask_of(w->seed);
 
+  if (small && m <= kSegRows) {
+    // the decode-block kernel: one launch, activation-dependent work only
+    // after the dependency wait (see tq4_decode.cu)
+    const int nb = m > 16 ? 2 : 1;
+    const int64_t KI = (w->k + 127) / 128;
+    const int split = choose_decode_split(L.tiles, KI, sms, nb);
+    if (split > 0) {
+      alignas(64) CUtensorMap tc;
+      if (!map_codes(&tc, w)) return TQ_ERR_CUDA;
+      DecodeArgs d{};
+      d.n = static_cast<int32_t>(w->n);
+      d.k = static_cast<int32_t>(w->k);
+      d.m = static_cast<int32_t>(m);
+      d.nb = nb;
+      d.row_tiles = static_cast<int32_t>(L.tiles);
+      d.k_iters = static_cast<int32_t>(KI);
+      d.split = split;
+      d.static_w = (w->flags & TQ_WEIGHT_STATIC) ? 1 : 0;
+      d.x = x;
+      d.scales = w->scales;
+      d.y = y;
+      sign_xor_words(mask, d.x_sign);
+      return cuda_rc(launch_decode(&tc, d, st));
+    }
+  }
   if (small) {
     const int64_t T = L.tiles * ((w->k + 127) / 128);
     if (T > INT32_MAX) return TQ_ERR_INVALID_ARG;   // 32-bit iteration space

@@ -1,0 +1,589 @@
+// Decode-block dequant-GEMM for sm_100a: y[m][n] = bf16(x W_hat^T) for
+// m <= 32 tokens (a 16-token denoise block), one launch per call.
+//
+// Route B (as in the stream-K kernel): the activations are rotated instead of
+// inverse-rotating the weight, x' = R x per 32-slice with R = r H diag(s)
+// ("What Config-I means": per-32-block randomized Walsh-Hadamard rotation;
+// R is orthogonal, so x W_hat^T = x' (c[code] d)^T), and the weight side is a
+// table lookup and a multiply per weight pair: the rotated-domain levels
+// fp16(256 c[code]) * d go to tensor memory as the A operand of tcgen05.mma
+// (M = 128 weight rows, N = 16 tokens per block, K = 16), x' (fp16, scaled by
+// a power of two per token) is the B operand in shared memory, fp32
+// accumulation, exact scaling back in the epilogue.
+//
+// One CTA = one 128-row tile of W and one k range of at most 8 iterations of
+// 128 k; the `split` CTAs of a tile form a thread-block cluster and reduce
+// their fp32 partial tiles through distributed shared memory in rank order
+// (deterministic).  What this kernel is built around is the chain of calls a
+// layer stack makes -- each call's input is the previous call's output --
+// where per-call latency, not bandwidth, is the limit:
+//   * a CTA is small enough (about 105 KB of shared memory, 256 tensor-memory
+//     columns, 512 threads at <= 64 registers) that two fit on an SM, and it
+//     lets the next kernel launch as soon as all its CTAs are running, so the
+//     next call's CTAs set up (barriers, level table, tensor memory) and --
+//     for a weight flagged static -- stream their weight tiles into shared
+//     memory while this call still computes;
+//   * only the activation-dependent work waits for the previous kernel: one
+//     warp per token loads its k range of x with coalesced 16-byte loads,
+//     rotates each lane's 32-slice in registers, takes the token's scale from
+//     a warp maximum and writes x' straight into the swizzled B tiles (no
+//     second pass, no shared-memory atomics);
+//   * dequantization, MMA issue and the epilogue run as separate roles.
+//
+// Warps (512 threads):
+//   0      lane 0: TMA producer of the codes tiles (4-stage ring);
+//   1-3    lane 0: MMA issuer of dequant group 0-2;
+//   0-3    epilogue (thread = tile row) once the MMAs are done;
+//   4-15   three dequant groups of four warps (thread = tile row): per
+//          iteration 16 B of codes + 8 scales -> 128 fp16 levels -> tensor
+//          memory, as two 64-k halves signalled separately;
+//   0-15   before their roles: the x rotation (warp = token).
+#include <mutex>
+
+#include "tq4_internal.h"
+
+namespace tq4 {
+namespace {
+
+constexpr int kGroups = 3;                 // dequant groups
+constexpr int kFirstDqWarp = 4;
+constexpr int kThreads = (kFirstDqWarp + 4 * kGroups) * 32;   // 512
+constexpr int kStagesD = 4;                // codes ring
+constexpr int kMaxIters = kFusedMaxIters;  // iterations (128 k) per CTA
+constexpr int kCodesTile = 128 * 64;       // codes of one iteration: 128 rows x 64 B
+constexpr int kLutBytesD = 256 * 32 * 4;   // fp16 level-pair table, one copy per lane
+constexpr int kAColsD = 64;                // tensor-memory columns of one A stage (128 k of fp16)
+constexpr float kLevelScaleD = 256.0f;
+
+struct DecodeShared {
+  uint64_t full[kStagesD];           // codes tile landed (TMA bytes)
+  uint64_t empty[kStagesD];          // the dequant group read the tile (4 warp arrivals)
+  uint64_t afull[kGroups][2];        // half A stage holds fresh levels (4 warp arrivals)
+  uint64_t afree[kGroups][2];        // the MMAs reading a half A stage completed
+  uint64_t xready;                   // every token's x' is in the B tiles (16 warp arrivals)
+  uint64_t dfull;                    // every issuer's MMAs completed (kGroups arrivals)
+  uint64_t idone[kGroups];           // an issuer's own MMAs completed (teardown)
+  float row_scale[kSegRows];         // 2^e of each token
+  uint32_t tmem_base;
+  int abort_flag;
+};
+
+// Dynamic shared memory: codes ring | B tiles [iters][2 halves][16 nb rows x 128 B] |
+// level table | cluster reduction buffer [split][rows per CTA][16 nb] fp32.
+__host__ __device__ constexpr int b_half_bytes(int nb) { return 16 * nb * 128; }
+__host__ __device__ constexpr int off_b() { return kStagesD * kCodesTile; }
+__host__ __device__ constexpr int off_lut(int nb) { return off_b() + kMaxIters * 2 * b_half_bytes(nb); }
+__host__ __device__ constexpr int off_red(int nb) { return off_lut(nb) + kLutBytesD; }
+// (the reduction buffer holds split * ceil(128 / split) <= 135 rows)
+__host__ __device__ constexpr int smem_total(int nb) { return off_red(nb) + 136 * 16 * nb * 4 + 1024; }
+
+struct LevelTableD {
+  uint32_t h[16];   // fp16 bits of 256 * levels[0..15]
+  float max_level;
+};
+
+// Dequantize one half-block (16 codes in q0, q1; dd = {d, d} fp16) through
+// the lane's copy of the level-pair table: out[i] = {level(2i) d, level(2i+1) d}.
+__device__ __forceinline__ void dq_half(uint32_t q0, uint32_t q1, uint32_t dd, uint32_t lut_lane, uint32_t* out) {
+#pragma unroll
+  for (int w = 0; w < 2; ++w) {
+    const uint32_t q = w ? q1 : q0;
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const uint32_t idx = prmt(q, 0u, 0x4440u + static_cast<uint32_t>(b));
+      uint32_t v;
+      asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(lut_lane + idx * 128u));
+      uint32_t r;
+      asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(v), "r"(dd));
+      out[4 * w + b] = r;
+    }
+  }
+}
+
+__device__ __forceinline__ bool wwait(uint64_t* bar, uint32_t parity, volatile int* abortp) {
+  int ok = 0;
+  if ((threadIdx.x & 31) == 0) ok = mbar_wait(bar, parity, abortp) ? 1 : 0;
+  return __shfl_sync(0xFFFFFFFFu, ok, 0) != 0;
+}
+
+__device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
+  const uint32_t addr = smem_u32(bar);
+  const uint64_t t0 = global_timer();
+  while (!mbar_try_wait(addr, parity)) {
+    if (global_timer() - t0 > TQ_WAIT_NS) {
+      raise_status(TQ_DEV_TIMEOUT);
+      return;
+    }
+  }
+}
+
+__device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, float a, float b, float c, float d) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
+}
+
+template <int NB>
+__global__ void __launch_bounds__(kThreads, 2)
+    decode_kernel(const __grid_constant__ CUtensorMap tm_codes, const DecodeArgs a,
+                  const __grid_constant__ LevelTableD lt) {
+  __shared__ DecodeShared sh;
+  extern __shared__ uint8_t dyn_smem[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
+  uint8_t* btiles = smem + off_b();
+  uint8_t* lut = smem + off_lut(NB);
+  uint8_t* red = smem + off_red(NB);
+  constexpr int kHalf = b_half_bytes(NB);
+  constexpr int kAccW = 16 * NB;          // accumulator columns per group
+  constexpr int kACol0 = kGroups * kAccW; // first A-stage column
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = a.split;
+  const int tile = blockIdx.x / split;
+  const int rank = blockIdx.x - tile * split;
+  const int KI = a.k_iters;
+  const int it0 = rank * KI / split, it1 = (rank + 1) * KI / split;
+  const int cnt = it1 - it0;   // >= 1 (split <= KI), <= kMaxIters (host)
+  const int row0 = tile * 128;
+  const bool stat = a.static_w != 0;
+
+  if (warp == 0) {
+    for (int i = lane; i < 2 * kStagesD + 5 * kGroups + 2; i += 32) {
+      if (i < kStagesD) mbar_init(&sh.full[i], 1);
+      else if (i < 2 * kStagesD) mbar_init(&sh.empty[i - kStagesD], 4);
+      else if (i < 2 * kStagesD + 2 * kGroups) mbar_init(&sh.afull[(i - 2 * kStagesD) >> 1][i & 1], 4);
+      else if (i < 2 * kStagesD + 4 * kGroups) mbar_init(&sh.afree[(i - 2 * kStagesD - 2 * kGroups) >> 1][i & 1], 1);
+      else if (i == 2 * kStagesD + 4 * kGroups) mbar_init(&sh.xready, kThreads / 32);
+      else if (i == 2 * kStagesD + 4 * kGroups + 1) mbar_init(&sh.dfull, kGroups);
+      else mbar_init(&sh.idone[i - 2 * kStagesD - 4 * kGroups - 2], 1);
+    }
+    if (lane == 0) {
+      sh.abort_flag = 0;
+      tma_prefetch_desc(&tm_codes);
+    }
+    fence_mbar_init();
+  } else if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, NB == 1 ? 256 : 512);
+    tmem_relinquish();
+  }
+  {
+    // level-pair table: entry b (a code byte) of lane l's copy at byte
+    // 128 b + 4 l holds {256 c[b & 15], 256 c[b >> 4]} * (fp16 pair)
+    uint32_t* lw = reinterpret_cast<uint32_t*>(lut);
+    for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
+      const int b = i >> 5;
+      lw[i] = lt.h[b & 15] | (lt.h[b >> 4] << 16);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // All CTAs of this grid are resident once every one of them is here: the
+  // next kernel may launch now.  Its CTAs take free SM slots (two CTAs of this
+  // kernel fit on an SM) and do their own set-up meanwhile; anything of theirs
+  // that reads this kernel's output waits in griddepcontrol.wait.
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  const uint32_t tmem = sh.tmem_base;
+  volatile int* abortp = &sh.abort_flag;
+
+  // A weight flagged static is not written by any kernel still in flight,
+  // so its tiles may be read before the wait; otherwise the previous kernel
+  // may have written it (a quantize) and everything waits.
+  auto issue_codes = [&](int li) {
+    const int s = li % kStagesD;
+    mbar_arrive_expect_tx(&sh.full[s], kCodesTile);
+    tma_load_3d(smem + s * kCodesTile, &tm_codes, &sh.full[s], (it0 + li) * 64, row0, 0);
+  };
+  const int npre = cnt < kStagesD ? cnt : kStagesD;
+  if (stat && warp == 0 && lane == 0)
+    for (int li = 0; li < npre; ++li) issue_codes(li);
+
+  // dequant threads: the scales of their (up to 3) iterations, 16 B each
+  const int dq_group = (warp >= kFirstDqWarp) ? (warp - kFirstDqWarp) >> 2 : -1;
+  const int trow = (warp & 3) * 32 + lane;   // tile row of this thread (dequant and epilogue)
+  uint32_t sraw[3][4];
+  auto load_scales = [&]() {
+    const int row = row0 + trow;
+    const int kh16 = a.k / 16;
+#pragma unroll
+    for (int u = 0; u < 3; ++u) {
+      const int li = dq_group + kGroups * u;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sraw[u][j] = 0u;
+      if (li < cnt && row < a.n) {
+        const int kit = it0 + li;
+        const uint32_t* sp = reinterpret_cast<const uint32_t*>(a.scales + static_cast<int64_t>(row) * kh16 + kit * 8);
+        if ((kh16 & 7) == 0) {
+          const uint4 v = __ldcg(reinterpret_cast<const uint4*>(sp));
+          sraw[u][0] = v.x;
+          sraw[u][1] = v.y;
+          sraw[u][2] = v.z;
+          sraw[u][3] = v.w;
+        } else {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) sraw[u][j] = (kit * 8 + 2 * j < kh16) ? __ldcg(sp + j) : 0u;
+        }
+      }
+    }
+  };
+  if (stat && dq_group >= 0) load_scales();
+
+  pdl_wait();
+  if (!stat && warp == 0 && lane == 0)
+    for (int li = 0; li < npre; ++li) issue_codes(li);
+  if (!stat && dq_group >= 0) load_scales();
+
+  // ------------------------------------------------------------ x rotation
+  // Warp w rotates tokens w and w + 16 (NB == 2).  Lane l owns the 32-slice
+  // at k = 128 it0 + 32 l of its token (slices past the CTA's range are not
+  // written; slices past k are zero).  Signs flip bf16 sign bits; the
+  // butterfly runs in registers in the fixed stage order; e puts the token's
+  // largest |x'| in [2^13, 2^14) (fp16 cannot overflow); x' 2^-e is rounded
+  // to fp16 and stored in the B tile layout the MMA reads (K-major rows of
+  // 128 B, 8-row groups 1024 B apart, 16-byte chunks XOR-swizzled by row).
+  {
+    const int nsl = cnt * 4;
+    const float r = __uint_as_float(0x3E3504F3u);
+#pragma unroll 1
+    for (int tk = warp; tk < 16 * NB; tk += 16) {
+      float v[32];
+      const int kk = (it0 * 4 + lane) * 32;   // first k of this lane's slice
+      const bool live = lane < nsl && tk < a.m && kk < a.k;
+      if (live) {
+        const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(tk) * a.k + kk);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const uint4 w4 = __ldcg(src + q);   // (L2: x is the previous kernel's output)
+          const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const uint32_t sw = ww[e] ^ a.x_sign[4 * q + e];
+            v[8 * q + 2 * e] = __uint_as_float(sw << 16);
+            v[8 * q + 2 * e + 1] = __uint_as_float(sw & 0xFFFF0000u);
+          }
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
+      }
+#pragma unroll
+      for (int h = 1; h < 32; h <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+          if (!(j & h)) {
+            const float p = v[j], q = v[j + h];
+            v[j] = __fadd_rn(p, q);
+            v[j + h] = __fsub_rn(p, q);
+          }
+        }
+      }
+      float mx = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(v[i]));
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+      int e = 0;
+      const float bound = __fmul_rn(mx, r);   // the token's largest |x'|
+      if (bound > 0.0f && isfinite(bound)) {
+        int ex;
+        frexpf(bound, &ex);   // bound in [2^(ex-1), 2^ex)
+        e = ex - 14;
+        e = e < -100 ? -100 : (e > 100 ? 100 : e);
+      }
+      if (lane == 0) sh.row_scale[tk] = ldexpf(1.0f, e);
+      const float rd = __fmul_rn(r, ldexpf(1.0f, -e));   // exact
+      if (lane < nsl) {
+        const int li = lane >> 2, h = (lane >> 1) & 1, c0 = (lane & 1) * 4;
+        uint8_t* rowp = btiles + (li * 2 + h) * kHalf + (tk >> 3) * 1024 + (tk & 7) * 128;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t hw[4];
+#pragma unroll
+          for (int c2 = 0; c2 < 4; ++c2) {
+            const __half2 hh = __floats2half2_rn(__fmul_rn(v[8 * q + 2 * c2], rd), __fmul_rn(v[8 * q + 2 * c2 + 1], rd));
+            hw[c2] = *reinterpret_cast<const uint32_t*>(&hh);
+          }
+          *reinterpret_cast<uint4*>(rowp + (((c0 + q) ^ (tk & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+        }
+      }
+    }
+    fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.xready);
+  }
+
+  if (dq_group >= 0) {
+    // ------------------------------------------------------------ dequant
+    const int g = dq_group;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t a_stage = tmem + kACol0 + g * kAColsD;
+    const uint32_t lut_lane = smem_u32(lut) + 4u * static_cast<uint32_t>(lane);
+    uint32_t dmax = 0u;
+    int use = 0;
+#pragma unroll 1
+    for (int li = g; li < cnt; li += kGroups, ++use) {
+      const int s = li % kStagesD;
+      if (!wwait(&sh.full[s], (li / kStagesD) & 1, abortp)) break;
+      const uint8_t* cb = smem + s * kCodesTile + trow * 64;
+      uint4 c[4];
+#pragma unroll
+      for (int kb = 0; kb < 4; ++kb) c[kb] = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((trow >> 1) & 3)));
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.empty[s]);   // the producer may refill the stage
+      uint32_t sr[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        sr[j] = (use == 0) ? sraw[0][j] : (use == 1 ? sraw[1][j] : sraw[2][j]);
+        asm("max.f16x2 %0, %1, %2;" : "=r"(dmax) : "r"(dmax), "r"(sr[j]));
+      }
+      bool ok = true;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (use > 0 && !wwait(&sh.afree[g][h], (use - 1) & 1, abortp)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kb2 = 0; kb2 < 2; ++kb2) {
+          const int kb = 2 * h + kb2;
+          uint32_t o[16];
+          dq_half(c[kb].x, c[kb].y, prmt(sr[kb], 0u, 0x1010u), lut_lane, o);
+          dq_half(c[kb].z, c[kb].w, prmt(sr[kb], 0u, 0x3232u), lut_lane, o + 8);
+          tmem_st16(a_stage + lane_base + 16 * kb, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.afull[g][h]);
+      }
+      if (!ok) break;
+    }
+    const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
+    if (fmaxf(dm.x, dm.y) * lt.max_level >= 65520.0f) raise_status(TQ_DEV_SCALE_RANGE);
+  } else {
+    if (warp == 0 && lane == 0) {
+      // ------------------------------------------------------------ producer
+      int armed = -1;   // last iteration whose copy was issued
+      armed = npre - 1;
+#pragma unroll 1
+      for (int li = npre; li < cnt; ++li) {
+        const int s = li % kStagesD;
+        if (!mbar_wait(&sh.empty[s], ((li / kStagesD) - 1) & 1, abortp)) break;
+        issue_codes(li);
+        armed = li;
+      }
+      if (*abortp) {
+        // wind down: every issued copy lands before the CTA exits
+        for (int li = (armed - kStagesD + 1 > 0 ? armed - kStagesD + 1 : 0); li <= armed; ++li)
+          drain(&sh.full[li % kStagesD], (li / kStagesD) & 1);
+      }
+    } else if (warp >= 1 && lane == 0) {
+      // ------------------------------------------------------------ MMA issue
+      const int g = warp - 1;
+      const uint32_t acc = tmem + g * kAccW;
+      const uint32_t a_stage = tmem + kACol0 + g * kAColsD;
+      const uint32_t idesc = idesc_f16(128, 16 * NB);
+      bool ok = mbar_wait(&sh.xready, 0, abortp);
+      int use = 0;
+      for (int li = g; ok && li < cnt; li += kGroups, ++use) {
+        for (int h = 0; h < 2; ++h) {
+          if (!mbar_wait(&sh.afull[g][h], use & 1, abortp)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint64_t bdesc = sdesc_k128(smem_u32(btiles + (li * 2 + h) * kHalf));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
+                   (use == 0 && h == 0 && kk == 0) ? 0u : 1u);
+          mma_commit(&sh.afree[g][h]);
+        }
+      }
+      if (use > 0) mma_commit(&sh.dfull);
+      else mbar_arrive(&sh.dfull);
+      // its MMAs complete before the CTA can release tensor memory
+      mma_commit(&sh.idone[g]);
+      drain(&sh.idone[g], 0);
+    }
+    __syncwarp();
+    // ------------------------------------------------------------ epilogue
+    // thread = tile row trow; the groups' accumulators summed in group order,
+    // scaled back by 2^e / 256 per token (exact)
+    // (xready also orders the token scales written by the rotation warps)
+    int ok = 0;
+    if (lane == 0) ok = (mbar_wait(&sh.xready, 0, abortp) && mbar_wait(&sh.dfull, 0, abortp)) ? 1 : 0;
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    tc_fence_after();
+    const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+    const int ngroups = cnt < kGroups ? cnt : kGroups;
+    if (ok) {
+#pragma unroll
+      for (int c = 0; c < NB; ++c) {
+        float v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = 0.0f;
+        for (int g = 0; g < ngroups; ++g) {
+          uint32_t rr[16];
+          tmem_ld16(tmem + lane_base + g * kAccW + 16 * c, rr);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __uint_as_float(rr[j]));
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], __fmul_rn(sh.row_scale[16 * c + j], 1.0f / kLevelScaleD));
+        if (split > 1) {
+          // row trow goes to the CTA that owns it: [source rank][row - owner's first row][token]
+          const int q = (trow * split) >> 7;
+          const int rpc = (128 + split - 1) / split;
+          const int tl = trow - (q * 128 + split - 1) / split;
+          const uint32_t dst = smem_u32(red) + static_cast<uint32_t>(((rank * rpc + tl) * 16 * NB + 16 * c) * 4);
+#pragma unroll
+          for (int j = 0; j < 16; j += 4)
+            st_dsmem_v4(dst + 4u * j, static_cast<uint32_t>(q), v[j], v[j + 1], v[j + 2], v[j + 3]);
+        } else {
+          const int row = row0 + trow;
+          if (row < a.n) {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (16 * c + j < a.m)
+                a.y[static_cast<int64_t>(16 * c + j) * a.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(v[j]));
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (split > 1) {
+    // Every thread of every CTA of the cluster reaches this barrier (each role
+    // runs to its end, on a timeout too), so it cannot hang; it orders the
+    // pushes above before the owners read them, and nothing touches another
+    // CTA's shared memory after it.
+    cluster_sync_all();
+    if (!sh.abort_flag) {
+      const int rpc = (128 + split - 1) / split;
+      const int r0 = (rank * 128 + split - 1) / split, r1 = ((rank + 1) * 128 + split - 1) / split;
+      const int nrow = r1 - r0;
+      const float* rb = reinterpret_cast<const float*>(red);
+      for (int idx = threadIdx.x; idx < nrow * a.m; idx += kThreads) {
+        const int j = idx / nrow, tl = idx - j * nrow;
+        const int row = row0 + r0 + tl;
+        if (row >= a.n) continue;
+        float acc = 0.0f;
+        for (int q = 0; q < split; ++q) acc = __fadd_rn(acc, rb[(q * rpc + tl) * 16 * NB + j]);
+        a.y[static_cast<int64_t>(j) * a.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+      }
+    }
+  }
+  if (warp == 1) tmem_dealloc(tmem, NB == 1 ? 256 : 512);
+}
+
+template <int NB>
+cudaError_t launch_decode_nb(const void* tm_codes, const DecodeArgs& a, cudaStream_t st) {
+  static bool attr_set = false;
+  const int smem = smem_total(NB);
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    if (e == cudaSuccess)
+      e = cudaFuncSetAttribute(decode_kernel<NB>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  static const LevelTableD lt = [] {
+    LevelTableD t;
+    const CodebookF32& cb = codebook();
+    for (int i = 0; i < 16; ++i)
+      t.h[i] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(cb.levels[i] * kLevelScaleD)));
+    t.max_level = __half2float(__float2half_rn(cb.levels[15] * kLevelScaleD));
+    return t;
+  }();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(a.row_tiles * a.split));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem);
+  cfg.stream = st;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (a.split > 1) {
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = static_cast<unsigned>(a.split);
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cfg.numAttrs = 2;
+  }
+  const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NB>, m0, a, lt);
+  if (e != cudaSuccess) return e;
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+template <int NB>
+int decode_max_clusters_nb(int s) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(static_cast<unsigned>(s));
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_total(NB));
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = static_cast<unsigned>(s);
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaFuncSetAttribute(decode_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_total(NB)) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<NB>, &cfg) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+}  // namespace
+
+size_t decode_smem_bytes(int nb) { return static_cast<size_t>(nb == 1 ? smem_total(1) : smem_total(2)); }
+
+cudaError_t launch_decode(const void* tm_codes, const DecodeArgs& a, cudaStream_t st) {
+  return a.nb == 1 ? launch_decode_nb<1>(tm_codes, a, st) : launch_decode_nb<2>(tm_codes, a, st);
+}
+
+int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb) {
+  // the largest s in [1, 8] with s <= k_iters, at most kMaxIters iterations
+  // per CTA, one CTA per SM (tiles * s <= sms) and all clusters resident at
+  // once; 0 if none fits.  Cluster capacities are queried once per device.
+  static std::mutex mu;
+  static int cap[64][2][9];   // resident clusters + 1 (0 = not queried yet)
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
+    cudaGetLastError();
+    return 0;
+  }
+  for (int s = 8; s >= 1; --s) {
+    if (s > k_iters || (k_iters + s - 1) / s > kMaxIters || tiles * s > sms) continue;
+    if (s == 1) return 1;
+    int c;
+    {
+      std::lock_guard<std::mutex> g(mu);
+      int& slot = cap[dev][nb == 1 ? 0 : 1][s];
+      if (slot == 0) slot = (nb == 1 ? decode_max_clusters_nb<1>(s) : decode_max_clusters_nb<2>(s)) + 1;
+      c = slot - 1;
+    }
+    if (tiles <= c) return s;
+  }
+  return 0;
+}
+
+}  // namespace tq4

@@ -126,6 +126,25 @@ int choose_cluster_split(int64_t tiles, int64_t k_iters, int sms);
 cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const void* tm_x3, const StreamKArgs& a, int grid,
                            cudaStream_t st);
 
+// ---------------------------------------------------------------- decode
+// The decode-block kernel: m <= 32 tokens, one CTA per (128-row tile, k
+// range of at most kFusedMaxIters iterations), `split` CTAs per tile in a
+// cluster.  tm_codes: the codes plane (map_codes).
+struct DecodeArgs {
+  int32_t n, k, m, nb;          // rows, columns, tokens, 16-token blocks (1 or 2)
+  int32_t row_tiles, k_iters;   // ceil(n / 128), ceil(k / 128)
+  int32_t split;                // CTAs per row tile (>= 1, <= k_iters)
+  int32_t static_w;             // the weight may be read before the dependency wait
+  const uint16_t* x;            // bf16 [m][k]
+  const uint16_t* scales;       // [n][k/16] fp16 bits
+  uint16_t* y;                  // bf16 [m][n]
+  uint32_t x_sign[16];          // sign mask as XOR words on bf16 pairs
+};
+cudaError_t launch_decode(const void* tm_codes, const DecodeArgs& a, cudaStream_t st);
+// The split for a decode launch of `tiles` row tiles (0: the kernel does not fit).
+int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb);
+size_t decode_smem_bytes(int nb);
+
 // ---------------------------------------------------------------- GEMM
 // y[m][n] = bf16( x[m][k] * w[n][k]^T ), bf16 operands via TMA tensor maps.
 cudaError_t launch_gemm_bf16(const void* tm_x, const void* tm_w, uint16_t* y, int32_t m, int32_t n, int32_t k,

@@ -69,7 +69,7 @@ using namespace tq4;
 TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y,
                                        tq4_stream_t stream) {
   if (!w) return TQ_ERR_INVALID_ARG;
-  if (w->n <= 0 || w->k <= 0 || (w->k % 32) != 0 || w->num_experts != 1 || w->reserved != 0 || m < 0)
+  if (w->n <= 0 || w->k <= 0 || (w->k % 32) != 0 || w->num_experts != 1 || (w->flags & ~TQ_WEIGHT_STATIC) != 0 || m < 0)
     return TQ_ERR_INVALID_ARG;
   if (!w->codes || !w->scales) return TQ_ERR_INVALID_ARG;
   if (m > kStaticMaxM || w->k > kStaticMaxK || w->n > kStaticMaxN) return TQ_ERR_SCRATCH_LIMIT;

@@ -76,12 +76,25 @@ enum {
 /* Input dtypes of tq4_1s_quantize. */
 enum { TQ_DTYPE_F32 = 0, TQ_DTYPE_BF16 = 1 };
 
+/* Bits of tq4_1s_weight.flags.
+ *   TQ_WEIGHT_STATIC: the caller guarantees that no kernel that may still be
+ *   running when a call reading this weight is enqueued writes its codes or
+ *   scales -- every write to them (tq4_1s_quantize included) has completed,
+ *   e.g. the stream or device was synchronized after it, as when weights are
+ *   quantized or loaded once at start-up.  The decode-block kernel of
+ *   tq4_1s_linear may then start streaming the weight before the previous
+ *   kernel on the stream has finished (its own input still waits).  Without
+ *   the bit every read of the weight waits for the previous kernel.  Setting
+ *   it for a weight that an unfinished kernel writes gives undefined results.
+ * Other bits must be 0. */
+enum { TQ_WEIGHT_STATIC = 1 };
+
 /* A packed TQ4_1S tensor or stack of num_experts tensors of shape [n][k]. */
 typedef struct {
   int64_t n;            /* rows (output features), > 0                          */
   int64_t k;            /* columns (input features), > 0, multiple of 32        */
   int32_t num_experts;  /* 1 for a dense layer                                  */
-  int32_t reserved;     /* must be 0                                            */
+  int32_t flags;        /* TQ_WEIGHT_* bits; 0 by default                      */
   uint64_t seed;        /* RHT seed; the sign mask is derived from it           */
   uint8_t* codes;       /* device, [num_experts][n][k/2], 16-byte aligned       */
   uint16_t* scales;     /* device, [num_experts][n][k/16], 16-byte aligned      */

@@ -4,9 +4,9 @@ Plugin hosts and serving runtimes that fix their device memory at start-up
 cannot hand tq4_1s_linear a workspace; tq4_1s_linear_static keeps its scratch
 in a fixed array inside the library instead.  This test calls it through the
 C ABI twice in a row (the second call runs on the scratch the first one left
-behind) and checks each result against tq4_1s_linear, which uses a caller
-workspace, with the same tolerances as the parity tests.  It lives in a file
-of its own that pytest collects last.
+behind) and checks each result against the CPU oracle and against
+tq4_1s_linear, which uses a caller workspace, with the same tolerances as the
+parity tests.  It lives in a file of its own that pytest collects last.
 """
 import ctypes
 
@@ -14,6 +14,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle
 import synth
 from tests._parity import assert_close
 
@@ -36,17 +37,21 @@ def test_static_scratch_linear_matches_workspace_linear():
     fn = lib.tq4_1s_linear_static
     fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(tq._Weight), ctypes.c_void_p, ctypes.c_void_p]
     fn.restype = ctypes.c_int
-    W = torch.from_numpy(synth.student_t_f32((4096, 4096), 2, 5.0, 0.02)).to(dev)
-    p = tq.tq4_1s_quantize(W, seed=2)
+    Wh = synth.student_t_f32((4096, 4096), 2, 5.0, 0.02)
+    p = tq.tq4_1s_quantize(torch.from_numpy(Wh).to(dev), seed=2)
+    codes, scales, _ = oracle.quantize(Wh, 2)
     wst = p.c_struct()
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
     for call, (m, seed) in enumerate([(16, 3), (13, 5)]):
-        x = _to_dev(synth.activations_bf16(m, 4096, seed), dev)
+        xh = synth.activations_bf16(m, 4096, seed)
+        x = _to_dev(xh, dev)
         ref = tq.tq4_1s_linear(x, p)
         y = torch.empty((m, 4096), dtype=torch.bfloat16, device=dev)
         rc = fn(ctypes.c_void_p(x.data_ptr()), m, ctypes.byref(wst), ctypes.c_void_p(y.data_ptr()), stream)
         assert rc == 0, tq.tq4_1s_error_string(rc)
         torch.cuda.synchronize()
+        y_ref, _ = oracle.linear(xh, codes, scales, 2)
+        assert_close(_bits(y), y_ref, f"static call {call} vs oracle")
         ref_f = _bits(ref).astype(np.uint32) << 16
         assert_close(_bits(y), ref_f.view(np.float32).astype(np.float64), f"static call {call}")
     assert tq.tq4_1s_get_status() == 0
@@ -68,16 +73,20 @@ def test_static_scratch_other_modes(m, n, k, seed):
     fn = lib.tq4_1s_linear_static
     fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(tq._Weight), ctypes.c_void_p, ctypes.c_void_p]
     fn.restype = ctypes.c_int
-    W = torch.from_numpy(synth.normal_f32((n, k), seed, 0.02)).to(dev)
-    p = tq.tq4_1s_quantize(W, seed=seed)
+    Wh = synth.normal_f32((n, k), seed, 0.02)
+    p = tq.tq4_1s_quantize(torch.from_numpy(Wh).to(dev), seed=seed)
     wst = p.c_struct()
     stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
-    x = _to_dev(synth.activations_bf16(m, k, seed + 1), dev)
+    xh = synth.activations_bf16(m, k, seed + 1)
+    x = _to_dev(xh, dev)
     ref = tq.tq4_1s_linear(x, p)
     y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
     rc = fn(ctypes.c_void_p(x.data_ptr()), m, ctypes.byref(wst), ctypes.c_void_p(y.data_ptr()), stream)
     assert rc == 0, tq.tq4_1s_error_string(rc)
     torch.cuda.synchronize()
+    codes, scales, _ = oracle.quantize(Wh, seed)
+    y_ref, _ = oracle.linear(xh, codes, scales, seed)
+    assert_close(_bits(y), y_ref, f"static m={m} n={n} k={k} vs oracle")
     ref_f = _bits(ref).astype(np.uint32) << 16
     assert_close(_bits(y), ref_f.view(np.float32).astype(np.float64), f"static m={m} n={n} k={k}")
     assert tq.tq4_1s_get_status() == 0
