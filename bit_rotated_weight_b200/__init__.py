@@ -25,7 +25,7 @@ __all__ = [
     "tq4_1s_version", "tq4_1s_error_string", "tq4_1s_packed_bytes", "tq4_1s_sign_mask", "tq4_1s_codebook",
     "tq4_1s_quantize", "tq4_1s_quantize_batched", "tq4_1s_dequantize", "tq4_1s_linear_workspace", "tq4_1s_linear",
     "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_logits", "tq4_1s_router_topk", "tq4_1s_moe_route", "tq4_1s_get_status", "tq4_1s_launch_count",
-    "tq4_1s_linear_static",
+    "tq4_1s_linear_static", "tq4_1s_debug_hook",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -35,6 +35,7 @@ TQ_OK = 0
 TQ_DTYPE_F32, TQ_DTYPE_BF16 = 0, 1
 TQ_DEV_TIMEOUT, TQ_DEV_BAD_ROUTING, TQ_DEV_NONFINITE, TQ_DEV_SCALE_RANGE = 1, 2, 4, 8
 TQ_WEIGHT_STATIC = 1
+TQ_HOOK_FAIL_NEXT_CALLS, TQ_HOOK_WAIT_NS, TQ_HOOK_WITHHOLD_ARRIVAL = 1, 2, 3
 
 
 class TQ4Error(RuntimeError):
@@ -84,6 +85,7 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                 "tq4_1s_router_topk": ([P, I64, I32, I32, P, P, P], ctypes.c_int),
                 "tq4_1s_get_status": ([P, ctypes.POINTER(I32)], ctypes.c_int),
                 "tq4_1s_launch_count": ([], ctypes.c_uint64),
+                "tq4_1s_debug_hook": ([ctypes.c_int, I64], ctypes.c_int),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -357,3 +359,8 @@ def tq4_1s_linear_static(x: torch.Tensor, w: Packed, out: torch.Tensor | None = 
     _check(load_library().tq4_1s_linear_static(_ptr(x), x.shape[0], ctypes.byref(wst), _ptr(out),
                                                _stream(x.device)), "linear_static")
     return out
+
+
+def tq4_1s_debug_hook(what: int, value: int) -> None:
+    """Test hooks of the library (fault injection, short device waits); see include/tq4_1s.h."""
+    _check(load_library().tq4_1s_debug_hook(what, value), "debug_hook")

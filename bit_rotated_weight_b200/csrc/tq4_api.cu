@@ -65,6 +65,16 @@ const CodebookF32& codebook() {
 static std::atomic<uint64_t> g_launches{0};
 void note_launches(int n) { g_launches.fetch_add(static_cast<uint64_t>(n), std::memory_order_relaxed); }
 
+static std::atomic<int64_t> g_fail_next{0};
+static std::atomic<int> g_withhold{0};
+bool take_injected_failure() {
+  int64_t v = g_fail_next.load(std::memory_order_relaxed);
+  while (v > 0)
+    if (g_fail_next.compare_exchange_weak(v, v - 1, std::memory_order_relaxed)) return true;
+  return false;
+}
+bool withhold_arrival_hook() { return g_withhold.load(std::memory_order_relaxed) != 0; }
+
 // SplitMix64 (Steele, Lea, Flood, OOPSLA 2014): first output from `state`.
 static uint32_t sign_mask_of(uint64_t state) {
   uint64_t z = state + 0x9E3779B97F4A7C15ull;
@@ -373,6 +383,7 @@ TQ_API int tq4_1s_quantize(const void* W, int dtype, const tq4_1s_weight* out, t
   if (!W || (dtype != TQ_DTYPE_F32 && dtype != TQ_DTYPE_BF16)) return TQ_ERR_INVALID_ARG;
   if (!aligned16(W)) return TQ_ERR_ALIGNMENT;
   if ((rc = check_device(nullptr))) return rc;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
   const int64_t rows = out->n * out->num_experts;
   return cuda_rc(launch_quantize(W, dtype, out->codes, out->scales, rows, out->k, sign_mask_of(out->seed),
                                  codebook(), reinterpret_cast<cudaStream_t>(stream)));
@@ -391,6 +402,7 @@ TQ_API int tq4_1s_quantize_batched(const void* const* W, int dtype, const tq4_1s
   }
   int rc = check_device(nullptr);
   if (rc) return rc;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
   std::vector<QuantItem> items(static_cast<size_t>(count));
   for (int32_t i = 0; i < count; ++i)
     items[i] = QuantItem{W[i], outs[i].codes, outs[i].scales, outs[i].n * outs[i].num_experts, outs[i].k,
@@ -404,6 +416,7 @@ TQ_API int tq4_1s_dequantize(const tq4_1s_weight* w, float* W_out, tq4_stream_t 
   if (!W_out) return TQ_ERR_INVALID_ARG;
   if (!aligned16(W_out)) return TQ_ERR_ALIGNMENT;
   if ((rc = check_device(nullptr))) return rc;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
   return cuda_rc(launch_dequantize_f32(w->codes, w->scales, W_out, w->n * w->num_experts, w->k,
                                        sign_mask_of(w->seed), codebook(), reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -436,6 +449,7 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
   const size_t need = small ? L.total : align256(static_cast<size_t>(w->n) * static_cast<size_t>(w->k) * 2);
   if (!ws || ws_bytes < need) return TQ_ERR_WORKSPACE;
   if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   const uint32_t mask = sign_mask_of(w->seed);
@@ -458,6 +472,7 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
       d.k_iters = static_cast<int32_t>(KI);
       d.split = split;
       d.static_w = (w->flags & TQ_WEIGHT_STATIC) ? 1 : 0;
+      d.test_withhold = withhold_arrival_hook() ? 1 : 0;
       d.x = x;
       d.scales = w->scales;
       d.y = y;
@@ -562,6 +577,7 @@ static int moe_impl(const uint16_t* x, int64_t m, const int32_t* topk_ids, const
     return TQ_ERR_INVALID_ARG;   // 32-bit iteration space
   if (!ws || ws_bytes < L.total) return TQ_ERR_WORKSPACE;
   if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
   uint8_t* base = static_cast<uint8_t*>(ws);
   const int64_t E = up->num_experts, H = up->k, I = up->n;
@@ -663,6 +679,7 @@ TQ_API int tq4_1s_router_topk(const float* logits, int64_t m, int32_t num_expert
   if (!logits || !ids || !weights) return TQ_ERR_INVALID_ARG;
   int rc = check_device(nullptr);
   if (rc) return rc;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
   return cuda_rc(launch_router(logits, m, num_experts, topk, ids, weights, reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -675,6 +692,28 @@ TQ_API int tq4_1s_moe_route(const int32_t* topk_ids, int64_t m, int32_t topk, in
   if (rc) return rc;
   return cuda_rc(launch_moe_route(topk_ids, m * topk, num_experts, offsets, pairs, nullptr, nullptr, kSegRows,
                                   nullptr, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+TQ_API int tq4_1s_debug_hook(int what, int64_t value) {
+  switch (what) {
+    case TQ_HOOK_FAIL_NEXT_CALLS:
+      if (value < 0) return TQ_ERR_INVALID_ARG;
+      g_fail_next.store(value, std::memory_order_relaxed);
+      return TQ_OK;
+    case TQ_HOOK_WAIT_NS: {
+      if (value < 0) return TQ_ERR_INVALID_ARG;
+      const int rc = check_device(nullptr);
+      if (rc) return rc;
+      const unsigned long long ns = value == 0 ? TQ_WAIT_NS_DEFAULT : static_cast<unsigned long long>(value);
+      return cudaMemcpyToSymbol(g_wait_ns, &ns, sizeof(ns)) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+    }
+    case TQ_HOOK_WITHHOLD_ARRIVAL:
+      if (value != 0 && value != 1) return TQ_ERR_INVALID_ARG;
+      g_withhold.store(static_cast<int>(value), std::memory_order_relaxed);
+      return TQ_OK;
+    default:
+      return TQ_ERR_INVALID_ARG;
+  }
 }
 
 TQ_API uint64_t tq4_1s_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }

@@ -2,7 +2,7 @@
 // for mbarriers, TMA tensor copies and the tcgen05 tensor-core / tensor-memory
 // instructions, bounded waits, and the device status word.
 //
-// Every wait in these kernels is bounded: after TQ_WAIT_NS of global time the
+// Every wait in these kernels is bounded: after g_wait_ns of global time the
 // waiting warp records TQ_DEV_TIMEOUT in the status word, raises the CTA's
 // abort flag and returns false, so that the kernel winds down instead of
 // hanging the GPU.
@@ -17,10 +17,14 @@
 
 namespace tq4 {
 
-constexpr unsigned long long TQ_WAIT_NS = 2000000000ull;   // 2 s per wait
+constexpr unsigned long long TQ_WAIT_NS_DEFAULT = 2000000000ull;   // 2 s per wait
 
 // Device status word, read and cleared by tq4_1s_get_status().
 extern __device__ int g_status;
+// The limit of every bounded wait, in ns of global time (TQ_WAIT_NS_DEFAULT
+// unless a test shortened it through tq4_1s_debug_hook).
+extern __device__ unsigned long long g_wait_ns;
+#define TQ_WAIT_NS (*const_cast<volatile unsigned long long*>(&g_wait_ns))
 
 __device__ __forceinline__ void raise_status(int flag) { atomicOr(&g_status, flag); }
 

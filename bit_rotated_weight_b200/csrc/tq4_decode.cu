@@ -63,6 +63,8 @@ struct DecodeShared {
   uint64_t xready;                   // every token's x' is in the B tiles (16 warp arrivals)
   uint64_t dfull;                    // every issuer's MMAs completed (kGroups arrivals)
   uint64_t idone[kGroups];           // an issuer's own MMAs completed (teardown)
+  uint64_t eready;                   // every dequant thread wrote its row exponent (12 warp arrivals)
+  int8_t rexp[kGroups][128];         // row exponent of each group's levels (see the dequant)
   float row_scale[kSegRows];         // 2^e of each token
   uint32_t tmem_base;
   int abort_flag;
@@ -149,14 +151,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool stat = a.static_w != 0;
 
   if (warp == 0) {
-    for (int i = lane; i < 2 * kStagesD + 5 * kGroups + 2; i += 32) {
+    for (int i = lane; i < 2 * kStagesD + 5 * kGroups + 3; i += 32) {
       if (i < kStagesD) mbar_init(&sh.full[i], 1);
       else if (i < 2 * kStagesD) mbar_init(&sh.empty[i - kStagesD], 4);
       else if (i < 2 * kStagesD + 2 * kGroups) mbar_init(&sh.afull[(i - 2 * kStagesD) >> 1][i & 1], 4);
       else if (i < 2 * kStagesD + 4 * kGroups) mbar_init(&sh.afree[(i - 2 * kStagesD - 2 * kGroups) >> 1][i & 1], 1);
       else if (i == 2 * kStagesD + 4 * kGroups) mbar_init(&sh.xready, kThreads / 32);
       else if (i == 2 * kStagesD + 4 * kGroups + 1) mbar_init(&sh.dfull, kGroups);
-      else mbar_init(&sh.idone[i - 2 * kStagesD - 4 * kGroups - 2], 1);
+      else if (i < 2 * kStagesD + 5 * kGroups + 2) mbar_init(&sh.idone[i - 2 * kStagesD - 4 * kGroups - 2], 1);
+      else mbar_init(&sh.eready, 4 * kGroups);
     }
     if (lane == 0) {
       sh.abort_flag = 0;
@@ -310,7 +313,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sh.xready);
+    if (lane == 0 && !(a.test_withhold && warp == 7)) mbar_arrive(&sh.xready);
   }
 
   if (dq_group >= 0) {
@@ -319,7 +322,33 @@ __global__ void __launch_bounds__(kThreads, 2)
     const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const uint32_t a_stage = tmem + kACol0 + g * kAColsD;
     const uint32_t lut_lane = smem_u32(lut) + 4u * static_cast<uint32_t>(lane);
-    uint32_t dmax = 0u;
+    // Row exponent of this group's levels: the scales of the group's
+    // iterations are multiplied by 2^-e (exact) so that the largest lies in
+    // [32, 64) -- levels fp16(256 c) * d 2^-e then stay normal and finite for
+    // every finite fp16 scale -- and the epilogue multiplies the group's
+    // accumulator by 2^e (exact).
+    uint32_t ff;
+    {
+      uint32_t dmax = 0u;
+#pragma unroll
+      for (int u = 0; u < 3; ++u)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) asm("max.f16x2 %0, %1, %2;" : "=r"(dmax) : "r"(dmax), "r"(sraw[u][j]));
+      const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
+      const float mx = fmaxf(dm.x, dm.y);
+      int e = 0;
+      if (mx > 0.0f && isfinite(mx)) {
+        int ex;
+        frexpf(mx, &ex);   // mx in [2^(ex-1), 2^ex)
+        e = ex - 6;
+        e = e < -15 ? -15 : (e > 14 ? 14 : e);
+      }
+      sh.rexp[g][trow] = static_cast<int8_t>(e);
+      const __half2 f2 = __float2half2_rn(ldexpf(1.0f, -e));   // a power of two, normal in fp16
+      ff = *reinterpret_cast<const uint32_t*>(&f2);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.eready);
+    }
     int use = 0;
 #pragma unroll 1
     for (int li = g; li < cnt; li += kGroups, ++use) {
@@ -335,7 +364,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         sr[j] = (use == 0) ? sraw[0][j] : (use == 1 ? sraw[1][j] : sraw[2][j]);
-        asm("max.f16x2 %0, %1, %2;" : "=r"(dmax) : "r"(dmax), "r"(sr[j]));
+        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(sr[j]) : "r"(sr[j]), "r"(ff));
       }
       bool ok = true;
 #pragma unroll
@@ -360,8 +389,6 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
       if (!ok) break;
     }
-    const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
-    if (fmaxf(dm.x, dm.y) * lt.max_level >= 65520.0f) raise_status(TQ_DEV_SCALE_RANGE);
   } else {
     if (warp == 0 && lane == 0) {
       // ------------------------------------------------------------ producer
@@ -414,7 +441,10 @@ __global__ void __launch_bounds__(kThreads, 2)
     // scaled back by 2^e / 256 per token (exact)
     // (xready also orders the token scales written by the rotation warps)
     int ok = 0;
-    if (lane == 0) ok = (mbar_wait(&sh.xready, 0, abortp) && mbar_wait(&sh.dfull, 0, abortp)) ? 1 : 0;
+    if (lane == 0)
+      ok = (mbar_wait(&sh.xready, 0, abortp) && mbar_wait(&sh.eready, 0, abortp) && mbar_wait(&sh.dfull, 0, abortp))
+               ? 1
+               : 0;
     ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
     tc_fence_after();
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
@@ -429,8 +459,9 @@ __global__ void __launch_bounds__(kThreads, 2)
           uint32_t rr[16];
           tmem_ld16(tmem + lane_base + g * kAccW + 16 * c, rr);
           tmem_wait_ld();
+          const float rs = ldexpf(1.0f, sh.rexp[g][trow]);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __uint_as_float(rr[j]));
+          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(rr[j]), rs));
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], __fmul_rn(sh.row_scale[16 * c + j], 1.0f / kLevelScaleD));

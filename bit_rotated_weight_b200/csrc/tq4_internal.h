@@ -16,6 +16,12 @@ struct CodebookF32 {
 // Count of kernel launches issued by the library (tq4_1s_launch_count).
 void note_launches(int n);
 
+// Test hooks (tq4_1s_debug_hook): a pending injected failure makes the next
+// launching call return TQ_ERR_CUDA before it launches anything; the
+// withhold flag is copied into decode launches.
+bool take_injected_failure();
+bool withhold_arrival_hook();
+
 // Host-side codebook computation (Lloyd iteration), run once per process.
 const CodebookF32& codebook();
 
@@ -135,6 +141,7 @@ struct DecodeArgs {
   int32_t row_tiles, k_iters;   // ceil(n / 128), ceil(k / 128)
   int32_t split;                // CTAs per row tile (>= 1, <= k_iters)
   int32_t static_w;             // the weight may be read before the dependency wait
+  int32_t test_withhold;        // test hook: rotation warp 7 never reports (its bounded waiters run out)
   const uint16_t* x;            // bf16 [m][k]
   const uint16_t* scales;       // [n][k/16] fp16 bits
   uint16_t* y;                  // bf16 [m][n]

@@ -14,6 +14,7 @@
 namespace tq4 {
 
 __device__ int g_status = 0;
+__device__ unsigned long long g_wait_ns = TQ_WAIT_NS_DEFAULT;
 
 // r = fp32(1/sqrt(32))
 __device__ __forceinline__ float rsqrt32() { return __uint_as_float(0x3E3504F3u); }

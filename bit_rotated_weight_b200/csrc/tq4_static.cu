@@ -89,6 +89,7 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   void* scratch = nullptr;
   int rc = scratch_address(&scratch);
   if (rc) return rc;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
 
   uint8_t* base = static_cast<uint8_t*>(scratch);
   uint16_t* xr = reinterpret_cast<uint16_t*>(base);

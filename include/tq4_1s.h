@@ -262,6 +262,23 @@ int tq4_1s_moe_route(const int32_t* topk_ids, int64_t m, int32_t topk, int32_t n
  * counts once, at capture. */
 uint64_t tq4_1s_launch_count(void);
 
+/* Test hooks -- fault injection for the library's failure-handling tests;
+ * not for production use.  (The model card has no counterpart.)
+ *   TQ_HOOK_FAIL_NEXT_CALLS, value n >= 0: the next n calls that would
+ *     launch kernels fail with TQ_ERR_CUDA after validating their arguments
+ *     and before launching anything (a host-side stand-in for a failed
+ *     launch); 0 cancels.  Host only.
+ *   TQ_HOOK_WAIT_NS, value ns >= 0: the limit of every bounded device wait
+ *     on the current device (0 restores the default of 2 s).
+ *   TQ_HOOK_WITHHOLD_ARRIVAL, value 0 or 1: while 1, the decode-block kernel
+ *     of tq4_1s_linear runs with one rotation warp that never reports its
+ *     activations ready, so the waits on them run out: the kernel sets
+ *     TQ_DEV_TIMEOUT, lets its copies and MMAs finish, frees its tensor
+ *     memory and returns (the output is then unspecified).
+ * Returns TQ_OK, or TQ_ERR_INVALID_ARG for an unknown hook or value. */
+enum { TQ_HOOK_FAIL_NEXT_CALLS = 1, TQ_HOOK_WAIT_NS = 2, TQ_HOOK_WITHHOLD_ARRIVAL = 3 };
+int tq4_1s_debug_hook(int what, int64_t value);
+
 /* Synchronize `stream`, then read and clear the current device's status
  * word (a mask of TQ_DEV_* bits) into *status (host). */
 int tq4_1s_get_status(tq4_stream_t stream, int32_t* status);

@@ -115,6 +115,23 @@ def test_static_entry_validation_and_scratch_limits():
     assert tq.tq4_1s_error_string(9).startswith("shape exceeds the fixed scratch")
 
 
+def test_debug_hooks_validation():
+    lib = tq.load_library()
+    assert lib.tq4_1s_debug_hook(99, 0) == 1                       # unknown hook
+    assert lib.tq4_1s_debug_hook(tq.TQ_HOOK_FAIL_NEXT_CALLS, -1) == 1
+    assert lib.tq4_1s_debug_hook(tq.TQ_HOOK_FAIL_NEXT_CALLS, 0) == 0
+    assert lib.tq4_1s_debug_hook(tq.TQ_HOOK_WITHHOLD_ARRIVAL, 2) == 1
+    assert lib.tq4_1s_debug_hook(tq.TQ_HOOK_WITHHOLD_ARRIVAL, 0) == 0
+    assert lib.tq4_1s_debug_hook(tq.TQ_HOOK_WAIT_NS, -5) == 1
+    if not torch.cuda.is_available():
+        assert lib.tq4_1s_debug_hook(tq.TQ_HOOK_WAIT_NS, 1000) == 3     # needs a device
+    # an armed failure is not consumed by calls that fail validation first
+    assert lib.tq4_1s_debug_hook(tq.TQ_HOOK_FAIL_NEXT_CALLS, 1) == 0
+    null = ctypes.c_void_p(0)
+    assert lib.tq4_1s_linear(null, 16, ctypes.byref(_weight()), null, null, 0, null) == 1
+    assert lib.tq4_1s_debug_hook(tq.TQ_HOOK_FAIL_NEXT_CALLS, 0) == 0
+
+
 def test_router_and_moe_logits_validation():
     lib = tq.load_library()
     null = ctypes.c_void_p(0)

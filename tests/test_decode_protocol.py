@@ -5,7 +5,7 @@ The kernel's roles synchronise only through mbarriers (plus one CTA barrier
 and one cluster barrier that every thread reaches): the TMA producer and the
 codes ring (full/empty), four-warp dequant groups filling half A stages
 (afull) that their MMA issuer frees (afree, by tcgen05.commit), the rotation
-warps' xready, the issuers' dfull and idone.  This model runs the roles as
+warps' xready, the dequant warps' eready, the issuers' dfull and idone.  This model runs the roles as
 actors in random interleavings, with TMA landings and MMA completions as
 asynchronous events, for every k-range length a CTA can have (1..8
 iterations), and checks that:
@@ -45,6 +45,7 @@ def test_source_constants_and_counts():
     assert "mbar_init(&sh.afull[(i - 2 * kStagesD) >> 1][i & 1], 4)" in SRC
     assert "mbar_init(&sh.xready, kThreads / 32)" in SRC             # one arrival per warp
     assert "mbar_init(&sh.dfull, kGroups)" in SRC
+    assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
 
 
 class Barrier:
@@ -83,6 +84,7 @@ def run(cnt, seed, withhold_xready=False):
     xready = bar("xready", WARPS)
     dfull = bar("dfull", GROUPS)
     idone = [bar(f"idone{g}", 1) for g in range(GROUPS)]
+    eready = bar("eready", 4 * GROUPS)
     state = {"abort": False, "landings": [], "mma": [], "issued": 0, "landed": 0, "mma_issued": 0, "mma_done": 0}
 
     def wait(b, p, bounded=True):
@@ -127,6 +129,8 @@ def run(cnt, seed, withhold_xready=False):
 
     def dequant(g, q):
         yield from rotation(FIRST_DQ + 4 * g + q)
+        yield ("step", "row exponent")
+        eready.arrive()
         use = 0
         for li in range(g, cnt, GROUPS):
             ok = yield from wait(full[li % STAGES], li // STAGES)
@@ -171,6 +175,7 @@ def run(cnt, seed, withhold_xready=False):
         if w == 0:
             yield from producer()
         ok = yield from wait(xready, 0)
+        ok = ok and (yield from wait(eready, 0))
         ok = ok and (yield from wait(dfull, 0))
 
     actors = [epilogue(0)]
@@ -240,7 +245,7 @@ def test_protocol_completes_with_exact_counts(cnt):
         assert not state["mma"] and state["mma_issued"] == 2 * cnt
         for b in B.values():
             assert b.arrived == 0, f"{b.name}: partial phase left at the end"
-        assert B["xready"].phase == 1 and B["dfull"].phase == 1
+        assert B["xready"].phase == 1 and B["dfull"].phase == 1 and B["eready"].phase == 1
         for s in range(STAGES):
             assert B[f"full{s}"].phase == len(range(s, cnt, STAGES))
 

@@ -203,11 +203,34 @@ def test_linear_activation_range(x_std):
     assert tq.tq4_1s_get_status() == 0
 
 
-def test_linear_scale_beyond_fp16_level_range_flagged():
-    # one weight row with half-block scales far above ~93.6: its fp16 levels
-    # overflow, the status word says so, and every other output column is
-    # still correct (accumulator rows are independent)
+def test_linear_any_finite_scale_decode_path():
+    # half-block scales far above ~93.6 (one row x 20000) and far below 2e-6
+    # (one row x 1e-5, fp16 subnormal scales): the decode kernel scales each
+    # dequant group's levels by a per-row power of two, so every output,
+    # those rows' columns included, matches the oracle and nothing is flagged
     m, n, k, seed = 16, 256, 256, 39
+    W = synth.normal_f32((n, k), seed, 0.02)
+    W[3] *= 20000.0
+    W[9] *= 1e-5
+    x = synth.activations_bf16(m, k, seed + 1)
+    p, codes, scales, _ = _quantize_both(W, seed)
+    assert scales[0][3].view(np.float16).astype(np.float32).max() > 94.0
+    y = tq.tq4_1s_linear(_bf16_dev(x), p)
+    torch.cuda.synchronize()
+    assert tq.tq4_1s_get_status() == 0
+    y_ref, _ = oracle.linear(x, codes[0], scales[0], seed)
+    yb = _bits(y)
+    keep = np.array([c for c in range(n) if c not in (3, 9)])
+    assert_close(yb[:, keep], y_ref[:, keep], "decode: ordinary rows")
+    assert_close(yb[:, [3]], y_ref[:, [3]], "decode: scales above the fp16 level range")
+    assert_close(yb[:, [9]], y_ref[:, [9]], "decode: subnormal scales")
+
+
+def test_linear_scale_beyond_fp16_level_range_flagged_stream_k():
+    # the TMA-fed stream-K path (more than 32 rows) still computes levels
+    # with a fixed factor: a row whose scales pass ~93.6 overflows, the
+    # status word says so, and every other output column is still correct
+    m, n, k, seed = 48, 256, 256, 39
     W = synth.normal_f32((n, k), seed, 0.02)
     W[3] *= 20000.0
     x = synth.activations_bf16(m, k, seed + 1)
@@ -217,7 +240,7 @@ def test_linear_scale_beyond_fp16_level_range_flagged():
     assert tq.tq4_1s_get_status() & tq.TQ_DEV_SCALE_RANGE
     y_ref, _ = oracle.linear(x, codes[0], scales[0], seed)
     keep = np.array([c for c in range(n) if c != 3])
-    assert_close(_bits(y)[:, keep], y_ref[:, keep], "linear with one out-of-range row")
+    assert_close(_bits(y)[:, keep], y_ref[:, keep], "stream-K with one out-of-range row")
 
 
 def test_linear_shared_workspace_across_shapes_and_paths():
