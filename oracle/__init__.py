@@ -15,6 +15,11 @@ listed at the top of the C file.  Parity status of each function:
 - router_topk: pinned by invariants (distinct ids, descending order, every
   chosen logit >= every other, weights positive summing to 1), equal-logit
   and single-choice special cases, and k = E against scipy's softmax.
+- f32_to_e4m3, e4m3_to_f64, to_fp8, fp8_dequantize, linear_fp8 (the fp8
+  weight cache of the model card's "Help wanted"): pinned by the format's
+  published values (largest finite 448, smallest subnormal 2^-9), round
+  trips of every code, ties to even, torch's float8_e4m3fn conversion,
+  the conversion's scale and error bounds, and numpy matmul.
 - moe: pinned through closed-form special cases (single slot, constant-level
   experts) and composition with the pinned linear; the squared-ReLU and the
   bf16 rounding of the hidden activation are fixed by the workload
@@ -91,6 +96,12 @@ def _load():
                                     P, P, ctypes.c_uint64, P, P, ctypes.c_uint64, P]
             lib.orc_moe.restype = I64
             lib.orc_router_topk.argtypes = [P, I64, ctypes.c_int, ctypes.c_int, P, P]
+            lib.orc_f32_to_e4m3_sat.argtypes = [ctypes.c_float]
+            lib.orc_f32_to_e4m3_sat.restype = ctypes.c_uint8
+            lib.orc_e4m3_to_f64.argtypes = [ctypes.c_uint8]
+            lib.orc_e4m3_to_f64.restype = ctypes.c_double
+            lib.orc_to_fp8.argtypes = [P, P, I64, I64, ctypes.c_uint64, P, P]
+            lib.orc_linear_fp8.argtypes = [P, I64, I64, P, P, I64, P]
             _lib = lib
     return _lib
 
@@ -283,6 +294,43 @@ def router_topk(z, topk: int):
     w = np.zeros((m, topk), np.float32)
     _load().orc_router_topk(_ptr(z), m, E, topk, _ptr(ids), _ptr(w))
     return ids, w
+
+
+def f32_to_e4m3(x: float) -> int:
+    """fp32 -> OCP E4M3 bits, round to nearest even, saturating at +-448."""
+    return int(_load().orc_f32_to_e4m3_sat(float(np.float32(x))))
+
+
+def e4m3_to_f64(b: int) -> float:
+    return float(_load().orc_e4m3_to_f64(int(b)))
+
+
+def to_fp8(codes, scales, seed: int):
+    """fp8-resident cache of a TQ4_1S weight [n][k]: (q uint8 [n][k] E4M3 bits,
+    row scales float32 [n]); the cached weight is s[n] * q[n][k]."""
+    codes = _c(codes, np.uint8); scales = _c(scales, np.uint16)
+    n, k = codes.shape[0], codes.shape[1] * 2
+    q = np.zeros((n, k), np.uint8)
+    s = np.zeros(n, np.float32)
+    _load().orc_to_fp8(_ptr(codes), _ptr(scales), n, k, seed, _ptr(q), _ptr(s))
+    return q, s
+
+
+def fp8_dequantize(q, s) -> np.ndarray:
+    """The cached weight s[n] * e4m3(q[n][k]) in fp64."""
+    q = _c(q, np.uint8)
+    lut = np.array([e4m3_to_f64(b) for b in range(256)], np.float64)
+    return np.asarray(s, np.float64)[:, None] * lut[q]
+
+
+def linear_fp8(x_bf16, q, s):
+    """y = x * (s q)^T with the sum in fp64: returns (y_f64, y_bf16_bits)."""
+    x = _c(x_bf16, np.uint16); q = _c(q, np.uint8); s = _c(s, np.float32)
+    m, k = x.shape
+    n = q.shape[0]
+    y = np.zeros((m, n), np.float64)
+    _load().orc_linear_fp8(_ptr(x), m, k, _ptr(q), _ptr(s), n, _ptr(y))
+    return y, round_bf16(y)
 
 
 def moe(x_bf16, ids, w, up_codes, up_scales, up_seed, dn_codes, dn_scales, dn_seed):

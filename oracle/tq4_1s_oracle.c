@@ -424,3 +424,72 @@ int64_t orc_moe(const uint16_t *x, int64_t m, int64_t H, int64_t I,
     free(Wup); free(Wdn); free(z); free(u); free(hv);
     return bad;
 }
+
+/* ------------------------------------------------------------------ */
+/* fp8-resident weight cache (model card "Nemotron-TheHobbit-30B-A3B",
+ * section "Help wanted": dequantize once to fp8 and keep the weights
+ * resident, ~63 GB, to remove the per-forward dequantization).  Reading:
+ * fp8 = OCP E4M3 (1 sign, 4 exponent bits with bias 7, 3 mantissa bits, no
+ * infinities, largest finite 448); one fp32 scale per output row n,
+ * s_n = fp32(amax_n / 448) with amax_n = max_k |W_hat[n][k]|; codes
+ * q = e4m3(fp32(W_hat / s_n)) rounded to nearest even, saturating at +-448;
+ * a zero row has s_n = 0 and all codes 0.  The cached weight is s_n * q.  */
+
+/* float -> E4M3 bits, round to nearest even, saturating to +-448; NaN -> 0x7F. */
+uint8_t orc_f32_to_e4m3_sat(float f) {
+    uint8_t sign = signbit(f) ? 0x80 : 0;
+    if (isnan(f)) return 0x7F;
+    double a = fabs((double)f);
+    if (a >= 448.0) return sign | 0x7E;            /* 1.75 * 2^8, the largest finite */
+    if (a < ldexp(1.0, -6)) {                      /* subnormal range: m * 2^-9, m = 0..8 */
+        double m = rint(ldexp(a, 9));
+        return sign | (uint8_t)m;                  /* m == 8 encodes 2^-6 */
+    }
+    int e;
+    frexp(a, &e);
+    e -= 1;                                        /* a in [2^e, 2^(e+1)) */
+    double q = rint(ldexp(a, 3 - e));              /* 8 .. 16 */
+    if (q >= 16.0) { q = 8.0; e += 1; }
+    if (e > 8 || (e == 8 && q > 14.0)) return sign | 0x7E;
+    return sign | (uint8_t)(((e + 7) << 3) | ((int)q - 8));
+}
+
+double orc_e4m3_to_f64(uint8_t b) {
+    int s = (b >> 7) & 1, e = (b >> 3) & 0xF, m = b & 7;
+    double v;
+    if (e == 15 && m == 7) return NAN;
+    if (e == 0) v = ldexp((double)m, -9);
+    else v = ldexp((double)(8 + m), e - 10);
+    return s ? -v : v;
+}
+
+/* TQ4_1S weight [n][k] -> fp8 cache: codes q [n][k] and row scales s [n]. */
+void orc_to_fp8(const uint8_t *codes, const uint16_t *scales, int64_t n, int64_t k, uint64_t seed,
+                uint8_t *q, float *s) {
+    float *W = (float *)malloc(sizeof(float) * (size_t)(n * k));
+    orc_dequantize(codes, scales, n, k, seed, W);
+    for (int64_t i = 0; i < n; i++) {
+        float amax = 0.0f;
+        for (int64_t j = 0; j < k; j++) {
+            float a = fabsf(W[i * k + j]);
+            if (a > amax) amax = a;
+        }
+        float sc = amax / 448.0f;
+        s[i] = sc;
+        for (int64_t j = 0; j < k; j++)
+            q[i * k + j] = (sc == 0.0f) ? 0 : orc_f32_to_e4m3_sat(W[i * k + j] / sc);
+    }
+    free(W);
+}
+
+/* y = x * (s_n q[n][k])^T in fp64 (x bf16 [m][k]). */
+void orc_linear_fp8(const uint16_t *x, int64_t m, int64_t k, const uint8_t *q, const float *s, int64_t n,
+                    double *y) {
+    for (int64_t i = 0; i < m; i++)
+        for (int64_t j = 0; j < n; j++) {
+            double acc = 0.0;
+            for (int64_t kk = 0; kk < k; kk++)
+                acc += orc_bf16_to_f64(x[i * k + kk]) * ((double)s[j] * orc_e4m3_to_f64(q[j * k + kk]));
+            y[i * n + j] = acc;
+        }
+}

@@ -456,3 +456,66 @@ def test_boundary_near_flags_a_value_on_a_threshold_and_a_scale_on_a_midpoint():
     W = _rotate_inverse_f64(v, seed).astype(np.float32).reshape(1, 32)
     near = oracle.boundary_near(W, seed)
     assert near["codes"] == 0 and near["scales"] == 0
+
+
+# ----------------------------------------------------------------- fp8 cache
+def test_e4m3_format_values_and_round_trips():
+    # OCP E4M3: largest finite 448 (0x7E), smallest subnormal 2^-9 (0x01),
+    # smallest normal 2^-6 (0x08), 0x7F is NaN; every finite code decodes and
+    # re-encodes to itself
+    assert oracle.e4m3_to_f64(0x7E) == 448.0 and oracle.e4m3_to_f64(0xFE) == -448.0
+    assert oracle.e4m3_to_f64(0x01) == 2.0 ** -9 and oracle.e4m3_to_f64(0x08) == 2.0 ** -6
+    assert oracle.e4m3_to_f64(0x38) == 1.0 and oracle.e4m3_to_f64(0x3F) == 1.875
+    assert np.isnan(oracle.e4m3_to_f64(0x7F))
+    for b in range(256):
+        if b & 0x7F == 0x7F:
+            continue
+        v = oracle.e4m3_to_f64(b)
+        assert oracle.f32_to_e4m3(v) == b
+    # saturation and ties to even (1 + 1/16 lies between 1 and 1.125: even is 1)
+    assert oracle.f32_to_e4m3(1e6) == 0x7E and oracle.f32_to_e4m3(-500.0) == 0xFE
+    assert oracle.f32_to_e4m3(1.0625) == 0x38 and oracle.f32_to_e4m3(1.1875) == 0x3A
+    assert oracle.f32_to_e4m3(2.0 ** -10) == 0x00 and oracle.f32_to_e4m3(3 * 2.0 ** -10) == 0x02
+
+
+def test_e4m3_rounding_matches_torch_float8():
+    import torch
+    x = np.concatenate([synth.normal_f32(20000, 150, 3.0), synth.normal_f32(5000, 151, 0.01),
+                        np.float32([0.0, 447.0, -447.9, 2.0 ** -9, 5 * 2.0 ** -11])]).astype(np.float32)
+    mine = np.array([oracle.f32_to_e4m3(v) for v in x], np.uint8)
+    ref = torch.from_numpy(x).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    assert np.array_equal(mine, ref)
+
+
+def test_fp8_cache_conversion_bounds():
+    W = synth.student_t_f32((40, 256), 152, 5.0, 0.02)
+    W[7] = 0.0
+    codes, scales, _ = oracle.quantize(W, 152)
+    q, s = oracle.to_fp8(codes, scales, 152)
+    Wh = oracle.dequantize(codes, scales, 152).astype(np.float64)
+    Wc = oracle.fp8_dequantize(q, s)
+    amax = np.abs(Wh).max(axis=1)
+    # the row scale maps the row's largest |w| to 448 exactly once rounded
+    assert np.array_equal(s, (amax.astype(np.float32) / np.float32(448.0)).astype(np.float32))
+    assert s[7] == 0.0 and np.all(q[7] == 0)
+    nz = [i for i in range(40) if i != 7]
+    assert all(np.any((q[i] & 0x7F) == 0x7E) for i in nz)
+    # E4M3 keeps 3 mantissa bits: relative error at most 2^-4 above the
+    # subnormal range, absolute error at most 2^-10 s below it
+    err = np.abs(Wc - Wh)
+    bound = np.maximum(np.abs(Wh) * 2.0 ** -4, s[:, None].astype(np.float64) * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(err <= bound)
+    # cosine of the cached weight against the TQ4_1S reconstruction
+    for i in nz:
+        c = Wh[i] @ Wc[i] / np.linalg.norm(Wh[i]) / np.linalg.norm(Wc[i])
+        assert c > 0.998
+
+
+def test_fp8_linear_matches_numpy_matmul():
+    W = synth.normal_f32((24, 96), 153, 0.02)
+    codes, scales, _ = oracle.quantize(W, 153)
+    q, s = oracle.to_fp8(codes, scales, 153)
+    x = synth.activations_bf16(5, 96, 154)
+    y, yb = oracle.linear_fp8(x, q, s)
+    ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ oracle.fp8_dequantize(q, s).T
+    assert np.allclose(y, ref, rtol=1e-12, atol=1e-15)
