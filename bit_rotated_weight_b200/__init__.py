@@ -25,7 +25,7 @@ __all__ = [
     "tq4_1s_version", "tq4_1s_error_string", "tq4_1s_packed_bytes", "tq4_1s_sign_mask", "tq4_1s_codebook",
     "tq4_1s_quantize", "tq4_1s_quantize_batched", "tq4_1s_dequantize", "tq4_1s_linear_workspace", "tq4_1s_linear",
     "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_logits", "tq4_1s_router_topk", "tq4_1s_moe_route", "tq4_1s_get_status", "tq4_1s_launch_count",
-    "tq4_1s_linear_static", "tq4_1s_debug_hook",
+    "tq4_1s_linear_static", "tq4_1s_debug_hook", "Fp8Weight", "tq4_1s_to_fp8", "tq4_1s_linear_fp8",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -86,6 +86,9 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                 "tq4_1s_get_status": ([P, ctypes.POINTER(I32)], ctypes.c_int),
                 "tq4_1s_launch_count": ([], ctypes.c_uint64),
                 "tq4_1s_debug_hook": ([ctypes.c_int, I64], ctypes.c_int),
+                "tq4_1s_to_fp8": ([W, P, P, P], ctypes.c_int),
+                "tq4_1s_linear_fp8_workspace": ([I64, I64, I64], SZ),
+                "tq4_1s_linear_fp8": ([P, I64, P, P, I64, I64, I32, P, P, SZ, P], ctypes.c_int),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -364,3 +367,42 @@ def tq4_1s_linear_static(x: torch.Tensor, w: Packed, out: torch.Tensor | None = 
 def tq4_1s_debug_hook(what: int, value: int) -> None:
     """Test hooks of the library (fault injection, short device waits); see include/tq4_1s.h."""
     _check(load_library().tq4_1s_debug_hook(what, value), "debug_hook")
+
+
+@dataclass
+class Fp8Weight:
+    """The fp8-resident cache of a TQ4_1S weight: E4M3 codes q [rows][k] (uint8)
+    and one float32 scale per row; the cached weight is wscale[n] * q[n][k]."""
+    q: torch.Tensor
+    wscale: torch.Tensor
+    n: int
+    k: int
+    flags: int = 0
+
+
+def tq4_1s_to_fp8(w: Packed, flags: int = 0) -> Fp8Weight:
+    """Convert a packed TQ4_1S weight (stack) to the fp8 cache (rows = n * E)."""
+    rows = w.n * w.num_experts
+    q = torch.empty((rows, w.k), dtype=torch.uint8, device=w.codes.device)
+    sc = torch.empty(rows, dtype=torch.float32, device=w.codes.device)
+    ws = w.c_struct()
+    _check(load_library().tq4_1s_to_fp8(ctypes.byref(ws), _ptr(q), _ptr(sc), _stream(q.device)), "to_fp8")
+    return Fp8Weight(q, sc, rows, w.k, flags)
+
+
+def tq4_1s_linear_fp8(x: torch.Tensor, w: Fp8Weight, out: torch.Tensor | None = None,
+                      workspace: torch.Tensor | None = None) -> torch.Tensor:
+    """y = bf16(x @ (wscale * q)^T) with the fp8 cache, x bfloat16 [m][k] on CUDA."""
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a CUDA bfloat16 [m][k] tensor")
+    x = x.contiguous()
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device)
+    lib = load_library()
+    if workspace is None:   # (used only when the decode kernel does not take the shape)
+        workspace = _workspace(lib.tq4_1s_linear_fp8_workspace(m, w.n, w.k), x.device, "fp8_large")
+    wsz = 0 if workspace is None else workspace.numel()
+    _check(lib.tq4_1s_linear_fp8(_ptr(x), m, _ptr(w.q), _ptr(w.wscale), w.n, w.k, w.flags, _ptr(out),
+                                 _ptr(workspace), wsz, _stream(x.device)), "linear_fp8")
+    return out

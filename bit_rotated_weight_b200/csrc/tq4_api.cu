@@ -240,6 +240,16 @@ static bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t col
   });
 }
 
+// fp8 cache codes [n][k] bytes, box 128 B x 128 rows, 128-byte swizzle.
+static bool map_fp8(CUtensorMap* m, const uint8_t* q, int64_t n, int64_t k) {
+  return cached_map(m, MapKey{3, q, n, k, 1}, [&](CUtensorMap* out) {
+    const uint64_t dims[3] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n), 1};
+    const uint64_t strides[2] = {static_cast<uint64_t>(k), static_cast<uint64_t>(n * k)};
+    const uint32_t box[3] = {128, 128, 1};
+    return make_map(out, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, q, dims, strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
+  });
+}
+
 static size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 // Small-m path threshold: up to this many rows, the stream-K kernel streams
@@ -535,6 +545,81 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
   const int grid = static_cast<int>(tiles < sms ? tiles : sms);
   return cuda_rc(launch_gemm_bf16(&tx, &tw, y, static_cast<int32_t>(m), static_cast<int32_t>(w->n),
                                   static_cast<int32_t>(w->k), grid, st));
+}
+
+// ------------------------------------------------------------------ fp8 cache
+TQ_API int tq4_1s_to_fp8(const tq4_1s_weight* w, uint8_t* q, float* wscale, tq4_stream_t stream) {
+  int rc = weight_ok(w, true);
+  if (rc) return rc;
+  if (!q || !wscale) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(wscale)) return TQ_ERR_ALIGNMENT;
+  if ((rc = check_device(nullptr))) return rc;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
+  return cuda_rc(launch_to_fp8(w->codes, w->scales, q, wscale, w->n * w->num_experts, w->k, sign_mask_of(w->seed),
+                               codebook(), reinterpret_cast<cudaStream_t>(stream)));
+}
+
+static int fp8_check(int64_t m, int64_t n, int64_t k) {
+  if (m < 0 || m > (1ll << 24) || n <= 0 || k <= 0 || k % 32 != 0 || n > (1ll << 30) || k > (1ll << 30))
+    return TQ_ERR_INVALID_ARG;
+  return TQ_OK;
+}
+
+TQ_API size_t tq4_1s_linear_fp8_workspace(int64_t m, int64_t n, int64_t k) {
+  if (fp8_check(m, n, k) != TQ_OK || m == 0) return 0;
+  return align256(static_cast<size_t>(n) * static_cast<size_t>(k) * 2);   // the bf16 weight of the large-m path
+}
+
+TQ_API int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, const float* wscale, int64_t n,
+                             int64_t k, int32_t flags, uint16_t* y, void* ws, size_t ws_bytes, tq4_stream_t stream) {
+  int rc = fp8_check(m, n, k);
+  if (rc) return rc;
+  if ((flags & ~TQ_WEIGHT_STATIC) != 0) return TQ_ERR_INVALID_ARG;
+  if (m == 0) return TQ_OK;
+  if (!x || !q || !wscale || !y) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(q) || !aligned16(wscale) || !aligned16(y)) return TQ_ERR_ALIGNMENT;
+  int sms = 0;
+  if ((rc = check_device(&sms))) return rc;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  const int64_t tiles = (n + 127) / 128, KI = (k + 127) / 128;
+  if (m <= kSegRows) {
+    const int nb = m > 16 ? 2 : 1;
+    const int split = choose_decode_split(tiles, KI, sms, nb, true);
+    if (split > 0) {
+      if (take_injected_failure()) return TQ_ERR_CUDA;
+      alignas(64) CUtensorMap tc;
+      if (!map_fp8(&tc, q, n, k)) return TQ_ERR_CUDA;
+      DecodeArgs d{};
+      d.n = static_cast<int32_t>(n);
+      d.k = static_cast<int32_t>(k);
+      d.m = static_cast<int32_t>(m);
+      d.nb = nb;
+      d.row_tiles = static_cast<int32_t>(tiles);
+      d.k_iters = static_cast<int32_t>(KI);
+      d.split = split;
+      d.static_w = (flags & TQ_WEIGHT_STATIC) ? 1 : 0;
+      d.test_withhold = withhold_arrival_hook() ? 1 : 0;
+      d.fp8 = 1;
+      d.wscale = wscale;
+      d.x = x;
+      d.y = y;
+      return cuda_rc(launch_decode(&tc, d, st));
+    }
+  }
+  // large m (or a shape the decode kernel does not take): the bf16 weight in
+  // the workspace, then the tensor-core GEMM
+  const size_t need = align256(static_cast<size_t>(n) * static_cast<size_t>(k) * 2);
+  if (!ws || ws_bytes < need) return TQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
+  uint16_t* wh = static_cast<uint16_t*>(ws);
+  if (launch_fp8_to_bf16(q, wscale, wh, n, k, st) != cudaSuccess) return TQ_ERR_CUDA;
+  alignas(64) CUtensorMap tx, tw;
+  if (!map_bf16(&tx, x, m, k, 128) || !map_bf16(&tw, wh, n, k, 256)) return TQ_ERR_CUDA;
+  const int64_t gt = ((m + 127) / 128) * ((n + 255) / 256);
+  const int grid = static_cast<int>(gt < sms ? gt : sms);
+  return cuda_rc(launch_gemm_bf16(&tx, &tw, y, static_cast<int32_t>(m), static_cast<int32_t>(n),
+                                  static_cast<int32_t>(k), grid, st));
 }
 
 static int64_t H_of(const tq4_1s_weight* up) { return up->k; }

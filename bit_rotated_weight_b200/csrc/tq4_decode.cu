@@ -71,13 +71,15 @@ struct DecodeShared {
 };
 
 // Dynamic shared memory: codes ring | B tiles [iters][2 halves][16 nb rows x 128 B] |
-// level table | cluster reduction buffer [split][rows per CTA][16 nb] fp32.
+// level table (TQ4_1S only) | cluster reduction buffer [split][rows per CTA][16 nb] fp32.
+// The fp8 cache (f8) streams 128 B of codes per row and iteration and needs no table.
+__host__ __device__ constexpr int tile_bytes(bool f8) { return f8 ? 2 * kCodesTile : kCodesTile; }
 __host__ __device__ constexpr int b_half_bytes(int nb) { return 16 * nb * 128; }
-__host__ __device__ constexpr int off_b() { return kStagesD * kCodesTile; }
-__host__ __device__ constexpr int off_lut(int nb) { return off_b() + kMaxIters * 2 * b_half_bytes(nb); }
-__host__ __device__ constexpr int off_red(int nb) { return off_lut(nb) + kLutBytesD; }
+__host__ __device__ constexpr int off_b(bool f8) { return kStagesD * tile_bytes(f8); }
+__host__ __device__ constexpr int off_lut(int nb, bool f8) { return off_b(f8) + kMaxIters * 2 * b_half_bytes(nb); }
+__host__ __device__ constexpr int off_red(int nb, bool f8) { return off_lut(nb, f8) + (f8 ? 0 : kLutBytesD); }
 // (the reduction buffer holds split * ceil(128 / split) <= 135 rows)
-__host__ __device__ constexpr int smem_total(int nb) { return off_red(nb) + 136 * 16 * nb * 4 + 1024; }
+__host__ __device__ constexpr int smem_total(int nb, bool f8) { return off_red(nb, f8) + 136 * 16 * nb * 4 + 1024; }
 
 struct LevelTableD {
   uint32_t h[16];   // fp16 bits of 256 * levels[0..15]
@@ -126,16 +128,22 @@ __device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, 
                : "memory");
 }
 
-template <int NB>
+// F8: the weight is the fp8-resident cache (E4M3 codes [n][k], one fp32
+// scale per row; "Help wanted": dequantize once, keep fp8 resident) instead of
+// TQ4_1S: no rotation (the cache is in the weight's own domain), levels are
+// the E4M3 values converted to fp16 (exact), and the row scale multiplies the
+// accumulator in the epilogue.
+template <int NB, bool F8>
 __global__ void __launch_bounds__(kThreads, 2)
     decode_kernel(const __grid_constant__ CUtensorMap tm_codes, const DecodeArgs a,
                   const __grid_constant__ LevelTableD lt) {
   __shared__ DecodeShared sh;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
-  uint8_t* btiles = smem + off_b();
-  uint8_t* lut = smem + off_lut(NB);
-  uint8_t* red = smem + off_red(NB);
+  constexpr int kTile = tile_bytes(F8);
+  uint8_t* btiles = smem + off_b(F8);
+  uint8_t* lut = smem + off_lut(NB, F8);
+  uint8_t* red = smem + off_red(NB, F8);
   constexpr int kHalf = b_half_bytes(NB);
   constexpr int kAccW = 16 * NB;          // accumulator columns per group
   constexpr int kACol0 = kGroups * kAccW; // first A-stage column
@@ -170,7 +178,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     tmem_alloc(&sh.tmem_base, NB == 1 ? 256 : 512);
     tmem_relinquish();
   }
-  {
+  if (!F8) {
     // level-pair table: entry b (a code byte) of lane l's copy at byte
     // 128 b + 4 l holds {256 c[b & 15], 256 c[b >> 4]} * (fp16 pair)
     uint32_t* lw = reinterpret_cast<uint32_t*>(lut);
@@ -195,8 +203,8 @@ __global__ void __launch_bounds__(kThreads, 2)
   // may have written it (a quantize) and everything waits.
   auto issue_codes = [&](int li) {
     const int s = li % kStagesD;
-    mbar_arrive_expect_tx(&sh.full[s], kCodesTile);
-    tma_load_3d(smem + s * kCodesTile, &tm_codes, &sh.full[s], (it0 + li) * 64, row0, 0);
+    mbar_arrive_expect_tx(&sh.full[s], kTile);
+    tma_load_3d(smem + s * kTile, &tm_codes, &sh.full[s], (it0 + li) * (F8 ? 128 : 64), row0, 0);
   };
   const int npre = cnt < kStagesD ? cnt : kStagesD;
   if (stat && warp == 0 && lane == 0)
@@ -214,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       const int li = dq_group + kGroups * u;
 #pragma unroll
       for (int j = 0; j < 4; ++j) sraw[u][j] = 0u;
-      if (li < cnt && row < a.n) {
+      if (!F8 && li < cnt && row < a.n) {
         const int kit = it0 + li;
         const uint32_t* sp = reinterpret_cast<const uint32_t*>(a.scales + static_cast<int64_t>(row) * kh16 + kit * 8);
         if ((kh16 & 7) == 0) {
@@ -261,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const uint32_t sw = ww[e] ^ a.x_sign[4 * q + e];
+            const uint32_t sw = F8 ? ww[e] : (ww[e] ^ a.x_sign[4 * q + e]);
             v[8 * q + 2 * e] = __uint_as_float(sw << 16);
             v[8 * q + 2 * e + 1] = __uint_as_float(sw & 0xFFFF0000u);
           }
@@ -270,14 +278,16 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
         for (int i = 0; i < 32; ++i) v[i] = 0.0f;
       }
+      if (!F8) {
 #pragma unroll
-      for (int h = 1; h < 32; h <<= 1) {
+        for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          if (!(j & h)) {
-            const float p = v[j], q = v[j + h];
-            v[j] = __fadd_rn(p, q);
-            v[j + h] = __fsub_rn(p, q);
+          for (int j = 0; j < 32; ++j) {
+            if (!(j & h)) {
+              const float p = v[j], q = v[j + h];
+              v[j] = __fadd_rn(p, q);
+              v[j + h] = __fsub_rn(p, q);
+            }
           }
         }
       }
@@ -287,7 +297,7 @@ __global__ void __launch_bounds__(kThreads, 2)
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
       int e = 0;
-      const float bound = __fmul_rn(mx, r);   // the token's largest |x'|
+      const float bound = F8 ? mx : __fmul_rn(mx, r);   // the token's largest |x'| (|x| for the fp8 cache)
       if (bound > 0.0f && isfinite(bound)) {
         int ex;
         frexpf(bound, &ex);   // bound in [2^(ex-1), 2^ex)
@@ -295,7 +305,7 @@ __global__ void __launch_bounds__(kThreads, 2)
         e = e < -100 ? -100 : (e > 100 ? 100 : e);
       }
       if (lane == 0) sh.row_scale[tk] = ldexpf(1.0f, e);
-      const float rd = __fmul_rn(r, ldexpf(1.0f, -e));   // exact
+      const float rd = F8 ? ldexpf(1.0f, -e) : __fmul_rn(r, ldexpf(1.0f, -e));   // exact
       if (lane < nsl) {
         const int li = lane >> 2, h = (lane >> 1) & 1, c0 = (lane & 1) * 4;
         uint8_t* rowp = btiles + (li * 2 + h) * kHalf + (tk >> 3) * 1024 + (tk & 7) * 128;
@@ -351,10 +361,52 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     int use = 0;
 #pragma unroll 1
-    for (int li = g; li < cnt; li += kGroups, ++use) {
+    for (int li = g; F8 && li < cnt; li += kGroups, ++use) {
+      // fp8 cache: 128 B of E4M3 codes per row (128-byte swizzle: 16-byte
+      // chunk c of row t at chunk c ^ (t & 7)); each byte pair converts to an
+      // fp16 pair exactly
       const int s = li % kStagesD;
       if (!wwait(&sh.full[s], (li / kStagesD) & 1, abortp)) break;
-      const uint8_t* cb = smem + s * kCodesTile + trow * 64;
+      const uint8_t* cb = smem + s * kTile + trow * 128;
+      bool ok = true;
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (use > 0 && !wwait(&sh.afree[g][h], (use - 1) & 1, abortp)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+#pragma unroll
+        for (int kb2 = 0; kb2 < 2; ++kb2) {
+          const int kb = 2 * h + kb2;
+          uint32_t o[16];
+#pragma unroll
+          for (int ch = 0; ch < 2; ++ch) {
+            const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * ((2 * kb + ch) ^ (trow & 7)));
+            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+                  "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+                  : "=r"(o[8 * ch + 2 * j]), "=r"(o[8 * ch + 2 * j + 1])
+                  : "r"(cw[j]));
+          }
+          tmem_st16(a_stage + lane_base + 16 * kb, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.afull[g][h]);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.empty[s]);   // the stage was read in full
+      if (!ok) break;
+    }
+#pragma unroll 1
+    for (int li = g; !F8 && li < cnt; li += kGroups, ++use) {
+      const int s = li % kStagesD;
+      if (!wwait(&sh.full[s], (li / kStagesD) & 1, abortp)) break;
+      const uint8_t* cb = smem + s * kTile + trow * 64;
       uint4 c[4];
 #pragma unroll
       for (int kb = 0; kb < 4; ++kb) c[kb] = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((trow >> 1) & 3)));
@@ -449,6 +501,8 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int ngroups = cnt < kGroups ? cnt : kGroups;
+    // TQ4_1S: levels carry a factor 256; fp8 cache: the row's scale
+    const float wsc = F8 ? ((row0 + trow < a.n) ? __ldcg(a.wscale + row0 + trow) : 0.0f) : 1.0f / kLevelScaleD;
     if (ok) {
 #pragma unroll
       for (int c = 0; c < NB; ++c) {
@@ -464,7 +518,7 @@ __global__ void __launch_bounds__(kThreads, 2)
           for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(rr[j]), rs));
         }
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], __fmul_rn(sh.row_scale[16 * c + j], 1.0f / kLevelScaleD));
+        for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], __fmul_rn(sh.row_scale[16 * c + j], wsc));
         if (split > 1) {
           // row trow goes to the CTA that owns it: [source rank][row - owner's first row][token]
           const int q = (trow * split) >> 7;
@@ -514,14 +568,14 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (warp == 1) tmem_dealloc(tmem, NB == 1 ? 256 : 512);
 }
 
-template <int NB>
+template <int NB, bool F8>
 cudaError_t launch_decode_nb(const void* tm_codes, const DecodeArgs& a, cudaStream_t st) {
   static bool attr_set = false;
-  const int smem = smem_total(NB);
+  const int smem = smem_total(NB, F8);
   if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(decode_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    cudaError_t e = cudaFuncSetAttribute(decode_kernel<NB, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
-      e = cudaFuncSetAttribute(decode_kernel<NB>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      e = cudaFuncSetAttribute(decode_kernel<NB, F8>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     if (e != cudaSuccess) return e;
     attr_set = true;
   }
@@ -551,18 +605,18 @@ cudaError_t launch_decode_nb(const void* tm_codes, const DecodeArgs& a, cudaStre
     cfg.numAttrs = 2;
   }
   const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NB>, m0, a, lt);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NB, F8>, m0, a, lt);
   if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();
 }
 
-template <int NB>
+template <int NB, bool F8>
 int decode_max_clusters_nb(int s) {
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(s));
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = static_cast<size_t>(smem_total(NB));
+  cfg.dynamicSmemBytes = static_cast<size_t>(smem_total(NB, F8));
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = static_cast<unsigned>(s);
@@ -570,13 +624,13 @@ int decode_max_clusters_nb(int s) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaFuncSetAttribute(decode_kernel<NB>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_total(NB)) !=
+  if (cudaFuncSetAttribute(decode_kernel<NB, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_total(NB, F8)) !=
       cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<NB>, &cfg) != cudaSuccess) {
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel<NB, F8>, &cfg) != cudaSuccess) {
     cudaGetLastError();
     return 0;
   }
@@ -585,18 +639,22 @@ int decode_max_clusters_nb(int s) {
 
 }  // namespace
 
-size_t decode_smem_bytes(int nb) { return static_cast<size_t>(nb == 1 ? smem_total(1) : smem_total(2)); }
-
-cudaError_t launch_decode(const void* tm_codes, const DecodeArgs& a, cudaStream_t st) {
-  return a.nb == 1 ? launch_decode_nb<1>(tm_codes, a, st) : launch_decode_nb<2>(tm_codes, a, st);
+size_t decode_smem_bytes(int nb, bool f8) {
+  return static_cast<size_t>(nb == 1 ? (f8 ? smem_total(1, true) : smem_total(1, false))
+                                     : (f8 ? smem_total(2, true) : smem_total(2, false)));
 }
 
-int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb) {
+cudaError_t launch_decode(const void* tm_codes, const DecodeArgs& a, cudaStream_t st) {
+  if (a.fp8) return a.nb == 1 ? launch_decode_nb<1, true>(tm_codes, a, st) : launch_decode_nb<2, true>(tm_codes, a, st);
+  return a.nb == 1 ? launch_decode_nb<1, false>(tm_codes, a, st) : launch_decode_nb<2, false>(tm_codes, a, st);
+}
+
+int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb, bool f8) {
   // the largest s in [1, 8] with s <= k_iters, at most kMaxIters iterations
   // per CTA, one CTA per SM (tiles * s <= sms) and all clusters resident at
   // once; 0 if none fits.  Cluster capacities are queried once per device.
   static std::mutex mu;
-  static int cap[64][2][9];   // resident clusters + 1 (0 = not queried yet)
+  static int cap[64][4][9];   // per (nb, format): resident clusters + 1 (0 = not queried yet)
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) {
     cudaGetLastError();
@@ -608,8 +666,11 @@ int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb) {
     int c;
     {
       std::lock_guard<std::mutex> g(mu);
-      int& slot = cap[dev][nb == 1 ? 0 : 1][s];
-      if (slot == 0) slot = (nb == 1 ? decode_max_clusters_nb<1>(s) : decode_max_clusters_nb<2>(s)) + 1;
+      int& slot = cap[dev][(nb == 1 ? 0 : 1) + (f8 ? 2 : 0)][s];
+      if (slot == 0)
+        slot = (f8 ? (nb == 1 ? decode_max_clusters_nb<1, true>(s) : decode_max_clusters_nb<2, true>(s))
+                   : (nb == 1 ? decode_max_clusters_nb<1, false>(s) : decode_max_clusters_nb<2, false>(s))) +
+               1;
       c = slot - 1;
     }
     if (tiles <= c) return s;

@@ -47,6 +47,12 @@ cudaError_t launch_dequantize_f32(const uint8_t* codes, const uint16_t* scales, 
                                   uint32_t mask, const CodebookF32& cb, cudaStream_t st);
 cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales, uint16_t* out, int64_t rows,
                                    int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st);
+// The fp8-resident cache: TQ4_1S rows -> E4M3 codes [rows][k] + fp32 row
+// scales, and the cache -> bf16 weight (large-m path of the fp8 linear).
+cudaError_t launch_to_fp8(const uint8_t* codes, const uint16_t* scales, uint8_t* q, float* wscale, int64_t rows,
+                          int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st);
+cudaError_t launch_fp8_to_bf16(const uint8_t* q, const float* wscale, uint16_t* out, int64_t rows, int64_t k,
+                               cudaStream_t st);
 // Activation rotation for the stream-K GEMM: x' = r H diag(s) x per 32-slice
 // of each row, scaled by a per-row power of two 2^-e and rounded to fp16
 // [rows][k]; row_scale[row] = 2^e.  Row r reads x row
@@ -142,6 +148,8 @@ struct DecodeArgs {
   int32_t split;                // CTAs per row tile (>= 1, <= k_iters)
   int32_t static_w;             // the weight may be read before the dependency wait
   int32_t test_withhold;        // test hook: rotation warp 7 never reports (its bounded waiters run out)
+  int32_t fp8;                  // the weight is the fp8 cache (codes = E4M3 [n][k], wscale [n]), else TQ4_1S
+  const float* wscale;          // fp8 cache: one fp32 scale per row
   const uint16_t* x;            // bf16 [m][k]
   const uint16_t* scales;       // [n][k/16] fp16 bits
   uint16_t* y;                  // bf16 [m][n]
@@ -149,8 +157,8 @@ struct DecodeArgs {
 };
 cudaError_t launch_decode(const void* tm_codes, const DecodeArgs& a, cudaStream_t st);
 // The split for a decode launch of `tiles` row tiles (0: the kernel does not fit).
-int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb);
-size_t decode_smem_bytes(int nb);
+int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb, bool f8 = false);
+size_t decode_smem_bytes(int nb, bool f8);
 
 // ---------------------------------------------------------------- GEMM
 // y[m][n] = bf16( x[m][k] * w[n][k]^T ), bf16 operands via TMA tensor maps.

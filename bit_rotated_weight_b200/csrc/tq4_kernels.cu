@@ -9,6 +9,8 @@
 // warp and runs the same butterfly through lane shuffles.
 #include <climits>
 
+#include <cuda_fp8.h>
+
 #include "tq4_internal.h"
 
 namespace tq4 {
@@ -211,6 +213,27 @@ __global__ void __launch_bounds__(256) quantize_kernel(const __grid_constant__ Q
 }
 
 // ------------------------------------------------------------------ dequantize
+// W_hat of one 32-block in fp32: levels c[code] * d, the butterfly, x r, the
+// signs -- one rounding per operation in this fixed order.
+__device__ __forceinline__ void dequant_block_f32(const uint4 cw, uint32_t sw, uint32_t mask, const float* s_c,
+                                                  float (&a)[32]) {
+  const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
+  const float d0 = __half2float(__ushort_as_half(static_cast<uint16_t>(sw & 0xFFFFu)));
+  const float d1 = __half2float(__ushort_as_half(static_cast<uint16_t>(sw >> 16)));
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const uint32_t code = (words[e >> 3] >> (4 * (e & 7))) & 0xFu;
+    a[e] = __fmul_rn(s_c[code], e < 16 ? d0 : d1);
+  }
+  fwht32_regs(a);
+  const float r = rsqrt32();
+#pragma unroll
+  for (int e = 0; e < 32; ++e) {
+    const float x = __fmul_rn(a[e], r);
+    a[e] = ((mask >> e) & 1u) ? -x : x;
+  }
+}
+
 // W_hat = diag(s) * r * H * (c[code] * d), fp32 or bf16 output; one thread per
 // 32-block, butterfly in registers.
 template <typename TO>
@@ -222,28 +245,14 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
   __syncthreads();
   const int64_t kb_per_row = k / 32;
   const int64_t nblocks = rows * kb_per_row;
-  const float r = rsqrt32();
   for (int64_t b = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; b < nblocks;
        b += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t row = b / kb_per_row, kb = b - row * kb_per_row;
     const uint4 cw = __ldg(reinterpret_cast<const uint4*>(codes + row * (k / 2) + kb * 16));
     const uint32_t sw = __ldg(reinterpret_cast<const uint32_t*>(scales + row * (k / 16) + kb * 2));
-    const uint32_t words[4] = {cw.x, cw.y, cw.z, cw.w};
-    const float d0 = __half2float(__ushort_as_half(static_cast<uint16_t>(sw & 0xFFFFu)));
-    const float d1 = __half2float(__ushort_as_half(static_cast<uint16_t>(sw >> 16)));
     float a[32];
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const uint32_t code = (words[e >> 3] >> (4 * (e & 7))) & 0xFu;
-      a[e] = __fmul_rn(s_c[code], e < 16 ? d0 : d1);
-    }
-    fwht32_regs(a);
+    dequant_block_f32(cw, sw, mask, s_c, a);
     TO* o = out + row * k + kb * 32;
-#pragma unroll
-    for (int e = 0; e < 32; ++e) {
-      const float x = __fmul_rn(a[e], r);
-      a[e] = ((mask >> e) & 1u) ? -x : x;
-    }
     if constexpr (sizeof(TO) == 4) {
       float4* o4 = reinterpret_cast<float4*>(o);
 #pragma unroll
@@ -255,6 +264,94 @@ __global__ void __launch_bounds__(256) dequantize_kernel(const uint8_t* __restri
         o4[i] = make_uint4(pack_bf16x2(a[8 * i], a[8 * i + 1]), pack_bf16x2(a[8 * i + 2], a[8 * i + 3]),
                            pack_bf16x2(a[8 * i + 4], a[8 * i + 5]), pack_bf16x2(a[8 * i + 6], a[8 * i + 7]));
     }
+  }
+}
+
+// ------------------------------------------------------------------ fp8 cache
+// TQ4_1S -> the fp8-resident cache of the model card's "Help wanted" (dequantize
+// once, keep the weight resident in fp8): per row n, s_n = fp32(amax_n / 448)
+// over the row's W_hat, codes = E4M3(fp32(W_hat / s_n)) rounded to nearest
+// even and saturating; a zero row gets s_n = 0 and zero codes.  One CTA per
+// row: a first pass takes the row maximum, a second dequantizes again and
+// converts (W_hat is not kept).
+__global__ void __launch_bounds__(256) to_fp8_kernel(const uint8_t* __restrict__ codes,
+                                                     const uint16_t* __restrict__ scales, uint8_t* __restrict__ q,
+                                                     float* __restrict__ wscale, int64_t rows, int64_t k,
+                                                     uint32_t mask, CodebookF32 cb) {
+  __shared__ float s_c[16];
+  __shared__ float s_max[8];
+  if (threadIdx.x < 16) s_c[threadIdx.x] = cb.levels[threadIdx.x];
+  __syncthreads();
+  const int64_t nkb = k / 32;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const uint8_t* cr = codes + row * (k / 2);
+    const uint16_t* sr = scales + row * (k / 16);
+    float mx = 0.0f;
+    for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) {
+      float a[32];
+      dequant_block_f32(__ldg(reinterpret_cast<const uint4*>(cr + kb * 16)),
+                        __ldg(reinterpret_cast<const uint32_t*>(sr + kb * 2)), mask, s_c, a);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) mx = fmaxf(mx, fabsf(a[e]));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if ((threadIdx.x & 31) == 0) s_max[threadIdx.x >> 5] = mx;
+    __syncthreads();
+    mx = s_max[0];
+    for (int w = 1; w < 8; ++w) mx = fmaxf(mx, s_max[w]);
+    __syncthreads();   // s_max is rewritten for the next row
+    const float sc = __fdiv_rn(mx, 448.0f);
+    if (threadIdx.x == 0) wscale[row] = sc;
+    for (int64_t kb = threadIdx.x; kb < nkb; kb += blockDim.x) {
+      float a[32];
+      dequant_block_f32(__ldg(reinterpret_cast<const uint4*>(cr + kb * 16)),
+                        __ldg(reinterpret_cast<const uint32_t*>(sr + kb * 2)), mask, s_c, a);
+      uint32_t w[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        uint32_t word = 0u;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const float v = (sc == 0.0f) ? 0.0f : __fdiv_rn(a[4 * i + j], sc);
+          const uint32_t b = static_cast<uint32_t>(__nv_cvt_float_to_fp8(v, __NV_SATFINITE, __NV_E4M3));
+          word |= b << (8 * j);
+        }
+        w[i] = word;
+      }
+      uint4* dst = reinterpret_cast<uint4*>(q + row * k + kb * 32);
+      dst[0] = make_uint4(w[0], w[1], w[2], w[3]);
+      dst[1] = make_uint4(w[4], w[5], w[6], w[7]);
+    }
+  }
+}
+
+// fp8 cache -> bf16 weight: out[n][k] = bf16(s_n * e4m3(q[n][k])) (the large-m
+// path of the fp8 linear); a thread converts 16 codes.
+__global__ void __launch_bounds__(256) fp8_to_bf16_kernel(const uint8_t* __restrict__ q,
+                                                          const float* __restrict__ wscale,
+                                                          uint16_t* __restrict__ out, int64_t rows, int64_t k) {
+  const int64_t per_row = k / 16, total = rows * per_row;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = i / per_row, c = i - row * per_row;
+    const uint4 v = __ldg(reinterpret_cast<const uint4*>(q + row * k + c * 16));
+    const float sc = __ldg(wscale + row);
+    const uint32_t vw[4] = {v.x, v.y, v.z, v.w};
+    uint32_t o[8];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const __half2_raw hr = __nv_cvt_fp8x2_to_halfraw2(static_cast<__nv_fp8x2_storage_t>(vw[j] >> (16 * h)),
+                                                          __NV_E4M3);
+        const float2 f = __half22float2(*reinterpret_cast<const __half2*>(&hr));
+        o[2 * j + h] = pack_bf16x2(__fmul_rn(f.x, sc), __fmul_rn(f.y, sc));
+      }
+    }
+    uint4* dst = reinterpret_cast<uint4*>(out + row * k + c * 16);
+    dst[0] = make_uint4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_uint4(o[4], o[5], o[6], o[7]);
   }
 }
 
@@ -600,6 +697,21 @@ cudaError_t launch_dequantize_bf16(const uint8_t* codes, const uint16_t* scales,
                                    int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
   dequantize_kernel<uint16_t><<<grid_threads(rows * (k / 32), 256), 256, 0, st>>>(codes, scales, out, rows, k,
                                                                                    mask, cb);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_to_fp8(const uint8_t* codes, const uint16_t* scales, uint8_t* q, float* wscale, int64_t rows,
+                          int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st) {
+  const int64_t g = rows < 148LL * 8 ? rows : 148LL * 8;
+  to_fp8_kernel<<<static_cast<unsigned>(g), 256, 0, st>>>(codes, scales, q, wscale, rows, k, mask, cb);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp8_to_bf16(const uint8_t* q, const float* wscale, uint16_t* out, int64_t rows, int64_t k,
+                               cudaStream_t st) {
+  fp8_to_bf16_kernel<<<grid_threads(rows * (k / 16), 256), 256, 0, st>>>(q, wscale, out, rows, k);
   note_launches(1);
   return cudaGetLastError();
 }

@@ -179,6 +179,35 @@ size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
 int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, void* ws, size_t ws_bytes,
                   tq4_stream_t stream);
 
+/* The fp8-resident weight cache of the model card's "Help wanted" section:
+ * dequantize the TQ4_1S weight once and keep it resident in fp8 (about 8
+ * bits per weight instead of 5), so no forward pass dequantizes TQ4_1S.
+ * Format (reading; the card names only "fp8"): OCP E4M3 codes q [rows][k]
+ * (row-major bytes, rows = n * num_experts) and one fp32 scale per row,
+ *   s_n = fp32(amax_n / 448),  q[n][k] = E4M3(fp32(W_hat[n][k] / s_n))
+ * with W_hat the dequantized weight (as tq4_1s_dequantize computes it),
+ * amax_n the largest |W_hat| of row n, rounding to nearest even, saturating
+ * at +-448; a zero row has s_n = 0 and zero codes.  The cached weight is
+ * s_n * q[n][k].
+ *   q      device uint8 [rows][k], 16-byte aligned, written;
+ *   wscale device float [rows], 16-byte aligned, written. */
+int tq4_1s_to_fp8(const tq4_1s_weight* w, uint8_t* q, float* wscale, tq4_stream_t stream);
+
+/* Workspace bytes of tq4_1s_linear_fp8 (the bf16 weight of its large-m
+ * path); 0 on invalid arguments or m == 0. */
+size_t tq4_1s_linear_fp8_workspace(int64_t m, int64_t n, int64_t k);
+
+/* y[m][n] = bf16(x * (s q)^T) with the fp8 cache (q [n][k], wscale [n]) of
+ * tq4_1s_to_fp8; fp32 accumulation on the tensor cores.  For m <= 32 this is
+ * the decode-block kernel of tq4_1s_linear streaming 1 byte per weight (the
+ * E4M3 values convert to fp16 exactly; x is scaled per row by a power of two
+ * and rounded to fp16; no workspace is used and ws may be NULL); otherwise
+ * the cache is expanded to a bf16 weight in the workspace and multiplied by
+ * the tensor-core GEMM.  flags: TQ_WEIGHT_STATIC or 0, as for tq4_1s_weight.
+ * k % 32 == 0; m == 0 is a no-op. */
+int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, const float* wscale, int64_t n, int64_t k,
+                      int32_t flags, uint16_t* y, void* ws, size_t ws_bytes, tq4_stream_t stream);
+
 /* tq4_1s_linear for callers that cannot allocate device memory.  (The model
  * card has no counterpart: this is a deployment variant of the layer above.)
  * Plugin hosts and serving runtimes that fix every device allocation at

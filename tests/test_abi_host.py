@@ -115,6 +115,22 @@ def test_static_entry_validation_and_scratch_limits():
     assert tq.tq4_1s_error_string(9).startswith("shape exceeds the fixed scratch")
 
 
+def test_fp8_cache_validation():
+    lib = tq.load_library()
+    null = ctypes.c_void_p(0)
+    good = ctypes.c_void_p(4096)
+    assert lib.tq4_1s_to_fp8(ctypes.byref(_weight()), null, good, null) == 1
+    assert lib.tq4_1s_to_fp8(ctypes.byref(_weight()), ctypes.c_void_p(4104), good, null) == 2
+    assert lib.tq4_1s_to_fp8(ctypes.byref(_weight(k=48)), good, good, null) == 1
+    assert lib.tq4_1s_linear_fp8_workspace(16, 4096, 4096) == 4096 * 4096 * 2
+    assert lib.tq4_1s_linear_fp8_workspace(16, 4096, 4016) == 0            # k % 32 != 0
+    assert lib.tq4_1s_linear_fp8(good, 0, good, good, 64, 64, 0, good, null, 0, null) == 0   # m == 0
+    assert lib.tq4_1s_linear_fp8(good, 16, good, good, 64, 48, 0, good, null, 0, null) == 1
+    assert lib.tq4_1s_linear_fp8(good, 16, good, good, 64, 64, 2, good, null, 0, null) == 1  # unknown flag
+    assert lib.tq4_1s_linear_fp8(null, 16, good, good, 64, 64, 0, good, null, 0, null) == 1
+    assert lib.tq4_1s_linear_fp8(good, 16, ctypes.c_void_p(4097), good, 64, 64, 0, good, null, 0, null) == 2
+
+
 def test_debug_hooks_validation():
     lib = tq.load_library()
     assert lib.tq4_1s_debug_hook(99, 0) == 1                       # unknown hook
