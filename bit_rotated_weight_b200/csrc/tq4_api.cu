@@ -92,7 +92,7 @@ struct DeviceInfo {
   int sms = 0;
 };
 
-static int check_device(int* sms_out) {
+int check_device(int* sms_out) {
   static std::mutex mu;
   static DeviceInfo info[64];
   int dev = 0;
@@ -207,7 +207,7 @@ static bool cached_map(CUtensorMap* m, const MapKey& key, Encode encode) {
 }
 
 // Codes plane [E][n][k/2] bytes, box 64 B x 128 rows, 64-byte swizzle.
-static bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
+bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
   return cached_map(m, MapKey{0, w->codes, w->n, w->k, w->num_experts}, [&](CUtensorMap* out) {
     const uint64_t dims[3] = {static_cast<uint64_t>(w->k / 2), static_cast<uint64_t>(w->n),
                               static_cast<uint64_t>(w->num_experts)};
@@ -220,7 +220,7 @@ static bool map_codes(CUtensorMap* m, const tq4_1s_weight* w) {
 // x [rows][cols] (cols % 64 == 0) viewed as [cols/64][rows][64] 16-bit,
 // box 64 x 32 x 2*kFusedMaxIters, 128-byte swizzle: one copy fills the B
 // tiles of all stages of a fused CTA.
-static bool map_x3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
+bool map_x3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
   return cached_map(m, MapKey{1, base, rows, cols, 0}, [&](CUtensorMap* out) {
     const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / 64)};
     const uint64_t strides[2] = {static_cast<uint64_t>(cols * 2), 128};
@@ -231,7 +231,7 @@ static bool map_x3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols)
 
 // 16-bit matrix [rows][cols] row-major (bf16 or fp16), box 64 x box_rows,
 // 128-byte swizzle.
-static bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
+bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
   return cached_map(m, MapKey{2, base, rows, cols, box_rows}, [&](CUtensorMap* out) {
     const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
     const uint64_t strides[1] = {static_cast<uint64_t>(cols * 2)};

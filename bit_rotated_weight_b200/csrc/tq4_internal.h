@@ -25,6 +25,16 @@ bool withhold_arrival_hook();
 // Host-side codebook computation (Lloyd iteration), run once per process.
 const CodebookF32& codebook();
 
+// Host helpers of the entry points (tq4_api.cu): the current device's check
+// (compute capability 10.0; SM count cached per device) and cached TMA tensor
+// maps -- the codes plane [E][n][k/2] (box 64 B x 128 rows, 64-byte swizzle),
+// a 16-bit [rows][cols] matrix (box 64 x box_rows, 128-byte swizzle) and
+// the same viewed as [cols/64][rows][64] (box 64 x 32 x 2 kFusedMaxIters).
+int check_device(int* sms_out);
+bool map_codes(CUtensorMap* m, const tq4_1s_weight* w);
+bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows);
+bool map_x3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols);
+
 // One segment of rows of the rotated activations multiplied by one expert:
 // x = expert, y = first row, z = row count (<= 16 * nb_max <= kSegRows),
 // w unused.

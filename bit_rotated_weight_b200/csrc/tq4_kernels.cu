@@ -125,13 +125,14 @@ struct QuantBatch {
 // one block from the tile in registers and stores its 16 code bytes and two
 // scales (coalesced too).  Tile rows are one block each, their 16-byte
 // pieces XOR-swizzled so that neither the writes nor the per-lane row reads
-// conflict on banks.  The next chunk's loads are issued before the current
-// chunk is quantized.
+// conflict on banks.  The arithmetic per block is long (a correctly rounded
+// division per element), so latency is hidden by occupancy: few registers,
+// four CTAs per SM.
 template <typename T>
-__global__ void __launch_bounds__(256) quantize_kernel(const __grid_constant__ QuantBatch qb, CodebookF32 cb) {
+__global__ void __launch_bounds__(256, 4) quantize_kernel(const __grid_constant__ QuantBatch qb, CodebookF32 cb) {
   constexpr int kRowBytes = 32 * static_cast<int>(sizeof(T));   // one block: 128 B (fp32) or 64 B (bf16)
   constexpr int kPieces = kRowBytes / 16;                        // 16-byte pieces per block
-  constexpr int kLoads = 32 * kPieces / 32;                      // 16-byte loads per lane per chunk
+  constexpr int kLoads = kPieces;                                // 16-byte loads per lane per chunk
   __shared__ float s_t[16];
   __shared__ __align__(16) uint8_t tile[8][32 * kRowBytes];
   if (threadIdx.x < 16) s_t[threadIdx.x] = cb.thresholds[threadIdx.x];
@@ -145,39 +146,25 @@ __global__ void __launch_bounds__(256) quantize_kernel(const __grid_constant__ Q
   };
   const int64_t nwarps = static_cast<int64_t>(gridDim.x) * 8;
   int tix = 0;   // tensor of the current chunk (chunks are visited in increasing order)
-  auto locate = [&](int64_t ch, int& ti) {
-    while (ti + 1 < qb.count && ch >= qb.t[ti + 1].chunk0) ++ti;
-  };
-  uint4 buf[kLoads];
-  auto load_chunk = [&](int64_t ch, int ti) {
-    const QuantTensor& q = qb.t[ti];
+  for (int64_t ch = static_cast<int64_t>(blockIdx.x) * 8 + warp; ch < qb.nchunks; ch += nwarps) {
+    while (tix + 1 < qb.count && ch >= qb.t[tix + 1].chunk0) ++tix;
+    const QuantTensor& q = qb.t[tix];
     const int64_t b0 = (ch - q.chunk0) * 32;
-    const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(q.W) + b0 * 32);
+    {
+      const uint4* src = reinterpret_cast<const uint4*>(static_cast<const T*>(q.W) + b0 * 32);
+      uint4 buf[kLoads];
 #pragma unroll
-    for (int i = 0; i < kLoads; ++i) {
-      const int piece = lane + 32 * i;   // 16-byte piece of the chunk
-      const int b = piece / kPieces;
-      buf[i] = (b0 + b < q.nblocks) ? __ldg(src + piece) : make_uint4(0u, 0u, 0u, 0u);
-    }
-  };
-  int64_t ch = static_cast<int64_t>(blockIdx.x) * 8 + warp;
-  if (ch < qb.nchunks) {
-    locate(ch, tix);
-    load_chunk(ch, tix);
-  }
-  for (; ch < qb.nchunks; ch += nwarps) {
+      for (int i = 0; i < kLoads; ++i) {
+        const int piece = lane + 32 * i;   // 16-byte piece of the chunk
+        buf[i] = (b0 + piece / kPieces < q.nblocks) ? __ldg(src + piece) : make_uint4(0u, 0u, 0u, 0u);
+      }
 #pragma unroll
-    for (int i = 0; i < kLoads; ++i) {
-      const int piece = lane + 32 * i;
-      *reinterpret_cast<uint4*>(my + tpos(piece / kPieces, piece % kPieces)) = buf[i];
+      for (int i = 0; i < kLoads; ++i) {
+        const int piece = lane + 32 * i;
+        *reinterpret_cast<uint4*>(my + tpos(piece / kPieces, piece % kPieces)) = buf[i];
+      }
     }
     __syncwarp();
-    const int cur = tix;
-    const int64_t nxt = ch + nwarps;
-    if (nxt < qb.nchunks) {
-      locate(nxt, tix);
-      load_chunk(nxt, tix);
-    }
     float a[32];
     if constexpr (sizeof(T) == 4) {
 #pragma unroll
@@ -201,8 +188,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(const __grid_constant__ Q
       }
     }
     __syncwarp();   // the tile is rewritten with the next chunk after this
-    const QuantTensor& q = qb.t[cur];
-    const int64_t b = (ch - q.chunk0) * 32 + lane;
+    const int64_t b = b0 + lane;
     if (b < q.nblocks) {
       uint32_t words[4], dpair;
       quantize_block(a, q.mask, s_t, words, dpair);
@@ -666,7 +652,7 @@ cudaError_t launch_quantize_batch(const QuantItem* items, int count, int dtype, 
     qb.nchunks = chunks;
     if (chunks == 0) continue;
     int64_t blocks = (chunks + 7) / 8;
-    const int64_t cap = 148LL * 6;
+    const int64_t cap = 148LL * 4 * 4;
     if (blocks > cap) blocks = cap;
     if (dtype == TQ_DTYPE_F32)
       quantize_kernel<float><<<static_cast<int>(blocks), 256, 0, st>>>(qb, cb);

@@ -9,9 +9,12 @@
 // runs the same two kernels as tq4_1s_linear's small-m path (activation
 // rotation, then the stream-K dequant-GEMM) but keeps their scratch -- the
 // rotated activations and their row scales, the stream-K partial sums and the
-// tile counters -- in
-// one file-scope device array of fixed size, allocated once per GPU when the
-// library's module loads there and held until the process exits.
+// tile counters -- in one file-scope device array of fixed size.  The array is
+// reserved on a GPU when the library's device code is loaded there: with
+// CUDA's default lazy module loading that is the first call of the library
+// on that GPU that needs it (the first call of this entry point looks up the
+// array's address, which loads the module), after which it is held until the
+// process exits.
 #include <mutex>
 
 #include "tq4_internal.h"
@@ -77,18 +80,11 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   if (!x || !y) return TQ_ERR_INVALID_ARG;
   auto a16 = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
   if (!a16(x) || !a16(y) || !a16(w->codes) || !a16(w->scales)) return TQ_ERR_ALIGNMENT;
-  int dev = 0, major = 0, minor = 0, sms = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
-      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
-    cudaGetLastError();
-    return TQ_ERR_UNSUPPORTED_DEVICE;
-  }
-  if (major != 10 || minor != 0) return TQ_ERR_UNSUPPORTED_DEVICE;
-  void* scratch = nullptr;
-  int rc = scratch_address(&scratch);
+  int sms = 0;
+  int rc = check_device(&sms);
   if (rc) return rc;
+  void* scratch = nullptr;
+  if ((rc = scratch_address(&scratch))) return rc;
   if (take_injected_failure()) return TQ_ERR_CUDA;
 
   uint8_t* base = static_cast<uint8_t*>(scratch);
@@ -115,41 +111,13 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   const bool fused = split > 1 || (T + grid - 1) / grid <= kFusedMaxIters;
   if (!fused && launch_rotate_scaled(x, w->k, nullptr, 1, nullptr, m, m, xr, xscale, mask, st) != cudaSuccess)
     return TQ_ERR_CUDA;
-  alignas(64) CUtensorMap tc, tx;
-  {
-    // same tensor maps as tq4_1s_linear: codes [1][n][k/2] (64 B x 128 rows),
-    // x' (TMA-fed mode) or x (fused mode) [m][k] (64 x 16)
-    typedef CUresult (*EncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
-                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
-                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
-    static EncodeFn fn = nullptr;
-    static std::once_flag once;
-    std::call_once(once, [] {
-      void* p = nullptr;
-      cudaDriverEntryPointQueryResult q;
-      if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
-          q == cudaDriverEntryPointSuccess)
-        fn = reinterpret_cast<EncodeFn>(p);
-      else
-        cudaGetLastError();
-    });
-    if (!fn) return TQ_ERR_CUDA;
-    const cuuint32_t es[3] = {1, 1, 1};
-    const cuuint64_t cd[3] = {static_cast<cuuint64_t>(w->k / 2), static_cast<cuuint64_t>(w->n), 1};
-    const cuuint64_t cs[2] = {static_cast<cuuint64_t>(w->k / 2), static_cast<cuuint64_t>(w->n * (w->k / 2))};
-    const cuuint32_t cb[3] = {64, 128, 1};
-    const cuuint64_t xd[2] = {static_cast<cuuint64_t>(w->k), static_cast<cuuint64_t>(m)};
-    const cuuint64_t xs[1] = {static_cast<cuuint64_t>(w->k * 2)};
-    const cuuint32_t xb[2] = {64, 16};
-    if (fn(&tc, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, w->codes, cd, cs, cb, es, CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-            CUDA_SUCCESS ||
-        fn(&tx, CU_TENSOR_MAP_DATA_TYPE_UINT16, 2, fused ? const_cast<uint16_t*>(x) : xr, xd, xs, xb, es,
-           CU_TENSOR_MAP_INTERLEAVE_NONE,
-           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) !=
-            CUDA_SUCCESS)
-      return TQ_ERR_CUDA;
-  }
+  // the cached tensor maps of tq4_1s_linear: codes [1][n][k/2] (64 B x 128
+  // rows), x' (TMA-fed mode) or x (fused mode) [m][k] (64 x 16), and in the
+  // cluster split-K mode x as one 3-D box per CTA
+  alignas(64) CUtensorMap tc, tx, tx3;
+  if (!map_codes(&tc, w) || !map_bf16(&tx, fused ? static_cast<const void*>(x) : xr, m, w->k, 16)) return TQ_ERR_CUDA;
+  const bool box3 = split > 1 && (w->k % 64) == 0;
+  if (box3 && !map_x3(&tx3, x, m, w->k)) return TQ_ERR_CUDA;
   StreamKArgs a{};
   a.n = static_cast<int32_t>(w->n);
   a.k = static_cast<int32_t>(w->k);
@@ -166,10 +134,11 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   }
   a.epoch = next_epoch();
   a.cluster_s = split;
+  a.x_box3 = box3 ? 1 : 0;
   a.mode = EPI_DENSE;
   a.out_a = y;
   a.partials = partials;
   a.counters = counters;
   a.max_tiles = static_cast<int32_t>(tiles);
-  return launch_streamk(&tc, &tx, nullptr, a, grid, st) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
+  return launch_streamk(&tc, &tx, box3 ? &tx3 : nullptr, a, grid, st) == cudaSuccess ? TQ_OK : TQ_ERR_CUDA;
 }

@@ -214,8 +214,12 @@ int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, const floa
  * start-up and forbid new ones later cannot hand tq4_1s_linear a workspace;
  * this entry point takes only x, w and y and keeps its scratch (rotated
  * activations, stream-K partial sums, tile counters) in a fixed device array
- * inside the library: about 5.2 MiB, reserved on every GPU that loads the
- * library and held until the process exits.
+ * inside the library: about 5.2 MiB per GPU, reserved when the library's
+ * device code is loaded on that GPU -- under CUDA's default lazy module
+ * loading, at the first call there (this entry point's first call loads it)
+ * -- and held until the process exits.  A caller with a fixed memory budget
+ * makes one warm-up call at start-up, outside any stream capture, so that
+ * the reservation happens then.
  *   Limits: m <= 32, w->k <= 8192, w->n <= 32768, dense weight; larger
  *   shapes return TQ_ERR_SCRATCH_LIMIT and launch nothing.
  *   The first call on a device looks up the array's device address (with

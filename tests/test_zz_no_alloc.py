@@ -90,3 +90,81 @@ def test_static_scratch_other_modes(m, n, k, seed):
     ref_f = _bits(ref).astype(np.uint32) << 16
     assert_close(_bits(y), ref_f.view(np.float32).astype(np.float64), f"static m={m} n={n} k={k}")
     assert tq.tq4_1s_get_status() == 0
+
+
+def _static_fn():
+    lib = tq.load_library()
+    fn = lib.tq4_1s_linear_static
+    fn.argtypes = [ctypes.c_void_p, ctypes.c_int64, ctypes.POINTER(tq._Weight), ctypes.c_void_p, ctypes.c_void_p]
+    fn.restype = ctypes.c_int
+    return fn
+
+
+def test_static_scratch_takes_no_memory_and_replays_in_a_graph():
+    # After one warm-up call (which may load the library's device code and
+    # with it the fixed array), further calls change neither the device's
+    # free memory nor torch's allocations; a captured call replayed over
+    # changing inputs reproduces each input's eager result.
+    dev = torch.device("cuda:0")
+    fn = _static_fn()
+    n, k, m = 2048, 2048, 16
+    p = tq.tq4_1s_quantize(synth.normal_f32_device((n, k), 62, 0.02, dev), seed=62)
+    wst = p.c_struct()
+    xs = [_to_dev(synth.activations_bf16(m, k, 63 + i), dev) for i in range(3)]
+    y = torch.empty((m, n), dtype=torch.bfloat16, device=dev)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+    def call(x, st=stream):
+        assert fn(ctypes.c_void_p(x.data_ptr()), m, ctypes.byref(wst), ctypes.c_void_p(y.data_ptr()), st) == 0
+
+    call(xs[0])
+    torch.cuda.synchronize()
+    free0, alloc0 = torch.cuda.mem_get_info(dev)[0], torch.cuda.memory_allocated(dev)
+    refs = []
+    for x in xs:
+        call(x)
+        torch.cuda.synchronize()
+        refs.append(y.clone())
+    assert torch.cuda.mem_get_info(dev)[0] == free0 and torch.cuda.memory_allocated(dev) == alloc0
+    x_in = xs[0].clone()
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream(dev)
+    with torch.cuda.graph(g, stream=s):
+        call(x_in, ctypes.c_void_p(s.cuda_stream))
+    bad = 0
+    for r in range(9):
+        x_in.copy_(xs[r % 3])
+        y.zero_()
+        g.replay()
+        torch.cuda.synchronize()
+        bad += int(not torch.equal(y.view(torch.int16), refs[r % 3].view(torch.int16)))
+    del g
+    assert bad == 0
+    assert tq.tq4_1s_get_status() == 0
+
+
+def test_static_scratch_at_its_limits():
+    # m = 32, k = 8192, n = 32768 (the last tile counter): sampled output
+    # columns against the oracle, and guard rows around y left untouched
+    dev = torch.device("cuda:0")
+    fn = _static_fn()
+    m, n, k, seed = 32, 32768, 8192, 64
+    W = synth.normal_f32_device((n, k), seed, 0.02, dev)
+    p = tq.tq4_1s_quantize(W, seed=seed)
+    xh = synth.activations_bf16(m, k, seed + 1)
+    x = _to_dev(xh, dev)
+    guard = 0x5A5A
+    buf = torch.full((m + 2, n), guard, dtype=torch.int16, device=dev)
+    y = buf[1:m + 1].view(torch.bfloat16)
+    stream = ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+    wst = p.c_struct()
+    for _ in range(2):
+        assert fn(ctypes.c_void_p(x.data_ptr()), m, ctypes.byref(wst), ctypes.c_void_p(y.data_ptr()), stream) == 0
+    torch.cuda.synchronize()
+    assert tq.tq4_1s_get_status() == 0
+    assert bool((buf[0] == guard).all()) and bool((buf[m + 1] == guard).all())
+    rows = np.array(sorted(set([0, 1, 127, 128, n - 129, n - 1] + list(range(5, n, 997)))))
+    Ws = W[torch.from_numpy(rows).to(dev)].cpu().numpy()
+    codes, scales, _ = oracle.quantize(Ws, seed)
+    y_ref, _ = oracle.linear(xh, codes, scales, seed)
+    assert_close(_bits(y)[:, rows], y_ref, "static at its limits, sampled columns")
