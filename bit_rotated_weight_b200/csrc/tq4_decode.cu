@@ -16,28 +16,30 @@
 // their fp32 partial tiles through distributed shared memory in rank order
 // (deterministic).  What this kernel is built around is the chain of calls a
 // layer stack makes -- each call's input is the previous call's output --
-// where per-call latency, not bandwidth, is the limit:
-//   * a CTA is small enough (about 105 KB of shared memory, 256 tensor-memory
-//     columns, 512 threads at <= 64 registers) that two fit on an SM, and it
-//     lets the next kernel launch as soon as all its CTAs are running, so the
-//     next call's CTAs set up (barriers, level table, tensor memory) and --
-//     for a weight flagged static -- stream their weight tiles into shared
-//     memory while this call still computes;
-//   * only the activation-dependent work waits for the previous kernel: one
-//     warp per token loads its k range of x with coalesced 16-byte loads,
-//     rotates each lane's 32-slice in registers, takes the token's scale from
-//     a warp maximum and writes x' straight into the swizzled B tiles (no
-//     second pass, no shared-memory atomics);
-//   * dequantization, MMA issue and the epilogue run as separate roles.
+// where per-call latency, not bandwidth, is the limit, so it moves as much
+// work as it can in front of the wait for the previous kernel:
+//   * it lets the next kernel launch as soon as all its CTAs are running: the
+//     next call's CTAs take SMs as this call's CTAs leave (and the SMs this
+//     grid does not use) and do their own set-up meanwhile;
+//   * every codes tile of the CTA is requested at once (one shared-memory
+//     stage per iteration; no ring whose refills would queue behind other
+//     traffic), before the wait when the weight is flagged static;
+//   * the dequant warps then turn as many tiles as tensor memory holds (7 of
+//     8 at 16 tokens) into A operands before the wait;
+//   * only the activation-dependent work follows the wait: one warp per
+//     token loads its k range of x with coalesced 16-byte loads, rotates each
+//     lane's 32-slice in registers, takes the token's scale from a warp
+//     maximum and writes x' straight into the swizzled B tiles; the MMAs, the
+//     remaining tile and the epilogue.
 //
-// Warps (512 threads):
-//   0      lane 0: TMA producer of the codes tiles (4-stage ring);
+// Warps (512 threads, one CTA per SM):
+//   0      lane 0: TMA producer of the codes tiles;
 //   1-3    lane 0: MMA issuer of dequant group 0-2;
 //   0-3    epilogue (thread = tile row) once the MMAs are done;
 //   4-15   three dequant groups of four warps (thread = tile row): per
 //          iteration 16 B of codes + 8 scales -> 128 fp16 levels -> tensor
 //          memory, as two 64-k halves signalled separately;
-//   0-15   before their roles: the x rotation (warp = token).
+//   0-15   the x rotation (warp = token) after the wait.
 #include <mutex>
 
 #include "tq4_internal.h"
@@ -48,18 +50,20 @@ namespace {
 constexpr int kGroups = 3;                 // dequant groups
 constexpr int kFirstDqWarp = 4;
 constexpr int kThreads = (kFirstDqWarp + 4 * kGroups) * 32;   // 512
-constexpr int kStagesD = 4;                // codes ring
 constexpr int kMaxIters = kFusedMaxIters;  // iterations (128 k) per CTA
+constexpr int kStagesD = kMaxIters;        // one codes stage per iteration
 constexpr int kCodesTile = 128 * 64;       // codes of one iteration: 128 rows x 64 B
 constexpr int kLutBytesD = 256 * 32 * 4;   // fp16 level-pair table, one copy per lane
 constexpr int kAColsD = 64;                // tensor-memory columns of one A stage (128 k of fp16)
+constexpr int kTmemColsD = 512;
 constexpr float kLevelScaleD = 256.0f;
+// A stages: the tensor memory beside the accumulators (16 nb columns per group)
+__host__ __device__ constexpr int a_stages(int nb) { return (kTmemColsD - kGroups * 16 * nb) / kAColsD; }
 
 struct DecodeShared {
   uint64_t full[kStagesD];           // codes tile landed (TMA bytes)
-  uint64_t empty[kStagesD];          // the dequant group read the tile (4 warp arrivals)
-  uint64_t afull[kGroups][2];        // half A stage holds fresh levels (4 warp arrivals)
-  uint64_t afree[kGroups][2];        // the MMAs reading a half A stage completed
+  uint64_t afull[kMaxIters][2];      // A stage s, half h holds fresh levels (4 warp arrivals)
+  uint64_t afree[kMaxIters][2];      // the MMAs reading A stage s, half h completed
   uint64_t xready;                   // every token's x' is in the B tiles (16 warp arrivals)
   uint64_t dfull;                    // every issuer's MMAs completed (kGroups arrivals)
   uint64_t idone[kGroups];           // an issuer's own MMAs completed (teardown)
@@ -70,7 +74,7 @@ struct DecodeShared {
   int abort_flag;
 };
 
-// Dynamic shared memory: codes ring | B tiles [iters][2 halves][16 nb rows x 128 B] |
+// Dynamic shared memory: codes stages | B tiles [iters][2 halves][16 nb rows x 128 B] |
 // level table (TQ4_1S only) | cluster reduction buffer [split][rows per CTA][16 nb] fp32.
 // The fp8 cache (f8) streams 128 B of codes per row and iteration and needs no table.
 __host__ __device__ constexpr int tile_bytes(bool f8) { return f8 ? 2 * kCodesTile : kCodesTile; }
@@ -134,7 +138,7 @@ __device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, 
 // the E4M3 values converted to fp16 (exact), and the row scale multiplies the
 // accumulator in the epilogue.
 template <int NB, bool F8>
-__global__ void __launch_bounds__(kThreads, 2)
+__global__ void __launch_bounds__(kThreads, 1)
     decode_kernel(const __grid_constant__ CUtensorMap tm_codes, const DecodeArgs a,
                   const __grid_constant__ LevelTableD lt) {
   __shared__ DecodeShared sh;
@@ -147,6 +151,7 @@ __global__ void __launch_bounds__(kThreads, 2)
   constexpr int kHalf = b_half_bytes(NB);
   constexpr int kAccW = 16 * NB;          // accumulator columns per group
   constexpr int kACol0 = kGroups * kAccW; // first A-stage column
+  constexpr int kNA = a_stages(NB);       // A stages (7 at NB == 1, 6 at NB == 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = a.split;
@@ -159,14 +164,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   const bool stat = a.static_w != 0;
 
   if (warp == 0) {
-    for (int i = lane; i < 2 * kStagesD + 5 * kGroups + 3; i += 32) {
+    constexpr int kBars = kStagesD + 4 * kMaxIters + 2 + kGroups + 1;
+    for (int i = lane; i < kBars; i += 32) {
       if (i < kStagesD) mbar_init(&sh.full[i], 1);
-      else if (i < 2 * kStagesD) mbar_init(&sh.empty[i - kStagesD], 4);
-      else if (i < 2 * kStagesD + 2 * kGroups) mbar_init(&sh.afull[(i - 2 * kStagesD) >> 1][i & 1], 4);
-      else if (i < 2 * kStagesD + 4 * kGroups) mbar_init(&sh.afree[(i - 2 * kStagesD - 2 * kGroups) >> 1][i & 1], 1);
-      else if (i == 2 * kStagesD + 4 * kGroups) mbar_init(&sh.xready, kThreads / 32);
-      else if (i == 2 * kStagesD + 4 * kGroups + 1) mbar_init(&sh.dfull, kGroups);
-      else if (i < 2 * kStagesD + 5 * kGroups + 2) mbar_init(&sh.idone[i - 2 * kStagesD - 4 * kGroups - 2], 1);
+      else if (i < kStagesD + 2 * kMaxIters) mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4);
+      else if (i < kStagesD + 4 * kMaxIters)
+        mbar_init(&sh.afree[(i - kStagesD - 2 * kMaxIters) >> 1][(i - kStagesD) & 1], 1);
+      else if (i == kStagesD + 4 * kMaxIters) mbar_init(&sh.xready, kThreads / 32);
+      else if (i == kStagesD + 4 * kMaxIters + 1) mbar_init(&sh.dfull, kGroups);
+      else if (i < kStagesD + 4 * kMaxIters + 2 + kGroups) mbar_init(&sh.idone[i - kStagesD - 4 * kMaxIters - 2], 1);
       else mbar_init(&sh.eready, 4 * kGroups);
     }
     if (lane == 0) {
@@ -175,7 +181,7 @@ __global__ void __launch_bounds__(kThreads, 2)
     }
     fence_mbar_init();
   } else if (warp == 1) {
-    tmem_alloc(&sh.tmem_base, NB == 1 ? 256 : 512);
+    tmem_alloc(&sh.tmem_base, kTmemColsD);
     tmem_relinquish();
   }
   if (!F8) {
@@ -191,28 +197,32 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   // All CTAs of this grid are resident once every one of them is here: the
-  // next kernel may launch now.  Its CTAs take free SM slots (two CTAs of this
-  // kernel fit on an SM) and do their own set-up meanwhile; anything of theirs
-  // that reads this kernel's output waits in griddepcontrol.wait.
+  // next kernel may launch now.  Its CTAs take the SMs this grid leaves free
+  // and those its CTAs release, and set up meanwhile; anything of theirs that
+  // reads this kernel's output waits in griddepcontrol.wait.
   if (threadIdx.x == 0) pdl_launch_dependents();
   const uint32_t tmem = sh.tmem_base;
   volatile int* abortp = &sh.abort_flag;
 
   // A weight flagged static is not written by any kernel still in flight,
-  // so its tiles may be read before the wait; otherwise the previous kernel
-  // may have written it (a quantize) and everything waits.
+  // so its tiles and scales may be read before the wait; otherwise the
+  // previous kernel may have written it (a quantize) and they are read after
+  // it, with L2 prefetches issued now (a prefetch is only a hint and L2 is
+  // the device's point of coherence, so it is safe either way).
   auto issue_codes = [&](int li) {
-    const int s = li % kStagesD;
-    mbar_arrive_expect_tx(&sh.full[s], kTile);
-    tma_load_3d(smem + s * kTile, &tm_codes, &sh.full[s], (it0 + li) * (F8 ? 128 : 64), row0, 0);
+    mbar_arrive_expect_tx(&sh.full[li], kTile);
+    tma_load_3d(smem + li * kTile, &tm_codes, &sh.full[li], (it0 + li) * (F8 ? 128 : 64), row0, 0);
   };
-  const int npre = cnt < kStagesD ? cnt : kStagesD;
-  if (stat && warp == 0 && lane == 0)
-    for (int li = 0; li < npre; ++li) issue_codes(li);
+  if (warp == 0 && lane == 0) {
+    for (int li = 0; li < cnt; ++li) {
+      if (stat) issue_codes(li);
+      else tma_prefetch_l2_3d(&tm_codes, (it0 + li) * (F8 ? 128 : 64), row0, 0);
+    }
+  }
 
-  // dequant threads: the scales of their (up to 3) iterations, 16 B each
   const int dq_group = (warp >= kFirstDqWarp) ? (warp - kFirstDqWarp) >> 2 : -1;
   const int trow = (warp & 3) * 32 + lane;   // tile row of this thread (dequant and epilogue)
+  // dequant threads: the scales of their (up to 3) iterations, 16 B each
   uint32_t sraw[3][4];
   auto load_scales = [&]() {
     const int row = row0 + trow;
@@ -238,11 +248,119 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   };
-  if (stat && dq_group >= 0) load_scales();
+
+  // ------------------------------------------------------------ dequant
+  // Group g dequantizes iterations g, g + 3, g + 6 of the CTA into A stage
+  // li % kNA; an iteration past the first kNA reuses a stage once the MMAs of
+  // the iteration kNA before it have read it.  Before the wait (static
+  // weight) a group does the iterations that need no stage back; the rest
+  // after the rotation.
+  uint32_t ff = 0u;   // {2^-e, 2^-e}: this thread's row exponent (see below)
+  int dq_done = 0;    // iterations of this group dequantized so far
+  auto dq_exponent = [&]() {
+    // Row exponent of this group's levels: the scales of the group's
+    // iterations are multiplied by 2^-e (exact) so that the largest lies in
+    // [32, 64) -- levels fp16(256 c) * d 2^-e then stay normal and finite for
+    // every finite fp16 scale -- and the epilogue multiplies the group's
+    // accumulator by 2^e (exact).
+    uint32_t dmax = 0u;
+#pragma unroll
+    for (int u = 0; u < 3; ++u)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) asm("max.f16x2 %0, %1, %2;" : "=r"(dmax) : "r"(dmax), "r"(sraw[u][j]));
+    const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
+    const float mx = fmaxf(dm.x, dm.y);
+    int e = 0;
+    if (mx > 0.0f && isfinite(mx)) {
+      int ex;
+      frexpf(mx, &ex);   // mx in [2^(ex-1), 2^ex)
+      e = ex - 6;
+      e = e < -15 ? -15 : (e > 14 ? 14 : e);
+    }
+    sh.rexp[dq_group][trow] = static_cast<int8_t>(e);
+    const __half2 f2 = __float2half2_rn(ldexpf(1.0f, -e));   // a power of two, normal in fp16
+    ff = *reinterpret_cast<const uint32_t*>(&f2);
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sh.eready);
+  };
+  // Dequantize this group's iterations up to (excluding) `li_end`; false on abort.
+  auto dq_run = [&](int li_end) -> bool {
+    const int g = dq_group;
+    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t lut_lane = smem_u32(lut) + 4u * static_cast<uint32_t>(lane);
+    for (;;) {
+      const int li = g + kGroups * dq_done;
+      if (li >= li_end || li >= cnt) return true;
+      const int sa = li % kNA;
+      const uint32_t a_stage = tmem + kACol0 + sa * kAColsD;
+      if (!wwait(&sh.full[li], 0, abortp)) return false;
+      const uint8_t* cb = smem + li * kTile + trow * (F8 ? 128 : 64);
+      uint32_t sr[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        sr[j] = (dq_done == 0) ? sraw[0][j] : (dq_done == 1 ? sraw[1][j] : sraw[2][j]);
+        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(sr[j]) : "r"(sr[j]), "r"(ff));
+      }
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        if (li >= kNA && !wwait(&sh.afree[sa][h], ((li / kNA) - 1) & 1, abortp)) return false;
+        tc_fence_after();
+#pragma unroll
+        for (int kb2 = 0; kb2 < 2; ++kb2) {
+          const int kb = 2 * h + kb2;
+          uint32_t o[16];
+          if (F8) {
+            // fp8 cache: 128 B of E4M3 codes per row (128-byte swizzle: 16-byte
+            // chunk c of row t at chunk c ^ (t & 7)); each byte pair converts to
+            // an fp16 pair exactly
+#pragma unroll
+            for (int ch = 0; ch < 2; ++ch) {
+              const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * ((2 * kb + ch) ^ (trow & 7)));
+              const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
+#pragma unroll
+              for (int j = 0; j < 4; ++j)
+                asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
+                    "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
+                    : "=r"(o[8 * ch + 2 * j]), "=r"(o[8 * ch + 2 * j + 1])
+                    : "r"(cw[j]));
+            }
+          } else {
+            // TQ4_1S: 16 B of codes (64-byte swizzle: chunk kb of row t at
+            // kb ^ ((t >> 1) & 3)), each byte a pair of codes looked up in the
+            // lane's table, times the pair of scaled half-block scales
+            const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((trow >> 1) & 3)));
+            dq_half(c.x, c.y, prmt(sr[kb], 0u, 0x1010u), lut_lane, o);
+            dq_half(c.z, c.w, prmt(sr[kb], 0u, 0x3232u), lut_lane, o + 8);
+          }
+          tmem_st16(a_stage + lane_base + 16 * kb, o);
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.afull[sa][h]);
+      }
+      ++dq_done;
+    }
+  };
+  bool dq_ok = true;
+  if (stat && dq_group >= 0) {
+    load_scales();
+    dq_exponent();
+    dq_ok = dq_run(kNA);
+  }
+
+  if (!stat && dq_group >= 0 && !F8 && row0 + trow < a.n) {
+    // the scales this thread will load after the wait, pulled into L2 now
+    const uint16_t* sp0 = a.scales + static_cast<int64_t>(row0 + trow) * (a.k / 16);
+    for (int u = 0; u < 3; ++u) {
+      const int li = dq_group + kGroups * u;
+      if (li < cnt) asm volatile("prefetch.global.L2 [%0];" ::"l"(sp0 + (it0 + li) * 8));
+    }
+  }
 
   pdl_wait();
   if (!stat && warp == 0 && lane == 0)
-    for (int li = 0; li < npre; ++li) issue_codes(li);
+    for (int li = 0; li < cnt; ++li) issue_codes(li);
   if (!stat && dq_group >= 0) load_scales();
 
   // ------------------------------------------------------------ x rotation
@@ -327,171 +445,50 @@ __global__ void __launch_bounds__(kThreads, 2)
   }
 
   if (dq_group >= 0) {
-    // ------------------------------------------------------------ dequant
-    const int g = dq_group;
-    const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t a_stage = tmem + kACol0 + g * kAColsD;
-    const uint32_t lut_lane = smem_u32(lut) + 4u * static_cast<uint32_t>(lane);
-    // Row exponent of this group's levels: the scales of the group's
-    // iterations are multiplied by 2^-e (exact) so that the largest lies in
-    // [32, 64) -- levels fp16(256 c) * d 2^-e then stay normal and finite for
-    // every finite fp16 scale -- and the epilogue multiplies the group's
-    // accumulator by 2^e (exact).
-    uint32_t ff;
-    {
-      uint32_t dmax = 0u;
-#pragma unroll
-      for (int u = 0; u < 3; ++u)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) asm("max.f16x2 %0, %1, %2;" : "=r"(dmax) : "r"(dmax), "r"(sraw[u][j]));
-      const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
-      const float mx = fmaxf(dm.x, dm.y);
-      int e = 0;
-      if (mx > 0.0f && isfinite(mx)) {
-        int ex;
-        frexpf(mx, &ex);   // mx in [2^(ex-1), 2^ex)
-        e = ex - 6;
-        e = e < -15 ? -15 : (e > 14 ? 14 : e);
-      }
-      sh.rexp[g][trow] = static_cast<int8_t>(e);
-      const __half2 f2 = __float2half2_rn(ldexpf(1.0f, -e));   // a power of two, normal in fp16
-      ff = *reinterpret_cast<const uint32_t*>(&f2);
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.eready);
-    }
+    if (!stat) dq_exponent();
+    if (dq_ok) dq_run(kMaxIters);
+  } else if (warp == 0 && lane == 0) {
+    // ------------------------------------------------------------ producer
+    // (every tile was issued above; on an abort, let them land before exit)
+    if (*abortp)
+      for (int li = 0; li < cnt; ++li) drain(&sh.full[li], 0);
+  } else if (warp >= 1 && warp <= kGroups && lane == 0) {
+    // ------------------------------------------------------------ MMA issue
+    const int g = warp - 1;
+    const uint32_t acc = tmem + g * kAccW;
+    const uint32_t idesc = idesc_f16(128, 16 * NB);
+    bool ok = mbar_wait(&sh.xready, 0, abortp);
     int use = 0;
-#pragma unroll 1
-    for (int li = g; F8 && li < cnt; li += kGroups, ++use) {
-      // fp8 cache: 128 B of E4M3 codes per row (128-byte swizzle: 16-byte
-      // chunk c of row t at chunk c ^ (t & 7)); each byte pair converts to an
-      // fp16 pair exactly
-      const int s = li % kStagesD;
-      if (!wwait(&sh.full[s], (li / kStagesD) & 1, abortp)) break;
-      const uint8_t* cb = smem + s * kTile + trow * 128;
-      bool ok = true;
-#pragma unroll
+    for (int li = g; ok && li < cnt; li += kGroups, ++use) {
+      const int sa = li % kNA;
+      const uint32_t a_stage = tmem + kACol0 + sa * kAColsD;
       for (int h = 0; h < 2; ++h) {
-        if (use > 0 && !wwait(&sh.afree[g][h], (use - 1) & 1, abortp)) {
+        if (!mbar_wait(&sh.afull[sa][h], (li / kNA) & 1, abortp)) {
           ok = false;
           break;
         }
         tc_fence_after();
+        const uint64_t bdesc = sdesc_k128(smem_u32(btiles + (li * 2 + h) * kHalf));
 #pragma unroll
-        for (int kb2 = 0; kb2 < 2; ++kb2) {
-          const int kb = 2 * h + kb2;
-          uint32_t o[16];
-#pragma unroll
-          for (int ch = 0; ch < 2; ++ch) {
-            const uint4 c = *reinterpret_cast<const uint4*>(cb + 16 * ((2 * kb + ch) ^ (trow & 7)));
-            const uint32_t cw[4] = {c.x, c.y, c.z, c.w};
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              asm("{\n\t.reg .b16 lo, hi;\n\tmov.b32 {lo, hi}, %2;\n\t"
-                  "cvt.rn.f16x2.e4m3x2 %0, lo;\n\tcvt.rn.f16x2.e4m3x2 %1, hi;\n\t}"
-                  : "=r"(o[8 * ch + 2 * j]), "=r"(o[8 * ch + 2 * j + 1])
-                  : "r"(cw[j]));
-          }
-          tmem_st16(a_stage + lane_base + 16 * kb, o);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.afull[g][h]);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
+                 (use == 0 && h == 0 && kk == 0) ? 0u : 1u);
+        mma_commit(&sh.afree[sa][h]);
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.empty[s]);   // the stage was read in full
-      if (!ok) break;
     }
-#pragma unroll 1
-    for (int li = g; !F8 && li < cnt; li += kGroups, ++use) {
-      const int s = li % kStagesD;
-      if (!wwait(&sh.full[s], (li / kStagesD) & 1, abortp)) break;
-      const uint8_t* cb = smem + s * kTile + trow * 64;
-      uint4 c[4];
-#pragma unroll
-      for (int kb = 0; kb < 4; ++kb) c[kb] = *reinterpret_cast<const uint4*>(cb + 16 * (kb ^ ((trow >> 1) & 3)));
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.empty[s]);   // the producer may refill the stage
-      uint32_t sr[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        sr[j] = (use == 0) ? sraw[0][j] : (use == 1 ? sraw[1][j] : sraw[2][j]);
-        asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(sr[j]) : "r"(sr[j]), "r"(ff));
-      }
-      bool ok = true;
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {
-        if (use > 0 && !wwait(&sh.afree[g][h], (use - 1) & 1, abortp)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-#pragma unroll
-        for (int kb2 = 0; kb2 < 2; ++kb2) {
-          const int kb = 2 * h + kb2;
-          uint32_t o[16];
-          dq_half(c[kb].x, c[kb].y, prmt(sr[kb], 0u, 0x1010u), lut_lane, o);
-          dq_half(c[kb].z, c[kb].w, prmt(sr[kb], 0u, 0x3232u), lut_lane, o + 8);
-          tmem_st16(a_stage + lane_base + 16 * kb, o);
-        }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&sh.afull[g][h]);
-      }
-      if (!ok) break;
-    }
-  } else {
-    if (warp == 0 && lane == 0) {
-      // ------------------------------------------------------------ producer
-      int armed = -1;   // last iteration whose copy was issued
-      armed = npre - 1;
-#pragma unroll 1
-      for (int li = npre; li < cnt; ++li) {
-        const int s = li % kStagesD;
-        if (!mbar_wait(&sh.empty[s], ((li / kStagesD) - 1) & 1, abortp)) break;
-        issue_codes(li);
-        armed = li;
-      }
-      if (*abortp) {
-        // wind down: every issued copy lands before the CTA exits
-        for (int li = (armed - kStagesD + 1 > 0 ? armed - kStagesD + 1 : 0); li <= armed; ++li)
-          drain(&sh.full[li % kStagesD], (li / kStagesD) & 1);
-      }
-    } else if (warp >= 1 && lane == 0) {
-      // ------------------------------------------------------------ MMA issue
-      const int g = warp - 1;
-      const uint32_t acc = tmem + g * kAccW;
-      const uint32_t a_stage = tmem + kACol0 + g * kAColsD;
-      const uint32_t idesc = idesc_f16(128, 16 * NB);
-      bool ok = mbar_wait(&sh.xready, 0, abortp);
-      int use = 0;
-      for (int li = g; ok && li < cnt; li += kGroups, ++use) {
-        for (int h = 0; h < 2; ++h) {
-          if (!mbar_wait(&sh.afull[g][h], use & 1, abortp)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint64_t bdesc = sdesc_k128(smem_u32(btiles + (li * 2 + h) * kHalf));
-#pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
-                   (use == 0 && h == 0 && kk == 0) ? 0u : 1u);
-          mma_commit(&sh.afree[g][h]);
-        }
-      }
-      if (use > 0) mma_commit(&sh.dfull);
-      else mbar_arrive(&sh.dfull);
-      // its MMAs complete before the CTA can release tensor memory
-      mma_commit(&sh.idone[g]);
-      drain(&sh.idone[g], 0);
-    }
+    if (use > 0) mma_commit(&sh.dfull);
+    else mbar_arrive(&sh.dfull);
+    // its MMAs complete before the CTA can release tensor memory
+    mma_commit(&sh.idone[g]);
+    drain(&sh.idone[g], 0);
+  }
+  if (warp < 4) {
     __syncwarp();
     // ------------------------------------------------------------ epilogue
     // thread = tile row trow; the groups' accumulators summed in group order,
-    // scaled back by 2^e / 256 per token (exact)
-    // (xready also orders the token scales written by the rotation warps)
+    // each scaled back by its row exponent, then by the token's 2^e and the
+    // level factor (TQ4_1S) or the row's scale (fp8 cache) -- all exact but
+    // the last.  (xready also orders the token scales the rotation wrote.)
     int ok = 0;
     if (lane == 0)
       ok = (mbar_wait(&sh.xready, 0, abortp) && mbar_wait(&sh.eready, 0, abortp) && mbar_wait(&sh.dfull, 0, abortp))
@@ -501,7 +498,6 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_after();
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int ngroups = cnt < kGroups ? cnt : kGroups;
-    // TQ4_1S: levels carry a factor 256; fp8 cache: the row's scale
     const float wsc = F8 ? ((row0 + trow < a.n) ? __ldcg(a.wscale + row0 + trow) : 0.0f) : 1.0f / kLevelScaleD;
     if (ok) {
 #pragma unroll
@@ -565,7 +561,7 @@ __global__ void __launch_bounds__(kThreads, 2)
       }
     }
   }
-  if (warp == 1) tmem_dealloc(tmem, NB == 1 ? 256 : 512);
+  if (warp == 1) tmem_dealloc(tmem, kTmemColsD);
 }
 
 template <int NB, bool F8>

@@ -2,10 +2,13 @@
 on the CPU.
 
 The kernel's roles synchronise only through mbarriers (plus one CTA barrier
-and one cluster barrier that every thread reaches): the TMA producer and the
-codes ring (full/empty), four-warp dequant groups filling half A stages
-(afull) that their MMA issuer frees (afree, by tcgen05.commit), the rotation
-warps' xready, the dequant warps' eready, the issuers' dfull and idone.  This model runs the roles as
+and one cluster barrier that every thread reaches): the TMA producer's codes
+tiles (full, one stage per iteration), four-warp dequant groups filling half
+A stages (afull) -- iterations past the tensor memory's stage count reuse a
+stage once the MMAs reading it complete (afree, by tcgen05.commit) -- the
+rotation warps' xready, the dequant warps' eready, the issuers' dfull and
+idone.  Static weights are dequantized in part before the wait for the
+previous kernel.  This model runs the roles as
 actors in random interleavings, with TMA landings and MMA completions as
 asynchronous events, for every k-range length a CTA can have (1..8
 iterations), and checks that:
@@ -33,19 +36,26 @@ def _const(name):
 
 
 GROUPS = _const("kGroups")
-STAGES = _const("kStagesD")
 FIRST_DQ = _const("kFirstDqWarp")
 WARPS = FIRST_DQ + 4 * GROUPS
+MAX_ITERS = 8                                    # kFusedMaxIters
+TMEM_COLS = _const("kTmemColsD")
+
+
+def a_stages(nb):
+    # as a_stages() in the kernel: tensor memory beside the accumulators
+    return (TMEM_COLS - GROUPS * 16 * nb) // 64
 
 
 def test_source_constants_and_counts():
-    # the init counts the model assumes, as written in the kernel
-    assert (GROUPS, STAGES, FIRST_DQ) == (3, 4, 4)
-    assert "mbar_init(&sh.empty[i - kStagesD], 4)" in SRC           # one arrival per dequant warp
-    assert "mbar_init(&sh.afull[(i - 2 * kStagesD) >> 1][i & 1], 4)" in SRC
+    # the init counts and layout the model assumes, as written in the kernel
+    assert (GROUPS, FIRST_DQ, TMEM_COLS) == (3, 4, 512)
+    assert "constexpr int kStagesD = kMaxIters;" in SRC              # one codes stage per iteration
+    assert "mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4)" in SRC   # one arrival per warp
     assert "mbar_init(&sh.xready, kThreads / 32)" in SRC             # one arrival per warp
     assert "mbar_init(&sh.dfull, kGroups)" in SRC
     assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
+    assert (a_stages(1), a_stages(2)) == (7, 6)
 
 
 class Barrier:
@@ -69,23 +79,24 @@ class Timeout(Exception):
     pass
 
 
-def run(cnt, seed, withhold_xready=False):
+def run(cnt, seed, withhold_xready=False, static=True, nb=1):
     rng = random.Random(seed)
+    na = a_stages(nb)
     B = {}
 
     def bar(name, count):
         B[name] = Barrier(name, count)
         return B[name]
 
-    full = [bar(f"full{s}", 1) for s in range(STAGES)]
-    empty = [bar(f"empty{s}", 4) for s in range(STAGES)]
-    afull = [[bar(f"afull{g}{h}", 4) for h in range(2)] for g in range(GROUPS)]
-    afree = [[bar(f"afree{g}{h}", 1) for h in range(2)] for g in range(GROUPS)]
+    full = [bar(f"full{s}", 1) for s in range(MAX_ITERS)]
+    afull = [[bar(f"afull{s}{h}", 4) for h in range(2)] for s in range(MAX_ITERS)]
+    afree = [[bar(f"afree{s}{h}", 1) for h in range(2)] for s in range(MAX_ITERS)]
     xready = bar("xready", WARPS)
     dfull = bar("dfull", GROUPS)
     idone = [bar(f"idone{g}", 1) for g in range(GROUPS)]
     eready = bar("eready", 4 * GROUPS)
-    state = {"abort": False, "landings": [], "mma": [], "issued": 0, "landed": 0, "mma_issued": 0, "mma_done": 0}
+    state = {"abort": False, "landings": [], "mma": [], "issued": 0, "landed": 0, "mma_issued": 0,
+             "waited": False}
 
     def wait(b, p, bounded=True):
         # a bounded wait: yields until the phase completed; after an abort it
@@ -101,52 +112,49 @@ def run(cnt, seed, withhold_xready=False):
                 return False
         return True
 
-    def issue(li):
-        state["issued"] += 1
-        state["landings"].append(full[li % STAGES])
-
-    def producer():
-        # warp 0, lane 0: the first copies, the warp's rotation, then the ring
-        npre = min(cnt, STAGES)
-        for li in range(npre):
-            issue(li)
-        yield from rotation(0)
-        armed = npre - 1
-        for li in range(npre, cnt):
-            ok = yield from wait(empty[li % STAGES], li // STAGES - 1)
-            if not ok:
-                break
-            issue(li)
-            armed = li
-        if state["abort"]:
-            for li in range(max(armed - STAGES + 1, 0), armed + 1):
-                yield from wait(full[li % STAGES], li // STAGES, bounded=False)
+    def issue_all():
+        for li in range(cnt):
+            state["issued"] += 1
+            state["landings"].append(full[li])
 
     def rotation(w):
         yield ("step", "rotate")
         if not (withhold_xready and w == 7):
             xready.arrive()
 
-    def dequant(g, q):
-        yield from rotation(FIRST_DQ + 4 * g + q)
-        yield ("step", "row exponent")
-        eready.arrive()
-        use = 0
-        for li in range(g, cnt, GROUPS):
-            ok = yield from wait(full[li % STAGES], li // STAGES)
+    def dq_run(g, done, li_end):
+        # dequantize this group's iterations g + 3 done, ... below li_end
+        while True:
+            li = g + GROUPS * done[0]
+            if li >= li_end or li >= cnt:
+                return True
+            sa = li % na
+            ok = yield from wait(full[li], 0)
             if not ok:
-                break
-            empty[li % STAGES].arrive()
+                return False
             for h in range(2):
-                if use > 0:
-                    ok = yield from wait(afree[g][h], use - 1)
+                if li >= na:
+                    ok = yield from wait(afree[sa][h], li // na - 1)
                     if not ok:
-                        break
+                        return False
                 yield ("step", "dequant")
-                afull[g][h].arrive()
-            if not ok:
-                break
-            use += 1
+                afull[sa][h].arrive()
+            done[0] += 1
+
+    def dequant(g, q):
+        done = [0]
+        ok = True
+        if static:
+            yield ("step", "row exponent")
+            eready.arrive()
+            ok = yield from dq_run(g, done, na)      # before the wait: stages not reused
+        yield ("step", "wait for the previous kernel")
+        yield from rotation(FIRST_DQ + 4 * g + q)
+        if not static:
+            yield ("step", "row exponent")
+            eready.arrive()
+        if ok:
+            yield from dq_run(g, done, MAX_ITERS)
 
     def issuer(g):
         yield from rotation(1 + g)
@@ -155,12 +163,13 @@ def run(cnt, seed, withhold_xready=False):
         for li in range(g, cnt, GROUPS):
             if not ok:
                 break
+            sa = li % na
             for h in range(2):
-                ok = yield from wait(afull[g][h], use)
+                ok = yield from wait(afull[sa][h], li // na)
                 if not ok:
                     break
                 state["mma_issued"] += 1
-                state["mma"].append(afree[g][h])      # commit: arrives when the MMAs complete
+                state["mma"].append(afree[sa][h])      # commit: arrives when the MMAs complete
             if not ok:
                 break
             use += 1
@@ -170,6 +179,18 @@ def run(cnt, seed, withhold_xready=False):
             dfull.arrive()
         state["mma"].append(idone[g])
         yield from wait(idone[g], 0, bounded=False)
+
+    def producer():
+        # warp 0, lane 0: every tile at once (before the wait when static)
+        if static:
+            issue_all()
+        yield ("step", "wait for the previous kernel")
+        if not static:
+            issue_all()
+        yield from rotation(0)
+        if state["abort"]:
+            for li in range(cnt):
+                yield from wait(full[li], 0, bounded=False)
 
     def epilogue(w):
         if w == 0:
@@ -181,7 +202,7 @@ def run(cnt, seed, withhold_xready=False):
     actors = [epilogue(0)]
     actors += [issuer(g) for g in range(GROUPS)]
     actors += [dequant(g, q) for g in range(GROUPS) for q in range(4)]
-    # the issuers' warps and warps 1-3 join the epilogue after their roles
+    # the issuers' warps 1-3 join the epilogue after their roles
     actors += [epilogue(w) for w in range(1, 4)]
     live = list(actors)
     pending = {id(a): None for a in live}
@@ -209,7 +230,6 @@ def run(cnt, seed, withhold_xready=False):
         if pick == "mma":
             # MMAs of one CTA complete in issue order
             state["mma"].pop(0).arrive()
-            state["mma_done"] += 1
             continue
         a = pick
         tag = pending[id(a)]
@@ -223,7 +243,6 @@ def run(cnt, seed, withhold_xready=False):
                 return B[t[1]].phase > t[2] or (t[3] and state["abort"])
             progress_possible = bool(events) or any(can_move(o) for o in live)
             if not progress_possible:
-                # nothing can move: the bounded wait of this actor runs out
                 try:
                     pending[id(a)] = a.throw(Timeout())
                 except StopIteration:
@@ -237,23 +256,27 @@ def run(cnt, seed, withhold_xready=False):
 
 
 @pytest.mark.parametrize("cnt", range(1, 9))
-def test_protocol_completes_with_exact_counts(cnt):
-    for seed in range(40):
-        B, state = run(cnt, seed)
+@pytest.mark.parametrize("static,nb", [(True, 1), (False, 1), (True, 2)])
+def test_protocol_completes_with_exact_counts(cnt, static, nb):
+    for seed in range(30):
+        B, state = run(cnt, seed, static=static, nb=nb)
         assert not state["abort"], f"cnt={cnt} seed={seed}: a wait ran out in a correct run"
         assert state["landed"] == state["issued"] == cnt
         assert not state["mma"] and state["mma_issued"] == 2 * cnt
         for b in B.values():
             assert b.arrived == 0, f"{b.name}: partial phase left at the end"
         assert B["xready"].phase == 1 and B["dfull"].phase == 1 and B["eready"].phase == 1
-        for s in range(STAGES):
-            assert B[f"full{s}"].phase == len(range(s, cnt, STAGES))
+        na = a_stages(nb)
+        for s in range(MAX_ITERS):
+            uses = len(range(s, cnt, na)) if s < na else 0
+            assert B[f"afull{s}0"].phase == uses and B[f"afree{s}1"].phase == uses
 
 
-@pytest.mark.parametrize("cnt", [1, 3, 4, 8])
-def test_withheld_arrival_winds_down(cnt):
-    for seed in range(40):
-        B, state = run(cnt, seed, withhold_xready=True)
+@pytest.mark.parametrize("cnt", [1, 3, 7, 8])
+@pytest.mark.parametrize("static", [True, False])
+def test_withheld_arrival_winds_down(cnt, static):
+    for seed in range(30):
+        B, state = run(cnt, seed, withhold_xready=True, static=static)
         assert state["abort"], "the withheld arrival must make a wait run out"
         assert state["landed"] == state["issued"], "a TMA copy still in flight at exit"
         assert not state["mma"], "an MMA still in flight when tensor memory is released"
