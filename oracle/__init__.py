@@ -20,6 +20,10 @@ listed at the top of the C file.  Parity status of each function:
   published values (largest finite 448, smallest subnormal 2^-9), round
   trips of every code, ties to even, torch's float8_e4m3fn conversion,
   the conversion's scale and error bounds, and numpy matmul.
+- affine_quantize, affine_dequantize (the MLX-style affine group format of
+  the MLX port's README, for the bytes-versus-accuracy comparison): pinned
+  by brute-force nearest grid points, the half-step error bound, exactly
+  representable grids, constant groups and the bit-stream packing.
 - moe: pinned through closed-form special cases (single slot, constant-level
   experts) and composition with the pinned linear; the squared-ReLU and the
   bf16 rounding of the hidden activation are fixed by the workload
@@ -102,6 +106,8 @@ def _load():
             lib.orc_e4m3_to_f64.restype = ctypes.c_double
             lib.orc_to_fp8.argtypes = [P, P, I64, I64, ctypes.c_uint64, P, P]
             lib.orc_linear_fp8.argtypes = [P, I64, I64, P, P, I64, P]
+            lib.orc_affine_quantize.argtypes = [P, I64, I64, ctypes.c_int, P, P, P]
+            lib.orc_affine_dequantize.argtypes = [P, P, P, I64, I64, ctypes.c_int, P]
             _lib = lib
     return _lib
 
@@ -331,6 +337,32 @@ def linear_fp8(x_bf16, q, s):
     y = np.zeros((m, n), np.float64)
     _load().orc_linear_fp8(_ptr(x), m, k, _ptr(q), _ptr(s), n, _ptr(y))
     return y, round_bf16(y)
+
+
+AFFINE_GROUP = 64
+
+
+def affine_quantize(W, bits: int):
+    """MLX-style affine group quantization of W fp32 [n][k] (groups of 64 along
+    k): returns (codes uint8 [n][k*bits/8] bit stream, scales bf16 bits
+    [n][k/64], biases bf16 bits [n][k/64])."""
+    W = _c(W, np.float32)
+    n, k = W.shape
+    assert bits in (4, 6, 8) and k % AFFINE_GROUP == 0
+    codes = np.zeros((n, k * bits // 8), np.uint8)
+    scales = np.zeros((n, k // AFFINE_GROUP), np.uint16)
+    biases = np.zeros((n, k // AFFINE_GROUP), np.uint16)
+    _load().orc_affine_quantize(_ptr(W), n, k, bits, _ptr(codes), _ptr(scales), _ptr(biases))
+    return codes, scales, biases
+
+
+def affine_dequantize(codes, scales, biases, bits: int) -> np.ndarray:
+    codes = _c(codes, np.uint8); scales = _c(scales, np.uint16); biases = _c(biases, np.uint16)
+    n = codes.shape[0]
+    k = codes.shape[1] * 8 // bits
+    W = np.zeros((n, k), np.float32)
+    _load().orc_affine_dequantize(_ptr(codes), _ptr(scales), _ptr(biases), n, k, bits, _ptr(W))
+    return W
 
 
 def moe(x_bf16, ids, w, up_codes, up_scales, up_seed, dn_codes, dn_scales, dn_seed):

@@ -493,3 +493,77 @@ void orc_linear_fp8(const uint16_t *x, int64_t m, int64_t k, const uint8_t *q, c
             y[i * n + j] = acc;
         }
 }
+
+/* ------------------------------------------------------------------ */
+/* MLX-style affine group quantization ("Nemotron-Labs-TwoTower-30B-A3B --
+ * MLX 6-bit", section "Quantization (6-bit, scheme mixed_v1)": the bulk of
+ * the weights at 6 bits, embeddings and heads at >= 8 bits, the family at 4,
+ * 6 and 8 bits).  Reading of what the README leaves open: groups of 64
+ * consecutive weights of a row; scale = (max - min) / (2^b - 1) and
+ * bias = min, both computed in fp32 and stored as bf16 (the checkpoint's
+ * dtype); q = clamp(rint(fp32(fp32(w - bias) / scale)), 0, 2^b - 1) against
+ * the stored bf16 values (a zero scale gives q = 0); codes of a row packed as
+ * one little-endian bit stream, element i in bits [b i, b i + b).
+ * Dequantized weight: fp32(fp32(scale * q) + bias).                       */
+
+#define ORC_AFF_GROUP 64
+
+static float orc_bf16_to_f32(uint16_t b) {
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, 4);
+    return f;
+}
+
+/* fp32 -> bf16 bits, round to nearest even (finite inputs). */
+static uint16_t orc_f32_to_bf16(float f) { return orc_f64_to_bf16((double)f); }
+
+void orc_affine_quantize(const float *W, int64_t n, int64_t k, int bits, uint8_t *codes, uint16_t *scales,
+                         uint16_t *biases) {
+    const int64_t ng = k / ORC_AFF_GROUP, row_bytes = k * bits / 8;
+    const float qmax = (float)((1 << bits) - 1);
+    memset(codes, 0, (size_t)(n * row_bytes));
+    for (int64_t i = 0; i < n; i++)
+        for (int64_t g = 0; g < ng; g++) {
+            const float *w = W + i * k + g * ORC_AFF_GROUP;
+            float lo = w[0], hi = w[0];
+            for (int j = 1; j < ORC_AFF_GROUP; j++) {
+                if (w[j] < lo) lo = w[j];
+                if (w[j] > hi) hi = w[j];
+            }
+            const uint16_t sb = orc_f32_to_bf16((hi - lo) / qmax), bb = orc_f32_to_bf16(lo);
+            scales[i * ng + g] = sb;
+            biases[i * ng + g] = bb;
+            const float sc = orc_bf16_to_f32(sb), bi = orc_bf16_to_f32(bb);
+            for (int j = 0; j < ORC_AFF_GROUP; j++) {
+                float q = 0.0f;
+                if (sc != 0.0f) {
+                    const float t = (w[j] - bi) / sc;
+                    q = rintf(t);
+                    if (q < 0.0f) q = 0.0f;
+                    if (q > qmax) q = qmax;
+                }
+                const uint32_t v = (uint32_t)q;
+                const int64_t bit = (g * ORC_AFF_GROUP + j) * bits;
+                for (int b = 0; b < bits; b++)
+                    if ((v >> b) & 1u) codes[i * row_bytes + (bit + b) / 8] |= (uint8_t)(1u << ((bit + b) % 8));
+            }
+        }
+}
+
+void orc_affine_dequantize(const uint8_t *codes, const uint16_t *scales, const uint16_t *biases, int64_t n,
+                           int64_t k, int bits, float *W) {
+    const int64_t ng = k / ORC_AFF_GROUP, row_bytes = k * bits / 8;
+    for (int64_t i = 0; i < n; i++)
+        for (int64_t e = 0; e < k; e++) {
+            uint32_t v = 0;
+            for (int b = 0; b < bits; b++) {
+                const int64_t bit = e * bits + b;
+                v |= (uint32_t)((codes[i * row_bytes + bit / 8] >> (bit % 8)) & 1u) << b;
+            }
+            const int64_t g = e / ORC_AFF_GROUP;
+            const float sc = orc_bf16_to_f32(scales[i * ng + g]), bi = orc_bf16_to_f32(biases[i * ng + g]);
+            const float t = sc * (float)v;
+            W[i * k + e] = t + bi;
+        }
+}

@@ -519,3 +519,69 @@ def test_fp8_linear_matches_numpy_matmul():
     y, yb = oracle.linear_fp8(x, q, s)
     ref = synth.bf16_bits_to_f32(x).astype(np.float64) @ oracle.fp8_dequantize(q, s).T
     assert np.allclose(y, ref, rtol=1e-12, atol=1e-15)
+
+
+# ----------------------------------------------------------------- affine (MLX-style) format
+def _unpack_bits(codes, bits):
+    # an independent reading of the little-endian bit stream (numpy's unpackbits)
+    b = np.unpackbits(codes, axis=1, bitorder="little")
+    n, nbits = b.shape
+    b = b.reshape(n, nbits // bits, bits).astype(np.uint32)
+    return (b << np.arange(bits, dtype=np.uint32)).sum(axis=2)
+
+
+def _bf16(bits):
+    return synth.bf16_bits_to_f32(np.asarray(bits, np.uint16)).astype(np.float64)
+
+
+@pytest.mark.parametrize("bits", [4, 6, 8])
+def test_affine_codes_are_nearest_grid_points(bits):
+    W = synth.student_t_f32((16, 256), 170 + bits, 5.0, 0.02)
+    codes, scales, biases = oracle.affine_quantize(W, bits)
+    q = _unpack_bits(codes, bits)
+    sc = np.repeat(_bf16(scales), 64, axis=1)
+    bi = np.repeat(_bf16(biases), 64, axis=1)
+    qmax = 2 ** bits - 1
+    grid = sc[..., None] * np.arange(qmax + 1)[None, None, :] + bi[..., None]
+    dist = np.abs(grid - W[..., None].astype(np.float64))
+    best = dist.argmin(axis=2)
+    d_sel = np.take_along_axis(dist, q[..., None].astype(np.int64), axis=2)[..., 0]
+    # the chosen point is a nearest one (up to fp32 rounding of the quotient)
+    assert np.all(d_sel <= dist.min(axis=2) + 1e-6 * sc)
+    assert np.mean(q == best) > 0.999
+    # scale = (max - min) / (2^b - 1) and bias = min, rounded to bf16
+    g = W.reshape(16, 4, 64).astype(np.float32)
+    lo, hi = g.min(axis=2), g.max(axis=2)
+    assert np.array_equal(scales, synth.f32_to_bf16_bits((hi - lo) / np.float32(qmax)))
+    assert np.array_equal(biases, synth.f32_to_bf16_bits(lo))
+    # the dequantized weight is the chosen grid point, and within half a step
+    Wd = oracle.affine_dequantize(codes, scales, biases, bits).astype(np.float64)
+    assert np.allclose(Wd, sc * q + bi, rtol=1e-6, atol=1e-9)
+    # (bf16 rounding of the bias shifts the grid, of the scale stretches it:
+    # the extremes of a group may lie that much beyond the grid's ends)
+    slack = np.abs(bi - np.repeat(lo.astype(np.float64), 64, axis=1))
+    slack += qmax * np.abs(sc - np.repeat(((hi - lo) / np.float32(qmax)).astype(np.float64), 64, axis=1))
+    assert np.all(np.abs(Wd - W) <= 0.5 * sc + slack + 1e-7)
+
+
+def test_affine_exact_grid_constant_group_and_packing():
+    bits = 6
+    rng = np.random.default_rng(175)
+    q = rng.integers(0, 64, size=(3, 128))
+    q[:, 0], q[:, 1] = 0, 63          # each group spans the full range
+    q[:, 64], q[:, 65] = 0, 63
+    sc, bi = np.float32(2.0 ** -9), np.float32(-0.0625)
+    W = (bi + sc * q).astype(np.float32)
+    W[2, 64:] = np.float32(0.3)       # a constant group: zero scale, codes 0
+    codes, scales, biases = oracle.affine_quantize(W, bits)
+    got = _unpack_bits(codes, bits)
+    assert np.array_equal(got[:2], q[:2]) and np.array_equal(got[2, :64], q[2, :64])
+    assert np.all(got[2, 64:] == 0) and _bf16(scales)[2, 1] == 0.0
+    Wd = oracle.affine_dequantize(codes, scales, biases, bits)
+    assert np.array_equal(Wd[:2], W[:2]) and np.array_equal(Wd[2, :64], W[2, :64])
+    assert np.all(Wd[2, 64:] == _bf16(synth.f32_to_bf16_bits(np.float32([0.3])))[0])
+    # 4 and 8 bits: the stream is plain nibbles (even element low) and bytes
+    c4, _, _ = oracle.affine_quantize(W, 4)
+    assert np.array_equal(_unpack_bits(c4, 4)[:, 0::2], (c4 & 0xF)) and np.array_equal(_unpack_bits(c4, 4)[:, 1::2], c4 >> 4)
+    c8, _, _ = oracle.affine_quantize(W, 8)
+    assert np.array_equal(_unpack_bits(c8, 8), c8)
