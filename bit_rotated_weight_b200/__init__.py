@@ -26,6 +26,7 @@ __all__ = [
     "tq4_1s_quantize", "tq4_1s_quantize_batched", "tq4_1s_dequantize", "tq4_1s_linear_workspace", "tq4_1s_linear",
     "tq4_1s_moe_workspace", "tq4_1s_moe", "tq4_1s_moe_logits", "tq4_1s_router_topk", "tq4_1s_moe_route", "tq4_1s_get_status", "tq4_1s_launch_count",
     "tq4_1s_linear_static", "tq4_1s_debug_hook", "Fp8Weight", "tq4_1s_to_fp8", "tq4_1s_linear_fp8",
+    "AffineWeight", "tq4_1s_affine_quantize", "tq4_1s_affine_dequantize", "tq4_1s_affine_linear",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -49,6 +50,13 @@ class _Weight(ctypes.Structure):
         ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("num_experts", ctypes.c_int32),
         ("flags", ctypes.c_int32), ("seed", ctypes.c_uint64),
         ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+    ]
+
+
+class _AffineWeight(ctypes.Structure):
+    _fields_ = [
+        ("n", ctypes.c_int64), ("k", ctypes.c_int64), ("bits", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p), ("biases", ctypes.c_void_p),
     ]
 
 
@@ -89,6 +97,10 @@ def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
                 "tq4_1s_to_fp8": ([W, P, P, P], ctypes.c_int),
                 "tq4_1s_linear_fp8_workspace": ([I64, I64, I64], SZ),
                 "tq4_1s_linear_fp8": ([P, I64, P, P, I64, I64, I32, P, P, SZ, P], ctypes.c_int),
+                "tq4_1s_affine_quantize": ([P, ctypes.POINTER(_AffineWeight), P], ctypes.c_int),
+                "tq4_1s_affine_dequantize": ([ctypes.POINTER(_AffineWeight), P, P], ctypes.c_int),
+                "tq4_1s_affine_linear_workspace": ([I64, ctypes.POINTER(_AffineWeight)], SZ),
+                "tq4_1s_affine_linear": ([P, I64, ctypes.POINTER(_AffineWeight), P, P, SZ, P], ctypes.c_int),
             }
             for name, (args, res) in sig.items():
                 fn = getattr(lib, name)
@@ -405,4 +417,61 @@ def tq4_1s_linear_fp8(x: torch.Tensor, w: Fp8Weight, out: torch.Tensor | None = 
     wsz = 0 if workspace is None else workspace.numel()
     _check(lib.tq4_1s_linear_fp8(_ptr(x), m, _ptr(w.q), _ptr(w.wscale), w.n, w.k, w.flags, _ptr(out),
                                  _ptr(workspace), wsz, _stream(x.device)), "linear_fp8")
+    return out
+
+
+@dataclass
+class AffineWeight:
+    """The MLX-style affine format: codes [n][k*bits/8] (bit stream), bf16
+    scales and biases [n][k/64] (as int16 bit patterns)."""
+    codes: torch.Tensor
+    scales: torch.Tensor
+    biases: torch.Tensor
+    n: int
+    k: int
+    bits: int
+
+    def c_struct(self) -> _AffineWeight:
+        return _AffineWeight(self.n, self.k, self.bits, 0, self.codes.data_ptr(), self.scales.data_ptr(),
+                             self.biases.data_ptr())
+
+    @property
+    def nbytes(self) -> int:
+        return self.codes.numel() + 2 * (self.scales.numel() + self.biases.numel())
+
+
+def tq4_1s_affine_quantize(W: torch.Tensor, bits: int) -> AffineWeight:
+    """Quantize W (float32 [n][k], CUDA, k % 64 == 0) to the affine format."""
+    if W.dim() != 2 or W.dtype != torch.float32 or not W.is_cuda:
+        raise ValueError("W must be a CUDA float32 [n][k] tensor")
+    W = W.contiguous()
+    n, k = W.shape
+    out = AffineWeight(torch.empty((n, k * bits // 8), dtype=torch.uint8, device=W.device),
+                       torch.empty((n, k // 64), dtype=torch.int16, device=W.device),
+                       torch.empty((n, k // 64), dtype=torch.int16, device=W.device), n, k, bits)
+    st = out.c_struct()
+    _check(load_library().tq4_1s_affine_quantize(_ptr(W), ctypes.byref(st), _stream(W.device)), "affine_quantize")
+    return out
+
+
+def tq4_1s_affine_dequantize(w: AffineWeight) -> torch.Tensor:
+    out = torch.empty((w.n, w.k), dtype=torch.float32, device=w.codes.device)
+    st = w.c_struct()
+    _check(load_library().tq4_1s_affine_dequantize(ctypes.byref(st), _ptr(out), _stream(out.device)),
+           "affine_dequantize")
+    return out
+
+
+def tq4_1s_affine_linear(x: torch.Tensor, w: AffineWeight, out: torch.Tensor | None = None) -> torch.Tensor:
+    if x.dtype != torch.bfloat16 or x.dim() != 2 or not x.is_cuda:
+        raise ValueError("x must be a CUDA bfloat16 [m][k] tensor")
+    x = x.contiguous()
+    m = x.shape[0]
+    if out is None:
+        out = torch.empty((m, w.n), dtype=torch.bfloat16, device=x.device)
+    st = w.c_struct()
+    lib = load_library()
+    ws = _workspace(lib.tq4_1s_affine_linear_workspace(m, ctypes.byref(st)), x.device, "affine")
+    _check(lib.tq4_1s_affine_linear(_ptr(x), m, ctypes.byref(st), _ptr(out), _ptr(ws), ws.numel(),
+                                    _stream(x.device)), "affine_linear")
     return out

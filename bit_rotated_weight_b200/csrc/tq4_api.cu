@@ -622,6 +622,72 @@ TQ_API int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, con
                                   static_cast<int32_t>(k), grid, st));
 }
 
+// ------------------------------------------------------------------ affine format
+static int affine_ok(const tq4_1s_affine_weight* w, bool need_ptrs) {
+  if (!w) return TQ_ERR_INVALID_ARG;
+  if (w->n <= 0 || w->k <= 0 || (w->k % 64) != 0 || w->reserved != 0) return TQ_ERR_INVALID_ARG;
+  if (w->bits != 4 && w->bits != 6 && w->bits != 8) return TQ_ERR_INVALID_ARG;
+  if (w->n > (1ll << 30) || w->k > (1ll << 30)) return TQ_ERR_INVALID_ARG;
+  if (need_ptrs) {
+    if (!w->codes || !w->scales || !w->biases) return TQ_ERR_INVALID_ARG;
+    if (!aligned16(w->codes) || !aligned16(w->scales) || !aligned16(w->biases)) return TQ_ERR_ALIGNMENT;
+  }
+  return TQ_OK;
+}
+
+TQ_API int tq4_1s_affine_quantize(const float* W, const tq4_1s_affine_weight* out, tq4_stream_t stream) {
+  int rc = affine_ok(out, true);
+  if (rc) return rc;
+  if (!W) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(W)) return TQ_ERR_ALIGNMENT;
+  if ((rc = check_device(nullptr))) return rc;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
+  return cuda_rc(launch_affine_quantize(W, out->codes, out->scales, out->biases, out->n, out->k, out->bits,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+TQ_API int tq4_1s_affine_dequantize(const tq4_1s_affine_weight* w, float* W_out, tq4_stream_t stream) {
+  int rc = affine_ok(w, true);
+  if (rc) return rc;
+  if (!W_out) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(W_out)) return TQ_ERR_ALIGNMENT;
+  if ((rc = check_device(nullptr))) return rc;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
+  return cuda_rc(launch_affine_dequantize(w->codes, w->scales, w->biases, W_out, false, w->n, w->k, w->bits,
+                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+TQ_API size_t tq4_1s_affine_linear_workspace(int64_t m, const tq4_1s_affine_weight* w) {
+  if (m <= 0 || m > (1ll << 24) || affine_ok(w, false) != TQ_OK) return 0;
+  return align256(static_cast<size_t>(w->n) * static_cast<size_t>(w->k) * 2);
+}
+
+TQ_API int tq4_1s_affine_linear(const uint16_t* x, int64_t m, const tq4_1s_affine_weight* w, uint16_t* y, void* ws,
+                                size_t ws_bytes, tq4_stream_t stream) {
+  int rc = affine_ok(w, true);
+  if (rc) return rc;
+  if (m < 0 || m > (1ll << 24)) return TQ_ERR_INVALID_ARG;
+  if (m == 0) return TQ_OK;
+  if (!x || !y) return TQ_ERR_INVALID_ARG;
+  if (!aligned16(x) || !aligned16(y)) return TQ_ERR_ALIGNMENT;
+  int sms = 0;
+  if ((rc = check_device(&sms))) return rc;
+  const size_t need = align256(static_cast<size_t>(w->n) * static_cast<size_t>(w->k) * 2);
+  if (!ws || ws_bytes < need) return TQ_ERR_WORKSPACE;
+  if (!aligned16(ws)) return TQ_ERR_ALIGNMENT;
+  if (take_injected_failure()) return TQ_ERR_CUDA;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  uint16_t* wh = static_cast<uint16_t*>(ws);
+  if (launch_affine_dequantize(w->codes, w->scales, w->biases, wh, true, w->n, w->k, w->bits, st) != cudaSuccess)
+    return TQ_ERR_CUDA;
+  alignas(64) CUtensorMap tx, tw;
+  if (!map_bf16(&tx, x, m, w->k, 128) || !map_bf16(&tw, wh, w->n, w->k, 256)) return TQ_ERR_CUDA;
+  const int64_t gt = ((m + 127) / 128) * ((w->n + 255) / 256);
+  const int grid = static_cast<int>(gt < sms ? gt : sms);
+  return cuda_rc(launch_gemm_bf16(&tx, &tw, y, static_cast<int32_t>(m), static_cast<int32_t>(w->n),
+                                  static_cast<int32_t>(w->k), grid, st));
+}
+
 static int64_t H_of(const tq4_1s_weight* up) { return up->k; }
 
 static int moe_check(int64_t m, int32_t topk, const tq4_1s_weight* up, const tq4_1s_weight* down, bool ptrs) {

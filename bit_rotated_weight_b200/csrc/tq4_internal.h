@@ -63,6 +63,12 @@ cudaError_t launch_to_fp8(const uint8_t* codes, const uint16_t* scales, uint8_t*
                           int64_t k, uint32_t mask, const CodebookF32& cb, cudaStream_t st);
 cudaError_t launch_fp8_to_bf16(const uint8_t* q, const float* wscale, uint16_t* out, int64_t rows, int64_t k,
                                cudaStream_t st);
+// The MLX-style affine format: fp32 rows -> bit-stream codes + bf16
+// scales/biases per group of 64, and back (fp32 or bf16 out).
+cudaError_t launch_affine_quantize(const float* W, uint8_t* codes, uint16_t* scales, uint16_t* biases, int64_t rows,
+                                   int64_t k, int bits, cudaStream_t st);
+cudaError_t launch_affine_dequantize(const uint8_t* codes, const uint16_t* scales, const uint16_t* biases, void* out,
+                                     bool bf16_out, int64_t rows, int64_t k, int bits, cudaStream_t st);
 // Activation rotation for the stream-K GEMM: x' = r H diag(s) x per 32-slice
 // of each row, scaled by a per-row power of two 2^-e and rounded to fp16
 // [rows][k]; row_scale[row] = 2^e.  Row r reads x row

@@ -341,6 +341,85 @@ __global__ void __launch_bounds__(256) fp8_to_bf16_kernel(const uint8_t* __restr
   }
 }
 
+// ------------------------------------------------------------------ affine format
+// MLX-style affine group quantization (the MLX port's README, "Quantization
+// (6-bit, scheme mixed_v1)"; 4/6/8-bit family): groups of 64 weights of a
+// row, scale = (max - min) / (2^b - 1) and bias = min in fp32, stored as bf16;
+// q = clamp(rint(fp32(fp32(w - bias) / scale)), 0, 2^b - 1) against the stored
+// values (zero scale: q = 0); codes as one little-endian bit stream per row.
+// One thread per group; a group's codes are 8 b bytes, byte-aligned.
+constexpr int kAffGroup = 64;
+
+__global__ void __launch_bounds__(256) affine_quantize_kernel(const float* __restrict__ W, uint8_t* __restrict__ codes,
+                                                              uint16_t* __restrict__ scales,
+                                                              uint16_t* __restrict__ biases, int64_t groups,
+                                                              int bits) {
+  const float qmax = static_cast<float>((1 << bits) - 1);
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const float4* w4 = reinterpret_cast<const float4*>(W + g * kAffGroup);
+    float lo = INFINITY, hi = -INFINITY;
+    for (int i = 0; i < kAffGroup / 4; ++i) {
+      const float4 f = __ldg(w4 + i);
+      lo = fminf(fminf(lo, f.x), fminf(f.y, fminf(f.z, f.w)));
+      hi = fmaxf(fmaxf(hi, f.x), fmaxf(f.y, fmaxf(f.z, f.w)));
+    }
+    const __nv_bfloat16 sb = __float2bfloat16_rn(__fdiv_rn(__fsub_rn(hi, lo), qmax));
+    const __nv_bfloat16 bb = __float2bfloat16_rn(lo);
+    scales[g] = __bfloat16_as_ushort(sb);
+    biases[g] = __bfloat16_as_ushort(bb);
+    const float sc = __bfloat162float(sb), bi = __bfloat162float(bb);
+    // pack into 32-bit words through a 64-bit accumulator
+    uint32_t* out = reinterpret_cast<uint32_t*>(codes + g * (8 * bits));
+    unsigned long long accb = 0ull;
+    int nacc = 0, nw = 0;
+    for (int i = 0; i < kAffGroup / 4; ++i) {
+      const float4 f = __ldg(w4 + i);
+      const float fv[4] = {f.x, f.y, f.z, f.w};
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float q = 0.0f;
+        if (sc != 0.0f) q = fminf(fmaxf(rintf(__fdiv_rn(__fsub_rn(fv[j], bi), sc)), 0.0f), qmax);
+        accb |= static_cast<unsigned long long>(static_cast<uint32_t>(q)) << nacc;
+        nacc += bits;
+        if (nacc >= 32) {
+          out[nw++] = static_cast<uint32_t>(accb);
+          accb >>= 32;
+          nacc -= 32;
+        }
+      }
+    }
+  }
+}
+
+template <typename TO>
+__global__ void __launch_bounds__(256) affine_dequantize_kernel(const uint8_t* __restrict__ codes,
+                                                                const uint16_t* __restrict__ scales,
+                                                                const uint16_t* __restrict__ biases,
+                                                                TO* __restrict__ out, int64_t groups, int bits) {
+  const uint32_t mask = (1u << bits) - 1u;
+  for (int64_t g = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; g < groups;
+       g += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const uint32_t* in = reinterpret_cast<const uint32_t*>(codes + g * (8 * bits));
+    const float sc = bf16_bits_to_f32(__ldg(scales + g)), bi = bf16_bits_to_f32(__ldg(biases + g));
+    TO* o = out + g * kAffGroup;
+    unsigned long long accb = 0ull;
+    int nacc = 0, nr = 0;
+    for (int i = 0; i < kAffGroup; ++i) {
+      if (nacc < bits) {
+        accb |= static_cast<unsigned long long>(__ldg(in + nr++)) << nacc;
+        nacc += 32;
+      }
+      const uint32_t q = static_cast<uint32_t>(accb) & mask;
+      accb >>= bits;
+      nacc -= bits;
+      const float v = __fadd_rn(__fmul_rn(sc, static_cast<float>(q)), bi);
+      if constexpr (sizeof(TO) == 4) o[i] = v;
+      else o[i] = __bfloat16_as_ushort(__float2bfloat16_rn(v));
+    }
+  }
+}
+
 // ------------------------------------------------------------------ activations
 // The activation side of route B: x' = r H diag(s) x per 32-slice of each row
 // (rotating x by the weight's RHT instead of inverse-rotating the weight;
@@ -631,6 +710,28 @@ static int grid_threads(int64_t threads_needed, int threads) {
   if (blocks < 1) blocks = 1;
   return static_cast<int>(blocks);
 }
+
+cudaError_t launch_affine_quantize(const float* W, uint8_t* codes, uint16_t* scales, uint16_t* biases, int64_t rows,
+                                   int64_t k, int bits, cudaStream_t st) {
+  const int64_t groups = rows * (k / kAffGroup);
+  affine_quantize_kernel<<<grid_threads(groups, 256), 256, 0, st>>>(W, codes, scales, biases, groups, bits);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_affine_dequantize(const uint8_t* codes, const uint16_t* scales, const uint16_t* biases, void* out,
+                                     bool bf16_out, int64_t rows, int64_t k, int bits, cudaStream_t st) {
+  const int64_t groups = rows * (k / kAffGroup);
+  if (bf16_out)
+    affine_dequantize_kernel<uint16_t><<<grid_threads(groups, 256), 256, 0, st>>>(
+        codes, scales, biases, static_cast<uint16_t*>(out), groups, bits);
+  else
+    affine_dequantize_kernel<float><<<grid_threads(groups, 256), 256, 0, st>>>(codes, scales, biases,
+                                                                               static_cast<float*>(out), groups, bits);
+  note_launches(1);
+  return cudaGetLastError();
+}
+
 
 cudaError_t launch_quantize_batch(const QuantItem* items, int count, int dtype, const CodebookF32& cb,
                                   cudaStream_t st) {

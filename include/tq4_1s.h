@@ -208,6 +208,44 @@ size_t tq4_1s_linear_fp8_workspace(int64_t m, int64_t n, int64_t k);
 int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, const float* wscale, int64_t n, int64_t k,
                       int32_t flags, uint16_t* y, void* ws, size_t ws_bytes, tq4_stream_t stream);
 
+/* A second weight format, for a bytes-versus-accuracy comparison with
+ * TQ4_1S: the MLX port's affine group quantization ("Nemotron-Labs-TwoTower-
+ * 30B-A3B -- MLX 6-bit", section "Quantization (6-bit, scheme mixed_v1)":
+ * the bulk of the weights at 6 bits, embeddings and heads at >= 8 bits; the
+ * family also at 4 bits).  Reading of what the README leaves open: groups
+ * of 64 consecutive weights of a row; per group scale = (max - min) /
+ * (2^bits - 1) and bias = min, computed in fp32 and stored as bf16;
+ * q = clamp(rint(fp32(fp32(w - bias) / scale)), 0, 2^bits - 1) against the
+ * stored values (a zero scale gives q = 0); the codes of a row are one
+ * little-endian bit stream (element i in bits [bits i, bits i + bits)).
+ * Dequantized weight: fp32(fp32(scale * q) + bias).  bits + 0.5 bits per
+ * weight (4.5, 6.5, 8.5). */
+typedef struct {
+  int64_t n;          /* rows, > 0                                             */
+  int64_t k;          /* columns, > 0, multiple of 64                          */
+  int32_t bits;       /* 4, 6 or 8                                             */
+  int32_t reserved;   /* must be 0                                             */
+  uint8_t* codes;     /* device, [n][k * bits / 8], 16-byte aligned            */
+  uint16_t* scales;   /* device, bf16 bits [n][k / 64], 16-byte aligned        */
+  uint16_t* biases;   /* device, bf16 bits [n][k / 64], 16-byte aligned        */
+} tq4_1s_affine_weight;
+
+/* Quantize W (device fp32 [n][k], 16-byte aligned) into out's planes. */
+int tq4_1s_affine_quantize(const float* W, const tq4_1s_affine_weight* out, tq4_stream_t stream);
+
+/* Dequantize to fp32 W_out (device [n][k]). */
+int tq4_1s_affine_dequantize(const tq4_1s_affine_weight* w, float* W_out, tq4_stream_t stream);
+
+/* Workspace bytes of tq4_1s_affine_linear (the bf16 weight); 0 on invalid
+ * arguments. */
+size_t tq4_1s_affine_linear_workspace(int64_t m, const tq4_1s_affine_weight* w);
+
+/* y[m][n] = bf16(x * W_hat^T) for the affine format: the weight dequantized
+ * to bf16 in the workspace, then the tensor-core GEMM (the comparison path;
+ * the TQ4_1S decode kernel is the streaming one).  m == 0 is a no-op. */
+int tq4_1s_affine_linear(const uint16_t* x, int64_t m, const tq4_1s_affine_weight* w, uint16_t* y, void* ws,
+                         size_t ws_bytes, tq4_stream_t stream);
+
 /* tq4_1s_linear for callers that cannot allocate device memory.  (The model
  * card has no counterpart: this is a deployment variant of the layer above.)
  * Plugin hosts and serving runtimes that fix every device allocation at

@@ -131,6 +131,23 @@ def test_fp8_cache_validation():
     assert lib.tq4_1s_linear_fp8(good, 16, ctypes.c_void_p(4097), good, 64, 64, 0, good, null, 0, null) == 2
 
 
+def test_affine_validation():
+    lib = tq.load_library()
+    null = ctypes.c_void_p(0)
+    good = ctypes.c_void_p(4096)
+
+    def aw(n=64, k=128, bits=6, codes=16, scales=16, biases=16):
+        return tq._AffineWeight(n, k, bits, 0, codes, scales, biases)
+
+    assert lib.tq4_1s_affine_quantize(good, ctypes.byref(aw(bits=5)), null) == 1      # bits not 4/6/8
+    assert lib.tq4_1s_affine_quantize(good, ctypes.byref(aw(k=96)), null) == 1        # k % 64 != 0
+    assert lib.tq4_1s_affine_quantize(null, ctypes.byref(aw()), null) == 1
+    assert lib.tq4_1s_affine_quantize(good, ctypes.byref(aw(biases=0)), null) == 1
+    assert lib.tq4_1s_affine_quantize(good, ctypes.byref(aw(scales=24)), null) == 2
+    assert lib.tq4_1s_affine_linear_workspace(16, ctypes.byref(aw(n=4096, k=4096))) == 4096 * 4096 * 2
+    assert lib.tq4_1s_affine_linear(good, 0, ctypes.byref(aw()), good, null, 0, null) == 0        # m == 0
+
+
 def test_debug_hooks_validation():
     lib = tq.load_library()
     assert lib.tq4_1s_debug_hook(99, 0) == 1                       # unknown hook
