@@ -474,12 +474,80 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     out["quantize"] = q
     del up, dn
     torch.cuda.empty_cache()
+    out["formats"] = formats_comparison(tq, synth, dev, pk, timed)
+    torch.cuda.empty_cache()
     # the 52-layer denoise sweep: whole step in one CUDA graph, 2 timed steps
     meas, layers, b, _ = sweep_measure(tq, synth, dev, pk, timed, steps=2, warmup=1)
     out["denoise_sweep_52"] = meas
     del layers, b
     torch.cuda.empty_cache()
     return out
+
+
+def formats_comparison(tq, synth, dev, pk, timed):
+    """Bytes versus accuracy of the weight formats on the decode workload
+    (4096 x 4096, 16 tokens, chained 16-call graphs over 16 distinct copies):
+    TQ4_1S (5 bits/weight), its fp8-resident cache (8 bits + a row scale) and
+    the MLX-style affine format at 4/6/8 bits (+0.5 bit of bf16 scale and
+    bias per 64).  Accuracy: relative RMS error and cosine of the
+    reconstructed weight against the drawn one (fp64 on the device), for
+    Student-t(5) (the decode weight) and Gaussian weights."""
+    import torch
+    n = k = 4096
+    res = {}
+    Ws = {"student_t5": torch.from_numpy(synth.student_t_f32((n, k), 2, 5.0, 0.02)).to(dev),
+          "gaussian": synth.normal_f32_device((n, k), 8, 0.02, dev)}
+
+    def acc(W, Wh):
+        d = (Wh.double() - W.double())
+        return {"rel_rms_err": float(d.norm() / W.double().norm()),
+                "cosine": float((Wh.double() * W.double()).sum() / Wh.double().norm() / W.double().norm())}
+
+    xs = torch.from_numpy(synth.activations_bf16(16, k, 3).view(np.int16)).to(dev).view(torch.bfloat16)
+    y = torch.empty((16, 16, n), dtype=torch.bfloat16, device=dev)
+
+    def chain_us(call):
+        g = torch.cuda.CUDAGraph()
+        call_chain = lambda: [call(xs if j == 0 else y[j - 1], j, y[j]) for j in range(16)]
+        call_chain()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=torch.cuda.Stream(dev)):
+            call_chain()
+        for _ in range(3):
+            g.replay()
+        ms = timed(lambda i: g.replay(), 10) / 10
+        del g
+        return ms * 1e3 / 16
+
+    for dist, W in Ws.items():
+        p = tq.tq4_1s_quantize(W, seed=2)
+        row = {"tq4_1s": {"bits_per_weight": 5.0, **acc(W, tq.tq4_1s_dequantize(p)[0])}}
+        f = tq.tq4_1s_to_fp8(p)
+        Wf = f.wscale[:, None] * f.q.view(torch.float8_e4m3fn).float()
+        row["fp8_cache_of_tq4_1s"] = {"bits_per_weight": 8 + 32 / k, **acc(W, Wf)}
+        for bits in (4, 6, 8):
+            a = tq.tq4_1s_affine_quantize(W, bits)
+            row[f"affine_{bits}bit"] = {"bits_per_weight": bits + 0.5, **acc(W, tq.tq4_1s_affine_dequantize(a))}
+        res[dist] = row
+        if dist == "student_t5":
+            torch.cuda.synchronize()
+            copies = [tq.Packed(p.codes.clone(), p.scales.clone(), n, k, 1, 2, flags=tq.TQ_WEIGHT_STATIC)
+                      for _ in range(16)]
+            fcop = [tq.Fp8Weight(f.q.clone(), f.wscale.clone(), n, k, flags=tq.TQ_WEIGHT_STATIC) for _ in range(16)]
+            a6 = tq.tq4_1s_affine_quantize(W, 6)
+            torch.cuda.synchronize()
+            us_tq4 = chain_us(lambda x, j, o: tq.tq4_1s_linear(x, copies[j], out=o))
+            us_f8 = chain_us(lambda x, j, o: tq.tq4_1s_linear_fp8(x, fcop[j], out=o))
+            us_a6 = chain_us(lambda x, j, o: tq.tq4_1s_affine_linear(x, a6, out=o))
+            res["decode_m16_chained_us_per_call"] = {
+                "tq4_1s": us_tq4, "fp8_cache": us_f8, "affine_6bit_dequant_gemm": us_a6,
+                "streamed_bytes": {"tq4_1s": n * k * 5 // 8, "fp8_cache": n * k + 4 * n,
+                                   "affine_6bit": n * k * 13 // 16},
+                "note": "TQ4_1S and the fp8 cache in the decode kernel (weights static, 16 distinct copies); "
+                        "the affine format through a bf16 weight + tensor-core GEMM (one weight, L2-warm)"}
+            del copies, fcop, a6
+        del p, f
+    return res
 
 
 # ------------------------------------------------------------------ denoise sweep

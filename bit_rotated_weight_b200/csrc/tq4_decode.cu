@@ -32,9 +32,9 @@
 //     maximum and writes x' straight into the swizzled B tiles; the MMAs, the
 //     remaining tile and the epilogue.
 //
-// Warps (512 threads, one CTA per SM):
-//   0      lane 0: TMA producer of the codes tiles;
-//   1-3    lane 0: MMA issuer of dequant group 0-2;
+// Warps (640 threads, one CTA per SM):
+//   16     lane 0: TMA producer of the codes tiles;
+//   1-3, 17-19  lane 0: MMA issuers, one per (dequant group, 64-k half);
 //   0-3    epilogue (thread = tile row) once the MMAs are done;
 //   4-15   three dequant groups of four warps (thread = tile row): per
 //          iteration 16 B of codes + 8 scales -> 128 fp16 levels -> tensor
@@ -49,7 +49,11 @@ namespace {
 
 constexpr int kGroups = 3;                 // dequant groups
 constexpr int kFirstDqWarp = 4;
-constexpr int kThreads = (kFirstDqWarp + 4 * kGroups) * 32;   // 512
+constexpr int kRotWarps = kFirstDqWarp + 4 * kGroups;          // warps 0-15 rotate x (one token each)
+constexpr int kProducerWarp = kRotWarps;                        // warp 16: TMA producer
+constexpr int kFirstHiIssuerWarp = kProducerWarp + 1;           // warps 17-19: issuers of the second halves
+constexpr int kIssuers = 2 * kGroups;                           // one per (group, 64-k half)
+constexpr int kThreads = (kFirstHiIssuerWarp + kGroups) * 32;   // 640
 constexpr int kMaxIters = kFusedMaxIters;  // iterations (128 k) per CTA
 constexpr int kStagesD = kMaxIters;        // one codes stage per iteration
 constexpr int kCodesTile = 128 * 64;       // codes of one iteration: 128 rows x 64 B
@@ -58,15 +62,15 @@ constexpr int kAColsD = 64;                // tensor-memory columns of one A sta
 constexpr int kTmemColsD = 512;
 constexpr float kLevelScaleD = 256.0f;
 // A stages: the tensor memory beside the accumulators (16 nb columns per group)
-__host__ __device__ constexpr int a_stages(int nb) { return (kTmemColsD - kGroups * 16 * nb) / kAColsD; }
+__host__ __device__ constexpr int a_stages(int nb) { return (kTmemColsD - kIssuers * 16 * nb) / kAColsD; }
 
 struct DecodeShared {
   uint64_t full[kStagesD];           // codes tile landed (TMA bytes)
   uint64_t afull[kMaxIters][2];      // A stage s, half h holds fresh levels (4 warp arrivals)
   uint64_t afree[kMaxIters][2];      // the MMAs reading A stage s, half h completed
   uint64_t xready;                   // every token's x' is in the B tiles (16 warp arrivals)
-  uint64_t dfull;                    // every issuer's MMAs completed (kGroups arrivals)
-  uint64_t idone[kGroups];           // an issuer's own MMAs completed (teardown)
+  uint64_t dfull;                    // every issuer's MMAs completed (kIssuers arrivals)
+  uint64_t idone[kIssuers];          // an issuer's own MMAs completed (teardown)
   uint64_t eready;                   // every dequant thread wrote its row exponent (12 warp arrivals)
   int8_t rexp[kGroups][128];         // row exponent of each group's levels (see the dequant)
   float row_scale[kSegRows];         // 2^e of each token
@@ -149,9 +153,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* lut = smem + off_lut(NB, F8);
   uint8_t* red = smem + off_red(NB, F8);
   constexpr int kHalf = b_half_bytes(NB);
-  constexpr int kAccW = 16 * NB;          // accumulator columns per group
-  constexpr int kACol0 = kGroups * kAccW; // first A-stage column
-  constexpr int kNA = a_stages(NB);       // A stages (7 at NB == 1, 6 at NB == 2)
+  constexpr int kAccW = 16 * NB;           // columns of one accumulator
+  constexpr int kACol0 = kIssuers * kAccW; // first A-stage column: an accumulator per (group, half)
+  constexpr int kNA = a_stages(NB);        // A stages (6 at NB == 1, 5 at NB == 2)
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = a.split;
@@ -164,15 +168,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   const bool stat = a.static_w != 0;
 
   if (warp == 0) {
-    constexpr int kBars = kStagesD + 4 * kMaxIters + 2 + kGroups + 1;
+    constexpr int kBars = kStagesD + 4 * kMaxIters + 2 + kIssuers + 1;
     for (int i = lane; i < kBars; i += 32) {
       if (i < kStagesD) mbar_init(&sh.full[i], 1);
       else if (i < kStagesD + 2 * kMaxIters) mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4);
       else if (i < kStagesD + 4 * kMaxIters)
         mbar_init(&sh.afree[(i - kStagesD - 2 * kMaxIters) >> 1][(i - kStagesD) & 1], 1);
-      else if (i == kStagesD + 4 * kMaxIters) mbar_init(&sh.xready, kThreads / 32);
-      else if (i == kStagesD + 4 * kMaxIters + 1) mbar_init(&sh.dfull, kGroups);
-      else if (i < kStagesD + 4 * kMaxIters + 2 + kGroups) mbar_init(&sh.idone[i - kStagesD - 4 * kMaxIters - 2], 1);
+      else if (i == kStagesD + 4 * kMaxIters) mbar_init(&sh.xready, kRotWarps);
+      else if (i == kStagesD + 4 * kMaxIters + 1) mbar_init(&sh.dfull, kIssuers);
+      else if (i < kStagesD + 4 * kMaxIters + 2 + kIssuers) mbar_init(&sh.idone[i - kStagesD - 4 * kMaxIters - 2], 1);
       else mbar_init(&sh.eready, 4 * kGroups);
     }
     if (lane == 0) {
@@ -186,12 +190,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   if (!F8) {
     // level-pair table: entry b (a code byte) of lane l's copy at byte
-    // 128 b + 4 l holds {256 c[b & 15], 256 c[b >> 4]} * (fp16 pair)
+    // 128 b + 4 l holds {256 c[b & 15], 256 c[b >> 4]} * (fp16 pair); a warp
+    // writes whole entries, so its parameter reads are uniform
     uint32_t* lw = reinterpret_cast<uint32_t*>(lut);
-    for (int i = threadIdx.x; i < 256 * 32; i += kThreads) {
-      const int b = i >> 5;
-      lw[i] = lt.h[b & 15] | (lt.h[b >> 4] << 16);
-    }
+    for (int b = warp; b < 256; b += kThreads / 32) lw[b * 32 + lane] = lt.h[b & 15] | (lt.h[b >> 4] << 16);
   }
   tc_fence_before();
   __syncthreads();
@@ -213,14 +215,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_arrive_expect_tx(&sh.full[li], kTile);
     tma_load_3d(smem + li * kTile, &tm_codes, &sh.full[li], (it0 + li) * (F8 ? 128 : 64), row0, 0);
   };
-  if (warp == 0 && lane == 0) {
+  if (warp == kProducerWarp && lane == 0) {
     for (int li = 0; li < cnt; ++li) {
       if (stat) issue_codes(li);
       else tma_prefetch_l2_3d(&tm_codes, (it0 + li) * (F8 ? 128 : 64), row0, 0);
     }
   }
 
-  const int dq_group = (warp >= kFirstDqWarp) ? (warp - kFirstDqWarp) >> 2 : -1;
+  const int dq_group = (warp >= kFirstDqWarp && warp < kRotWarps) ? (warp - kFirstDqWarp) >> 2 : -1;
   const int trow = (warp & 3) * 32 + lane;   // tile row of this thread (dequant and epilogue)
   // dequant threads: the scales of their (up to 3) iterations, 16 B each
   uint32_t sraw[3][4];
@@ -359,7 +361,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   pdl_wait();
-  if (!stat && warp == 0 && lane == 0)
+  if (!stat && warp == kProducerWarp && lane == 0)
     for (int li = 0; li < cnt; ++li) issue_codes(li);
   if (!stat && dq_group >= 0) load_scales();
 
@@ -375,7 +377,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int nsl = cnt * 4;
     const float r = __uint_as_float(0x3E3504F3u);
 #pragma unroll 1
-    for (int tk = warp; tk < 16 * NB; tk += 16) {
+    for (int tk = warp; warp < kRotWarps && tk < 16 * NB; tk += kRotWarps) {
       float v[32];
       const int kk = (it0 * 4 + lane) * 32;   // first k of this lane's slice
       const bool live = lane < nsl && tk < a.m && kk < a.k;
@@ -441,46 +443,49 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
     __syncwarp();
-    if (lane == 0 && !(a.test_withhold && warp == 7)) mbar_arrive(&sh.xready);
+    if (warp < kRotWarps && lane == 0 && !(a.test_withhold && warp == 7)) mbar_arrive(&sh.xready);
   }
 
   if (dq_group >= 0) {
     if (!stat) dq_exponent();
     if (dq_ok) dq_run(kMaxIters);
-  } else if (warp == 0 && lane == 0) {
+  } else if (warp == kProducerWarp && lane == 0) {
     // ------------------------------------------------------------ producer
     // (every tile was issued above; on an abort, let them land before exit)
     if (*abortp)
       for (int li = 0; li < cnt; ++li) drain(&sh.full[li], 0);
-  } else if (warp >= 1 && warp <= kGroups && lane == 0) {
+  } else if (((warp >= 1 && warp <= kGroups) || warp >= kFirstHiIssuerWarp) && lane == 0) {
     // ------------------------------------------------------------ MMA issue
-    const int g = warp - 1;
-    const uint32_t acc = tmem + g * kAccW;
+    // Issuer (g, h): the 4 MMAs of half h of each of group g's iterations,
+    // into its own accumulator (single-thread issue costs ~65 cycles per
+    // instruction at this N, so six threads issue in parallel).
+    const int g = warp >= kFirstHiIssuerWarp ? warp - kFirstHiIssuerWarp : warp - 1;
+    const int h = warp >= kFirstHiIssuerWarp ? 1 : 0;
+    const int ii = 2 * g + h;
+    const uint32_t acc = tmem + ii * kAccW;
     const uint32_t idesc = idesc_f16(128, 16 * NB);
     bool ok = mbar_wait(&sh.xready, 0, abortp);
     int use = 0;
     for (int li = g; ok && li < cnt; li += kGroups, ++use) {
       const int sa = li % kNA;
       const uint32_t a_stage = tmem + kACol0 + sa * kAColsD;
-      for (int h = 0; h < 2; ++h) {
-        if (!mbar_wait(&sh.afull[sa][h], (li / kNA) & 1, abortp)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint64_t bdesc = sdesc_k128(smem_u32(btiles + (li * 2 + h) * kHalf));
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
-                 (use == 0 && h == 0 && kk == 0) ? 0u : 1u);
-        mma_commit(&sh.afree[sa][h]);
+      if (!mbar_wait(&sh.afull[sa][h], (li / kNA) & 1, abortp)) {
+        ok = false;
+        break;
       }
+      tc_fence_after();
+      const uint64_t bdesc = sdesc_k128(smem_u32(btiles + (li * 2 + h) * kHalf));
+#pragma unroll
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
+               (use == 0 && kk == 0) ? 0u : 1u);
+      mma_commit(&sh.afree[sa][h]);
     }
     if (use > 0) mma_commit(&sh.dfull);
     else mbar_arrive(&sh.dfull);
     // its MMAs complete before the CTA can release tensor memory
-    mma_commit(&sh.idone[g]);
-    drain(&sh.idone[g], 0);
+    mma_commit(&sh.idone[ii]);
+    drain(&sh.idone[ii], 0);
   }
   if (warp < 4) {
     __syncwarp();
@@ -497,7 +502,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
     tc_fence_after();
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-    const int ngroups = cnt < kGroups ? cnt : kGroups;
+    const int ngroups = cnt < kGroups ? cnt : kGroups;   // groups (and their two accumulators) with work
     const float wsc = F8 ? ((row0 + trow < a.n) ? __ldcg(a.wscale + row0 + trow) : 0.0f) : 1.0f / kLevelScaleD;
     if (ok) {
 #pragma unroll
@@ -505,11 +510,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-        for (int g = 0; g < ngroups; ++g) {
+        for (int ii = 0; ii < 2 * ngroups; ++ii) {
           uint32_t rr[16];
-          tmem_ld16(tmem + lane_base + g * kAccW + 16 * c, rr);
+          tmem_ld16(tmem + lane_base + ii * kAccW + 16 * c, rr);
           tmem_wait_ld();
-          const float rs = ldexpf(1.0f, sh.rexp[g][trow]);
+          const float rs = ldexpf(1.0f, sh.rexp[ii >> 1][trow]);
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(rr[j]), rs));
         }

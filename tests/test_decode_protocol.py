@@ -37,14 +37,15 @@ def _const(name):
 
 GROUPS = _const("kGroups")
 FIRST_DQ = _const("kFirstDqWarp")
-WARPS = FIRST_DQ + 4 * GROUPS
+WARPS = FIRST_DQ + 4 * GROUPS          # rotation warps (one token each)
+ISSUERS = 2 * GROUPS                   # one per (group, 64-k half)
 MAX_ITERS = 8                                    # kFusedMaxIters
 TMEM_COLS = _const("kTmemColsD")
 
 
 def a_stages(nb):
     # as a_stages() in the kernel: tensor memory beside the accumulators
-    return (TMEM_COLS - GROUPS * 16 * nb) // 64
+    return (TMEM_COLS - ISSUERS * 16 * nb) // 64
 
 
 def test_source_constants_and_counts():
@@ -52,10 +53,11 @@ def test_source_constants_and_counts():
     assert (GROUPS, FIRST_DQ, TMEM_COLS) == (3, 4, 512)
     assert "constexpr int kStagesD = kMaxIters;" in SRC              # one codes stage per iteration
     assert "mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4)" in SRC   # one arrival per warp
-    assert "mbar_init(&sh.xready, kThreads / 32)" in SRC             # one arrival per warp
-    assert "mbar_init(&sh.dfull, kGroups)" in SRC
+    assert "mbar_init(&sh.xready, kRotWarps)" in SRC                 # one arrival per rotation warp
+    assert "constexpr int kRotWarps = kFirstDqWarp + 4 * kGroups;" in SRC
+    assert "mbar_init(&sh.dfull, kIssuers)" in SRC and "constexpr int kIssuers = 2 * kGroups;" in SRC
     assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
-    assert (a_stages(1), a_stages(2)) == (7, 6)
+    assert (a_stages(1), a_stages(2)) == (6, 5)
 
 
 class Barrier:
@@ -92,8 +94,8 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
     afull = [[bar(f"afull{s}{h}", 4) for h in range(2)] for s in range(MAX_ITERS)]
     afree = [[bar(f"afree{s}{h}", 1) for h in range(2)] for s in range(MAX_ITERS)]
     xready = bar("xready", WARPS)
-    dfull = bar("dfull", GROUPS)
-    idone = [bar(f"idone{g}", 1) for g in range(GROUPS)]
+    dfull = bar("dfull", ISSUERS)
+    idone = [bar(f"idone{i}", 1) for i in range(ISSUERS)]
     eready = bar("eready", 4 * GROUPS)
     state = {"abort": False, "landings": [], "mma": [], "issued": 0, "landed": 0, "mma_issued": 0,
              "waited": False}
@@ -156,51 +158,50 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
         if ok:
             yield from dq_run(g, done, MAX_ITERS)
 
-    def issuer(g):
-        yield from rotation(1 + g)
+    def issuer(g, h):
+        # lane 0 of warps 1-3 (h = 0, also rotation warps) and 17-19 (h = 1)
+        if h == 0:
+            yield from rotation(1 + g)
         ok = yield from wait(xready, 0)
         use = 0
         for li in range(g, cnt, GROUPS):
             if not ok:
                 break
             sa = li % na
-            for h in range(2):
-                ok = yield from wait(afull[sa][h], li // na)
-                if not ok:
-                    break
-                state["mma_issued"] += 1
-                state["mma"].append(afree[sa][h])      # commit: arrives when the MMAs complete
+            ok = yield from wait(afull[sa][h], li // na)
             if not ok:
                 break
+            state["mma_issued"] += 1
+            state["mma"].append(afree[sa][h])          # commit: arrives when the MMAs complete
             use += 1
         if use > 0:
             state["mma"].append(dfull)
         else:
             dfull.arrive()
-        state["mma"].append(idone[g])
-        yield from wait(idone[g], 0, bounded=False)
+        state["mma"].append(idone[2 * g + h])
+        yield from wait(idone[2 * g + h], 0, bounded=False)
 
     def producer():
-        # warp 0, lane 0: every tile at once (before the wait when static)
+        # warp 16, lane 0: every tile at once (before the wait when static)
         if static:
             issue_all()
         yield ("step", "wait for the previous kernel")
         if not static:
             issue_all()
-        yield from rotation(0)
+        yield ("step", "the others rotate")
         if state["abort"]:
             for li in range(cnt):
                 yield from wait(full[li], 0, bounded=False)
 
     def epilogue(w):
         if w == 0:
-            yield from producer()
+            yield from rotation(0)
         ok = yield from wait(xready, 0)
         ok = ok and (yield from wait(eready, 0))
         ok = ok and (yield from wait(dfull, 0))
 
-    actors = [epilogue(0)]
-    actors += [issuer(g) for g in range(GROUPS)]
+    actors = [epilogue(0), producer()]
+    actors += [issuer(g, h) for g in range(GROUPS) for h in range(2)]
     actors += [dequant(g, q) for g in range(GROUPS) for q in range(4)]
     # the issuers' warps 1-3 join the epilogue after their roles
     actors += [epilogue(w) for w in range(1, 4)]

@@ -117,14 +117,14 @@ def test_static_scratch_takes_no_memory_and_replays_in_a_graph():
     def call(x, st=stream):
         assert fn(ctypes.c_void_p(x.data_ptr()), m, ctypes.byref(wst), ctypes.c_void_p(y.data_ptr()), st) == 0
 
+    refs = torch.empty((3, m, n), dtype=torch.bfloat16, device=dev)
     call(xs[0])
     torch.cuda.synchronize()
     free0, alloc0 = torch.cuda.mem_get_info(dev)[0], torch.cuda.memory_allocated(dev)
-    refs = []
-    for x in xs:
+    for i, x in enumerate(xs):
         call(x)
         torch.cuda.synchronize()
-        refs.append(y.clone())
+        refs[i].copy_(y)
     assert torch.cuda.mem_get_info(dev)[0] == free0 and torch.cuda.memory_allocated(dev) == alloc0
     x_in = xs[0].clone()
     g = torch.cuda.CUDAGraph()
