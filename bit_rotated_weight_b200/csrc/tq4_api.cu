@@ -772,6 +772,7 @@ static int moe_impl(const uint16_t* x, int64_t m, const int32_t* topk_ids, const
   a.row_scale = xscale;
   a.epoch = next_epoch();
   a.cluster_s = 1;
+  a.x_resident = (L.nb_max == 1 && H <= kResidentMaxK) ? 1 : 0;
   a.mode = EPI_UP;
   a.out_a = h;
   a.partials = reinterpret_cast<float*>(base + L.partials);
@@ -789,6 +790,7 @@ static int moe_impl(const uint16_t* x, int64_t m, const int32_t* topk_ids, const
   b.k_iters = static_cast<int32_t>((I + 127) / 128);
   b.scales = down->scales;
   b.row_scale = hscale;
+  b.x_resident = (L.nb_max == 1 && I <= kResidentMaxK) ? 1 : 0;
   b.epoch = next_epoch();
   b.mode = EPI_DOWN;
   b.out_a = nullptr;

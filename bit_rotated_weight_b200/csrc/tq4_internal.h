@@ -115,6 +115,8 @@ struct StreamKArgs {
   int32_t cluster_s;         // >= 2: fused split-K mode -- grid = tiles * cluster_s, one cluster per
                              // tile, partials reduced through distributed shared memory; else 1
   int32_t x_box3;            // cluster mode with k % 64 == 0: x arrives as one 3-D box (tm_x3)
+  int32_t x_resident;        // grouped mode, segments of <= 16 rows, k <= kResidentMaxK: a segment's
+                             // x' for all of k is loaded once into shared memory (no per-iteration x')
   int32_t mode;              // EpilogueMode
   uint16_t* out_a;           // dense: y [m][n]; up: h = relu(u)^2 [P][n] (bf16)
   float* out_f;              // down: z*w [m*topk][n]
@@ -128,6 +130,9 @@ struct StreamKArgs {
 // Iterations per CTA up to which the dense kernel can rotate x in its
 // prologue (one pipeline stage per iteration, no stage reuse).
 constexpr int kFusedMaxIters = 8;
+
+// Largest k whose 16-row x' (fp16) fits the stream-K kernel's B tiles at once.
+constexpr int kResidentMaxK = 3072;
 
 // A fresh counter tag for each stream-K launch.
 uint32_t next_epoch();

@@ -112,6 +112,8 @@ struct SharedState {
   uint64_t issuer_done[kDequantGroups];
   uint64_t xready;             // fused mode: every stage's x' tile is written (one arrival per prologue warp)
   uint64_t xland[kFusedMaxIters];   // fused mode: the raw x tiles of a stage landed (TMA)
+  uint64_t rland;              // resident mode: the current segment's x' (all of k) landed
+  uint64_t rfree;              // resident mode: the MMAs reading the previous segment's x' completed (4 commits)
   float row_scale[kSegRows];   // fused mode: 2^e of each row
   unsigned row_max[kSegRows];  // fused mode: max |x| of each row over this CTA's k range (float bits)
   uint32_t tmem_base;
@@ -325,7 +327,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // the barriers, spread over the lanes of warp 0
-    constexpr int kBars = 2 * kStages + 4 * kDequantGroups + 12 + 1 + kFusedMaxIters;
+    constexpr int kBars = 2 * kStages + 4 * kDequantGroups + 12 + 1 + kFusedMaxIters + 2;
     for (int i = lane; i < kBars; i += 32) {
       if (i < kStages) mbar_init(&sh.full[i], 1);
       else if (i < 2 * kStages) mbar_init(&sh.done[i - kStages], 1);
@@ -343,8 +345,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(&sh.issuer_done[i - 2 * kStages - 4 * kDequantGroups - 8], 1);
       } else if (i == 2 * kStages + 4 * kDequantGroups + 12) {
         mbar_init(&sh.xready, kPrologueThreads / 32);
-      } else {
+      } else if (i < 2 * kStages + 4 * kDequantGroups + 13 + kFusedMaxIters) {
         mbar_init(&sh.xland[i - 2 * kStages - 4 * kDequantGroups - 13], 1);
+      } else if (i == 2 * kStages + 4 * kDequantGroups + 13 + kFusedMaxIters) {
+        mbar_init(&sh.rland, 1);
+      } else {
+        mbar_init(&sh.rfree, kDequantGroups);
       }
     }
     static_assert(kSegRows == 32, "one row maximum per lane");
@@ -518,7 +524,22 @@ __global__ void __launch_bounds__(kThreads, 1)
       // and does not write the weight.  Fused mode: any kernel may come
       // before, so wait first.
       const int npre = cnt < kStages ? cnt : kStages;
-      const uint32_t xbytes = fused ? 0u : 2u * 2048u;   // per 16-row block: two k-halves of 16 x 128 B
+      // per 16-row block: two k-halves of 16 x 128 B of x' per iteration (none
+      // in fused mode; none in resident mode, where a segment's x' for all of
+      // k is loaded once when the CTA reaches the segment)
+      const bool resident = a.x_resident != 0;
+      const uint32_t xbytes = (fused || resident) ? 0u : 2u * 2048u;
+      int rseg = -1, rcount = 0;   // resident mode: segment whose x' is loaded, loads so far
+      auto load_resident = [&](int sgi, const Seg& sg) -> bool {
+        // every MMA of the previous segment has read its x' (the issuers'
+        // commits), then all 2 KI 64-k halves of this one, 16 rows each
+        if (rcount > 0 && !mbar_wait(&sh.rfree, (rcount - 1) & 1, abortp)) return false;
+        mbar_arrive_expect_tx(&sh.rland, static_cast<uint32_t>(2 * KI) * 2048u);
+        for (int kh = 0; kh < 2 * KI; ++kh) tma_load_2d(smem + kBOff + kh * 2048, &tm_x, &sh.rland, 64 * kh, sg.row0);
+        rseg = sgi;
+        ++rcount;
+        return true;
+      };
       Cursor cur;
       cur.init(it_begin, KI, a.row_tiles);
       const Cursor first = cur;
@@ -544,17 +565,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       Seg sg = get_seg(a, cur.sgi);
       int seg_of = cur.sgi;
+      bool rok = true;
       for (int li = 0; li < npre; ++li, cur.advance(1, KI, a.row_tiles)) {
         if (cur.sgi != seg_of) {
           seg_of = cur.sgi;
           sg = get_seg(a, seg_of);
         }
+        if (resident && cur.sgi != rseg && !(rok = load_resident(cur.sgi, sg))) break;
         const int nb = (sg.count + 15) >> 4;
         mbar_arrive_expect_tx(&sh.full[li], kCodesBytes + nb * xbytes);
         armed[li] = 0;
         tma_load_3d(codes_of(li), &tm_codes, &sh.full[li], cur.kit * 64, cur.rt * 128, sg.e);
       }
-      if (!fused) {
+      if (!fused && !resident) {
         pdl_wait();   // x' and its row scales are the rotation kernel's output
         Cursor c2 = first;
         Seg sg2 = get_seg(a, c2.sgi);
@@ -568,7 +591,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
       // (fused mode: cnt <= kStages, so the loop below does not run)
-      for (int li = npre; li < cnt; ++li, cur.advance(1, KI, a.row_tiles)) {
+      for (int li = npre; rok && li < cnt; ++li, cur.advance(1, KI, a.row_tiles)) {
         const int s = li % kStages;
         const uint32_t ph = (li / kStages) & 1;
         if (!mbar_wait(&sh.done[s], ph ^ 1u, abortp)) break;
@@ -576,11 +599,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           seg_of = cur.sgi;
           sg = get_seg(a, seg_of);
         }
+        if (resident && cur.sgi != rseg && !(rok = load_resident(cur.sgi, sg))) break;
         const int nb = (sg.count + 15) >> 4;
         mbar_arrive_expect_tx(&sh.full[s], kCodesBytes + nb * xbytes);
         armed[s] = static_cast<int>(ph);
         tma_load_3d(codes_of(s), &tm_codes, &sh.full[s], cur.kit * 64, cur.rt * 128, sg.e);
-        load_x(s, cur.kit, sg, nb, &sh.full[s]);
+        if (!resident) load_x(s, cur.kit, sg, nb, &sh.full[s]);
       }
       if (*abortp) {
         // wind down: let every armed copy land before the CTA exits
@@ -588,6 +612,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (armed[i] >= 0) drain_wait(&sh.full[i], static_cast<uint32_t>(armed[i]));
         if (fused)
           for (int i = 0; i < (a.x_box3 ? 1 : cnt); ++i) drain_wait(&sh.xland[i], 0);
+        if (resident && rcount > 0) drain_wait(&sh.rland, (rcount - 1) & 1);
       }
     }
   } else if (warp >= kFirstDequantWarp && warp < kFirstEpilogueWarp) {
@@ -687,6 +712,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int w = issuer_group(warp);
     int use = 0;   // fills of the group's A stage consumed so far
     bool ok = !fused || mbar_wait(&sh.xready, 0, abortp);   // fused mode: the B tiles are written
+    const bool resident = a.x_resident != 0;
+    int iseg = -1, rn = 0;   // resident mode: segment whose x' the MMAs read, loads waited for
     for (int pi = 0; pi < nportions && ok; ++pi) {
       const int tile = tile_begin + pi;
       const int pf = (tile * KI > it_begin ? tile * KI : it_begin) - it_begin;
@@ -701,6 +728,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       const Seg sg = get_seg(a, tile / a.row_tiles);
       const int nb = (sg.count + 15) >> 4;
       const uint32_t idesc = idesc_f16(128, 16 * nb);
+      if (resident && tile / a.row_tiles != iseg) {
+        // a new segment: release the previous one's x' once these MMAs are
+        // done, then wait for this one's
+        if (iseg >= 0) mma_commit(&sh.rfree);
+        if (!mbar_wait(&sh.rland, rn & 1, abortp)) {
+          ok = false;
+          break;
+        }
+        ++rn;
+        iseg = tile / a.row_tiles;
+      }
       const uint32_t acc = tmem + db * (kAccRegion / nsets) + w * acc_w;
       const uint32_t a_stage = tmem + kACol0 + w * kAColsPerStage;
       bool started = false;
@@ -708,7 +746,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int li = pf + ((w - pf) % kDequantGroups + kDequantGroups) % kDequantGroups; li < pe && ok;
            li += kDequantGroups) {
         const int s = li % kStages;
-        const uint32_t xb = smem_u32(btile_of(s));
+        // resident mode: the iteration's k slice of the segment's x'; else the stage's B tile
+        const int kit_li = it_begin + li - tile * KI;
+        const uint32_t xb = resident ? smem_u32(smem + kBOff + kit_li * 2 * 2048) : smem_u32(btile_of(s));
         // the B tile (x') of this stage must have landed too
         if (!mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) {
           ok = false;
@@ -722,7 +762,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           // half h of the stage's B tile is k-half h of x'; the descriptor's
           // start address (16-byte units) advances by 2 per 16-k step
-          const uint64_t bdesc0 = sdesc_k128(xb + h * kXHalfBytes);
+          const uint64_t bdesc0 = sdesc_k128(xb + h * (resident ? 2048 : kXHalfBytes));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
             mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc0 + static_cast<uint64_t>(2 * kk), idesc,
