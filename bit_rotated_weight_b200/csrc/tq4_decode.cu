@@ -26,20 +26,20 @@
 //     traffic), before the wait when the weight is flagged static;
 //   * the dequant warps then turn as many tiles as tensor memory holds (7 of
 //     8 at 16 tokens) into A operands before the wait;
-//   * only the activation-dependent work follows the wait: one warp per
-//     token loads its k range of x with coalesced 16-byte loads, rotates each
-//     lane's 32-slice in registers, takes the token's scale from a warp
-//     maximum and writes x' straight into the swizzled B tiles; the MMAs, the
-//     remaining tile and the epilogue.
+//   * only the activation-dependent work follows the wait: eight warps that
+//     do not dequantize load x (two tokens each, coalesced 16-byte loads),
+//     rotate each lane's 32-slice in registers, take each token's scale from
+//     a warp maximum and write x' straight into the swizzled B tiles; then
+//     the MMAs, the remaining tiles and the epilogue.
 //
 // Warps (640 threads, one CTA per SM):
-//   16     lane 0: TMA producer of the codes tiles;
+//   4      lane 0: TMA producer of the codes tiles (it only issues);
 //   1-3, 17-19  lane 0: MMA issuers, one per (dequant group, 64-k half);
 //   0-3    epilogue (thread = tile row) once the MMAs are done;
 //   4-15   three dequant groups of four warps (thread = tile row): per
 //          iteration 16 B of codes + 8 scales -> 128 fp16 levels -> tensor
 //          memory, as two 64-k halves signalled separately;
-//   0-15   the x rotation (warp = token) after the wait.
+//   0-3, 16-19  the x rotation (two tokens per warp) after the wait.
 #include <mutex>
 
 #include "tq4_internal.h"
@@ -48,12 +48,13 @@ namespace tq4 {
 namespace {
 
 constexpr int kGroups = 3;                 // dequant groups
-constexpr int kFirstDqWarp = 4;
-constexpr int kRotWarps = kFirstDqWarp + 4 * kGroups;          // warps 0-15 rotate x (one token each)
-constexpr int kProducerWarp = kRotWarps;                        // warp 16: TMA producer
-constexpr int kFirstHiIssuerWarp = kProducerWarp + 1;           // warps 17-19: issuers of the second halves
+constexpr int kFirstDqWarp = 4;            // warps 4-15: dequant
+constexpr int kHiWarp = kFirstDqWarp + 4 * kGroups;             // warps 16-19: rotation (17-19 also issue)
+constexpr int kFirstHiIssuerWarp = kHiWarp + 1;                 // warps 17-19: issuers of the second halves
+constexpr int kProducerWarp = kFirstDqWarp;                     // warp 4, lane 0: TMA producer (issue only)
+constexpr int kRotWarps = 8;                                    // warps 0-3 and 16-19 rotate x
 constexpr int kIssuers = 2 * kGroups;                           // one per (group, 64-k half)
-constexpr int kThreads = (kFirstHiIssuerWarp + kGroups) * 32;   // 640
+constexpr int kThreads = (kHiWarp + 4) * 32;                    // 640
 constexpr int kMaxIters = kFusedMaxIters;  // iterations (128 k) per CTA
 constexpr int kStagesD = kMaxIters;        // one codes stage per iteration
 constexpr int kCodesTile = 128 * 64;       // codes of one iteration: 128 rows x 64 B
@@ -68,7 +69,7 @@ struct DecodeShared {
   uint64_t full[kStagesD];           // codes tile landed (TMA bytes)
   uint64_t afull[kMaxIters][2];      // A stage s, half h holds fresh levels (4 warp arrivals)
   uint64_t afree[kMaxIters][2];      // the MMAs reading A stage s, half h completed
-  uint64_t xready;                   // every token's x' is in the B tiles (16 warp arrivals)
+  uint64_t xready;                   // every token's x' is in the B tiles (8 warp arrivals)
   uint64_t dfull;                    // every issuer's MMAs completed (kIssuers arrivals)
   uint64_t idone[kIssuers];          // an issuer's own MMAs completed (teardown)
   uint64_t eready;                   // every dequant thread wrote its row exponent (12 warp arrivals)
@@ -222,7 +223,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  const int dq_group = (warp >= kFirstDqWarp && warp < kRotWarps) ? (warp - kFirstDqWarp) >> 2 : -1;
+  const int dq_group = (warp >= kFirstDqWarp && warp < kHiWarp) ? (warp - kFirstDqWarp) >> 2 : -1;
   const int trow = (warp & 3) * 32 + lane;   // tile row of this thread (dequant and epilogue)
   // dequant threads: the scales of their (up to 3) iterations, 16 B each
   uint32_t sraw[3][4];
@@ -366,37 +367,46 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (!stat && dq_group >= 0) load_scales();
 
   // ------------------------------------------------------------ x rotation
-  // Warp w rotates tokens w and w + 16 (NB == 2).  Lane l owns the 32-slice
-  // at k = 128 it0 + 32 l of its token (slices past the CTA's range are not
-  // written; slices past k are zero).  Signs flip bf16 sign bits; the
-  // butterfly runs in registers in the fixed stage order; e puts the token's
-  // largest |x'| in [2^13, 2^14) (fp16 cannot overflow); x' 2^-e is rounded
-  // to fp16 and stored in the B tile layout the MMA reads (K-major rows of
-  // 128 B, 8-row groups 1024 B apart, 16-byte chunks XOR-swizzled by row).
-  {
+  // The eight warps that do not dequantize (0-3 and 16-19) rotate x, so the
+  // dequant warps never hold it up: rotation warp r takes tokens r and r + 8
+  // (and r + 16, r + 24 at NB == 2), loading both tokens' slices before
+  // rotating either.  Lane l owns the 32-slice at k = 128 it0 + 32 l of a
+  // token (slices past the CTA's range are not written; slices past k are
+  // zero).  Signs flip bf16 sign bits; the butterfly runs in registers in the
+  // fixed stage order; e puts the token's largest |x'| in [2^13, 2^14) (fp16
+  // cannot overflow); x' 2^-e is rounded to fp16 and stored in the B tile
+  // layout the MMA reads (K-major rows of 128 B, 8-row groups 1024 B apart,
+  // 16-byte chunks XOR-swizzled by row).
+  const int rot = warp < 4 ? warp : ((warp >= kHiWarp && warp < kHiWarp + 4) ? warp - kHiWarp + 4 : -1);
+  if (rot >= 0) {
     const int nsl = cnt * 4;
     const float r = __uint_as_float(0x3E3504F3u);
+    const int kk = (it0 * 4 + lane) * 32;   // first k of this lane's slice
 #pragma unroll 1
-    for (int tk = warp; warp < kRotWarps && tk < 16 * NB; tk += kRotWarps) {
-      float v[32];
-      const int kk = (it0 * 4 + lane) * 32;   // first k of this lane's slice
-      const bool live = lane < nsl && tk < a.m && kk < a.k;
-      if (live) {
+    for (int round = 0; round < NB; ++round) {
+      uint4 raw[2][4];
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const int tk = rot + 8 * t + 16 * round;
+        const bool live = lane < nsl && tk < a.m && kk < a.k;
         const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(tk) * a.k + kk);
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const uint4 w4 = __ldcg(src + q);   // (L2: x is the previous kernel's output)
-          const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+        for (int q = 0; q < 4; ++q) raw[t][q] = live ? __ldcg(src + q) : make_uint4(0u, 0u, 0u, 0u);
+      }
+#pragma unroll 1
+      for (int t = 0; t < 2; ++t) {
+      const int tk = rot + 8 * t + 16 * round;
+      float v[32];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const uint32_t sw = F8 ? ww[e] : (ww[e] ^ a.x_sign[4 * q + e]);
-            v[8 * q + 2 * e] = __uint_as_float(sw << 16);
-            v[8 * q + 2 * e + 1] = __uint_as_float(sw & 0xFFFF0000u);
-          }
+      for (int q = 0; q < 4; ++q) {
+        const uint4 w4 = t ? raw[1][q] : raw[0][q];   // (L2: x is the previous kernel's output)
+        const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t sw = F8 ? ww[e] : (ww[e] ^ a.x_sign[4 * q + e]);
+          v[8 * q + 2 * e] = __uint_as_float(sw << 16);
+          v[8 * q + 2 * e + 1] = __uint_as_float(sw & 0xFFFF0000u);
         }
-      } else {
-#pragma unroll
-        for (int i = 0; i < 32; ++i) v[i] = 0.0f;
       }
       if (!F8) {
 #pragma unroll
@@ -440,19 +450,18 @@ __global__ void __launch_bounds__(kThreads, 1)
           *reinterpret_cast<uint4*>(rowp + (((c0 + q) ^ (tk & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
         }
       }
+      }
     }
     fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
     __syncwarp();
-    if (warp < kRotWarps && lane == 0 && !(a.test_withhold && warp == 7)) mbar_arrive(&sh.xready);
+    if (lane == 0 && !(a.test_withhold && rot == 7)) mbar_arrive(&sh.xready);
   }
 
   if (dq_group >= 0) {
     if (!stat) dq_exponent();
     if (dq_ok) dq_run(kMaxIters);
-  } else if (warp == kProducerWarp && lane == 0) {
-    // ------------------------------------------------------------ producer
-    // (every tile was issued above; on an abort, let them land before exit)
-    if (*abortp)
+    // the producer (every tile was issued above): on an abort, let them land before exit
+    if (warp == kProducerWarp && lane == 0 && *abortp)
       for (int li = 0; li < cnt; ++li) drain(&sh.full[li], 0);
   } else if (((warp >= 1 && warp <= kGroups) || warp >= kFirstHiIssuerWarp) && lane == 0) {
     // ------------------------------------------------------------ MMA issue
@@ -510,13 +519,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-        for (int ii = 0; ii < 2 * ngroups; ++ii) {
-          uint32_t rr[16];
-          tmem_ld16(tmem + lane_base + ii * kAccW + 16 * c, rr);
+        for (int g = 0; g < ngroups; ++g) {
+          // the group's two accumulators (its 64-k halves), one wait for both
+          uint32_t r0[16], r1[16];
+          tmem_ld16(tmem + lane_base + (2 * g) * kAccW + 16 * c, r0);
+          tmem_ld16(tmem + lane_base + (2 * g + 1) * kAccW + 16 * c, r1);
           tmem_wait_ld();
-          const float rs = ldexpf(1.0f, sh.rexp[ii >> 1][trow]);
+          const float rs = ldexpf(1.0f, sh.rexp[g][trow]);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(rr[j]), rs));
+          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(r0[j]), rs));
+#pragma unroll
+          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(r1[j]), rs));
         }
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], __fmul_rn(sh.row_scale[16 * c + j], wsc));

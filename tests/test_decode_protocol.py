@@ -37,7 +37,7 @@ def _const(name):
 
 GROUPS = _const("kGroups")
 FIRST_DQ = _const("kFirstDqWarp")
-WARPS = FIRST_DQ + 4 * GROUPS          # rotation warps (one token each)
+WARPS = _const("kRotWarps")            # rotation warps: 0-3 and 16-19
 ISSUERS = 2 * GROUPS                   # one per (group, 64-k half)
 MAX_ITERS = 8                                    # kFusedMaxIters
 TMEM_COLS = _const("kTmemColsD")
@@ -54,7 +54,11 @@ def test_source_constants_and_counts():
     assert "constexpr int kStagesD = kMaxIters;" in SRC              # one codes stage per iteration
     assert "mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4)" in SRC   # one arrival per warp
     assert "mbar_init(&sh.xready, kRotWarps)" in SRC                 # one arrival per rotation warp
-    assert "constexpr int kRotWarps = kFirstDqWarp + 4 * kGroups;" in SRC
+    assert WARPS == 8 and "constexpr int kProducerWarp = kFirstDqWarp;" in SRC
+    # dequant warps 4-15, rotation warps 0-3 and 16-19
+    assert "(warp >= kFirstDqWarp && warp < kHiWarp) ? (warp - kFirstDqWarp) >> 2 : -1" in SRC
+    assert "constexpr int kHiWarp = kFirstDqWarp + 4 * kGroups;" in SRC
+    assert "warp < 4 ? warp : ((warp >= kHiWarp && warp < kHiWarp + 4) ? warp - kHiWarp + 4 : -1)" in SRC
     assert "mbar_init(&sh.dfull, kIssuers)" in SRC and "constexpr int kIssuers = 2 * kGroups;" in SRC
     assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
     assert (a_stages(1), a_stages(2)) == (6, 5)
@@ -119,9 +123,10 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
             state["issued"] += 1
             state["landings"].append(full[li])
 
-    def rotation(w):
+    def rotation(r):
+        # rotation warp r (0-3: warps 0-3; 4-7: warps 16-19)
         yield ("step", "rotate")
-        if not (withhold_xready and w == 7):
+        if not (withhold_xready and r == 7):
             xready.arrive()
 
     def dq_run(g, done, li_end):
@@ -144,6 +149,10 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
             done[0] += 1
 
     def dequant(g, q):
+        # warp 4 + 4g + q; lane 0 of warp 4 is also the TMA producer
+        producer = (g, q) == (0, 0)
+        if producer and static:
+            issue_all()
         done = [0]
         ok = True
         if static:
@@ -151,17 +160,21 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
             eready.arrive()
             ok = yield from dq_run(g, done, na)      # before the wait: stages not reused
         yield ("step", "wait for the previous kernel")
-        yield from rotation(FIRST_DQ + 4 * g + q)
+        if producer and not static:
+            issue_all()
         if not static:
             yield ("step", "row exponent")
             eready.arrive()
         if ok:
             yield from dq_run(g, done, MAX_ITERS)
+        if producer and state["abort"]:
+            # every tile was issued: let them land before exit
+            for li in range(cnt):
+                yield from wait(full[li], 0, bounded=False)
 
     def issuer(g, h):
-        # lane 0 of warps 1-3 (h = 0, also rotation warps) and 17-19 (h = 1)
-        if h == 0:
-            yield from rotation(1 + g)
+        # lane 0 of warps 1-3 (h = 0) and 17-19 (h = 1), all rotation warps
+        yield from rotation(1 + g if h == 0 else 5 + g)
         ok = yield from wait(xready, 0)
         use = 0
         for li in range(g, cnt, GROUPS):
@@ -181,18 +194,6 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
         state["mma"].append(idone[2 * g + h])
         yield from wait(idone[2 * g + h], 0, bounded=False)
 
-    def producer():
-        # warp 16, lane 0: every tile at once (before the wait when static)
-        if static:
-            issue_all()
-        yield ("step", "wait for the previous kernel")
-        if not static:
-            issue_all()
-        yield ("step", "the others rotate")
-        if state["abort"]:
-            for li in range(cnt):
-                yield from wait(full[li], 0, bounded=False)
-
     def epilogue(w):
         if w == 0:
             yield from rotation(0)
@@ -200,7 +201,11 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
         ok = ok and (yield from wait(eready, 0))
         ok = ok and (yield from wait(dfull, 0))
 
-    actors = [epilogue(0), producer()]
+    def plain_rotation():
+        # warp 16 rotates and does nothing else
+        yield from rotation(4)
+
+    actors = [epilogue(0), plain_rotation()]
     actors += [issuer(g, h) for g in range(GROUPS) for h in range(2)]
     actors += [dequant(g, q) for g in range(GROUPS) for q in range(4)]
     # the issuers' warps 1-3 join the epilogue after their roles
