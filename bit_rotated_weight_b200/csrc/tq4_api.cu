@@ -471,8 +471,11 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     const int64_t KI = (w->k + 127) / 128;
     const int split = choose_decode_split(L.tiles, KI, sms, nb);
     if (split > 0) {
-      alignas(64) CUtensorMap tc;
-      if (!map_codes(&tc, w)) return TQ_ERR_CUDA;
+      alignas(64) CUtensorMap tc, tx, ts;
+      const bool sc_tma = (w->k % 128) == 0;
+      if (!map_codes(&tc, w) || !map_bf16(&tx, x, m, w->k, static_cast<uint32_t>(16 * nb)) ||
+          (sc_tma && !map_bf16(&ts, w->scales, w->n, w->k / 16, 128)))
+        return TQ_ERR_CUDA;
       DecodeArgs d{};
       d.n = static_cast<int32_t>(w->n);
       d.k = static_cast<int32_t>(w->k);
@@ -485,9 +488,10 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
       d.test_withhold = withhold_arrival_hook() ? 1 : 0;
       d.x = x;
       d.scales = w->scales;
+      d.scales_tma = sc_tma ? 1 : 0;
       d.y = y;
       sign_xor_words(mask, d.x_sign);
-      return cuda_rc(launch_decode(&tc, d, st));
+      return cuda_rc(launch_decode(&tc, &tx, &ts, d, st));
     }
   }
   if (small) {
@@ -587,8 +591,8 @@ TQ_API int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, con
     const int split = choose_decode_split(tiles, KI, sms, nb, true);
     if (split > 0) {
       if (take_injected_failure()) return TQ_ERR_CUDA;
-      alignas(64) CUtensorMap tc;
-      if (!map_fp8(&tc, q, n, k)) return TQ_ERR_CUDA;
+      alignas(64) CUtensorMap tc, tx;
+      if (!map_fp8(&tc, q, n, k) || !map_bf16(&tx, x, m, k, static_cast<uint32_t>(16 * nb))) return TQ_ERR_CUDA;
       DecodeArgs d{};
       d.n = static_cast<int32_t>(n);
       d.k = static_cast<int32_t>(k);
@@ -603,7 +607,7 @@ TQ_API int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, con
       d.wscale = wscale;
       d.x = x;
       d.y = y;
-      return cuda_rc(launch_decode(&tc, d, st));
+      return cuda_rc(launch_decode(&tc, &tx, &tc, d, st));
     }
   }
   // large m (or a shape the decode kernel does not take): the bf16 weight in

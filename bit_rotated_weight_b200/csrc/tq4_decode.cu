@@ -64,6 +64,10 @@ constexpr int kTmemColsD = 512;
 constexpr float kLevelScaleD = 256.0f;
 // A stages: the tensor memory beside the accumulators (16 nb columns per group)
 __host__ __device__ constexpr int a_stages(int nb) { return (kTmemColsD - kIssuers * 16 * nb) / kAColsD; }
+// A stages in shared memory (the MMA reads A from there), where it has room:
+// at 16 tokens of TQ4_1S, 6 + 2 = 8 stages hold every iteration of a CTA.
+__host__ __device__ constexpr int smem_a_stages(int nb, bool f8) { return (nb == 1 && !f8) ? 2 : 0; }
+constexpr int kATileBytes = 2 * 128 * 128;   // 128 rows x 128 k fp16: [2 halves][128 rows][128 B]
 
 struct DecodeShared {
   uint64_t full[kStagesD];           // codes tile landed (TMA bytes)
@@ -73,20 +77,28 @@ struct DecodeShared {
   uint64_t dfull;                    // every issuer's MMAs completed (kIssuers arrivals)
   uint64_t idone[kIssuers];          // an issuer's own MMAs completed (teardown)
   uint64_t eready;                   // every dequant thread wrote its row exponent (12 warp arrivals)
+  uint64_t xland;                    // the x tiles landed (TMA bytes)
+  uint64_t sfull;                    // the scales tile landed (TMA bytes)
   int8_t rexp[kGroups][128];         // row exponent of each group's levels (see the dequant)
   float row_scale[kSegRows];         // 2^e of each token
+  uint32_t tok_max[kSegRows];        // max |x| of each token over the CTA's k range (fp32 bits)
+  int own[3];                        // cluster reduction: rows per CTA, first and count of this CTA's rows
   uint32_t tmem_base;
   int abort_flag;
 };
 
 // Dynamic shared memory: codes stages | B tiles [iters][2 halves][16 nb rows x 128 B] |
-// level table (TQ4_1S only) | cluster reduction buffer [split][rows per CTA][16 nb] fp32.
-// The fp8 cache (f8) streams 128 B of codes per row and iteration and needs no table.
+// A stages in shared memory | level table and scales tile [128 rows][64
+// scales] (TQ4_1S only) | cluster reduction buffer [split][rows per CTA][16 nb] fp32.  The fp8 cache (f8)
+// streams 128 B of codes per row and iteration and needs neither.
 __host__ __device__ constexpr int tile_bytes(bool f8) { return f8 ? 2 * kCodesTile : kCodesTile; }
 __host__ __device__ constexpr int b_half_bytes(int nb) { return 16 * nb * 128; }
 __host__ __device__ constexpr int off_b(bool f8) { return kStagesD * tile_bytes(f8); }
-__host__ __device__ constexpr int off_lut(int nb, bool f8) { return off_b(f8) + kMaxIters * 2 * b_half_bytes(nb); }
-__host__ __device__ constexpr int off_red(int nb, bool f8) { return off_lut(nb, f8) + (f8 ? 0 : kLutBytesD); }
+__host__ __device__ constexpr int off_asm(int nb, bool f8) { return off_b(f8) + kMaxIters * 2 * b_half_bytes(nb); }
+__host__ __device__ constexpr int off_lut(int nb, bool f8) { return off_asm(nb, f8) + smem_a_stages(nb, f8) * kATileBytes; }
+__host__ __device__ constexpr int off_sc(int nb, bool f8) { return off_lut(nb, f8) + (f8 ? 0 : kLutBytesD); }
+constexpr int kScTileBytes = 128 * 128;   // 128 rows x 64 fp16 scales (8 iterations)
+__host__ __device__ constexpr int off_red(int nb, bool f8) { return off_sc(nb, f8) + (f8 ? 0 : kScTileBytes); }
 // (the reduction buffer holds split * ceil(128 / split) <= 135 rows)
 __host__ __device__ constexpr int smem_total(int nb, bool f8) { return off_red(nb, f8) + 136 * 16 * nb * 4 + 1024; }
 
@@ -130,6 +142,14 @@ __device__ __forceinline__ void drain(uint64_t* bar, uint32_t parity) {
   }
 }
 
+// Position of 4-token group gi of local row tl in the reduction buffer's row:
+// the groups are XOR-swizzled so that eight consecutive rows' float4 at the
+// same gi fall in eight different 16-byte bank groups.
+template <int NB>
+__device__ __forceinline__ int red_pos(int tl, int gi) {
+  return NB == 1 ? (gi ^ ((tl >> 1) & 3)) : (gi ^ (tl & 7));
+}
+
 __device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, float a, float b, float c, float d) {
   uint32_t remote;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
@@ -144,8 +164,8 @@ __device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, 
 // accumulator in the epilogue.
 template <int NB, bool F8>
 __global__ void __launch_bounds__(kThreads, 1)
-    decode_kernel(const __grid_constant__ CUtensorMap tm_codes, const DecodeArgs a,
-                  const __grid_constant__ LevelTableD lt) {
+    decode_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
+                  const __grid_constant__ CUtensorMap tm_sc, const DecodeArgs a, const __grid_constant__ LevelTableD lt) {
   __shared__ DecodeShared sh;
   extern __shared__ uint8_t dyn_smem[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dyn_smem) + 1023) & ~uintptr_t(1023));
@@ -153,10 +173,13 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* btiles = smem + off_b(F8);
   uint8_t* lut = smem + off_lut(NB, F8);
   uint8_t* red = smem + off_red(NB, F8);
+  const uint8_t* sctile = smem + off_sc(NB, F8);
   constexpr int kHalf = b_half_bytes(NB);
   constexpr int kAccW = 16 * NB;           // columns of one accumulator
   constexpr int kACol0 = kIssuers * kAccW; // first A-stage column: an accumulator per (group, half)
-  constexpr int kNA = a_stages(NB);        // A stages (6 at NB == 1, 5 at NB == 2)
+  constexpr int kNA = a_stages(NB);        // A stages in tensor memory (6 at NB == 1, 5 at NB == 2)
+  constexpr int kNS = kNA + smem_a_stages(NB, F8);   // all A stages (those past kNA in shared memory)
+  uint8_t* atiles = smem + off_asm(NB, F8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = a.split;
@@ -167,67 +190,57 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int cnt = it1 - it0;   // >= 1 (split <= KI), <= kMaxIters (host)
   const int row0 = tile * 128;
   const bool stat = a.static_w != 0;
-
-  if (warp == 0) {
-    constexpr int kBars = kStagesD + 4 * kMaxIters + 2 + kIssuers + 1;
-    for (int i = lane; i < kBars; i += 32) {
-      if (i < kStagesD) mbar_init(&sh.full[i], 1);
-      else if (i < kStagesD + 2 * kMaxIters) mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4);
-      else if (i < kStagesD + 4 * kMaxIters)
-        mbar_init(&sh.afree[(i - kStagesD - 2 * kMaxIters) >> 1][(i - kStagesD) & 1], 1);
-      else if (i == kStagesD + 4 * kMaxIters) mbar_init(&sh.xready, kRotWarps);
-      else if (i == kStagesD + 4 * kMaxIters + 1) mbar_init(&sh.dfull, kIssuers);
-      else if (i < kStagesD + 4 * kMaxIters + 2 + kIssuers) mbar_init(&sh.idone[i - kStagesD - 4 * kMaxIters - 2], 1);
-      else mbar_init(&sh.eready, 4 * kGroups);
-    }
-    if (lane == 0) {
-      sh.abort_flag = 0;
-      tma_prefetch_desc(&tm_codes);
-    }
-    fence_mbar_init();
-  } else if (warp == 1) {
-    tmem_alloc(&sh.tmem_base, kTmemColsD);
-    tmem_relinquish();
-  }
-  if (!F8) {
-    // level-pair table: entry b (a code byte) of lane l's copy at byte
-    // 128 b + 4 l holds {256 c[b & 15], 256 c[b >> 4]} * (fp16 pair); a warp
-    // writes whole entries, so its parameter reads are uniform
-    uint32_t* lw = reinterpret_cast<uint32_t*>(lut);
-    for (int b = warp; b < 256; b += kThreads / 32) lw[b * 32 + lane] = lt.h[b & 15] | (lt.h[b >> 4] << 16);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  // All CTAs of this grid are resident once every one of them is here: the
-  // next kernel may launch now.  Its CTAs take the SMs this grid leaves free
-  // and those its CTAs release, and set up meanwhile; anything of theirs that
-  // reads this kernel's output waits in griddepcontrol.wait.
-  if (threadIdx.x == 0) pdl_launch_dependents();
-  const uint32_t tmem = sh.tmem_base;
   volatile int* abortp = &sh.abort_flag;
 
-  // A weight flagged static is not written by any kernel still in flight,
-  // so its tiles and scales may be read before the wait; otherwise the
-  // previous kernel may have written it (a quantize) and they are read after
-  // it, with L2 prefetches issued now (a prefetch is only a hint and L2 is
-  // the device's point of coherence, so it is safe either way).
-  auto issue_codes = [&](int li) {
-    mbar_arrive_expect_tx(&sh.full[li], kTile);
-    tma_load_3d(smem + li * kTile, &tm_codes, &sh.full[li], (it0 + li) * (F8 ? 128 : 64), row0, 0);
+  // The codes tiles and the scales tile are requested first of all: the
+  // producer initialises their barriers and issues the copies before the
+  // rest of the set-up, so HBM latency overlaps it.  A weight flagged static
+  // is not written by any kernel still in flight, so it may be read before
+  // the wait for the previous kernel; otherwise the tiles are only pulled
+  // into L2 now and loaded after the wait (by the x producer, below).
+  const bool sc_tma = !F8 && a.scales_tma != 0;
+  auto issue_weight = [&]() {
+    for (int li = 0; li < cnt; ++li) {
+      mbar_arrive_expect_tx(&sh.full[li], kTile);
+      tma_load_3d(smem + li * kTile, &tm_codes, &sh.full[li], (it0 + li) * (F8 ? 128 : 64), row0, 0);
+    }
+    if (sc_tma) {
+      mbar_arrive_expect_tx(&sh.sfull, kScTileBytes);
+      tma_load_2d(const_cast<uint8_t*>(sctile), &tm_sc, &sh.sfull, it0 * 8, row0);
+    }
   };
   if (warp == kProducerWarp && lane == 0) {
-    for (int li = 0; li < cnt; ++li) {
-      if (stat) issue_codes(li);
-      else tma_prefetch_l2_3d(&tm_codes, (it0 + li) * (F8 ? 128 : 64), row0, 0);
+    for (int li = 0; li < cnt; ++li) mbar_init(&sh.full[li], 1);
+    mbar_init(&sh.sfull, 1);
+    fence_mbar_init();
+    if (stat) {
+      issue_weight();
+    } else {
+      for (int li = 0; li < cnt; ++li) tma_prefetch_l2_3d(&tm_codes, (it0 + li) * (F8 ? 128 : 64), row0, 0);
+      if (sc_tma) tma_prefetch_l2_2d(&tm_sc, it0 * 8, row0);
     }
   }
-
   const int dq_group = (warp >= kFirstDqWarp && warp < kHiWarp) ? (warp - kFirstDqWarp) >> 2 : -1;
   const int trow = (warp & 3) * 32 + lane;   // tile row of this thread (dequant and epilogue)
   // dequant threads: the scales of their (up to 3) iterations, 16 B each
   uint32_t sraw[3][4];
   auto load_scales = [&]() {
+    if (sc_tma) {
+      // the tile [128 rows][64 scales] (128-byte swizzle: chunk c of row t at
+      // c ^ (t & 7)); iteration li's 8 scales are chunk li of the row
+      const bool ok = wwait(&sh.sfull, 0, abortp);
+#pragma unroll
+      for (int u = 0; u < 3; ++u) {
+        const int li = dq_group + kGroups * u;
+        uint4 v = make_uint4(0u, 0u, 0u, 0u);
+        if (ok && li < cnt) v = *reinterpret_cast<const uint4*>(sctile + trow * 128 + ((li ^ (trow & 7)) << 4));
+        sraw[u][0] = v.x;
+        sraw[u][1] = v.y;
+        sraw[u][2] = v.z;
+        sraw[u][3] = v.w;
+      }
+      return;
+    }
     const int row = row0 + trow;
     const int kh16 = a.k / 16;
 #pragma unroll
@@ -251,13 +264,63 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   };
+  if (warp == 0) {
+    constexpr int kBars = kStagesD + 4 * kMaxIters + 2 + kIssuers + 1;
+    for (int i = kStagesD + lane; i < kBars; i += 32) {
+      if (i < kStagesD + 2 * kMaxIters) mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4);
+      else if (i < kStagesD + 4 * kMaxIters)
+        mbar_init(&sh.afree[(i - kStagesD - 2 * kMaxIters) >> 1][(i - kStagesD) & 1], 1);
+      else if (i == kStagesD + 4 * kMaxIters) mbar_init(&sh.xready, kRotWarps);
+      else if (i == kStagesD + 4 * kMaxIters + 1) mbar_init(&sh.dfull, kIssuers);
+      else if (i < kStagesD + 4 * kMaxIters + 2 + kIssuers) mbar_init(&sh.idone[i - kStagesD - 4 * kMaxIters - 2], 1);
+      else mbar_init(&sh.eready, 4 * kGroups);
+    }
+    if (lane == 0) {
+      mbar_init(&sh.xland, 1);
+      sh.abort_flag = 0;
+    }
+    sh.tok_max[lane] = 0u;
+    fence_mbar_init();
+  } else if (warp == 1) {
+    tmem_alloc(&sh.tmem_base, kTmemColsD);
+    tmem_relinquish();
+  }
+  if (!F8) {
+    // level-pair table: entry b (a code byte) of lane l's copy at byte
+    // 128 b + 4 l holds {256 c[b & 15], 256 c[b >> 4]} (fp16 pair).  Lane j
+    // of each warp holds level j; one 16-byte store per lane writes four
+    // entries per warp (lane l: entry 4 s + (l >> 3), copies 4 (l & 7) + 0..3),
+    // taking the two levels by shuffles.
+    const uint32_t hl = lt.h[lane & 15];
+    uint4* lw4 = reinterpret_cast<uint4*>(lut);
+#pragma unroll
+    for (int it = 0; it < (64 + kThreads / 32 - 1) / (kThreads / 32); ++it) {
+      const int s4 = warp + (kThreads / 32) * it;   // warp-uniform
+      if (s4 < 64) {
+        const int b = 4 * s4 + (lane >> 3);
+        const uint32_t lo = __shfl_sync(0xFFFFFFFFu, hl, b & 15), hi = __shfl_sync(0xFFFFFFFFu, hl, b >> 4);
+        const uint32_t v = lo | (hi << 16);
+        lw4[b * 8 + (lane & 7)] = make_uint4(v, v, v, v);
+      }
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  // All CTAs of this grid are resident once every one of them is here: the
+  // next kernel may launch now.  Its CTAs take the SMs this grid leaves free
+  // and those its CTAs release, and set up meanwhile; anything of theirs that
+  // reads this kernel's output waits in griddepcontrol.wait.
+  if (threadIdx.x == 0) pdl_launch_dependents();
+  const uint32_t tmem = sh.tmem_base;
 
   // ------------------------------------------------------------ dequant
   // Group g dequantizes iterations g, g + 3, g + 6 of the CTA into A stage
-  // li % kNA; an iteration past the first kNA reuses a stage once the MMAs of
-  // the iteration kNA before it have read it.  Before the wait (static
-  // weight) a group does the iterations that need no stage back; the rest
-  // after the rotation.
+  // li % kNS (tensor memory for the first kNA, shared memory past them); an
+  // iteration past the first kNS reuses a stage once the MMAs of the
+  // iteration kNS before it have read it.  Before the wait (static weight) a
+  // group does the iterations that need no stage back; the rest after the
+  // rotation.
   uint32_t ff = 0u;   // {2^-e, 2^-e}: this thread's row exponent (see below)
   int dq_done = 0;    // iterations of this group dequantized so far
   auto dq_exponent = [&]() {
@@ -294,7 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (;;) {
       const int li = g + kGroups * dq_done;
       if (li >= li_end || li >= cnt) return true;
-      const int sa = li % kNA;
+      const int sa = li % kNS;
       const uint32_t a_stage = tmem + kACol0 + sa * kAColsD;
       if (!wwait(&sh.full[li], 0, abortp)) return false;
       const uint8_t* cb = smem + li * kTile + trow * (F8 ? 128 : 64);
@@ -306,7 +369,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        if (li >= kNA && !wwait(&sh.afree[sa][h], ((li / kNA) - 1) & 1, abortp)) return false;
+        if (li >= kNS && !wwait(&sh.afree[sa][h], ((li / kNS) - 1) & 1, abortp)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kb2 = 0; kb2 < 2; ++kb2) {
@@ -335,10 +398,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             dq_half(c.x, c.y, prmt(sr[kb], 0u, 0x1010u), lut_lane, o);
             dq_half(c.z, c.w, prmt(sr[kb], 0u, 0x3232u), lut_lane, o + 8);
           }
-          tmem_st16(a_stage + lane_base + 16 * kb, o);
+          if (kNS > kNA && sa >= kNA) {
+            // shared-memory stage, the layout a TMA copy with 128-byte
+            // swizzle would give: half h [128 rows][128 B], 8-row groups
+            // 1024 B apart, 16-byte chunk c of row t at c ^ (t & 7)
+            uint8_t* at = atiles + (sa - kNA) * kATileBytes + h * (kATileBytes / 2) + (trow >> 3) * 1024 +
+                          (trow & 7) * 128;
+#pragma unroll
+            for (int j = 0; j < 4; ++j)
+              *reinterpret_cast<uint4*>(at + (((4 * kb2 + j) ^ (trow & 7)) << 4)) =
+                  make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
+          } else {
+            tmem_st16(a_stage + lane_base + 16 * kb, o);
+          }
         }
-        tmem_wait_st();
-        tc_fence_before();
+        if (kNS > kNA && sa >= kNA) {
+          fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
+        } else {
+          tmem_wait_st();
+          tc_fence_before();
+        }
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.afull[sa][h]);
       }
@@ -349,10 +428,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (stat && dq_group >= 0) {
     load_scales();
     dq_exponent();
-    dq_ok = dq_run(kNA);
+    dq_ok = dq_run(kNS);
   }
 
-  if (!stat && dq_group >= 0 && !F8 && row0 + trow < a.n) {
+  if (!stat && dq_group >= 0 && !sc_tma && !F8 && row0 + trow < a.n) {
     // the scales this thread will load after the wait, pulled into L2 now
     const uint16_t* sp0 = a.scales + static_cast<int64_t>(row0 + trow) * (a.k / 16);
     for (int u = 0; u < 3; ++u) {
@@ -362,107 +441,136 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   pdl_wait();
-  if (!stat && warp == kProducerWarp && lane == 0)
-    for (int li = 0; li < cnt; ++li) issue_codes(li);
+  // The x producer (lane 0 of warp 16, which has nothing to do before the
+  // wait): the x tiles, and a weight not flagged static.
+  if (warp == kHiWarp && lane == 0) {
+    mbar_arrive_expect_tx(&sh.xland, static_cast<uint32_t>(2 * cnt * kHalf));
+    for (int u = 0; u < 2 * cnt; ++u) tma_load_2d(btiles + u * kHalf, &tm_x, &sh.xland, (2 * it0 + u) * 64, 0);
+    if (!stat) issue_weight();
+  }
   if (!stat && dq_group >= 0) load_scales();
 
   // ------------------------------------------------------------ x rotation
-  // The eight warps that do not dequantize (0-3 and 16-19) rotate x, so the
-  // dequant warps never hold it up: rotation warp r takes tokens r and r + 8
-  // (and r + 16, r + 24 at NB == 2), loading both tokens' slices before
-  // rotating either.  Lane l owns the 32-slice at k = 128 it0 + 32 l of a
-  // token (slices past the CTA's range are not written; slices past k are
-  // zero).  Signs flip bf16 sign bits; the butterfly runs in registers in the
-  // fixed stage order; e puts the token's largest |x'| in [2^13, 2^14) (fp16
-  // cannot overflow); x' 2^-e is rounded to fp16 and stored in the B tile
-  // layout the MMA reads (K-major rows of 128 B, 8-row groups 1024 B apart,
-  // 16-byte chunks XOR-swizzled by row).
+  // x came by TMA straight into the B tiles: half tile u = 2 li + h holds the
+  // 16 nb tokens' 64 k of iteration li, half h, as bf16 in the layout the MMA
+  // reads (K-major rows of 128 B, 8-row groups 1024 B apart, 16-byte chunks
+  // XOR-swizzled by row; tokens past m and k past the end are zero).  A
+  // 32-slice of a token is four chunks of one row, so it is rotated in place:
+  // bf16 in, fp16 x' 2^-e out, the same bytes.  The eight warps that do not
+  // dequantize (0-3 and 16-19) take the half tiles round-robin; lane l takes
+  // the slice at chunks 4 (l >> 4) + 0..3 of token l & 15 (and of token
+  // 16 + (l & 15) at nb = 2), so the eight lanes of a quarter warp touch
+  // eight different chunk positions: no bank conflicts.  The scale 2^e of a
+  // token is common to its whole k range in the CTA (one accumulator): a
+  // first pass takes max |x| per token (shared-memory atomic max, then a
+  // barrier of the rotation warps), and e puts 5.66 max |x| >= sqrt(32)
+  // max |x| -- a bound on |x'|, each x' being r = 1/sqrt(32) times a sum of
+  // 32 signed x -- in [2^13, 2^14), so fp16 cannot overflow.  Signs flip bf16
+  // sign bits; the butterfly runs in registers in the fixed stage order.
   const int rot = warp < 4 ? warp : ((warp >= kHiWarp && warp < kHiWarp + 4) ? warp - kHiWarp + 4 : -1);
   if (rot >= 0) {
-    const int nsl = cnt * 4;
-    const float r = __uint_as_float(0x3E3504F3u);
-    const int kk = (it0 * 4 + lane) * 32;   // first k of this lane's slice
-#pragma unroll 1
-    for (int round = 0; round < NB; ++round) {
-      uint4 raw[2][4];
+    const bool xok = wwait(&sh.xland, 0, abortp);
+    const int nunits = 2 * cnt;
+    const int tl = lane & 15, c0 = (lane >> 4) * 4;
+    if (xok) {
+      uint32_t m16[NB];
 #pragma unroll
-      for (int t = 0; t < 2; ++t) {
-        const int tk = rot + 8 * t + 16 * round;
-        const bool live = lane < nsl && tk < a.m && kk < a.k;
-        const uint4* src = reinterpret_cast<const uint4*>(a.x + static_cast<int64_t>(tk) * a.k + kk);
+      for (int rr = 0; rr < NB; ++rr) m16[rr] = 0u;
+      for (int u = rot; u < nunits; u += kRotWarps) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) raw[t][q] = live ? __ldcg(src + q) : make_uint4(0u, 0u, 0u, 0u);
-      }
-#pragma unroll 1
-      for (int t = 0; t < 2; ++t) {
-      const int tk = rot + 8 * t + 16 * round;
-      float v[32];
+        for (int rr = 0; rr < NB; ++rr) {
+          const int t = tl + 16 * rr;
+          const uint8_t* rowp = btiles + u * kHalf + (t >> 3) * 1024 + (t & 7) * 128;
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const uint4 w4 = t ? raw[1][q] : raw[0][q];   // (L2: x is the previous kernel's output)
-        const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          const uint32_t sw = F8 ? ww[e] : (ww[e] ^ a.x_sign[4 * q + e]);
-          v[8 * q + 2 * e] = __uint_as_float(sw << 16);
-          v[8 * q + 2 * e + 1] = __uint_as_float(sw & 0xFFFF0000u);
+          for (int q = 0; q < 4; ++q) {
+            const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + (((c0 + q) ^ (t & 7)) << 4));
+            m16[rr] = __vmaxu2(m16[rr], w4.x & 0x7FFF7FFFu);
+            m16[rr] = __vmaxu2(m16[rr], w4.y & 0x7FFF7FFFu);
+            m16[rr] = __vmaxu2(m16[rr], w4.z & 0x7FFF7FFFu);
+            m16[rr] = __vmaxu2(m16[rr], w4.w & 0x7FFF7FFFu);
+          }
         }
       }
-      if (!F8) {
 #pragma unroll
-        for (int h = 1; h < 32; h <<= 1) {
+      for (int rr = 0; rr < NB; ++rr) {
+        uint32_t mb = m16[rr] >> 16 > (m16[rr] & 0xFFFFu) ? m16[rr] >> 16 : (m16[rr] & 0xFFFFu);
+        const uint32_t ob = __shfl_xor_sync(0xFFFFFFFFu, mb, 16);   // the token's other slice position
+        mb = mb > ob ? mb : ob;
+        if (lane < 16 && mb != 0u) atomicMax(&sh.tok_max[tl + 16 * rr], mb << 16);
+      }
+    }
+    named_bar_sync(1, kRotWarps * 32);
+    if (xok) {
+      const float r = __uint_as_float(0x3E3504F3u);
+#pragma unroll 1
+      for (int u = rot; u < nunits; u += kRotWarps) {
+#pragma unroll 1
+        for (int rr = 0; rr < NB; ++rr) {
+          const int t = tl + 16 * rr;
+          const float tmx = __uint_as_float(sh.tok_max[t]);   // max |x| (NaN, Inf: bits above Inf)
+          const float bound = F8 ? tmx : __fmul_rn(tmx, 5.66f);
+          int e = 0;
+          if (bound > 0.0f && isfinite(bound)) {
+            int ex;
+            frexpf(bound, &ex);   // bound in [2^(ex-1), 2^ex)
+            e = ex - 14;
+            e = e < -100 ? -100 : (e > 100 ? 100 : e);
+          }
+          if (rot == 0 && u == 0 && lane < 16) sh.row_scale[t] = ldexpf(1.0f, e);
+          const float rd = F8 ? ldexpf(1.0f, -e) : __fmul_rn(r, ldexpf(1.0f, -e));   // exact
+          uint8_t* rowp = btiles + u * kHalf + (t >> 3) * 1024 + (t & 7) * 128;
+          float v[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            if (!(j & h)) {
-              const float p = v[j], q = v[j + h];
-              v[j] = __fadd_rn(p, q);
-              v[j + h] = __fsub_rn(p, q);
+          for (int q = 0; q < 4; ++q) {
+            const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + (((c0 + q) ^ (t & 7)) << 4));
+            const uint32_t ww[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+            for (int e2 = 0; e2 < 4; ++e2) {
+              const uint32_t sw = F8 ? ww[e2] : (ww[e2] ^ a.x_sign[4 * q + e2]);
+              v[8 * q + 2 * e2] = __uint_as_float(sw << 16);
+              v[8 * q + 2 * e2 + 1] = __uint_as_float(sw & 0xFFFF0000u);
             }
           }
-        }
-      }
-      float mx = 0.0f;
+          if (!F8) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) mx = fmaxf(mx, fabsf(v[i]));
+            for (int h = 1; h < 32; h <<= 1) {
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-      int e = 0;
-      const float bound = F8 ? mx : __fmul_rn(mx, r);   // the token's largest |x'| (|x| for the fp8 cache)
-      if (bound > 0.0f && isfinite(bound)) {
-        int ex;
-        frexpf(bound, &ex);   // bound in [2^(ex-1), 2^ex)
-        e = ex - 14;
-        e = e < -100 ? -100 : (e > 100 ? 100 : e);
-      }
-      if (lane == 0) sh.row_scale[tk] = ldexpf(1.0f, e);
-      const float rd = F8 ? ldexpf(1.0f, -e) : __fmul_rn(r, ldexpf(1.0f, -e));   // exact
-      if (lane < nsl) {
-        const int li = lane >> 2, h = (lane >> 1) & 1, c0 = (lane & 1) * 4;
-        uint8_t* rowp = btiles + (li * 2 + h) * kHalf + (tk >> 3) * 1024 + (tk & 7) * 128;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t hw[4];
-#pragma unroll
-          for (int c2 = 0; c2 < 4; ++c2) {
-            const __half2 hh = __floats2half2_rn(__fmul_rn(v[8 * q + 2 * c2], rd), __fmul_rn(v[8 * q + 2 * c2 + 1], rd));
-            hw[c2] = *reinterpret_cast<const uint32_t*>(&hh);
+              for (int j = 0; j < 32; ++j) {
+                if (!(j & h)) {
+                  const float p = v[j], q = v[j + h];
+                  v[j] = __fadd_rn(p, q);
+                  v[j + h] = __fsub_rn(p, q);
+                }
+              }
+            }
           }
-          *reinterpret_cast<uint4*>(rowp + (((c0 + q) ^ (tk & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            uint32_t hw[4];
+#pragma unroll
+            for (int c2 = 0; c2 < 4; ++c2) {
+              const __half2 hh = __floats2half2_rn(__fmul_rn(v[8 * q + 2 * c2], rd), __fmul_rn(v[8 * q + 2 * c2 + 1], rd));
+              hw[c2] = *reinterpret_cast<const uint32_t*>(&hh);
+            }
+            *reinterpret_cast<uint4*>(rowp + (((c0 + q) ^ (t & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          }
         }
-      }
       }
     }
     fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
     __syncwarp();
     if (lane == 0 && !(a.test_withhold && rot == 7)) mbar_arrive(&sh.xready);
+    // the x producer: on an abort, every copy it or the weight producer issued lands before exit
+    if (warp == kHiWarp && lane == 0 && *abortp) {
+      for (int li = 0; li < cnt; ++li) drain(&sh.full[li], 0);
+      if (sc_tma) drain(&sh.sfull, 0);
+      drain(&sh.xland, 0);
+    }
   }
 
   if (dq_group >= 0) {
     if (!stat) dq_exponent();
     if (dq_ok) dq_run(kMaxIters);
-    // the producer (every tile was issued above): on an abort, let them land before exit
-    if (warp == kProducerWarp && lane == 0 && *abortp)
-      for (int li = 0; li < cnt; ++li) drain(&sh.full[li], 0);
   } else if (((warp >= 1 && warp <= kGroups) || warp >= kFirstHiIssuerWarp) && lane == 0) {
     // ------------------------------------------------------------ MMA issue
     // Issuer (g, h): the 4 MMAs of half h of each of group g's iterations,
@@ -476,18 +584,26 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = mbar_wait(&sh.xready, 0, abortp);
     int use = 0;
     for (int li = g; ok && li < cnt; li += kGroups, ++use) {
-      const int sa = li % kNA;
+      const int sa = li % kNS;
       const uint32_t a_stage = tmem + kACol0 + sa * kAColsD;
-      if (!mbar_wait(&sh.afull[sa][h], (li / kNA) & 1, abortp)) {
+      if (!mbar_wait(&sh.afull[sa][h], (li / kNS) & 1, abortp)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint64_t bdesc = sdesc_k128(smem_u32(btiles + (li * 2 + h) * kHalf));
+      if (kNS > kNA && sa >= kNA) {
+        const uint64_t adesc = sdesc_k128(smem_u32(atiles + (sa - kNA) * kATileBytes + h * (kATileBytes / 2)));
 #pragma unroll
-      for (int kk = 0; kk < 4; ++kk)
-        mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
-               (use == 0 && kk == 0) ? 0u : 1u);
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(acc, adesc + static_cast<uint64_t>(2 * kk), bdesc + static_cast<uint64_t>(2 * kk), idesc,
+                 (use == 0 && kk == 0) ? 0u : 1u);
+      } else {
+#pragma unroll
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
+                 (use == 0 && kk == 0) ? 0u : 1u);
+      }
       mma_commit(&sh.afree[sa][h]);
     }
     if (use > 0) mma_commit(&sh.dfull);
@@ -503,12 +619,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     // each scaled back by its row exponent, then by the token's 2^e and the
     // level factor (TQ4_1S) or the row's scale (fp8 cache) -- all exact but
     // the last.  (xready also orders the token scales the rotation wrote.)
+    // (the owner and local row of this thread's row, and the rows this CTA
+    // owns, before the waits)
+    const int q_own = (trow * split) >> 7;
+    const int rpc = (128 + split - 1) / split;
+    const int tl_own = trow - (q_own * 128 + split - 1) / split;
+    if (threadIdx.x == 0) {
+      const int r0 = (rank * 128 + split - 1) / split;
+      sh.own[0] = rpc;
+      sh.own[1] = r0;
+      sh.own[2] = ((rank + 1) * 128 + split - 1) / split - r0;
+    }
     int ok = 0;
     if (lane == 0)
       ok = (mbar_wait(&sh.xready, 0, abortp) && mbar_wait(&sh.eready, 0, abortp) && mbar_wait(&sh.dfull, 0, abortp))
                ? 1
                : 0;
-    ok = __shfl_sync(0xFFFFFFFFu, ok, 0);
+    ok = __shfl_sync(0xFFFFFFFFu, ok, 0) && !*abortp;   // (a timed-out role: no output)
     tc_fence_after();
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int ngroups = cnt < kGroups ? cnt : kGroups;   // groups (and their two accumulators) with work
@@ -534,14 +661,13 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], __fmul_rn(sh.row_scale[16 * c + j], wsc));
         if (split > 1) {
-          // row trow goes to the CTA that owns it: [source rank][row - owner's first row][token]
-          const int q = (trow * split) >> 7;
-          const int rpc = (128 + split - 1) / split;
-          const int tl = trow - (q * 128 + split - 1) / split;
-          const uint32_t dst = smem_u32(red) + static_cast<uint32_t>(((rank * rpc + tl) * 16 * NB + 16 * c) * 4);
+          // row trow goes to the CTA that owns it: [source rank][row - owner's
+          // first row][16 nb tokens], its 4-token groups swizzled (red_pos)
+          const uint32_t dst = smem_u32(red) + static_cast<uint32_t>((rank * rpc + tl_own) * 16 * NB * 4);
 #pragma unroll
           for (int j = 0; j < 16; j += 4)
-            st_dsmem_v4(dst + 4u * j, static_cast<uint32_t>(q), v[j], v[j + 1], v[j + 2], v[j + 3]);
+            st_dsmem_v4(dst + 16u * static_cast<uint32_t>(red_pos<NB>(tl_own, 4 * c + j / 4)),
+                        static_cast<uint32_t>(q_own), v[j], v[j + 1], v[j + 2], v[j + 3]);
         } else {
           const int row = row0 + trow;
           if (row < a.n) {
@@ -565,17 +691,31 @@ __global__ void __launch_bounds__(kThreads, 1)
     // CTA's shared memory after it.
     cluster_sync_all();
     if (!sh.abort_flag) {
-      const int rpc = (128 + split - 1) / split;
-      const int r0 = (rank * 128 + split - 1) / split, r1 = ((rank + 1) * 128 + split - 1) / split;
-      const int nrow = r1 - r0;
-      const float* rb = reinterpret_cast<const float*>(red);
-      for (int idx = threadIdx.x; idx < nrow * a.m; idx += kThreads) {
-        const int j = idx / nrow, tl = idx - j * nrow;
-        const int row = row0 + r0 + tl;
-        if (row >= a.n) continue;
-        float acc = 0.0f;
-        for (int q = 0; q < split; ++q) acc = __fadd_rn(acc, rb[(q * rpc + tl) * 16 * NB + j]);
-        a.y[static_cast<int64_t>(j) * a.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(acc));
+      // thread -> (local row tl, 4-token group gi), lanes along rows: the
+      // float4 reads are free of bank conflicts and the stores of one token
+      // are coalesced; partials summed in source-rank order
+      constexpr int kG = 4 * NB;   // 4-token groups per row
+      const int rpc_own = sh.own[0], r0_own = sh.own[1], nrow_own = sh.own[2];
+      const int idx = threadIdx.x;
+      const int tl = (idx & 31) + 32 * ((idx >> 5) / kG), gi = (idx >> 5) % kG;
+      if (tl < nrow_own && 4 * gi < a.m) {
+        const int row = row0 + r0_own + tl;
+        float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        const float* rb = reinterpret_cast<const float*>(red) + 4 * red_pos<NB>(tl, gi);
+        for (int q = 0; q < split; ++q) {
+          const float4 p = *reinterpret_cast<const float4*>(rb + (q * rpc_own + tl) * 16 * NB);
+          acc.x = __fadd_rn(acc.x, p.x);
+          acc.y = __fadd_rn(acc.y, p.y);
+          acc.z = __fadd_rn(acc.z, p.z);
+          acc.w = __fadd_rn(acc.w, p.w);
+        }
+        if (row < a.n) {
+          const float av[4] = {acc.x, acc.y, acc.z, acc.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+            if (4 * gi + u < a.m)
+              a.y[static_cast<int64_t>(4 * gi + u) * a.n + row] = __bfloat16_as_ushort(__float2bfloat16_rn(av[u]));
+        }
       }
     }
   }
@@ -583,7 +723,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 template <int NB, bool F8>
-cudaError_t launch_decode_nb(const void* tm_codes, const DecodeArgs& a, cudaStream_t st) {
+cudaError_t launch_decode_nb(const void* tm_codes, const void* tm_x, const void* tm_scales, const DecodeArgs& a,
+                             cudaStream_t st) {
   static bool attr_set = false;
   const int smem = smem_total(NB, F8);
   if (!attr_set) {
@@ -619,7 +760,10 @@ cudaError_t launch_decode_nb(const void* tm_codes, const DecodeArgs& a, cudaStre
     cfg.numAttrs = 2;
   }
   const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);
-  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NB, F8>, m0, a, lt);
+  const CUtensorMap& m1 = *static_cast<const CUtensorMap*>(tm_x);
+  // (no scales map: any valid map stands in; the kernel does not read it)
+  const CUtensorMap& m2 = *static_cast<const CUtensorMap*>(a.scales_tma ? tm_scales : tm_codes);
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, decode_kernel<NB, F8>, m0, m1, m2, a, lt);
   if (e != cudaSuccess) return e;
   note_launches(1);
   return cudaGetLastError();
@@ -658,9 +802,13 @@ size_t decode_smem_bytes(int nb, bool f8) {
                                      : (f8 ? smem_total(2, true) : smem_total(2, false)));
 }
 
-cudaError_t launch_decode(const void* tm_codes, const DecodeArgs& a, cudaStream_t st) {
-  if (a.fp8) return a.nb == 1 ? launch_decode_nb<1, true>(tm_codes, a, st) : launch_decode_nb<2, true>(tm_codes, a, st);
-  return a.nb == 1 ? launch_decode_nb<1, false>(tm_codes, a, st) : launch_decode_nb<2, false>(tm_codes, a, st);
+cudaError_t launch_decode(const void* tm_codes, const void* tm_x, const void* tm_scales, const DecodeArgs& a,
+                          cudaStream_t st) {
+  if (a.fp8)
+    return a.nb == 1 ? launch_decode_nb<1, true>(tm_codes, tm_x, tm_scales, a, st)
+                     : launch_decode_nb<2, true>(tm_codes, tm_x, tm_scales, a, st);
+  return a.nb == 1 ? launch_decode_nb<1, false>(tm_codes, tm_x, tm_scales, a, st)
+                   : launch_decode_nb<2, false>(tm_codes, tm_x, tm_scales, a, st);
 }
 
 int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb, bool f8) {

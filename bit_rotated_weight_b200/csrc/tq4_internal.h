@@ -170,13 +170,18 @@ struct DecodeArgs {
   int32_t static_w;             // the weight may be read before the dependency wait
   int32_t test_withhold;        // test hook: rotation warp 7 never reports (its bounded waiters run out)
   int32_t fp8;                  // the weight is the fp8 cache (codes = E4M3 [n][k], wscale [n]), else TQ4_1S
+  int32_t scales_tma;           // TQ4_1S with k % 128 == 0: the scales come by TMA (tm_scales), else by loads
   const float* wscale;          // fp8 cache: one fp32 scale per row
   const uint16_t* x;            // bf16 [m][k]
   const uint16_t* scales;       // [n][k/16] fp16 bits
   uint16_t* y;                  // bf16 [m][n]
   uint32_t x_sign[16];          // sign mask as XOR words on bf16 pairs
 };
-cudaError_t launch_decode(const void* tm_codes, const DecodeArgs& a, cudaStream_t st);
+// tm_codes: the codes plane (or the fp8 cache); tm_x: x [m][k] bf16, box 64 x 16 nb,
+// 128-byte swizzle; tm_scales: the scales [n][k/16], box 64 x 128, 128-byte
+// swizzle (read only when a.scales_tma).
+cudaError_t launch_decode(const void* tm_codes, const void* tm_x, const void* tm_scales, const DecodeArgs& a,
+                          cudaStream_t st);
 // The split for a decode launch of `tiles` row tiles (0: the kernel does not fit).
 int choose_decode_split(int64_t tiles, int64_t k_iters, int sms, int nb, bool f8 = false);
 size_t decode_smem_bytes(int nb, bool f8);

@@ -1,14 +1,15 @@
 """The mbarrier protocol of the decode-block kernel (tq4_decode.cu), modelled
 on the CPU.
 
-The kernel's roles synchronise only through mbarriers (plus one CTA barrier
-and one cluster barrier that every thread reaches): the TMA producer's codes
-tiles (full, one stage per iteration), four-warp dequant groups filling half
-A stages (afull) -- iterations past the tensor memory's stage count reuse a
-stage once the MMAs reading it complete (afree, by tcgen05.commit) -- the
-rotation warps' xready, the dequant warps' eready, the issuers' dfull and
-idone.  Static weights are dequantized in part before the wait for the
-previous kernel.  This model runs the roles as
+The kernel's roles synchronise through mbarriers (plus one CTA barrier and
+one cluster barrier that every thread reaches, and one named barrier of the
+eight rotation warps): the weight producer's codes tiles (full, one stage per
+iteration) and scales tile (sfull), the x producer's x tiles (xland),
+four-warp dequant groups filling half A stages (afull) -- iterations past the
+tensor memory's stage count reuse a stage once the MMAs reading it complete
+(afree, by tcgen05.commit) -- the rotation warps' xready, the dequant warps'
+eready, the issuers' dfull and idone.  Static weights are requested at entry
+and dequantized in part before the wait for the previous kernel.  This model runs the roles as
 actors in random interleavings, with TMA landings and MMA completions as
 asynchronous events, for every k-range length a CTA can have (1..8
 iterations), and checks that:
@@ -19,7 +20,9 @@ iterations), and checks that:
   * with one arrival withheld (a rotation warp that never reports), the
     bounded waits run out, every role still ends, every issued TMA copy has
     landed and every issued MMA has completed before tensor memory would be
-    released -- the wind-down the kernel promises on a timeout.
+    released -- the wind-down the kernel promises on a timeout;
+  * a withheld x copy (xland never completes) also winds down, through the
+    rotation warps' named barrier.
 The arrival counts and ring depth are read from the kernel source, so a
 change there is checked as it stands."""
 import os
@@ -48,6 +51,11 @@ def a_stages(nb):
     return (TMEM_COLS - ISSUERS * 16 * nb) // 64
 
 
+def all_stages(nb):
+    # plus the shared-memory A stages (smem_a_stages() in the kernel, TQ4_1S)
+    return a_stages(nb) + (2 if nb == 1 else 0)
+
+
 def test_source_constants_and_counts():
     # the init counts and layout the model assumes, as written in the kernel
     assert (GROUPS, FIRST_DQ, TMEM_COLS) == (3, 4, 512)
@@ -61,7 +69,11 @@ def test_source_constants_and_counts():
     assert "warp < 4 ? warp : ((warp >= kHiWarp && warp < kHiWarp + 4) ? warp - kHiWarp + 4 : -1)" in SRC
     assert "mbar_init(&sh.dfull, kIssuers)" in SRC and "constexpr int kIssuers = 2 * kGroups;" in SRC
     assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
+    assert "mbar_init(&sh.xland, 1)" in SRC and "mbar_init(&sh.sfull, 1)" in SRC
+    assert "named_bar_sync(1, kRotWarps * 32)" in SRC                 # the eight rotation warps
     assert (a_stages(1), a_stages(2)) == (6, 5)
+    assert "return (nb == 1 && !f8) ? 2 : 0;" in SRC and (all_stages(1), all_stages(2)) == (8, 5)
+    assert "const int sa = li % kNS;" in SRC and "dq_ok = dq_run(kNS);" in SRC
 
 
 class Barrier:
@@ -85,9 +97,9 @@ class Timeout(Exception):
     pass
 
 
-def run(cnt, seed, withhold_xready=False, static=True, nb=1):
+def run(cnt, seed, withhold_xready=False, static=True, nb=1, withhold_x=False):
     rng = random.Random(seed)
-    na = a_stages(nb)
+    na = all_stages(nb)
     B = {}
 
     def bar(name, count):
@@ -101,6 +113,9 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
     dfull = bar("dfull", ISSUERS)
     idone = [bar(f"idone{i}", 1) for i in range(ISSUERS)]
     eready = bar("eready", 4 * GROUPS)
+    xland = bar("xland", 1)
+    sfull = bar("sfull", 1)
+    rotbar = bar("rotbar", WARPS)      # the named barrier (hardware: no timeout)
     state = {"abort": False, "landings": [], "mma": [], "issued": 0, "landed": 0, "mma_issued": 0,
              "waited": False}
 
@@ -119,13 +134,22 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
         return True
 
     def issue_all():
+        # codes tiles and the scales tile
         for li in range(cnt):
             state["issued"] += 1
             state["landings"].append(full[li])
+        state["issued"] += 1
+        state["landings"].append(sfull)
 
     def rotation(r):
         # rotation warp r (0-3: warps 0-3; 4-7: warps 16-19)
-        yield ("step", "rotate")
+        xok = yield from wait(xland, 0)
+        if xok:
+            yield ("step", "max |x|")
+        rotbar.arrive()
+        yield from wait(rotbar, 0, bounded=False)
+        if xok:
+            yield ("step", "rotate")
         if not (withhold_xready and r == 7):
             xready.arrive()
 
@@ -149,28 +173,25 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
             done[0] += 1
 
     def dequant(g, q):
-        # warp 4 + 4g + q; lane 0 of warp 4 is also the TMA producer
-        producer = (g, q) == (0, 0)
-        if producer and static:
-            issue_all()
+        # warp 4 + 4g + q; lane 0 of warp 4 is also the weight producer
+        if (g, q) == (0, 0) and static:
+            issue_all()                              # at entry
+        yield ("step", "set-up (CTA barrier)")
         done = [0]
         ok = True
         if static:
+            ok = yield from wait(sfull, 0)           # the scales tile
             yield ("step", "row exponent")
             eready.arrive()
-            ok = yield from dq_run(g, done, na)      # before the wait: stages not reused
+            if ok:
+                ok = yield from dq_run(g, done, na)  # before the wait: stages not reused
         yield ("step", "wait for the previous kernel")
-        if producer and not static:
-            issue_all()
         if not static:
+            ok = yield from wait(sfull, 0)
             yield ("step", "row exponent")
             eready.arrive()
         if ok:
             yield from dq_run(g, done, MAX_ITERS)
-        if producer and state["abort"]:
-            # every tile was issued: let them land before exit
-            for li in range(cnt):
-                yield from wait(full[li], 0, bounded=False)
 
     def issuer(g, h):
         # lane 0 of warps 1-3 (h = 0) and 17-19 (h = 1), all rotation warps
@@ -201,11 +222,27 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1):
         ok = ok and (yield from wait(eready, 0))
         ok = ok and (yield from wait(dfull, 0))
 
-    def plain_rotation():
-        # warp 16 rotates and does nothing else
+    def x_producer_rotation():
+        # warp 16: lane 0 issues the x tiles (and a weight not flagged static)
+        # after the wait, the warp rotates, and on an abort lane 0 waits for
+        # every copy to land
+        yield ("step", "wait for the previous kernel")
+        state["issued"] += 1
+        if not withhold_x:
+            state["landings"].append(xland)
+        else:
+            state["issued"] -= 1                      # the copy never completes (models a lost transfer)
+        if not static:
+            issue_all()
         yield from rotation(4)
+        if state["abort"]:
+            for li in range(cnt):
+                yield from wait(full[li], 0, bounded=False)
+            yield from wait(sfull, 0, bounded=False)
+            if not withhold_x:
+                yield from wait(xland, 0, bounded=False)
 
-    actors = [epilogue(0), plain_rotation()]
+    actors = [epilogue(0), x_producer_rotation()]
     actors += [issuer(g, h) for g in range(GROUPS) for h in range(2)]
     actors += [dequant(g, q) for g in range(GROUPS) for q in range(4)]
     # the issuers' warps 1-3 join the epilogue after their roles
@@ -267,12 +304,13 @@ def test_protocol_completes_with_exact_counts(cnt, static, nb):
     for seed in range(30):
         B, state = run(cnt, seed, static=static, nb=nb)
         assert not state["abort"], f"cnt={cnt} seed={seed}: a wait ran out in a correct run"
-        assert state["landed"] == state["issued"] == cnt
+        assert state["landed"] == state["issued"] == cnt + 2   # codes, scales, x
         assert not state["mma"] and state["mma_issued"] == 2 * cnt
         for b in B.values():
             assert b.arrived == 0, f"{b.name}: partial phase left at the end"
         assert B["xready"].phase == 1 and B["dfull"].phase == 1 and B["eready"].phase == 1
-        na = a_stages(nb)
+        assert B["xland"].phase == 1 and B["sfull"].phase == 1 and B["rotbar"].phase == 1
+        na = all_stages(nb)
         for s in range(MAX_ITERS):
             uses = len(range(s, cnt, na)) if s < na else 0
             assert B[f"afull{s}0"].phase == uses and B[f"afree{s}1"].phase == uses
@@ -287,3 +325,14 @@ def test_withheld_arrival_winds_down(cnt, static):
         assert state["landed"] == state["issued"], "a TMA copy still in flight at exit"
         assert not state["mma"], "an MMA still in flight when tensor memory is released"
         assert B["xready"].phase == 0
+
+
+@pytest.mark.parametrize("cnt", [1, 4, 8])
+@pytest.mark.parametrize("static", [True, False])
+def test_lost_x_copy_winds_down(cnt, static):
+    for seed in range(20):
+        B, state = run(cnt, seed, withhold_x=True, static=static)
+        assert state["abort"], "a lost x copy must make a wait run out"
+        assert state["landed"] == state["issued"], "a TMA copy still in flight at exit"
+        assert not state["mma"], "an MMA still in flight when tensor memory is released"
+        assert B["xready"].phase == 1 and B["rotbar"].phase == 1
