@@ -491,6 +491,7 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
       d.scales_tma = sc_tma ? 1 : 0;
       d.y = y;
       sign_xor_words(mask, d.x_sign);
+      d.sign_bits = mask;
       return cuda_rc(launch_decode(&tc, &tx, &ts, d, st));
     }
   }

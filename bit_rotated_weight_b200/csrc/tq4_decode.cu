@@ -79,6 +79,7 @@ struct DecodeShared {
   uint64_t eready;                   // every dequant thread wrote its row exponent (12 warp arrivals)
   uint64_t xland;                    // the x tiles landed (TMA bytes)
   uint64_t sfull;                    // the scales tile landed (TMA bytes)
+  uint64_t rdone;                    // the rotation MMAs completed (tensor-core rotation)
   int8_t rexp[kGroups][128];         // row exponent of each group's levels (see the dequant)
   float row_scale[kSegRows];         // 2^e of each token
   uint32_t tok_max[kSegRows];        // max |x| of each token over the CTA's k range (fp32 bits)
@@ -98,7 +99,12 @@ __host__ __device__ constexpr int off_asm(int nb, bool f8) { return off_b(f8) + 
 __host__ __device__ constexpr int off_lut(int nb, bool f8) { return off_asm(nb, f8) + smem_a_stages(nb, f8) * kATileBytes; }
 __host__ __device__ constexpr int off_sc(int nb, bool f8) { return off_lut(nb, f8) + (f8 ? 0 : kLutBytesD); }
 constexpr int kScTileBytes = 128 * 128;   // 128 rows x 64 fp16 scales (8 iterations)
-__host__ __device__ constexpr int off_red(int nb, bool f8) { return off_sc(nb, f8) + (f8 ? 0 : kScTileBytes); }
+// The rotation runs on the tensor core at 16 tokens of TQ4_1S (tc_rotation):
+// the B operand is the 64 x 64 block-diagonal matrix diag(H S, H S) in bf16.
+__host__ __device__ constexpr bool tc_rotation(int nb, bool f8) { return nb == 1 && !f8; }
+constexpr int kRotBBytes = 64 * 128;
+__host__ __device__ constexpr int off_rb(int nb, bool f8) { return off_sc(nb, f8) + (f8 ? 0 : kScTileBytes); }
+__host__ __device__ constexpr int off_red(int nb, bool f8) { return off_rb(nb, f8) + (tc_rotation(nb, f8) ? kRotBBytes : 0); }
 // (the reduction buffer holds split * ceil(128 / split) <= 135 rows)
 __host__ __device__ constexpr int smem_total(int nb, bool f8) { return off_red(nb, f8) + 136 * 16 * nb * 4 + 1024; }
 
@@ -176,7 +182,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint8_t* sctile = smem + off_sc(NB, F8);
   constexpr int kHalf = b_half_bytes(NB);
   constexpr int kAccW = 16 * NB;           // columns of one accumulator
-  constexpr int kACol0 = kIssuers * kAccW; // first A-stage column: an accumulator per (group, half)
+  constexpr int kACol0 = 0;                // A stages first, then an accumulator per (group, half)
+  constexpr int kAccCol0 = a_stages(NB) * kAColsD;
+  constexpr bool kTcRot = tc_rotation(NB, F8);
   constexpr int kNA = a_stages(NB);        // A stages in tensor memory (6 at NB == 1, 5 at NB == 2)
   constexpr int kNS = kNA + smem_a_stages(NB, F8);   // all A stages (those past kNA in shared memory)
   uint8_t* atiles = smem + off_asm(NB, F8);
@@ -277,6 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) {
       mbar_init(&sh.xland, 1);
+      mbar_init(&sh.rdone, 1);
       sh.abort_flag = 0;
     }
     sh.tok_max[lane] = 0u;
@@ -303,6 +312,35 @@ __global__ void __launch_bounds__(kThreads, 1)
         lw4[b * 8 + (lane & 7)] = make_uint4(v, v, v, v);
       }
     }
+  }
+  if (kTcRot) {
+    // The rotation's B operand: row n (output k of a 64-k half tile), column
+    // i (input k) holds H[n % 32][i % 32] s[i % 32] when n and i lie in the
+    // same 32-slice, else 0 -- H the Walsh-Hadamard matrix in natural order
+    // ((-1)^popcount(n & i)), s the signs.  bf16 +-1 and 0 are exact.  K-major,
+    // 128-byte swizzle: 8 entries (16 B) per store, chunk c of row n at c ^ (n & 7).
+    uint8_t* rb = smem + off_rb(NB, F8);
+    for (int t = threadIdx.x; t < 64 * 8; t += kThreads) {
+      const int n = t >> 3, c = t & 7;   // chunk c: inputs 8 c .. 8 c + 7
+      uint32_t w[4] = {0u, 0u, 0u, 0u};
+      if ((n >> 5) == (c >> 2)) {
+        // bit i of hb: parity of popcount((n % 32) & i), the sign of H[n][i]
+        const int nn = n & 31;
+        uint32_t hb = 0u;
+        if (nn & 1) hb ^= 0xAAAAAAAAu;
+        if (nn & 2) hb ^= 0xCCCCCCCCu;
+        if (nn & 4) hb ^= 0xF0F0F0F0u;
+        if (nn & 8) hb ^= 0xFF00FF00u;
+        if (nn & 16) hb ^= 0xFFFF0000u;
+        const uint32_t bits = ((hb ^ a.sign_bits) >> (8 * (c & 3))) & 0xFFu;
+#pragma unroll
+        for (int e2 = 0; e2 < 4; ++e2)
+          w[e2] = 0x3F803F80u | (((bits >> (2 * e2)) & 1u) << 15) | (((bits >> (2 * e2 + 1)) & 1u) << 31);
+      }
+      *reinterpret_cast<uint4*>(rb + (n >> 3) * 1024 + (n & 7) * 128 + ((c ^ (n & 7)) << 4)) =
+          make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    fence_proxy_async_smem();
   }
   tc_fence_before();
   __syncthreads();
@@ -468,7 +506,101 @@ __global__ void __launch_bounds__(kThreads, 1)
   // 32 signed x -- in [2^13, 2^14), so fp16 cannot overflow.  Signs flip bf16
   // sign bits; the butterfly runs in registers in the fixed stage order.
   const int rot = warp < 4 ? warp : ((warp >= kHiWarp && warp < kHiWarp + 4) ? warp - kHiWarp + 4 : -1);
-  if (rot >= 0) {
+  if (rot >= 0 && kTcRot) {
+    // Tensor-core rotation (16 tokens of TQ4_1S): the x tiles as A (bf16,
+    // 128 rows = 8 half tiles x 16 tokens per block, K = 64 k) times the
+    // block-diagonal sign-folded Hadamard matrix as B give x' / r in tensor
+    // memory (the accumulators' columns, free until the main MMAs).  Rotation
+    // warp (w & 3, block w >= 16) reads row 32 (w & 3) + lane of its block:
+    // half tile 8 block + row / 16, token row % 16.
+    const bool xok = wwait(&sh.xland, 0, abortp);
+    if (warp == kHiWarp && lane == 0) {
+      if (xok) {
+        tc_fence_after();
+        const uint64_t rbd = sdesc_k128(smem_u32(smem + off_rb(NB, F8)));
+        const uint32_t idr = idesc_bf16(128, 64);
+        for (int b = 0; b < (cnt > 4 ? 2 : 1); ++b) {
+          const uint64_t ad = sdesc_k128(smem_u32(btiles + b * 8 * kHalf));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            mma_ss(tmem + kAccCol0 + 64 * b, ad + static_cast<uint64_t>(2 * kk), rbd + static_cast<uint64_t>(2 * kk),
+                   idr, kk > 0 ? 1u : 0u);
+        }
+        mma_commit(&sh.rdone);
+      } else {
+        mbar_arrive(&sh.rdone);
+      }
+    }
+    __syncwarp();
+    const int trw = (warp & 3) * 32 + lane;      // row of the block (tensor-memory lane)
+    const int blk = warp >= kHiWarp ? 1 : 0;
+    const int u = 8 * blk + (trw >> 4), t = trw & 15;
+    const bool live = xok && u < 2 * cnt;
+    uint8_t* rowp = btiles + u * kHalf + (t >> 3) * 1024 + (t & 7) * 128;
+    const bool rok = wwait(&sh.rdone, 0, abortp);
+    tc_fence_after();
+    const uint32_t taddr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kAccCol0 + 64 * blk;
+    // pass 1: max |x' / r| of the row (64 k) from tensor memory, the token's
+    // two rows of this warp combined, then a shared-memory atomic max over
+    // the warps (non-negative floats order as their bits)
+    float mx = 0.0f;
+    if (xok && rok) {
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t rv[32];
+        tmem_ld32(taddr + 32 * hh, rv);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fabsf(__uint_as_float(rv[j])));
+      }
+    }
+    if (!live) mx = 0.0f;
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
+    if (lane < 16 && mx > 0.0f) atomicMax(&sh.tok_max[t], __float_as_uint(mx));
+    named_bar_sync(1, kRotWarps * 32);
+    if (xok && rok) {
+      const float tmx = __uint_as_float(sh.tok_max[t]);
+      const float bound = __fmul_rn(tmx, __uint_as_float(0x3E3504F3u));   // the token's largest |x'|
+      int e = 0;
+      if (bound > 0.0f && isfinite(bound)) {
+        int ex;
+        frexpf(bound, &ex);   // bound in [2^(ex-1), 2^ex)
+        e = ex - 14;
+        e = e < -100 ? -100 : (e > 100 ? 100 : e);
+      }
+      if (blk == 0 && trw < 16) sh.row_scale[t] = ldexpf(1.0f, e);
+      const float rd = __fmul_rn(__uint_as_float(0x3E3504F3u), ldexpf(1.0f, -e));   // r 2^-e
+#pragma unroll
+      for (int hh = 0; hh < 2; ++hh) {
+        uint32_t rv[32];
+        tmem_ld32(taddr + 32 * hh, rv);
+        tmem_wait_ld();
+        if (live) {
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            uint32_t hw[4];
+#pragma unroll
+            for (int c2 = 0; c2 < 4; ++c2) {
+              const __half2 hh2 = __floats2half2_rn(__fmul_rn(__uint_as_float(rv[8 * j + 2 * c2]), rd),
+                                                    __fmul_rn(__uint_as_float(rv[8 * j + 2 * c2 + 1]), rd));
+              hw[c2] = *reinterpret_cast<const uint32_t*>(&hh2);
+            }
+            *reinterpret_cast<uint4*>(rowp + (((4 * hh + j) ^ (t & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          }
+        }
+      }
+    }
+    tc_fence_before();          // the tensor-memory reads, before the main MMAs reuse the columns
+    fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
+    __syncwarp();
+    if (lane == 0 && !(a.test_withhold && rot == 7)) mbar_arrive(&sh.xready);
+    if (warp == kHiWarp && lane == 0 && *abortp) {
+      for (int li = 0; li < cnt; ++li) drain(&sh.full[li], 0);
+      if (sc_tma) drain(&sh.sfull, 0);
+      drain(&sh.xland, 0);
+      drain(&sh.rdone, 0);
+    }
+  } else if (rot >= 0) {
     const bool xok = wwait(&sh.xland, 0, abortp);
     const int nunits = 2 * cnt;
     const int tl = lane & 15, c0 = (lane >> 4) * 4;
@@ -579,7 +711,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int g = warp >= kFirstHiIssuerWarp ? warp - kFirstHiIssuerWarp : warp - 1;
     const int h = warp >= kFirstHiIssuerWarp ? 1 : 0;
     const int ii = 2 * g + h;
-    const uint32_t acc = tmem + ii * kAccW;
+    const uint32_t acc = tmem + kAccCol0 + ii * kAccW;
     const uint32_t idesc = idesc_f16(128, 16 * NB);
     bool ok = mbar_wait(&sh.xready, 0, abortp);
     int use = 0;
@@ -649,8 +781,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int g = 0; g < ngroups; ++g) {
           // the group's two accumulators (its 64-k halves), one wait for both
           uint32_t r0[16], r1[16];
-          tmem_ld16(tmem + lane_base + (2 * g) * kAccW + 16 * c, r0);
-          tmem_ld16(tmem + lane_base + (2 * g + 1) * kAccW + 16 * c, r1);
+          tmem_ld16(tmem + lane_base + kAccCol0 + (2 * g) * kAccW + 16 * c, r0);
+          tmem_ld16(tmem + lane_base + kAccCol0 + (2 * g + 1) * kAccW + 16 * c, r1);
           tmem_wait_ld();
           const float rs = ldexpf(1.0f, sh.rexp[g][trow]);
 #pragma unroll

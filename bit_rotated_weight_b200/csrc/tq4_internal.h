@@ -176,6 +176,7 @@ struct DecodeArgs {
   const uint16_t* scales;       // [n][k/16] fp16 bits
   uint16_t* y;                  // bf16 [m][n]
   uint32_t x_sign[16];          // sign mask as XOR words on bf16 pairs
+  uint32_t sign_bits;           // the same mask, bit i = sign of element i of a 32-slice
 };
 // tm_codes: the codes plane (or the fp8 cache); tm_x: x [m][k] bf16, box 64 x 16 nb,
 // 128-byte swizzle; tm_scales: the scales [n][k/16], box 64 x 128, 128-byte

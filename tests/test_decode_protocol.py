@@ -71,6 +71,7 @@ def test_source_constants_and_counts():
     assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
     assert "mbar_init(&sh.xland, 1)" in SRC and "mbar_init(&sh.sfull, 1)" in SRC
     assert "named_bar_sync(1, kRotWarps * 32)" in SRC                 # the eight rotation warps
+    assert "mbar_init(&sh.rdone, 1)" in SRC and "mma_commit(&sh.rdone)" in SRC and "drain(&sh.rdone, 0)" in SRC
     assert (a_stages(1), a_stages(2)) == (6, 5)
     assert "return (nb == 1 && !f8) ? 2 : 0;" in SRC and (all_stages(1), all_stages(2)) == (8, 5)
     assert "const int sa = li % kNS;" in SRC and "dq_ok = dq_run(kNS);" in SRC
@@ -116,6 +117,7 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1, withhold_x=False):
     xland = bar("xland", 1)
     sfull = bar("sfull", 1)
     rotbar = bar("rotbar", WARPS)      # the named barrier (hardware: no timeout)
+    rdone = bar("rdone", 1)            # the rotation MMAs (16 tokens of TQ4_1S: on the tensor core)
     state = {"abort": False, "landings": [], "mma": [], "issued": 0, "landed": 0, "mma_issued": 0,
              "waited": False}
 
@@ -142,13 +144,21 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1, withhold_x=False):
         state["landings"].append(sfull)
 
     def rotation(r):
-        # rotation warp r (0-3: warps 0-3; 4-7: warps 16-19)
+        # rotation warp r (0-3: warps 0-3; 4-7: warps 16-19); lane 0 of warp
+        # 16 issues the rotation MMAs once x landed (else arrives itself)
         xok = yield from wait(xland, 0)
+        if r == 4:
+            if xok:
+                state["mma_issued"] += 1
+                state["mma"].append(rdone)
+            else:
+                rdone.arrive()
         if xok:
             yield ("step", "max |x|")
         rotbar.arrive()
         yield from wait(rotbar, 0, bounded=False)
-        if xok:
+        rok = yield from wait(rdone, 0)
+        if xok and rok:
             yield ("step", "rotate")
         if not (withhold_xready and r == 7):
             xready.arrive()
@@ -241,6 +251,7 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1, withhold_x=False):
             yield from wait(sfull, 0, bounded=False)
             if not withhold_x:
                 yield from wait(xland, 0, bounded=False)
+            yield from wait(rdone, 0, bounded=False)
 
     actors = [epilogue(0), x_producer_rotation()]
     actors += [issuer(g, h) for g in range(GROUPS) for h in range(2)]
@@ -305,7 +316,7 @@ def test_protocol_completes_with_exact_counts(cnt, static, nb):
         B, state = run(cnt, seed, static=static, nb=nb)
         assert not state["abort"], f"cnt={cnt} seed={seed}: a wait ran out in a correct run"
         assert state["landed"] == state["issued"] == cnt + 2   # codes, scales, x
-        assert not state["mma"] and state["mma_issued"] == 2 * cnt
+        assert not state["mma"] and state["mma_issued"] == 2 * cnt + 1   # + the rotation MMAs
         for b in B.values():
             assert b.arrived == 0, f"{b.name}: partial phase left at the end"
         assert B["xready"].phase == 1 and B["dfull"].phase == 1 and B["eready"].phase == 1
