@@ -64,10 +64,6 @@ constexpr int kTmemColsD = 512;
 constexpr float kLevelScaleD = 256.0f;
 // A stages: the tensor memory beside the accumulators (16 nb columns per group)
 __host__ __device__ constexpr int a_stages(int nb) { return (kTmemColsD - kIssuers * 16 * nb) / kAColsD; }
-// A stages in shared memory (the MMA reads A from there), where it has room:
-// at 16 tokens of TQ4_1S, 6 + 2 = 8 stages hold every iteration of a CTA.
-__host__ __device__ constexpr int smem_a_stages(int nb, bool f8) { return (nb == 1 && !f8) ? 2 : 0; }
-constexpr int kATileBytes = 2 * 128 * 128;   // 128 rows x 128 k fp16: [2 halves][128 rows][128 B]
 
 struct DecodeShared {
   uint64_t full[kStagesD];           // codes tile landed (TMA bytes)
@@ -89,14 +85,14 @@ struct DecodeShared {
 };
 
 // Dynamic shared memory: codes stages | B tiles [iters][2 halves][16 nb rows x 128 B] |
-// A stages in shared memory | level table and scales tile [128 rows][64
-// scales] (TQ4_1S only) | cluster reduction buffer [split][rows per CTA][16 nb] fp32.  The fp8 cache (f8)
+// level table and scales tile [128 rows][64 scales] (TQ4_1S only) | the
+// rotation's B operand (16 tokens of TQ4_1S) | cluster reduction buffer
+// [split][rows per CTA][16 nb] fp32.  The fp8 cache (f8)
 // streams 128 B of codes per row and iteration and needs neither.
 __host__ __device__ constexpr int tile_bytes(bool f8) { return f8 ? 2 * kCodesTile : kCodesTile; }
 __host__ __device__ constexpr int b_half_bytes(int nb) { return 16 * nb * 128; }
 __host__ __device__ constexpr int off_b(bool f8) { return kStagesD * tile_bytes(f8); }
-__host__ __device__ constexpr int off_asm(int nb, bool f8) { return off_b(f8) + kMaxIters * 2 * b_half_bytes(nb); }
-__host__ __device__ constexpr int off_lut(int nb, bool f8) { return off_asm(nb, f8) + smem_a_stages(nb, f8) * kATileBytes; }
+__host__ __device__ constexpr int off_lut(int nb, bool f8) { return off_b(f8) + kMaxIters * 2 * b_half_bytes(nb); }
 __host__ __device__ constexpr int off_sc(int nb, bool f8) { return off_lut(nb, f8) + (f8 ? 0 : kLutBytesD); }
 constexpr int kScTileBytes = 128 * 128;   // 128 rows x 64 fp16 scales (8 iterations)
 // The rotation runs on the tensor core at 16 tokens of TQ4_1S (tc_rotation):
@@ -186,8 +182,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kAccCol0 = a_stages(NB) * kAColsD;
   constexpr bool kTcRot = tc_rotation(NB, F8);
   constexpr int kNA = a_stages(NB);        // A stages in tensor memory (6 at NB == 1, 5 at NB == 2)
-  constexpr int kNS = kNA + smem_a_stages(NB, F8);   // all A stages (those past kNA in shared memory)
-  uint8_t* atiles = smem + off_asm(NB, F8);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int split = a.split;
@@ -354,11 +348,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   // ------------------------------------------------------------ dequant
   // Group g dequantizes iterations g, g + 3, g + 6 of the CTA into A stage
-  // li % kNS (tensor memory for the first kNA, shared memory past them); an
-  // iteration past the first kNS reuses a stage once the MMAs of the
-  // iteration kNS before it have read it.  Before the wait (static weight) a
-  // group does the iterations that need no stage back; the rest after the
-  // rotation.
+  // li % kNA; an iteration past the first kNA reuses a stage once the MMAs of
+  // the iteration kNA before it have read it.  Before the wait (static
+  // weight) a group does the iterations that need no stage back; the rest
+  // after the rotation.  (A stages in shared memory, tried for the last two
+  // iterations, were slower: their 16-byte stores double the dequant's
+  // shared-memory traffic, which already bounds its rate.)
   uint32_t ff = 0u;   // {2^-e, 2^-e}: this thread's row exponent (see below)
   int dq_done = 0;    // iterations of this group dequantized so far
   auto dq_exponent = [&]() {
@@ -395,7 +390,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (;;) {
       const int li = g + kGroups * dq_done;
       if (li >= li_end || li >= cnt) return true;
-      const int sa = li % kNS;
+      const int sa = li % kNA;
       const uint32_t a_stage = tmem + kACol0 + sa * kAColsD;
       if (!wwait(&sh.full[li], 0, abortp)) return false;
       const uint8_t* cb = smem + li * kTile + trow * (F8 ? 128 : 64);
@@ -407,7 +402,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        if (li >= kNS && !wwait(&sh.afree[sa][h], ((li / kNS) - 1) & 1, abortp)) return false;
+        if (li >= kNA && !wwait(&sh.afree[sa][h], ((li / kNA) - 1) & 1, abortp)) return false;
         tc_fence_after();
 #pragma unroll
         for (int kb2 = 0; kb2 < 2; ++kb2) {
@@ -436,26 +431,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             dq_half(c.x, c.y, prmt(sr[kb], 0u, 0x1010u), lut_lane, o);
             dq_half(c.z, c.w, prmt(sr[kb], 0u, 0x3232u), lut_lane, o + 8);
           }
-          if (kNS > kNA && sa >= kNA) {
-            // shared-memory stage, the layout a TMA copy with 128-byte
-            // swizzle would give: half h [128 rows][128 B], 8-row groups
-            // 1024 B apart, 16-byte chunk c of row t at c ^ (t & 7)
-            uint8_t* at = atiles + (sa - kNA) * kATileBytes + h * (kATileBytes / 2) + (trow >> 3) * 1024 +
-                          (trow & 7) * 128;
-#pragma unroll
-            for (int j = 0; j < 4; ++j)
-              *reinterpret_cast<uint4*>(at + (((4 * kb2 + j) ^ (trow & 7)) << 4)) =
-                  make_uint4(o[4 * j], o[4 * j + 1], o[4 * j + 2], o[4 * j + 3]);
-          } else {
-            tmem_st16(a_stage + lane_base + 16 * kb, o);
-          }
+          tmem_st16(a_stage + lane_base + 16 * kb, o);
         }
-        if (kNS > kNA && sa >= kNA) {
-          fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
-        } else {
-          tmem_wait_st();
-          tc_fence_before();
-        }
+        tmem_wait_st();
+        tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&sh.afull[sa][h]);
       }
@@ -466,7 +445,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (stat && dq_group >= 0) {
     load_scales();
     dq_exponent();
-    dq_ok = dq_run(kNS);
+    dq_ok = dq_run(kNA);
   }
 
   if (!stat && dq_group >= 0 && !sc_tma && !F8 && row0 + trow < a.n) {
@@ -716,26 +695,18 @@ __global__ void __launch_bounds__(kThreads, 1)
     bool ok = mbar_wait(&sh.xready, 0, abortp);
     int use = 0;
     for (int li = g; ok && li < cnt; li += kGroups, ++use) {
-      const int sa = li % kNS;
+      const int sa = li % kNA;
       const uint32_t a_stage = tmem + kACol0 + sa * kAColsD;
-      if (!mbar_wait(&sh.afull[sa][h], (li / kNS) & 1, abortp)) {
+      if (!mbar_wait(&sh.afull[sa][h], (li / kNA) & 1, abortp)) {
         ok = false;
         break;
       }
       tc_fence_after();
       const uint64_t bdesc = sdesc_k128(smem_u32(btiles + (li * 2 + h) * kHalf));
-      if (kNS > kNA && sa >= kNA) {
-        const uint64_t adesc = sdesc_k128(smem_u32(atiles + (sa - kNA) * kATileBytes + h * (kATileBytes / 2)));
 #pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ss(acc, adesc + static_cast<uint64_t>(2 * kk), bdesc + static_cast<uint64_t>(2 * kk), idesc,
-                 (use == 0 && kk == 0) ? 0u : 1u);
-      } else {
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk)
-          mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
-                 (use == 0 && kk == 0) ? 0u : 1u);
-      }
+      for (int kk = 0; kk < 4; ++kk)
+        mma_ts(acc, a_stage + 32 * h + 8 * kk, bdesc + static_cast<uint64_t>(2 * kk), idesc,
+               (use == 0 && kk == 0) ? 0u : 1u);
       mma_commit(&sh.afree[sa][h]);
     }
     if (use > 0) mma_commit(&sh.dfull);

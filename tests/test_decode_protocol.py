@@ -52,8 +52,7 @@ def a_stages(nb):
 
 
 def all_stages(nb):
-    # plus the shared-memory A stages (smem_a_stages() in the kernel, TQ4_1S)
-    return a_stages(nb) + (2 if nb == 1 else 0)
+    return a_stages(nb)
 
 
 def test_source_constants_and_counts():
@@ -73,8 +72,7 @@ def test_source_constants_and_counts():
     assert "named_bar_sync(1, kRotWarps * 32)" in SRC                 # the eight rotation warps
     assert "mbar_init(&sh.rdone, 1)" in SRC and "mma_commit(&sh.rdone)" in SRC and "drain(&sh.rdone, 0)" in SRC
     assert (a_stages(1), a_stages(2)) == (6, 5)
-    assert "return (nb == 1 && !f8) ? 2 : 0;" in SRC and (all_stages(1), all_stages(2)) == (8, 5)
-    assert "const int sa = li % kNS;" in SRC and "dq_ok = dq_run(kNS);" in SRC
+    assert "const int sa = li % kNA;" in SRC and "dq_ok = dq_run(kNA);" in SRC
 
 
 class Barrier:
