@@ -75,7 +75,8 @@ struct DecodeShared {
   uint64_t eready;                   // every dequant thread wrote its row exponent (12 warp arrivals)
   uint64_t xland;                    // the x tiles landed (TMA bytes)
   uint64_t sfull;                    // the scales tile landed (TMA bytes)
-  uint64_t rdone;                    // the rotation MMAs completed (tensor-core rotation)
+  uint64_t rdone;                    // the rotation MMAs completed (tensor-core rotation; one commit per block)
+  uint64_t redfull;                  // cluster reduction: every CTA's partial rows of this CTA landed (bytes)
   int8_t rexp[kGroups][128];         // row exponent of each group's levels (see the dequant)
   float row_scale[kSegRows];         // 2^e of each token
   uint32_t tok_max[kSegRows];        // max |x| of each token over the CTA's k range (fp32 bits)
@@ -152,10 +153,15 @@ __device__ __forceinline__ int red_pos(int tl, int gi) {
   return NB == 1 ? (gi ^ ((tl >> 1) & 3)) : (gi ^ (tl & 7));
 }
 
-__device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, float a, float b, float c, float d) {
-  uint32_t remote;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(remote) : "r"(local_addr), "r"(rank));
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(remote), "f"(a), "f"(b), "f"(c), "f"(d)
+// Asynchronous 16-byte store into CTA `rank` of the cluster; its completion
+// counts the bytes on that CTA's mbarrier at the same offset as local_bar.
+__device__ __forceinline__ void st_async_v4(uint32_t local_addr, uint32_t local_bar, uint32_t rank, float a, float b,
+                                            float c, float d) {
+  uint32_t ra, rb;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(rb) : "r"(local_bar), "r"(rank));
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.v4.f32 [%0], {%1, %2, %3, %4}, [%5];" ::"r"(ra),
+               "f"(a), "f"(b), "f"(c), "f"(d), "r"(rb)
                : "memory");
 }
 
@@ -279,7 +285,14 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (lane == 0) {
       mbar_init(&sh.xland, 1);
-      mbar_init(&sh.rdone, 1);
+      mbar_init(&sh.rdone, 2);
+      mbar_init(&sh.redfull, 1);
+      // the bytes this CTA receives in the cluster reduction: its rows from
+      // every CTA of the cluster, itself included
+      if (split > 1)
+        mbar_arrive_expect_tx(&sh.redfull, static_cast<uint32_t>(split * (((rank + 1) * 128 + split - 1) / split -
+                                                                           (rank * 128 + split - 1) / split) *
+                                                                 16 * NB * 4));
       sh.abort_flag = 0;
     }
     sh.tok_max[lane] = 0u;
@@ -344,6 +357,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   // and those its CTAs release, and set up meanwhile; anything of theirs that
   // reads this kernel's output waits in griddepcontrol.wait.
   if (threadIdx.x == 0) pdl_launch_dependents();
+  // Every CTA of the cluster has initialised its barriers once all have
+  // arrived here; the epilogue waits for that before its first remote store.
+  if (split > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
   const uint32_t tmem = sh.tmem_base;
 
   // ------------------------------------------------------------ dequant
@@ -493,18 +509,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     // warp (w & 3, block w >= 16) reads row 32 (w & 3) + lane of its block:
     // half tile 8 block + row / 16, token row % 16.
     const bool xok = wwait(&sh.xland, 0, abortp);
-    if (warp == kHiWarp && lane == 0) {
-      if (xok) {
+    if ((warp == kHiWarp || warp == kHiWarp + 1) && lane == 0) {
+      // lane 0 of warp 16 issues block 0, of warp 17 block 1 (when the CTA
+      // has more than 4 iterations), each committing once to rdone
+      const int b = warp - kHiWarp;
+      if (xok && (b == 0 || cnt > 4)) {
         tc_fence_after();
         const uint64_t rbd = sdesc_k128(smem_u32(smem + off_rb(NB, F8)));
         const uint32_t idr = idesc_bf16(128, 64);
-        for (int b = 0; b < (cnt > 4 ? 2 : 1); ++b) {
-          const uint64_t ad = sdesc_k128(smem_u32(btiles + b * 8 * kHalf));
+        const uint64_t ad = sdesc_k128(smem_u32(btiles + b * 8 * kHalf));
 #pragma unroll
-          for (int kk = 0; kk < 4; ++kk)
-            mma_ss(tmem + kAccCol0 + 64 * b, ad + static_cast<uint64_t>(2 * kk), rbd + static_cast<uint64_t>(2 * kk),
-                   idr, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < 4; ++kk)
+          mma_ss(tmem + kAccCol0 + 64 * b, ad + static_cast<uint64_t>(2 * kk), rbd + static_cast<uint64_t>(2 * kk), idr,
+                 kk > 0 ? 1u : 0u);
         mma_commit(&sh.rdone);
       } else {
         mbar_arrive(&sh.rdone);
@@ -743,13 +760,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int ngroups = cnt < kGroups ? cnt : kGroups;   // groups (and their two accumulators) with work
     const float wsc = F8 ? ((row0 + trow < a.n) ? __ldcg(a.wscale + row0 + trow) : 0.0f) : 1.0f / kLevelScaleD;
-    if (ok) {
+    if (split > 1) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    // the cluster reduction counts bytes: every CTA sends all its rows, zeros
+    // when a role timed out
+    if (ok || split > 1) {
 #pragma unroll
       for (int c = 0; c < NB; ++c) {
         float v[16];
 #pragma unroll
         for (int j = 0; j < 16; ++j) v[j] = 0.0f;
-        for (int g = 0; g < ngroups; ++g) {
+        for (int g = 0; ok && g < ngroups; ++g) {
           // the group's two accumulators (its 64-k halves), one wait for both
           uint32_t r0[16], r1[16];
           tmem_ld16(tmem + lane_base + kAccCol0 + (2 * g) * kAccW + 16 * c, r0);
@@ -761,15 +781,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(r1[j]), rs));
         }
+        if (ok) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], __fmul_rn(sh.row_scale[16 * c + j], wsc));
+          for (int j = 0; j < 16; ++j) v[j] = __fmul_rn(v[j], __fmul_rn(sh.row_scale[16 * c + j], wsc));
+        }
         if (split > 1) {
           // row trow goes to the CTA that owns it: [source rank][row - owner's
           // first row][16 nb tokens], its 4-token groups swizzled (red_pos)
           const uint32_t dst = smem_u32(red) + static_cast<uint32_t>((rank * rpc + tl_own) * 16 * NB * 4);
 #pragma unroll
           for (int j = 0; j < 16; j += 4)
-            st_dsmem_v4(dst + 16u * static_cast<uint32_t>(red_pos<NB>(tl_own, 4 * c + j / 4)),
+            st_async_v4(dst + 16u * static_cast<uint32_t>(red_pos<NB>(tl_own, 4 * c + j / 4)), smem_u32(&sh.redfull),
                         static_cast<uint32_t>(q_own), v[j], v[j + 1], v[j + 2], v[j + 3]);
         } else {
           const int row = row0 + trow;
@@ -788,12 +810,29 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   if (split > 1) {
-    // Every thread of every CTA of the cluster reaches this barrier (each role
-    // runs to its end, on a timeout too), so it cannot hang; it orders the
-    // pushes above before the owners read them, and nothing touches another
-    // CTA's shared memory after it.
-    cluster_sync_all();
-    if (!sh.abort_flag) {
+    // The other warps' half of the cluster barrier (the epilogue warps passed
+    // it before their stores).  Then this CTA's rows from every CTA of the
+    // cluster: the byte count completes even when a role timed out (zeros
+    // are sent), so once it has, no other CTA writes here and this CTA may
+    // leave whenever it is done.
+    if (warp >= 4) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+    // (a bounded wait that does not give up on this CTA's abort flag: the
+    // other CTAs' stores must land before this CTA may exit)
+    int rok = 1;
+    if (lane == 0) {
+      const uint32_t addr = smem_u32(&sh.redfull);
+      const uint64_t t0 = global_timer();
+      while (!mbar_try_wait(addr, 0)) {
+        if (global_timer() - t0 > TQ_WAIT_NS) {
+          raise_status(TQ_DEV_TIMEOUT);
+          *abortp = 1;
+          rok = 0;
+          break;
+        }
+      }
+    }
+    rok = __shfl_sync(0xFFFFFFFFu, rok, 0);
+    if (rok && !sh.abort_flag) {
       // thread -> (local row tl, 4-token group gi), lanes along rows: the
       // float4 reads are free of bank conflicts and the stores of one token
       // are coalesced; partials summed in source-rank order

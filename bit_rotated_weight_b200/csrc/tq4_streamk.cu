@@ -104,7 +104,8 @@ constexpr float kLevelScale = 256.0f;
 
 struct SharedState {
   uint64_t full[kStages];      // the stage's codes and x' tiles landed
-  uint64_t done[kStages];      // the MMAs of the iteration that used this stage completed
+  uint64_t done[kStages];      // the stage may be refilled: the MMAs of the iteration that used it completed
+                               // (x' in the stage), or its four dequant warps read its codes (resident x')
   uint64_t afull[kDequantGroups][2];   // a half A stage (64 k) holds fresh levels (128 arrivals)
   uint64_t afree[kDequantGroups][2];   // the MMAs reading a half A stage completed
   uint64_t dfull[4];           // all four groups finished a portion (4 arrivals), per set
@@ -330,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     constexpr int kBars = 2 * kStages + 4 * kDequantGroups + 12 + 1 + kFusedMaxIters + 2;
     for (int i = lane; i < kBars; i += 32) {
       if (i < kStages) mbar_init(&sh.full[i], 1);
-      else if (i < 2 * kStages) mbar_init(&sh.done[i - kStages], 1);
+      else if (i < 2 * kStages) mbar_init(&sh.done[i - kStages], a.x_resident ? 4 : 1);
       else if (i < 2 * kStages + 2 * kDequantGroups) {
         const int g = i - 2 * kStages;
         mbar_init(&sh.afull[g >> 1][g & 1], 128);
@@ -698,6 +699,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_arrive(&sh.afull[wg][h]);
       }
       if (!ok) break;
+      // resident x': the MMAs read only tensor memory and the resident x', so
+      // the codes stage is free as soon as this warp has read it (the refill
+      // gets the MMAs' latency as extra lead)
+      if (a.x_resident) {
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sh.done[s]);
+      }
     }
     // a scale whose largest level overflows fp16 made some levels infinite
     const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
@@ -770,7 +778,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&sh.afree[w][h]);
         }
         if (!ok) break;
-        mma_commit(&sh.done[s]);
+        if (!resident) mma_commit(&sh.done[s]);
         started = true;
         ++use;
       }

@@ -70,7 +70,14 @@ def test_source_constants_and_counts():
     assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
     assert "mbar_init(&sh.xland, 1)" in SRC and "mbar_init(&sh.sfull, 1)" in SRC
     assert "named_bar_sync(1, kRotWarps * 32)" in SRC                 # the eight rotation warps
-    assert "mbar_init(&sh.rdone, 1)" in SRC and "mma_commit(&sh.rdone)" in SRC and "drain(&sh.rdone, 0)" in SRC
+    assert "mbar_init(&sh.rdone, 2)" in SRC
+    # the cluster reduction: asynchronous stores counted in bytes on the
+    # owner's barrier; every CTA sends all its rows (zeros after a timeout)
+    # and waits for its own with a wait that ignores its abort flag, so no
+    # store can reach a CTA that has left
+    assert "if (ok || split > 1) {" in SRC and "st_async_v4(" in SRC
+    assert "while (!mbar_try_wait(addr, 0)) {" in SRC and "wwait(&sh.redfull" not in SRC
+    assert SRC.count("barrier.cluster.arrive") == 1 and SRC.count("barrier.cluster.wait") == 2 and "mma_commit(&sh.rdone)" in SRC and "drain(&sh.rdone, 0)" in SRC
     assert (a_stages(1), a_stages(2)) == (6, 5)
     assert "const int sa = li % kNA;" in SRC and "dq_ok = dq_run(kNA);" in SRC
 
@@ -115,7 +122,7 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1, withhold_x=False):
     xland = bar("xland", 1)
     sfull = bar("sfull", 1)
     rotbar = bar("rotbar", WARPS)      # the named barrier (hardware: no timeout)
-    rdone = bar("rdone", 1)            # the rotation MMAs (16 tokens of TQ4_1S: on the tensor core)
+    rdone = bar("rdone", 2)            # the rotation MMAs (16 tokens of TQ4_1S: on the tensor core), per block
     state = {"abort": False, "landings": [], "mma": [], "issued": 0, "landed": 0, "mma_issued": 0,
              "waited": False}
 
@@ -145,8 +152,9 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1, withhold_x=False):
         # rotation warp r (0-3: warps 0-3; 4-7: warps 16-19); lane 0 of warp
         # 16 issues the rotation MMAs once x landed (else arrives itself)
         xok = yield from wait(xland, 0)
-        if r == 4:
-            if xok:
+        if r in (4, 5):
+            # lane 0 of warp 16 (block 0) and 17 (block 1, more than 4 iterations)
+            if xok and (r == 4 or cnt > 4):
                 state["mma_issued"] += 1
                 state["mma"].append(rdone)
             else:
@@ -314,7 +322,7 @@ def test_protocol_completes_with_exact_counts(cnt, static, nb):
         B, state = run(cnt, seed, static=static, nb=nb)
         assert not state["abort"], f"cnt={cnt} seed={seed}: a wait ran out in a correct run"
         assert state["landed"] == state["issued"] == cnt + 2   # codes, scales, x
-        assert not state["mma"] and state["mma_issued"] == 2 * cnt + 1   # + the rotation MMAs
+        assert not state["mma"] and state["mma_issued"] == 2 * cnt + (2 if cnt > 4 else 1)   # + the rotation MMAs
         for b in B.values():
             assert b.arrived == 0, f"{b.name}: partial phase left at the end"
         assert B["xready"].phase == 1 and B["dfull"].phase == 1 and B["eready"].phase == 1
