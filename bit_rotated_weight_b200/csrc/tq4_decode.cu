@@ -227,6 +227,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int li = 0; li < cnt; ++li) tma_prefetch_l2_3d(&tm_codes, (it0 + li) * (F8 ? 128 : 64), row0, 0);
       if (sc_tma) tma_prefetch_l2_2d(&tm_sc, it0 * 8, row0);
     }
+    // then the other barriers, first used after the set-up barrier (the
+    // producer's warp takes no part in the set-up stores below, so this
+    // serial work runs beside them)
+    for (int i = 0; i < kMaxIters; ++i) {
+      mbar_init(&sh.afull[i][0], 4);
+      mbar_init(&sh.afull[i][1], 4);
+      mbar_init(&sh.afree[i][0], 1);
+      mbar_init(&sh.afree[i][1], 1);
+    }
+    mbar_init(&sh.xready, kRotWarps);
+    mbar_init(&sh.dfull, kIssuers);
+    for (int i = 0; i < kIssuers; ++i) mbar_init(&sh.idone[i], 1);
+    mbar_init(&sh.eready, 4 * kGroups);
+    mbar_init(&sh.xland, 1);
+    mbar_init(&sh.rdone, 2);
+    mbar_init(&sh.redfull, 1);
+    // the bytes this CTA receives in the cluster reduction: its rows from
+    // every CTA of the cluster, itself included
+    if (split > 1)
+      mbar_arrive_expect_tx(&sh.redfull, static_cast<uint32_t>(split * (((rank + 1) * 128 + split - 1) / split -
+                                                                         (rank * 128 + split - 1) / split) *
+                                                               16 * NB * 4));
+    fence_mbar_init();
   }
   const int dq_group = (warp >= kFirstDqWarp && warp < kHiWarp) ? (warp - kFirstDqWarp) >> 2 : -1;
   const int trow = (warp & 3) * 32 + lane;   // tile row of this thread (dequant and epilogue)
@@ -272,31 +295,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   };
+  // the set-up stores below are shared by the warps other than the producer's
+  constexpr int kSetupWarps = kThreads / 32 - 1;
+  const int setup_warp = warp < kProducerWarp ? warp : warp - 1;
   if (warp == 0) {
-    constexpr int kBars = kStagesD + 4 * kMaxIters + 2 + kIssuers + 1;
-    for (int i = kStagesD + lane; i < kBars; i += 32) {
-      if (i < kStagesD + 2 * kMaxIters) mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4);
-      else if (i < kStagesD + 4 * kMaxIters)
-        mbar_init(&sh.afree[(i - kStagesD - 2 * kMaxIters) >> 1][(i - kStagesD) & 1], 1);
-      else if (i == kStagesD + 4 * kMaxIters) mbar_init(&sh.xready, kRotWarps);
-      else if (i == kStagesD + 4 * kMaxIters + 1) mbar_init(&sh.dfull, kIssuers);
-      else if (i < kStagesD + 4 * kMaxIters + 2 + kIssuers) mbar_init(&sh.idone[i - kStagesD - 4 * kMaxIters - 2], 1);
-      else mbar_init(&sh.eready, 4 * kGroups);
-    }
-    if (lane == 0) {
-      mbar_init(&sh.xland, 1);
-      mbar_init(&sh.rdone, 2);
-      mbar_init(&sh.redfull, 1);
-      // the bytes this CTA receives in the cluster reduction: its rows from
-      // every CTA of the cluster, itself included
-      if (split > 1)
-        mbar_arrive_expect_tx(&sh.redfull, static_cast<uint32_t>(split * (((rank + 1) * 128 + split - 1) / split -
-                                                                           (rank * 128 + split - 1) / split) *
-                                                                 16 * NB * 4));
-      sh.abort_flag = 0;
-    }
+    if (lane == 0) sh.abort_flag = 0;
     sh.tok_max[lane] = 0u;
-    fence_mbar_init();
   } else if (warp == 1) {
     tmem_alloc(&sh.tmem_base, kTmemColsD);
     tmem_relinquish();
@@ -310,9 +314,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     const uint32_t hl = lt.h[lane & 15];
     uint4* lw4 = reinterpret_cast<uint4*>(lut);
 #pragma unroll
-    for (int it = 0; it < (64 + kThreads / 32 - 1) / (kThreads / 32); ++it) {
-      const int s4 = warp + (kThreads / 32) * it;   // warp-uniform
-      if (s4 < 64) {
+    for (int it = 0; it < (64 + kSetupWarps - 1) / kSetupWarps; ++it) {
+      const int s4 = setup_warp + kSetupWarps * it;   // warp-uniform
+      if (warp != kProducerWarp && s4 < 64) {
         const int b = 4 * s4 + (lane >> 3);
         const uint32_t lo = __shfl_sync(0xFFFFFFFFu, hl, b & 15), hi = __shfl_sync(0xFFFFFFFFu, hl, b >> 4);
         const uint32_t v = lo | (hi << 16);
@@ -327,7 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ((-1)^popcount(n & i)), s the signs.  bf16 +-1 and 0 are exact.  K-major,
     // 128-byte swizzle: 8 entries (16 B) per store, chunk c of row n at c ^ (n & 7).
     uint8_t* rb = smem + off_rb(NB, F8);
-    for (int t = threadIdx.x; t < 64 * 8; t += kThreads) {
+    for (int t = setup_warp * 32 + lane; warp != kProducerWarp && t < 64 * 8; t += kSetupWarps * 32) {
       const int n = t >> 3, c = t & 7;   // chunk c: inputs 8 c .. 8 c + 7
       uint32_t w[4] = {0u, 0u, 0u, 0u};
       if ((n >> 5) == (c >> 2)) {

@@ -59,7 +59,7 @@ def test_source_constants_and_counts():
     # the init counts and layout the model assumes, as written in the kernel
     assert (GROUPS, FIRST_DQ, TMEM_COLS) == (3, 4, 512)
     assert "constexpr int kStagesD = kMaxIters;" in SRC              # one codes stage per iteration
-    assert "mbar_init(&sh.afull[(i - kStagesD) >> 1][(i - kStagesD) & 1], 4)" in SRC   # one arrival per warp
+    assert "mbar_init(&sh.afull[i][0], 4);" in SRC and "mbar_init(&sh.afull[i][1], 4);" in SRC   # one arrival per warp
     assert "mbar_init(&sh.xready, kRotWarps)" in SRC                 # one arrival per rotation warp
     assert WARPS == 8 and "constexpr int kProducerWarp = kFirstDqWarp;" in SRC
     # dequant warps 4-15, rotation warps 0-3 and 16-19
