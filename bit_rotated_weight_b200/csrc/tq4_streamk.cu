@@ -757,8 +757,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         // resident mode: the iteration's k slice of the segment's x'; else the stage's B tile
         const int kit_li = it_begin + li - tile * KI;
         const uint32_t xb = resident ? smem_u32(smem + kBOff + kit_li * 2 * 2048) : smem_u32(btile_of(s));
-        // the B tile (x') of this stage must have landed too
-        if (!mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) {
+        // the B tile (x') of this stage must have landed too (resident x':
+        // the stage holds only codes, which the dequant warps waited for --
+        // and may already be refilled, so its barrier is not waited on here)
+        if (!resident && !mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) {
           ok = false;
           break;
         }

@@ -222,3 +222,15 @@ def test_gemm_roles_and_named_barriers():
         r = _role_of(arms, env, tid // 32, tid % 32, False)
         counts[r] = counts.get(r, 0) + 1
     assert counts[len(arms) - 1] == 128   # epilogue: one thread per tensor-memory lane
+
+
+def test_streamk_resident_stage_release_has_no_second_waiter():
+    # With the resident x' a codes stage is released by the dequant warps as
+    # soon as they read it (4 arrivals), so it may be refilled before the
+    # group's issuer gets to that iteration: the issuer must not wait on the
+    # stage's `full` barrier then (its parity wait could be two phases
+    # behind).  The refill waits for the dequant warps, not the MMAs.
+    src = _read("tq4_streamk.cu")
+    assert "mbar_init(&sh.done[i - kStages], a.x_resident ? 4 : 1)" in src
+    assert "if (!resident && !mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) {" in src
+    assert "if (!resident) mma_commit(&sh.done[s]);" in src
