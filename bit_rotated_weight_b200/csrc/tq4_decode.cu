@@ -461,23 +461,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       ++dq_done;
     }
   };
-  bool dq_ok = true;
-  if (stat && dq_group >= 0) {
+  // The dequant warps read the weight only through the tiles the producers
+  // copy -- after the wait for the previous kernel when it is not flagged
+  // static -- except for the scales when they come by plain loads: only then
+  // do they wait for the previous kernel themselves.  (One call site of the
+  // dequant loop keeps the kernel's code compact.)
+  if (dq_group >= 0) {
+    if (!stat && !sc_tma) {
+      if (!F8 && row0 + trow < a.n) {
+        // the scales this thread will load after the wait, pulled into L2 now
+        const uint16_t* sp0 = a.scales + static_cast<int64_t>(row0 + trow) * (a.k / 16);
+        for (int u = 0; u < 3; ++u) {
+          const int li = dq_group + kGroups * u;
+          if (li < cnt) asm volatile("prefetch.global.L2 [%0];" ::"l"(sp0 + (it0 + li) * 8));
+        }
+      }
+      pdl_wait();
+    }
     load_scales();
     dq_exponent();
-    dq_ok = dq_run(kNA);
+    dq_run(kMaxIters);
+  } else {
+    pdl_wait();
   }
-
-  if (!stat && dq_group >= 0 && !sc_tma && !F8 && row0 + trow < a.n) {
-    // the scales this thread will load after the wait, pulled into L2 now
-    const uint16_t* sp0 = a.scales + static_cast<int64_t>(row0 + trow) * (a.k / 16);
-    for (int u = 0; u < 3; ++u) {
-      const int li = dq_group + kGroups * u;
-      if (li < cnt) asm volatile("prefetch.global.L2 [%0];" ::"l"(sp0 + (it0 + li) * 8));
-    }
-  }
-
-  pdl_wait();
   // The x producer (lane 0 of warp 16, which has nothing to do before the
   // wait): the x tiles, and a weight not flagged static.
   if (warp == kHiWarp && lane == 0) {
@@ -485,7 +491,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int u = 0; u < 2 * cnt; ++u) tma_load_2d(btiles + u * kHalf, &tm_x, &sh.xland, (2 * it0 + u) * 64, 0);
     if (!stat) issue_weight();
   }
-  if (!stat && dq_group >= 0) load_scales();
 
   // ------------------------------------------------------------ x rotation
   // x came by TMA straight into the B tiles: half tile u = 2 li + h holds the
@@ -700,10 +705,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
 
-  if (dq_group >= 0) {
-    if (!stat) dq_exponent();
-    if (dq_ok) dq_run(kMaxIters);
-  } else if (((warp >= 1 && warp <= kGroups) || warp >= kFirstHiIssuerWarp) && lane == 0) {
+  if (((warp >= 1 && warp <= kGroups) || warp >= kFirstHiIssuerWarp) && lane == 0) {
     // ------------------------------------------------------------ MMA issue
     // Issuer (g, h): the 4 MMAs of half h of each of group g's iterations,
     // into its own accumulator (single-thread issue costs ~65 cycles per
