@@ -48,9 +48,9 @@ CALLS = 16
 COPIES = 64
 PACKED_PER_CALL = N_OUT * K_IN // 2 + N_OUT * (K_IN // 16) * 2   # 10,485,760 B
 # DRAM bytes (read + write) of one decode launch: ncu dram__bytes_read.sum +
-# dram__bytes_write.sum of decode_kernel<1, 0> on this workload (10,683,392 +
+# dram__bytes_write.sum of decode_kernel<1, 0> on this workload (10,689,536 +
 # 0); set back to None whenever the kernel changes until taken again.
-TRAFFIC_PER_CALL = None
+TRAFFIC_PER_CALL = 10689536
 WORKLOAD = ("decode_linear_4096: x bf16 [16][4096] N(0,1), W 4096x4096 Student-t(5)*0.02 TQ4_1S, "
             "16 calls per step (denoising steps)")
 
