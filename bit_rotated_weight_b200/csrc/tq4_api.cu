@@ -229,6 +229,17 @@ bool map_x3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols) {
   });
 }
 
+bool map_x3d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows, uint32_t box_chunks) {
+  return cached_map(m, MapKey{4, base, rows, cols, static_cast<int64_t>(box_rows) * 1024 + box_chunks},
+                    [&](CUtensorMap* out) {
+                      const uint64_t dims[3] = {64, static_cast<uint64_t>(rows), static_cast<uint64_t>(cols / 64)};
+                      const uint64_t strides[2] = {static_cast<uint64_t>(cols * 2), 128};
+                      const uint32_t box[3] = {64, box_rows, box_chunks};
+                      return make_map(out, CU_TENSOR_MAP_DATA_TYPE_UINT16, 3, base, dims, strides, box,
+                                      CU_TENSOR_MAP_SWIZZLE_128B);
+                    });
+}
+
 // 16-bit matrix [rows][cols] row-major (bf16 or fp16), box 64 x box_rows,
 // 128-byte swizzle.
 bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
@@ -473,7 +484,10 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     if (split > 0) {
       alignas(64) CUtensorMap tc, tx, ts;
       const bool sc_tma = (w->k % 128) == 0;
-      if (!map_codes(&tc, w) || !map_bf16(&tx, x, m, w->k, static_cast<uint32_t>(16 * nb)) ||
+      const bool box3 = (w->k % 64) == 0;
+      if (!map_codes(&tc, w) ||
+          !(box3 ? map_x3d(&tx, x, m, w->k, static_cast<uint32_t>(16 * nb), 2 * kFusedMaxIters)
+                 : map_bf16(&tx, x, m, w->k, static_cast<uint32_t>(16 * nb))) ||
           (sc_tma && !map_bf16(&ts, w->scales, w->n, w->k / 16, 128)))
         return TQ_ERR_CUDA;
       DecodeArgs d{};
@@ -489,6 +503,7 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
       d.x = x;
       d.scales = w->scales;
       d.scales_tma = sc_tma ? 1 : 0;
+      d.x_box3 = box3 ? 1 : 0;
       d.y = y;
       sign_xor_words(mask, d.x_sign);
       d.sign_bits = mask;
@@ -593,7 +608,11 @@ TQ_API int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, con
     if (split > 0) {
       if (take_injected_failure()) return TQ_ERR_CUDA;
       alignas(64) CUtensorMap tc, tx;
-      if (!map_fp8(&tc, q, n, k) || !map_bf16(&tx, x, m, k, static_cast<uint32_t>(16 * nb))) return TQ_ERR_CUDA;
+      const bool box3 = (k % 64) == 0;
+      if (!map_fp8(&tc, q, n, k) ||
+          !(box3 ? map_x3d(&tx, x, m, k, static_cast<uint32_t>(16 * nb), 2 * kFusedMaxIters)
+                 : map_bf16(&tx, x, m, k, static_cast<uint32_t>(16 * nb))))
+        return TQ_ERR_CUDA;
       DecodeArgs d{};
       d.n = static_cast<int32_t>(n);
       d.k = static_cast<int32_t>(k);
@@ -605,6 +624,7 @@ TQ_API int tq4_1s_linear_fp8(const uint16_t* x, int64_t m, const uint8_t* q, con
       d.static_w = (flags & TQ_WEIGHT_STATIC) ? 1 : 0;
       d.test_withhold = withhold_arrival_hook() ? 1 : 0;
       d.fp8 = 1;
+      d.x_box3 = box3 ? 1 : 0;
       d.wscale = wscale;
       d.x = x;
       d.y = y;

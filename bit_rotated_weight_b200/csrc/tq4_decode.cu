@@ -487,8 +487,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // The x producer (lane 0 of warp 16, which has nothing to do before the
   // wait): the x tiles, and a weight not flagged static.
   if (warp == kHiWarp && lane == 0) {
-    mbar_arrive_expect_tx(&sh.xland, static_cast<uint32_t>(2 * cnt * kHalf));
-    for (int u = 0; u < 2 * cnt; ++u) tma_load_2d(btiles + u * kHalf, &tm_x, &sh.xland, (2 * it0 + u) * 64, 0);
+    if (a.x_box3) {
+      // one 3-D box: all 2 kMaxIters half tiles from this CTA's first k
+      // (those past its range land in B tiles it does not use)
+      mbar_arrive_expect_tx(&sh.xland, static_cast<uint32_t>(2 * kMaxIters * kHalf));
+      tma_load_3d(btiles, &tm_x, &sh.xland, 0, 0, 2 * it0);
+    } else {
+      mbar_arrive_expect_tx(&sh.xland, static_cast<uint32_t>(2 * cnt * kHalf));
+      for (int u = 0; u < 2 * cnt; ++u) tma_load_2d(btiles + u * kHalf, &tm_x, &sh.xland, (2 * it0 + u) * 64, 0);
+    }
     if (!stat) issue_weight();
   }
 
@@ -542,30 +549,36 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int u = 8 * blk + (trw >> 4), t = trw & 15;
     const bool live = xok && u < 2 * cnt;
     uint8_t* rowp = btiles + u * kHalf + (t >> 3) * 1024 + (t & 7) * 128;
+    // pass 1, while the rotation MMAs run: max |x| of the row (64 k, bf16 in
+    // shared memory), the token's two rows of this warp combined, then a
+    // shared-memory atomic max over the warps (non-negative values order as
+    // their bits)
+    uint32_t m16 = 0u;
+    if (live) {
+#pragma unroll
+      for (int c = 0; c < 8; ++c) {
+        const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + ((c ^ (t & 7)) << 4));
+        m16 = __vmaxu2(m16, w4.x & 0x7FFF7FFFu);
+        m16 = __vmaxu2(m16, w4.y & 0x7FFF7FFFu);
+        m16 = __vmaxu2(m16, w4.z & 0x7FFF7FFFu);
+        m16 = __vmaxu2(m16, w4.w & 0x7FFF7FFFu);
+      }
+    }
+    {
+      uint32_t mb = m16 >> 16 > (m16 & 0xFFFFu) ? m16 >> 16 : (m16 & 0xFFFFu);
+      const uint32_t ob = __shfl_xor_sync(0xFFFFFFFFu, mb, 16);
+      mb = mb > ob ? mb : ob;
+      if (lane < 16 && mb != 0u) atomicMax(&sh.tok_max[t], mb << 16);
+    }
+    named_bar_sync(1, kRotWarps * 32);
     const bool rok = wwait(&sh.rdone, 0, abortp);
     tc_fence_after();
     const uint32_t taddr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kAccCol0 + 64 * blk;
-    // pass 1: max |x' / r| of the row (64 k) from tensor memory, the token's
-    // two rows of this warp combined, then a shared-memory atomic max over
-    // the warps (non-negative floats order as their bits)
-    float mx = 0.0f;
     if (xok && rok) {
-#pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {
-        uint32_t rv[32];
-        tmem_ld32(taddr + 32 * hh, rv);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) mx = fmaxf(mx, fabsf(__uint_as_float(rv[j])));
-      }
-    }
-    if (!live) mx = 0.0f;
-    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 16));
-    if (lane < 16 && mx > 0.0f) atomicMax(&sh.tok_max[t], __float_as_uint(mx));
-    named_bar_sync(1, kRotWarps * 32);
-    if (xok && rok) {
+      // e from the bound sqrt(32) max |x| >= max |x'| (each x' is r times a
+      // sum of 32 signed x), as in the register path
       const float tmx = __uint_as_float(sh.tok_max[t]);
-      const float bound = __fmul_rn(tmx, __uint_as_float(0x3E3504F3u));   // the token's largest |x'|
+      const float bound = __fmul_rn(tmx, 5.66f);
       int e = 0;
       if (bound > 0.0f && isfinite(bound)) {
         int ex;

@@ -34,6 +34,9 @@ int check_device(int* sms_out);
 bool map_codes(CUtensorMap* m, const tq4_1s_weight* w);
 bool map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows);
 bool map_x3(CUtensorMap* m, const void* base, int64_t rows, int64_t cols);
+// x [rows][cols] (cols % 64 == 0) viewed as [cols/64][rows][64] 16-bit, box 64 x
+// box_rows x box_chunks, 128-byte swizzle.
+bool map_x3d(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows, uint32_t box_chunks);
 
 // One segment of rows of the rotated activations multiplied by one expert:
 // x = expert, y = first row, z = row count (<= 16 * nb_max <= kSegRows),
@@ -171,6 +174,7 @@ struct DecodeArgs {
   int32_t test_withhold;        // test hook: rotation warp 7 never reports (its bounded waiters run out)
   int32_t fp8;                  // the weight is the fp8 cache (codes = E4M3 [n][k], wscale [n]), else TQ4_1S
   int32_t scales_tma;           // TQ4_1S with k % 128 == 0: the scales come by TMA (tm_scales), else by loads
+  int32_t x_box3;               // k % 64 == 0: tm_x views x as [k/64][m][64] (one 3-D box per CTA), else 2-D
   const float* wscale;          // fp8 cache: one fp32 scale per row
   const uint16_t* x;            // bf16 [m][k]
   const uint16_t* scales;       // [n][k/16] fp16 bits
@@ -179,7 +183,7 @@ struct DecodeArgs {
   uint32_t sign_bits;           // the same mask, bit i = sign of element i of a 32-slice
 };
 // tm_codes: the codes plane (or the fp8 cache); tm_x: x [m][k] bf16, box 64 x 16 nb,
-// 128-byte swizzle; tm_scales: the scales [n][k/16], box 64 x 128, 128-byte
+// 128-byte swizzle (a.x_box3: the map_x3d view, box 64 x 16 nb x 16); tm_scales: the scales [n][k/16], box 64 x 128, 128-byte
 // swizzle (read only when a.scales_tma).
 cudaError_t launch_decode(const void* tm_codes, const void* tm_x, const void* tm_scales, const DecodeArgs& a,
                           cudaStream_t st);
