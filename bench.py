@@ -51,6 +51,10 @@ PACKED_PER_CALL = N_OUT * K_IN // 2 + N_OUT * (K_IN // 16) * 2   # 10,485,760 B
 # dram__bytes_write.sum of decode_kernel<1, 0> on this workload (10,689,536 +
 # 0); set back to None whenever the kernel changes until taken again.
 TRAFFIC_PER_CALL = 10689536
+# DRAM bytes of one stream-K launch of the MoE layer (an up projection, the
+# routing of seed 7: 223,318,272 read + 6,119,424 written), against about
+# 216 MB of touched packed bytes per projection.
+MOE_TRAFFIC_PER_PROJECTION = 223318272 + 6119424
 WORKLOAD = ("decode_linear_4096: x bf16 [16][4096] N(0,1), W 4096x4096 Student-t(5)*0.02 TQ4_1S, "
             "16 calls per step (denoising steps)")
 
@@ -454,7 +458,10 @@ def secondary_workloads(tq, synth, dev, pk, timed):
     gbs = (sum(touched) / 4) / (ms * 1e-3) / 1e9
     out["moe_128x_top6_m16"] = {"value": gbs, "unit": "GB/s", "ms_per_call": ms,
                                 "touched_bytes_per_call": sum(touched) / 4,
-                                "frac_of_hbm": gbs / pk["hbm_gbs"]}
+                                "frac_of_hbm": gbs / pk["hbm_gbs"],
+                                "traffic_per_projection": MOE_TRAFFIC_PER_PROJECTION,
+                                "traffic_source": "ncu dram__bytes_read.sum + dram__bytes_write.sum of one "
+                                                  "streamk_kernel launch (an up projection; routing seed 7)"}
     # quantize throughput: the up-projection expert stack (638M fp32 weights,
     # 4 B read + 0.625 B written per weight) and the decode weight
     q = {}
