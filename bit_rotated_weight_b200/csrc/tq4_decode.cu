@@ -21,25 +21,31 @@
 //   * it lets the next kernel launch as soon as all its CTAs are running: the
 //     next call's CTAs take SMs as this call's CTAs leave (and the SMs this
 //     grid does not use) and do their own set-up meanwhile;
-//   * every codes tile of the CTA is requested at once (one shared-memory
-//     stage per iteration; no ring whose refills would queue behind other
-//     traffic), before the wait when the weight is flagged static;
-//   * the dequant warps then turn as many tiles as tensor memory holds (7 of
-//     8 at 16 tokens) into A operands before the wait;
-//   * only the activation-dependent work follows the wait: eight warps that
-//     do not dequantize load x (two tokens each, coalesced 16-byte loads),
-//     rotate each lane's 32-slice in registers, take each token's scale from
-//     a warp maximum and write x' straight into the swizzled B tiles; then
+//   * every codes tile of the CTA and its scales tile are requested at entry
+//     (one shared-memory stage per iteration; no ring whose refills would
+//     queue behind other traffic), before the wait when the weight is
+//     flagged static;
+//   * the dequant warps then turn as many tiles as tensor memory holds (6 of
+//     8 at 16 tokens) into A operands, whether or not the wait has ended;
+//   * only the activation-dependent work follows the wait: x comes by TMA
+//     straight into the swizzled B tiles; at 16 tokens of TQ4_1S the tensor
+//     core multiplies it by the block-diagonal sign-folded Hadamard matrix
+//     (elsewhere eight warps butterfly each 32-slice in registers), the
+//     token scales come from max |x|, and x' is written back in place; then
 //     the MMAs, the remaining tiles and the epilogue.
 //
 // Warps (640 threads, one CTA per SM):
-//   4      lane 0: TMA producer of the codes tiles (it only issues);
+//   4      lane 0: producer of the codes and scales tiles, and of every
+//          barrier (its warp takes no part in the set-up stores);
+//   16     lane 0: producer of the x tiles (and of a weight not flagged
+//          static) after the wait; 16 and 17 lane 0 issue the rotation MMAs;
 //   1-3, 17-19  lane 0: MMA issuers, one per (dequant group, 64-k half);
-//   0-3    epilogue (thread = tile row) once the MMAs are done;
+//   0-3    epilogue (thread = tile row) once the MMAs are done, then the
+//          cluster reduction of the rows this CTA owns (all warps);
 //   4-15   three dequant groups of four warps (thread = tile row): per
 //          iteration 16 B of codes + 8 scales -> 128 fp16 levels -> tensor
 //          memory, as two 64-k halves signalled separately;
-//   0-3, 16-19  the x rotation (two tokens per warp) after the wait.
+//   0-3, 16-19  the x rotation after the wait.
 #include <mutex>
 
 #include "tq4_internal.h"
