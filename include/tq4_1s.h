@@ -167,14 +167,16 @@ size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
  * rounds it to fp16, and multiplies the rotated-domain levels
  * fp16(256 c[code]) * d (fp16 product) by x' on the tensor cores, streaming
  * the packed weight once and scaling back exactly.  For m <= 32 with a short
- * k range per CTA this is one kernel launch (the GEMM kernel rotates x
- * itself; the CTAs sharing a row tile form a cluster and reduce their
- * partial sums on chip); otherwise a rotation kernel writes x' to the
- * workspace first and a stream-K kernel splits the weight stream evenly over
- * the SMs.  Levels are finite for half-block scales d up to
- * 65504 / fp16(256 c_max) (about 93.6); a larger scale sets
- * TQ_DEV_SCALE_RANGE and makes the affected outputs non-finite.  Large m
- * dequantizes W_hat to bf16 in the workspace and runs a tensor-core GEMM.
+ * k range per CTA this is one kernel launch (the kernel rotates x itself;
+ * the CTAs sharing a row tile form a cluster and reduce their partial sums
+ * on chip), and a power of two per row and dequant group keeps the levels
+ * normal and finite for every finite half-block scale.  Otherwise a
+ * rotation kernel writes x' to the workspace first and a stream-K kernel
+ * splits the weight stream evenly over the SMs; there levels are finite for
+ * half-block scales d up to 65504 / fp16(256 c_max) (about 93.6), and a
+ * larger scale sets TQ_DEV_SCALE_RANGE and makes the affected outputs
+ * non-finite.  Large m dequantizes W_hat to bf16 in the workspace and runs a
+ * tensor-core GEMM.
  * m == 0 is a no-op. */
 int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, void* ws, size_t ws_bytes,
                   tq4_stream_t stream);
