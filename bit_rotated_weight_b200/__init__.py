@@ -67,6 +67,8 @@ _lib = None
 def load_library(path: str = LIB_PATH) -> ctypes.CDLL:
     """Load libtq4_1s.so (built by ``__graft_entry__.build()``); raise if absent."""
     global _lib
+    if _lib is not None and path == LIB_PATH:
+        return _lib
     with _lock:
         if _lib is None:
             if not os.path.exists(path):
@@ -115,12 +117,20 @@ def _check(rc: int, what: str):
         raise TQ4Error(rc, what)
 
 
+# torch's own raw accessor of the current stream (what its generated code
+# calls); the public Stream object costs several microseconds per call
+_raw_stream = getattr(torch._C, "_cuda_getCurrentRawStream", None)
+
+
 def _stream(device: torch.device | None = None):
-    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+    if _raw_stream is not None:
+        index = device.index if device is not None and device.index is not None else torch.cuda.current_device()
+        return _raw_stream(index)
+    return torch.cuda.current_stream(device).cuda_stream
 
 
 def _ptr(t: torch.Tensor | None):
-    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+    return 0 if t is None else t.data_ptr()
 
 
 @dataclass

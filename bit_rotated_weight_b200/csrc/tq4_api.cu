@@ -169,8 +169,11 @@ static bool make_map(CUtensorMap* m, CUtensorMapDataType dt, int rank, const voi
 }
 
 // Tensor maps depend only on the address, shape and box they describe, so
-// recently encoded ones are kept: a weight, or an activation buffer, used
-// call after call is encoded once.
+// encoded ones are kept: a weight, or an activation buffer, used call after
+// call is encoded once.  The cache is 4-way set associative (512 sets, the
+// set chosen by a hash of the key, round-robin replacement in a set), so a
+// model's few hundred weights and buffers all stay resident and a lookup
+// costs four compares.
 struct MapKey {
   int kind;
   const void* ptr;
@@ -178,31 +181,40 @@ struct MapKey {
   bool operator==(const MapKey& o) const {
     return kind == o.kind && ptr == o.ptr && d0 == o.d0 && d1 == o.d1 && d2 == o.d2;
   }
+  uint64_t hash() const {
+    uint64_t h = reinterpret_cast<uintptr_t>(ptr) ^ (static_cast<uint64_t>(kind) << 56);
+    for (const int64_t v : {d0, d1, d2}) h = (h ^ static_cast<uint64_t>(v)) * 0x9E3779B97F4A7C15ull;
+    return h ^ (h >> 29);
+  }
 };
 
 template <typename Encode>
 static bool cached_map(CUtensorMap* m, const MapKey& key, Encode encode) {
   struct Entry {
     MapKey key;
+    bool valid;
     CUtensorMap map;
   };
-  constexpr int kEntries = 128;
+  constexpr int kSets = 512, kWays = 4;
   static std::mutex mu;
-  static Entry cache[kEntries];
-  static int used = 0, next = 0;
+  static Entry cache[kSets][kWays];
+  static uint8_t next[kSets];
+  const int set = static_cast<int>(key.hash() & (kSets - 1));
   {
     std::lock_guard<std::mutex> g(mu);
-    for (int i = 0; i < used; ++i)
-      if (cache[i].key == key) {
-        *m = cache[i].map;
+    for (int i = 0; i < kWays; ++i)
+      if (cache[set][i].valid && cache[set][i].key == key) {
+        *m = cache[set][i].map;
         return true;
       }
   }
   if (!encode(m)) return false;
   std::lock_guard<std::mutex> g(mu);
-  cache[next] = Entry{key, *m};
-  next = (next + 1) % kEntries;
-  if (used < kEntries) ++used;
+  Entry& e = cache[set][next[set]];
+  next[set] = static_cast<uint8_t>((next[set] + 1) % kWays);
+  e.key = key;
+  e.map = *m;
+  e.valid = true;
   return true;
 }
 
@@ -359,7 +371,7 @@ static int cuda_rc(cudaError_t e) { return e == cudaSuccess ? TQ_OK : TQ_ERR_CUD
 using namespace tq4;
 
 // ==================================================================== ABI
-TQ_API int tq4_1s_version(void) { return 101; }
+TQ_API int tq4_1s_version(void) { return 102; }
 
 TQ_API const char* tq4_1s_error_string(int code) {
   switch (code) {
@@ -540,6 +552,8 @@ TQ_API int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, u
     a.m_host = static_cast<int32_t>(m);
     a.nb_max = m > 16 ? 2 : 1;
     a.scales = w->scales;
+    a.codes = w->codes;
+    a.xr = fused ? nullptr : xr;
     a.row_scale = xscale;
     if (fused) {
       a.x_raw = x;
@@ -794,6 +808,8 @@ static int moe_impl(const uint16_t* x, int64_t m, const int32_t* topk_ids, const
   a.nseg_dev = nseg;
   a.nb_max = L.nb_max;   // segments hold at most 16 * nb_max rows (the route's chunk)
   a.scales = up->scales;
+  a.codes = up->codes;
+  a.xr = xr;
   a.row_scale = xscale;
   a.epoch = next_epoch();
   a.cluster_s = 1;
@@ -814,6 +830,8 @@ static int moe_impl(const uint16_t* x, int64_t m, const int32_t* topk_ids, const
   b.row_tiles = static_cast<int32_t>(L.rt_dn);
   b.k_iters = static_cast<int32_t>((I + 127) / 128);
   b.scales = down->scales;
+  b.codes = down->codes;
+  b.xr = hr;
   b.row_scale = hscale;
   b.x_resident = (L.nb_max == 1 && I <= kResidentMaxK) ? 1 : 0;
   b.epoch = next_epoch();

@@ -892,15 +892,15 @@ __global__ void __launch_bounds__(kThreads, 1)
 template <int NB, bool F8>
 cudaError_t launch_decode_nb(const void* tm_codes, const void* tm_x, const void* tm_scales, const DecodeArgs& a,
                              cudaStream_t st) {
-  static bool attr_set = false;
+  static std::atomic<uint64_t> attr_done{0};
   const int smem = smem_total(NB, F8);
-  if (!attr_set) {
+  cudaError_t e0 = once_per_device(attr_done, [&] {
     cudaError_t e = cudaFuncSetAttribute(decode_kernel<NB, F8>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e == cudaSuccess)
       e = cudaFuncSetAttribute(decode_kernel<NB, F8>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+    return e;
+  });
+  if (e0 != cudaSuccess) return e0;
   static const LevelTableD lt = [] {
     LevelTableD t;
     const CodebookF32& cb = codebook();

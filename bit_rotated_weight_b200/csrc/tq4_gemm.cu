@@ -201,14 +201,13 @@ size_t gemm_smem_bytes() { return static_cast<size_t>(kStages) * kStageBytes + 1
 
 cudaError_t launch_gemm_bf16(const void* tm_x, const void* tm_w, uint16_t* y, int32_t m, int32_t n, int32_t k,
                              int grid, cudaStream_t st) {
-  static bool attr_set = false;
+  static std::atomic<uint64_t> attr_done{0};
   const size_t smem = gemm_smem_bytes();
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  const cudaError_t e = once_per_device(attr_done, [&] {
+    return cudaFuncSetAttribute(gemm_bf16_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                static_cast<int>(smem));
+  });
+  if (e != cudaSuccess) return e;
   gemm_bf16_kernel<<<grid, kThreads, smem, st>>>(*static_cast<const CUtensorMap*>(tm_x),
                                                  *static_cast<const CUtensorMap*>(tm_w), y, m, n, k);
   note_launches(1);

@@ -1,11 +1,28 @@
 // Internal declarations shared by the library's translation units.
 #pragma once
+#include <atomic>
 #include <cstdint>
 #include <cuda_runtime.h>
 
 #include "tq4_common.cuh"
 
 namespace tq4 {
+
+// Kernel attributes (dynamic shared-memory size, carveout) belong to each
+// device's context: `set` runs once per device, and again after a failure.
+// Two threads that race on the first call both run it (it is idempotent).
+template <typename Set>
+cudaError_t once_per_device(std::atomic<uint64_t>& done, Set set) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 64) return cudaErrorInvalidDevice;
+  const uint64_t bit = uint64_t(1) << dev;
+  if (done.load(std::memory_order_acquire) & bit) return cudaSuccess;
+  e = set();
+  if (e == cudaSuccess) done.fetch_or(bit, std::memory_order_acq_rel);
+  return e;
+}
 
 // The fp32 codebook handed to kernels by value (kernel parameter space).
 struct CodebookF32 {
@@ -109,6 +126,8 @@ struct StreamKArgs {
   const int4* segs;          // device segment list (MoE) or nullptr
   const int32_t* nseg_dev;   // device segment count (MoE) or nullptr
   const uint16_t* scales;    // [E][n][k/16]
+  const uint8_t* codes;      // [E][n][k/2] (read by the exact fallback of the epilogue only)
+  const uint16_t* xr;        // x' fp16 [rows][k] in memory (TMA-fed and grouped modes); nullptr in fused mode
   const float* row_scale;    // x' row r holds x'_r * 2^-e_r; row_scale[r] = 2^e_r (TMA-fed mode)
   const uint16_t* x_raw;     // fused mode (dense, m <= kSegRows, <= kFusedMaxIters iterations per CTA):
                              // raw bf16 x [m][k], rotated by the kernel itself; nullptr otherwise

@@ -807,15 +807,13 @@ cudaError_t launch_rotate_scaled(const uint16_t* x, int64_t k, const int32_t* ga
                                  const int32_t* rows_valid_dev, int64_t rows_valid_host, int64_t rows_alloc,
                                  uint16_t* xr, float* row_scale, uint32_t mask, cudaStream_t st) {
   if (rows_alloc <= 0) return cudaSuccess;
-  static bool attr_set = false;
-  if (!attr_set) {
-    // the stream-K kernel runs with the largest shared-memory carveout; an SM
-    // hosts CTAs of two kernels at once only if their carveouts agree
-    const cudaError_t e =
-        cudaFuncSetAttribute(rotate_scaled_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  // the stream-K kernel runs with the largest shared-memory carveout; an SM
+  // hosts CTAs of two kernels at once only if their carveouts agree
+  static std::atomic<uint64_t> attr_done{0};
+  const cudaError_t ea = once_per_device(attr_done, [] {
+    return cudaFuncSetAttribute(rotate_scaled_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+  });
+  if (ea != cudaSuccess) return ea;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(static_cast<unsigned>(rows_alloc));
   cfg.blockDim = dim3(kRotThreads);

@@ -127,6 +127,8 @@ TQ_STATIC_API int tq4_1s_linear_static(const uint16_t* x, int64_t m, const tq4_1
   a.m_host = static_cast<int32_t>(m);
   a.nb_max = m > 16 ? 2 : 1;
   a.scales = w->scales;
+  a.codes = w->codes;
+  a.xr = fused ? nullptr : xr;
   a.row_scale = xscale;
   if (fused) {
     a.x_raw = x;

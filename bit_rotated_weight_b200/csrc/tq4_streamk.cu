@@ -99,7 +99,9 @@ static_assert(kACol0 + kDequantGroups * kAColsPerStage <= kTmemCols, "tensor mem
 static_assert(kFusedMaxIters <= kStages, "fused mode gives each iteration its own stage");
 // fp16 levels carry a factor 256 (2^8): with it, half-block scales d from
 // ~2e-6 up to 65504 / fp16(256 * max level) ~ 93.6 give normal, finite fp16
-// levels.  Larger scales overflow; the dequant warps flag them.
+// levels.  A larger scale overflows its levels, which makes the row's sums
+// non-finite; the epilogue then recomputes that row's portion exactly
+// (exact_row_portion).
 constexpr float kLevelScale = 256.0f;
 
 struct SharedState {
@@ -225,12 +227,6 @@ __device__ __forceinline__ void dequant_half(uint32_t q0, uint32_t q1, uint32_t 
   }
 }
 
-__device__ __forceinline__ uint32_t hmax2(uint32_t a, uint32_t b) {
-  uint32_t d;
-  asm("max.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-  return d;
-}
-
 // 32-point Sylvester butterfly on a register array (stages h = 1..16).
 __device__ __forceinline__ void fwht32_regs_sk(float (&a)[32]) {
 #pragma unroll
@@ -282,8 +278,38 @@ __device__ __forceinline__ void epilogue_store(const StreamKArgs& a, const float
 
 struct LevelTable {
   uint32_t h[16];    // fp16 bits of 256 * levels[0..15]
-  float max_level;   // fp16(256 * levels[15]) as a float
 };
+
+// The exact path for one weight row of one tile portion, taken when the
+// row's sums came out non-finite: a level fp16(256 c) * d overflows fp16
+// for a half-block scale d above ~93.6.  Recomputes the sums of tokens
+// j0 .. j0 + ntok - 1 (ntok <= 16) over the portion's columns [kc0, kc1) on
+// the CUDA cores with fp32 levels 256 c d, in the accumulator's domain:
+// out[j] = sum_k 256 c[code_k] d_k x'[j0 + j][k].  x' comes from memory
+// (xg: row j at xg + j * k_row) or, in fused mode (xg == nullptr), from the
+// CTA's B tiles (xs: local iteration li's tile at xs + li * kXBytes, as the
+// prologue left it: row j at 128 j in each 64-k half, chunk c at c ^ (j & 7)),
+// with column kc0 in local iteration li0.  Tokens past ntok are zero.
+__device__ __noinline__ void exact_row_portion(const uint8_t* crow, const uint16_t* srow, int kc0, int kc1,
+                                               const uint16_t* xg, int k_row, const uint8_t* xs, int li0, int j0,
+                                               int ntok, const uint32_t* lvl, float* out) {
+  for (int j = 0; j < 16; ++j) out[j] = 0.0f;
+  for (int kk = kc0; kk < kc1; ++kk) {
+    const uint32_t b = crow[kk >> 1];
+    const uint32_t code = (kk & 1) ? (b >> 4) : (b & 15u);
+    const float w = __fmul_rn(__half2float(__ushort_as_half(static_cast<unsigned short>(lvl[code]))),
+                              __half2float(__ushort_as_half(srow[kk >> 4])));
+    const int li = li0 + (kk >> 7) - (kc0 >> 7), e = kk & 127, e64 = e & 63;
+    for (int j = 0; j < ntok; ++j) {
+      const int jj = j0 + j;
+      const uint16_t xb =
+          xg ? xg[static_cast<int64_t>(jj) * k_row + kk]
+             : *reinterpret_cast<const uint16_t*>(xs + li * kXBytes + (e >> 6) * kXHalfBytes + jj * 128 +
+                                                  ((((e64 >> 3) ^ (jj & 7))) << 4) + (e64 & 7) * 2);
+      out[j] = __fmaf_rn(w, __half2float(__ushort_as_half(xb)), out[j]);
+    }
+  }
+}
 
 __global__ void __launch_bounds__(kThreads, 1)
     streamk_kernel(const __grid_constant__ CUtensorMap tm_codes, const __grid_constant__ CUtensorMap tm_x,
@@ -652,17 +678,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     };
     uint32_t next_raw[4] = {first_raw[0], first_raw[1], first_raw[2], first_raw[3]};
-    uint32_t dmax = 0u;   // running max of the scales seen (fp16 pairs)
     Cursor ahead;         // the iteration whose scales are in flight
     ahead.init(it_begin + wg, KI, a.row_tiles);
     int use = 0;    // how many times this group has filled its A stage
     for (int li = wg; li < cnt; li += kDequantGroups, ++use) {
       uint32_t sraw[4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        sraw[j] = next_raw[j];
-        dmax = hmax2(dmax, sraw[j]);
-      }
+      for (int j = 0; j < 4; ++j) sraw[j] = next_raw[j];
       if (li + kDequantGroups < cnt) {
         if (fused) {
 #pragma unroll
@@ -707,9 +729,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) mbar_arrive(&sh.done[s]);
       }
     }
-    // a scale whose largest level overflows fp16 made some levels infinite
-    const float2 dm = __half22float2(*reinterpret_cast<const __half2*>(&dmax));
-    if (fmaxf(dm.x, dm.y) * lt.max_level >= 65520.0f) raise_status(TQ_DEV_SCALE_RANGE);
   } else if ((warp == 1 || warp >= kFirstIssuerWarp) && lane == 0) {
     // ------------------------------------------------------------ MMA issue
     // Issuer of group w: the iterations li = w (mod 4), in order.  Per half A
@@ -842,6 +861,29 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __uint_as_float(rr[j]));
+        }
+        {
+          // a non-finite sum: some level overflowed fp16 (a half-block scale
+          // above ~93.6), or the inputs hold an Inf or NaN; the row's portion
+          // is recomputed exactly (the latter stays non-finite, as it should).
+          // v * 0 is 0 for a finite v and NaN otherwise, so one test covers the
+          // 16 columns (a padding column only costs a needless recompute).
+          const int ntok = sg.count - 16 * c < 16 ? sg.count - 16 * c : 16;
+          float z = 0.0f;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) z = __fmaf_rn(v[j], 0.0f, z);
+          const bool bad = z != z;
+          if (bad && row < a.n) {
+            const int kc0 = (portion_first - tile_first) * 128;
+            const int kc1 = min((portion_end - tile_first) * 128, a.k);
+            const int64_t wrow = static_cast<int64_t>(sg.e) * a.n + row;
+            float ex[16];   // (its own array: v stays in registers)
+            exact_row_portion(a.codes + wrow * (a.k / 2), a.scales + wrow * (a.k / 16), kc0, kc1,
+                              a.xr ? a.xr + static_cast<int64_t>(sg.row0) * a.k : nullptr, a.k,
+                              smem + kBOff, lpf, 16 * c, ntok, lt.h, ex);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) v[j] = ex[j];
+          }
         }
         // back from the scaled domain: times 2^e / 256 per token (exact), with
         // 2^e from the prologue in fused mode (it may differ between the CTAs
@@ -1071,7 +1113,6 @@ cudaError_t launch_streamk(const void* tm_codes, const void* tm_x, const void* t
     const CodebookF32& cb = codebook();
     for (int i = 0; i < 16; ++i)
       t.h[i] = static_cast<uint32_t>(__half_as_ushort(__float2half_rn(cb.levels[i] * kLevelScale)));
-    t.max_level = __half2float(__float2half_rn(cb.levels[15] * kLevelScale));
     return t;
   }();
   const CUtensorMap& m0 = *static_cast<const CUtensorMap*>(tm_codes);

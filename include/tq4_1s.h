@@ -70,7 +70,7 @@ enum {
   TQ_DEV_TIMEOUT = 1,
   TQ_DEV_BAD_ROUTING = 2,
   TQ_DEV_NONFINITE = 4,
-  TQ_DEV_SCALE_RANGE = 8   /* linear/moe: a half-block scale above ~93.6 (see tq4_1s_linear) */
+  TQ_DEV_SCALE_RANGE = 8   /* reserved: set by no kernel since ABI 1.02 (every finite scale is handled) */
 };
 
 /* Input dtypes of tq4_1s_quantize. */
@@ -169,14 +169,15 @@ size_t tq4_1s_linear_workspace(int64_t m, const tq4_1s_weight* w);
  * the packed weight once and scaling back exactly.  For m <= 32 with a short
  * k range per CTA this is one kernel launch (the kernel rotates x itself;
  * the CTAs sharing a row tile form a cluster and reduce their partial sums
- * on chip), and a power of two per row and dequant group keeps the levels
- * normal and finite for every finite half-block scale.  Otherwise a
- * rotation kernel writes x' to the workspace first and a stream-K kernel
- * splits the weight stream evenly over the SMs; there levels are finite for
- * half-block scales d up to 65504 / fp16(256 c_max) (about 93.6), and a
- * larger scale sets TQ_DEV_SCALE_RANGE and makes the affected outputs
- * non-finite.  Large m dequantizes W_hat to bf16 in the workspace and runs a
- * tensor-core GEMM.
+ * on chip); there a power of two per row and dequant group, taken from the
+ * row's largest half-block scale, keeps the levels normal and finite for
+ * every finite scale.  Otherwise a stream-K kernel splits the weight stream
+ * evenly over the SMs (x' from a rotation kernel through the workspace, or
+ * rotated in the kernel); its levels are finite for half-block scales up to
+ * 65504 / fp16(256 c_max) (about 93.6), and where a larger scale makes a
+ * row's sums non-finite the kernel recomputes that row's part exactly on
+ * the CUDA cores (slower, same result).  Large m dequantizes W_hat to bf16
+ * in the workspace and runs a tensor-core GEMM.
  * m == 0 is a no-op. */
 int tq4_1s_linear(const uint16_t* x, int64_t m, const tq4_1s_weight* w, uint16_t* y, void* ws, size_t ws_bytes,
                   tq4_stream_t stream);

@@ -34,7 +34,7 @@ def test_library_exports_every_declared_symbol():
 
 
 def test_version_and_error_strings():
-    assert tq.tq4_1s_version() == 101
+    assert tq.tq4_1s_version() == 102
     for code in range(0, 9):
         s = tq.tq4_1s_error_string(code)
         assert s and s != "unknown error code"

@@ -226,21 +226,33 @@ def test_linear_any_finite_scale_decode_path():
     assert_close(yb[:, [9]], y_ref[:, [9]], "decode: subnormal scales")
 
 
-def test_linear_scale_beyond_fp16_level_range_flagged_stream_k():
-    # the TMA-fed stream-K path (more than 32 rows) still computes levels
-    # with a fixed factor: a row whose scales pass ~93.6 overflows, the
-    # status word says so, and every other output column is still correct
-    m, n, k, seed = 48, 256, 256, 39
+@pytest.mark.parametrize("m,n,k,seed", [
+    (48, 256, 256, 39),      # TMA-fed stream-K (two segments)
+    (48, 256, 544, 46),      # ragged k: rows of scales not 16-byte aligned
+    (16, 19072, 256, 47),    # 149 row tiles: past the decode kernel's one wave (fused
+                             # stream-K: x' only in the CTA's shared memory)
+])
+def test_linear_any_finite_scale_stream_k(m, n, k, seed):
+    # scales far above ~93.6 (one row x 20000) overflow the stream-K
+    # kernel's fp16 levels; the row's sums come out non-finite and the
+    # epilogue recomputes them exactly, so every column matches the oracle
+    # and nothing is flagged; scales far below 2e-6 (one row x 1e-5) give
+    # fp16-subnormal levels, still within the tolerance
     W = synth.normal_f32((n, k), seed, 0.02)
     W[3] *= 20000.0
+    W[9] *= 1e-5
     x = synth.activations_bf16(m, k, seed + 1)
     p, codes, scales, _ = _quantize_both(W, seed)
+    assert scales[0][3].view(np.float16).astype(np.float32).max() > 94.0
     y = tq.tq4_1s_linear(_bf16_dev(x), p)
     torch.cuda.synchronize()
-    assert tq.tq4_1s_get_status() & tq.TQ_DEV_SCALE_RANGE
+    assert tq.tq4_1s_get_status() == 0
     y_ref, _ = oracle.linear(x, codes[0], scales[0], seed)
-    keep = np.array([c for c in range(n) if c != 3])
-    assert_close(_bits(y)[:, keep], y_ref[:, keep], "stream-K with one out-of-range row")
+    yb = _bits(y)
+    keep = np.array([c for c in range(n) if c not in (3, 9)])
+    assert_close(yb[:, keep], y_ref[:, keep], "stream-K: ordinary rows")
+    assert_close(yb[:, [3]], y_ref[:, [3]], "stream-K: scales above the unscaled fp16 level range")
+    assert_close(yb[:, [9]], y_ref[:, [9]], "stream-K: subnormal scales")
 
 
 def test_linear_shared_workspace_across_shapes_and_paths():
@@ -312,12 +324,15 @@ def test_moe_route_bad_ids_flagged():
     assert tq.tq4_1s_get_status() & tq.TQ_DEV_BAD_ROUTING
 
 
-def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False, x_std=1.0, zero_rows=(), ids=None):
+def _moe_case(E, H, I, m, topk, seeds, dist_std=0.02, bad_ids=False, x_std=1.0, zero_rows=(), ids=None,
+              mutate=None):
     up_seed, dn_seed, x_seed, r_seed = seeds
     up = synth.normal_f32((E, I, H), up_seed, dist_std)
     dn = synth.normal_f32((E, H, I), dn_seed, dist_std)
     routed, w = synth.gumbel_topk_router(m, E, topk, r_seed)
     ids = routed if ids is None else np.ascontiguousarray(ids, np.int32)
+    if mutate is not None:
+        mutate(up, dn, ids)
     if bad_ids:
         ids[0, 1] = E + 1
     x = synth.f32_to_bf16_bits(synth.normal_f32((m, H), x_seed, x_std))
@@ -365,6 +380,41 @@ def test_moe_activation_range(x_std, w_std):
     y, y_ref, _ = _moe_case(4, 128, 96, 6, 2, (34, 35, 36, 37), dist_std=w_std, x_std=x_std)
     assert np.all(np.isfinite(y.float().cpu().numpy()))
     assert_close(_bits(y), y_ref, f"moe range x_std={x_std}")
+
+
+def test_moe_any_finite_scale():
+    # one routed expert with its whole up projection x 20000 and one down row
+    # x 20000 (half-block scales far above ~93.6), another with an up row
+    # x 1e-5 (fp16 subnormal scales): the stream-K kernel's exact recompute of
+    # the rows whose sums overflowed keeps every output finite and matching
+    # the oracle, unflagged, in both projections.  (The
+    # whole up projection is scaled, not one row: a single dominant
+    # h = bf16(relu(u)^2) would make a whole token row hinge on one bf16
+    # rounding, which the fp16 operands may legitimately flip.)  Outputs of
+    # different magnitude are compared apart: the tokens routed to the big
+    # expert (its column 2 on its own), and the other tokens.
+    routed = {}
+
+    def mutate(up, dn, ids):
+        e = routed["e"] = int(ids[0, 0])
+        routed["ids"] = ids.copy()
+        up[e] *= 20000.0
+        dn[e, 2] *= 20000.0
+        small = next(int(v) for v in ids.ravel() if int(v) != e)
+        up[small, 7] *= 1e-5
+
+    m = 16
+    y, y_ref, _ = _moe_case(8, 256, 128, m, 2, (54, 55, 56, 57), mutate=mutate)
+    assert tq.tq4_1s_get_status() == 0
+    assert np.all(np.isfinite(y.float().cpu().numpy()))
+    yb = _bits(y)
+    big = np.array([t for t in range(m) if routed["e"] in routed["ids"][t]])
+    other = np.array([t for t in range(m) if t not in big])
+    assert len(big) and len(other)
+    keep = np.array([c for c in range(256) if c != 2])
+    assert_close(yb[np.ix_(big, keep)], y_ref[np.ix_(big, keep)], "moe large scales: tokens of the big expert")
+    assert_close(yb[big][:, [2]], y_ref[big][:, [2]], "moe large scales: the big down row")
+    assert_close(yb[other], y_ref[other], "moe large scales: the other tokens")
 
 
 def test_moe_128_experts_top6_full():

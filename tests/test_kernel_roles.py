@@ -234,3 +234,20 @@ def test_streamk_resident_stage_release_has_no_second_waiter():
     assert "mbar_init(&sh.done[i - kStages], a.x_resident ? 4 : 1)" in src
     assert "if (!resident && !mbar_wait(&sh.full[s], (li / kStages) & 1, abortp)) {" in src
     assert "if (!resident) mma_commit(&sh.done[s]);" in src
+
+
+def test_streamk_overflowing_levels_fall_back_to_the_exact_path():
+    # a half-block scale above ~93.6 overflows the fp16 levels: the epilogue
+    # detects the non-finite sums (one NaN test over v * 0) and recomputes the
+    # row's portion with fp32 levels, reading x' from memory or, in fused
+    # mode, from the B tiles; no kernel raises the scale-range status any more
+    src = _read("tq4_streamk.cu")
+    assert "z = __fmaf_rn(v[j], 0.0f, z);" in src and "const bool bad = z != z;" in src
+    assert "exact_row_portion(a.codes + wrow * (a.k / 2), a.scales + wrow * (a.k / 16), kc0, kc1," in src
+    assert "a.xr ? a.xr + static_cast<int64_t>(sg.row0) * a.k : nullptr" in src
+    for name in ("tq4_streamk.cu", "tq4_decode.cu", "tq4_kernels.cu", "tq4_gemm.cu", "tq4_api.cu", "tq4_static.cu"):
+        assert "raise_status(TQ_DEV_SCALE_RANGE)" not in _read(name), name
+    api = _read("tq4_api.cu") + _read("tq4_static.cu")
+    assert api.count("a.codes = w->codes;") == 2 and "a.xr = fused ? nullptr : xr;" in api
+    assert "a.codes = up->codes;" in api and "b.codes = down->codes;" in api
+    assert "a.xr = xr;" in api and "b.xr = hr;" in api

@@ -9,6 +9,7 @@ tq4_1s_linear, which uses a caller workspace, with the same tolerances as the
 parity tests.  It lives in a file of its own that pytest collects last.
 """
 import ctypes
+import gc
 
 import numpy as np
 import pytest
@@ -120,12 +121,20 @@ def test_static_scratch_takes_no_memory_and_replays_in_a_graph():
     refs = torch.empty((3, m, n), dtype=torch.bfloat16, device=dev)
     call(xs[0])
     torch.cuda.synchronize()
-    free0, alloc0 = torch.cuda.mem_get_info(dev)[0], torch.cuda.memory_allocated(dev)
-    for i, x in enumerate(xs):
-        call(x)
-        torch.cuda.synchronize()
-        refs[i].copy_(y)
-    assert torch.cuda.mem_get_info(dev)[0] == free0 and torch.cuda.memory_allocated(dev) == alloc0
+    # (the collector is paused over the measured calls: objects of earlier
+    # tests freed or finalised meanwhile would move torch's counters)
+    gc.collect()
+    gc.disable()
+    try:
+        free0, alloc0 = torch.cuda.mem_get_info(dev)[0], torch.cuda.memory_allocated(dev)
+        for i, x in enumerate(xs):
+            call(x)
+            torch.cuda.synchronize()
+            refs[i].copy_(y)
+        free1, alloc1 = torch.cuda.mem_get_info(dev)[0], torch.cuda.memory_allocated(dev)
+    finally:
+        gc.enable()
+    assert free1 == free0 and alloc1 == alloc0
     x_in = xs[0].clone()
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream(dev)
