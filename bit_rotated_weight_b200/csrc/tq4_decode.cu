@@ -30,9 +30,10 @@
 //   * only the activation-dependent work follows the wait: x comes by TMA
 //     straight into the swizzled B tiles; at 16 tokens of TQ4_1S the tensor
 //     core multiplies it by the block-diagonal sign-folded Hadamard matrix
-//     (elsewhere eight warps butterfly each 32-slice in registers), the
-//     token scales come from max |x|, and x' is written back in place; then
-//     the MMAs, the remaining tiles and the epilogue.
+//     (elsewhere eight warps butterfly each 32-slice in registers), x' is
+//     written back in place as fp16 with a power-of-two scale per token
+//     (1 for any activation of ordinary range); then the MMAs, the
+//     remaining tiles and the epilogue.
 //
 // Warps (640 threads, one CTA per SM):
 //   4      lane 0: producer of the codes and scales tiles, and of every
@@ -516,12 +517,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // the slice at chunks 4 (l >> 4) + 0..3 of token l & 15 (and of token
   // 16 + (l & 15) at nb = 2), so the eight lanes of a quarter warp touch
   // eight different chunk positions: no bank conflicts.  The scale 2^e of a
-  // token is common to its whole k range in the CTA (one accumulator): a
-  // first pass takes max |x| per token (shared-memory atomic max, then a
-  // barrier of the rotation warps), and e puts 5.66 max |x| >= sqrt(32)
-  // max |x| -- a bound on |x'|, each x' being r = 1/sqrt(32) times a sum of
-  // 32 signed x -- in [2^13, 2^14), so fp16 cannot overflow.  Signs flip bf16
-  // sign bits; the butterfly runs in registers in the fixed stage order.
+  // token is common to its whole k range in the CTA (one accumulator).  On
+  // the tensor-core path x' is converted at e = 0 while its exact max |x'|
+  // per token is taken, and only tokens whose max falls outside [2^-4, 2^15)
+  // are converted again (see there).  On the register path a first pass
+  // takes max |x| per token (shared-memory atomic max, then a barrier of the
+  // rotation warps), and e puts 5.66 max |x| >= sqrt(32) max |x| -- a bound
+  // on |x'|, each x' being r = 1/sqrt(32) times a sum of 32 signed x -- in
+  // [2^13, 2^14), so fp16 cannot overflow.  Signs flip bf16 sign bits; the
+  // butterfly runs in registers in the fixed stage order.
   const int rot = warp < 4 ? warp : ((warp >= kHiWarp && warp < kHiWarp + 4) ? warp - kHiWarp + 4 : -1);
   if (rot >= 0 && kTcRot) {
     // Tensor-core rotation (16 tokens of TQ4_1S): the x tiles as A (bf16,
@@ -555,45 +559,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int u = 8 * blk + (trw >> 4), t = trw & 15;
     const bool live = xok && u < 2 * cnt;
     uint8_t* rowp = btiles + u * kHalf + (t >> 3) * 1024 + (t & 7) * 128;
-    // pass 1, while the rotation MMAs run: max |x| of the row (64 k, bf16 in
-    // shared memory), the token's two rows of this warp combined, then a
-    // shared-memory atomic max over the warps (non-negative values order as
-    // their bits)
-    uint32_t m16 = 0u;
-    if (live) {
-#pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint4 w4 = *reinterpret_cast<const uint4*>(rowp + ((c ^ (t & 7)) << 4));
-        m16 = __vmaxu2(m16, w4.x & 0x7FFF7FFFu);
-        m16 = __vmaxu2(m16, w4.y & 0x7FFF7FFFu);
-        m16 = __vmaxu2(m16, w4.z & 0x7FFF7FFFu);
-        m16 = __vmaxu2(m16, w4.w & 0x7FFF7FFFu);
-      }
-    }
-    {
-      uint32_t mb = m16 >> 16 > (m16 & 0xFFFFu) ? m16 >> 16 : (m16 & 0xFFFFu);
-      const uint32_t ob = __shfl_xor_sync(0xFFFFFFFFu, mb, 16);
-      mb = mb > ob ? mb : ob;
-      if (lane < 16 && mb != 0u) atomicMax(&sh.tok_max[t], mb << 16);
-    }
-    named_bar_sync(1, kRotWarps * 32);
     const bool rok = wwait(&sh.rdone, 0, abortp);
     tc_fence_after();
     const uint32_t taddr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kAccCol0 + 64 * blk;
-    if (xok && rok) {
-      // e from the bound sqrt(32) max |x| >= max |x'| (each x' is r times a
-      // sum of 32 signed x), as in the register path
-      const float tmx = __uint_as_float(sh.tok_max[t]);
-      const float bound = __fmul_rn(tmx, 5.66f);
-      int e = 0;
-      if (bound > 0.0f && isfinite(bound)) {
-        int ex;
-        frexpf(bound, &ex);   // bound in [2^(ex-1), 2^ex)
-        e = ex - 14;
-        e = e < -100 ? -100 : (e > 100 ? 100 : e);
-      }
-      if (blk == 0 && trw < 16) sh.row_scale[t] = ldexpf(1.0f, e);
-      const float rd = __fmul_rn(__uint_as_float(0x3E3504F3u), ldexpf(1.0f, -e));   // r 2^-e
+    // x' = r (x R2) from tensor memory to fp16, in place.  A token's scale
+    // 2^-e is common to its whole k range in the CTA, and every x' of it
+    // must come out finite and, to keep full precision, not too small: the
+    // first pass converts with e = 0 and takes the token's exact max |x'|
+    // (a shared-memory atomic max over the rows of the token; non-negative
+    // floats order as their bits, NaN above Inf).  Tokens whose max lies in
+    // [2^-4, 2^15) -- about any activation -- keep it; the others are
+    // converted again with the e that puts the max in [2^13, 2^14) (e = 0 for
+    // a non-finite max, which then shows in the output as it should).
+    const float r = __uint_as_float(0x3E3504F3u);
+    auto convert = [&](float rd) -> uint32_t {
+      uint32_t mx = 0u;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t rv[32];
@@ -605,14 +585,41 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t hw[4];
 #pragma unroll
             for (int c2 = 0; c2 < 4; ++c2) {
-              const __half2 hh2 = __floats2half2_rn(__fmul_rn(__uint_as_float(rv[8 * j + 2 * c2]), rd),
-                                                    __fmul_rn(__uint_as_float(rv[8 * j + 2 * c2 + 1]), rd));
+              const float v0 = __fmul_rn(__uint_as_float(rv[8 * j + 2 * c2]), rd);
+              const float v1 = __fmul_rn(__uint_as_float(rv[8 * j + 2 * c2 + 1]), rd);
+              const uint32_t b0 = __float_as_uint(v0) & 0x7FFFFFFFu, b1 = __float_as_uint(v1) & 0x7FFFFFFFu;
+              mx = b0 > mx ? b0 : mx;
+              mx = b1 > mx ? b1 : mx;
+              const __half2 hh2 = __floats2half2_rn(v0, v1);
               hw[c2] = *reinterpret_cast<const uint32_t*>(&hh2);
             }
             *reinterpret_cast<uint4*>(rowp + (((4 * hh + j) ^ (t & 7)) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
           }
         }
       }
+      return mx;
+    };
+    if (xok && rok) {
+      uint32_t mb = convert(r);   // |x'| max of this row, e = 0
+      // the token's two rows of this warp combined, then over the warps
+      const uint32_t ob = __shfl_xor_sync(0xFFFFFFFFu, mb, 16);
+      mb = mb > ob ? mb : ob;
+      if (lane < 16 && mb != 0u) atomicMax(&sh.tok_max[t], mb);
+    }
+    named_bar_sync(1, kRotWarps * 32);
+    if (xok && rok) {
+      const uint32_t tb = sh.tok_max[t];
+      int e = 0;
+      const bool keep = tb == 0u || (tb >= 0x3D800000u && tb < 0x47000000u);   // 0, or [2^-4, 2^15)
+      if (!keep && tb < 0x7F800000u) {
+        int ex;
+        frexpf(__uint_as_float(tb), &ex);   // max in [2^(ex-1), 2^ex)
+        e = ex - 14;
+        e = e < -100 ? -100 : (e > 100 ? 100 : e);
+      }
+      if (blk == 0 && trw < 16) sh.row_scale[t] = ldexpf(1.0f, e);
+      // (warp-uniform: tcgen05.ld is warp-collective)
+      if (__any_sync(0xFFFFFFFFu, !keep && e != 0)) convert(__fmul_rn(r, ldexpf(1.0f, -e)));
     }
     tc_fence_before();          // the tensor-memory reads, before the main MMAs reuse the columns
     fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them

@@ -70,6 +70,15 @@ def test_source_constants_and_counts():
     assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
     assert "mbar_init(&sh.xland, 1)" in SRC and "mbar_init(&sh.sfull, 1)" in SRC
     assert "named_bar_sync(1, kRotWarps * 32)" in SRC                 # the eight rotation warps
+    # tensor-core rotation: the bounded rdone wait, then the first conversion
+    # and the token max, then the named barrier (every warp reaches it), then
+    # the check of the token range and the second conversion where needed
+    i_rdone = SRC.index("const bool rok = wwait(&sh.rdone, 0, abortp);")
+    i_first = SRC.index("uint32_t mb = convert(r);")
+    i_bar = SRC.index("named_bar_sync(1, kRotWarps * 32);", i_first)
+    i_keep = SRC.index("const bool keep = tb == 0u || (tb >= 0x3D800000u && tb < 0x47000000u);")
+    i_again = SRC.index("if (__any_sync(0xFFFFFFFFu, !keep && e != 0)) convert(__fmul_rn(r, ldexpf(1.0f, -e)));")
+    assert i_rdone < i_first < i_bar < i_keep < i_again
     assert "mbar_init(&sh.rdone, 2)" in SRC
     # the cluster reduction: asynchronous stores counted in bytes on the
     # owner's barrier; every CTA sends all its rows (zeros after a timeout)
@@ -159,13 +168,13 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1, withhold_x=False):
                 state["mma"].append(rdone)
             else:
                 rdone.arrive()
-        if xok:
-            yield ("step", "max |x|")
-        rotbar.arrive()
-        yield from wait(rotbar, 0, bounded=False)
         rok = yield from wait(rdone, 0)
         if xok and rok:
-            yield ("step", "rotate")
+            yield ("step", "x' to fp16 at e = 0, token max |x'|")
+        rotbar.arrive()
+        yield from wait(rotbar, 0, bounded=False)
+        if xok and rok:
+            yield ("step", "tokens outside [2^-4, 2^15) converted again")
         if not (withhold_xready and r == 7):
             xready.arrive()
 
