@@ -112,6 +112,10 @@ __host__ __device__ constexpr int off_red(int nb, bool f8) { return off_rb(nb, f
 // (the reduction buffer holds split * ceil(128 / split) <= 135 rows)
 __host__ __device__ constexpr int smem_total(int nb, bool f8) { return off_red(nb, f8) + 136 * 16 * nb * 4 + 1024; }
 
+// 2^e for an integer e in [-126, 127], from its exponent bits (the library
+// call costs tens of instructions on paths where every cycle counts).
+__device__ __forceinline__ float exp2i(int e) { return __int_as_float((127 + e) << 23); }
+
 struct LevelTableD {
   uint32_t h[16];   // fp16 bits of 256 * levels[0..15]
   float max_level;
@@ -404,8 +408,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       e = e < -15 ? -15 : (e > 14 ? 14 : e);
     }
     sh.rexp[dq_group][trow] = static_cast<int8_t>(e);
-    const __half2 f2 = __float2half2_rn(ldexpf(1.0f, -e));   // a power of two, normal in fp16
-    ff = *reinterpret_cast<const uint32_t*>(&f2);
+    ff = static_cast<uint32_t>(15 - e) * 0x04000400u;   // {2^-e, 2^-e} in fp16 (normal for e in [-15, 14])
     __syncwarp();
     if (lane == 0) mbar_arrive(&sh.eready);
   };
@@ -617,9 +620,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         e = ex - 14;
         e = e < -100 ? -100 : (e > 100 ? 100 : e);
       }
-      if (blk == 0 && trw < 16) sh.row_scale[t] = ldexpf(1.0f, e);
+      if (blk == 0 && trw < 16) sh.row_scale[t] = exp2i(e);
       // (warp-uniform: tcgen05.ld is warp-collective)
-      if (__any_sync(0xFFFFFFFFu, !keep && e != 0)) convert(__fmul_rn(r, ldexpf(1.0f, -e)));
+      if (__any_sync(0xFFFFFFFFu, !keep && e != 0)) convert(__fmul_rn(r, exp2i(-e)));
     }
     tc_fence_before();          // the tensor-memory reads, before the main MMAs reuse the columns
     fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
@@ -679,8 +682,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             e = ex - 14;
             e = e < -100 ? -100 : (e > 100 ? 100 : e);
           }
-          if (rot == 0 && u == 0 && lane < 16) sh.row_scale[t] = ldexpf(1.0f, e);
-          const float rd = F8 ? ldexpf(1.0f, -e) : __fmul_rn(r, ldexpf(1.0f, -e));   // exact
+          if (rot == 0 && u == 0 && lane < 16) sh.row_scale[t] = exp2i(e);
+          const float rd = F8 ? exp2i(-e) : __fmul_rn(r, exp2i(-e));   // exact
           uint8_t* rowp = btiles + u * kHalf + (t >> 3) * 1024 + (t & 7) * 128;
           float v[32];
 #pragma unroll
@@ -807,11 +810,13 @@ __global__ void __launch_bounds__(kThreads, 1)
           tmem_ld16(tmem + lane_base + kAccCol0 + (2 * g) * kAccW + 16 * c, r0);
           tmem_ld16(tmem + lane_base + kAccCol0 + (2 * g + 1) * kAccW + 16 * c, r1);
           tmem_wait_ld();
-          const float rs = ldexpf(1.0f, sh.rexp[g][trow]);
+          // 2^e from its exponent bits (e in [-15, 14]); r * 2^e is exact, so
+          // the fused multiply-add rounds as the separate add would
+          const float rs = exp2i(sh.rexp[g][trow]);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(r0[j]), rs));
+          for (int j = 0; j < 16; ++j) v[j] = __fmaf_rn(__uint_as_float(r0[j]), rs, v[j]);
 #pragma unroll
-          for (int j = 0; j < 16; ++j) v[j] = __fadd_rn(v[j], __fmul_rn(__uint_as_float(r1[j]), rs));
+          for (int j = 0; j < 16; ++j) v[j] = __fmaf_rn(__uint_as_float(r1[j]), rs, v[j]);
         }
         if (ok) {
 #pragma unroll
