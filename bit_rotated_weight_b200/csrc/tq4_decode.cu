@@ -48,6 +48,7 @@
 //          memory, as two 64-k halves signalled separately;
 //   0-3, 16-19  the x rotation after the wait.
 #include <mutex>
+#include <type_traits>
 
 #include "tq4_internal.h"
 
@@ -565,18 +566,19 @@ __global__ void __launch_bounds__(kThreads, 1)
     const bool rok = wwait(&sh.rdone, 0, abortp);
     tc_fence_after();
     const uint32_t taddr = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16) + kAccCol0 + 64 * blk;
-    // x' = r (x R2) from tensor memory to fp16, in place.  A token's scale
-    // 2^-e is common to its whole k range in the CTA, and every x' of it
-    // must come out finite and, to keep full precision, not too small: the
-    // first pass converts with e = 0 and takes the token's exact max |x'|
-    // (a shared-memory atomic max over the rows of the token; non-negative
-    // floats order as their bits, NaN above Inf).  Tokens whose max lies in
-    // [2^-4, 2^15) -- about any activation -- keep it; the others are
-    // converted again with the e that puts the max in [2^13, 2^14) (e = 0 for
-    // a non-finite max, which then shows in the output as it should).
-    const float r = __uint_as_float(0x3E3504F3u);
-    auto convert = [&](float rd) -> uint32_t {
-      uint32_t mx = 0u;
+    // x R2 = x' / r from tensor memory to fp16, in place (the factor r joins
+    // the token scale of the epilogue).  A token's scale 2^-e is common to
+    // its whole k range in the CTA, and every value of it must come out
+    // finite and, to keep full precision, not too small: the first pass
+    // converts with e = 0 and takes the token's exact max |x R2| (a
+    // shared-memory atomic max over the rows of the token; non-negative
+    // floats order as their bits; a NaN is left out of the max and shows in
+    // the output).  Tokens whose max lies in [2^-4, 2^15) -- about any
+    // activation -- keep it; the others are converted again with the e that
+    // puts the max in [2^13, 2^14) (e = 0 for an infinite max, which then
+    // shows in the output as it should).
+    auto convert = [&](auto scaled, float rd) -> float {
+      float mx = 0.0f;
 #pragma unroll
       for (int hh = 0; hh < 2; ++hh) {
         uint32_t rv[32];
@@ -588,11 +590,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             uint32_t hw[4];
 #pragma unroll
             for (int c2 = 0; c2 < 4; ++c2) {
-              const float v0 = __fmul_rn(__uint_as_float(rv[8 * j + 2 * c2]), rd);
-              const float v1 = __fmul_rn(__uint_as_float(rv[8 * j + 2 * c2 + 1]), rd);
-              const uint32_t b0 = __float_as_uint(v0) & 0x7FFFFFFFu, b1 = __float_as_uint(v1) & 0x7FFFFFFFu;
-              mx = b0 > mx ? b0 : mx;
-              mx = b1 > mx ? b1 : mx;
+              float v0 = __uint_as_float(rv[8 * j + 2 * c2]), v1 = __uint_as_float(rv[8 * j + 2 * c2 + 1]);
+              if constexpr (decltype(scaled)::value) {
+                v0 = __fmul_rn(v0, rd);
+                v1 = __fmul_rn(v1, rd);
+              } else {
+                mx = fmaxf(mx, fmaxf(fabsf(v0), fabsf(v1)));
+              }
               const __half2 hh2 = __floats2half2_rn(v0, v1);
               hw[c2] = *reinterpret_cast<const uint32_t*>(&hh2);
             }
@@ -603,7 +607,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       return mx;
     };
     if (xok && rok) {
-      uint32_t mb = convert(r);   // |x'| max of this row, e = 0
+      uint32_t mb = __float_as_uint(convert(std::false_type{}, 1.0f));   // max |x R2| of this row, e = 0
       // the token's two rows of this warp combined, then over the warps
       const uint32_t ob = __shfl_xor_sync(0xFFFFFFFFu, mb, 16);
       mb = mb > ob ? mb : ob;
@@ -622,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       if (blk == 0 && trw < 16) sh.row_scale[t] = exp2i(e);
       // (warp-uniform: tcgen05.ld is warp-collective)
-      if (__any_sync(0xFFFFFFFFu, !keep && e != 0)) convert(__fmul_rn(r, exp2i(-e)));
+      if (__any_sync(0xFFFFFFFFu, !keep && e != 0)) convert(std::true_type{}, exp2i(-e));
     }
     tc_fence_before();          // the tensor-memory reads, before the main MMAs reuse the columns
     fence_proxy_async_smem();   // generic-proxy writes, before the tensor core reads them
@@ -794,7 +798,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
     const int ngroups = cnt < kGroups ? cnt : kGroups;   // groups (and their two accumulators) with work
-    const float wsc = F8 ? ((row0 + trow < a.n) ? __ldcg(a.wscale + row0 + trow) : 0.0f) : 1.0f / kLevelScaleD;
+    // (the tensor-core rotation leaves the factor r = 1/sqrt(32) of x' to here)
+    const float wsc = F8 ? ((row0 + trow < a.n) ? __ldcg(a.wscale + row0 + trow) : 0.0f)
+                         : (kTcRot ? __uint_as_float(0x3E3504F3u) / kLevelScaleD : 1.0f / kLevelScaleD);
     if (split > 1) asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
     // the cluster reduction counts bytes: every CTA sends all its rows, zeros
     // when a role timed out

@@ -74,11 +74,13 @@ def test_source_constants_and_counts():
     # and the token max, then the named barrier (every warp reaches it), then
     # the check of the token range and the second conversion where needed
     i_rdone = SRC.index("const bool rok = wwait(&sh.rdone, 0, abortp);")
-    i_first = SRC.index("uint32_t mb = convert(r);")
+    i_first = SRC.index("uint32_t mb = __float_as_uint(convert(std::false_type{}, 1.0f));")
     i_bar = SRC.index("named_bar_sync(1, kRotWarps * 32);", i_first)
     i_keep = SRC.index("const bool keep = tb == 0u || (tb >= 0x3D800000u && tb < 0x47000000u);")
-    i_again = SRC.index("if (__any_sync(0xFFFFFFFFu, !keep && e != 0)) convert(__fmul_rn(r, ldexpf(1.0f, -e)));")
+    i_again = SRC.index("if (__any_sync(0xFFFFFFFFu, !keep && e != 0)) convert(std::true_type{}, exp2i(-e));")
     assert i_rdone < i_first < i_bar < i_keep < i_again
+    # the factor r of x' is applied in the epilogue on this path
+    assert "(kTcRot ? __uint_as_float(0x3E3504F3u) / kLevelScaleD : 1.0f / kLevelScaleD)" in SRC
     assert "mbar_init(&sh.rdone, 2)" in SRC
     # the cluster reduction: asynchronous stores counted in bytes on the
     # owner's barrier; every CTA sends all its rows (zeros after a timeout)
