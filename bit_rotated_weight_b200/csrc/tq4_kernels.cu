@@ -81,18 +81,36 @@ __device__ __forceinline__ void quantize_block(float (&a)[32], uint32_t mask, co
     const uint16_t dbits = f16_sat_bits(rms);
     dpair |= static_cast<uint32_t>(dbits) << (16 * h);
     const float d = __half2float(__ushort_as_half(dbits));
+    // u = fl(a / d), correctly rounded.  With y = RN(1/d) once per half
+    // block, q = RN(a y), the exact residual r = a - q d (one fma) and
+    // RN(q + r y) give the correctly rounded quotient whenever nothing
+    // overflows (Markstein's theorem; checked against the division on every
+    // positive fp16 d).  A finite sum of squares bounds |a| by 2^63, and then
+    // |a / d| stays near 4 or below; otherwise (an Inf or NaN in the block)
+    // the division itself runs.
+    float u[16];
+    if (isfinite(p[0]) && d != 0.0f) {
+      const float y = __frcp_rn(d);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float q = __fmul_rn(a[16 * h + i], y);
+        u[i] = __fmaf_rn(__fmaf_rn(-q, d, a[16 * h + i]), y, q);
+      }
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) u[i] = __fdiv_rn(a[16 * h + i], d);
+    }
 #pragma unroll
     for (int i = 0; i < 16; ++i) {
       uint32_t code;
       if (d == 0.0f) {
         code = 7u;
       } else {
-        const float u = __fdiv_rn(a[16 * h + i], d);
         // number of thresholds strictly below u (binary search, sorted t)
-        code = (u > s_t[7]) ? 8u : 0u;
-        code += (u > s_t[code + 3]) ? 4u : 0u;
-        code += (u > s_t[code + 1]) ? 2u : 0u;
-        code += (u > s_t[code]) ? 1u : 0u;
+        code = (u[i] > s_t[7]) ? 8u : 0u;
+        code += (u[i] > s_t[code + 3]) ? 4u : 0u;
+        code += (u[i] > s_t[code + 1]) ? 2u : 0u;
+        code += (u[i] > s_t[code]) ? 1u : 0u;
       }
       const int e = 16 * h + i;   // element index; nibble e of the 16-byte block
       words[e >> 3] |= code << (4 * (e & 7));
