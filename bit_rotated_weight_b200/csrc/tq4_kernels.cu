@@ -47,21 +47,32 @@ __device__ __forceinline__ void fwht32_regs(float (&a)[32]) {
   }
 }
 
+// Thresholds of the quantizer in shared memory: t[0..14] (sorted, t[15]
+// unused), then, when the codebook is symmetric (t[14 - k] == -t[k], so
+// t[7] == 0), the positive thresholds p[j] = t[8 + j] and the largest float
+// below each, b[j] (x >= p[j] exactly when x > b[j]), j < 7; sym says which.
+struct QuantThresholds {
+  float t[16];
+  float p[8];
+  float b[8];
+  int sym;
+};
+
 // Quantize one 32-element block held in registers (sign flip, butterfly, x r,
 // per-half RMS by the pairwise tree, fp16 scale, nearest level by the
 // thresholds, nibble packing) -- the fixed fp32 operation order that the
 // packing's bit-exactness rests on.  words = the 16 code bytes, dpair = the
-// two fp16 scales (half 0 in the low 16 bits).
-__device__ __forceinline__ void quantize_block(float (&a)[32], uint32_t mask, const float* s_t, uint32_t (&words)[4],
-                                               uint32_t& dpair) {
+// two fp16 scales (half 0 in the low 16 bits).  Returns false when a half
+// block's sum of squares is not finite: an input was Inf or NaN (which makes
+// every output of the butterfly non-finite), or a finite input was above
+// ~2^63; the caller then checks the inputs themselves.
+__device__ __forceinline__ bool quantize_block(float (&a)[32], uint32_t mask, const QuantThresholds& th,
+                                               uint32_t (&words)[4], uint32_t& dpair) {
   const float r = rsqrt32();
-  bool finite = true;
+  bool sums_finite = true;
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    finite = finite && isfinite(a[i]);
+  for (int i = 0; i < 32; ++i)
     if ((mask >> i) & 1u) a[i] = -a[i];
-  }
-  if (!finite) raise_status(TQ_DEV_NONFINITE);
   fwht32_regs(a);
 #pragma unroll
   for (int i = 0; i < 32; ++i) a[i] = __fmul_rn(a[i], r);
@@ -81,41 +92,58 @@ __device__ __forceinline__ void quantize_block(float (&a)[32], uint32_t mask, co
     const uint16_t dbits = f16_sat_bits(rms);
     dpair |= static_cast<uint32_t>(dbits) << (16 * h);
     const float d = __half2float(__ushort_as_half(dbits));
-    // u = fl(a / d), correctly rounded.  With y = RN(1/d) once per half
-    // block, q = RN(a y), the exact residual r = a - q d (one fma) and
-    // RN(q + r y) give the correctly rounded quotient whenever nothing
-    // overflows (Markstein's theorem; checked against the division on every
-    // positive fp16 d).  A finite sum of squares bounds |a| by 2^63, and then
-    // |a / d| stays near 4 or below; otherwise (an Inf or NaN in the block)
-    // the division itself runs.
-    float u[16];
-    if (isfinite(p[0]) && d != 0.0f) {
+    // u = fl(a / d), correctly rounded, and its code: the number of
+    // thresholds strictly below u.
+    const bool fin = isfinite(p[0]);
+    sums_finite = sums_finite && fin;
+    if (fin && d != 0.0f) {
+      // With y = RN(1/d) once per half block, q = RN(a y), the exact
+      // residual r = a - q d (one fma) and RN(q + r y) give the correctly
+      // rounded quotient whenever nothing overflows (Markstein's theorem;
+      // checked against the division on every positive fp16 d): a finite sum
+      // of squares bounds |a| by 2^63, and |a / d| then stays near 4 or below.
       const float y = __frcp_rn(d);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float q = __fmul_rn(a[16 * h + i], y);
-        u[i] = __fmaf_rn(__fmaf_rn(-q, d, a[16 * h + i]), y, q);
+        const float u = __fmaf_rn(__fmaf_rn(-q, d, a[16 * h + i]), y, q);
+        uint32_t code;
+        if (th.sym) {
+          // symmetric thresholds: u > 0 has 8 + #{p[j] < u} below it, u <= 0
+          // has #{t[k] < u, k < 7} = #{p[j] > |u|} = 7 - #{|u| > b[j]}
+          const bool pos = u > 0.0f;
+          const float au = fabsf(u);
+          const float* tb = pos ? th.p : th.b;
+          uint32_t c = (au > tb[3]) ? 4u : 0u;
+          c += (au > tb[c + 1]) ? 2u : 0u;
+          c += (au > tb[c]) ? 1u : 0u;
+          code = pos ? 8u + c : 7u - c;
+        } else {
+          code = (u > th.t[7]) ? 8u : 0u;
+          code += (u > th.t[code + 3]) ? 4u : 0u;
+          code += (u > th.t[code + 1]) ? 2u : 0u;
+          code += (u > th.t[code]) ? 1u : 0u;
+        }
+        const int e = 16 * h + i;   // element index; nibble e of the 16-byte block
+        words[e >> 3] |= code << (4 * (e & 7));
       }
     } else {
 #pragma unroll
-      for (int i = 0; i < 16; ++i) u[i] = __fdiv_rn(a[16 * h + i], d);
-    }
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      uint32_t code;
-      if (d == 0.0f) {
-        code = 7u;
-      } else {
-        // number of thresholds strictly below u (binary search, sorted t)
-        code = (u[i] > s_t[7]) ? 8u : 0u;
-        code += (u[i] > s_t[code + 3]) ? 4u : 0u;
-        code += (u[i] > s_t[code + 1]) ? 2u : 0u;
-        code += (u[i] > s_t[code]) ? 1u : 0u;
+      for (int i = 0; i < 16; ++i) {
+        uint32_t code = 7u;   // d == 0: the zero level's code
+        if (d != 0.0f) {
+          const float u = __fdiv_rn(a[16 * h + i], d);
+          code = (u > th.t[7]) ? 8u : 0u;
+          code += (u > th.t[code + 3]) ? 4u : 0u;
+          code += (u > th.t[code + 1]) ? 2u : 0u;
+          code += (u > th.t[code]) ? 1u : 0u;
+        }
+        const int e = 16 * h + i;
+        words[e >> 3] |= code << (4 * (e & 7));
       }
-      const int e = 16 * h + i;   // element index; nibble e of the 16-byte block
-      words[e >> 3] |= code << (4 * (e & 7));
     }
   }
+  return sums_finite;
 }
 
 // The tensors of one quantize launch.  A tensor of B blocks (B = rows * k / 32,
@@ -151,9 +179,19 @@ __global__ void __launch_bounds__(256, 4) quantize_kernel(const __grid_constant_
   constexpr int kRowBytes = 32 * static_cast<int>(sizeof(T));   // one block: 128 B (fp32) or 64 B (bf16)
   constexpr int kPieces = kRowBytes / 16;                        // 16-byte pieces per block
   constexpr int kLoads = kPieces;                                // 16-byte loads per lane per chunk
-  __shared__ float s_t[16];
+  __shared__ QuantThresholds th;
   __shared__ __align__(16) uint8_t tile[8][32 * kRowBytes];
-  if (threadIdx.x < 16) s_t[threadIdx.x] = cb.thresholds[threadIdx.x];
+  if (threadIdx.x < 16) th.t[threadIdx.x] = cb.thresholds[threadIdx.x];
+  if (threadIdx.x < 8) {
+    const float pj = threadIdx.x < 7 ? cb.thresholds[8 + threadIdx.x] : INFINITY;
+    th.p[threadIdx.x] = pj;
+    th.b[threadIdx.x] = threadIdx.x < 7 ? __uint_as_float(__float_as_uint(pj) - 1u) : INFINITY;
+  }
+  if (threadIdx.x == 0) {
+    bool sym = cb.thresholds[7] == 0.0f;
+    for (int k = 0; k < 7; ++k) sym = sym && cb.thresholds[14 - k] == -cb.thresholds[k] && cb.thresholds[8 + k] > 0.0f;
+    th.sym = sym ? 1 : 0;
+  }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   uint8_t* my = tile[warp];
@@ -209,10 +247,28 @@ __global__ void __launch_bounds__(256, 4) quantize_kernel(const __grid_constant_
     const int64_t b = b0 + lane;
     if (b < q.nblocks) {
       uint32_t words[4], dpair;
-      quantize_block(a, q.mask, s_t, words, dpair);
+      if (!quantize_block(a, q.mask, th, words, dpair)) {
+        // a sum of squares was not finite: flag an input that is Inf or NaN
+        bool finite = true;
+#pragma unroll
+        for (int c = 0; c < kPieces; ++c) {
+          const uint4 w = *reinterpret_cast<const uint4*>(my + tpos(lane, c));
+          const uint32_t v[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            if constexpr (sizeof(T) == 4) {
+              finite = finite && isfinite(__uint_as_float(v[j]));
+            } else {
+              finite = finite && isfinite(__uint_as_float(v[j] << 16)) && isfinite(__uint_as_float(v[j] & 0xFFFF0000u));
+            }
+          }
+        }
+        if (!finite) raise_status(TQ_DEV_NONFINITE);
+      }
       *reinterpret_cast<uint4*>(q.codes + b * 16) = make_uint4(words[0], words[1], words[2], words[3]);
       *reinterpret_cast<uint32_t*>(q.scales + b * 2) = dpair;
     }
+    __syncwarp();   // every lane is done with the tile (the check above reads it)
   }
 }
 

@@ -244,3 +244,44 @@ def test_missing_library_raises(tmp_path):
             tq.load_library(str(tmp_path / "nope.so"))
         finally:
             tq._lib = tq._lib_saved
+
+
+def test_symmetric_threshold_search_counts_like_the_full_search():
+    # The quantize kernel, on finite half blocks, finds a code with a 3-step
+    # search on |u| over the 7 positive thresholds p[j] (u > 0: 8 + #{p[j] < u})
+    # or, for u <= 0, the largest floats b[j] below them (7 - #{|u| > b[j]}).
+    # On the library's own fp32 thresholds (symmetric: t[14 - k] == -t[k]),
+    # that must equal the number of thresholds strictly below u for every u,
+    # ties included: checked at each threshold, +-4 ulps around it, both signs.
+    _, th = tq.tq4_1s_codebook()
+    t = th.numpy().astype(np.float32)
+    assert t[7] == 0.0 and all(t[14 - k] == -t[k] for k in range(7))
+    p = t[8:15]
+    b = (p.view(np.uint32) - np.uint32(1)).view(np.float32)
+    assert np.all(np.nextafter(p, np.float32(0)) == b)
+
+    def full(u):
+        return int(np.sum(t < u))
+
+    def symmetric(u):
+        pos = u > 0
+        au = np.float32(abs(u))
+        tb = p if pos else b
+        c = 4 if au > tb[3] else 0
+        c += 2 if au > tb[c + 1] else 0
+        c += 1 if au > tb[c] else 0
+        return 8 + c if pos else 7 - c
+
+    cases = [np.float32(0.0), np.float32(-0.0), np.float32(1e-30), np.float32(-1e-30), np.float32(7.0),
+             np.float32(-7.0)]
+    for x in t:
+        for sgn in (1, -1):
+            v = np.float32(sgn * x)
+            bits = v.view(np.uint32).astype(np.int64)
+            for dlt in range(-4, 5):
+                if v == 0.0:
+                    continue
+                cases.append(np.array([bits + dlt], dtype=np.int64).astype(np.uint32).view(np.float32)[0])
+    assert len(cases) > 200
+    for u in cases:
+        assert symmetric(u) == full(u), (float(u), symmetric(u), full(u))

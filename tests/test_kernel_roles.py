@@ -251,3 +251,24 @@ def test_streamk_overflowing_levels_fall_back_to_the_exact_path():
     assert api.count("a.codes = w->codes;") == 2 and "a.xr = fused ? nullptr : xr;" in api
     assert "a.codes = up->codes;" in api and "b.codes = down->codes;" in api
     assert "a.xr = xr;" in api and "b.xr = hr;" in api
+
+
+def test_quantize_fast_path_matches_the_checked_forms():
+    # the symmetric search and the quotient sequence are the forms that
+    # test_abi_host.py and the GPU probe of the division checked: b[j] is the
+    # float just below p[j]; the search runs only on symmetric thresholds and
+    # finite half blocks; other half blocks keep the division and full search
+    src = _read("tq4_kernels.cu")
+    for s in ("th.b[threadIdx.x] = threadIdx.x < 7 ? __uint_as_float(__float_as_uint(pj) - 1u) : INFINITY;",
+              "const float* tb = pos ? th.p : th.b;",
+              "uint32_t c = (au > tb[3]) ? 4u : 0u;",
+              "c += (au > tb[c + 1]) ? 2u : 0u;",
+              "c += (au > tb[c]) ? 1u : 0u;",
+              "code = pos ? 8u + c : 7u - c;",
+              "if (fin && d != 0.0f) {",
+              "const float y = __frcp_rn(d);",
+              "const float u = __fmaf_rn(__fmaf_rn(-q, d, a[16 * h + i]), y, q);",
+              "const float u = __fdiv_rn(a[16 * h + i], d);",
+              "if (!finite) raise_status(TQ_DEV_NONFINITE);",
+              "__syncwarp();   // every lane is done with the tile (the check above reads it)"):
+        assert s in src, s
