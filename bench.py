@@ -50,7 +50,7 @@ PACKED_PER_CALL = N_OUT * K_IN // 2 + N_OUT * (K_IN // 16) * 2   # 10,485,760 B
 # DRAM bytes (read + write) of one decode launch: ncu dram__bytes_read.sum +
 # dram__bytes_write.sum of decode_kernel<1, 0> on this workload (10,691,072 +
 # 0); set back to None whenever the kernel changes until taken again.
-TRAFFIC_PER_CALL = 10691072
+TRAFFIC_PER_CALL = None
 # DRAM bytes of one stream-K launch of the MoE layer (an up projection, the
 # routing of seed 7: 223,320,320 read + 5,106,688 written), against about
 # 216 MB of touched packed bytes per projection.

@@ -252,7 +252,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&sh.dfull, kIssuers);
     for (int i = 0; i < kIssuers; ++i) mbar_init(&sh.idone[i], 1);
     mbar_init(&sh.eready, 4 * kGroups);
-    mbar_init(&sh.xland, 1);
     mbar_init(&sh.rdone, 2);
     mbar_init(&sh.redfull, 1);
     // the bytes this CTA receives in the cluster reduction: its rows from
@@ -262,6 +261,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                                                                          (rank * 128 + split - 1) / split) *
                                                                16 * NB * 4));
     fence_mbar_init();
+  }
+  // The x producer (lane 0 of warp 16; its warp takes no part in the set-up
+  // stores): its own barrier, the wait for the previous kernel (x is its
+  // output), and the x tiles at once, so that they land while the set-up
+  // runs.  (The B tiles are written by nothing else before the rotation.)
+  if (warp == kHiWarp && lane == 0) {
+    mbar_init(&sh.xland, 1);
+    fence_mbar_init();
+    pdl_wait();
+    if (a.x_box3) {
+      // one 3-D box: all 2 kMaxIters half tiles from this CTA's first k
+      // (those past its range land in B tiles it does not use)
+      mbar_arrive_expect_tx(&sh.xland, static_cast<uint32_t>(2 * kMaxIters * kHalf));
+      tma_load_3d(btiles, &tm_x, &sh.xland, 0, 0, 2 * it0);
+    } else {
+      mbar_arrive_expect_tx(&sh.xland, static_cast<uint32_t>(2 * cnt * kHalf));
+      for (int u = 0; u < 2 * cnt; ++u) tma_load_2d(btiles + u * kHalf, &tm_x, &sh.xland, (2 * it0 + u) * 64, 0);
+    }
   }
   const int dq_group = (warp >= kFirstDqWarp && warp < kHiWarp) ? (warp - kFirstDqWarp) >> 2 : -1;
   const int trow = (warp & 3) * 32 + lane;   // tile row of this thread (dequant and epilogue)
@@ -307,9 +324,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
     }
   };
-  // the set-up stores below are shared by the warps other than the producer's
-  constexpr int kSetupWarps = kThreads / 32 - 1;
-  const int setup_warp = warp < kProducerWarp ? warp : warp - 1;
+  // the set-up stores below are shared by the warps other than the two
+  // producers' (4 and 16)
+  constexpr int kSetupWarps = kThreads / 32 - 2;
+  const int setup_warp = warp < kProducerWarp ? warp : (warp < kHiWarp ? warp - 1 : warp - 2);
+  const bool setup_role = warp != kProducerWarp && warp != kHiWarp;
   if (warp == 0) {
     if (lane == 0) sh.abort_flag = 0;
     sh.tok_max[lane] = 0u;
@@ -328,7 +347,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
     for (int it = 0; it < (64 + kSetupWarps - 1) / kSetupWarps; ++it) {
       const int s4 = setup_warp + kSetupWarps * it;   // warp-uniform
-      if (warp != kProducerWarp && s4 < 64) {
+      if (setup_role && s4 < 64) {
         const int b = 4 * s4 + (lane >> 3);
         const uint32_t lo = __shfl_sync(0xFFFFFFFFu, hl, b & 15), hi = __shfl_sync(0xFFFFFFFFu, hl, b >> 4);
         const uint32_t v = lo | (hi << 16);
@@ -343,7 +362,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ((-1)^popcount(n & i)), s the signs.  bf16 +-1 and 0 are exact.  K-major,
     // 128-byte swizzle: 8 entries (16 B) per store, chunk c of row n at c ^ (n & 7).
     uint8_t* rb = smem + off_rb(NB, F8);
-    for (int t = setup_warp * 32 + lane; warp != kProducerWarp && t < 64 * 8; t += kSetupWarps * 32) {
+    for (int t = setup_warp * 32 + lane; setup_role && t < 64 * 8; t += kSetupWarps * 32) {
       const int n = t >> 3, c = t & 7;   // chunk c: inputs 8 c .. 8 c + 7
       uint32_t w[4] = {0u, 0u, 0u, 0u};
       if ((n >> 5) == (c >> 2)) {
@@ -365,14 +384,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     fence_proxy_async_smem();
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
   // All CTAs of this grid are resident once every one of them is here: the
   // next kernel may launch now.  Its CTAs take the SMs this grid leaves free
   // and those its CTAs release, and set up meanwhile; anything of theirs that
-  // reads this kernel's output waits in griddepcontrol.wait.
+  // reads this kernel's output waits in griddepcontrol.wait.  (Before the
+  // set-up barrier, which the x producer reaches only after its wait.)
   if (threadIdx.x == 0) pdl_launch_dependents();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
   // Every CTA of the cluster has initialised its barriers once all have
   // arrived here; the epilogue waits for that before its first remote store.
   if (split > 1) asm volatile("barrier.cluster.arrive.relaxed.aligned;" ::: "memory");
@@ -495,20 +515,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     pdl_wait();
   }
-  // The x producer (lane 0 of warp 16, which has nothing to do before the
-  // wait): the x tiles, and a weight not flagged static.
-  if (warp == kHiWarp && lane == 0) {
-    if (a.x_box3) {
-      // one 3-D box: all 2 kMaxIters half tiles from this CTA's first k
-      // (those past its range land in B tiles it does not use)
-      mbar_arrive_expect_tx(&sh.xland, static_cast<uint32_t>(2 * kMaxIters * kHalf));
-      tma_load_3d(btiles, &tm_x, &sh.xland, 0, 0, 2 * it0);
-    } else {
-      mbar_arrive_expect_tx(&sh.xland, static_cast<uint32_t>(2 * cnt * kHalf));
-      for (int u = 0; u < 2 * cnt; ++u) tma_load_2d(btiles + u * kHalf, &tm_x, &sh.xland, (2 * it0 + u) * 64, 0);
-    }
-    if (!stat) issue_weight();
-  }
+  // A weight not flagged static is copied after the wait too, by the x
+  // producer (its barriers come from the set-up).
+  if (warp == kHiWarp && lane == 0 && !stat) issue_weight();
 
   // ------------------------------------------------------------ x rotation
   // x came by TMA straight into the B tiles: half tile u = 2 li + h holds the

@@ -69,6 +69,16 @@ def test_source_constants_and_counts():
     assert "mbar_init(&sh.dfull, kIssuers)" in SRC and "constexpr int kIssuers = 2 * kGroups;" in SRC
     assert "mbar_init(&sh.eready, 4 * kGroups)" in SRC               # one arrival per dequant warp
     assert "mbar_init(&sh.xland, 1)" in SRC and "mbar_init(&sh.sfull, 1)" in SRC
+    # the x producer initialises its own barrier, waits and copies x before
+    # the set-up barrier; its warp takes no part in the set-up stores; the
+    # next-launch trigger precedes the set-up barrier (which the x producer
+    # reaches only after its wait)
+    i_xp = SRC.index("  if (warp == kHiWarp && lane == 0) {\n    mbar_init(&sh.xland, 1);\n    fence_mbar_init();\n    pdl_wait();")
+    i_trig = SRC.index("  if (threadIdx.x == 0) pdl_launch_dependents();\n  tc_fence_before();\n  __syncthreads();")
+    assert i_xp < i_trig
+    assert SRC.count("mbar_init(&sh.xland, 1)") == 1
+    assert "const bool setup_role = warp != kProducerWarp && warp != kHiWarp;" in SRC
+    assert "if (warp == kHiWarp && lane == 0 && !stat) issue_weight();" in SRC
     assert "named_bar_sync(1, kRotWarps * 32)" in SRC                 # the eight rotation warps
     # tensor-core rotation: the bounded rdone wait, then the first conversion
     # and the token max, then the named barrier (every warp reaches it), then
@@ -250,8 +260,10 @@ def run(cnt, seed, withhold_xready=False, static=True, nb=1, withhold_x=False):
         ok = ok and (yield from wait(dfull, 0))
 
     def x_producer_rotation():
-        # warp 16: lane 0 issues the x tiles (and a weight not flagged static)
-        # after the wait, the warp rotates, and on an abort lane 0 waits for
+        # warp 16: lane 0 initialises xland, waits for the previous kernel and
+        # issues the x tiles before the set-up barrier (the set-up is not
+        # modelled: every actor here starts after it), then a weight not
+        # flagged static; the warp rotates, and on an abort lane 0 waits for
         # every copy to land
         yield ("step", "wait for the previous kernel")
         state["issued"] += 1
