@@ -220,13 +220,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   // into L2 now and loaded after the wait (by the x producer, below).
   const bool sc_tma = !F8 && a.scales_tma != 0;
   auto issue_weight = [&]() {
-    for (int li = 0; li < cnt; ++li) {
-      mbar_arrive_expect_tx(&sh.full[li], kTile);
-      tma_load_3d(smem + li * kTile, &tm_codes, &sh.full[li], (it0 + li) * (F8 ? 128 : 64), row0, 0);
-    }
+    // the scales tile first: every dequant thread needs it before its first
+    // iteration, and copies land in about the order they are issued
     if (sc_tma) {
       mbar_arrive_expect_tx(&sh.sfull, kScTileBytes);
       tma_load_2d(const_cast<uint8_t*>(sctile), &tm_sc, &sh.sfull, it0 * 8, row0);
+    }
+    for (int li = 0; li < cnt; ++li) {
+      mbar_arrive_expect_tx(&sh.full[li], kTile);
+      tma_load_3d(smem + li * kTile, &tm_codes, &sh.full[li], (it0 + li) * (F8 ? 128 : 64), row0, 0);
     }
   };
   if (warp == kProducerWarp && lane == 0) {
