@@ -48,9 +48,9 @@ CALLS = 16
 COPIES = 64
 PACKED_PER_CALL = N_OUT * K_IN // 2 + N_OUT * (K_IN // 16) * 2   # 10,485,760 B
 # DRAM bytes (read + write) of one decode launch: ncu dram__bytes_read.sum +
-# dram__bytes_write.sum of decode_kernel<1, 0> on this workload (10,691,072 +
+# dram__bytes_write.sum of decode_kernel<1, 0> on this workload (10,694,400 +
 # 0); set back to None whenever the kernel changes until taken again.
-TRAFFIC_PER_CALL = None
+TRAFFIC_PER_CALL = 10694400
 # DRAM bytes of one stream-K launch of the MoE layer (an up projection, the
 # routing of seed 7: 223,320,320 read + 5,106,688 written), against about
 # 216 MB of touched packed bytes per projection.
