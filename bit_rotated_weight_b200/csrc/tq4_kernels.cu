@@ -48,14 +48,22 @@ __device__ __forceinline__ void fwht32_regs(float (&a)[32]) {
 }
 
 // Thresholds of the quantizer in shared memory: t[0..14] (sorted, t[15]
-// unused), then, when the codebook is symmetric (t[14 - k] == -t[k], so
-// t[7] == 0), the positive thresholds p[j] = t[8 + j] and the largest float
-// below each, b[j] (x >= p[j] exactly when x > b[j]), j < 7; sym says which.
+// unused), and a bucket table over |u| for a symmetric codebook
+// (t[14 - k] == -t[k], so t[7] == 0), whose positive thresholds are
+// p[j] = t[8 + j], j < 7.  Bucket i >= 1 holds the floats whose bits >> 19
+// (exponent and top 4 mantissa bits) equal kQBucket0 + i - 1, i.e.
+// [2^-5, 2^3) in 128 buckets; bucket 0 is below 2^-5, the last one 2^3 and
+// above.  Entry i: x = the bits of the p[j] inside the bucket (those of
+// +inf if none), y = the number of p[j] below the bucket.  Non-negative
+// floats order as their bits, so |u| > p[j] is bits(|u|) > x and
+// |u| >= p[j] is bits(|u|) + 1 > x.  fast: the codebook is symmetric and no
+// bucket holds two thresholds (else the full search runs).
+constexpr int kQBucket0 = 122 << 4;   // bits of 2^-5, >> 19
+constexpr int kQBuckets = 130;
 struct QuantThresholds {
   float t[16];
-  float p[8];
-  float b[8];
-  int sym;
+  uint2 bucket[kQBuckets];
+  int fast;
 };
 
 // Quantize one 32-element block held in registers (sign flip, butterfly, x r,
@@ -108,15 +116,17 @@ __device__ __forceinline__ bool quantize_block(float (&a)[32], uint32_t mask, co
         const float q = __fmul_rn(a[16 * h + i], y);
         const float u = __fmaf_rn(__fmaf_rn(-q, d, a[16 * h + i]), y, q);
         uint32_t code;
-        if (th.sym) {
+        if (th.fast) {
           // symmetric thresholds: u > 0 has 8 + #{p[j] < u} below it, u <= 0
-          // has #{t[k] < u, k < 7} = #{p[j] > |u|} = 7 - #{|u| > b[j]}
+          // has #{t[k] < u, k < 7} = #{p[j] > |u|} = 7 - #{p[j] <= |u|}; both
+          // counts from |u|'s bucket: the thresholds below it, plus the one
+          // inside it if |u| passes it (> for u > 0, >= for u <= 0)
           const bool pos = u > 0.0f;
-          const float au = fabsf(u);
-          const float* tb = pos ? th.p : th.b;
-          uint32_t c = (au > tb[3]) ? 4u : 0u;
-          c += (au > tb[c + 1]) ? 2u : 0u;
-          c += (au > tb[c]) ? 1u : 0u;
+          const uint32_t ab = __float_as_uint(u) & 0x7FFFFFFFu;
+          int q = static_cast<int>(ab >> 19) - (kQBucket0 - 1);
+          q = q < 0 ? 0 : (q > kQBuckets - 1 ? kQBuckets - 1 : q);
+          const uint2 e = th.bucket[q];
+          const uint32_t c = e.y + ((ab + (pos ? 0u : 1u) > e.x) ? 1u : 0u);
           code = pos ? 8u + c : 7u - c;
         } else {
           code = (u > th.t[7]) ? 8u : 0u;
@@ -182,15 +192,33 @@ __global__ void __launch_bounds__(256, 4) quantize_kernel(const __grid_constant_
   __shared__ QuantThresholds th;
   __shared__ __align__(16) uint8_t tile[8][32 * kRowBytes];
   if (threadIdx.x < 16) th.t[threadIdx.x] = cb.thresholds[threadIdx.x];
-  if (threadIdx.x < 8) {
-    const float pj = threadIdx.x < 7 ? cb.thresholds[8 + threadIdx.x] : INFINITY;
-    th.p[threadIdx.x] = pj;
-    th.b[threadIdx.x] = threadIdx.x < 7 ? __uint_as_float(__float_as_uint(pj) - 1u) : INFINITY;
+  auto bucket_of = [](float x) {   // x >= 0
+    const int q = static_cast<int>(__float_as_uint(x) >> 19) - (kQBucket0 - 1);
+    return q < 0 ? 0 : (q > kQBuckets - 1 ? kQBuckets - 1 : q);
+  };
+  for (int i = threadIdx.x; i < kQBuckets; i += blockDim.x) {
+    const float lo = i == 0 ? 0.0f : __uint_as_float(static_cast<uint32_t>(kQBucket0 + i - 1) << 19);
+    const float hi = i == kQBuckets - 1 ? INFINITY : __uint_as_float(static_cast<uint32_t>(kQBucket0 + i) << 19);
+    uint32_t below = 0u, inside = 0x7F800000u;   // (+inf)
+#pragma unroll
+    for (int j = 0; j < 7; ++j) {
+      const float pj = cb.thresholds[8 + j];
+      if (pj < lo) {
+        ++below;
+      } else if (pj < hi) {
+        inside = __float_as_uint(pj);
+      }
+    }
+    th.bucket[i] = make_uint2(inside, below);
   }
   if (threadIdx.x == 0) {
-    bool sym = cb.thresholds[7] == 0.0f;
-    for (int k = 0; k < 7; ++k) sym = sym && cb.thresholds[14 - k] == -cb.thresholds[k] && cb.thresholds[8 + k] > 0.0f;
-    th.sym = sym ? 1 : 0;
+    // symmetric, positive, and no two (sorted) thresholds in one bucket
+    bool fast = cb.thresholds[7] == 0.0f;
+#pragma unroll
+    for (int k = 0; k < 7; ++k) fast = fast && cb.thresholds[14 - k] == -cb.thresholds[k] && cb.thresholds[8 + k] > 0.0f;
+#pragma unroll
+    for (int j = 0; j + 1 < 7; ++j) fast = fast && bucket_of(cb.thresholds[8 + j]) != bucket_of(cb.thresholds[9 + j]);
+    th.fast = fast ? 1 : 0;
   }
   __syncthreads();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;

@@ -246,42 +246,61 @@ def test_missing_library_raises(tmp_path):
             tq._lib = tq._lib_saved
 
 
-def test_symmetric_threshold_search_counts_like_the_full_search():
-    # The quantize kernel, on finite half blocks, finds a code with a 3-step
-    # search on |u| over the 7 positive thresholds p[j] (u > 0: 8 + #{p[j] < u})
-    # or, for u <= 0, the largest floats b[j] below them (7 - #{|u| > b[j]}).
-    # On the library's own fp32 thresholds (symmetric: t[14 - k] == -t[k]),
-    # that must equal the number of thresholds strictly below u for every u,
-    # ties included: checked at each threshold, +-4 ulps around it, both signs.
+def test_bucket_threshold_search_counts_like_the_full_search():
+    # The quantize kernel, on finite half blocks of a symmetric codebook, takes
+    # a code from |u|'s bucket (bits >> 19 = exponent and top 4 mantissa bits,
+    # 2^-5 .. 2^3 in 128 buckets, one bucket below and one above): the number
+    # of positive thresholds below the bucket, plus the one inside it if
+    # |u| passes it, compared as float bits (> for u > 0, >= for u <= 0).
+    # Built here as the kernel builds it from the library's fp32 thresholds,
+    # and checked against the strict count t < u on every float of every
+    # bucket that holds a threshold, both signs, and at both ends of the others.
     _, th = tq.tq4_1s_codebook()
     t = th.numpy().astype(np.float32)
-    assert t[7] == 0.0 and all(t[14 - k] == -t[k] for k in range(7))
     p = t[8:15]
-    b = (p.view(np.uint32) - np.uint32(1)).view(np.float32)
-    assert np.all(np.nextafter(p, np.float32(0)) == b)
+    q0, nb = 122 << 4, 130
 
-    def full(u):
-        return int(np.sum(t < u))
+    def bucket_of_bits(bits):
+        q = (bits >> 19).astype(np.int64) - (q0 - 1)
+        return np.clip(q, 0, nb - 1)
 
-    def symmetric(u):
+    pb = p.view(np.uint32)
+    assert len(set(bucket_of_bits(pb).tolist())) == 7          # one threshold per bucket at most
+    inside = np.full(nb, 0x7F800000, np.uint64)
+    below = np.zeros(nb, np.int64)
+    for i in range(nb):
+        lo = 0.0 if i == 0 else np.array([(q0 + i - 1) << 19], np.uint32).view(np.float32)[0]
+        hi = np.inf if i == nb - 1 else np.array([(q0 + i) << 19], np.uint32).view(np.float32)[0]
+        for pj in p:
+            if pj < lo:
+                below[i] += 1
+            elif pj < hi:
+                inside[i] = int(np.array([pj], np.float32).view(np.uint32)[0])
+
+    def bucket_code(u):
         pos = u > 0
-        au = np.float32(abs(u))
-        tb = p if pos else b
-        c = 4 if au > tb[3] else 0
-        c += 2 if au > tb[c + 1] else 0
-        c += 1 if au > tb[c] else 0
-        return 8 + c if pos else 7 - c
+        ab = u.view(np.uint32) & np.uint32(0x7FFFFFFF)
+        q = bucket_of_bits(ab)
+        c = below[q] + ((ab.astype(np.uint64) + np.where(pos, 0, 1).astype(np.uint64)) > inside[q]).astype(np.int64)
+        return np.where(pos, 8 + c, 7 - c)
 
-    cases = [np.float32(0.0), np.float32(-0.0), np.float32(1e-30), np.float32(-1e-30), np.float32(7.0),
-             np.float32(-7.0)]
-    for x in t:
-        for sgn in (1, -1):
-            v = np.float32(sgn * x)
-            bits = v.view(np.uint32).astype(np.int64)
-            for dlt in range(-4, 5):
-                if v == 0.0:
-                    continue
-                cases.append(np.array([bits + dlt], dtype=np.int64).astype(np.uint32).view(np.float32)[0])
-    assert len(cases) > 200
-    for u in cases:
-        assert symmetric(u) == full(u), (float(u), symmetric(u), full(u))
+    def full_code(u):
+        return (t[None, :] < u[:, None]).sum(axis=1)
+
+    for pj in pb:
+        b = int(pj >> 19)
+        bits = np.arange(b << 19, (b + 1) << 19, dtype=np.uint64).astype(np.uint32)
+        for sgn in (0, 0x80000000):
+            u = (bits | np.uint32(sgn)).view(np.float32)
+            for chunk in range(0, len(u), 1 << 16):
+                uu = u[chunk:chunk + (1 << 16)]
+                assert np.array_equal(bucket_code(uu), full_code(uu))
+    ends = []
+    for i in range(nb):
+        for bits in ((q0 + i - 1) << 19, ((q0 + i) << 19) - 1):
+            if 0 < bits < 0x7F800000:
+                ends.append(bits)
+    ends += [0, 1, 0x00800000, 0x3D000000 - 1, 0x3D000000, 0x41000000 - 1, 0x41000000, 0x7F7FFFFF]
+    e = np.array(ends, np.uint32)
+    u = np.concatenate([e, e | np.uint32(0x80000000)]).view(np.float32)
+    assert np.array_equal(bucket_code(u), full_code(u))

@@ -254,16 +254,21 @@ def test_streamk_overflowing_levels_fall_back_to_the_exact_path():
 
 
 def test_quantize_fast_path_matches_the_checked_forms():
-    # the symmetric search and the quotient sequence are the forms that
-    # test_abi_host.py and the GPU probe of the division checked: b[j] is the
-    # float just below p[j]; the search runs only on symmetric thresholds and
-    # finite half blocks; other half blocks keep the division and full search
+    # the bucket search and the quotient sequence are the forms that
+    # test_abi_host.py (exhaustively on the threshold buckets) and the GPU
+    # probe of the division checked: the table as built there, the search
+    # only on symmetric thresholds with one per bucket and on finite half
+    # blocks; other half blocks keep the division and the full search
     src = _read("tq4_kernels.cu")
-    for s in ("th.b[threadIdx.x] = threadIdx.x < 7 ? __uint_as_float(__float_as_uint(pj) - 1u) : INFINITY;",
-              "const float* tb = pos ? th.p : th.b;",
-              "uint32_t c = (au > tb[3]) ? 4u : 0u;",
-              "c += (au > tb[c + 1]) ? 2u : 0u;",
-              "c += (au > tb[c]) ? 1u : 0u;",
+    for s in ("constexpr int kQBucket0 = 122 << 4;",
+              "constexpr int kQBuckets = 130;",
+              "const float lo = i == 0 ? 0.0f : __uint_as_float(static_cast<uint32_t>(kQBucket0 + i - 1) << 19);",
+              "const float hi = i == kQBuckets - 1 ? INFINITY : __uint_as_float(static_cast<uint32_t>(kQBucket0 + i) << 19);",
+              "th.bucket[i] = make_uint2(inside, below);",
+              "fast = fast && bucket_of(cb.thresholds[8 + j]) != bucket_of(cb.thresholds[9 + j]);",
+              "int q = static_cast<int>(ab >> 19) - (kQBucket0 - 1);",
+              "q = q < 0 ? 0 : (q > kQBuckets - 1 ? kQBuckets - 1 : q);",
+              "const uint32_t c = e.y + ((ab + (pos ? 0u : 1u) > e.x) ? 1u : 0u);",
               "code = pos ? 8u + c : 7u - c;",
               "if (fin && d != 0.0f) {",
               "const float y = __frcp_rn(d);",
