@@ -36,10 +36,14 @@
 //     remaining tiles and the epilogue.
 //
 // Warps (640 threads, one CTA per SM):
-//   4      lane 0: producer of the codes and scales tiles, and of every
-//          barrier (its warp takes no part in the set-up stores);
-//   16     lane 0: producer of the x tiles (and of a weight not flagged
-//          static) after the wait; 16 and 17 lane 0 issue the rotation MMAs;
+//   4      lane 0: producer of the scales and codes tiles (in that order)
+//          and of every barrier but xland (its warp takes no part in the
+//          set-up stores);
+//   16     lane 0: producer of the x tiles -- its own barrier, the wait and
+//          the copy at entry, so that x lands during the set-up (its warp
+//          takes no part in the set-up stores either) -- and of a weight not
+//          flagged static after the set-up; 16 and 17 lane 0 issue the
+//          rotation MMAs;
 //   1-3, 17-19  lane 0: MMA issuers, one per (dequant group, 64-k half);
 //   0-3    epilogue (thread = tile row) once the MMAs are done, then the
 //          cluster reduction of the rows this CTA owns (all warps);
