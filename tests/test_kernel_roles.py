@@ -277,3 +277,33 @@ def test_quantize_fast_path_matches_the_checked_forms():
               "if (!finite) raise_status(TQ_DEV_NONFINITE);",
               "__syncwarp();   // every lane is done with the tile (the check above reads it)"):
         assert s in src, s
+
+
+def test_streamk_exact_path_reads_x_where_the_fused_prologue_wrote_it():
+    # In fused mode x' lives only in the CTA's B tiles.  The prologue writes
+    # unit u = (iteration li, slice sl, token j) as four 16-byte chunks q at
+    # btile(li) + (sl >> 1) * kXHalfBytes + 128 j + ((q ^ cx) << 4), with
+    # cx = 4 (sl & 1) ^ (j & 7), element t of chunk q at byte 2 t.  The exact
+    # fallback of the epilogue reads column kk of local iteration li at the
+    # address below.  Both as written in the source, and the same byte for
+    # every (li, sl, j, q, t).
+    src = _read("tq4_streamk.cu")
+    assert "cx = ((sl & 1) * 4) ^ (j & 7);   // chunk q sits at chunk q ^ cx" in src
+    assert "return btile_of(li) + (sl >> 1) * kXHalfBytes + j * 128;" in src
+    assert "*reinterpret_cast<uint4*>(rowp + ((q ^ cx) << 4)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);" in src
+    assert ": *reinterpret_cast<const uint16_t*>(xs + li * kXBytes + (e >> 6) * kXHalfBytes + jj * 128 +" in src
+    assert "((((e64 >> 3) ^ (jj & 7))) << 4) + (e64 & 7) * 2);" in src
+    assert "const int li = li0 + (kk >> 7) - (kc0 >> 7), e = kk & 127, e64 = e & 63;" in src
+    env = _constants(_read("tq4_internal.h"), src)
+    half, full = env["kXHalfBytes"], env["kXBytes"]
+    for li in range(env["kFusedMaxIters"]):
+        for sl in range(4):
+            for j in range(env["kSegRows"]):
+                cx = ((sl & 1) * 4) ^ (j & 7)
+                for q in range(4):
+                    for t in range(8):
+                        written = li * full + (sl >> 1) * half + j * 128 + ((q ^ cx) << 4) + 2 * t
+                        e = 32 * sl + 8 * q + t
+                        e64 = e & 63
+                        read = li * full + (e >> 6) * half + j * 128 + (((e64 >> 3) ^ (j & 7)) << 4) + (e64 & 7) * 2
+                        assert written == read, (li, sl, j, q, t)
